@@ -1,0 +1,326 @@
+/*
+ * s6_oracle.c -- plain, slow, fp64 CPU oracle for the selective scan (S6).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test-suite, the smoke check and the
+ * CPU-baseline leg of the benchmark may load this library.  The product path
+ * (the CUDA library and its Python binding) shares no code with it and never
+ * calls it.
+ *
+ * Sources (page title, section):
+ *  [KN1]  "Mamba: Linear-Time Sequence Modeling with Selective State Spaces"
+ *         (chapterpal.com), Knowl 1 "Selective State Space Layer (S6)":
+ *         steps 2-4 and the per-element loop (discretize, update, readout).
+ *  [KN4]  same page, Knowl 4 "Equivalence of Zero-Order Hold Selective SSM to
+ *         Gated Recurrent Units" (Theorem 1).
+ *  [PG33] "Mamba: Linear-Time Sequence Modeling with Selective State Spaces"
+ *         (paper-graph-ui summary), section 3.4, "Algorithm 2 (Selective S6)"
+ *         and "The specific functional forms" (softplus), and "The Mamba
+ *         Architecture" (SiLU gate branch).
+ *  [TP-II6] "Mamba: Linear-Time Sequence Modeling with Selective State Spaces"
+ *         (trishampatil.com engineering walk-through), Part II section 4
+ *         (h_0 = 0) and section 6 (Algorithm 2 shapes).
+ *  [TP-III4] same page, Part III section 4 (recomputation in the backward).
+ *
+ * What is computed (forward), for every batch b and channel d independently:
+ *     Delta_t = softplus(delta[b,d,t] + bias[d])                     [PG33]
+ *     for n:  Abar = exp(Delta_t * A[d,n])                           [KN1 step 3]
+ *             Bbar = (exp(Delta_t * A[d,n]) - 1) / A[d,n] * B[b,n,t] [KN1 step 3]
+ *             h[n] = Abar * h[n] + Bbar * u[b,d,t]                   [KN1 step 4]
+ *     y0_t = sum_n C[b,n,t] * h[n]  (+ D[d] * u[b,d,t] if D given)   [KN1 step 4]
+ *     y_t  = y0_t * silu(z[b,d,t])  (if z given)                     [PG33 block]
+ * with h = 0 before the first step [TP-II6 s.4] and last_state = h after the
+ * last step.
+ *
+ * Readings where the pages are silent or ambiguous (each one is listed in the
+ * design notes of the repository):
+ *  - Bbar is the exact zero-order-hold value for a diagonal A, evaluated as
+ *    Delta * psi(Delta*A) * B with psi(x) = expm1(x)/x (psi(0) = 1), which is
+ *    the same quantity written without the cancellation of exp(x) - 1 and
+ *    without the division by A (so A = 0 is the limit Delta*B).
+ *  - softplus is exact (stable form, no large-argument cutoff).
+ *  - The D skip and the z gate are not on the pages; y = (C.h + D*u)*silu(z).
+ *
+ * The backward is the adjoint of the forward above, derived by hand from it
+ * (the pages give no gradient formulas).  States are recomputed forward per
+ * channel and kept in fp64 (the oracle has no memory constraint), then a
+ * reverse sweep accumulates gradients [TP-III4].
+ *
+ * Parity pins (the tests check this file against): Theorem 1 closed form,
+ * the LTI convolution form, brute-force unrolling, an independent ZOH via the
+ * matrix exponential, the exact ODE solution for a step input, finite
+ * differences and autograd for the backward, and exact hand-derived values.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdlib.h>
+#include <string.h>
+
+typedef long long i64;
+
+/* softplus(v) = log(1 + e^v), stable form. */
+static double softplus(double v) {
+  if (v > 0.0) return v + log1p(exp(-v));
+  return log1p(exp(v));
+}
+
+/* logistic sigmoid, stable form. */
+static double sigmoid(double v) {
+  if (v >= 0.0) return 1.0 / (1.0 + exp(-v));
+  double e = exp(v);
+  return e / (1.0 + e);
+}
+
+/* psi(x) = (exp(x) - 1) / x, psi(0) = 1. */
+static double psi(double x) {
+  if (x == 0.0) return 1.0;
+  return expm1(x) / x;
+}
+
+/* phi(x) = d psi / dx = (x e^x - expm1(x)) / x^2; series near 0. */
+static double phi(double x) {
+  if (fabs(x) < 1e-2) {
+    /* sum_k (k+1)/(k+2)! x^k */
+    return 0.5 + x * (1.0 / 3.0 + x * (1.0 / 8.0 + x * (1.0 / 30.0 + x * (1.0 / 144.0))));
+  }
+  return (x * exp(x) - expm1(x)) / (x * x);
+}
+
+typedef struct {
+  const double *u, *delta, *bias, *A, *B, *C, *D, *z, *dy;
+  double *y, *last_state;
+  double *du, *ddelta, *dz;
+  double *dA_part, *dD_part, *dbias_part; /* per (b,d) partials */
+  double *dB_acc, *dC_acc;                /* per-thread (batch,N,L) accumulators */
+  i64 batch, dim, L, N;
+  i64 first, last; /* range of flattened (b,d) this worker owns */
+} job_t;
+
+/* ---------------------------------------------------------------- forward */
+
+static void fwd_channel(const job_t *j, i64 b, i64 d, double *h) {
+  const i64 L = j->L, N = j->N, dim = j->dim;
+  const double *u = j->u + (b * dim + d) * L;
+  const double *dl = j->delta + (b * dim + d) * L;
+  const double *z = j->z ? j->z + (b * dim + d) * L : NULL;
+  const double *Bm = j->B + b * N * L;
+  const double *Cm = j->C + b * N * L;
+  const double *A = j->A + d * N;
+  const double bias = j->bias ? j->bias[d] : 0.0;
+  const double Dd = j->D ? j->D[d] : 0.0;
+  double *y = j->y + (b * dim + d) * L;
+  for (i64 n = 0; n < N; ++n) h[n] = 0.0;
+  for (i64 t = 0; t < L; ++t) {
+    const double Delta = softplus(dl[t] + bias);
+    double y0 = 0.0;
+    for (i64 n = 0; n < N; ++n) {
+      const double x = Delta * A[n];
+      const double Abar = exp(x);
+      const double Bbar = Delta * psi(x) * Bm[n * L + t];
+      h[n] = Abar * h[n] + Bbar * u[t];
+      y0 += Cm[n * L + t] * h[n];
+    }
+    if (j->D) y0 += Dd * u[t];
+    if (z) y0 *= z[t] * sigmoid(z[t]);
+    y[t] = y0;
+  }
+  if (j->last_state) {
+    double *ls = j->last_state + (b * dim + d) * N;
+    for (i64 n = 0; n < N; ++n) ls[n] = h[n];
+  }
+}
+
+static void *fwd_worker(void *arg) {
+  job_t *j = (job_t *)arg;
+  double *h = (double *)malloc(sizeof(double) * (size_t)j->N);
+  for (i64 i = j->first; i < j->last; ++i) fwd_channel(j, i / j->dim, i % j->dim, h);
+  free(h);
+  return NULL;
+}
+
+/* --------------------------------------------------------------- backward */
+
+static void bwd_channel(job_t *j, i64 b, i64 d, double *H, double *G) {
+  const i64 L = j->L, N = j->N, dim = j->dim;
+  const i64 off = (b * dim + d) * L;
+  const double *u = j->u + off, *dl = j->delta + off, *dy = j->dy + off;
+  const double *z = j->z ? j->z + off : NULL;
+  const double *Bm = j->B + b * N * L, *Cm = j->C + b * N * L;
+  const double *A = j->A + d * N;
+  const double bias = j->bias ? j->bias[d] : 0.0;
+  const double Dd = j->D ? j->D[d] : 0.0;
+
+  /* Recompute the forward states; H[(t+1)*N + n] = h_t, H[n] = h_{-1} = 0. */
+  for (i64 n = 0; n < N; ++n) H[n] = 0.0;
+  for (i64 t = 0; t < L; ++t) {
+    const double Delta = softplus(dl[t] + bias);
+    for (i64 n = 0; n < N; ++n) {
+      const double x = Delta * A[n];
+      H[(t + 1) * N + n] = exp(x) * H[t * N + n] + Delta * psi(x) * Bm[n * L + t] * u[t];
+    }
+  }
+
+  /* Reverse sweep.  G[n] is the adjoint of h_t (total derivative of the loss
+   * sum_t dy_t * y_t with respect to h_t). */
+  for (i64 n = 0; n < N; ++n) G[n] = 0.0;
+  double dD = 0.0, dbias = 0.0;
+  double *dA = j->dA_part + (b * dim + d) * N;
+  for (i64 n = 0; n < N; ++n) dA[n] = 0.0;
+  double *dBacc = j->dB_acc, *dCacc = j->dC_acc;
+  double Abar_next[64];
+  for (i64 n = 0; n < N; ++n) Abar_next[n] = 0.0; /* Abar_{L} unused: G_{L} = 0 */
+  for (i64 t = L - 1; t >= 0; --t) {
+    const double v = dl[t] + bias;
+    const double Delta = softplus(v);
+    double y0 = 0.0;
+    for (i64 n = 0; n < N; ++n) y0 += Cm[n * L + t] * H[(t + 1) * N + n];
+    if (j->D) y0 += Dd * u[t];
+    double dy0 = dy[t];
+    if (z) {
+      const double s = sigmoid(z[t]);
+      j->dz[off + t] = dy[t] * y0 * s * (1.0 + z[t] * (1.0 - s));
+      dy0 = dy[t] * z[t] * s;
+    }
+    double du = j->D ? Dd * dy0 : 0.0;
+    double dDelta = 0.0;
+    if (j->D) dD += dy0 * u[t];
+    for (i64 n = 0; n < N; ++n) {
+      const double x = Delta * A[n];
+      const double Abar = exp(x);
+      const double hprev = H[t * N + n];
+      /* G_t = C_t dy0_t + Abar_{t+1} G_{t+1} */
+      G[n] = Cm[n * L + t] * dy0 + Abar_next[n] * G[n];
+      Abar_next[n] = Abar;
+      const double Bt = Bm[n * L + t];
+      const double Ebar = Delta * psi(x); /* Bbar / B */
+      du += G[n] * Ebar * Bt;
+      /* d/dDelta of (Abar h_prev + Bbar u) = A Abar h_prev + Abar B u */
+      dDelta += G[n] * Abar * (A[n] * hprev + Bt * u[t]);
+      /* d/dA of (Abar h_prev + Bbar u) = Delta Abar h_prev + B u Delta^2 phi(x) */
+      dA[n] += G[n] * (Delta * Abar * hprev + Bt * u[t] * Delta * Delta * phi(x));
+      dBacc[(b * N + n) * L + t] += G[n] * u[t] * Ebar;
+      dCacc[(b * N + n) * L + t] += dy0 * H[(t + 1) * N + n];
+    }
+    const double dd = dDelta * sigmoid(v);
+    j->du[off + t] = du;
+    j->ddelta[off + t] = dd;
+    dbias += dd;
+  }
+  j->dD_part[b * dim + d] = dD;
+  j->dbias_part[b * dim + d] = dbias;
+}
+
+static void *bwd_worker(void *arg) {
+  job_t *j = (job_t *)arg;
+  double *H = (double *)malloc(sizeof(double) * (size_t)((j->L + 1) * j->N));
+  double *G = (double *)malloc(sizeof(double) * (size_t)j->N);
+  for (i64 i = j->first; i < j->last; ++i) bwd_channel(j, i / j->dim, i % j->dim, H, G);
+  free(H);
+  free(G);
+  return NULL;
+}
+
+/* ------------------------------------------------------------- driver */
+
+static int run_workers(job_t *base, i64 nthreads, void *(*fn)(void *), int per_thread_acc) {
+  const i64 total = base->batch * base->dim;
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > total) nthreads = total > 0 ? total : 1;
+  job_t *jobs = (job_t *)calloc((size_t)nthreads, sizeof(job_t));
+  pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+  if (!jobs || !th) { free(jobs); free(th); return -1; }
+  const size_t accn = (size_t)(base->batch * base->N * base->L);
+  int rc = 0;
+  for (i64 k = 0; k < nthreads; ++k) {
+    jobs[k] = *base;
+    jobs[k].first = total * k / nthreads;
+    jobs[k].last = total * (k + 1) / nthreads;
+    if (per_thread_acc) {
+      jobs[k].dB_acc = (double *)calloc(accn ? accn : 1, sizeof(double));
+      jobs[k].dC_acc = (double *)calloc(accn ? accn : 1, sizeof(double));
+      if (!jobs[k].dB_acc || !jobs[k].dC_acc) rc = -1;
+    }
+  }
+  if (rc == 0) {
+    for (i64 k = 1; k < nthreads; ++k) pthread_create(&th[k], NULL, fn, &jobs[k]);
+    fn(&jobs[0]);
+    for (i64 k = 1; k < nthreads; ++k) pthread_join(th[k], NULL);
+  }
+  if (per_thread_acc && rc == 0) {
+    /* fixed-order reduction of the per-thread accumulators */
+    for (size_t i = 0; i < accn; ++i) {
+      double sb = 0.0, sc = 0.0;
+      for (i64 k = 0; k < nthreads; ++k) { sb += jobs[k].dB_acc[i]; sc += jobs[k].dC_acc[i]; }
+      base->dB_acc[i] = sb;
+      base->dC_acc[i] = sc;
+    }
+  }
+  if (per_thread_acc)
+    for (i64 k = 0; k < nthreads; ++k) { free(jobs[k].dB_acc); free(jobs[k].dC_acc); }
+  free(jobs);
+  free(th);
+  return rc;
+}
+
+/* Forward.  Layouts: u, delta, z, y: (batch, dim, L); B, C: (batch, N, L);
+ * A: (dim, N); bias, D: (dim); last_state: (batch, dim, N).  bias, D, z and
+ * last_state may be NULL.  Returns 0 on success. */
+int s6_oracle_fwd(const double *u, const double *delta, const double *bias, const double *A,
+                  const double *B, const double *C, const double *D, const double *z,
+                  double *y, double *last_state, i64 batch, i64 dim, i64 L, i64 N,
+                  i64 nthreads) {
+  if (batch < 0 || dim < 0 || L < 0 || N < 1 || N > 64) return -2;
+  job_t j;
+  memset(&j, 0, sizeof(j));
+  j.u = u; j.delta = delta; j.bias = bias; j.A = A; j.B = B; j.C = C; j.D = D; j.z = z;
+  j.y = y; j.last_state = last_state;
+  j.batch = batch; j.dim = dim; j.L = L; j.N = N;
+  if (batch * dim == 0) return 0;
+  return run_workers(&j, nthreads, fwd_worker, 0);
+}
+
+/* Backward of the loss sum(dy * y).  Outputs: du, ddelta, dz (batch, dim, L);
+ * dB, dC (batch, N, L); dA (dim, N); dD, dbias (dim).  dz must be non-NULL iff
+ * z is; dD must be non-NULL iff D is; dbias may be NULL.  Returns 0 on
+ * success. */
+int s6_oracle_bwd(const double *u, const double *delta, const double *bias, const double *A,
+                  const double *B, const double *C, const double *D, const double *z,
+                  const double *dy, double *du, double *ddelta, double *dA, double *dB,
+                  double *dC, double *dD, double *dz, double *dbias, i64 batch, i64 dim, i64 L,
+                  i64 N, i64 nthreads) {
+  if (batch < 0 || dim < 0 || L < 0 || N < 1 || N > 64) return -2;
+  if ((z == NULL) != (dz == NULL)) return -2;
+  if ((D == NULL) != (dD == NULL)) return -2;
+  const size_t bd = (size_t)(batch * dim);
+  job_t j;
+  memset(&j, 0, sizeof(j));
+  j.u = u; j.delta = delta; j.bias = bias; j.A = A; j.B = B; j.C = C; j.D = D; j.z = z;
+  j.dy = dy; j.du = du; j.ddelta = ddelta; j.dz = dz;
+  j.batch = batch; j.dim = dim; j.L = L; j.N = N;
+  j.dB_acc = dB; j.dC_acc = dC;
+  memset(dB, 0, sizeof(double) * (size_t)(batch * N * L));
+  memset(dC, 0, sizeof(double) * (size_t)(batch * N * L));
+  memset(dA, 0, sizeof(double) * (size_t)(dim * N));
+  if (dD) memset(dD, 0, sizeof(double) * (size_t)dim);
+  if (dbias) memset(dbias, 0, sizeof(double) * (size_t)dim);
+  if (bd == 0) return 0;
+  j.dA_part = (double *)calloc(bd * (size_t)N, sizeof(double));
+  j.dD_part = (double *)calloc(bd, sizeof(double));
+  j.dbias_part = (double *)calloc(bd, sizeof(double));
+  int rc = -1;
+  if (j.dA_part && j.dD_part && j.dbias_part) {
+    rc = run_workers(&j, nthreads, bwd_worker, 1);
+    if (rc == 0) {
+      /* parameters are shared over the batch: sum the per-(b,d) partials in b order */
+      for (i64 b = 0; b < batch; ++b)
+        for (i64 d = 0; d < dim; ++d) {
+          for (i64 n = 0; n < N; ++n) dA[d * N + n] += j.dA_part[(b * dim + d) * N + n];
+          if (dD) dD[d] += j.dD_part[b * dim + d];
+          if (dbias) dbias[d] += j.dbias_part[b * dim + d];
+        }
+    }
+  }
+  free(j.dA_part);
+  free(j.dD_part);
+  free(j.dbias_part);
+  return rc;
+}
