@@ -1,0 +1,161 @@
+/*
+ * mamba_scan.h -- C ABI of libmambascan, the B200 (sm_100a) fused selective
+ * scan (S6).
+ *
+ * The operation (forward) follows "Mamba: Linear-Time Sequence Modeling with
+ * Selective State Spaces" (chapterpal.com), Knowl 1 "Selective State Space
+ * Layer (S6)" (steps 2-4 and its per-element loop), with the softplus of
+ * section 3.4 "The specific functional forms" and the SiLU gate branch of
+ * "The Mamba Architecture" on the paper-graph-ui summary page.  For every
+ * batch b and channel d, with an N-dimensional diagonal state h (h = 0 before
+ * the first step):
+ *
+ *     Delta_t = softplus(delta[b,d,t] + delta_bias[d])
+ *     Abar_tn = exp(Delta_t * A[d,n])
+ *     Bbar_tn = (exp(Delta_t * A[d,n]) - 1) / A[d,n] * B[b,n,t]   (Delta_t*B at A = 0)
+ *     h_tn    = Abar_tn * h_{t-1,n} + Bbar_tn * u[b,d,t]
+ *     y[b,d,t] = (sum_n C[b,n,t] * h_tn + D[d] * u[b,d,t]) * silu(z[b,d,t])
+ *     last_state[b,d,n] = h_{L-1,n}
+ *
+ * The backward recomputes the states from the inputs instead of reading
+ * stored ones (the recomputation of section 3.3 of the paper-graph-ui page and
+ * Part III section 4 of the trishampatil.com walk-through) and returns the
+ * gradients of sum(dy * y) with respect to every input.
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers on the current CUDA device, owned
+ *    by the caller.  The library never frees them and keeps no reference after
+ *    the call returns.  Tensors are dense and contiguous in the stated layout
+ *    (last index fastest) and aligned to their element size; 16-byte aligned
+ *    tensors whose rows are 16-byte multiples take the fastest kernels.
+ *  - `dtype` selects the I/O type of u, delta, z, B, C, y, dy, du, ddelta, dz,
+ *    dB and dC.  A, D, delta_bias, last_state, dA, dD and ddelta_bias are
+ *    always float32.  Arithmetic is float32 throughout; bf16 values are
+ *    widened exactly on load and rounded to nearest-even once on store.
+ *  - Calls only enqueue work on `stream` (NULL = the legacy default stream)
+ *    and return.  The status reports argument validation and launch errors.
+ *    Errors raised later on the device (a bounded wait that expired) are
+ *    recorded in a per-device sticky error word read by
+ *    mamba_scan_stream_status().
+ *  - Temporary device memory (chunk-boundary states, partial sums) is taken
+ *    with cudaMallocAsync/cudaFreeAsync on `stream`; failure returns
+ *    MAMBA_ERR_OUT_OF_MEMORY.
+ *  - Outputs are overwritten, never accumulated into.  No exception, abort,
+ *    printf or trap crosses or happens behind this interface.  Calls are
+ *    thread-safe; concurrent calls on different streams are independent.
+ *  - batch, dim or L equal to 0 is an empty problem: nothing is computed, and
+ *    outputs of size 0 are left alone; last_state (L = 0) is set to 0 and the
+ *    parameter gradients dA, dD, ddelta_bias are set to 0.
+ */
+#ifndef MAMBA_SCAN_H
+#define MAMBA_SCAN_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MAMBA_SCAN_API __attribute__((visibility("default")))
+#else
+#define MAMBA_SCAN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *mamba_stream_t;
+
+typedef enum { MAMBA_F32 = 0, MAMBA_BF16 = 1 } mamba_dtype_t;
+
+typedef enum {
+  MAMBA_OK = 0,
+  MAMBA_ERR_INVALID_ARG = 1,   /* null/misaligned/overlapping/host pointer, bad size */
+  MAMBA_ERR_UNSUPPORTED = 2,   /* N outside 1..16, or a shape beyond the limits */
+  MAMBA_ERR_CUDA = 3,          /* a CUDA runtime call or a launch failed */
+  MAMBA_ERR_OUT_OF_MEMORY = 4, /* the stream-ordered workspace could not be allocated */
+  MAMBA_ERR_DEVICE_TIMEOUT = 5 /* a bounded device-side wait expired (sticky) */
+} mamba_status_t;
+
+/* Kernel-path selection for mamba_scan_fwd_ex / mamba_scan_bwd_ex. */
+typedef enum {
+  MAMBA_PATH_AUTO = 0,       /* pick by shape and A (the default of the plain calls) */
+  MAMBA_PATH_REFERENCE = 1,  /* one thread per channel, plain loads, any A */
+  MAMBA_PATH_GENERIC = 2,    /* staged, chunked kernel, one exp per state element */
+  MAMBA_PATH_STRUCTURED = 3  /* staged, chunked kernel for A[d,n] = (n+1)*A[d,0] < 0;
+                                channels that do not have this form fall back to the
+                                generic arithmetic inside the same launch */
+} mamba_path_t;
+
+typedef struct {
+  int32_t path;        /* a mamba_path_t */
+  int32_t chunk_len;   /* time steps per chunk of the chunked kernels; 0 = automatic.
+                          Must be a positive multiple of 64 when set. */
+  int32_t reserved[6]; /* must be 0 */
+} mamba_scan_options_t;
+
+/*
+ * Forward.
+ *   u, delta, z, y : (batch, dim, L), dtype
+ *   B, C           : (batch, N, L), dtype (input-dependent, one row per step)
+ *   A              : (dim, N) float32 (diagonal of the state matrix per channel)
+ *   delta_bias, D  : (dim) float32
+ *   last_state     : (batch, dim, N) float32, the state after step L-1
+ * Nullable: delta_bias (treated as 0), D (no skip), z (no gate), last_state
+ * (not written).  1 <= N <= 16.
+ */
+MAMBA_SCAN_API mamba_status_t mamba_scan_fwd(const void *u, const void *delta, const float *delta_bias,
+                              const float *A, const void *B, const void *C, const float *D,
+                              const void *z, void *y, float *last_state, int64_t batch,
+                              int64_t dim, int64_t L, int64_t N, mamba_dtype_t dtype,
+                              mamba_stream_t stream);
+
+/* Forward with an explicit kernel path (options may be NULL = defaults). */
+MAMBA_SCAN_API mamba_status_t mamba_scan_fwd_ex(const void *u, const void *delta, const float *delta_bias,
+                                 const float *A, const void *B, const void *C, const float *D,
+                                 const void *z, void *y, float *last_state, int64_t batch,
+                                 int64_t dim, int64_t L, int64_t N, mamba_dtype_t dtype,
+                                 const mamba_scan_options_t *options, mamba_stream_t stream);
+
+/*
+ * Backward of the scalar sum(dy * y), recomputing the states from the inputs.
+ *   inputs as in mamba_scan_fwd, plus dy : (batch, dim, L) dtype
+ *   du, ddelta, dz : (batch, dim, L) dtype
+ *   dB, dC         : (batch, N, L) dtype (summed over channels)
+ *   dA             : (dim, N) float32, dD, ddelta_bias : (dim) float32
+ *                    (summed over batch and time)
+ * dz must be non-NULL exactly when z is, dD exactly when D is; ddelta_bias
+ * may be NULL.  The reductions run in a fixed order: results are bitwise
+ * reproducible run to run on the same device and shape.
+ */
+MAMBA_SCAN_API mamba_status_t mamba_scan_bwd(const void *u, const void *delta, const float *delta_bias,
+                              const float *A, const void *B, const void *C, const float *D,
+                              const void *z, const void *dy, void *du, void *ddelta, float *dA,
+                              void *dB, void *dC, float *dD, void *dz, float *ddelta_bias,
+                              int64_t batch, int64_t dim, int64_t L, int64_t N,
+                              mamba_dtype_t dtype, mamba_stream_t stream);
+
+MAMBA_SCAN_API mamba_status_t mamba_scan_bwd_ex(const void *u, const void *delta, const float *delta_bias,
+                                 const float *A, const void *B, const void *C, const float *D,
+                                 const void *z, const void *dy, void *du, void *ddelta,
+                                 float *dA, void *dB, void *dC, float *dD, void *dz,
+                                 float *ddelta_bias, int64_t batch, int64_t dim, int64_t L,
+                                 int64_t N, mamba_dtype_t dtype,
+                                 const mamba_scan_options_t *options, mamba_stream_t stream);
+
+/* Synchronizes `stream`, then returns MAMBA_ERR_CUDA for a pending CUDA error,
+ * else MAMBA_ERR_DEVICE_TIMEOUT if a kernel of this library recorded an
+ * expired wait on the current device since the last call (the record is
+ * cleared), else MAMBA_OK. */
+MAMBA_SCAN_API mamba_status_t mamba_scan_stream_status(mamba_stream_t stream);
+
+/* Static, human-readable name of a status code (never NULL). */
+MAMBA_SCAN_API const char *mamba_scan_status_string(mamba_status_t status);
+
+/* Version of this ABI (incremented on any incompatible change). */
+MAMBA_SCAN_API int mamba_scan_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MAMBA_SCAN_H */

@@ -1,0 +1,241 @@
+// bwd_reference.cuh -- backward of sum(dy * y) with recomputed states.
+//
+// The states h_t (batch, dim, L, N) are never stored: a first forward sweep
+// keeps only the state at the start of every block of kBwdTC steps; the
+// reverse sweep then, block by block from the end, recomputes the block's
+// states into shared memory and walks it backwards with the adjoint
+//     G_t = C_t dy0_t + Abar_{t+1} G_{t+1},   dy0_t = dy_t silu(z_t),
+// accumulating the local gradients (the recomputation of section 3.3 of the
+// paper-graph-ui page, "Recomputation for the backward pass").  The adjoint
+// itself is derived from the forward; the pages give no gradient formulas.
+//
+// One thread per (batch, channel); a CTA holds kBwdThreads channels of one
+// batch row.  Reductions are deterministic: dB and dC (summed over channels)
+// are reduced per warp by a butterfly reduce-scatter, per CTA in shared
+// memory, then across CTAs by the finalize kernel in a fixed order; dA, dD
+// and the bias gradient (summed over batch and time) go through per-channel
+// partials.
+#pragma once
+#include "common.cuh"
+
+namespace mscan {
+
+constexpr int kBwdTC = 16;
+constexpr int kBwdThreads = 64;
+constexpr int kBwdSlots = 2 * kMaxN;  // dB in slots 0..15, dC in slots 16..31
+
+struct BwdWork {
+  float *ckpt;      // (batch*dim, n_chunks, NM) chunk-start states
+  float *part_bc;   // (n_dblk, batch, kBwdSlots, L) per-CTA sums of dB / dC
+  float *part_A;    // (batch*dim, N)
+  float *part_D;    // (batch*dim)
+  float *part_bias; // (batch*dim)
+  int64_t n_chunks, n_dblk;
+};
+
+// Butterfly reduce-scatter of 32 values over a warp: lane l returns the warp
+// sum of value index l.
+__device__ __forceinline__ float warp_reduce_scatter32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < o; ++i) {
+      const float send = up ? v[i] : v[i + o];
+      const float keep = up ? v[i + o] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  return v[0];
+}
+
+template <typename T, int NM>
+__global__ void __launch_bounds__(kBwdThreads) bwd_reference_kernel(BwdArgs a, BwdWork w) {
+  extern __shared__ float smem[];
+  float *hs = smem;                                // [kBwdTC][NM][kBwdThreads]
+  float *wsum = smem + kBwdTC * NM * kBwdThreads;  // [2 warps][kBwdSlots][kBwdTC]
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t b = blockIdx.y;
+  const int64_t d_raw = (int64_t)blockIdx.x * kBwdThreads + tid;
+  const bool valid = d_raw < a.dim;
+  const int64_t d = valid ? d_raw : a.dim - 1;  // loads stay in bounds
+  const int64_t ch = b * a.dim + d;
+  const int64_t L = a.L;
+  const int N = a.N;
+  const T *u = static_cast<const T *>(a.u) + ch * L;
+  const T *dl = static_cast<const T *>(a.delta) + ch * L;
+  const T *z = a.z ? static_cast<const T *>(a.z) + ch * L : nullptr;
+  const T *dy = static_cast<const T *>(a.dy) + ch * L;
+  const T *Bp = static_cast<const T *>(a.B) + b * N * L;
+  const T *Cp = static_cast<const T *>(a.C) + b * N * L;
+  const float bias = a.bias ? a.bias[d] : 0.f;
+  const float Dd = a.D ? a.D[d] : 0.f;
+  float *ckpt = w.ckpt + ch * w.n_chunks * NM;
+
+  float Av[NM], invA[NM], h[NM];
+#pragma unroll
+  for (int n = 0; n < NM; ++n) {
+    Av[n] = n < N ? a.A[d * N + n] : -1.f;
+    invA[n] = Av[n] != 0.f ? 1.f / Av[n] : 0.f;
+    h[n] = 0.f;
+  }
+
+  // Forward sweep: keep the state at the start of every block.
+  for (int64_t t = 0; t < L; ++t) {
+    if (t % kBwdTC == 0) {
+#pragma unroll
+      for (int n = 0; n < NM; ++n) ckpt[(t / kBwdTC) * NM + n] = h[n];
+    }
+    const float Delta = softplus_acc(to_f(dl[t]) + bias);
+    const float ut = to_f(u[t]);
+#pragma unroll
+    for (int n = 0; n < NM; ++n) {
+      if (n < N) {
+        const float x = Delta * Av[n];
+        const float E = Av[n] != 0.f ? expm1f(x) * invA[n] : Delta;
+        h[n] = expf(x) * h[n] + E * to_f(Bp[n * L + t]) * ut;
+      }
+    }
+  }
+
+  float G[NM], Anext[NM], dAacc[NM];
+#pragma unroll
+  for (int n = 0; n < NM; ++n) G[n] = Anext[n] = dAacc[n] = 0.f;
+  float dDacc = 0.f, dbacc = 0.f;
+
+  for (int64_t c = w.n_chunks - 1; c >= 0; --c) {
+    const int64_t t0 = c * kBwdTC;
+    const int steps = (int)((L - t0) < kBwdTC ? (L - t0) : kBwdTC);
+    // Recompute the block's states; hs[s] holds the state before step t0+s.
+#pragma unroll
+    for (int n = 0; n < NM; ++n) h[n] = ckpt[c * NM + n];
+    for (int s = 0; s < steps; ++s) {
+      const int64_t t = t0 + s;
+#pragma unroll
+      for (int n = 0; n < NM; ++n) hs[(s * NM + n) * kBwdThreads + tid] = h[n];
+      const float Delta = softplus_acc(to_f(dl[t]) + bias);
+      const float ut = to_f(u[t]);
+#pragma unroll
+      for (int n = 0; n < NM; ++n) {
+        if (n < N) {
+          const float x = Delta * Av[n];
+          const float E = Av[n] != 0.f ? expm1f(x) * invA[n] : Delta;
+          h[n] = expf(x) * h[n] + E * to_f(Bp[n * L + t]) * ut;
+        }
+      }
+    }
+    // Reverse sweep over the block.
+    for (int s = steps - 1; s >= 0; --s) {
+      const int64_t t = t0 + s;
+      const float v = to_f(dl[t]) + bias;
+      const float Delta = softplus_acc(v);
+      const float sv = sigmoid_acc(v);
+      const float ut = to_f(u[t]);
+      const float dyt = to_f(dy[t]);
+      float dy0 = dyt, zt = 0.f, sz = 0.f;
+      if (z) {
+        zt = to_f(z[t]);
+        sz = sigmoid_acc(zt);
+        dy0 = dyt * zt * sz;
+      }
+      float y0 = a.D ? Dd * ut : 0.f;
+      float du = a.D ? Dd * dy0 : 0.f;
+      float dDelta = 0.f;
+      float vals[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) vals[i] = 0.f;
+#pragma unroll
+      for (int n = 0; n < NM; ++n) {
+        if (n < N) {
+          const float hprev = hs[(s * NM + n) * kBwdThreads + tid];
+          const float x = Delta * Av[n];
+          const float Abar = expf(x);
+          const float E = Av[n] != 0.f ? expm1f(x) * invA[n] : Delta;
+          const float Bt = to_f(Bp[n * L + t]);
+          const float Ct = to_f(Cp[n * L + t]);
+          const float hcur = Abar * hprev + E * Bt * ut;
+          y0 += Ct * hcur;
+          G[n] = Ct * dy0 + Anext[n] * G[n];
+          Anext[n] = Abar;
+          du += G[n] * E * Bt;
+          dDelta += G[n] * Abar * (Av[n] * hprev + Bt * ut);
+          dAacc[n] += G[n] * (Delta * Abar * hprev + Bt * ut * Delta * Delta * dpsi_acc(x));
+          if (valid) {
+            vals[n] = G[n] * ut * E;
+            vals[kMaxN + n] = dy0 * hcur;
+          }
+        }
+      }
+      const float ddl = dDelta * sv;
+      if (valid) {
+        static_cast<T *>(a.du)[ch * L + t] = from_f<T>(du);
+        static_cast<T *>(a.ddelta)[ch * L + t] = from_f<T>(ddl);
+        if (z) static_cast<T *>(a.dz)[ch * L + t] = from_f<T>(dyt * y0 * sz * (1.f + zt * (1.f - sz)));
+        dDacc += dy0 * ut;
+        dbacc += ddl;
+      }
+      const float r = warp_reduce_scatter32(vals, lane);
+      wsum[(warp * kBwdSlots + lane) * kBwdTC + s] = r;
+    }
+    __syncthreads();
+    // CTA partial of dB / dC for this block.
+    for (int idx = tid; idx < kBwdSlots * kBwdTC; idx += kBwdThreads) {
+      const int slot = idx / kBwdTC, s = idx % kBwdTC;
+      if (s < steps) {
+        const float sum = wsum[(0 * kBwdSlots + slot) * kBwdTC + s] +
+                          wsum[(1 * kBwdSlots + slot) * kBwdTC + s];
+        w.part_bc[((blockIdx.x * a.batch + b) * kBwdSlots + slot) * L + t0 + s] = sum;
+      }
+    }
+    __syncthreads();
+  }
+  if (valid) {
+#pragma unroll
+    for (int n = 0; n < NM; ++n)
+      if (n < N) w.part_A[ch * N + n] = dAacc[n];
+    w.part_D[ch] = dDacc;
+    w.part_bias[ch] = dbacc;
+  }
+}
+
+// dB[b,n,t] / dC[b,n,t]: sum of the per-CTA partials over channel blocks.
+template <typename T>
+__global__ void bwd_finalize_bc_kernel(BwdArgs a, BwdWork w) {
+  const int64_t total = a.batch * a.N * a.L;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = i % a.L, n = (i / a.L) % a.N, b = i / (a.L * a.N);
+    float sb = 0.f, sc = 0.f;
+    for (int64_t k = 0; k < w.n_dblk; ++k) {
+      const float *p = w.part_bc + ((k * a.batch + b) * kBwdSlots) * a.L + t;
+      sb += p[n * a.L];
+      sc += p[(kMaxN + n) * a.L];
+    }
+    static_cast<T *>(a.dB)[i] = from_f<T>(sb);
+    static_cast<T *>(a.dC)[i] = from_f<T>(sc);
+  }
+}
+
+// dA[d,n], dD[d], dbias[d]: sum of the per-channel partials over the batch.
+__global__ void bwd_finalize_params_kernel(BwdArgs a, BwdWork w) {
+  const int64_t total = a.dim * a.N;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t d = i / a.N, n = i % a.N;
+    float s = 0.f;
+    for (int64_t b = 0; b < a.batch; ++b) s += w.part_A[(b * a.dim + d) * a.N + n];
+    a.dA[i] = s;
+    if (n == 0) {
+      float sd = 0.f, sb = 0.f;
+      for (int64_t b = 0; b < a.batch; ++b) {
+        sd += w.part_D[b * a.dim + d];
+        sb += w.part_bias[b * a.dim + d];
+      }
+      if (a.dD) a.dD[d] = sd;
+      if (a.dbias) a.dbias[d] = sb;
+    }
+  }
+}
+
+}  // namespace mscan

@@ -1,0 +1,342 @@
+// mamba_scan.cu -- the C ABI of libmambascan: argument validation, workspace,
+// kernel selection and launch.  The operation is documented in
+// include/mamba_scan.h.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/mamba_scan.h"
+#include "bwd_reference.cuh"
+#include "common.cuh"
+#include "fwd_reference.cuh"
+#include "fwd_staged.cuh"
+
+using namespace mscan;
+
+namespace {
+
+constexpr int kAbiVersion = 1;
+
+struct Range {
+  uintptr_t lo, hi;
+};
+
+size_t dtype_size(mamba_dtype_t dt) { return dt == MAMBA_BF16 ? 2 : 4; }
+
+// A pointer the kernels may dereference: device (or managed) memory visible
+// from the current device.
+bool is_device_ptr(const void *p, int dev) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  if (at.type == cudaMemoryTypeManaged) return true;
+  return at.type == cudaMemoryTypeDevice && at.device == dev;
+}
+
+struct Checker {
+  int dev = 0;
+  mamba_status_t st = MAMBA_OK;
+  Range ranges[24];
+  bool is_out[24];
+  int n = 0;
+
+  // Records a buffer of `bytes` bytes; `required` buffers may not be NULL.
+  void buf(const void *p, size_t bytes, size_t align, bool required, bool output) {
+    if (st != MAMBA_OK) return;
+    if (!p) {
+      if (required && bytes > 0) st = MAMBA_ERR_INVALID_ARG;
+      return;
+    }
+    if (bytes == 0) return;
+    if (reinterpret_cast<uintptr_t>(p) % align != 0 || !is_device_ptr(p, dev)) {
+      st = MAMBA_ERR_INVALID_ARG;
+      return;
+    }
+    const uintptr_t lo = reinterpret_cast<uintptr_t>(p);
+    for (int i = 0; i < n; ++i) {
+      const bool overlap = lo < ranges[i].hi && ranges[i].lo < lo + bytes;
+      if (overlap && (output || is_out[i])) {
+        st = MAMBA_ERR_INVALID_ARG;
+        return;
+      }
+    }
+    ranges[n] = {lo, lo + bytes};
+    is_out[n] = output;
+    ++n;
+  }
+};
+
+mamba_status_t check_shape(int64_t batch, int64_t dim, int64_t L, int64_t N, mamba_dtype_t dt) {
+  if (dt != MAMBA_F32 && dt != MAMBA_BF16) return MAMBA_ERR_INVALID_ARG;
+  if (batch < 0 || dim < 0 || L < 0) return MAMBA_ERR_INVALID_ARG;
+  if (N < 1 || N > kMaxN) return MAMBA_ERR_UNSUPPORTED;
+  // Keep every flattened index inside int64 with room to spare, and the batch
+  // inside a grid dimension.
+  if (batch > 65535 || dim > (int64_t(1) << 31) || L > (int64_t(1) << 40)) return MAMBA_ERR_UNSUPPORTED;
+  const double elems = double(batch) * double(dim) * double(L);
+  if (elems > 9.0e15) return MAMBA_ERR_UNSUPPORTED;
+  return MAMBA_OK;
+}
+
+mamba_status_t check_options(const mamba_scan_options_t *o) {
+  if (!o) return MAMBA_OK;
+  if (o->path < MAMBA_PATH_AUTO || o->path > MAMBA_PATH_STRUCTURED) return MAMBA_ERR_INVALID_ARG;
+  if (o->chunk_len < 0 || (o->chunk_len > 0 && o->chunk_len % 64 != 0)) return MAMBA_ERR_INVALID_ARG;
+  for (int i = 0; i < 6; ++i)
+    if (o->reserved[i] != 0) return MAMBA_ERR_INVALID_ARG;
+  return MAMBA_OK;
+}
+
+mamba_status_t launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) return MAMBA_OK;
+  return e == cudaErrorMemoryAllocation ? MAMBA_ERR_OUT_OF_MEMORY : MAMBA_ERR_CUDA;
+}
+
+// Dispatch on N (rounded up to 1, 2, 4, 8 or 16; the padding states carry
+// B = C = 0 and so stay 0) and on the I/O type.
+template <template <typename, int> class Launcher, typename... Args>
+mamba_status_t dispatch(mamba_dtype_t dt, int N, Args &&...args) {
+#define MSCAN_CASE(NMV)                                                            \
+  if (N <= NMV) {                                                                  \
+    return dt == MAMBA_BF16 ? Launcher<__nv_bfloat16, NMV>::run(args...)          \
+                            : Launcher<float, NMV>::run(args...);                  \
+  }
+  MSCAN_CASE(1)
+  MSCAN_CASE(2)
+  MSCAN_CASE(4)
+  MSCAN_CASE(8)
+  MSCAN_CASE(16)
+#undef MSCAN_CASE
+  return MAMBA_ERR_UNSUPPORTED;
+}
+
+template <typename T, int NM>
+struct FwdReferenceLauncher {
+  static mamba_status_t run(const FwdArgs &a, cudaStream_t s) {
+    const int64_t ch = a.batch * a.dim;
+    const int64_t grid = (ch + kRefThreads - 1) / kRefThreads;
+    fwd_reference_kernel<T, NM><<<(unsigned)grid, kRefThreads, 0, s>>>(a);
+    return launch_status();
+  }
+};
+
+template <typename T, int NM>
+struct FwdStagedLauncher {
+  static mamba_status_t run(const FwdArgs &a, int path, int chunk_len, cudaStream_t s) {
+    return staged_forward<T, NM>(a, path, chunk_len, s);
+  }
+};
+
+template <typename T, int NM>
+struct BwdReferenceLauncher {
+  static mamba_status_t run(const BwdArgs &a, cudaStream_t s) {
+    BwdWork w;
+    w.n_chunks = (a.L + kBwdTC - 1) / kBwdTC;
+    w.n_dblk = (a.dim + kBwdThreads - 1) / kBwdThreads;
+    const size_t bd = size_t(a.batch * a.dim);
+    const size_t n_ckpt = bd * size_t(w.n_chunks) * NM;
+    const size_t n_bc = size_t(w.n_dblk) * size_t(a.batch) * kBwdSlots * size_t(a.L);
+    const size_t n_A = bd * size_t(a.N);
+    const size_t total = n_ckpt + n_bc + n_A + 2 * bd;
+    float *ws = nullptr;
+    if (cudaMallocAsync(reinterpret_cast<void **>(&ws), total * sizeof(float), s) != cudaSuccess) {
+      cudaGetLastError();
+      return MAMBA_ERR_OUT_OF_MEMORY;
+    }
+    w.ckpt = ws;
+    w.part_bc = w.ckpt + n_ckpt;
+    w.part_A = w.part_bc + n_bc;
+    w.part_D = w.part_A + n_A;
+    w.part_bias = w.part_D + bd;
+    const size_t smem = sizeof(float) * (kBwdTC * NM * kBwdThreads + 2 * kBwdSlots * kBwdTC);
+    mamba_status_t st = MAMBA_OK;
+    if (cudaFuncSetAttribute(bwd_reference_kernel<T, NM>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
+      st = MAMBA_ERR_CUDA;
+    }
+    if (st == MAMBA_OK) {
+      dim3 grid((unsigned)w.n_dblk, (unsigned)a.batch);
+      bwd_reference_kernel<T, NM><<<grid, kBwdThreads, smem, s>>>(a, w);
+      st = launch_status();
+    }
+    if (st == MAMBA_OK) {
+      const int64_t nbc = a.batch * a.N * a.L;
+      const int64_t g = std::min<int64_t>((nbc + 255) / 256, 148 * 16);
+      bwd_finalize_bc_kernel<T><<<(unsigned)g, 256, 0, s>>>(a, w);
+      st = launch_status();
+    }
+    if (st == MAMBA_OK) {
+      const int64_t np = a.dim * a.N;
+      const int64_t g = std::min<int64_t>((np + 255) / 256, 148 * 16);
+      bwd_finalize_params_kernel<<<(unsigned)g, 256, 0, s>>>(a, w);
+      st = launch_status();
+    }
+    if (cudaFreeAsync(ws, s) != cudaSuccess && st == MAMBA_OK) st = MAMBA_ERR_CUDA;
+    return st;
+  }
+};
+
+}  // namespace
+
+extern "C" {
+
+int mamba_scan_abi_version(void) { return kAbiVersion; }
+
+const char *mamba_scan_status_string(mamba_status_t s) {
+  switch (s) {
+    case MAMBA_OK: return "MAMBA_OK";
+    case MAMBA_ERR_INVALID_ARG: return "MAMBA_ERR_INVALID_ARG";
+    case MAMBA_ERR_UNSUPPORTED: return "MAMBA_ERR_UNSUPPORTED";
+    case MAMBA_ERR_CUDA: return "MAMBA_ERR_CUDA";
+    case MAMBA_ERR_OUT_OF_MEMORY: return "MAMBA_ERR_OUT_OF_MEMORY";
+    case MAMBA_ERR_DEVICE_TIMEOUT: return "MAMBA_ERR_DEVICE_TIMEOUT";
+  }
+  return "MAMBA_ERR_UNKNOWN";
+}
+
+mamba_status_t mamba_scan_stream_status(mamba_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return MAMBA_ERR_CUDA;
+  }
+  unsigned int word = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess ||
+      cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) {
+    cudaGetLastError();
+    return MAMBA_ERR_CUDA;
+  }
+  return (word & kErrTimeout) ? MAMBA_ERR_DEVICE_TIMEOUT : MAMBA_OK;
+}
+
+mamba_status_t mamba_scan_fwd_ex(const void *u, const void *delta, const float *delta_bias,
+                                 const float *A, const void *B, const void *C, const float *D,
+                                 const void *z, void *y, float *last_state, int64_t batch,
+                                 int64_t dim, int64_t L, int64_t N, mamba_dtype_t dtype,
+                                 const mamba_scan_options_t *options, mamba_stream_t stream) {
+  mamba_status_t st = check_shape(batch, dim, L, N, dtype);
+  if (st != MAMBA_OK) return st;
+  if ((st = check_options(options)) != MAMBA_OK) return st;
+  Checker ck;
+  if (cudaGetDevice(&ck.dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MAMBA_ERR_CUDA;
+  }
+  const size_t es = dtype_size(dtype);
+  const size_t nbdl = size_t(batch) * size_t(dim) * size_t(L);
+  const size_t nbnl = size_t(batch) * size_t(N) * size_t(L);
+  ck.buf(u, nbdl * es, es, true, false);
+  ck.buf(delta, nbdl * es, es, true, false);
+  ck.buf(z, nbdl * es, es, false, false);
+  ck.buf(B, nbnl * es, es, true, false);
+  ck.buf(C, nbnl * es, es, true, false);
+  ck.buf(A, size_t(dim) * N * 4, 4, true, false);
+  ck.buf(D, size_t(dim) * 4, 4, false, false);
+  ck.buf(delta_bias, size_t(dim) * 4, 4, false, false);
+  ck.buf(y, nbdl * es, es, true, true);
+  ck.buf(last_state, size_t(batch) * dim * N * 4, 4, false, true);
+  if (ck.st != MAMBA_OK) return ck.st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (batch == 0 || dim == 0) return MAMBA_OK;
+  if (L == 0) {
+    if (last_state && cudaMemsetAsync(last_state, 0, size_t(batch) * dim * N * 4, s) != cudaSuccess)
+      return launch_status();
+    return MAMBA_OK;
+  }
+  FwdArgs a;
+  a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
+  a.bias = delta_bias; a.A = A; a.D = D; a.y = y; a.last_state = last_state;
+  a.batch = batch; a.dim = dim; a.L = L; a.N = (int)N;
+  const int path = options ? options->path : MAMBA_PATH_AUTO;
+  const int chunk_len = options ? options->chunk_len : 0;
+  if (path == MAMBA_PATH_REFERENCE || !staged_supported(a, es)) {
+    if (path == MAMBA_PATH_GENERIC || path == MAMBA_PATH_STRUCTURED) return MAMBA_ERR_UNSUPPORTED;
+    return dispatch<FwdReferenceLauncher>(dtype, (int)N, a, s);
+  }
+  return dispatch<FwdStagedLauncher>(dtype, (int)N, a, path, chunk_len, s);
+}
+
+mamba_status_t mamba_scan_fwd(const void *u, const void *delta, const float *delta_bias,
+                              const float *A, const void *B, const void *C, const float *D,
+                              const void *z, void *y, float *last_state, int64_t batch,
+                              int64_t dim, int64_t L, int64_t N, mamba_dtype_t dtype,
+                              mamba_stream_t stream) {
+  return mamba_scan_fwd_ex(u, delta, delta_bias, A, B, C, D, z, y, last_state, batch, dim, L, N,
+                           dtype, nullptr, stream);
+}
+
+mamba_status_t mamba_scan_bwd_ex(const void *u, const void *delta, const float *delta_bias,
+                                 const float *A, const void *B, const void *C, const float *D,
+                                 const void *z, const void *dy, void *du, void *ddelta,
+                                 float *dA, void *dB, void *dC, float *dD, void *dz,
+                                 float *ddelta_bias, int64_t batch, int64_t dim, int64_t L,
+                                 int64_t N, mamba_dtype_t dtype,
+                                 const mamba_scan_options_t *options, mamba_stream_t stream) {
+  mamba_status_t st = check_shape(batch, dim, L, N, dtype);
+  if (st != MAMBA_OK) return st;
+  if ((st = check_options(options)) != MAMBA_OK) return st;
+  if ((z == nullptr) != (dz == nullptr) || (D == nullptr) != (dD == nullptr))
+    return MAMBA_ERR_INVALID_ARG;
+  Checker ck;
+  if (cudaGetDevice(&ck.dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MAMBA_ERR_CUDA;
+  }
+  const size_t es = dtype_size(dtype);
+  const size_t nbdl = size_t(batch) * size_t(dim) * size_t(L);
+  const size_t nbnl = size_t(batch) * size_t(N) * size_t(L);
+  ck.buf(u, nbdl * es, es, true, false);
+  ck.buf(delta, nbdl * es, es, true, false);
+  ck.buf(z, nbdl * es, es, false, false);
+  ck.buf(dy, nbdl * es, es, true, false);
+  ck.buf(B, nbnl * es, es, true, false);
+  ck.buf(C, nbnl * es, es, true, false);
+  ck.buf(A, size_t(dim) * N * 4, 4, true, false);
+  ck.buf(D, size_t(dim) * 4, 4, false, false);
+  ck.buf(delta_bias, size_t(dim) * 4, 4, false, false);
+  ck.buf(du, nbdl * es, es, true, true);
+  ck.buf(ddelta, nbdl * es, es, true, true);
+  ck.buf(dz, nbdl * es, es, false, true);
+  ck.buf(dB, nbnl * es, es, true, true);
+  ck.buf(dC, nbnl * es, es, true, true);
+  ck.buf(dA, size_t(dim) * N * 4, 4, true, true);
+  ck.buf(dD, size_t(dim) * 4, 4, false, true);
+  ck.buf(ddelta_bias, size_t(dim) * 4, 4, false, true);
+  if (ck.st != MAMBA_OK) return ck.st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (dim == 0) return MAMBA_OK;
+  if (batch == 0 || L == 0) {
+    // Empty sum: parameter gradients are zero, and dB / dC have no elements
+    // unless batch > 0 and L > 0.
+    if (cudaMemsetAsync(dA, 0, size_t(dim) * N * 4, s) != cudaSuccess) return launch_status();
+    if (dD && cudaMemsetAsync(dD, 0, size_t(dim) * 4, s) != cudaSuccess) return launch_status();
+    if (ddelta_bias && cudaMemsetAsync(ddelta_bias, 0, size_t(dim) * 4, s) != cudaSuccess)
+      return launch_status();
+    return MAMBA_OK;
+  }
+  BwdArgs a;
+  a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C; a.dy = dy;
+  a.bias = delta_bias; a.A = A; a.D = D;
+  a.du = du; a.ddelta = ddelta; a.dz = dz; a.dB = dB; a.dC = dC;
+  a.dA = dA; a.dD = dD; a.dbias = ddelta_bias;
+  a.batch = batch; a.dim = dim; a.L = L; a.N = (int)N;
+  const int path = options ? options->path : MAMBA_PATH_AUTO;
+  if (path == MAMBA_PATH_GENERIC || path == MAMBA_PATH_STRUCTURED) return MAMBA_ERR_UNSUPPORTED;
+  return dispatch<BwdReferenceLauncher>(dtype, (int)N, a, s);
+}
+
+mamba_status_t mamba_scan_bwd(const void *u, const void *delta, const float *delta_bias,
+                              const float *A, const void *B, const void *C, const float *D,
+                              const void *z, const void *dy, void *du, void *ddelta, float *dA,
+                              void *dB, void *dC, float *dD, void *dz, float *ddelta_bias,
+                              int64_t batch, int64_t dim, int64_t L, int64_t N,
+                              mamba_dtype_t dtype, mamba_stream_t stream) {
+  return mamba_scan_bwd_ex(u, delta, delta_bias, A, B, C, D, z, dy, du, ddelta, dA, dB, dC, dD,
+                           dz, ddelta_bias, batch, dim, L, N, dtype, nullptr, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,201 @@
+"""Python binding of libmambascan (ctypes).  Argument marshalling only: every
+step of the selective scan runs in the library's CUDA kernels.  There is no
+CPU fallback; a missing library or device raises.
+
+Low-level calls (same names and argument order as ``include/mamba_scan.h``):
+``mamba_scan_fwd``, ``mamba_scan_bwd``, ``mamba_scan_stream_status``.
+Convenience wrappers that allocate the outputs: ``selective_scan_fwd`` and
+``selective_scan_bwd``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libmambascan.so")
+
+MAMBA_F32, MAMBA_BF16 = 0, 1
+PATH_AUTO, PATH_REFERENCE, PATH_GENERIC, PATH_STRUCTURED = 0, 1, 2, 3
+PATHS = {"auto": PATH_AUTO, "reference": PATH_REFERENCE, "generic": PATH_GENERIC,
+         "structured": PATH_STRUCTURED}
+STATUS = {0: "MAMBA_OK", 1: "MAMBA_ERR_INVALID_ARG", 2: "MAMBA_ERR_UNSUPPORTED",
+          3: "MAMBA_ERR_CUDA", 4: "MAMBA_ERR_OUT_OF_MEMORY", 5: "MAMBA_ERR_DEVICE_TIMEOUT"}
+
+
+class MambaScanError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+class _Options(ctypes.Structure):
+    _fields_ = [("path", ctypes.c_int32), ("chunk_len", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 6)]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load libmambascan.so (built in-tree by ``selective_state_space_21_b200.build``)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise RuntimeError(
+                    f"libmambascan.so not found at {_LIB_PATH}; build it with "
+                    "`python -m selective_state_space_21_b200.build`")
+            lib = ctypes.CDLL(_LIB_PATH)
+            vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+            opt = ctypes.POINTER(_Options)
+            lib.mamba_scan_fwd.argtypes = [vp] * 10 + [i64] * 4 + [i32, vp]
+            lib.mamba_scan_fwd_ex.argtypes = [vp] * 10 + [i64] * 4 + [i32, opt, vp]
+            lib.mamba_scan_bwd.argtypes = [vp] * 17 + [i64] * 4 + [i32, vp]
+            lib.mamba_scan_bwd_ex.argtypes = [vp] * 17 + [i64] * 4 + [i32, opt, vp]
+            for f in ("mamba_scan_fwd", "mamba_scan_fwd_ex", "mamba_scan_bwd",
+                      "mamba_scan_bwd_ex", "mamba_scan_stream_status"):
+                getattr(lib, f).restype = ctypes.c_int
+            lib.mamba_scan_stream_status.argtypes = [vp]
+            lib.mamba_scan_status_string.argtypes = [ctypes.c_int]
+            lib.mamba_scan_status_string.restype = ctypes.c_char_p
+            lib.mamba_scan_abi_version.argtypes = []
+            lib.mamba_scan_abi_version.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.float32:
+        return MAMBA_F32
+    if t == torch.bfloat16:
+        return MAMBA_BF16
+    raise TypeError(f"unsupported I/O dtype {t} (float32 or bfloat16)")
+
+
+def _ptr(t: Optional[torch.Tensor], dtype=None, shape=None, name=""):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t.data_ptr() if t.numel() > 0 else None
+
+
+def _stream_handle(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if isinstance(stream, torch.cuda.Stream) else int(stream)
+
+
+def _options(path, chunk_len):
+    o = _Options()
+    o.path = PATHS[path] if isinstance(path, str) else int(path)
+    o.chunk_len = int(chunk_len)
+    return o
+
+
+def _check(rc: int, where: str):
+    if rc != 0:
+        raise MambaScanError(rc, where)
+
+
+def mamba_scan_fwd(u, delta, delta_bias, A, B, C, D, z, y, last_state, *, path="auto",
+                   chunk_len=0, stream=None):
+    """Enqueue the forward on ``stream`` (torch's current stream by default).
+    Tensors as in ``include/mamba_scan.h``; ``y`` (and ``last_state``) are
+    written."""
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    dt = u.dtype
+    f32 = torch.float32
+    args = [
+        _ptr(u, dt, (batch, dim, L), "u"), _ptr(delta, dt, (batch, dim, L), "delta"),
+        _ptr(delta_bias, f32, (dim,), "delta_bias"), _ptr(A, f32, (dim, N), "A"),
+        _ptr(B, dt, (batch, N, L), "B"), _ptr(C, dt, (batch, N, L), "C"),
+        _ptr(D, f32, (dim,), "D"), _ptr(z, dt, (batch, dim, L), "z"),
+        _ptr(y, dt, (batch, dim, L), "y"), _ptr(last_state, f32, (batch, dim, N), "last_state"),
+        batch, dim, L, N, _dtype_code(dt)]
+    lib = load_library()
+    if path == "auto" and not chunk_len:
+        rc = lib.mamba_scan_fwd(*args, _stream_handle(stream))
+    else:
+        rc = lib.mamba_scan_fwd_ex(*args, ctypes.byref(_options(path, chunk_len)),
+                                   _stream_handle(stream))
+    _check(rc, "mamba_scan_fwd")
+
+
+def mamba_scan_bwd(u, delta, delta_bias, A, B, C, D, z, dy, du, ddelta, dA, dB, dC, dD, dz,
+                   ddelta_bias, *, path="auto", chunk_len=0, stream=None):
+    """Enqueue the backward of sum(dy * y) on ``stream``; the gradient tensors
+    are written."""
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    dt = u.dtype
+    f32 = torch.float32
+    bdl, bnl = (batch, dim, L), (batch, N, L)
+    args = [
+        _ptr(u, dt, bdl, "u"), _ptr(delta, dt, bdl, "delta"),
+        _ptr(delta_bias, f32, (dim,), "delta_bias"), _ptr(A, f32, (dim, N), "A"),
+        _ptr(B, dt, bnl, "B"), _ptr(C, dt, bnl, "C"), _ptr(D, f32, (dim,), "D"),
+        _ptr(z, dt, bdl, "z"), _ptr(dy, dt, bdl, "dy"), _ptr(du, dt, bdl, "du"),
+        _ptr(ddelta, dt, bdl, "ddelta"), _ptr(dA, f32, (dim, N), "dA"),
+        _ptr(dB, dt, bnl, "dB"), _ptr(dC, dt, bnl, "dC"), _ptr(dD, f32, (dim,), "dD"),
+        _ptr(dz, dt, bdl, "dz"), _ptr(ddelta_bias, f32, (dim,), "ddelta_bias"),
+        batch, dim, L, N, _dtype_code(dt)]
+    lib = load_library()
+    if path == "auto" and not chunk_len:
+        rc = lib.mamba_scan_bwd(*args, _stream_handle(stream))
+    else:
+        rc = lib.mamba_scan_bwd_ex(*args, ctypes.byref(_options(path, chunk_len)),
+                                   _stream_handle(stream))
+    _check(rc, "mamba_scan_bwd")
+
+
+def mamba_scan_stream_status(stream=None) -> int:
+    """Synchronize the stream and return (and clear) the sticky device status."""
+    return load_library().mamba_scan_stream_status(_stream_handle(stream))
+
+
+def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
+                       return_last_state=False, path="auto", chunk_len=0, stream=None):
+    """Allocate y (and last_state) and run the forward; returns y or (y, last_state)."""
+    batch, dim, L = u.shape
+    y = torch.empty_like(u)
+    last = (torch.empty(batch, dim, A.shape[1], device=u.device, dtype=torch.float32)
+            if return_last_state else None)
+    mamba_scan_fwd(u, delta, delta_bias, A, B, C, D, z, y, last, path=path,
+                   chunk_len=chunk_len, stream=stream)
+    return (y, last) if return_last_state else y
+
+
+def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, path="auto",
+                       chunk_len=0, stream=None) -> dict:
+    """Allocate the gradients and run the backward; returns a dict of them."""
+    dim, N = A.shape
+    f32 = torch.float32
+    g = {
+        "du": torch.empty_like(u), "ddelta": torch.empty_like(u),
+        "dA": torch.empty(dim, N, device=u.device, dtype=f32),
+        "dB": torch.empty_like(B), "dC": torch.empty_like(C),
+        "dD": torch.empty(dim, device=u.device, dtype=f32) if D is not None else None,
+        "dz": torch.empty_like(u) if z is not None else None,
+        "ddelta_bias": torch.empty(dim, device=u.device, dtype=f32),
+    }
+    mamba_scan_bwd(u, delta, delta_bias, A, B, C, D, z, dy, g["du"], g["ddelta"], g["dA"],
+                   g["dB"], g["dC"], g["dD"], g["dz"], g["ddelta_bias"], path=path,
+                   chunk_len=chunk_len, stream=stream)
+    return {k: v for k, v in g.items() if v is not None}

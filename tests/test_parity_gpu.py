@@ -1,0 +1,267 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded inputs.  Normwise max error <= 1e-4 for fp32 I/O and <= 2e-2 for
+bf16 I/O (fp32 state and accumulation)."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import gpu_cases as gc
+from selective_state_space_21_b200 import build, scan
+from selective_state_space_21_b200.inputs import (WORKLOADS, gated_case, lti_case, make_inputs,
+                                                  workload_inputs)
+
+pytestmark = pytest.mark.gpu
+
+PATHS = ["auto", "reference"]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    build.build()
+    scan.load_library()
+
+
+def _fwd_case(x_host, path="auto", chunk_len=0):
+    x = gc.to_device(x_host)
+    y, last = gc.gpu_fwd(x, path=path, chunk_len=chunk_len)
+    y_ref, last_ref = gc.oracle_fwd(x_host)
+    tol = gc.TOL[x_host["u"].dtype]
+    ey = gc.normwise(y.cpu().double().numpy(), y_ref)
+    el = gc.normwise(last.cpu().double().numpy(), last_ref)
+    assert ey <= tol and el <= max(tol, 1e-4), f"y err {ey:.2e}, last_state err {el:.2e}"
+    return ey, el
+
+
+# ------------------------------------------------------------- forward, small
+
+@pytest.mark.parametrize("path", PATHS)
+def test_fwd_tiny_workload(path):
+    _fwd_case(workload_inputs(0), path)
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_fwd_theorem1_gated_case(path):
+    _fwd_case(gated_case(L=64, dim=4), path)
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_fwd_lti_case(path):
+    _fwd_case(lti_case(batch=1, dim=4, L=64, N=4), path)
+
+
+GRID = [  # (batch, dim, L, N) -- several tiles plus ragged tails in dim and L
+    (2, 200, 1000, 16), (1, 130, 4099, 16), (3, 7, 65, 3), (2, 64, 512, 8), (1, 33, 257, 1),
+]
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("shape", GRID, ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("path", PATHS)
+def test_fwd_grid(shape, dtype, path):
+    b, d, L, N = shape
+    _fwd_case(make_inputs(b, d, L, N, dtype, seed=100 + L), path)
+
+
+@pytest.mark.parametrize("has_z,has_D,has_bias", [(False, False, False), (True, False, True),
+                                                   (False, True, False)])
+def test_fwd_optional_inputs(has_z, has_D, has_bias):
+    x = make_inputs(2, 96, 300, 16, torch.float32, seed=5, has_z=has_z, has_D=has_D)
+    if not has_bias:
+        x["delta_bias"] = None
+    _fwd_case(x)
+
+
+def test_fwd_generic_A():
+    """A that is not of the S4D-Real form (random negative diagonal)."""
+    x = make_inputs(2, 100, 700, 16, torch.float32, seed=6)
+    g = torch.Generator().manual_seed(9)
+    x["A"] = -torch.exp(torch.randn(100, 16, generator=g))
+    _fwd_case(x)
+
+
+# -------------------------------------------------- forward, full workloads
+
+@pytest.mark.parametrize("index", [1, 2, 3], ids=lambda i: WORKLOADS[i].name)
+def test_fwd_full_workload_sampled(index):
+    """The full-size workloads in the launch configuration the benchmark
+    times (auto path), checked on sampled channels over their full length."""
+    w = WORKLOADS[index]
+    x = workload_inputs(index, device="cuda", with_dy=False)
+    y, last = gc.gpu_fwd(x)
+    k = 12 if w.L > 100_000 else 48
+    ey, el = gc.check_fwd_sampled(x, y, last, k=k, seed=index)
+    tol = gc.TOL[w.dtype]
+    assert ey <= tol and el <= tol, f"{w.name}: y err {ey:.2e}, last_state err {el:.2e}"
+    assert torch.isfinite(y).all()
+
+
+# ------------------------------------------------------------------ backward
+
+GRAD_KEYS = ["du", "ddelta", "dz", "dA", "dB", "dC", "dD", "ddelta_bias"]
+
+
+def _bwd_case(x_host, path="auto"):
+    x = gc.to_device(x_host)
+    g = gc.gpu_bwd(x, path=path)
+    ref = gc.oracle_bwd(x_host)
+    tol = gc.TOL[x_host["u"].dtype]
+    errs = {}
+    for k in GRAD_KEYS:
+        if k in ref and k in g:
+            errs[k] = gc.normwise(g[k].cpu().double().numpy(), ref[k])
+    bad = {k: v for k, v in errs.items() if not v <= tol}
+    assert not bad, f"gradient errors above {tol}: {bad} (all: {errs})"
+    return errs
+
+
+def test_bwd_tiny_workload():
+    _bwd_case(workload_inputs(0))
+
+
+def test_bwd_theorem1_gated_case():
+    _bwd_case(gated_case(L=64, dim=4))
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("shape", [(2, 100, 333, 16), (1, 70, 1025, 8), (2, 5, 40, 1)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_bwd_grid(shape, dtype):
+    b, d, L, N = shape
+    _bwd_case(make_inputs(b, d, L, N, dtype, seed=200 + L, with_dy=True))
+
+
+def test_bwd_full_workload_sampled():
+    """Forward + recompute backward at the full bf16 4 x 2048 x 4096 size:
+    per-channel gradients on sampled channels, dB / dC on one full batch row
+    (they sum over all channels), dA / dD / dbias on sampled channels."""
+    index = 4
+    w = WORKLOADS[index]
+    x = workload_inputs(index, device="cuda")
+    y, last = gc.gpu_fwd(x)
+    ey, el = gc.check_fwd_sampled(x, y, last, k=16, seed=index)
+    assert ey <= gc.TOL[w.dtype] and el <= gc.TOL[w.dtype]
+    g = gc.gpu_bwd(x)
+    gh = {k: v.cpu() for k, v in g.items()}
+    xh = gc.to_host(x)
+    tol = gc.TOL[w.dtype]
+    # one full batch row for the channel-summed dB, dC
+    b = w.batch - 1
+    row = gc.sub_problem(xh, b, list(range(w.dim)))
+    ref = gc.oracle_bwd(row)
+    for k in ("dB", "dC"):
+        e = gc.normwise(gh[k][b].double().numpy(), ref[k][0])
+        assert e <= tol, f"{k}: {e:.2e}"
+    samples = gc.sample_channels(w.batch, w.dim, 16, seed=7)
+    for bb, ds in samples.items():
+        idx = torch.tensor(ds)
+        if bb == b:
+            r = {k: v[0][ds] for k, v in ref.items() if k in ("du", "ddelta", "dz")}
+        else:
+            r = {k: v[0] for k, v in gc.oracle_bwd(gc.sub_problem(xh, bb, ds)).items()
+                 if k in ("du", "ddelta", "dz")}
+        for k, v in r.items():
+            e = gc.normwise(gh[k][bb].index_select(0, idx).double().numpy(), v)
+            assert e <= tol, f"{k} (batch {bb}): {e:.2e}"
+    # parameter gradients sum over the batch: all rows for a few channels
+    ds = [0, 1, 777, w.dim - 1]
+    idx = torch.tensor(ds)
+    sub = {k: (v.index_select(1, idx).contiguous() if k in ("u", "delta", "z", "dy") else v)
+           for k, v in xh.items()}
+    sub.update(A=xh["A"][idx].contiguous(), D=xh["D"][idx].contiguous(),
+               delta_bias=xh["delta_bias"][idx].contiguous())
+    pref = gc.oracle_bwd(sub)
+    for k in ("dA", "dD", "ddelta_bias"):
+        e = gc.normwise(gh[k].index_select(0, idx).double().numpy(), pref[k])
+        assert e <= tol, f"{k}: {e:.2e}"
+
+
+# ----------------------------------------------------------------- contract
+
+def test_fwd_deterministic_and_overwrites_nan():
+    x = gc.to_device(make_inputs(2, 150, 600, 16, torch.bfloat16, seed=3))
+    y1 = torch.full_like(x["u"], float("nan"))
+    last1 = torch.full((2, 150, 16), float("nan"), device="cuda")
+    scan.mamba_scan_fwd(x["u"], x["delta"], x["delta_bias"], x["A"], x["B"], x["C"], x["D"],
+                        x["z"], y1, last1)
+    y2, last2 = gc.gpu_fwd(x)
+    assert torch.isfinite(y1.float()).all() and torch.isfinite(last1).all()
+    assert torch.equal(y1, y2) and torch.equal(last1, last2)
+
+
+def test_bwd_deterministic():
+    x = gc.to_device(make_inputs(2, 150, 300, 16, torch.bfloat16, seed=4, with_dy=True))
+    g1, g2 = gc.gpu_bwd(x), gc.gpu_bwd(x)
+    for k in g1:
+        assert torch.equal(g1[k], g2[k]), k
+
+
+def test_guard_bands_untouched():
+    x = gc.to_device(make_inputs(1, 40, 128, 16, torch.float32, seed=8))
+    n = x["u"].numel()
+    buf = torch.full((n + 2048,), 7.0, device="cuda")
+    y = buf[1024:1024 + n].view_as(x["u"])
+    scan.mamba_scan_fwd(x["u"], x["delta"], x["delta_bias"], x["A"], x["B"], x["C"], x["D"],
+                        x["z"], y, None)
+    torch.cuda.synchronize()
+    assert (buf[:1024] == 7.0).all() and (buf[1024 + n:] == 7.0).all()
+    y_ref, _ = gc.oracle_fwd(gc.to_host(x))
+    assert gc.normwise(y.cpu().double().numpy(), y_ref) <= 1e-4
+
+
+def test_empty_and_degenerate_shapes():
+    # L = 0: last_state is the initial state 0
+    x = gc.to_device(make_inputs(2, 3, 0, 4, torch.float32))
+    y, last = gc.gpu_fwd(x)
+    assert y.numel() == 0 and torch.equal(last, torch.zeros_like(last))
+    # batch = 0 and dim = 0 are accepted and do nothing
+    for b, d in ((0, 3), (2, 0)):
+        xe = gc.to_device(make_inputs(b, d, 16, 4, torch.float32))
+        ye, _ = gc.gpu_fwd(xe)
+        assert ye.numel() == 0
+    # L = 0 backward: parameter gradients are 0
+    x = gc.to_device(make_inputs(2, 3, 0, 4, torch.float32, with_dy=True))
+    g = gc.gpu_bwd(x)
+    assert torch.equal(g["dA"], torch.zeros_like(g["dA"]))
+    # L = 1
+    _fwd_case(make_inputs(3, 9, 1, 16, torch.float32, seed=2))
+
+
+def _raw_fwd(u_ptr, y_ptr, batch=1, dim=2, L=8, N=4, dtype=0, A_ptr=None, B_ptr=None):
+    lib = scan.load_library()
+    return lib.mamba_scan_fwd(u_ptr, u_ptr, None, A_ptr, B_ptr, B_ptr, None, None, y_ptr, None,
+                              batch, dim, L, N, dtype, None)
+
+
+def test_invalid_arguments_are_rejected_on_the_host():
+    u = torch.zeros(1, 2, 8, device="cuda")
+    y = torch.zeros(1, 2, 8, device="cuda")
+    A = -torch.ones(2, 4, device="cuda")
+    B = torch.zeros(1, 4, 8, device="cuda")
+    host = np.zeros(16, np.float32)
+    ok = _raw_fwd(u.data_ptr(), y.data_ptr(), A_ptr=A.data_ptr(), B_ptr=B.data_ptr())
+    assert ok == 0
+    # host pointer for an input
+    assert _raw_fwd(host.ctypes.data, y.data_ptr(), A_ptr=A.data_ptr(), B_ptr=B.data_ptr()) == 1
+    # output overlapping an input
+    assert _raw_fwd(u.data_ptr(), u.data_ptr(), A_ptr=A.data_ptr(), B_ptr=B.data_ptr()) == 1
+    # missing required pointer
+    assert _raw_fwd(u.data_ptr(), y.data_ptr(), A_ptr=None, B_ptr=B.data_ptr()) == 1
+    # misaligned fp32 pointer
+    assert _raw_fwd(u.data_ptr() + 2, y.data_ptr(), A_ptr=A.data_ptr(), B_ptr=B.data_ptr()) == 1
+    # N outside 1..16, bad dtype, negative size
+    A17 = -torch.ones(2, 17, device="cuda")
+    B17 = torch.zeros(1, 17, 8, device="cuda")
+    assert _raw_fwd(u.data_ptr(), y.data_ptr(), N=17, A_ptr=A17.data_ptr(),
+                    B_ptr=B17.data_ptr()) == 2
+    assert _raw_fwd(u.data_ptr(), y.data_ptr(), dtype=7, A_ptr=A.data_ptr(),
+                    B_ptr=B.data_ptr()) == 1
+    assert _raw_fwd(u.data_ptr(), y.data_ptr(), L=-1, A_ptr=A.data_ptr(),
+                    B_ptr=B.data_ptr()) == 1
+    assert scan.mamba_scan_stream_status() == 0
+    # nothing was launched by the rejected calls: y still zero from the good call's input
+    torch.cuda.synchronize()
+    assert torch.isfinite(y).all()
