@@ -1,0 +1,482 @@
+#!/usr/bin/env python
+"""Benchmark of the fused selective scan (S6) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = the whole hot path over one batch of synthetic input: the forward
+(softplus, zero-order-hold discretization, scan, C readout, D skip, SiLU gate,
+store) and the recompute-based backward of sum(dy * y), on the bf16-I/O
+workload of batch 8, 5120 channels, 2048 steps and N = 16 (fp32 state and
+arithmetic).  Inputs are resident in HBM when the timed region starts and each
+of u, delta, z, dy (168 MB) is larger than the 126 MB L2, so every step reads
+them from DRAM.  Device time comes from CUDA events on the launching stream;
+for N > 1 (torchrun, one process per GPU) every rank runs its own independent
+batch (weak scaling, no data-path collective) and the step time is the max
+over ranks.
+
+Rank 0 prints one JSON line.  ``--impl reference`` times the fp64 CPU oracle
+on the host cores instead (bounded channel samples of the same workload).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from selective_state_space_21_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = ("selective-scan fwd/bwd GB/s and token·channels/s vs B200 HBM roofline (1 GPU)")
+UNIT = "token·channels/s"
+DEFAULT_WORKLOAD = 2
+FALLBACK_HBM_GBS = 6650.0
+
+
+# --------------------------------------------------------------- accounting
+
+def fwd_bytes(w, last_state=False) -> int:
+    """Algorithmic bytes of one forward: read u, delta, z and write y (4 s per
+    token-channel), read the B and C rows, the parameters, and write
+    last_state if asked."""
+    s = w.io_bytes
+    tc = w.token_channels
+    b = 4 * s * tc + 2 * w.batch * w.N * w.L * s + 4 * (w.dim * w.N + 2 * w.dim)
+    return b + (4 * w.batch * w.dim * w.N if last_state else 0)
+
+
+def bwd_bytes(w) -> int:
+    """Algorithmic bytes of one backward: read u, delta, z, dy and write du,
+    ddelta, dz (7 s per token-channel), read B, C and write dB, dC, read A, D,
+    bias and write dA, dD, dbias."""
+    s = w.io_bytes
+    tc = w.token_channels
+    return 7 * s * tc + 4 * w.batch * w.N * w.L * s + 8 * (w.dim * w.N + 2 * w.dim)
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "source": "fallback"}
+
+
+def ncu_traffic(kernel_key: str):
+    """Per-launch DRAM bytes from a committed ncu summary, only if it was taken
+    on the current source of that kernel (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        e = d[kernel_key]
+        from selective_state_space_21_b200.build import source_digest
+        if e.get("source_digest") != source_digest():
+            return None
+        return e
+    except Exception:
+        return None
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.idx = device_index
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _sample(self):
+        nv = self.nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+        try:
+            mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            mask = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        for name, bit in self.REASONS.items():
+            if mask & bit and name != "gpu_idle":
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._t is not None:
+            self._stop.set()
+            self._t.join()
+            try:
+                self._sample()
+            except Exception:
+                pass
+
+    def summary(self) -> dict:
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [],
+                    "source": "unavailable"}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml"}
+
+
+# ------------------------------------------------------------- distributed
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(value: float, device) -> float:
+    """Max of a per-rank scalar over all ranks (identity with one rank)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def shard_seed(base_seed: int, rank: int) -> int:
+    """Each rank draws its own independent batch (weak scaling)."""
+    return base_seed + 1000 * rank
+
+
+def whole_job_rate(units_per_rank: float, world: int, max_seconds: float) -> float:
+    return units_per_rank * world / max_seconds
+
+
+# ------------------------------------------------------------- CPU oracle
+
+def oracle_sample_rate(x_host: dict, w, seconds: float = 10.0, min_blocks: int = 1):
+    """Time the fp64 oracle (forward + backward, as it stands) on channel
+    blocks of batch row 0 until `seconds` elapse; returns (tc/s, threads,
+    description)."""
+    import oracle
+    threads = oracle.default_threads()
+    k = max(8, 2 * threads)
+    done_tc = 0
+    blocks = 0
+    t0 = time.perf_counter()
+    d0 = 0
+    while True:
+        ds = [(d0 + i) % w.dim for i in range(k)]
+        d0 = (d0 + k) % w.dim
+        idx = torch.tensor(ds)
+        sub = {n: (x_host[n][0:1].index_select(1, idx).contiguous() if x_host[n] is not None
+                   else None) for n in ("u", "delta", "z", "dy")}
+        sub.update(B=x_host["B"][0:1].contiguous(), C=x_host["C"][0:1].contiguous(),
+                   A=x_host["A"][idx].contiguous(),
+                   D=None if x_host["D"] is None else x_host["D"][idx].contiguous(),
+                   delta_bias=x_host["delta_bias"][idx].contiguous())
+        oracle.s6_forward(sub["u"], sub["delta"], sub["A"], sub["B"], sub["C"],
+                          sub["delta_bias"], sub["D"], sub["z"], nthreads=threads)
+        oracle.s6_backward(sub["u"], sub["delta"], sub["A"], sub["B"], sub["C"], sub["dy"],
+                           sub["delta_bias"], sub["D"], sub["z"], nthreads=threads)
+        done_tc += k * w.L
+        blocks += 1
+        el = time.perf_counter() - t0
+        if el >= seconds and blocks >= min_blocks:
+            break
+    desc = (f"forward + backward of {blocks} blocks of {k} channels of batch row 0 "
+            f"(full L = {w.L}) of {w.name}: {blocks * k} of {w.batch * w.dim} channels, "
+            f"{el:.1f} s on {threads} threads")
+    return done_tc / el, threads, desc
+
+
+# ------------------------------------------------------------------- arms
+
+def run_ours(args, world, rank, device):
+    from selective_state_space_21_b200 import scan
+
+    w = WORKLOADS[args.workload]
+    x = make_inputs(w.batch, w.dim, w.L, w.N, w.dtype, device=device,
+                    seed=shard_seed(1234 + args.workload, rank), has_z=w.has_z,
+                    has_D=w.has_D, with_dy=True)
+    y = torch.empty_like(x["u"])
+    g = {"du": torch.empty_like(x["u"]), "ddelta": torch.empty_like(x["u"]),
+         "dz": torch.empty_like(x["u"]),
+         "dA": torch.empty(w.dim, w.N, device=device), "dB": torch.empty_like(x["B"]),
+         "dC": torch.empty_like(x["C"]), "dD": torch.empty(w.dim, device=device),
+         "dbias": torch.empty(w.dim, device=device)}
+
+    def fwd():
+        scan.mamba_scan_fwd(x["u"], x["delta"], x["delta_bias"], x["A"], x["B"], x["C"],
+                            x["D"], x["z"], y, None)
+
+    def bwd():
+        scan.mamba_scan_bwd(x["u"], x["delta"], x["delta_bias"], x["A"], x["B"], x["C"],
+                            x["D"], x["z"], x["dy"], g["du"], g["ddelta"], g["dA"], g["dB"],
+                            g["dC"], g["dD"], g["dz"], g["dbias"])
+
+    do_fwd = args.only in (None, "fwd")
+    do_bwd = args.only in (None, "bwd")
+    for _ in range(args.warmup):
+        if do_fwd:
+            fwd()
+        if do_bwd:
+            bwd()
+    torch.cuda.synchronize(device)
+    if scan.mamba_scan_stream_status() != 0:
+        raise RuntimeError("device error during warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = scan.launch_count()
+    sampler = ClockSampler(device.index if device.index is not None else 0)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    with sampler:
+        start.record()
+        for k in range(K):
+            ev[k][0].record()
+            if do_fwd:
+                fwd()
+            ev[k][1].record()
+            if do_bwd:
+                bwd()
+            ev[k][2].record()
+        end.record()
+        torch.cuda.synchronize(device)
+    barrier(device)
+    launches = scan.launch_count() - launches0
+    status = scan.mamba_scan_stream_status()
+    if status != 0:
+        raise RuntimeError(f"device error in the timed region: {status}")
+    total_ms = start.elapsed_time(end)
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    step_ms_local = total_ms / K
+    step_ms = max_over_ranks(step_ms_local, device)
+    fwd_ms_max = max_over_ranks(fwd_ms, device)
+    bwd_ms_max = max_over_ranks(bwd_ms, device)
+
+    peaks = measured_peaks()
+    peak = peaks["hbm_gbs"]
+    fb, bb = fwd_bytes(w), bwd_bytes(w)
+
+    def roof(name, nbytes, ms, kernels):
+        ach = nbytes / (ms * 1e-3) / 1e9
+        tr = ncu_traffic(name)
+        return {"bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(ach / peak, 4), "traffic": tr["bytes_per_launch"] if tr else None,
+                "kernel": name, "launch_group": kernels, "bytes_per_launch": nbytes,
+                "peak_source": f"{peaks['source']} hbm_gbs (copy bandwidth)",
+                "ms_per_launch": round(ms, 4)}
+
+    roof_fwd = roof("fwd", fb, fwd_ms_max, "mamba_scan_fwd call")
+    roof_bwd = roof("bwd", bb, bwd_ms_max, "mamba_scan_bwd call")
+    dominant = roof_bwd if bwd_ms_max >= fwd_ms_max else roof_fwd
+
+    tc_step = w.token_channels
+    value = whole_job_rate(tc_step, world, step_ms * 1e-3)
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(step_ms, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded N(0,1) u, delta, z, B, C, D, dy; log-uniform dt bias; "
+                "A = -(n+1))",
+        "config": {"workload": f"{w.name} (forward + recompute backward per step)",
+                   "batch": w.batch, "dim": w.dim, "L": w.L, "N": w.N, "io_dtype": "bf16",
+                   "state_dtype": "f32", "global_batch": w.batch * world,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (u, delta, z, dy 168 MB each; L2 126 MB)"},
+        "gbs": round((fb + bb) / (step_ms * 1e-3) / 1e9 * world, 1),
+        "fwd": {"ms": round(fwd_ms_max, 4), "tc_per_s": tc_step * world / (fwd_ms_max * 1e-3),
+                "gbs": roof_fwd["achieved"], "frac_hbm": roof_fwd["frac"]},
+        "bwd": {"ms": round(bwd_ms_max, 4), "tc_per_s": tc_step * world / (bwd_ms_max * 1e-3),
+                "gbs": roof_bwd["achieved"], "frac_hbm": roof_bwd["frac"]},
+        "roofline": dominant, "roofline_fwd": roof_fwd,
+        "gpu_launches": launches, "clocks": sampler.summary(),
+    }
+
+    if args.only:
+        result["note"] = f"--only {args.only}: a profiling run, not a benchmark result"
+    if not args.no_e2e and not args.only:
+        result["e2e"] = run_e2e(args, w, x, y, g, fwd, bwd, device, world)
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.only:
+        xh = {k: (v.cpu() if torch.is_tensor(v) else v) for k, v in x.items()}
+        rate, threads, desc = oracle_sample_rate(xh, w, seconds=args.cpu_seconds)
+        result["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": threads,
+                                  "kind": "oracle", "sample": desc}
+    return result
+
+
+def run_e2e(args, w, x, y, g, fwd, bwd, device, world):
+    """Same step through the public API with host buffers: each step copies its
+    inputs from pinned host memory to the device and reads every result back."""
+    names_in = ["u", "delta", "z", "B", "C", "A", "D", "delta_bias", "dy"]
+    host_in = {k: x[k].cpu().pin_memory() for k in names_in}
+    outs = {"y": y, **g}
+    host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in outs.items()}
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+
+    def step():
+        for k in names_in:
+            x[k].copy_(host_in[k], non_blocking=True)
+        fwd()
+        bwd()
+        for k, v in outs.items():
+            host_out[k].copy_(v, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize(device)
+    K = max(3, min(args.steps, 10))
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(device)
+    s.record()
+    for _ in range(K):
+        step()
+    e.record()
+    torch.cuda.synchronize(device)
+    barrier(device)
+    ms = max_over_ranks(s.elapsed_time(e) / K, device)
+    return {"value": w.token_channels * world / (ms * 1e-3), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3),
+            "steps": K}
+
+
+def run_reference(args, world, rank):
+    """The fp64 CPU oracle as it stands, on the host cores, over bounded channel
+    samples of the same workload (one sample per step)."""
+    import oracle
+    w = WORKLOADS[args.workload]
+    x = make_inputs(w.batch, w.dim, w.L, w.N, w.dtype, device="cpu",
+                    seed=1234 + args.workload, has_z=w.has_z, has_D=w.has_D, with_dy=True)
+    threads = oracle.default_threads()
+    k = max(8, 2 * threads)
+
+    def step(d0):
+        idx = torch.tensor([(d0 + i) % w.dim for i in range(k)])
+        sub = {n: x[n][0:1].index_select(1, idx).contiguous() for n in ("u", "delta", "z", "dy")}
+        A, D, bias = x["A"][idx].contiguous(), x["D"][idx].contiguous(), \
+            x["delta_bias"][idx].contiguous()
+        oracle.s6_forward(sub["u"], sub["delta"], A, x["B"][0:1], x["C"][0:1], bias, D,
+                          sub["z"], nthreads=threads)
+        oracle.s6_backward(sub["u"], sub["delta"], A, x["B"][0:1], x["C"][0:1], sub["dy"],
+                           bias, D, sub["z"], nthreads=threads)
+
+    for i in range(args.warmup):
+        step(i * k)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step((args.warmup + i) * k)
+    el = time.perf_counter() - t0
+    per = el / args.steps
+    value = k * w.L / per
+    desc = (f"each step: forward + backward of {k} channels of batch row 0 (full L = {w.L}) "
+            f"of {w.name}")
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(per * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{w.name} (forward + recompute backward per step)",
+                   "batch": w.batch, "dim": w.dim, "L": w.L, "N": w.N, "io_dtype": "bf16"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD,
+                    help="index into the workload list (default: the bf16 2K-length one)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--only", choices=["fwd", "bwd"], default=None,
+                    help="time one pass only (for profiling; not a benchmark result)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, world, rank)), flush=True)
+        return 0
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+    try:
+        result = run_ours(args, world, rank, device)
+        if rank == 0:
+            print(json.dumps(result), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -87,10 +87,17 @@ typedef enum {
 } mamba_path_t;
 
 typedef struct {
-  int32_t path;        /* a mamba_path_t */
-  int32_t chunk_len;   /* time steps per chunk of the chunked kernels; 0 = automatic.
-                          Must be a positive multiple of 64 when set. */
-  int32_t reserved[6]; /* must be 0 */
+  int32_t path;            /* a mamba_path_t */
+  int32_t chunk_len;       /* time steps per chunk of the chunked kernels; 0 = automatic,
+                              else a positive multiple of 64 */
+  int32_t carry;           /* how a chunk's end state reaches the next chunk: 0 = automatic,
+                              1 = sequential hand-off (a bounded wait on the predecessor),
+                              2 = three-phase (aggregate, scan over chunks, recompute) */
+  int32_t wait_timeout_us; /* bound of every device-side wait; 0 = 2,000,000 (2 s) */
+  int32_t test_hook;       /* 0 in normal use.  1: the first chunk of the first channel
+                              group never publishes its end state, so that the waits on it
+                              expire (tests MAMBA_ERR_DEVICE_TIMEOUT; outputs undefined) */
+  int32_t reserved[3];     /* must be 0 */
 } mamba_scan_options_t;
 
 /*
@@ -150,6 +157,10 @@ MAMBA_SCAN_API mamba_status_t mamba_scan_stream_status(mamba_stream_t stream);
 
 /* Static, human-readable name of a status code (never NULL). */
 MAMBA_SCAN_API const char *mamba_scan_status_string(mamba_status_t status);
+
+/* Number of CUDA kernels this library has launched in this process (all
+ * devices, all threads), for accounting in benchmarks. */
+MAMBA_SCAN_API uint64_t mamba_scan_launch_count(void);
 
 /* Version of this ABI (incremented on any incompatible change). */
 MAMBA_SCAN_API int mamba_scan_abi_version(void);

@@ -34,6 +34,18 @@ def deps():
         os.path.join(ROOT, "include", "mamba_scan.h")]
 
 
+def source_digest() -> str:
+    """Short hash of every source the library is built from (used to tell
+    whether a stored profile still describes the current kernels)."""
+    import hashlib
+    h = hashlib.sha256()
+    for p in deps():
+        h.update(os.path.basename(p).encode())
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def stale() -> bool:
     if not os.path.exists(LIB):
         return True

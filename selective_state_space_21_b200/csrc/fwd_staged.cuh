@@ -1,15 +1,792 @@
-// fwd_staged.cuh -- staged, chunked forward kernels (sm_100a).
+// fwd_staged.cuh -- the staged, chunked forward of the selective scan for
+// sm_100a.
+//
+// What it computes is the forward of Knowl 1 "Selective State Space Layer
+// (S6)" ("Mamba: Linear-Time Sequence Modeling with Selective State Spaces",
+// chapterpal.com) plus softplus on Delta, the D skip and the SiLU gate.  How it
+// is organised for B200:
+//
+//  * One thread owns one (batch, channel) and keeps its N <= 16 fp32 states in
+//    registers for the whole chunk; the expanded (B, L, D, N) tensors never
+//    exist anywhere (the fusion of section 3.3 of the paper-graph-ui page).
+//  * A CTA is 128 channels of one batch row.  TMA streams 64-byte-per-channel
+//    time tiles of u, delta and z (swizzled so that each thread reads its own
+//    row without bank conflicts) and the matching B and C rows through a
+//    3-stage mbarrier pipeline; y leaves through a TMA store.  Only u, delta,
+//    z, B, C, the parameters, y and the final state touch HBM.
+//  * Work is split into units = (channel group, time chunk) handed out by a
+//    ticket counter to persistent CTAs.  The state crosses chunk boundaries in
+//    one of two ways (the chunking of section 3.3, "Handling long sequences
+//    with chunking"):
+//      - SEQ: chunk k of a group waits (bounded) for chunk k-1 to publish its
+//        end state; tickets are issued chunk-major, so the predecessor was
+//        claimed earlier by a running CTA and the wait always ends.  Used when
+//        there are enough channel groups to fill the GPU.
+//      - PAR: an aggregate pass computes, for every chunk but the last, the
+//        state it produces from zero and the sum of its Delta; a small kernel
+//        scans those across chunks (the associative combine of affine maps,
+//        the total decay of a chunk being exp(A * sum Delta)); the main pass
+//        then runs every chunk from its true initial state.  Used for few
+//        channels and long sequences.
+//  * Arithmetic.  For channels whose A has the S4D-Real structure
+//    A[d,n] = (n+1) A[d,0] < 0, the decays of all states follow from one
+//    expm1 per (t, channel): with E(j) = expm1(j x), x = Delta A[d,0], the
+//    doubling relation E(m+k) = E(m) + exp(m x) E(k) gives E(1..16) in 15
+//    FMAs.  The zero-order-hold update is then
+//        h_n <- h_n + E(n+1) (h_n + B_n/(n+1) * u/A[d,0]),
+//    which equals Abar h + Bbar u with Abar = 1 + E(n+1) and
+//    Bbar = E(n+1)/A_n B.  When A[d,0] = -1, exp(-softplus(v)) = sigma(-v)
+//    (the identity in the proof of Theorem 1, Knowl 4 of the same page), so
+//    no log or expm1 is needed at all.  Other channels take the generic
+//    arithmetic: one exp per state element and Bbar/B = Delta psi(Delta A)
+//    with a series for small arguments.  Both use packed fma.rn.f32x2 where
+//    the work pairs up.
 #pragma once
+
+#include <algorithm>
+#include <type_traits>
+
 #include "../../include/mamba_scan.h"
 #include "common.cuh"
+#include "tma.cuh"
 
 namespace mscan {
 
-inline bool staged_supported(const FwdArgs &a, size_t es) { return false; }
+constexpr int kSThreads = 128;
+constexpr int kStages = 3;
+constexpr int kRowBytes = 64;
+constexpr int kTileBytes = kSThreads * kRowBytes;     // 8 KB per (u | delta | z | y) tile
+constexpr int kRawBytes = kMaxN * kRowBytes;          // 1 KB per B / C tile
+constexpr int kStageBytes = 3 * kTileBytes + 2 * kRawBytes;
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
+
+enum StagedKind { KIND_SEQ = 0, KIND_PAR = 1, KIND_AGG = 2 };
+enum UnitMode { MODE_SIG = 0, MODE_STRUCT = 1, MODE_GEN = 2 };
+
+struct StagedArgs {
+  FwdArgs f;
+  int G;           // channel groups (batch rows x groups per row)
+  int gpb;         // groups per batch row
+  int K;           // chunks per group
+  int chunk_len;   // time steps per chunk (a multiple of the tile length)
+  int n_units;     // units handled by this launch
+  int *counter;    // ticket counter, zero before the launch
+  int *flags;      // SEQ: per group, number of chunks whose end state is published
+  float *carry;    // SEQ: [G][NM][128] state handed to the next chunk
+  float *agg_h;    // PAR: [G][K][NM][128] state each chunk produces from zero
+  double *agg_S;   // PAR: [G][K][128] sum of Delta over each chunk
+  float *hin;      // PAR: [G][K][NM][128] state entering each chunk
+  uint64_t timeout_ns;
+  int test_hook;   // 1: unit (group 0, chunk 0) never publishes (tests the bounded wait)
+  int force_generic;  // 1: generic arithmetic for every channel
+};
+
+// ------------------------------------------------------------------ math
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+__device__ __forceinline__ float ex2f(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float lg2f(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcpf(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+using f2 = unsigned long long;  // two packed fp32 lanes for fma.rn.f32x2
+
+__device__ __forceinline__ f2 pk(float lo, float hi) {
+  f2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float lo_of(f2 v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return lo;
+}
+__device__ __forceinline__ float hi_of(f2 v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return hi;
+}
+__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
+  f2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+// log(1 + e^v): a 5-term series of log1p(w) for w = e^v < 1/16 (relative
+// error below 2e-7), log2(1 + w) ln 2 above, and v + e^-v for v > 15.
+__device__ __forceinline__ float softplus_fast(float v) {
+  const float w = ex2f(v * kLog2e);
+  const float s = w * (1.f - w * (0.5f - w * (1.f / 3.f - w * (0.25f - w * 0.2f))));
+  const float l = lg2f(1.f + w) * kLn2;
+  const float r = w < 0.0625f ? s : l;
+  return v > 15.f ? v + ex2f(-v * kLog2e) : r;
+}
+
+// expm1(x) for x <= 0: a degree-6 Taylor polynomial for x > -1/4 (relative
+// error below 6e-8), exp(x) - 1 below (no cancellation there).
+__device__ __forceinline__ float expm1_neg(float x) {
+  const float p = x * (1.f + x * (0.5f + x * (1.f / 6.f + x * (1.f / 24.f + x * (1.f / 120.f +
+                  x * (1.f / 720.f))))));
+  const float q = ex2f(x * kLog2e) - 1.f;
+  return x > -0.25f ? p : q;
+}
+
+// Decays E(j) = expm1(j x), j = 1..NM, as pairs (E(2i+1), E(2i+2)), from
+// E(1) and exp(x) = a1 by E(m+k) = E(m) + exp(m x) E(k).
+template <int NM>
+__device__ __forceinline__ void decay_pairs(float E1, float a1, f2 (&P)[NM / 2]) {
+  const float E2 = fmaf(a1, E1, E1);
+  P[0] = pk(E1, E2);
+  if constexpr (NM >= 4) {
+    const float a2 = 1.f + E2;
+    P[1] = fma2(pk(a2, a2), P[0], pk(E2, E2));
+  }
+  if constexpr (NM >= 8) {
+    const float E4 = hi_of(P[1]);
+    const float a4 = 1.f + E4;
+    const f2 A4 = pk(a4, a4), E4p = pk(E4, E4);
+    P[2] = fma2(A4, P[0], E4p);
+    P[3] = fma2(A4, P[1], E4p);
+  }
+  if constexpr (NM >= 16) {
+    const float E8 = hi_of(P[3]);
+    const float a8 = 1.f + E8;
+    const f2 A8 = pk(a8, a8), E8p = pk(E8, E8);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) P[4 + i] = fma2(A8, P[i], E8p);
+  }
+}
+
+// One structured step for one channel: h_n += E(n+1) (h_n + B'_n u'),
+// returns yinit + sum_n C_n h_n.  Brow / Crow are 16-byte aligned fp32 rows
+// of B' = B/(n+1) and C for this time step.
+template <int NM>
+__device__ __forceinline__ float struct_update(f2 (&H)[NM / 2], const f2 (&P)[NM / 2], float up,
+                                               float yinit, const float *Brow, const float *Crow) {
+  const f2 U = pk(up, up);
+  f2 Y = pk(yinit, 0.f);
+  if constexpr (NM == 2) {
+    const f2 b = *reinterpret_cast<const f2 *>(Brow);
+    const f2 c = *reinterpret_cast<const f2 *>(Crow);
+    H[0] = fma2(P[0], fma2(b, U, H[0]), H[0]);
+    Y = fma2(c, H[0], Y);
+  } else {
+#pragma unroll
+    for (int i = 0; i < NM / 2; i += 2) {
+      const ulonglong2 b = *reinterpret_cast<const ulonglong2 *>(Brow + 2 * i);
+      const ulonglong2 c = *reinterpret_cast<const ulonglong2 *>(Crow + 2 * i);
+      H[i] = fma2(P[i], fma2(b.x, U, H[i]), H[i]);
+      H[i + 1] = fma2(P[i + 1], fma2(b.y, U, H[i + 1]), H[i + 1]);
+      Y = fma2(c.x, H[i], Y);
+      Y = fma2(c.y, H[i + 1], Y);
+    }
+  }
+  return lo_of(Y) + hi_of(Y);
+}
+
+// One generic step for one channel (any A): per state, Abar = exp(Delta A_n)
+// and Bbar/B = Delta psi(Delta A_n) with psi(x) = expm1(x)/x.
+template <int NM>
+__device__ __forceinline__ float generic_update(float (&h)[NM], float Delta, float uv, float yinit,
+                                                const float (&A)[NM], const float (&A2)[NM],
+                                                const float (&invA)[NM], const float *Brow,
+                                                const float *Crow) {
+  float y = yinit;
+#pragma unroll
+  for (int n = 0; n < NM; ++n) {
+    const float x = Delta * A[n];
+    const float a = ex2f(Delta * A2[n]);
+    float p = fmaf(x, 1.f / 720.f, 1.f / 120.f);
+    p = fmaf(x, p, 1.f / 24.f);
+    p = fmaf(x, p, 1.f / 6.f);
+    p = fmaf(x, p, 0.5f);
+    p = fmaf(x, p, 1.f);
+    const float E = fabsf(x) < 0.25f ? Delta * p : (a - 1.f) * invA[n];
+    h[n] = fmaf(a, h[n], E * (Brow[n] * uv));
+    y = fmaf(Crow[n], h[n], y);
+  }
+  return y;
+}
+
+// ------------------------------------------------------------ tile access
+
+template <typename T> struct Vec;
+template <> struct Vec<__nv_bfloat16> {
+  static constexpr int kN = 8;
+  __device__ static void unpack(const uint4 &v, float (&o)[8]) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      o[2 * i] = __uint_as_float(w[i] << 16);
+      o[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+  __device__ static uint4 pack(const float (&o)[8]) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __nv_bfloat162 p = __floats2bfloat162_rn(o[2 * i], o[2 * i + 1]);
+      w[i] = *reinterpret_cast<uint32_t *>(&p);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+  }
+};
+template <> struct Vec<float> {
+  static constexpr int kN = 4;
+  __device__ static void unpack(const uint4 &v, float (&o)[4]) {
+    o[0] = __uint_as_float(v.x);
+    o[1] = __uint_as_float(v.y);
+    o[2] = __uint_as_float(v.z);
+    o[3] = __uint_as_float(v.w);
+  }
+  __device__ static uint4 pack(const float (&o)[4]) {
+    return make_uint4(__float_as_uint(o[0]), __float_as_uint(o[1]), __float_as_uint(o[2]),
+                      __float_as_uint(o[3]));
+  }
+};
+
+// Byte offset of 16-byte chunk j of row r in a 64-byte-row tile written by
+// TMA with 64-byte swizzling (chunk index XOR bits 8:7 of the address).
+__device__ __forceinline__ int swz64(int r, int j) { return r * kRowBytes + ((j ^ ((r >> 1) & 3)) << 4); }
+
+__device__ __forceinline__ float raw_to_f(const __nv_bfloat16 *p, int i) { return __bfloat162float(p[i]); }
+__device__ __forceinline__ float raw_to_f(const float *p, int i) { return p[i]; }
+
+// --------------------------------------------------------------- the kernel
 
 template <typename T, int NM>
-mamba_status_t staged_forward(const FwdArgs &a, int path, int chunk_len, cudaStream_t s) {
-  return MAMBA_ERR_UNSUPPORTED;
+struct StagedLayout {
+  static constexpr int TT = kRowBytes / (int)sizeof(T);  // time steps per tile
+  static constexpr int VEC = 16 / (int)sizeof(T);        // time steps per 16-byte chunk
+  static constexpr int NV = TT / VEC;                    // chunks per row
+  static constexpr int BSTR = (NM < 4 ? 4 : NM) + 4;     // fp32 row stride of B' / C
+  static constexpr int OFF_Y = kStages * kStageBytes;
+  static constexpr int OFF_BS = OFF_Y + 2 * kTileBytes;
+  static constexpr int OFF_CS = OFF_BS + TT * BSTR * 4;
+  static constexpr int OFF_BAR = OFF_CS + TT * BSTR * 4;
+  static constexpr int OFF_Q = OFF_BAR + 8 * kStages;
+  static constexpr int BYTES = OFF_Q + 16 * 4;
+  static constexpr int ALLOC = BYTES + 1024;  // slack to align the base to 1 KB
+};
+
+template <typename T, int NM, int KIND>
+__global__ void __launch_bounds__(kSThreads, 2)
+    fwd_staged_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_d,
+                      const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_y,
+                      const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_C,
+                      const StagedArgs p) {
+  using Lay = StagedLayout<T, NM>;
+  constexpr int TT = Lay::TT, VEC = Lay::VEC, NV = Lay::NV, BSTR = Lay::BSTR;
+  constexpr bool kOut = KIND != KIND_AGG;
+
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char *sm = reinterpret_cast<unsigned char *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sm + Lay::OFF_BAR);
+  int *q = reinterpret_cast<int *>(sm + Lay::OFF_Q);  // [0..7] ticket ring, [8] abort
+  float *Bs = reinterpret_cast<float *>(sm + Lay::OFF_BS);
+  float *Cs = reinterpret_cast<float *>(sm + Lay::OFF_CS);
+
+  const int tid = threadIdx.x;
+  const FwdArgs &f = p.f;
+  const int N = f.N;
+  const bool has_z = kOut && f.z != nullptr;
+  const uint32_t tile_bytes = (kOut ? (has_z ? 3u : 2u) : 2u) * kTileBytes +
+                              (kOut ? 2u : 1u) * uint32_t(N) * kRowBytes;
+
+  if (tid == 0) {
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
+    fence_barrier_init();
+    prefetch_tensormap(&tm_u);
+    prefetch_tensormap(&tm_d);
+    prefetch_tensormap(&tm_B);
+    if (kOut) {
+      prefetch_tensormap(&tm_C);
+      prefetch_tensormap(&tm_y);
+      if (has_z) prefetch_tensormap(&tm_z);
+    }
+    q[8] = 0;
+  }
+  __syncthreads();
+
+  // ---- producer state (meaningful in thread 0 only)
+  int p_ticket = 0, p_tile = 0, p_ntiles = 0, p_tail = 0, p_issued = 0;
+  bool p_done = false;
+
+  auto unit_tiles = [&](int ticket) {
+    const int k = ticket / p.G;
+    const int64_t t0 = int64_t(k) * p.chunk_len;
+    const int64_t t1 = std::min<int64_t>(f.L, t0 + p.chunk_len);
+    return int((t1 - t0 + TT - 1) / TT);
+  };
+
+  auto produce = [&](int stage) {
+    if (p_done) return;
+    if (p_tile == p_ntiles) {
+      p_ticket = atomicAdd(p.counter, 1);
+      q[p_tail & 7] = p_ticket;
+      ++p_tail;
+      if (p_ticket >= p.n_units) {
+        p_done = true;
+        return;
+      }
+      p_ntiles = unit_tiles(p_ticket);
+      p_tile = 0;
+    }
+    const int g = p_ticket % p.G, k = p_ticket / p.G;
+    const int b = g / p.gpb, d0 = (g % p.gpb) * kSThreads;
+    const int t0 = k * p.chunk_len + p_tile * TT;
+    unsigned char *st = sm + stage * kStageBytes;
+    uint64_t *bar = &bars[stage];
+    mbar_arrive_expect_tx(bar, tile_bytes);
+    tma_load_3d(st, &tm_u, bar, t0, d0, b);
+    tma_load_3d(st + kTileBytes, &tm_d, bar, t0, d0, b);
+    if (has_z) tma_load_3d(st + 2 * kTileBytes, &tm_z, bar, t0, d0, b);
+    tma_load_3d(st + 3 * kTileBytes, &tm_B, bar, t0, 0, b);
+    if (kOut) tma_load_3d(st + 3 * kTileBytes + kRawBytes, &tm_C, bar, t0, 0, b);
+    ++p_tile;
+    ++p_issued;
+  };
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) produce(s);
+  }
+
+  int head = 0;   // consumer position in the ticket ring
+  int ctile = 0;  // tiles consumed by this CTA
+  bool aborted = false;
+
+  while (true) {
+    __syncthreads();
+    const int ticket = q[head & 7];
+    ++head;
+    if (ticket >= p.n_units) break;
+    const int g = ticket % p.G, k = ticket / p.G;
+    const int b = g / p.gpb, d0 = (g % p.gpb) * kSThreads;
+    const int d = d0 + tid;
+    const bool valid = d < f.dim;
+    const int64_t tbeg = int64_t(k) * p.chunk_len;
+    const int64_t tend = std::min<int64_t>(f.L, tbeg + p.chunk_len);
+    const int ntiles = int((tend - tbeg + TT - 1) / TT);
+
+    // per-channel parameters and the arithmetic this unit can use
+    float Arow[NM];
+#pragma unroll
+    for (int n = 0; n < NM; ++n) Arow[n] = (valid && n < N) ? f.A[int64_t(d) * N + n] : -float(n + 1);
+    if (valid) {  // padding states (n >= N) carry B = C = 0; give them a finite A of the same form
+      const float pad0 = (Arow[0] < 0.f && isfinite(Arow[0])) ? Arow[0] : -1.f;
+#pragma unroll
+      for (int n = 1; n < NM; ++n)
+        if (n >= N) Arow[n] = float(n + 1) * pad0;
+    }
+    const float bias = (valid && f.bias) ? f.bias[d] : 0.f;
+    const float Dd = (valid && f.D && kOut) ? f.D[d] : 0.f;
+    bool structured = Arow[0] < 0.f && isfinite(Arow[0]);
+#pragma unroll
+    for (int n = 1; n < NM; ++n) structured = structured && (Arow[n] == float(n + 1) * Arow[0]);
+    const bool sig = structured && Arow[0] == -1.f;
+    int mode = MODE_GEN;
+    if (!p.force_generic) {
+      if (__syncthreads_and(sig)) mode = MODE_SIG;
+      else if (__syncthreads_and(structured)) mode = MODE_STRUCT;
+    }
+
+    // state entering the chunk
+    float hs[NM];
+#pragma unroll
+    for (int n = 0; n < NM; ++n) hs[n] = 0.f;
+    if (KIND == KIND_SEQ && k > 0) {
+      if (tid == 0 && !wait_flag_geq(p.flags + g, k, p.timeout_ns)) {
+        record_timeout();
+        q[8] = 1;
+      }
+      __syncthreads();
+      if (q[8]) {
+        aborted = true;
+        break;
+      }
+#pragma unroll
+      for (int n = 0; n < NM; ++n) hs[n] = __ldcg(p.carry + (int64_t(g) * NM + n) * kSThreads + tid);
+    } else if (KIND == KIND_PAR && k > 0) {
+#pragma unroll
+      for (int n = 0; n < NM; ++n)
+        hs[n] = __ldcg(p.hin + ((int64_t(g) * p.K + k) * NM + n) * kSThreads + tid);
+    }
+
+    double Ssum = 0.0;  // sum of Delta over the chunk (aggregate pass)
+
+    // Runs every tile of this unit with the arithmetic of mode M.
+    auto run = [&](auto mode_tag) {
+      constexpr int M = decltype(mode_tag)::value;
+      f2 H[NM / 2];
+      float h[NM];
+      float A2[NM], invA[NM];
+      if constexpr (M == MODE_GEN) {
+#pragma unroll
+        for (int n = 0; n < NM; ++n) {
+          h[n] = hs[n];
+          A2[n] = Arow[n] * kLog2e;
+          invA[n] = Arow[n] != 0.f ? 1.f / Arow[n] : 0.f;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < NM / 2; ++i) H[i] = pk(hs[2 * i], hs[2 * i + 1]);
+      }
+      const float A0 = Arow[0];
+      const float invA0 = 1.f / A0;
+
+      for (int it = 0; it < ntiles; ++it, ++ctile) {
+        const int stage = ctile % kStages;
+        const uint32_t parity = uint32_t(ctile / kStages) & 1u;
+        unsigned char *st = sm + stage * kStageBytes;
+        if (!mbar_wait_bounded(&bars[stage], parity, p.timeout_ns)) {
+          record_timeout();
+          q[8] = 1;
+        }
+        // B and C rows of this tile -> fp32, time-major, B scaled by 1/(n+1)
+        // for the structured arithmetic.
+        {
+          const T *Braw = reinterpret_cast<const T *>(st + 3 * kTileBytes);
+          const T *Craw = reinterpret_cast<const T *>(st + 3 * kTileBytes + kRawBytes);
+          constexpr int ITEMS = NM * (TT / 4);
+          for (int w = tid; w < (kOut ? 2 : 1) * ITEMS; w += kSThreads) {
+            const bool isC = w >= ITEMS;
+            const int r = isC ? w - ITEMS : w;
+            const int n = r % NM, tg = r / NM;
+            const T *src = (isC ? Craw : Braw) + n * TT + 4 * tg;
+            float *dst = (isC ? Cs : Bs) + 4 * tg * BSTR + n;
+            const float scale = (!isC && M != MODE_GEN) ? 1.f / float(n + 1) : 1.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i * BSTR] = n < N ? raw_to_f(src, i) * scale : 0.f;
+          }
+        }
+        __syncthreads();
+        if (q[8]) return;
+
+        const int64_t t0 = tbeg + int64_t(it) * TT;
+        const unsigned char *su = st;
+        const unsigned char *sd = st + kTileBytes;
+        const unsigned char *sz = st + 2 * kTileBytes;
+        unsigned char *sy = sm + Lay::OFF_Y + (ctile & 1) * kTileBytes;
+        for (int j = 0; j < NV; ++j) {
+          if (t0 + int64_t(j) * VEC >= tend) break;  // past the end of the sequence
+          const int off = swz64(tid, j);
+          float uv[VEC], dv[VEC], zv[VEC], yv[VEC];
+          Vec<T>::unpack(*reinterpret_cast<const uint4 *>(su + off), uv);
+          Vec<T>::unpack(*reinterpret_cast<const uint4 *>(sd + off), dv);
+          if (has_z) Vec<T>::unpack(*reinterpret_cast<const uint4 *>(sz + off), zv);
+#pragma unroll
+          for (int i = 0; i < VEC; ++i) {
+            const int tl = j * VEC + i;
+            const float *Brow = Bs + tl * BSTR;
+            const float *Crow = Cs + tl * BSTR;
+            const float v = dv[i] + bias;
+            float y0;
+            if constexpr (M == MODE_SIG) {
+              const float vc = fminf(fmaxf(v, -80.f), 80.f);
+              const float ev = ex2f(-vc * kLog2e);  // e^-v
+              const float s = rcpf(1.f + ev);      // sigma(v) = 1 - exp(-Delta)
+              f2 P[NM / 2];
+              decay_pairs<NM>(-s, ev * s, P);
+              if (kOut) {
+                y0 = struct_update<NM>(H, P, -uv[i], Dd * uv[i], Brow, Crow);
+              } else {
+                struct_update<NM>(H, P, -uv[i], 0.f, Brow, Brow);
+                Ssum += double(softplus_fast(v));
+              }
+            } else if constexpr (M == MODE_STRUCT) {
+              const float Delta = softplus_fast(v);
+              const float E1 = expm1_neg(Delta * A0);
+              f2 P[NM / 2];
+              decay_pairs<NM>(E1, 1.f + E1, P);
+              if (kOut) {
+                y0 = struct_update<NM>(H, P, uv[i] * invA0, Dd * uv[i], Brow, Crow);
+              } else {
+                struct_update<NM>(H, P, uv[i] * invA0, 0.f, Brow, Brow);
+                Ssum += double(Delta);
+              }
+            } else {
+              const float Delta = softplus_fast(v);
+              y0 = generic_update<NM>(h, Delta, uv[i], Dd * uv[i], Arow, A2, invA, Brow,
+                                      kOut ? Crow : Brow);
+              if (!kOut) Ssum += double(Delta);
+            }
+            if (kOut) {
+              if (has_z) {
+                const float ez = ex2f(-zv[i] * kLog2e);
+                y0 *= zv[i] * rcpf(1.f + ez);
+              }
+              yv[i] = y0;
+            }
+          }
+          if (kOut) *reinterpret_cast<uint4 *>(sy + off) = Vec<T>::pack(yv);
+        }
+        if (kOut) fence_proxy_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+          if (kOut) {
+            tma_store_3d(&tm_y, sy, int(t0), d0, b);
+            bulk_commit();
+            bulk_wait_read<1>();
+          }
+          produce(stage);
+        }
+      }
+      if constexpr (M == MODE_GEN) {
+#pragma unroll
+        for (int n = 0; n < NM; ++n) hs[n] = h[n];
+      } else {
+#pragma unroll
+        for (int i = 0; i < NM / 2; ++i) {
+          hs[2 * i] = lo_of(H[i]);
+          hs[2 * i + 1] = hi_of(H[i]);
+        }
+      }
+    };
+
+    if (mode == MODE_SIG) run(std::integral_constant<int, MODE_SIG>{});
+    else if (mode == MODE_STRUCT) run(std::integral_constant<int, MODE_STRUCT>{});
+    else run(std::integral_constant<int, MODE_GEN>{});
+    if (q[8]) {
+      aborted = true;
+      break;
+    }
+
+    // hand the end state on
+    if (KIND == KIND_AGG) {
+#pragma unroll
+      for (int n = 0; n < NM; ++n)
+        p.agg_h[((int64_t(g) * p.K + k) * NM + n) * kSThreads + tid] = hs[n];
+      p.agg_S[(int64_t(g) * p.K + k) * kSThreads + tid] = Ssum;
+    } else if (k == p.K - 1) {
+      if (valid && f.last_state) {
+#pragma unroll
+        for (int n = 0; n < NM; ++n)
+          if (n < N) f.last_state[(int64_t(b) * f.dim + d) * N + n] = hs[n];
+      }
+    } else if (KIND == KIND_SEQ) {
+#pragma unroll
+      for (int n = 0; n < NM; ++n) p.carry[(int64_t(g) * NM + n) * kSThreads + tid] = hs[n];
+      __threadfence();
+      __syncthreads();
+      if (tid == 0 && !(p.test_hook == 1 && g == 0 && k == 0)) st_release_gpu(p.flags + g, k + 1);
+    }
+  }
+
+  // Drain: every TMA load this CTA issued must land before it exits.
+  __syncthreads();
+  if (tid == 0) {
+    if (aborted) {
+      for (int t = ctile; t < p_issued; ++t)
+        mbar_wait_bounded(&bars[t % kStages], uint32_t(t / kStages) & 1u, p.timeout_ns);
+    }
+    bulk_wait<0>();
+  }
+}
+
+// Carry scan over chunks (PAR): h_in(0) = 0,
+// h_in(k+1) = exp(A_n S_k) h_in(k) + h_loc(k), one thread per (group, n, channel).
+template <int NM>
+__global__ void carry_scan_kernel(const StagedArgs p) {
+  const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t total = int64_t(p.G) * NM * kSThreads;
+  if (idx >= total) return;
+  const int c = int(idx % kSThreads);
+  const int n = int((idx / kSThreads) % NM);
+  const int g = int(idx / (int64_t(NM) * kSThreads));
+  const int d = (g % p.gpb) * kSThreads + c;
+  const double An = (d < p.f.dim && n < p.f.N) ? double(p.f.A[int64_t(d) * p.f.N + n]) : 0.0;
+  double h = 0.0;
+  for (int k = 0; k < p.K; ++k) {
+    const int64_t base = (int64_t(g) * p.K + k);
+    p.hin[(base * NM + n) * kSThreads + c] = float(h);
+    if (k < p.K - 1) h = exp(An * p.agg_S[base * kSThreads + c]) * h + double(p.agg_h[(base * NM + n) * kSThreads + c]);
+  }
+}
+
+// ------------------------------------------------------------------ host
+
+struct StagedPlan {
+  int kind;       // KIND_SEQ or KIND_PAR
+  int chunk_len;
+  int K;
+};
+
+inline int device_sm_count() {
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms > 0 ? sms : 148;
+}
+
+// Whether the staged kernels can take this problem: rows of 16-byte
+// multiples, 16-byte aligned bases, N >= 3.
+inline bool staged_supported(const FwdArgs &a, size_t es) {
+  auto al = [](const void *ptr) { return ptr == nullptr || (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; };
+  if (a.N < 3) return false;
+  if ((a.L * int64_t(es)) % 16 != 0) return false;
+  if (a.L > (int64_t(1) << 31) - 1024 || a.dim > (int64_t(1) << 31) - 1) return false;
+  return al(a.u) && al(a.delta) && al(a.z) && al(a.y) && al(a.B) && al(a.C);
+}
+
+template <typename T, int NM, int KIND>
+inline cudaError_t prepare_kernel(int *blocks_per_sm) {
+  auto kern = fwd_staged_kernel<T, NM, KIND>;
+  const int bytes = StagedLayout<T, NM>::ALLOC;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, kern, kSThreads, bytes);
+}
+
+template <typename T, int NM, int KIND>
+inline void launch_staged(const CUtensorMap (&maps)[6], const StagedArgs &sa, int grid, cudaStream_t s) {
+  fwd_staged_kernel<T, NM, KIND><<<grid, kSThreads, StagedLayout<T, NM>::ALLOC, s>>>(
+      maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], sa);
+}
+
+struct StagedOptions {
+  int path, chunk_len, carry, timeout_us, test_hook;
+};
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Picks the chunking: the sequential hand-off when the channel groups alone
+// fill the resident CTAs (about eight chunks per group keeps the tail short),
+// else the three-phase scheme with about four units per resident CTA.
+inline StagedPlan plan_staged(int64_t G, int64_t L, int slots, const StagedOptions &o) {
+  StagedPlan pl;
+  int carry = o.carry;
+  if (carry == 0) carry = G >= slots ? 1 : 2;
+  int64_t chunk = o.chunk_len;
+  if (chunk <= 0) {
+    if (carry == 1) {
+      const int64_t kt = std::max<int64_t>(1, (8 * int64_t(slots) + G / 2) / G);
+      chunk = std::max<int64_t>(256, ceil_div(ceil_div(L, kt), 64) * 64);
+    } else {
+      const int64_t kt = std::max<int64_t>(1, ceil_div(4 * int64_t(slots), G));
+      chunk = std::max<int64_t>(512, ceil_div(ceil_div(L, kt), 64) * 64);
+    }
+  }
+  chunk = std::min<int64_t>(chunk, ceil_div(L, 64) * 64);
+  pl.chunk_len = int(chunk);
+  pl.K = int(ceil_div(L, chunk));
+  pl.kind = (pl.K == 1) ? KIND_SEQ : (carry == 1 ? KIND_SEQ : KIND_PAR);
+  return pl;
+}
+
+// The staged forward: tensor maps, plan, stream-ordered workspace, launches.
+// Returns MAMBA_ERR_UNSUPPORTED (nothing enqueued) if the driver rejects a
+// tensor map.
+template <typename T, int NM>
+mamba_status_t staged_forward(const FwdArgs &a, const StagedOptions &o, cudaStream_t s,
+                              mamba_status_t (*launched)()) {
+  using Lay = StagedLayout<T, NM>;
+  constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
+  CUtensorMap maps[6];
+  const uint64_t L = a.L, dim = a.dim, batch = a.batch, N = a.N;
+  const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_64B, none = CU_TENSOR_MAP_SWIZZLE_NONE;
+  if (!make_map_3d(&maps[0], a.u, bf16, L, dim, batch, Lay::TT, kSThreads, sw) ||
+      !make_map_3d(&maps[1], a.delta, bf16, L, dim, batch, Lay::TT, kSThreads, sw) ||
+      !make_map_3d(&maps[2], a.z ? a.z : a.u, bf16, L, dim, batch, Lay::TT, kSThreads, sw) ||
+      !make_map_3d(&maps[3], a.y, bf16, L, dim, batch, Lay::TT, kSThreads, sw) ||
+      !make_map_3d(&maps[4], a.B, bf16, L, N, batch, Lay::TT, uint32_t(N), none) ||
+      !make_map_3d(&maps[5], a.C, bf16, L, N, batch, Lay::TT, uint32_t(N), none)) {
+    return MAMBA_ERR_UNSUPPORTED;
+  }
+  int bps_main = 0;
+  if (prepare_kernel<T, NM, KIND_SEQ>(&bps_main) != cudaSuccess) return MAMBA_ERR_CUDA;
+  const int sms = device_sm_count();
+  const int slots = sms * std::max(1, bps_main);
+  const int64_t gpb = ceil_div(a.dim, kSThreads);
+  const int64_t G = int64_t(a.batch) * gpb;
+  if (G > (int64_t(1) << 30)) return MAMBA_ERR_UNSUPPORTED;
+  const StagedPlan pl = plan_staged(G, a.L, slots, o);
+  if (G * pl.K > (int64_t(1) << 30)) return MAMBA_ERR_UNSUPPORTED;
+
+  StagedArgs sa;
+  sa.f = a;
+  sa.G = int(G);
+  sa.gpb = int(gpb);
+  sa.K = pl.K;
+  sa.chunk_len = pl.chunk_len;
+  sa.timeout_ns = o.timeout_us > 0 ? uint64_t(o.timeout_us) * 1000ull : kDefaultTimeoutNs;
+  sa.test_hook = o.test_hook;
+  sa.force_generic = o.path == MAMBA_PATH_GENERIC ? 1 : 0;
+  sa.flags = nullptr;
+  sa.carry = sa.agg_h = sa.hin = nullptr;
+  sa.agg_S = nullptr;
+
+  // workspace: [ints: 2 counters + G flags][carry | agg_h, agg_S, hin]
+  const size_t n_int = 2 + size_t(G);
+  const size_t int_bytes = ceil_div(n_int * 4, 256) * 256;
+  size_t bytes = int_bytes;
+  const size_t gk = size_t(G) * size_t(pl.K);
+  if (pl.kind == KIND_SEQ) {
+    bytes += size_t(G) * NM * kSThreads * 4;
+  } else {
+    bytes += gk * kSThreads * 8 + 2 * gk * NM * kSThreads * 4;
+  }
+  unsigned char *ws = nullptr;
+  if (cudaMallocAsync(reinterpret_cast<void **>(&ws), bytes, s) != cudaSuccess) {
+    cudaGetLastError();
+    return MAMBA_ERR_OUT_OF_MEMORY;
+  }
+  mamba_status_t st = MAMBA_OK;
+  if (cudaMemsetAsync(ws, 0, int_bytes, s) != cudaSuccess) st = MAMBA_ERR_CUDA;
+  int *counters = reinterpret_cast<int *>(ws);
+  sa.flags = counters + 2;
+  if (st == MAMBA_OK && pl.kind == KIND_SEQ) {
+    sa.carry = reinterpret_cast<float *>(ws + int_bytes);
+    sa.counter = counters;
+    sa.n_units = int(gk);
+    const int grid = int(std::min<int64_t>(gk, slots));
+    launch_staged<T, NM, KIND_SEQ>(maps, sa, grid, s);
+    st = launched();
+  } else if (st == MAMBA_OK) {
+    sa.agg_S = reinterpret_cast<double *>(ws + int_bytes);
+    sa.agg_h = reinterpret_cast<float *>(ws + int_bytes + gk * kSThreads * 8);
+    sa.hin = sa.agg_h + gk * NM * kSThreads;
+    int bps_agg = 0, bps_par = 0;
+    if (prepare_kernel<T, NM, KIND_AGG>(&bps_agg) != cudaSuccess ||
+        prepare_kernel<T, NM, KIND_PAR>(&bps_par) != cudaSuccess) {
+      st = MAMBA_ERR_CUDA;
+    }
+    if (st == MAMBA_OK) {
+      StagedArgs sg = sa;
+      sg.counter = counters;
+      sg.n_units = int(size_t(G) * size_t(pl.K - 1));
+      launch_staged<T, NM, KIND_AGG>(maps, sg, int(std::min<int64_t>(sg.n_units, sms * std::max(1, bps_agg))), s);
+      st = launched();
+    }
+    if (st == MAMBA_OK) {
+      const int64_t threads = G * NM * kSThreads;
+      carry_scan_kernel<NM><<<unsigned(ceil_div(threads, 256)), 256, 0, s>>>(sa);
+      st = launched();
+    }
+    if (st == MAMBA_OK) {
+      StagedArgs sm = sa;
+      sm.counter = counters + 1;
+      sm.n_units = int(gk);
+      launch_staged<T, NM, KIND_PAR>(maps, sm, int(std::min<int64_t>(gk, sms * std::max(1, bps_par))), s);
+      st = launched();
+    }
+  }
+  if (cudaFreeAsync(ws, s) != cudaSuccess && st == MAMBA_OK) st = MAMBA_ERR_CUDA;
+  return st;
 }
 
 }  // namespace mscan

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 
@@ -13,11 +14,31 @@
 #include "fwd_reference.cuh"
 #include "fwd_staged.cuh"
 
+namespace mscan {
+
+EncodeTiledFn get_encode_tiled() {
+  static const EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    return reinterpret_cast<EncodeTiledFn>(ptr);
+  }();
+  return fn;
+}
+
+}  // namespace mscan
+
 using namespace mscan;
 
 namespace {
 
 constexpr int kAbiVersion = 1;
+
+std::atomic<uint64_t> g_launches{0};
 
 struct Range {
   uintptr_t lo, hi;
@@ -86,15 +107,23 @@ mamba_status_t check_options(const mamba_scan_options_t *o) {
   if (!o) return MAMBA_OK;
   if (o->path < MAMBA_PATH_AUTO || o->path > MAMBA_PATH_STRUCTURED) return MAMBA_ERR_INVALID_ARG;
   if (o->chunk_len < 0 || (o->chunk_len > 0 && o->chunk_len % 64 != 0)) return MAMBA_ERR_INVALID_ARG;
-  for (int i = 0; i < 6; ++i)
+  if (o->carry < 0 || o->carry > 2 || o->wait_timeout_us < 0 || o->test_hook < 0 || o->test_hook > 1)
+    return MAMBA_ERR_INVALID_ARG;
+  for (int i = 0; i < 3; ++i)
     if (o->reserved[i] != 0) return MAMBA_ERR_INVALID_ARG;
   return MAMBA_OK;
 }
 
-mamba_status_t launch_status() {
+mamba_status_t cuda_status() {
   const cudaError_t e = cudaGetLastError();
   if (e == cudaSuccess) return MAMBA_OK;
   return e == cudaErrorMemoryAllocation ? MAMBA_ERR_OUT_OF_MEMORY : MAMBA_ERR_CUDA;
+}
+
+// Status of the kernel launch just made (counted for mamba_scan_launch_count).
+mamba_status_t launch_status() {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return cuda_status();
 }
 
 // Dispatch on N (rounded up to 1, 2, 4, 8 or 16; the padding states carry
@@ -125,12 +154,12 @@ struct FwdReferenceLauncher {
   }
 };
 
-template <typename T, int NM>
-struct FwdStagedLauncher {
-  static mamba_status_t run(const FwdArgs &a, int path, int chunk_len, cudaStream_t s) {
-    return staged_forward<T, NM>(a, path, chunk_len, s);
-  }
-};
+template <typename T>
+mamba_status_t staged_dispatch(const FwdArgs &a, const StagedOptions &o, cudaStream_t s) {
+  if (a.N <= 4) return staged_forward<T, 4>(a, o, s, &launch_status);
+  if (a.N <= 8) return staged_forward<T, 8>(a, o, s, &launch_status);
+  return staged_forward<T, 16>(a, o, s, &launch_status);
+}
 
 template <typename T, int NM>
 struct BwdReferenceLauncher {
@@ -186,6 +215,8 @@ struct BwdReferenceLauncher {
 extern "C" {
 
 int mamba_scan_abi_version(void) { return kAbiVersion; }
+
+uint64_t mamba_scan_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 const char *mamba_scan_status_string(mamba_status_t s) {
   switch (s) {
@@ -244,20 +275,27 @@ mamba_status_t mamba_scan_fwd_ex(const void *u, const void *delta, const float *
   if (batch == 0 || dim == 0) return MAMBA_OK;
   if (L == 0) {
     if (last_state && cudaMemsetAsync(last_state, 0, size_t(batch) * dim * N * 4, s) != cudaSuccess)
-      return launch_status();
+      return cuda_status();
     return MAMBA_OK;
   }
   FwdArgs a;
   a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
   a.bias = delta_bias; a.A = A; a.D = D; a.y = y; a.last_state = last_state;
   a.batch = batch; a.dim = dim; a.L = L; a.N = (int)N;
-  const int path = options ? options->path : MAMBA_PATH_AUTO;
-  const int chunk_len = options ? options->chunk_len : 0;
-  if (path == MAMBA_PATH_REFERENCE || !staged_supported(a, es)) {
-    if (path == MAMBA_PATH_GENERIC || path == MAMBA_PATH_STRUCTURED) return MAMBA_ERR_UNSUPPORTED;
+  StagedOptions so;
+  so.path = options ? options->path : MAMBA_PATH_AUTO;
+  so.chunk_len = options ? options->chunk_len : 0;
+  so.carry = options ? options->carry : 0;
+  so.timeout_us = options ? options->wait_timeout_us : 0;
+  so.test_hook = options ? options->test_hook : 0;
+  const bool stageable = staged_supported(a, es);
+  if (so.path == MAMBA_PATH_REFERENCE || (!stageable && so.path == MAMBA_PATH_AUTO))
     return dispatch<FwdReferenceLauncher>(dtype, (int)N, a, s);
-  }
-  return dispatch<FwdStagedLauncher>(dtype, (int)N, a, path, chunk_len, s);
+  if (!stageable) return MAMBA_ERR_UNSUPPORTED;
+  st = dtype == MAMBA_BF16 ? staged_dispatch<__nv_bfloat16>(a, so, s) : staged_dispatch<float>(a, so, s);
+  if (st == MAMBA_ERR_UNSUPPORTED && so.path == MAMBA_PATH_AUTO)
+    return dispatch<FwdReferenceLauncher>(dtype, (int)N, a, s);
+  return st;
 }
 
 mamba_status_t mamba_scan_fwd(const void *u, const void *delta, const float *delta_bias,
@@ -312,10 +350,10 @@ mamba_status_t mamba_scan_bwd_ex(const void *u, const void *delta, const float *
   if (batch == 0 || L == 0) {
     // Empty sum: parameter gradients are zero, and dB / dC have no elements
     // unless batch > 0 and L > 0.
-    if (cudaMemsetAsync(dA, 0, size_t(dim) * N * 4, s) != cudaSuccess) return launch_status();
-    if (dD && cudaMemsetAsync(dD, 0, size_t(dim) * 4, s) != cudaSuccess) return launch_status();
+    if (cudaMemsetAsync(dA, 0, size_t(dim) * N * 4, s) != cudaSuccess) return cuda_status();
+    if (dD && cudaMemsetAsync(dD, 0, size_t(dim) * 4, s) != cudaSuccess) return cuda_status();
     if (ddelta_bias && cudaMemsetAsync(ddelta_bias, 0, size_t(dim) * 4, s) != cudaSuccess)
-      return launch_status();
+      return cuda_status();
     return MAMBA_OK;
   }
   BwdArgs a;

@@ -34,7 +34,8 @@ class MambaScanError(RuntimeError):
 
 class _Options(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int32), ("chunk_len", ctypes.c_int32),
-                ("reserved", ctypes.c_int32 * 6)]
+                ("carry", ctypes.c_int32), ("wait_timeout_us", ctypes.c_int32),
+                ("test_hook", ctypes.c_int32), ("reserved", ctypes.c_int32 * 3)]
 
 
 _lock = threading.Lock()
@@ -67,6 +68,8 @@ def load_library():
             lib.mamba_scan_stream_status.argtypes = [vp]
             lib.mamba_scan_status_string.argtypes = [ctypes.c_int]
             lib.mamba_scan_status_string.restype = ctypes.c_char_p
+            lib.mamba_scan_launch_count.argtypes = []
+            lib.mamba_scan_launch_count.restype = ctypes.c_uint64
             lib.mamba_scan_abi_version.argtypes = []
             lib.mamba_scan_abi_version.restype = ctypes.c_int
             _lib = lib
@@ -101,10 +104,16 @@ def _stream_handle(stream) -> Optional[int]:
     return stream.cuda_stream if isinstance(stream, torch.cuda.Stream) else int(stream)
 
 
-def _options(path, chunk_len):
+CARRY = {"auto": 0, "sequential": 1, "three_phase": 2}
+
+
+def _options(path, chunk_len, carry="auto", wait_timeout_us=0, test_hook=0):
     o = _Options()
     o.path = PATHS[path] if isinstance(path, str) else int(path)
     o.chunk_len = int(chunk_len)
+    o.carry = CARRY[carry] if isinstance(carry, str) else int(carry)
+    o.wait_timeout_us = int(wait_timeout_us)
+    o.test_hook = int(test_hook)
     return o
 
 
@@ -114,7 +123,7 @@ def _check(rc: int, where: str):
 
 
 def mamba_scan_fwd(u, delta, delta_bias, A, B, C, D, z, y, last_state, *, path="auto",
-                   chunk_len=0, stream=None):
+                   chunk_len=0, carry="auto", wait_timeout_us=0, test_hook=0, stream=None):
     """Enqueue the forward on ``stream`` (torch's current stream by default).
     Tensors as in ``include/mamba_scan.h``; ``y`` (and ``last_state``) are
     written."""
@@ -130,11 +139,12 @@ def mamba_scan_fwd(u, delta, delta_bias, A, B, C, D, z, y, last_state, *, path="
         _ptr(y, dt, (batch, dim, L), "y"), _ptr(last_state, f32, (batch, dim, N), "last_state"),
         batch, dim, L, N, _dtype_code(dt)]
     lib = load_library()
-    if path == "auto" and not chunk_len:
+    if path == "auto" and not chunk_len and carry == "auto" and not wait_timeout_us \
+            and not test_hook:
         rc = lib.mamba_scan_fwd(*args, _stream_handle(stream))
     else:
-        rc = lib.mamba_scan_fwd_ex(*args, ctypes.byref(_options(path, chunk_len)),
-                                   _stream_handle(stream))
+        opts = _options(path, chunk_len, carry, wait_timeout_us, test_hook)
+        rc = lib.mamba_scan_fwd_ex(*args, ctypes.byref(opts), _stream_handle(stream))
     _check(rc, "mamba_scan_fwd")
 
 
@@ -165,20 +175,26 @@ def mamba_scan_bwd(u, delta, delta_bias, A, B, C, D, z, dy, du, ddelta, dA, dB, 
     _check(rc, "mamba_scan_bwd")
 
 
+def launch_count() -> int:
+    """Kernels launched by the library so far in this process."""
+    return int(load_library().mamba_scan_launch_count())
+
+
 def mamba_scan_stream_status(stream=None) -> int:
     """Synchronize the stream and return (and clear) the sticky device status."""
     return load_library().mamba_scan_stream_status(_stream_handle(stream))
 
 
 def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
-                       return_last_state=False, path="auto", chunk_len=0, stream=None):
+                       return_last_state=False, path="auto", chunk_len=0, carry="auto",
+                       stream=None):
     """Allocate y (and last_state) and run the forward; returns y or (y, last_state)."""
     batch, dim, L = u.shape
     y = torch.empty_like(u)
     last = (torch.empty(batch, dim, A.shape[1], device=u.device, dtype=torch.float32)
             if return_last_state else None)
     mamba_scan_fwd(u, delta, delta_bias, A, B, C, D, z, y, last, path=path,
-                   chunk_len=chunk_len, stream=stream)
+                   chunk_len=chunk_len, carry=carry, stream=stream)
     return (y, last) if return_last_state else y
 
 

@@ -27,10 +27,11 @@ def to_host(x: dict) -> dict:
     return {k: (v.cpu() if torch.is_tensor(v) else v) for k, v in x.items()}
 
 
-def gpu_fwd(x: dict, path="auto", chunk_len=0, last=True):
+def gpu_fwd(x: dict, path="auto", chunk_len=0, last=True, carry="auto"):
     out = scan.selective_scan_fwd(x["u"], x["delta"], x["A"], x["B"], x["C"], D=x["D"],
                                   z=x["z"], delta_bias=x["delta_bias"],
-                                  return_last_state=last, path=path, chunk_len=chunk_len)
+                                  return_last_state=last, path=path, chunk_len=chunk_len,
+                                  carry=carry)
     assert scan.mamba_scan_stream_status() == 0
     return out if last else (out, None)
 

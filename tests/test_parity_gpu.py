@@ -25,9 +25,9 @@ def _lib():
     scan.load_library()
 
 
-def _fwd_case(x_host, path="auto", chunk_len=0):
+def _fwd_case(x_host, path="auto", chunk_len=0, carry="auto"):
     x = gc.to_device(x_host)
-    y, last = gc.gpu_fwd(x, path=path, chunk_len=chunk_len)
+    y, last = gc.gpu_fwd(x, path=path, chunk_len=chunk_len, carry=carry)
     y_ref, last_ref = gc.oracle_fwd(x_host)
     tol = gc.TOL[x_host["u"].dtype]
     ey = gc.normwise(y.cpu().double().numpy(), y_ref)
@@ -75,12 +75,83 @@ def test_fwd_optional_inputs(has_z, has_D, has_bias):
     _fwd_case(x)
 
 
-def test_fwd_generic_A():
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_fwd_generic_A(dtype):
     """A that is not of the S4D-Real form (random negative diagonal)."""
-    x = make_inputs(2, 100, 700, 16, torch.float32, seed=6)
+    x = make_inputs(2, 100, 704, 16, dtype, seed=6)
     g = torch.Generator().manual_seed(9)
     x["A"] = -torch.exp(torch.randn(100, 16, generator=g))
     _fwd_case(x)
+
+
+STAGED = [  # shapes the staged kernels take (rows of 16-byte multiples, N >= 3)
+    (2, 300, 1024, 16), (1, 129, 2048, 4), (3, 40, 96, 16), (2, 256, 4096, 16), (1, 128, 64, 8),
+    (2, 70, 520, 3),
+]
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("shape", STAGED, ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("path", ["auto", "generic"])
+def test_fwd_staged_grid(shape, dtype, path):
+    b, d, L, N = shape
+    _fwd_case(make_inputs(b, d, L, N, dtype, seed=300 + L + d), path)
+
+
+@pytest.mark.parametrize("carry", ["sequential", "three_phase"])
+@pytest.mark.parametrize("chunk_len", [64, 192, 512])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_fwd_chunking_and_carry(carry, chunk_len, dtype):
+    """The state crosses chunk boundaries exactly (both hand-off schemes, chunk
+    lengths that do and do not divide L)."""
+    _fwd_case(make_inputs(2, 200, 1000, 16, dtype, seed=17), chunk_len=chunk_len, carry=carry)
+
+
+def test_fwd_chunk_size_independence():
+    """Different chunkings of the same problem agree to fp32 rounding."""
+    x = gc.to_device(make_inputs(2, 160, 2048, 16, torch.float32, seed=23))
+    outs = [gc.gpu_fwd(x, chunk_len=c, carry=m)
+            for c, m in ((2048, "sequential"), (256, "sequential"), (128, "three_phase"))]
+    for y, last in outs[1:]:
+        assert gc.normwise(y.cpu().numpy(), outs[0][0].cpu().numpy()) < 2e-6
+        assert gc.normwise(last.cpu().numpy(), outs[0][1].cpu().numpy()) < 2e-6
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_fwd_structured_scaled_A(dtype):
+    """A[d, n] = (n + 1) A[d, 0] with A[d, 0] != -1 (the general structured
+    arithmetic), one scale per channel."""
+    x = make_inputs(2, 260, 1024, 16, dtype, seed=31)
+    g = torch.Generator().manual_seed(2)
+    scale = torch.exp(torch.randn(260, 1, generator=g))
+    x["A"] = (-torch.arange(1, 17, dtype=torch.float32)[None, :] * scale).contiguous()
+    x["A"] = torch.where(torch.arange(16)[None, :] == 0, x["A"][:, :1], x["A"][:, :1] *
+                         torch.arange(1, 17, dtype=torch.float32)[None, :])
+    _fwd_case(x)
+
+
+def test_fwd_mixed_structure_groups():
+    """One channel of a group breaks the structure: that group falls back to
+    the generic arithmetic, the others keep the fast one."""
+    x = make_inputs(1, 384, 512, 16, torch.float32, seed=37)
+    x["A"][200, 5] = -5.5
+    x["A"][10, :] *= 0.5
+    _fwd_case(x)
+
+
+def test_fwd_sequential_wait_times_out_without_hanging():
+    """A chunk that never publishes its state makes the waits on it expire
+    (bounded by wait_timeout_us); the host reads MAMBA_ERR_DEVICE_TIMEOUT and
+    the context stays usable."""
+    x = gc.to_device(make_inputs(1, 256, 1024, 16, torch.bfloat16, seed=41))
+    y = torch.empty_like(x["u"])
+    scan.mamba_scan_fwd(x["u"], x["delta"], x["delta_bias"], x["A"], x["B"], x["C"], x["D"],
+                        x["z"], y, None, chunk_len=128, carry="sequential",
+                        wait_timeout_us=2000, test_hook=1)
+    assert scan.mamba_scan_stream_status() == 5  # MAMBA_ERR_DEVICE_TIMEOUT
+    assert scan.mamba_scan_stream_status() == 0  # the record is cleared
+    _fwd_case(make_inputs(1, 256, 1024, 16, torch.bfloat16, seed=41), chunk_len=128,
+              carry="sequential")
 
 
 # -------------------------------------------------- forward, full workloads
