@@ -177,12 +177,12 @@ template <int NM>
 __device__ __forceinline__ float struct_update(f2 (&H)[NM / 2], const f2 (&P)[NM / 2], float up,
                                                float yinit, const float *Brow, const float *Crow) {
   const f2 U = pk(up, up);
-  f2 Y = pk(yinit, 0.f);
+  f2 Y0 = pk(yinit, 0.f), Y1 = pk(0.f, 0.f);  // two accumulators halve the chain
   if constexpr (NM == 2) {
     const f2 b = *reinterpret_cast<const f2 *>(Brow);
     const f2 c = *reinterpret_cast<const f2 *>(Crow);
     H[0] = fma2(P[0], fma2(b, U, H[0]), H[0]);
-    Y = fma2(c, H[0], Y);
+    Y0 = fma2(c, H[0], Y0);
   } else {
 #pragma unroll
     for (int i = 0; i < NM / 2; i += 2) {
@@ -190,11 +190,11 @@ __device__ __forceinline__ float struct_update(f2 (&H)[NM / 2], const f2 (&P)[NM
       const ulonglong2 c = *reinterpret_cast<const ulonglong2 *>(Crow + 2 * i);
       H[i] = fma2(P[i], fma2(b.x, U, H[i]), H[i]);
       H[i + 1] = fma2(P[i + 1], fma2(b.y, U, H[i + 1]), H[i + 1]);
-      Y = fma2(c.x, H[i], Y);
-      Y = fma2(c.y, H[i + 1], Y);
+      Y0 = fma2(c.x, H[i], Y0);
+      Y1 = fma2(c.y, H[i + 1], Y1);
     }
   }
-  return lo_of(Y) + hi_of(Y);
+  return (lo_of(Y0) + hi_of(Y0)) + (lo_of(Y1) + hi_of(Y1));
 }
 
 // One generic step for one channel (any A): per state, Abar = exp(Delta A_n)
@@ -292,9 +292,11 @@ __global__ void __launch_bounds__(kSThreads, 2)
   constexpr int TT = Lay::TT, VEC = Lay::VEC, NV = Lay::NV, BSTR = Lay::BSTR;
   constexpr bool kOut = KIND != KIND_AGG;
 
-  extern __shared__ unsigned char smem_raw[];
-  unsigned char *sm = reinterpret_cast<unsigned char *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // Offsetting the __shared__ array itself (not a cast integer) keeps every
+  // derived pointer in the shared address space, so the compiler emits
+  // shared-memory loads and stores instead of generic ones.
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + Lay::OFF_BAR);
   int *q = reinterpret_cast<int *>(sm + Lay::OFF_Q);  // [0..7] ticket ring, [8] abort
   float *Bs = reinterpret_cast<float *>(sm + Lay::OFF_BS);
@@ -334,9 +336,14 @@ __global__ void __launch_bounds__(kSThreads, 2)
     return int((t1 - t0 + TT - 1) / TT);
   };
 
-  auto produce = [&](int stage) {
+  // Issues the next tile of this CTA's stream into stage p_issued % kStages.
+  // In the sequential hand-off the next unit is claimed only once the current
+  // one is finished (claiming early would let a unit be claimed while its
+  // predecessor is still queued behind another unit, and waits would pile up).
+  auto produce = [&](bool may_claim) {
     if (p_done) return;
     if (p_tile == p_ntiles) {
+      if (!may_claim) return;
       p_ticket = atomicAdd(p.counter, 1);
       q[p_tail & 7] = p_ticket;
       ++p_tail;
@@ -350,6 +357,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
     const int g = p_ticket % p.G, k = p_ticket / p.G;
     const int b = g / p.gpb, d0 = (g % p.gpb) * kSThreads;
     const int t0 = k * p.chunk_len + p_tile * TT;
+    const int stage = p_issued % kStages;
     unsigned char *st = sm + stage * kStageBytes;
     uint64_t *bar = &bars[stage];
     mbar_arrive_expect_tx(bar, tile_bytes);
@@ -362,8 +370,10 @@ __global__ void __launch_bounds__(kSThreads, 2)
     ++p_issued;
   };
 
+  constexpr bool kLookahead = KIND != KIND_SEQ;
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) produce(s);
+    produce(true);
+    for (int s = 1; s < kStages; ++s) produce(kLookahead);
   }
 
   int head = 0;   // consumer position in the ticket ring
@@ -543,7 +553,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
             bulk_commit();
             bulk_wait_read<1>();
           }
-          produce(stage);
+          produce(kLookahead);
         }
       }
       if constexpr (M == MODE_GEN) {
@@ -584,6 +594,10 @@ __global__ void __launch_bounds__(kSThreads, 2)
       __threadfence();
       __syncthreads();
       if (tid == 0 && !(p.test_hook == 1 && g == 0 && k == 0)) st_release_gpu(p.flags + g, k + 1);
+    }
+    if (!kLookahead && tid == 0) {  // claim the next unit and fill the free stages
+      produce(true);
+      while (!p_done && p_issued < ctile + kStages && p_tile < p_ntiles) produce(false);
     }
   }
 
