@@ -1,0 +1,781 @@
+// bwd_staged.cuh -- the staged backward of the selective scan for sm_100a.
+//
+// Gradients of the scalar sum(dy * y) with respect to every input, with the
+// states recomputed instead of stored (the recomputation of section 3.3 of
+// "Mamba: Linear-Time Sequence Modeling with Selective State Spaces",
+// paper-graph-ui summary, and of Part III section 4 of the trishampatil.com
+// walk-through).  The pages give no gradient formulas; the adjoint below is
+// derived from the forward of Knowl 1 (chapterpal.com page).
+//
+// Organisation:
+//  * The forward runs first in checkpoint mode (fwd_staged.cuh, no y): it
+//    stores the state before every 16th step, (batch, dim, L/16, N) fp32.
+//  * This kernel then walks every (channel group, chunk) unit from the last
+//    chunk to the first.  One thread owns one channel and its N states.  Per
+//    16-step tile (TMA-staged u, delta, z, dy, B, C, read in reverse order) it
+//    re-runs the tile forward from its checkpoint, keeping the state every 4
+//    steps in shared memory, then for each 4-step segment from the last
+//    re-runs the segment into registers and walks it backwards.
+//  * The adjoint of h_t is G_t = C_t dy0_t + Abar_{t+1} G_{t+1} with
+//    dy0 = dy silu(z); the thread carries Ga = Abar_t G_t, which is also the
+//    factor of dDelta.  With the structured A of the forward (decays E(n+1)
+//    from one expm1, Bbar = E(n+1) B/(n+1) / A[d,0]) the local gradients are
+//        du     = D dy0 + (1/A0) sum_n (G E) B'
+//        dDelta = A0 sum_n (n+1) Ga (h_{t-1} + B' u')        (Ga = (1+E) G)
+//        dB_n   = sum_d (G E) u' / (n+1),   dC_n = sum_d dy0 h_t
+//        dA_n   = (1/A_n) sum_t [A_n Delta (G dh/dDelta)_n - (G Bbar u)_n]
+//    the last from A_n dh/dA_n = Delta dh/dDelta - Bbar u, which needs no
+//    second derivative of psi.  Channels without that structure take the
+//    generic arithmetic (dA through psi'(x) = (x e^x - expm1 x)/x^2).
+//  * The adjoint crosses chunk boundaries backwards by the same bounded-wait
+//    hand-off as the forward (unit tickets are issued chunk-major from the
+//    end).  dB and dC (sums over channels) are reduced per warp by a
+//    butterfly, per CTA in shared memory, then across CTAs by a finalize
+//    kernel in a fixed order, as are dA, dD and the bias gradient: results
+//    are bitwise reproducible.
+#pragma once
+
+#include "bwd_reference.cuh"
+#include "fwd_staged.cuh"
+
+namespace mscan {
+
+constexpr int kBTT = kCkptEvery;  // time steps per backward tile
+constexpr int kBSeg = 4;          // time steps per recompute segment
+constexpr int kBNSeg = kBTT / kBSeg;
+constexpr int kBStages = 2;
+
+template <typename T, int NM>
+struct BwdLayout {
+  static constexpr int RB = kBTT * (int)sizeof(T);  // bytes of one channel row in a tile
+  static constexpr int TILE = kSThreads * RB;
+  static constexpr int RAW = kMaxN * RB;
+  static constexpr int STAGE = 4 * TILE + 2 * RAW;  // u, delta, z, dy, B, C
+  static constexpr int BSTR = NM + 4;
+  static constexpr int OFF_SUB = kBStages * STAGE;
+  static constexpr int OFF_BS = OFF_SUB + kBNSeg * NM * kSThreads * 4;
+  static constexpr int OFF_CS = OFF_BS + kBTT * BSTR * 4;
+  static constexpr int OFF_RED = OFF_CS + kBTT * BSTR * 4;
+  static constexpr int OFF_BAR = OFF_RED + (kSThreads / 32) * 32 * kBTT * 4;
+  static constexpr int OFF_Q = OFF_BAR + 8 * kBStages;
+  static constexpr int BYTES = OFF_Q + 16 * 4;
+  static constexpr int ALLOC = BYTES + 512;
+};
+
+struct BwdStagedArgs {
+  BwdArgs w;
+  int G, gpb, K, chunk_len, n_units;
+  int *counter;
+  int *flags;          // per group: number of later chunks whose adjoint is published
+  float *carry;        // [G][NM][128] Abar G handed to the previous chunk
+  const float *ckpt;   // [G][ceil(L/16)][NM][128] state before every 16th step
+  float *part_bc;      // [gpb][batch][32][L] per-CTA sums: dB in slots 0..15, dC in 16..31
+  float *part_A;       // [G][K][NM][128]
+  float *part_D;       // [G][K][128]
+  float *part_bias;    // [G][K][128]
+  uint64_t timeout_ns;
+  int force_generic;
+};
+
+// Byte offset of 16-byte chunk c of row r in a tile with RB-byte rows written
+// by TMA with RB-byte swizzling (chunk index XOR address bits from bit 7 up).
+template <int RB>
+__device__ __forceinline__ int swz_rows(int r, int c) {
+  return r * RB + ((c ^ ((r * RB >> 7) & (RB / 16 - 1))) << 4);
+}
+
+// kBSeg consecutive values of a row starting at segment `seg` (4 steps).
+template <typename T> struct SegIO;
+template <> struct SegIO<__nv_bfloat16> {
+  __device__ static void load(const unsigned char *tile, int r, int seg, float (&o)[4]) {
+    const uint2 v = *reinterpret_cast<const uint2 *>(tile + swz_rows<32>(r, seg >> 1) + (seg & 1) * 8);
+    o[0] = __uint_as_float(v.x << 16);
+    o[1] = __uint_as_float(v.x & 0xffff0000u);
+    o[2] = __uint_as_float(v.y << 16);
+    o[3] = __uint_as_float(v.y & 0xffff0000u);
+  }
+  __device__ static void store(__nv_bfloat16 *dst, const float (&o)[4]) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(o[0], o[1]);
+    __nv_bfloat162 b = __floats2bfloat162_rn(o[2], o[3]);
+    uint2 v;
+    v.x = *reinterpret_cast<uint32_t *>(&a);
+    v.y = *reinterpret_cast<uint32_t *>(&b);
+    *reinterpret_cast<uint2 *>(dst) = v;
+  }
+};
+template <> struct SegIO<float> {
+  __device__ static void load(const unsigned char *tile, int r, int seg, float (&o)[4]) {
+    const float4 v = *reinterpret_cast<const float4 *>(tile + swz_rows<64>(r, seg));
+    o[0] = v.x;
+    o[1] = v.y;
+    o[2] = v.z;
+    o[3] = v.w;
+  }
+  __device__ static void store(float *dst, const float (&o)[4]) {
+    *reinterpret_cast<float4 *>(dst) = make_float4(o[0], o[1], o[2], o[3]);
+  }
+};
+
+// psi'(x) = (x e^x - expm1(x)) / x^2 = sum_k (k+1)/(k+2)! x^k; the series
+// below |x| = 1/4 (truncation below 5e-8 relative), the closed form above.
+__device__ __forceinline__ float dpsi_fast(float x, float ex) {
+  const float p = 0.5f + x * (1.f / 3.f + x * (0.125f + x * (1.f / 30.f + x * (1.f / 144.f +
+                  x * (1.f / 840.f)))));
+  const float q = (x * ex - (ex - 1.f)) / (x * x);
+  return fabsf(x) < 0.25f ? p : q;
+}
+
+template <typename T, int NM>
+__global__ void __launch_bounds__(kSThreads, 2)
+    bwd_staged_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_d,
+                      const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_dy,
+                      const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_C,
+                      const BwdStagedArgs p) {
+  using Lay = BwdLayout<T, NM>;
+  constexpr int RB = Lay::RB, BSTR = Lay::BSTR;
+  constexpr int NP = NM / 2;
+
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char *sm = smem_raw + ((512u - (smem_u32(smem_raw) & 511u)) & 511u);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sm + Lay::OFF_BAR);
+  int *q = reinterpret_cast<int *>(sm + Lay::OFF_Q);
+  float *sub = reinterpret_cast<float *>(sm + Lay::OFF_SUB);  // [kBNSeg][NM][128]
+  float *Bs = reinterpret_cast<float *>(sm + Lay::OFF_BS);
+  float *Cs = reinterpret_cast<float *>(sm + Lay::OFF_CS);
+  float *red = reinterpret_cast<float *>(sm + Lay::OFF_RED);  // [4 warps][32][kBTT]
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const BwdArgs &f = p.w;
+  const int N = f.N;
+  const bool has_z = f.z != nullptr;
+  const int64_t n16 = (f.L + kBTT - 1) / kBTT;
+  const uint32_t tile_bytes = (has_z ? 4u : 3u) * Lay::TILE + 2u * uint32_t(N) * RB;
+
+  if (tid == 0) {
+#pragma unroll
+    for (int s = 0; s < kBStages; ++s) mbar_init(&bars[s], 1);
+    fence_barrier_init();
+    prefetch_tensormap(&tm_u);
+    prefetch_tensormap(&tm_d);
+    prefetch_tensormap(&tm_dy);
+    prefetch_tensormap(&tm_B);
+    prefetch_tensormap(&tm_C);
+    if (has_z) prefetch_tensormap(&tm_z);
+    q[8] = 0;
+  }
+  __syncthreads();
+
+  // ---- producer (thread 0): tiles of the current unit, last tile first
+  int p_ticket = 0, p_tile = 0, p_ntiles = 0, p_tail = 0, p_issued = 0;
+  bool p_done = false;
+  auto unit_tiles = [&](int ticket) {
+    const int k = p.K - 1 - ticket / p.G;
+    const int64_t t0 = int64_t(k) * p.chunk_len;
+    const int64_t t1 = std::min<int64_t>(f.L, t0 + p.chunk_len);
+    return int((t1 - t0 + kBTT - 1) / kBTT);
+  };
+  auto produce = [&](bool may_claim) {
+    if (p_done) return;
+    if (p_tile == p_ntiles) {
+      if (!may_claim) return;
+      p_ticket = atomicAdd(p.counter, 1);
+      q[p_tail & 7] = p_ticket;
+      ++p_tail;
+      if (p_ticket >= p.n_units) {
+        p_done = true;
+        return;
+      }
+      p_ntiles = unit_tiles(p_ticket);
+      p_tile = 0;
+    }
+    const int g = p_ticket % p.G, k = p.K - 1 - p_ticket / p.G;
+    const int b = g / p.gpb, d0 = (g % p.gpb) * kSThreads;
+    const int t0 = k * p.chunk_len + (p_ntiles - 1 - p_tile) * kBTT;
+    const int stage = p_issued % kBStages;
+    unsigned char *st = sm + stage * Lay::STAGE;
+    uint64_t *bar = &bars[stage];
+    mbar_arrive_expect_tx(bar, tile_bytes);
+    tma_load_3d(st, &tm_u, bar, t0, d0, b);
+    tma_load_3d(st + Lay::TILE, &tm_d, bar, t0, d0, b);
+    if (has_z) tma_load_3d(st + 2 * Lay::TILE, &tm_z, bar, t0, d0, b);
+    tma_load_3d(st + 3 * Lay::TILE, &tm_dy, bar, t0, d0, b);
+    tma_load_3d(st + 4 * Lay::TILE, &tm_B, bar, t0, 0, b);
+    tma_load_3d(st + 4 * Lay::TILE + Lay::RAW, &tm_C, bar, t0, 0, b);
+    ++p_tile;
+    ++p_issued;
+  };
+  if (tid == 0) {
+    produce(true);
+    for (int s = 1; s < kBStages; ++s) produce(false);
+  }
+
+  int head = 0, ctile = 0;
+  bool aborted = false;
+
+  while (true) {
+    __syncthreads();
+    const int ticket = q[head & 7];
+    ++head;
+    if (ticket >= p.n_units) break;
+    const int r = ticket / p.G;
+    const int g = ticket % p.G, k = p.K - 1 - r;
+    const int b = g / p.gpb, d0 = (g % p.gpb) * kSThreads;
+    const int d = d0 + tid;
+    const bool valid = d < f.dim;
+    const int64_t tbeg = int64_t(k) * p.chunk_len;
+    const int64_t tend = std::min<int64_t>(f.L, tbeg + p.chunk_len);
+    const int ntiles = int((tend - tbeg + kBTT - 1) / kBTT);
+    const int64_t row = (int64_t(b) * f.dim + (valid ? d : 0)) * f.L;  // row offset in (batch, dim, L)
+
+    float Arow[NM];
+#pragma unroll
+    for (int n = 0; n < NM; ++n) Arow[n] = (valid && n < N) ? f.A[int64_t(d) * N + n] : -float(n + 1);
+    if (valid) {
+      const float pad0 = (Arow[0] < 0.f && isfinite(Arow[0])) ? Arow[0] : -1.f;
+#pragma unroll
+      for (int n = 1; n < NM; ++n)
+        if (n >= N) Arow[n] = float(n + 1) * pad0;
+    }
+    const float bias = (valid && f.bias) ? f.bias[d] : 0.f;
+    const float Dd = (valid && f.D) ? f.D[d] : 0.f;
+    bool structured = Arow[0] < 0.f && isfinite(Arow[0]);
+#pragma unroll
+    for (int n = 1; n < NM; ++n) structured = structured && (Arow[n] == float(n + 1) * Arow[0]);
+    const bool sig = structured && Arow[0] == -1.f;
+    int mode = MODE_GEN;
+    if (!p.force_generic) {
+      if (__syncthreads_and(sig)) mode = MODE_SIG;
+      else if (__syncthreads_and(structured)) mode = MODE_STRUCT;
+    }
+
+    // adjoint entering from the later chunk
+    float gt[NM];
+#pragma unroll
+    for (int n = 0; n < NM; ++n) gt[n] = 0.f;
+    if (r > 0) {
+      if (tid == 0 && !wait_flag_geq(p.flags + g, r, p.timeout_ns)) {
+        record_timeout();
+        q[8] = 1;
+      }
+      __syncthreads();
+      if (q[8]) {
+        aborted = true;
+        break;
+      }
+#pragma unroll
+      for (int n = 0; n < NM; ++n) gt[n] = __ldcg(p.carry + (int64_t(g) * NM + n) * kSThreads + tid);
+    }
+    float dA[NM];
+    float dDsum = 0.f, dbsum = 0.f;
+
+    auto run = [&](auto mode_tag) {
+      constexpr int M = decltype(mode_tag)::value;
+      constexpr bool kS = M != MODE_GEN;
+      const float A0 = Arow[0];
+      const float invA0 = 1.f / A0;
+      // per-mode state: pairs for the structured arithmetic, scalars otherwise
+      f2 Gt[NP], Acc[NP];
+      float gs[NM], accs[NM], A2[NM], invA[NM];
+      if constexpr (kS) {
+#pragma unroll
+        for (int i = 0; i < NP; ++i) {
+          Gt[i] = pk(gt[2 * i], gt[2 * i + 1]);
+          Acc[i] = pk(0.f, 0.f);
+        }
+      } else {
+#pragma unroll
+        for (int n = 0; n < NM; ++n) {
+          gs[n] = gt[n];
+          accs[n] = 0.f;
+          A2[n] = Arow[n] * kLog2e;
+          invA[n] = Arow[n] != 0.f ? 1.f / Arow[n] : 0.f;
+        }
+      }
+
+      // Decays of one step: pairs (E(2i+1), E(2i+2)) for the structured
+      // arithmetic; also returns Delta and sigma(v).
+      auto step_decay = [&](float v, f2 (&P)[NP], float &Delta, float &sv) {
+        if constexpr (M == MODE_SIG) {
+          const float vc = fminf(fmaxf(v, -80.f), 80.f);
+          const float ev = ex2f(-vc * kLog2e);
+          const float s = rcpf(1.f + ev);
+          decay_pairs<NM>(-s, ev * s, P);
+          sv = s;
+          Delta = softplus_fast(v);
+        } else {
+          Delta = softplus_fast(v);
+          const float E1 = expm1_neg(Delta * A0);
+          decay_pairs<NM>(E1, 1.f + E1, P);
+          sv = rcpf(1.f + ex2f(-v * kLog2e));
+        }
+      };
+
+      for (int it = 0; it < ntiles; ++it, ++ctile) {
+        const int tile = ntiles - 1 - it;  // tiles run from the end of the chunk
+        const int64_t t0 = tbeg + int64_t(tile) * kBTT;
+        const int steps = int(std::min<int64_t>(kBTT, tend - t0));
+        const int nseg = steps / kBSeg;
+        const int stage = ctile % kBStages;
+        const uint32_t parity = uint32_t(ctile / kBStages) & 1u;
+        unsigned char *st = sm + stage * Lay::STAGE;
+        // checkpoint of the tile start (issued before the wait to overlap)
+        float h0[NM];
+        {
+          const float *ck = p.ckpt + ((int64_t(g) * n16 + t0 / kBTT) * NM) * kSThreads + tid;
+#pragma unroll
+          for (int n = 0; n < NM; ++n) h0[n] = __ldcg(ck + n * kSThreads);
+        }
+        if (!mbar_wait_bounded(&bars[stage], parity, p.timeout_ns)) {
+          record_timeout();
+          q[8] = 1;
+        }
+        {
+          const T *Braw = reinterpret_cast<const T *>(st + 4 * Lay::TILE);
+          const T *Craw = reinterpret_cast<const T *>(st + 4 * Lay::TILE + Lay::RAW);
+          constexpr int ITEMS = NM * (kBTT / 4);
+          for (int w = tid; w < 2 * ITEMS; w += kSThreads) {
+            const bool isC = w >= ITEMS;
+            const int rr = isC ? w - ITEMS : w;
+            const int n = rr % NM, tg = rr / NM;
+            const T *src = (isC ? Craw : Braw) + n * kBTT + 4 * tg;
+            float *dst = (isC ? Cs : Bs) + 4 * tg * BSTR + n;
+            const float scale = (!isC && kS) ? 1.f / float(n + 1) : 1.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i * BSTR] = n < N ? raw_to_f(src, i) * scale : 0.f;
+          }
+        }
+        __syncthreads();
+        if (q[8]) return;
+
+        const unsigned char *su = st;
+        const unsigned char *sd = st + Lay::TILE;
+        const unsigned char *sz = st + 2 * Lay::TILE;
+        const unsigned char *sdy = st + 3 * Lay::TILE;
+
+        // forward over the tile: the state before every segment -> shared memory
+        {
+          f2 H[NP];
+          float h[NM];
+          if constexpr (kS) {
+#pragma unroll
+            for (int i = 0; i < NP; ++i) H[i] = pk(h0[2 * i], h0[2 * i + 1]);
+          } else {
+#pragma unroll
+            for (int n = 0; n < NM; ++n) h[n] = h0[n];
+          }
+          for (int seg = 0; seg < nseg; ++seg) {
+            float *sp = sub + (seg * NM) * kSThreads + tid;
+            if constexpr (kS) {
+#pragma unroll
+              for (int i = 0; i < NP; ++i) {
+                sp[(2 * i) * kSThreads] = lo_of(H[i]);
+                sp[(2 * i + 1) * kSThreads] = hi_of(H[i]);
+              }
+            } else {
+#pragma unroll
+              for (int n = 0; n < NM; ++n) sp[n * kSThreads] = h[n];
+            }
+            if (seg == nseg - 1) break;  // the last segment is re-run below anyway
+            float uv[4], dv[4];
+            SegIO<T>::load(su, tid, seg, uv);
+            SegIO<T>::load(sd, tid, seg, dv);
+#pragma unroll
+            for (int i = 0; i < kBSeg; ++i) {
+              const float *Brow = Bs + (seg * kBSeg + i) * BSTR;
+              if constexpr (kS) {
+                f2 P[NP];
+                float Delta, sv;
+                step_decay(dv[i] + bias, P, Delta, sv);
+                struct_update<NM>(H, P, uv[i] * invA0, 0.f, Brow, Brow);
+              } else {
+                const float Delta = softplus_fast(dv[i] + bias);
+                generic_update<NM>(h, Delta, uv[i], 0.f, Arow, A2, invA, Brow, Brow);
+              }
+            }
+          }
+        }
+
+        // segments from the last: re-run into registers, then walk backwards
+        for (int seg = nseg - 1; seg >= 0; --seg) {
+          float uv[4], dv[4], zv[4], dyv[4];
+          SegIO<T>::load(su, tid, seg, uv);
+          SegIO<T>::load(sd, tid, seg, dv);
+          SegIO<T>::load(sdy, tid, seg, dyv);
+          if (has_z) SegIO<T>::load(sz, tid, seg, zv);
+          float du_o[4], dd_o[4], dz_o[4];
+          const float *sp = sub + (seg * NM) * kSThreads + tid;
+
+          if constexpr (kS) {
+            f2 Hs[kBSeg + 1][NP];
+#pragma unroll
+            for (int i = 0; i < NP; ++i)
+              Hs[0][i] = pk(sp[(2 * i) * kSThreads], sp[(2 * i + 1) * kSThreads]);
+#pragma unroll
+            for (int i = 0; i < kBSeg; ++i) {
+              const float *Brow = Bs + (seg * kBSeg + i) * BSTR;
+              f2 P[NP];
+              float Delta, sv;
+              step_decay(dv[i] + bias, P, Delta, sv);
+#pragma unroll
+              for (int j = 0; j < NP; ++j) Hs[i + 1][j] = Hs[i][j];
+              struct_update<NM>(Hs[i + 1], P, uv[i] * invA0, 0.f, Brow, Brow);
+            }
+#pragma unroll
+            for (int i = kBSeg - 1; i >= 0; --i) {
+              const int tl = seg * kBSeg + i;
+              const float *Brow = Bs + tl * BSTR;
+              const float *Crow = Cs + tl * BSTR;
+              f2 P[NP];
+              float Delta, sv;
+              step_decay(dv[i] + bias, P, Delta, sv);
+              float dy0 = dyv[i], sz = 0.f;
+              if (has_z) {
+                sz = rcpf(1.f + ex2f(-zv[i] * kLog2e));
+                dy0 *= zv[i] * sz;
+              }
+              const float up = uv[i] * invA0;
+              const float x1 = Delta * A0;
+              const f2 U = pk(up, up), DY = pk(dy0, dy0), X1n = pk(-x1, -x1), Z = pk(0.f, 0.f);
+              f2 DU = Z, DD = Z, Y0 = Z;
+              float vals[32];
+#pragma unroll
+              for (int j = 0; j < NP; j += 2) {
+                const ulonglong2 bq = *reinterpret_cast<const ulonglong2 *>(Brow + 2 * j);
+                const ulonglong2 cq2 = *reinterpret_cast<const ulonglong2 *>(Crow + 2 * j);
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                  const int jj = j + e;
+                  const f2 Bp = e ? bq.y : bq.x;
+                  const f2 Cp = e ? cq2.y : cq2.x;
+                  const f2 CN = pk(float(2 * jj + 1), float(2 * jj + 2));
+                  const f2 Gv = fma2(Cp, DY, Gt[jj]);
+                  const f2 Ga = fma2(Gv, P[jj], Gv);
+                  const f2 w = fma2(Gv, P[jj], Z);
+                  const f2 t1 = fma2(Bp, U, Hs[i][jj]);
+                  const f2 cq = fma2(fma2(Ga, t1, Z), CN, Z);
+                  DD = fma2(cq, pk(1.f, 1.f), DD);
+                  Acc[jj] = fma2(X1n, cq, Acc[jj]);
+                  const f2 dBc = fma2(w, U, Z);
+                  Acc[jj] = fma2(dBc, Bp, Acc[jj]);
+                  DU = fma2(w, Bp, DU);
+                  Y0 = fma2(Cp, Hs[i + 1][jj], Y0);
+                  const f2 dCc = fma2(DY, Hs[i + 1][jj], Z);
+                  Gt[jj] = Ga;
+                  vals[2 * jj] = lo_of(dBc);
+                  vals[2 * jj + 1] = hi_of(dBc);
+                  vals[kMaxN + 2 * jj] = lo_of(dCc);
+                  vals[kMaxN + 2 * jj + 1] = hi_of(dCc);
+                }
+              }
+#pragma unroll
+              for (int n = NM; n < kMaxN; ++n) vals[n] = vals[kMaxN + n] = 0.f;
+              if (!valid) {
+#pragma unroll
+                for (int n = 0; n < 32; ++n) vals[n] = 0.f;
+              }
+              const float du = fmaf(lo_of(DU) + hi_of(DU), invA0, Dd * dy0);
+              const float dd = A0 * (lo_of(DD) + hi_of(DD)) * sv;
+              const float y0 = (lo_of(Y0) + hi_of(Y0)) + Dd * uv[i];
+              du_o[i] = du;
+              dd_o[i] = dd;
+              dz_o[i] = has_z ? dyv[i] * y0 * sz * (1.f + zv[i] * (1.f - sz)) : 0.f;
+              dDsum = fmaf(dy0, uv[i], dDsum);
+              dbsum += dd;
+              const float rsum = warp_reduce_scatter32(vals, lane);
+              // lane l holds dB (l < 16, to be divided by l+1) or dC of state l-16
+              red[(warp * 32 + lane) * kBTT + tl] = (lane < kMaxN) ? rsum * (1.f / float(lane + 1)) : rsum;
+            }
+          } else {
+            float Hs[kBSeg + 1][NM];
+#pragma unroll
+            for (int n = 0; n < NM; ++n) Hs[0][n] = sp[n * kSThreads];
+#pragma unroll
+            for (int i = 0; i < kBSeg; ++i) {
+              const float *Brow = Bs + (seg * kBSeg + i) * BSTR;
+              const float Delta = softplus_fast(dv[i] + bias);
+#pragma unroll
+              for (int n = 0; n < NM; ++n) Hs[i + 1][n] = Hs[i][n];
+              generic_update<NM>(Hs[i + 1], Delta, uv[i], 0.f, Arow, A2, invA, Brow, Brow);
+            }
+#pragma unroll
+            for (int i = kBSeg - 1; i >= 0; --i) {
+              const int tl = seg * kBSeg + i;
+              const float *Brow = Bs + tl * BSTR;
+              const float *Crow = Cs + tl * BSTR;
+              const float v = dv[i] + bias;
+              const float Delta = softplus_fast(v);
+              const float sv = rcpf(1.f + ex2f(-v * kLog2e));
+              float dy0 = dyv[i], sz = 0.f;
+              if (has_z) {
+                sz = rcpf(1.f + ex2f(-zv[i] * kLog2e));
+                dy0 *= zv[i] * sz;
+              }
+              float du_acc = 0.f, dD_acc = 0.f, y0 = Dd * uv[i];
+              float vals[32];
+#pragma unroll
+              for (int n = 0; n < NM; ++n) {
+                const float x = Delta * Arow[n];
+                const float a = ex2f(Delta * A2[n]);
+                float pp = fmaf(x, 1.f / 720.f, 1.f / 120.f);
+                pp = fmaf(x, pp, 1.f / 24.f);
+                pp = fmaf(x, pp, 1.f / 6.f);
+                pp = fmaf(x, pp, 0.5f);
+                pp = fmaf(x, pp, 1.f);
+                const float Eb = fabsf(x) < 0.25f ? Delta * pp : (a - 1.f) * invA[n];  // Bbar / B
+                const float Bn = Brow[n], Cn = Crow[n];
+                const float hprev = Hs[i][n], hcur = Hs[i + 1][n];
+                const float Gv = fmaf(Cn, dy0, gs[n]);
+                const float Ga = a * Gv;
+                const float wv = Gv * Eb;
+                du_acc = fmaf(wv, Bn, du_acc);
+                dD_acc = fmaf(Ga, fmaf(Bn, uv[i], Arow[n] * hprev), dD_acc);
+                accs[n] = fmaf(Gv, Delta * a * hprev + Bn * uv[i] * Delta * Delta * dpsi_fast(x, a), accs[n]);
+                y0 = fmaf(Cn, hcur, y0);
+                vals[n] = wv * uv[i];
+                vals[kMaxN + n] = dy0 * hcur;
+                gs[n] = Ga;
+              }
+#pragma unroll
+              for (int n = NM; n < kMaxN; ++n) vals[n] = vals[kMaxN + n] = 0.f;
+              if (!valid) {
+#pragma unroll
+                for (int n = 0; n < 32; ++n) vals[n] = 0.f;
+              }
+              const float dd = dD_acc * sv;
+              du_o[i] = fmaf(Dd, dy0, du_acc);
+              dd_o[i] = dd;
+              dz_o[i] = has_z ? dyv[i] * y0 * sz * (1.f + zv[i] * (1.f - sz)) : 0.f;
+              dDsum = fmaf(dy0, uv[i], dDsum);
+              dbsum += dd;
+              red[(warp * 32 + lane) * kBTT + tl] = warp_reduce_scatter32(vals, lane);
+            }
+          }
+          if (valid) {
+            const int64_t o = row + t0 + seg * kBSeg;
+            SegIO<T>::store(static_cast<T *>(f.du) + o, du_o);
+            SegIO<T>::store(static_cast<T *>(f.ddelta) + o, dd_o);
+            if (has_z) SegIO<T>::store(static_cast<T *>(f.dz) + o, dz_o);
+          }
+        }
+        __syncthreads();
+        // CTA sums of dB / dC for this tile -> partials
+        for (int idx = tid; idx < 32 * kBTT; idx += kSThreads) {
+          const int slot = idx / kBTT, tl = idx % kBTT;
+          if (tl < steps) {
+            float sum = 0.f;
+#pragma unroll
+            for (int wv = 0; wv < kSThreads / 32; ++wv) sum += red[(wv * 32 + slot) * kBTT + tl];
+            p.part_bc[((int64_t(g % p.gpb) * f.batch + b) * 32 + slot) * f.L + t0 + tl] = sum;
+          }
+        }
+        if (tid == 0) produce(false);
+      }
+      // unit results
+      if constexpr (kS) {
+#pragma unroll
+        for (int i = 0; i < NP; ++i) {
+          gt[2 * i] = lo_of(Gt[i]);
+          gt[2 * i + 1] = hi_of(Gt[i]);
+          // Acc holds -A_n dA_n
+          dA[2 * i] = -lo_of(Acc[i]) / Arow[2 * i];
+          dA[2 * i + 1] = -hi_of(Acc[i]) / Arow[2 * i + 1];
+        }
+      } else {
+#pragma unroll
+        for (int n = 0; n < NM; ++n) {
+          gt[n] = gs[n];
+          dA[n] = accs[n];
+        }
+      }
+    };
+
+    if (mode == MODE_SIG) run(std::integral_constant<int, MODE_SIG>{});
+    else if (mode == MODE_STRUCT) run(std::integral_constant<int, MODE_STRUCT>{});
+    else run(std::integral_constant<int, MODE_GEN>{});
+    if (q[8]) {
+      aborted = true;
+      break;
+    }
+
+    const int64_t pu = int64_t(g) * p.K + k;
+#pragma unroll
+    for (int n = 0; n < NM; ++n) p.part_A[(pu * NM + n) * kSThreads + tid] = valid ? dA[n] : 0.f;
+    p.part_D[pu * kSThreads + tid] = valid ? dDsum : 0.f;
+    p.part_bias[pu * kSThreads + tid] = valid ? dbsum : 0.f;
+    if (k > 0) {
+#pragma unroll
+      for (int n = 0; n < NM; ++n) p.carry[(int64_t(g) * NM + n) * kSThreads + tid] = gt[n];
+      __threadfence();
+      __syncthreads();
+      if (tid == 0) st_release_gpu(p.flags + g, r + 1);
+    }
+    if (tid == 0) {  // claim the next unit and fill the free stages
+      produce(true);
+      while (!p_done && p_issued < ctile + kBStages && p_tile < p_ntiles) produce(false);
+    }
+  }
+
+  __syncthreads();
+  if (tid == 0 && aborted) {
+    for (int t = ctile; t < p_issued; ++t)
+      mbar_wait_bounded(&bars[t % kBStages], uint32_t(t / kBStages) & 1u, p.timeout_ns);
+  }
+}
+
+// dB / dC: sum of the per-CTA partials over the channel groups of a batch row.
+template <typename T>
+__global__ void bwd_staged_finalize_bc(const BwdStagedArgs p) {
+  const BwdArgs &f = p.w;
+  const int64_t total = f.batch * f.N * f.L;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t t = i % f.L, n = (i / f.L) % f.N, b = i / (f.L * f.N);
+    float sb = 0.f, sc = 0.f;
+    for (int j = 0; j < p.gpb; ++j) {
+      const float *pp = p.part_bc + ((int64_t(j) * f.batch + b) * 32) * f.L + t;
+      sb += pp[n * f.L];
+      sc += pp[(kMaxN + n) * f.L];
+    }
+    static_cast<T *>(f.dB)[i] = from_f<T>(sb);
+    static_cast<T *>(f.dC)[i] = from_f<T>(sc);
+  }
+}
+
+// dA, dD, dbias: sums over batch rows and chunks of the per-unit partials.
+template <int NM>
+__global__ void bwd_staged_finalize_params(const BwdStagedArgs p) {
+  const BwdArgs &f = p.w;
+  const int64_t total = f.dim * f.N;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t d = i / f.N, n = i % f.N;
+    const int64_t gi = d / kSThreads, c = d % kSThreads;
+    float s = 0.f, sd = 0.f, sb = 0.f;
+    for (int64_t b = 0; b < f.batch; ++b) {
+      const int64_t g = b * p.gpb + gi;
+      for (int k = 0; k < p.K; ++k) {
+        const int64_t pu = g * p.K + k;
+        s += p.part_A[(pu * NM + n) * kSThreads + c];
+        if (n == 0) {
+          sd += p.part_D[pu * kSThreads + c];
+          sb += p.part_bias[pu * kSThreads + c];
+        }
+      }
+    }
+    f.dA[i] = s;
+    if (n == 0) {
+      if (f.dD) f.dD[d] = sd;
+      if (f.dbias) f.dbias[d] = sb;
+    }
+  }
+}
+
+// Whether the staged backward takes this problem (as the staged forward).
+inline bool staged_bwd_supported(const BwdArgs &a, size_t es) {
+  auto al = [](const void *ptr) { return ptr == nullptr || (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; };
+  if (a.N < 3) return false;
+  if ((a.L * int64_t(es)) % 16 != 0 || a.L % kBSeg != 0) return false;
+  if (a.L > (int64_t(1) << 31) - 1024 || a.dim > (int64_t(1) << 31) - 1) return false;
+  return al(a.u) && al(a.delta) && al(a.z) && al(a.dy) && al(a.B) && al(a.C) && al(a.du) &&
+         al(a.ddelta) && al(a.dz);
+}
+
+template <typename T, int NM>
+mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStream_t s,
+                               mamba_status_t (*launched)()) {
+  using Lay = BwdLayout<T, NM>;
+  constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
+  const uint64_t L = a.L, dim = a.dim, batch = a.batch, N = a.N;
+  const CUtensorMapSwizzle sw = bf16 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B;
+  const CUtensorMapSwizzle none = CU_TENSOR_MAP_SWIZZLE_NONE;
+  CUtensorMap maps[6];
+  if (!make_map_3d(&maps[0], a.u, bf16, L, dim, batch, kBTT, kSThreads, sw) ||
+      !make_map_3d(&maps[1], a.delta, bf16, L, dim, batch, kBTT, kSThreads, sw) ||
+      !make_map_3d(&maps[2], a.z ? a.z : a.u, bf16, L, dim, batch, kBTT, kSThreads, sw) ||
+      !make_map_3d(&maps[3], a.dy, bf16, L, dim, batch, kBTT, kSThreads, sw) ||
+      !make_map_3d(&maps[4], a.B, bf16, L, N, batch, kBTT, uint32_t(N), none) ||
+      !make_map_3d(&maps[5], a.C, bf16, L, N, batch, kBTT, uint32_t(N), none)) {
+    return MAMBA_ERR_UNSUPPORTED;
+  }
+  auto kern = bwd_staged_kernel<T, NM>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::ALLOC) != cudaSuccess)
+    return MAMBA_ERR_CUDA;
+  int bps = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, kern, kSThreads, Lay::ALLOC) != cudaSuccess)
+    return MAMBA_ERR_CUDA;
+  const int sms = device_sm_count();
+  const int slots = sms * std::max(1, bps);
+  const int64_t gpb = ceil_div(a.dim, kSThreads);
+  const int64_t G = int64_t(a.batch) * gpb;
+  if (G > (int64_t(1) << 30)) return MAMBA_ERR_UNSUPPORTED;
+  StagedOptions ro = o;
+  ro.carry = 1;  // the adjoint crosses chunks by the sequential hand-off
+  StagedPlan pl = plan_staged(G, a.L, slots, ro);
+  if (G * pl.K > (int64_t(1) << 30)) return MAMBA_ERR_UNSUPPORTED;
+  const int64_t n16 = ceil_div(a.L, kBTT);
+
+  // workspace: [ints][ckpt][carry][part_bc][part_A][part_D][part_bias]
+  const size_t int_bytes = ceil_div((1 + size_t(G)) * 4, 256) * 256;
+  const size_t n_ckpt = size_t(G) * size_t(n16) * NM * kSThreads;
+  const size_t n_carry = size_t(G) * NM * kSThreads;
+  const size_t n_bc = size_t(gpb) * size_t(a.batch) * 32 * size_t(a.L);
+  const size_t gk = size_t(G) * size_t(pl.K);
+  const size_t n_A = gk * NM * kSThreads, n_D = gk * kSThreads;
+  const size_t bytes = int_bytes + 4 * (n_ckpt + n_carry + n_bc + n_A + 2 * n_D);
+  unsigned char *ws = nullptr;
+  if (cudaMallocAsync(reinterpret_cast<void **>(&ws), bytes, s) != cudaSuccess) {
+    cudaGetLastError();
+    return MAMBA_ERR_OUT_OF_MEMORY;
+  }
+  BwdStagedArgs bp;
+  bp.w = a;
+  bp.G = int(G);
+  bp.gpb = int(gpb);
+  bp.K = pl.K;
+  bp.chunk_len = pl.chunk_len;
+  bp.n_units = int(gk);
+  bp.counter = reinterpret_cast<int *>(ws);
+  bp.flags = bp.counter + 1;
+  float *fws = reinterpret_cast<float *>(ws + int_bytes);
+  float *ckpt = fws;
+  bp.ckpt = ckpt;
+  bp.carry = ckpt + n_ckpt;
+  bp.part_bc = bp.carry + n_carry;
+  bp.part_A = bp.part_bc + n_bc;
+  bp.part_D = bp.part_A + n_A;
+  bp.part_bias = bp.part_D + n_D;
+  bp.timeout_ns = o.timeout_us > 0 ? uint64_t(o.timeout_us) * 1000ull : kDefaultTimeoutNs;
+  bp.force_generic = o.path == MAMBA_PATH_GENERIC ? 1 : 0;
+
+  mamba_status_t st = MAMBA_OK;
+  if (cudaMemsetAsync(ws, 0, int_bytes, s) != cudaSuccess) st = MAMBA_ERR_CUDA;
+  if (st == MAMBA_OK) {
+    FwdArgs fa;
+    fa.u = a.u; fa.delta = a.delta; fa.z = nullptr; fa.B = a.B; fa.C = a.C;
+    fa.bias = a.bias; fa.A = a.A; fa.D = nullptr; fa.y = nullptr; fa.last_state = nullptr;
+    fa.batch = a.batch; fa.dim = a.dim; fa.L = a.L; fa.N = a.N;
+    StagedOptions fo = o;
+    fo.chunk_len = 0;
+    fo.carry = 0;
+    st = staged_forward<T, NM>(fa, fo, s, launched, ckpt);
+  }
+  if (st == MAMBA_OK) {
+    kern<<<unsigned(std::min<int64_t>(gk, slots)), kSThreads, Lay::ALLOC, s>>>(
+        maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], bp);
+    st = launched();
+  }
+  if (st == MAMBA_OK) {
+    const int64_t nbc = a.batch * a.N * a.L;
+    bwd_staged_finalize_bc<T><<<unsigned(std::min<int64_t>(ceil_div(nbc, 256), sms * 8)), 256, 0, s>>>(bp);
+    st = launched();
+  }
+  if (st == MAMBA_OK) {
+    const int64_t np = a.dim * a.N;
+    bwd_staged_finalize_params<NM><<<unsigned(std::min<int64_t>(ceil_div(np, 256), sms * 8)), 256, 0, s>>>(bp);
+    st = launched();
+  }
+  if (cudaFreeAsync(ws, s) != cudaSuccess && st == MAMBA_OK) st = MAMBA_ERR_CUDA;
+  return st;
+}
+
+}  // namespace mscan

@@ -60,7 +60,11 @@ constexpr int kRawBytes = kMaxN * kRowBytes;          // 1 KB per B / C tile
 constexpr int kStageBytes = 3 * kTileBytes + 2 * kRawBytes;
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
 
-enum StagedKind { KIND_SEQ = 0, KIND_PAR = 1, KIND_AGG = 2 };
+// SEQ / PAR: the forward with y.  AGG: chunk aggregates for PAR.  CKPT_SEQ /
+// CKPT_PAR: the forward without y that stores the state every kCkptEvery
+// steps (the checkpoints the backward recomputes from).
+enum StagedKind { KIND_SEQ = 0, KIND_PAR = 1, KIND_AGG = 2, KIND_CKPT_SEQ = 3, KIND_CKPT_PAR = 4 };
+constexpr int kCkptEvery = 16;
 enum UnitMode { MODE_SIG = 0, MODE_STRUCT = 1, MODE_GEN = 2 };
 
 struct StagedArgs {
@@ -76,6 +80,7 @@ struct StagedArgs {
   float *agg_h;    // PAR: [G][K][NM][128] state each chunk produces from zero
   double *agg_S;   // PAR: [G][K][128] sum of Delta over each chunk
   float *hin;      // PAR: [G][K][NM][128] state entering each chunk
+  float *ckpt;     // CKPT: [G][ceil(L/16)][NM][128] state before every 16th step
   uint64_t timeout_ns;
   int test_hook;   // 1: unit (group 0, chunk 0) never publishes (tests the bounded wait)
   int force_generic;  // 1: generic arithmetic for every channel
@@ -290,7 +295,10 @@ __global__ void __launch_bounds__(kSThreads, 2)
                       const StagedArgs p) {
   using Lay = StagedLayout<T, NM>;
   constexpr int TT = Lay::TT, VEC = Lay::VEC, NV = Lay::NV, BSTR = Lay::BSTR;
-  constexpr bool kOut = KIND != KIND_AGG;
+  constexpr bool kOut = KIND == KIND_SEQ || KIND == KIND_PAR;  // computes and stores y
+  constexpr bool kSeq = KIND == KIND_SEQ || KIND == KIND_CKPT_SEQ;
+  constexpr bool kPar = KIND == KIND_PAR || KIND == KIND_CKPT_PAR;
+  constexpr bool kCkpt = KIND == KIND_CKPT_SEQ || KIND == KIND_CKPT_PAR;
 
   // Offsetting the __shared__ array itself (not a cast integer) keeps every
   // derived pointer in the shared address space, so the compiler emits
@@ -370,7 +378,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
     ++p_issued;
   };
 
-  constexpr bool kLookahead = KIND != KIND_SEQ;
+  constexpr bool kLookahead = !kSeq;
   if (tid == 0) {
     produce(true);
     for (int s = 1; s < kStages; ++s) produce(kLookahead);
@@ -419,7 +427,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
     float hs[NM];
 #pragma unroll
     for (int n = 0; n < NM; ++n) hs[n] = 0.f;
-    if (KIND == KIND_SEQ && k > 0) {
+    if (kSeq && k > 0) {
       if (tid == 0 && !wait_flag_geq(p.flags + g, k, p.timeout_ns)) {
         record_timeout();
         q[8] = 1;
@@ -431,7 +439,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
       }
 #pragma unroll
       for (int n = 0; n < NM; ++n) hs[n] = __ldcg(p.carry + (int64_t(g) * NM + n) * kSThreads + tid);
-    } else if (KIND == KIND_PAR && k > 0) {
+    } else if (kPar && k > 0) {
 #pragma unroll
       for (int n = 0; n < NM; ++n)
         hs[n] = __ldcg(p.hin + ((int64_t(g) * p.K + k) * NM + n) * kSThreads + tid);
@@ -494,6 +502,23 @@ __global__ void __launch_bounds__(kSThreads, 2)
         unsigned char *sy = sm + Lay::OFF_Y + (ctile & 1) * kTileBytes;
         for (int j = 0; j < NV; ++j) {
           if (t0 + int64_t(j) * VEC >= tend) break;  // past the end of the sequence
+          if constexpr (kCkpt) {
+            const int64_t tj = t0 + int64_t(j) * VEC;
+            if (tj % kCkptEvery == 0) {
+              float *dst = p.ckpt + ((int64_t(g) * ((f.L + kCkptEvery - 1) / kCkptEvery) +
+                                      tj / kCkptEvery) * NM) * kSThreads + tid;
+              if constexpr (M == MODE_GEN) {
+#pragma unroll
+                for (int n = 0; n < NM; ++n) dst[n * kSThreads] = h[n];
+              } else {
+#pragma unroll
+                for (int i = 0; i < NM / 2; ++i) {
+                  dst[(2 * i) * kSThreads] = lo_of(H[i]);
+                  dst[(2 * i + 1) * kSThreads] = hi_of(H[i]);
+                }
+              }
+            }
+          }
           const int off = swz64(tid, j);
           float uv[VEC], dv[VEC], zv[VEC], yv[VEC];
           Vec<T>::unpack(*reinterpret_cast<const uint4 *>(su + off), uv);
@@ -516,7 +541,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
                 y0 = struct_update<NM>(H, P, -uv[i], Dd * uv[i], Brow, Crow);
               } else {
                 struct_update<NM>(H, P, -uv[i], 0.f, Brow, Brow);
-                Ssum += double(softplus_fast(v));
+                if constexpr (KIND == KIND_AGG) Ssum += double(softplus_fast(v));
               }
             } else if constexpr (M == MODE_STRUCT) {
               const float Delta = softplus_fast(v);
@@ -527,13 +552,13 @@ __global__ void __launch_bounds__(kSThreads, 2)
                 y0 = struct_update<NM>(H, P, uv[i] * invA0, Dd * uv[i], Brow, Crow);
               } else {
                 struct_update<NM>(H, P, uv[i] * invA0, 0.f, Brow, Brow);
-                Ssum += double(Delta);
+                if constexpr (KIND == KIND_AGG) Ssum += double(Delta);
               }
             } else {
               const float Delta = softplus_fast(v);
               y0 = generic_update<NM>(h, Delta, uv[i], Dd * uv[i], Arow, A2, invA, Brow,
                                       kOut ? Crow : Brow);
-              if (!kOut) Ssum += double(Delta);
+              if constexpr (KIND == KIND_AGG) Ssum += double(Delta);
             }
             if (kOut) {
               if (has_z) {
@@ -583,12 +608,12 @@ __global__ void __launch_bounds__(kSThreads, 2)
         p.agg_h[((int64_t(g) * p.K + k) * NM + n) * kSThreads + tid] = hs[n];
       p.agg_S[(int64_t(g) * p.K + k) * kSThreads + tid] = Ssum;
     } else if (k == p.K - 1) {
-      if (valid && f.last_state) {
+      if (kOut && valid && f.last_state) {
 #pragma unroll
         for (int n = 0; n < NM; ++n)
           if (n < N) f.last_state[(int64_t(b) * f.dim + d) * N + n] = hs[n];
       }
-    } else if (KIND == KIND_SEQ) {
+    } else if (kSeq) {
 #pragma unroll
       for (int n = 0; n < NM; ++n) p.carry[(int64_t(g) * NM + n) * kSThreads + tid] = hs[n];
       __threadfence();
@@ -705,9 +730,11 @@ inline StagedPlan plan_staged(int64_t G, int64_t L, int slots, const StagedOptio
 // The staged forward: tensor maps, plan, stream-ordered workspace, launches.
 // Returns MAMBA_ERR_UNSUPPORTED (nothing enqueued) if the driver rejects a
 // tensor map.
+// With `ckpt` non-null the forward runs without y and stores the state before
+// every kCkptEvery-th step into ckpt ([G][ceil(L/16)][NM][128] floats).
 template <typename T, int NM>
 mamba_status_t staged_forward(const FwdArgs &a, const StagedOptions &o, cudaStream_t s,
-                              mamba_status_t (*launched)()) {
+                              mamba_status_t (*launched)(), float *ckpt = nullptr) {
   using Lay = StagedLayout<T, NM>;
   constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
   CUtensorMap maps[6];
@@ -716,7 +743,7 @@ mamba_status_t staged_forward(const FwdArgs &a, const StagedOptions &o, cudaStre
   if (!make_map_3d(&maps[0], a.u, bf16, L, dim, batch, Lay::TT, kSThreads, sw) ||
       !make_map_3d(&maps[1], a.delta, bf16, L, dim, batch, Lay::TT, kSThreads, sw) ||
       !make_map_3d(&maps[2], a.z ? a.z : a.u, bf16, L, dim, batch, Lay::TT, kSThreads, sw) ||
-      !make_map_3d(&maps[3], a.y, bf16, L, dim, batch, Lay::TT, kSThreads, sw) ||
+      !make_map_3d(&maps[3], a.y ? a.y : a.u, bf16, L, dim, batch, Lay::TT, kSThreads, sw) ||
       !make_map_3d(&maps[4], a.B, bf16, L, N, batch, Lay::TT, uint32_t(N), none) ||
       !make_map_3d(&maps[5], a.C, bf16, L, N, batch, Lay::TT, uint32_t(N), none)) {
     return MAMBA_ERR_UNSUPPORTED;
@@ -743,6 +770,7 @@ mamba_status_t staged_forward(const FwdArgs &a, const StagedOptions &o, cudaStre
   sa.flags = nullptr;
   sa.carry = sa.agg_h = sa.hin = nullptr;
   sa.agg_S = nullptr;
+  sa.ckpt = ckpt;
 
   // workspace: [ints: 2 counters + G flags][carry | agg_h, agg_S, hin]
   const size_t n_int = 2 + size_t(G);
@@ -768,15 +796,22 @@ mamba_status_t staged_forward(const FwdArgs &a, const StagedOptions &o, cudaStre
     sa.counter = counters;
     sa.n_units = int(gk);
     const int grid = int(std::min<int64_t>(gk, slots));
-    launch_staged<T, NM, KIND_SEQ>(maps, sa, grid, s);
-    st = launched();
+    if (ckpt) {
+      int bps = 0;
+      if (prepare_kernel<T, NM, KIND_CKPT_SEQ>(&bps) != cudaSuccess) st = MAMBA_ERR_CUDA;
+      else launch_staged<T, NM, KIND_CKPT_SEQ>(maps, sa, int(std::min<int64_t>(gk, sms * std::max(1, bps))), s);
+    } else {
+      launch_staged<T, NM, KIND_SEQ>(maps, sa, grid, s);
+    }
+    if (st == MAMBA_OK) st = launched();
   } else if (st == MAMBA_OK) {
     sa.agg_S = reinterpret_cast<double *>(ws + int_bytes);
     sa.agg_h = reinterpret_cast<float *>(ws + int_bytes + gk * kSThreads * 8);
     sa.hin = sa.agg_h + gk * NM * kSThreads;
     int bps_agg = 0, bps_par = 0;
     if (prepare_kernel<T, NM, KIND_AGG>(&bps_agg) != cudaSuccess ||
-        prepare_kernel<T, NM, KIND_PAR>(&bps_par) != cudaSuccess) {
+        (ckpt ? prepare_kernel<T, NM, KIND_CKPT_PAR>(&bps_par)
+              : prepare_kernel<T, NM, KIND_PAR>(&bps_par)) != cudaSuccess) {
       st = MAMBA_ERR_CUDA;
     }
     if (st == MAMBA_OK) {
@@ -795,7 +830,9 @@ mamba_status_t staged_forward(const FwdArgs &a, const StagedOptions &o, cudaStre
       StagedArgs sm = sa;
       sm.counter = counters + 1;
       sm.n_units = int(gk);
-      launch_staged<T, NM, KIND_PAR>(maps, sm, int(std::min<int64_t>(gk, sms * std::max(1, bps_par))), s);
+      const int grid = int(std::min<int64_t>(gk, sms * std::max(1, bps_par)));
+      if (ckpt) launch_staged<T, NM, KIND_CKPT_PAR>(maps, sm, grid, s);
+      else launch_staged<T, NM, KIND_PAR>(maps, sm, grid, s);
       st = launched();
     }
   }

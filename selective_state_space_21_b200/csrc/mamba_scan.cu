@@ -10,6 +10,7 @@
 
 #include "../../include/mamba_scan.h"
 #include "bwd_reference.cuh"
+#include "bwd_staged.cuh"
 #include "common.cuh"
 #include "fwd_reference.cuh"
 #include "fwd_staged.cuh"
@@ -153,6 +154,13 @@ struct FwdReferenceLauncher {
     return launch_status();
   }
 };
+
+template <typename T>
+mamba_status_t staged_bwd_dispatch(const BwdArgs &a, const StagedOptions &o, cudaStream_t s) {
+  if (a.N <= 4) return staged_backward<T, 4>(a, o, s, &launch_status);
+  if (a.N <= 8) return staged_backward<T, 8>(a, o, s, &launch_status);
+  return staged_backward<T, 16>(a, o, s, &launch_status);
+}
 
 template <typename T>
 mamba_status_t staged_dispatch(const FwdArgs &a, const StagedOptions &o, cudaStream_t s) {
@@ -362,9 +370,21 @@ mamba_status_t mamba_scan_bwd_ex(const void *u, const void *delta, const float *
   a.du = du; a.ddelta = ddelta; a.dz = dz; a.dB = dB; a.dC = dC;
   a.dA = dA; a.dD = dD; a.dbias = ddelta_bias;
   a.batch = batch; a.dim = dim; a.L = L; a.N = (int)N;
-  const int path = options ? options->path : MAMBA_PATH_AUTO;
-  if (path == MAMBA_PATH_GENERIC || path == MAMBA_PATH_STRUCTURED) return MAMBA_ERR_UNSUPPORTED;
-  return dispatch<BwdReferenceLauncher>(dtype, (int)N, a, s);
+  StagedOptions so;
+  so.path = options ? options->path : MAMBA_PATH_AUTO;
+  so.chunk_len = options ? options->chunk_len : 0;
+  so.carry = options ? options->carry : 0;
+  so.timeout_us = options ? options->wait_timeout_us : 0;
+  so.test_hook = 0;
+  const bool stageable = staged_bwd_supported(a, es);
+  if (so.path == MAMBA_PATH_REFERENCE || (!stageable && so.path == MAMBA_PATH_AUTO))
+    return dispatch<BwdReferenceLauncher>(dtype, (int)N, a, s);
+  if (!stageable) return MAMBA_ERR_UNSUPPORTED;
+  st = dtype == MAMBA_BF16 ? staged_bwd_dispatch<__nv_bfloat16>(a, so, s)
+                           : staged_bwd_dispatch<float>(a, so, s);
+  if (st == MAMBA_ERR_UNSUPPORTED && so.path == MAMBA_PATH_AUTO)
+    return dispatch<BwdReferenceLauncher>(dtype, (int)N, a, s);
+  return st;
 }
 
 mamba_status_t mamba_scan_bwd(const void *u, const void *delta, const float *delta_bias,
