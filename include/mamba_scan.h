@@ -149,6 +149,40 @@ MAMBA_SCAN_API mamba_status_t mamba_scan_bwd_ex(const void *u, const void *delta
                                  int64_t N, mamba_dtype_t dtype,
                                  const mamba_scan_options_t *options, mamba_stream_t stream);
 
+/*
+ * Forward that allocates nothing.  (An addition of this library for callers
+ * that cannot allocate; the paper has no counterpart.)
+ *
+ * Same arguments, layouts and results as mamba_scan_fwd.  Meant for callers
+ * that cannot let a library allocate device memory -- programs that give all
+ * device memory to their own allocator up front, latency-critical loops that
+ * must not enter the CUDA allocator, code that runs where allocation calls
+ * are not allowed.  Instead of a workspace per call, the chunked kernel keeps
+ * its scratch (ticket counter, hand-off flags, carried chunk-end states) in a
+ * fixed 8 MiB array in the library's device memory; every GPU that loads the
+ * library holds that array until the process exits.  The call makes no
+ * cudaMalloc, cudaMallocAsync or cudaFree call.
+ *
+ *  - Limit: batch * ceil(dim / 128) channel groups must fit the array: at most
+ *    1016 groups when N > 8, 2032 when 4 < N <= 8, 4064 when N <= 4.  Larger
+ *    problems return MAMBA_ERR_UNSUPPORTED without enqueuing anything.  Shapes
+ *    that the staged kernels do not take (see mamba_scan_fwd) run the
+ *    one-thread-per-channel kernel, which needs no scratch.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) for that device; make that first call before any
+ *    stream capture.
+ *  - All calls on a device share the one array, and it keeps what the last
+ *    call left (each call clears the parts that must start at zero).  Calls
+ *    whose work overlaps on the GPU -- on different streams, or from
+ *    different threads -- race on it: order them.
+ */
+MAMBA_SCAN_API mamba_status_t mamba_scan_fwd_noalloc(const void *u, const void *delta,
+                                                     const float *delta_bias, const float *A,
+                                                     const void *B, const void *C, const float *D,
+                                                     const void *z, void *y, float *last_state,
+                                                     int64_t batch, int64_t dim, int64_t L, int64_t N,
+                                                     mamba_dtype_t dtype, mamba_stream_t stream);
+
 /* Synchronizes `stream`, then returns MAMBA_ERR_CUDA for a pending CUDA error,
  * else MAMBA_ERR_DEVICE_TIMEOUT if a kernel of this library recorded an
  * expired wait on the current device since the last call (the record is

@@ -7,6 +7,7 @@
 #include <atomic>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/mamba_scan.h"
 #include "bwd_reference.cuh"
@@ -398,3 +399,160 @@ mamba_status_t mamba_scan_bwd(const void *u, const void *delta, const float *del
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free forward (mamba_scan_fwd_noalloc).
+//
+// Some callers cannot let a library allocate device memory: programs that
+// hand all device memory to their own allocator at start-up (so an
+// allocation by the library fails, or breaks their budget), latency-critical
+// loops whose owners forbid any call into the CUDA allocator, and hosts that
+// call the scan from code that must not enter the allocator at all.  For
+// them the chunked forward keeps its scratch -- the unit ticket counter, the
+// per-group hand-off flags and the carried chunk-end states -- in the fixed
+// array below instead of taking a workspace per call.  The array is part of
+// the library's device code, so every GPU that loads the library holds it
+// (8 MiB) until the process exits.
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // per device
+constexpr size_t kNoAllocIntBytes = size_t(64) << 10;     // ticket counter + group flags
+constexpr int kNoAllocMaxDevices = 64;
+
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+std::mutex g_noalloc_mutex;
+unsigned char *g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on device `dev` (the current device).
+// In host code the array's name only stands for the symbol, so the address
+// is looked up with cudaGetSymbolAddress, once per device.
+mamba_status_t noalloc_scratch(int dev, unsigned char **out) {
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return MAMBA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) {
+      cudaGetLastError();
+      return MAMBA_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = static_cast<unsigned char *>(ptr);
+  }
+  *out = g_noalloc_ptr[dev];
+  return MAMBA_OK;
+}
+
+// The staged forward with the sequential hand-off, its scratch carved out of
+// the fixed array.  Enqueues a memset of the counter and flags and one kernel.
+template <typename T, int NM>
+mamba_status_t noalloc_forward(const FwdArgs &a, unsigned char *scratch, cudaStream_t s) {
+  using Lay = StagedLayout<T, NM>;
+  constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
+  const uint64_t L = a.L, dim = a.dim, batch = a.batch, N = a.N;
+  const int64_t gpb = ceil_div(a.dim, kSThreads);
+  const int64_t G = int64_t(a.batch) * gpb;
+  // the limit: counter + flags in the first 64 KiB, one carried state per group after it
+  if (size_t(G + 1) * 4 > kNoAllocIntBytes ||
+      size_t(G) * NM * kSThreads * 4 > kNoAllocScratchBytes - kNoAllocIntBytes)
+    return MAMBA_ERR_UNSUPPORTED;
+  CUtensorMap maps[6];
+  const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_64B, none = CU_TENSOR_MAP_SWIZZLE_NONE;
+  if (!make_map_3d(&maps[0], a.u, bf16, L, dim, batch, Lay::TT, kSThreads, sw) ||
+      !make_map_3d(&maps[1], a.delta, bf16, L, dim, batch, Lay::TT, kSThreads, sw) ||
+      !make_map_3d(&maps[2], a.z ? a.z : a.u, bf16, L, dim, batch, Lay::TT, kSThreads, sw) ||
+      !make_map_3d(&maps[3], a.y, bf16, L, dim, batch, Lay::TT, kSThreads, sw) ||
+      !make_map_3d(&maps[4], a.B, bf16, L, N, batch, Lay::TT, uint32_t(N), none) ||
+      !make_map_3d(&maps[5], a.C, bf16, L, N, batch, Lay::TT, uint32_t(N), none))
+    return MAMBA_ERR_UNSUPPORTED;
+  int bps = 0;
+  if (prepare_kernel<T, NM, KIND_SEQ>(&bps) != cudaSuccess) return MAMBA_ERR_CUDA;
+  const int slots = device_sm_count() * std::max(1, bps);
+  StagedOptions o;
+  o.path = MAMBA_PATH_AUTO;
+  o.chunk_len = 0;
+  o.carry = 1;
+  o.timeout_us = 0;
+  o.test_hook = 0;
+  const StagedPlan pl = plan_staged(G, a.L, slots, o);
+  if (G * pl.K > (int64_t(1) << 30)) return MAMBA_ERR_UNSUPPORTED;
+  StagedArgs sa;
+  sa.f = a;
+  sa.G = int(G);
+  sa.gpb = int(gpb);
+  sa.K = pl.K;
+  sa.chunk_len = pl.chunk_len;
+  sa.n_units = int(G * pl.K);
+  sa.counter = reinterpret_cast<int *>(scratch);
+  sa.flags = sa.counter + 1;
+  sa.carry = reinterpret_cast<float *>(scratch + kNoAllocIntBytes);
+  sa.agg_h = sa.hin = sa.ckpt = nullptr;
+  sa.agg_S = nullptr;
+  sa.timeout_ns = kDefaultTimeoutNs;
+  sa.test_hook = 0;
+  sa.force_generic = 0;
+  // The array keeps whatever the previous call left: the counter and the
+  // flags must start at zero (the carried states are written before read).
+  if (cudaMemsetAsync(scratch, 0, size_t(G + 1) * 4, s) != cudaSuccess) return cuda_status();
+  launch_staged<T, NM, KIND_SEQ>(maps, sa, int(std::min<int64_t>(G * pl.K, slots)), s);
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" mamba_status_t mamba_scan_fwd_noalloc(const void *u, const void *delta,
+                                                 const float *delta_bias, const float *A,
+                                                 const void *B, const void *C, const float *D,
+                                                 const void *z, void *y, float *last_state,
+                                                 int64_t batch, int64_t dim, int64_t L, int64_t N,
+                                                 mamba_dtype_t dtype, mamba_stream_t stream) {
+  mamba_status_t st = check_shape(batch, dim, L, N, dtype);
+  if (st != MAMBA_OK) return st;
+  Checker ck;
+  if (cudaGetDevice(&ck.dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MAMBA_ERR_CUDA;
+  }
+  const size_t es = dtype_size(dtype);
+  const size_t nbdl = size_t(batch) * size_t(dim) * size_t(L);
+  const size_t nbnl = size_t(batch) * size_t(N) * size_t(L);
+  ck.buf(u, nbdl * es, es, true, false);
+  ck.buf(delta, nbdl * es, es, true, false);
+  ck.buf(z, nbdl * es, es, false, false);
+  ck.buf(B, nbnl * es, es, true, false);
+  ck.buf(C, nbnl * es, es, true, false);
+  ck.buf(A, size_t(dim) * N * 4, 4, true, false);
+  ck.buf(D, size_t(dim) * 4, 4, false, false);
+  ck.buf(delta_bias, size_t(dim) * 4, 4, false, false);
+  ck.buf(y, nbdl * es, es, true, true);
+  ck.buf(last_state, size_t(batch) * dim * N * 4, 4, false, true);
+  if (ck.st != MAMBA_OK) return ck.st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (batch == 0 || dim == 0) return MAMBA_OK;
+  if (L == 0) {
+    if (last_state && cudaMemsetAsync(last_state, 0, size_t(batch) * dim * N * 4, s) != cudaSuccess)
+      return cuda_status();
+    return MAMBA_OK;
+  }
+  FwdArgs a;
+  a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
+  a.bias = delta_bias; a.A = A; a.D = D; a.y = y; a.last_state = last_state;
+  a.batch = batch; a.dim = dim; a.L = L; a.N = (int)N;
+  // Shapes the staged kernels do not take use the one-thread-per-channel
+  // kernel, which needs no scratch at all.
+  if (!staged_supported(a, es)) return dispatch<FwdReferenceLauncher>(dtype, (int)N, a, s);
+  unsigned char *scratch = nullptr;
+  if ((st = noalloc_scratch(ck.dev, &scratch)) != MAMBA_OK) return st;
+  if (dtype == MAMBA_BF16) {
+    if (N <= 4) return noalloc_forward<__nv_bfloat16, 4>(a, scratch, s);
+    if (N <= 8) return noalloc_forward<__nv_bfloat16, 8>(a, scratch, s);
+    return noalloc_forward<__nv_bfloat16, 16>(a, scratch, s);
+  }
+  if (N <= 4) return noalloc_forward<float, 4>(a, scratch, s);
+  if (N <= 8) return noalloc_forward<float, 8>(a, scratch, s);
+  return noalloc_forward<float, 16>(a, scratch, s);
+}

@@ -62,8 +62,9 @@ def load_library():
             lib.mamba_scan_fwd_ex.argtypes = [vp] * 10 + [i64] * 4 + [i32, opt, vp]
             lib.mamba_scan_bwd.argtypes = [vp] * 17 + [i64] * 4 + [i32, vp]
             lib.mamba_scan_bwd_ex.argtypes = [vp] * 17 + [i64] * 4 + [i32, opt, vp]
+            lib.mamba_scan_fwd_noalloc.argtypes = [vp] * 10 + [i64] * 4 + [i32, vp]
             for f in ("mamba_scan_fwd", "mamba_scan_fwd_ex", "mamba_scan_bwd",
-                      "mamba_scan_bwd_ex", "mamba_scan_stream_status"):
+                      "mamba_scan_bwd_ex", "mamba_scan_stream_status", "mamba_scan_fwd_noalloc"):
                 getattr(lib, f).restype = ctypes.c_int
             lib.mamba_scan_stream_status.argtypes = [vp]
             lib.mamba_scan_status_string.argtypes = [ctypes.c_int]
@@ -173,6 +174,27 @@ def mamba_scan_bwd(u, delta, delta_bias, A, B, C, D, z, dy, du, ddelta, dA, dB, 
         rc = lib.mamba_scan_bwd_ex(*args, ctypes.byref(_options(path, chunk_len)),
                                    _stream_handle(stream))
     _check(rc, "mamba_scan_bwd")
+
+
+def mamba_scan_fwd_noalloc(u, delta, delta_bias, A, B, C, D, z, y, last_state, *, stream=None):
+    """The forward without any device allocation by the library: for callers
+    that cannot let a library allocate (their own allocator owns device
+    memory, or allocation calls are not allowed where they run).  Scratch lives
+    in a fixed per-device array of the library; calls that overlap on the GPU
+    race on it.  Same tensors as ``mamba_scan_fwd``."""
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    dt = u.dtype
+    f32 = torch.float32
+    args = [
+        _ptr(u, dt, (batch, dim, L), "u"), _ptr(delta, dt, (batch, dim, L), "delta"),
+        _ptr(delta_bias, f32, (dim,), "delta_bias"), _ptr(A, f32, (dim, N), "A"),
+        _ptr(B, dt, (batch, N, L), "B"), _ptr(C, dt, (batch, N, L), "C"),
+        _ptr(D, f32, (dim,), "D"), _ptr(z, dt, (batch, dim, L), "z"),
+        _ptr(y, dt, (batch, dim, L), "y"), _ptr(last_state, f32, (batch, dim, N), "last_state"),
+        batch, dim, L, N, _dtype_code(dt)]
+    _check(load_library().mamba_scan_fwd_noalloc(*args, _stream_handle(stream)),
+           "mamba_scan_fwd_noalloc")
 
 
 def launch_count() -> int:
