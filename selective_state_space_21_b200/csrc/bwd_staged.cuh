@@ -13,9 +13,10 @@
 //  * This kernel then walks every (channel group, chunk) unit from the last
 //    chunk to the first.  One thread owns one channel and its N states.  Per
 //    16-step tile (TMA-staged u, delta, z, dy, B, C, read in reverse order) it
-//    re-runs the tile forward from its checkpoint, keeping the state every 4
-//    steps in shared memory, then for each 4-step segment from the last
-//    re-runs the segment into registers and walks it backwards.
+//    re-runs the tile forward from its checkpoint, keeping the state before
+//    every segment of 2 (bf16) or 4 (fp32) steps in shared memory, then for
+//    each segment from the last re-runs it into registers and walks it
+//    backwards.
 //  * The adjoint of h_t is G_t = C_t dy0_t + Abar_{t+1} G_{t+1} with
 //    dy0 = dy silu(z); the thread carries Ga = Abar_t G_t, which is also the
 //    factor of dDelta.  With the structured A of the forward (decays E(n+1)
@@ -41,8 +42,6 @@
 namespace mscan {
 
 constexpr int kBTT = kCkptEvery;  // time steps per backward tile
-constexpr int kBSeg = 4;          // time steps per recompute segment
-constexpr int kBNSeg = kBTT / kBSeg;
 constexpr int kBStages = 2;
 
 template <typename T, int NM>
@@ -51,12 +50,18 @@ struct BwdLayout {
   static constexpr int TILE = kSThreads * RB;
   static constexpr int RAW = kMaxN * RB;
   static constexpr int STAGE = 4 * TILE + 2 * RAW;  // u, delta, z, dy, B, C
+  // Steps per recompute segment: the states of one segment live in
+  // registers, the state before every segment in shared memory.  Two-step
+  // segments keep the register footprint down; fp32 tiles are twice as large,
+  // which leaves room for four-step segments only.
+  static constexpr int SEG = sizeof(T) == 2 ? 2 : 4;
+  static constexpr int NSEG = kBTT / SEG;
   static constexpr int BSTR = NM + 4;
   static constexpr int OFF_SUB = kBStages * STAGE;
-  static constexpr int OFF_BS = OFF_SUB + kBNSeg * NM * kSThreads * 4;
+  static constexpr int OFF_BS = OFF_SUB + NSEG * NM * kSThreads * 4;
   static constexpr int OFF_CS = OFF_BS + kBTT * BSTR * 4;
   static constexpr int OFF_RED = OFF_CS + kBTT * BSTR * 4;
-  static constexpr int OFF_BAR = OFF_RED + (kSThreads / 32) * 32 * kBTT * 4;
+  static constexpr int OFF_BAR = OFF_RED + (kSThreads / 32) * kBTT * 33 * 4;
   static constexpr int OFF_Q = OFF_BAR + 8 * kBStages;
   static constexpr int BYTES = OFF_Q + 16 * 4;
   static constexpr int ALLOC = BYTES + 512;
@@ -84,26 +89,20 @@ __device__ __forceinline__ int swz_rows(int r, int c) {
   return r * RB + ((c ^ ((r * RB >> 7) & (RB / 16 - 1))) << 4);
 }
 
-// kBSeg consecutive values of a row starting at segment `seg` (4 steps).
-template <typename T> struct SegIO;
-template <> struct SegIO<__nv_bfloat16> {
-  __device__ static void load(const unsigned char *tile, int r, int seg, float (&o)[4]) {
-    const uint2 v = *reinterpret_cast<const uint2 *>(tile + swz_rows<32>(r, seg >> 1) + (seg & 1) * 8);
-    o[0] = __uint_as_float(v.x << 16);
-    o[1] = __uint_as_float(v.x & 0xffff0000u);
-    o[2] = __uint_as_float(v.y << 16);
-    o[3] = __uint_as_float(v.y & 0xffff0000u);
+// The SEG consecutive values of row r that make segment `seg` of a tile.
+template <typename T, int SEG> struct SegIO;
+template <> struct SegIO<__nv_bfloat16, 2> {  // 32-byte rows: 2 chunks of 8 steps
+  __device__ static void load(const unsigned char *tile, int r, int seg, float (&o)[2]) {
+    const uint32_t v = *reinterpret_cast<const uint32_t *>(tile + swz_rows<32>(r, seg >> 2) + (seg & 3) * 4);
+    o[0] = __uint_as_float(v << 16);
+    o[1] = __uint_as_float(v & 0xffff0000u);
   }
-  __device__ static void store(__nv_bfloat16 *dst, const float (&o)[4]) {
+  __device__ static void store(__nv_bfloat16 *dst, const float (&o)[2]) {
     __nv_bfloat162 a = __floats2bfloat162_rn(o[0], o[1]);
-    __nv_bfloat162 b = __floats2bfloat162_rn(o[2], o[3]);
-    uint2 v;
-    v.x = *reinterpret_cast<uint32_t *>(&a);
-    v.y = *reinterpret_cast<uint32_t *>(&b);
-    *reinterpret_cast<uint2 *>(dst) = v;
+    *reinterpret_cast<uint32_t *>(dst) = *reinterpret_cast<uint32_t *>(&a);
   }
 };
-template <> struct SegIO<float> {
+template <> struct SegIO<float, 4> {  // 64-byte rows: 4 chunks of 4 steps
   __device__ static void load(const unsigned char *tile, int r, int seg, float (&o)[4]) {
     const float4 v = *reinterpret_cast<const float4 *>(tile + swz_rows<64>(r, seg));
     o[0] = v.x;
@@ -125,6 +124,32 @@ __device__ __forceinline__ float dpsi_fast(float x, float ex) {
   return fabsf(x) < 0.25f ? p : q;
 }
 
+// First butterfly stage for one state: lanes with bit 4 set keep the dC value
+// and receive their partner's dC; the others keep dB.  Folding this stage
+// into the per-state loop halves the values live at once.
+__device__ __forceinline__ float bfly_first(float db, float dc, bool up) {
+  const float send = up ? db : dc;
+  const float keep = up ? dc : db;
+  return keep + __shfl_xor_sync(0xffffffffu, send, 16);
+}
+
+// Remaining stages (lane bits 3..0) of the reduce-scatter over 16 values:
+// lane l returns the warp sum of value l (dB of state l for l < 16, dC of
+// state l - 16 otherwise).
+__device__ __forceinline__ float bfly_rest(float (&v)[16], int lane) {
+#pragma unroll
+  for (int o = 8; o >= 1; o >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < o; ++i) {
+      const float send = up ? v[i] : v[i + o];
+      const float keep = up ? v[i + o] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  return v[0];
+}
+
 template <typename T, int NM>
 __global__ void __launch_bounds__(kSThreads, 2)
     bwd_staged_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_d,
@@ -134,15 +159,17 @@ __global__ void __launch_bounds__(kSThreads, 2)
   using Lay = BwdLayout<T, NM>;
   constexpr int RB = Lay::RB, BSTR = Lay::BSTR;
   constexpr int NP = NM / 2;
+  constexpr int SEG = Lay::SEG;
+  using IO = SegIO<T, SEG>;
 
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *sm = smem_raw + ((512u - (smem_u32(smem_raw) & 511u)) & 511u);
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + Lay::OFF_BAR);
   int *q = reinterpret_cast<int *>(sm + Lay::OFF_Q);
-  float *sub = reinterpret_cast<float *>(sm + Lay::OFF_SUB);  // [kBNSeg][NM][128]
+  float *sub = reinterpret_cast<float *>(sm + Lay::OFF_SUB);  // [NSEG][NM][128]
   float *Bs = reinterpret_cast<float *>(sm + Lay::OFF_BS);
   float *Cs = reinterpret_cast<float *>(sm + Lay::OFF_CS);
-  float *red = reinterpret_cast<float *>(sm + Lay::OFF_RED);  // [4 warps][32][kBTT]
+  float *red = reinterpret_cast<float *>(sm + Lay::OFF_RED);  // [4 warps][kBTT][33] (padded rows)
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const BwdArgs &f = p.w;
@@ -314,7 +341,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
         const int tile = ntiles - 1 - it;  // tiles run from the end of the chunk
         const int64_t t0 = tbeg + int64_t(tile) * kBTT;
         const int steps = int(std::min<int64_t>(kBTT, tend - t0));
-        const int nseg = steps / kBSeg;
+        const int nseg = steps / SEG;
         const int stage = ctile % kBStages;
         const uint32_t parity = uint32_t(ctile / kBStages) & 1u;
         unsigned char *st = sm + stage * Lay::STAGE;
@@ -376,12 +403,12 @@ __global__ void __launch_bounds__(kSThreads, 2)
               for (int n = 0; n < NM; ++n) sp[n * kSThreads] = h[n];
             }
             if (seg == nseg - 1) break;  // the last segment is re-run below anyway
-            float uv[4], dv[4];
-            SegIO<T>::load(su, tid, seg, uv);
-            SegIO<T>::load(sd, tid, seg, dv);
+            float uv[SEG], dv[SEG];
+            IO::load(su, tid, seg, uv);
+            IO::load(sd, tid, seg, dv);
 #pragma unroll
-            for (int i = 0; i < kBSeg; ++i) {
-              const float *Brow = Bs + (seg * kBSeg + i) * BSTR;
+            for (int i = 0; i < SEG; ++i) {
+              const float *Brow = Bs + (seg * SEG + i) * BSTR;
               if constexpr (kS) {
                 f2 P[NP];
                 float Delta, sv;
@@ -397,22 +424,24 @@ __global__ void __launch_bounds__(kSThreads, 2)
 
         // segments from the last: re-run into registers, then walk backwards
         for (int seg = nseg - 1; seg >= 0; --seg) {
-          float uv[4], dv[4], zv[4], dyv[4];
-          SegIO<T>::load(su, tid, seg, uv);
-          SegIO<T>::load(sd, tid, seg, dv);
-          SegIO<T>::load(sdy, tid, seg, dyv);
-          if (has_z) SegIO<T>::load(sz, tid, seg, zv);
-          float du_o[4], dd_o[4], dz_o[4];
+          float uv[SEG], dv[SEG], zv[SEG], dyv[SEG];
+          IO::load(su, tid, seg, uv);
+          IO::load(sd, tid, seg, dv);
+          IO::load(sdy, tid, seg, dyv);
+          if (has_z) IO::load(sz, tid, seg, zv);
+          float du_o[SEG], dd_o[SEG], dz_o[SEG];
           const float *sp = sub + (seg * NM) * kSThreads + tid;
 
           if constexpr (kS) {
-            f2 Hs[kBSeg + 1][NP];
+            // states before each step of the segment (the state after a step
+            // is recomputed in the reverse step from h_{t-1} and t1)
+            f2 Hs[SEG][NP];
 #pragma unroll
             for (int i = 0; i < NP; ++i)
               Hs[0][i] = pk(sp[(2 * i) * kSThreads], sp[(2 * i + 1) * kSThreads]);
 #pragma unroll
-            for (int i = 0; i < kBSeg; ++i) {
-              const float *Brow = Bs + (seg * kBSeg + i) * BSTR;
+            for (int i = 0; i + 1 < SEG; ++i) {
+              const float *Brow = Bs + (seg * SEG + i) * BSTR;
               f2 P[NP];
               float Delta, sv;
               step_decay(dv[i] + bias, P, Delta, sv);
@@ -421,8 +450,8 @@ __global__ void __launch_bounds__(kSThreads, 2)
               struct_update<NM>(Hs[i + 1], P, uv[i] * invA0, 0.f, Brow, Brow);
             }
 #pragma unroll
-            for (int i = kBSeg - 1; i >= 0; --i) {
-              const int tl = seg * kBSeg + i;
+            for (int i = SEG - 1; i >= 0; --i) {
+              const int tl = seg * SEG + i;
               const float *Brow = Bs + tl * BSTR;
               const float *Crow = Cs + tl * BSTR;
               f2 P[NP];
@@ -437,7 +466,8 @@ __global__ void __launch_bounds__(kSThreads, 2)
               const float x1 = Delta * A0;
               const f2 U = pk(up, up), DY = pk(dy0, dy0), X1n = pk(-x1, -x1), Z = pk(0.f, 0.f);
               f2 DU = Z, DD = Z, Y0 = Z;
-              float vals[32];
+              const bool up16 = (lane & 16) != 0;
+              float v16[16];
 #pragma unroll
               for (int j = 0; j < NP; j += 2) {
                 const ulonglong2 bq = *reinterpret_cast<const ulonglong2 *>(Brow + 2 * j);
@@ -452,27 +482,23 @@ __global__ void __launch_bounds__(kSThreads, 2)
                   const f2 Ga = fma2(Gv, P[jj], Gv);
                   const f2 w = fma2(Gv, P[jj], Z);
                   const f2 t1 = fma2(Bp, U, Hs[i][jj]);
+                  const f2 hcur = fma2(P[jj], t1, Hs[i][jj]);  // h_t
                   const f2 cq = fma2(fma2(Ga, t1, Z), CN, Z);
                   DD = fma2(cq, pk(1.f, 1.f), DD);
                   Acc[jj] = fma2(X1n, cq, Acc[jj]);
                   const f2 dBc = fma2(w, U, Z);
                   Acc[jj] = fma2(dBc, Bp, Acc[jj]);
                   DU = fma2(w, Bp, DU);
-                  Y0 = fma2(Cp, Hs[i + 1][jj], Y0);
-                  const f2 dCc = fma2(DY, Hs[i + 1][jj], Z);
+                  Y0 = fma2(Cp, hcur, Y0);
+                  const f2 dCc = fma2(DY, hcur, Z);
                   Gt[jj] = Ga;
-                  vals[2 * jj] = lo_of(dBc);
-                  vals[2 * jj + 1] = hi_of(dBc);
-                  vals[kMaxN + 2 * jj] = lo_of(dCc);
-                  vals[kMaxN + 2 * jj + 1] = hi_of(dCc);
+                  const float vm = valid ? 1.f : 0.f;
+                  v16[2 * jj] = bfly_first(vm * lo_of(dBc), vm * lo_of(dCc), up16);
+                  v16[2 * jj + 1] = bfly_first(vm * hi_of(dBc), vm * hi_of(dCc), up16);
                 }
               }
 #pragma unroll
-              for (int n = NM; n < kMaxN; ++n) vals[n] = vals[kMaxN + n] = 0.f;
-              if (!valid) {
-#pragma unroll
-                for (int n = 0; n < 32; ++n) vals[n] = 0.f;
-              }
+              for (int n = NM; n < kMaxN; ++n) v16[n] = 0.f;
               const float du = fmaf(lo_of(DU) + hi_of(DU), invA0, Dd * dy0);
               const float dd = A0 * (lo_of(DD) + hi_of(DD)) * sv;
               const float y0 = (lo_of(Y0) + hi_of(Y0)) + Dd * uv[i];
@@ -481,25 +507,25 @@ __global__ void __launch_bounds__(kSThreads, 2)
               dz_o[i] = has_z ? dyv[i] * y0 * sz * (1.f + zv[i] * (1.f - sz)) : 0.f;
               dDsum = fmaf(dy0, uv[i], dDsum);
               dbsum += dd;
-              const float rsum = warp_reduce_scatter32(vals, lane);
+              const float rsum = bfly_rest(v16, lane);
               // lane l holds dB (l < 16, to be divided by l+1) or dC of state l-16
-              red[(warp * 32 + lane) * kBTT + tl] = (lane < kMaxN) ? rsum * (1.f / float(lane + 1)) : rsum;
+              red[(warp * kBTT + tl) * 33 + lane] = (lane < kMaxN) ? rsum * (1.f / float(lane + 1)) : rsum;
             }
           } else {
-            float Hs[kBSeg + 1][NM];
+            float Hs[SEG][NM];
 #pragma unroll
             for (int n = 0; n < NM; ++n) Hs[0][n] = sp[n * kSThreads];
 #pragma unroll
-            for (int i = 0; i < kBSeg; ++i) {
-              const float *Brow = Bs + (seg * kBSeg + i) * BSTR;
+            for (int i = 0; i + 1 < SEG; ++i) {
+              const float *Brow = Bs + (seg * SEG + i) * BSTR;
               const float Delta = softplus_fast(dv[i] + bias);
 #pragma unroll
               for (int n = 0; n < NM; ++n) Hs[i + 1][n] = Hs[i][n];
               generic_update<NM>(Hs[i + 1], Delta, uv[i], 0.f, Arow, A2, invA, Brow, Brow);
             }
 #pragma unroll
-            for (int i = kBSeg - 1; i >= 0; --i) {
-              const int tl = seg * kBSeg + i;
+            for (int i = SEG - 1; i >= 0; --i) {
+              const int tl = seg * SEG + i;
               const float *Brow = Bs + tl * BSTR;
               const float *Crow = Cs + tl * BSTR;
               const float v = dv[i] + bias;
@@ -511,7 +537,9 @@ __global__ void __launch_bounds__(kSThreads, 2)
                 dy0 *= zv[i] * sz;
               }
               float du_acc = 0.f, dD_acc = 0.f, y0 = Dd * uv[i];
-              float vals[32];
+              const bool up16 = (lane & 16) != 0;
+              const float vm = valid ? 1.f : 0.f;
+              float v16[16];
 #pragma unroll
               for (int n = 0; n < NM; ++n) {
                 const float x = Delta * Arow[n];
@@ -523,7 +551,8 @@ __global__ void __launch_bounds__(kSThreads, 2)
                 pp = fmaf(x, pp, 1.f);
                 const float Eb = fabsf(x) < 0.25f ? Delta * pp : (a - 1.f) * invA[n];  // Bbar / B
                 const float Bn = Brow[n], Cn = Crow[n];
-                const float hprev = Hs[i][n], hcur = Hs[i + 1][n];
+                const float hprev = Hs[i][n];
+                const float hcur = fmaf(a, hprev, Eb * (Bn * uv[i]));  // h_t, as in the forward
                 const float Gv = fmaf(Cn, dy0, gs[n]);
                 const float Ga = a * Gv;
                 const float wv = Gv * Eb;
@@ -531,30 +560,25 @@ __global__ void __launch_bounds__(kSThreads, 2)
                 dD_acc = fmaf(Ga, fmaf(Bn, uv[i], Arow[n] * hprev), dD_acc);
                 accs[n] = fmaf(Gv, Delta * a * hprev + Bn * uv[i] * Delta * Delta * dpsi_fast(x, a), accs[n]);
                 y0 = fmaf(Cn, hcur, y0);
-                vals[n] = wv * uv[i];
-                vals[kMaxN + n] = dy0 * hcur;
+                v16[n] = bfly_first(vm * wv * uv[i], vm * dy0 * hcur, up16);
                 gs[n] = Ga;
               }
 #pragma unroll
-              for (int n = NM; n < kMaxN; ++n) vals[n] = vals[kMaxN + n] = 0.f;
-              if (!valid) {
-#pragma unroll
-                for (int n = 0; n < 32; ++n) vals[n] = 0.f;
-              }
+              for (int n = NM; n < kMaxN; ++n) v16[n] = 0.f;
               const float dd = dD_acc * sv;
               du_o[i] = fmaf(Dd, dy0, du_acc);
               dd_o[i] = dd;
               dz_o[i] = has_z ? dyv[i] * y0 * sz * (1.f + zv[i] * (1.f - sz)) : 0.f;
               dDsum = fmaf(dy0, uv[i], dDsum);
               dbsum += dd;
-              red[(warp * 32 + lane) * kBTT + tl] = warp_reduce_scatter32(vals, lane);
+              red[(warp * kBTT + tl) * 33 + lane] = bfly_rest(v16, lane);
             }
           }
           if (valid) {
-            const int64_t o = row + t0 + seg * kBSeg;
-            SegIO<T>::store(static_cast<T *>(f.du) + o, du_o);
-            SegIO<T>::store(static_cast<T *>(f.ddelta) + o, dd_o);
-            if (has_z) SegIO<T>::store(static_cast<T *>(f.dz) + o, dz_o);
+            const int64_t o = row + t0 + seg * SEG;
+            IO::store(static_cast<T *>(f.du) + o, du_o);
+            IO::store(static_cast<T *>(f.ddelta) + o, dd_o);
+            if (has_z) IO::store(static_cast<T *>(f.dz) + o, dz_o);
           }
         }
         __syncthreads();
@@ -564,7 +588,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
           if (tl < steps) {
             float sum = 0.f;
 #pragma unroll
-            for (int wv = 0; wv < kSThreads / 32; ++wv) sum += red[(wv * 32 + slot) * kBTT + tl];
+            for (int wv = 0; wv < kSThreads / 32; ++wv) sum += red[(wv * kBTT + tl) * 33 + slot];
             p.part_bc[((int64_t(g % p.gpb) * f.batch + b) * 32 + slot) * f.L + t0 + tl] = sum;
           }
         }
@@ -577,8 +601,8 @@ __global__ void __launch_bounds__(kSThreads, 2)
           gt[2 * i] = lo_of(Gt[i]);
           gt[2 * i + 1] = hi_of(Gt[i]);
           // Acc holds -A_n dA_n
-          dA[2 * i] = -lo_of(Acc[i]) / Arow[2 * i];
-          dA[2 * i + 1] = -hi_of(Acc[i]) / Arow[2 * i + 1];
+          dA[2 * i] = -lo_of(Acc[i]) / (float(2 * i + 1) * A0);
+          dA[2 * i + 1] = -hi_of(Acc[i]) / (float(2 * i + 2) * A0);
         }
       } else {
 #pragma unroll
@@ -674,7 +698,7 @@ __global__ void bwd_staged_finalize_params(const BwdStagedArgs p) {
 inline bool staged_bwd_supported(const BwdArgs &a, size_t es) {
   auto al = [](const void *ptr) { return ptr == nullptr || (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; };
   if (a.N < 3) return false;
-  if ((a.L * int64_t(es)) % 16 != 0 || a.L % kBSeg != 0) return false;
+  if ((a.L * int64_t(es)) % 16 != 0 || a.L % 4 != 0) return false;
   if (a.L > (int64_t(1) << 31) - 1024 || a.dim > (int64_t(1) << 31) - 1) return false;
   return al(a.u) && al(a.delta) && al(a.z) && al(a.dy) && al(a.B) && al(a.C) && al(a.du) &&
          al(a.ddelta) && al(a.dz);
