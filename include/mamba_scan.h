@@ -38,7 +38,9 @@
  *    recorded in a per-device sticky error word read by
  *    mamba_scan_stream_status().
  *  - Temporary device memory (chunk-boundary states, partial sums) is taken
- *    with cudaMallocAsync/cudaFreeAsync on `stream`; failure returns
+ *    stream-ordered on `stream` from a memory pool the library creates once
+ *    per device; the pool keeps up to 4 GiB reserved between calls (until the
+ *    process exits) so that repeated calls do not re-map it.  Failure returns
  *    MAMBA_ERR_OUT_OF_MEMORY.
  *  - Outputs are overwritten, never accumulated into.  No exception, abort,
  *    printf or trap crosses or happens behind this interface.  Calls are

@@ -492,9 +492,10 @@ __global__ void __launch_bounds__(kSThreads, 2)
                   Y0 = fma2(Cp, hcur, Y0);
                   const f2 dCc = fma2(DY, hcur, Z);
                   Gt[jj] = Ga;
-                  const float vm = valid ? 1.f : 0.f;
-                  v16[2 * jj] = bfly_first(vm * lo_of(dBc), vm * lo_of(dCc), up16);
-                  v16[2 * jj + 1] = bfly_first(vm * hi_of(dBc), vm * hi_of(dCc), up16);
+                  // Channels past `dim` contribute exact zeros: TMA fills their
+                  // rows with 0, so dy0 = 0 and their adjoint stays 0.
+                  v16[2 * jj] = bfly_first(lo_of(dBc), lo_of(dCc), up16);
+                  v16[2 * jj + 1] = bfly_first(hi_of(dBc), hi_of(dCc), up16);
                 }
               }
 #pragma unroll
@@ -538,7 +539,6 @@ __global__ void __launch_bounds__(kSThreads, 2)
               }
               float du_acc = 0.f, dD_acc = 0.f, y0 = Dd * uv[i];
               const bool up16 = (lane & 16) != 0;
-              const float vm = valid ? 1.f : 0.f;
               float v16[16];
 #pragma unroll
               for (int n = 0; n < NM; ++n) {
@@ -560,7 +560,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
                 dD_acc = fmaf(Ga, fmaf(Bn, uv[i], Arow[n] * hprev), dD_acc);
                 accs[n] = fmaf(Gv, Delta * a * hprev + Bn * uv[i] * Delta * Delta * dpsi_fast(x, a), accs[n]);
                 y0 = fmaf(Cn, hcur, y0);
-                v16[n] = bfly_first(vm * wv * uv[i], vm * dy0 * hcur, up16);
+                v16[n] = bfly_first(wv * uv[i], dy0 * hcur, up16);  // zero past `dim`
                 gs[n] = Ga;
               }
 #pragma unroll
@@ -747,7 +747,7 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
   const size_t n_A = gk * NM * kSThreads, n_D = gk * kSThreads;
   const size_t bytes = int_bytes + 4 * (n_ckpt + n_carry + n_bc + n_A + 2 * n_D);
   unsigned char *ws = nullptr;
-  if (cudaMallocAsync(reinterpret_cast<void **>(&ws), bytes, s) != cudaSuccess) {
+  if (ws_alloc(reinterpret_cast<void **>(&ws), bytes, s) != cudaSuccess) {
     cudaGetLastError();
     return MAMBA_ERR_OUT_OF_MEMORY;
   }
@@ -798,7 +798,7 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
     bwd_staged_finalize_params<NM><<<unsigned(std::min<int64_t>(ceil_div(np, 256), sms * 8)), 256, 0, s>>>(bp);
     st = launched();
   }
-  if (cudaFreeAsync(ws, s) != cudaSuccess && st == MAMBA_OK) st = MAMBA_ERR_CUDA;
+  if (ws_free(ws, s) != cudaSuccess && st == MAMBA_OK) st = MAMBA_ERR_CUDA;
   return st;
 }
 

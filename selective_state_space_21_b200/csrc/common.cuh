@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 namespace mscan {
 
 constexpr int kMaxN = 16;
@@ -59,5 +61,49 @@ __device__ __forceinline__ float dpsi_acc(float x) {
   }
   return (x * expf(x) - expm1f(x)) / (x * x);
 }
+
+// ----------------------------------------------------------- host: workspace
+
+// Workspace comes stream-ordered from one library-owned memory pool per device
+// that keeps up to kPoolKeepBytes reserved between calls, so that repeated
+// calls do not map and unmap hundreds of megabytes each time (the default
+// pool gives memory back to the system at every synchronization).
+constexpr uint64_t kPoolKeepBytes = uint64_t(4) << 30;
+
+inline cudaMemPool_t library_pool() {
+  static std::mutex mu;
+  static cudaMemPool_t pools[64] = {};
+  static bool tried[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!tried[dev]) {
+    tried[dev] = true;
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    if (cudaMemPoolCreate(&pool, &props) == cudaSuccess) {
+      uint64_t keep = kPoolKeepBytes;
+      cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+      pools[dev] = pool;
+    } else {
+      cudaGetLastError();
+    }
+  }
+  return pools[dev];
+}
+
+inline cudaError_t ws_alloc(void **ptr, size_t bytes, cudaStream_t s) {
+  cudaMemPool_t pool = library_pool();
+  if (pool) return cudaMallocFromPoolAsync(ptr, bytes, pool, s);
+  return cudaMallocAsync(ptr, bytes, s);
+}
+
+inline cudaError_t ws_free(void *ptr, cudaStream_t s) { return cudaFreeAsync(ptr, s); }
 
 }  // namespace mscan

@@ -783,7 +783,7 @@ mamba_status_t staged_forward(const FwdArgs &a, const StagedOptions &o, cudaStre
     bytes += gk * kSThreads * 8 + 2 * gk * NM * kSThreads * 4;
   }
   unsigned char *ws = nullptr;
-  if (cudaMallocAsync(reinterpret_cast<void **>(&ws), bytes, s) != cudaSuccess) {
+  if (ws_alloc(reinterpret_cast<void **>(&ws), bytes, s) != cudaSuccess) {
     cudaGetLastError();
     return MAMBA_ERR_OUT_OF_MEMORY;
   }
@@ -836,7 +836,7 @@ mamba_status_t staged_forward(const FwdArgs &a, const StagedOptions &o, cudaStre
       st = launched();
     }
   }
-  if (cudaFreeAsync(ws, s) != cudaSuccess && st == MAMBA_OK) st = MAMBA_ERR_CUDA;
+  if (ws_free(ws, s) != cudaSuccess && st == MAMBA_OK) st = MAMBA_ERR_CUDA;
   return st;
 }
 

@@ -182,7 +182,7 @@ struct BwdReferenceLauncher {
     const size_t n_A = bd * size_t(a.N);
     const size_t total = n_ckpt + n_bc + n_A + 2 * bd;
     float *ws = nullptr;
-    if (cudaMallocAsync(reinterpret_cast<void **>(&ws), total * sizeof(float), s) != cudaSuccess) {
+    if (ws_alloc(reinterpret_cast<void **>(&ws), total * sizeof(float), s) != cudaSuccess) {
       cudaGetLastError();
       return MAMBA_ERR_OUT_OF_MEMORY;
     }
@@ -214,7 +214,7 @@ struct BwdReferenceLauncher {
       bwd_finalize_params_kernel<<<(unsigned)g, 256, 0, s>>>(a, w);
       st = launch_status();
     }
-    if (cudaFreeAsync(ws, s) != cudaSuccess && st == MAMBA_OK) st = MAMBA_ERR_CUDA;
+    if (ws_free(ws, s) != cudaSuccess && st == MAMBA_OK) st = MAMBA_ERR_CUDA;
     return st;
   }
 };
