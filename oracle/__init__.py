@@ -48,7 +48,7 @@ def load_library(path: str):
     lib = ctypes.CDLL(path)
     dp = ctypes.c_void_p
     i64 = ctypes.c_longlong
-    lib.s6_oracle_fwd.argtypes = [dp] * 10 + [i64] * 5
+    lib.s6_oracle_fwd.argtypes = [dp] * 11 + [i64] * 5
     lib.s6_oracle_fwd.restype = ctypes.c_int
     lib.s6_oracle_bwd.argtypes = [dp] * 17 + [i64] * 5
     lib.s6_oracle_bwd.restype = ctypes.c_int
@@ -80,12 +80,15 @@ def default_threads() -> int:
     return max(1, os.cpu_count() or 1)
 
 
-def s6_forward(u, delta, A, B, C, delta_bias=None, D=None, z=None, nthreads=None, lib=None):
+def s6_forward(u, delta, A, B, C, delta_bias=None, D=None, z=None, nthreads=None, lib=None,
+               initial_state=None):
     """fp64 forward.  Shapes: u, delta, z (batch, dim, L); B, C (batch, N, L);
-    A (dim, N); delta_bias, D (dim,).  Returns (y, last_state) as float64
+    A (dim, N); delta_bias, D (dim,); initial_state (batch, dim, N), the state
+    before the first step (None = 0).  Returns (y, last_state) as float64
     arrays of shapes (batch, dim, L) and (batch, dim, N)."""
     u, delta, A, B, C = (_f64(t) for t in (u, delta, A, B, C))
     delta_bias, D, z = _f64(delta_bias), _f64(D), _f64(z)
+    h0 = _f64(initial_state)
     batch, dim, L = u.shape
     N = A.shape[1]
     assert delta.shape == u.shape and B.shape == (batch, N, L) and C.shape == (batch, N, L)
@@ -94,7 +97,7 @@ def s6_forward(u, delta, A, B, C, delta_bias=None, D=None, z=None, nthreads=None
     last = np.empty((batch, dim, N), np.float64)
     rc = (lib or _load()).s6_oracle_fwd(
         _ptr(u), _ptr(delta), _ptr(delta_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
-        _ptr(y), _ptr(last), batch, dim, L, N, nthreads or default_threads())
+        _ptr(h0), _ptr(y), _ptr(last), batch, dim, L, N, nthreads or default_threads())
     if rc != 0:
         raise RuntimeError(f"s6_oracle_fwd failed ({rc})")
     return y, last

@@ -28,8 +28,10 @@
  *             h[n] = Abar * h[n] + Bbar * u[b,d,t]                   [KN1 step 4]
  *     y0_t = sum_n C[b,n,t] * h[n]  (+ D[d] * u[b,d,t] if D given)   [KN1 step 4]
  *     y_t  = y0_t * silu(z[b,d,t])  (if z given)                     [PG33 block]
- * with h = 0 before the first step [TP-II6 s.4] and last_state = h after the
- * last step.
+ * with h = 0 before the first step [TP-II6 s.4] (or a given initial state, to
+ * continue a sequence one call or one token at a time: the recurrent mode of
+ * [TP-II6] section 4, "best for autoregressive inference") and last_state = h
+ * after the last step.
  *
  * Readings where the pages are silent or ambiguous (each one is listed in the
  * design notes of the repository):
@@ -87,6 +89,7 @@ static double phi(double x) {
 
 typedef struct {
   const double *u, *delta, *bias, *A, *B, *C, *D, *z, *dy;
+  const double *h0; /* optional initial state (batch, dim, N); NULL = 0 */
   double *y, *last_state;
   double *du, *ddelta, *dz;
   double *dA_part, *dD_part, *dbias_part; /* per (b,d) partials */
@@ -108,7 +111,7 @@ static void fwd_channel(const job_t *j, i64 b, i64 d, double *h) {
   const double bias = j->bias ? j->bias[d] : 0.0;
   const double Dd = j->D ? j->D[d] : 0.0;
   double *y = j->y + (b * dim + d) * L;
-  for (i64 n = 0; n < N; ++n) h[n] = 0.0;
+  for (i64 n = 0; n < N; ++n) h[n] = j->h0 ? j->h0[(b * dim + d) * N + n] : 0.0;
   for (i64 t = 0; t < L; ++t) {
     const double Delta = softplus(dl[t] + bias);
     double y0 = 0.0;
@@ -262,16 +265,20 @@ static int run_workers(job_t *base, i64 nthreads, void *(*fn)(void *), int per_t
 }
 
 /* Forward.  Layouts: u, delta, z, y: (batch, dim, L); B, C: (batch, N, L);
- * A: (dim, N); bias, D: (dim); last_state: (batch, dim, N).  bias, D, z and
- * last_state may be NULL.  Returns 0 on success. */
+ * A: (dim, N); bias, D: (dim); initial_state, last_state: (batch, dim, N).
+ * bias, D, z, initial_state (the state before the first step; NULL = 0) and
+ * last_state may be NULL.  Returns 0 on success.  Continuing a sequence from
+ * the state another call left is the recurrent (one token at a time) mode of
+ * the selective SSM. */
 int s6_oracle_fwd(const double *u, const double *delta, const double *bias, const double *A,
                   const double *B, const double *C, const double *D, const double *z,
-                  double *y, double *last_state, i64 batch, i64 dim, i64 L, i64 N,
-                  i64 nthreads) {
+                  const double *initial_state, double *y, double *last_state, i64 batch,
+                  i64 dim, i64 L, i64 N, i64 nthreads) {
   if (batch < 0 || dim < 0 || L < 0 || N < 1 || N > 64) return -2;
   job_t j;
   memset(&j, 0, sizeof(j));
   j.u = u; j.delta = delta; j.bias = bias; j.A = A; j.B = B; j.C = C; j.D = D; j.z = z;
+  j.h0 = initial_state;
   j.y = y; j.last_state = last_state;
   j.batch = batch; j.dim = dim; j.L = L; j.N = N;
   if (batch * dim == 0) return 0;

@@ -373,10 +373,37 @@ def pin_threads_agree(lib=None):
     return err, 1e-15
 
 
+def pin_resume_from_state(lib=None):
+    """Splitting a sequence and continuing from the first part's final state
+    gives the unsplit result (the recurrence carries everything in h)."""
+    x = make_inputs(2, 3, 50, 4, seed=61)
+    sl = lambda t, a, b: None if t is None else t[..., a:b].contiguous()
+    full, last = oracle.s6_forward(x["u"], x["delta"], x["A"], x["B"], x["C"], x["delta_bias"],
+                                   x["D"], x["z"], lib=lib)
+    args = lambda a, b: (sl(x["u"], a, b), sl(x["delta"], a, b), x["A"], sl(x["B"], a, b),
+                         sl(x["C"], a, b), x["delta_bias"], x["D"], sl(x["z"], a, b))
+    y1, h1 = oracle.s6_forward(*args(0, 21), lib=lib)
+    y2, h2 = oracle.s6_forward(*args(21, 50), lib=lib, initial_state=h1)
+    e = max(normwise(np.concatenate([y1, y2], axis=2), full), normwise(h2, last))
+    return e, 1e-14
+
+
+def pin_initial_state_decay(lib=None):
+    """With u = 0 a starting state only decays: h_L = exp(A sum_t Delta_t) h_0."""
+    x = make_inputs(1, 3, 30, 5, seed=62, has_z=False, has_D=False)
+    h0 = np.random.default_rng(7).standard_normal((1, 3, 5))
+    zeros = torch.zeros_like(x["u"])
+    _, last = oracle.s6_forward(zeros, x["delta"], x["A"], x["B"], x["C"], x["delta_bias"],
+                                lib=lib, initial_state=h0)
+    Delta = _softplus(_np(x["delta"])[0] + _np(x["delta_bias"])[:, None])
+    ref = np.exp(_np(x["A"]) * Delta.sum(axis=1)[:, None]) * h0[0]
+    return normwise(last[0], ref), 1e-13
+
+
 ALL_PINS = [pin_golden, pin_theorem1, pin_zoh_expm, pin_lti_convolution, pin_brute_force,
             pin_held_input_exact, pin_skip_and_gate, pin_large_delta_limit,
             pin_small_delta_limit, pin_structure, pin_finite_differences, pin_autograd,
-            pin_threads_agree]
+            pin_threads_agree, pin_resume_from_state, pin_initial_state_decay]
 
 
 def run_all(lib=None):

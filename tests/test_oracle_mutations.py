@@ -27,6 +27,8 @@ MUTATIONS = {
     "sigmoid_gate_not_silu": ("if (z) y0 *= z[t] * sigmoid(z[t]);", "if (z) y0 *= sigmoid(z[t]);"),
     "bias_ignored": ("const double bias = j->bias ? j->bias[d] : 0.0;\n  const double Dd = j->D ? j->D[d] : 0.0;\n  double *y",
                      "const double bias = 0.0;\n  const double Dd = j->D ? j->D[d] : 0.0;\n  double *y"),
+    "initial_state_ignored": ("h[n] = j->h0 ? j->h0[(b * dim + d) * N + n] : 0.0;",
+                              "h[n] = 0.0;"),
     "bwd_dropped_phi_term": ("Bt * u[t] * Delta * Delta * phi(x)", "0.0"),
     "bwd_adjoint_uses_current_Abar": ("Abar_next[n] * G[n];", "Abar * G[n];"),
     "bwd_dz_missing_factor": ("s * (1.0 + z[t] * (1.0 - s))", "s"),
