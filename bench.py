@@ -343,6 +343,8 @@ def run_ours(args, world, rank, device):
         "gpu_launches": launches, "clocks": sampler.summary(),
     }
 
+    if not args.only and not args.no_decode:
+        result["decode"] = run_decode(w, x, device, peaks)
     if args.only:
         result["note"] = f"--only {args.only}: a profiling run, not a benchmark result"
     if not args.no_e2e and not args.only:
@@ -354,6 +356,73 @@ def run_ours(args, world, rank, device):
         result["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": threads,
                                   "kind": "oracle", "sample": desc}
     return result
+
+
+def decode_bytes(w) -> int:
+    """Algorithmic bytes of one decoding step: read and write the fp32 state
+    (8 N bytes per channel), read u, delta, z and write y (4 s per channel),
+    read the B and C rows and the parameters."""
+    s = w.io_bytes
+    ch = w.batch * w.dim
+    return ch * (8 * w.N + 4 * s) + 2 * w.batch * w.N * s + 4 * (w.dim * w.N + 2 * w.dim)
+
+
+def run_decode(w, x, device, peaks, steps=200):
+    """One token per batch row through mamba_scan_step, repeated `steps` times
+    on the workload's channels (a decoding loop after a prefill)."""
+    from selective_state_space_21_b200 import scan
+
+    tok = {k: x[k][:, :, 0].contiguous() for k in ("u", "delta", "z", "B", "C")}
+    state = torch.zeros(w.batch, w.dim, w.N, device=device)
+    y = torch.empty_like(tok["u"])
+
+    def step():
+        scan.mamba_scan_step(state, tok["u"], tok["delta"], x["delta_bias"], x["A"], tok["B"],
+                             tok["C"], x["D"], tok["z"], y)
+
+    for _ in range(10):
+        step()
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize(device)
+    if scan.mamba_scan_stream_status() != 0:
+        raise RuntimeError("device error in the decoding loop")
+    ms = e0.elapsed_time(e1) / steps
+    nb = decode_bytes(w)
+    gbs = nb / (ms * 1e-3) / 1e9
+    out = {"us_per_token_step": round(ms * 1e3, 3), "tokens_per_s": w.batch / (ms * 1e-3),
+           "bytes_per_step": nb, "gbs": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
+           "steps": steps, "launch": "eager (host-side argument checks every call)",
+           "shape": f"batch {w.batch} x dim {w.dim} x N {w.N}, one token per row"}
+    # The same loop replayed from a CUDA graph (how a decoding loop is usually
+    # run): device time per step without the per-call host work.
+    try:
+        s_cap = torch.cuda.Stream(device)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(s_cap):
+            step()
+            torch.cuda.synchronize(device)
+            with torch.cuda.graph(graph, stream=s_cap):
+                for _ in range(steps):
+                    step()
+        graph.replay()
+        torch.cuda.synchronize(device)
+        e0.record()
+        graph.replay()
+        e1.record()
+        torch.cuda.synchronize(device)
+        gms = e0.elapsed_time(e1) / steps
+        ggbs = nb / (gms * 1e-3) / 1e9
+        out["graph"] = {"us_per_token_step": round(gms * 1e3, 3),
+                        "tokens_per_s": w.batch / (gms * 1e-3), "gbs": round(ggbs, 1),
+                        "frac_hbm": round(ggbs / peaks["hbm_gbs"], 4)}
+    except Exception as e:  # capture not possible here: report the eager loop only
+        out["graph"] = {"unavailable": str(e)[:200]}
+    return out
 
 
 def run_e2e(args, w, x, y, g, fwd, bwd, device, world):
@@ -482,6 +551,7 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--only", choices=["fwd", "bwd"], default=None,
                     help="time one pass only (for profiling; not a benchmark result)")
     args = ap.parse_args(argv)

@@ -152,6 +152,29 @@ MAMBA_SCAN_API mamba_status_t mamba_scan_bwd_ex(const void *u, const void *delta
                                  const mamba_scan_options_t *options, mamba_stream_t stream);
 
 /*
+ * One decoding step: the recurrent mode of the selective SSM, one token per
+ * call with constant work per token ("Mamba: Linear-Time Sequence Modeling
+ * with Selective State Spaces", trishampatil.com walk-through, Part II
+ * section 4: recurrence for autoregressive inference).  For every batch b
+ * and channel d, with state[b,d,:] the state after the previous token:
+ *     Delta = softplus(delta[b,d] + delta_bias[d])
+ *     state[b,d,n] <- exp(Delta A[d,n]) state[b,d,n]
+ *                     + (exp(Delta A[d,n]) - 1)/A[d,n] B[b,n] u[b,d]
+ *     y[b,d] = (sum_n C[b,n] state[b,d,n] + D[d] u[b,d]) silu(z[b,d])
+ *   state          : (batch, dim, N) float32, read and overwritten in place
+ *                    (e.g. the last_state of mamba_scan_fwd over a prompt)
+ *   u, delta, z, y : (batch, dim) dtype;  B, C : (batch, N) dtype
+ *   A, D, delta_bias as in mamba_scan_fwd.  delta_bias, D and z may be NULL.
+ * Repeating the call over the tokens of a sequence gives the same result as
+ * mamba_scan_fwd over the whole sequence, up to rounding.
+ */
+MAMBA_SCAN_API mamba_status_t mamba_scan_step(float *state, const void *u, const void *delta,
+                                              const float *delta_bias, const float *A,
+                                              const void *B, const void *C, const float *D,
+                                              const void *z, void *y, int64_t batch, int64_t dim,
+                                              int64_t N, mamba_dtype_t dtype, mamba_stream_t stream);
+
+/*
  * Forward that allocates nothing.  (An addition of this library for callers
  * that cannot allocate; the paper has no counterpart.)
  *

@@ -13,6 +13,7 @@
 #include "bwd_reference.cuh"
 #include "bwd_staged.cuh"
 #include "common.cuh"
+#include "decode.cuh"
 #include "fwd_reference.cuh"
 #include "fwd_staged.cuh"
 
@@ -386,6 +387,56 @@ mamba_status_t mamba_scan_bwd_ex(const void *u, const void *delta, const float *
   if (st == MAMBA_ERR_UNSUPPORTED && so.path == MAMBA_PATH_AUTO)
     return dispatch<BwdReferenceLauncher>(dtype, (int)N, a, s);
   return st;
+}
+
+mamba_status_t mamba_scan_step(float *state, const void *u, const void *delta,
+                               const float *delta_bias, const float *A, const void *B, const void *C,
+                               const float *D, const void *z, void *y, int64_t batch, int64_t dim,
+                               int64_t N, mamba_dtype_t dtype, mamba_stream_t stream) {
+  mamba_status_t st = check_shape(batch, dim, 1, N, dtype);
+  if (st != MAMBA_OK) return st;
+  Checker ck;
+  if (cudaGetDevice(&ck.dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MAMBA_ERR_CUDA;
+  }
+  const size_t es = dtype_size(dtype);
+  const size_t nbd = size_t(batch) * size_t(dim);
+  ck.buf(u, nbd * es, es, true, false);
+  ck.buf(delta, nbd * es, es, true, false);
+  ck.buf(z, nbd * es, es, false, false);
+  ck.buf(B, size_t(batch) * N * es, es, true, false);
+  ck.buf(C, size_t(batch) * N * es, es, true, false);
+  ck.buf(A, size_t(dim) * N * 4, 4, true, false);
+  ck.buf(D, size_t(dim) * 4, 4, false, false);
+  ck.buf(delta_bias, size_t(dim) * 4, 4, false, false);
+  ck.buf(state, nbd * N * 4, 4, true, true);
+  ck.buf(y, nbd * es, es, true, true);
+  if (ck.st != MAMBA_OK) return ck.st;
+  if (nbd == 0) return MAMBA_OK;
+  DecodeArgs a;
+  a.state = state; a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
+  a.bias = delta_bias; a.A = A; a.D = D; a.y = y;
+  a.batch = batch; a.dim = dim; a.N = (int)N;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t grid = (int64_t(nbd) + kDecodeThreads - 1) / kDecodeThreads;
+  if (grid > (int64_t(1) << 31) - 1) return MAMBA_ERR_UNSUPPORTED;
+  auto launch = [&](auto tag, auto nm) {
+    using T = typename decltype(tag)::type;
+    decode_step_kernel<T, decltype(nm)::value><<<unsigned(grid), kDecodeThreads, 0, s>>>(a);
+  };
+  struct TF { using type = float; };
+  struct TB { using type = __nv_bfloat16; };
+  if (dtype == MAMBA_BF16) {
+    if (N <= 4) launch(TB{}, std::integral_constant<int, 4>{});
+    else if (N <= 8) launch(TB{}, std::integral_constant<int, 8>{});
+    else launch(TB{}, std::integral_constant<int, 16>{});
+  } else {
+    if (N <= 4) launch(TF{}, std::integral_constant<int, 4>{});
+    else if (N <= 8) launch(TF{}, std::integral_constant<int, 8>{});
+    else launch(TF{}, std::integral_constant<int, 16>{});
+  }
+  return launch_status();
 }
 
 mamba_status_t mamba_scan_bwd(const void *u, const void *delta, const float *delta_bias,

@@ -63,6 +63,8 @@ def load_library():
             lib.mamba_scan_bwd.argtypes = [vp] * 17 + [i64] * 4 + [i32, vp]
             lib.mamba_scan_bwd_ex.argtypes = [vp] * 17 + [i64] * 4 + [i32, opt, vp]
             lib.mamba_scan_fwd_noalloc.argtypes = [vp] * 10 + [i64] * 4 + [i32, vp]
+            lib.mamba_scan_step.argtypes = [vp] * 10 + [i64] * 3 + [i32, vp]
+            lib.mamba_scan_step.restype = ctypes.c_int
             for f in ("mamba_scan_fwd", "mamba_scan_fwd_ex", "mamba_scan_bwd",
                       "mamba_scan_bwd_ex", "mamba_scan_stream_status", "mamba_scan_fwd_noalloc"):
                 getattr(lib, f).restype = ctypes.c_int
@@ -195,6 +197,23 @@ def mamba_scan_fwd_noalloc(u, delta, delta_bias, A, B, C, D, z, y, last_state, *
         batch, dim, L, N, _dtype_code(dt)]
     _check(load_library().mamba_scan_fwd_noalloc(*args, _stream_handle(stream)),
            "mamba_scan_fwd_noalloc")
+
+
+def mamba_scan_step(state, u, delta, delta_bias, A, B, C, D, z, y, *, stream=None):
+    """One decoding step (one token per batch row): updates ``state``
+    (batch, dim, N) float32 in place and writes ``y`` (batch, dim).  u, delta,
+    z, y: (batch, dim); B, C: (batch, N), in the I/O dtype."""
+    batch, dim = u.shape
+    N = A.shape[1]
+    dt = u.dtype
+    f32 = torch.float32
+    args = [
+        _ptr(state, f32, (batch, dim, N), "state"), _ptr(u, dt, (batch, dim), "u"),
+        _ptr(delta, dt, (batch, dim), "delta"), _ptr(delta_bias, f32, (dim,), "delta_bias"),
+        _ptr(A, f32, (dim, N), "A"), _ptr(B, dt, (batch, N), "B"), _ptr(C, dt, (batch, N), "C"),
+        _ptr(D, f32, (dim,), "D"), _ptr(z, dt, (batch, dim), "z"), _ptr(y, dt, (batch, dim), "y"),
+        batch, dim, N, _dtype_code(dt)]
+    _check(load_library().mamba_scan_step(*args, _stream_handle(stream)), "mamba_scan_step")
 
 
 def launch_count() -> int:
