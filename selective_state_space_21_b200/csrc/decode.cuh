@@ -70,4 +70,66 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_step_kernel(const Decod
   static_cast<T *>(a.y)[ch] = from_f<T>(y0);
 }
 
+// The same step with four states per thread (N a multiple of 4, 16-byte
+// aligned state and A): a warp's state and A accesses are then contiguous
+// 16-byte vectors, and the NM/4 threads of a channel join their partial
+// readouts with shuffles.
+template <typename T> struct Quad;
+template <> struct Quad<float> {
+  __device__ static float4 load(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+};
+template <> struct Quad<__nv_bfloat16> {
+  __device__ static float4 load(const __nv_bfloat16 *p) {
+    const uint2 v = *reinterpret_cast<const uint2 *>(p);
+    return make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
+                       __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
+  }
+};
+
+template <typename T, int NM>
+__global__ void __launch_bounds__(kDecodeThreads) decode_step_vec4_kernel(const DecodeArgs a) {
+  constexpr int TPC = NM / 4;  // threads per channel
+  const int64_t gid = int64_t(blockIdx.x) * kDecodeThreads + threadIdx.x;
+  const int64_t ch = gid / TPC;
+  const int g = int(gid % TPC);
+  const bool live = ch < a.batch * a.dim;  // dead threads still join the shuffles
+  const int64_t chs = live ? ch : 0;
+  const int64_t b = chs / a.dim, d = chs % a.dim;
+  const float4 h = *reinterpret_cast<const float4 *>(a.state + chs * NM + 4 * g);
+  const float4 Av = *reinterpret_cast<const float4 *>(a.A + d * NM + 4 * g);
+  const float4 Bv = Quad<T>::load(static_cast<const T *>(a.B) + b * NM + 4 * g);
+  const float4 Cv = Quad<T>::load(static_cast<const T *>(a.C) + b * NM + 4 * g);
+  const float uv = to_f(static_cast<const T *>(a.u)[chs]);
+  const float v = to_f(static_cast<const T *>(a.delta)[chs]) + (a.bias ? a.bias[d] : 0.f);
+  const float Delta = softplus_fast(v);
+  const float hs[4] = {h.x, h.y, h.z, h.w}, As[4] = {Av.x, Av.y, Av.z, Av.w};
+  const float Bs_[4] = {Bv.x, Bv.y, Bv.z, Bv.w}, Cs_[4] = {Cv.x, Cv.y, Cv.z, Cv.w};
+  float hn[4], yp = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float x = Delta * As[i];
+    const float e = ex2f(x * kLog2e);
+    float p = fmaf(x, 1.f / 720.f, 1.f / 120.f);
+    p = fmaf(x, p, 1.f / 24.f);
+    p = fmaf(x, p, 1.f / 6.f);
+    p = fmaf(x, p, 0.5f);
+    p = fmaf(x, p, 1.f);
+    const float Eb = fabsf(x) < 0.25f ? Delta * p : (e - 1.f) / As[i];
+    hn[i] = fmaf(e, hs[i], Eb * Bs_[i] * uv);
+    yp = fmaf(Cs_[i], hn[i], yp);
+  }
+#pragma unroll
+  for (int o = 1; o < TPC; o <<= 1) yp += __shfl_xor_sync(0xffffffffu, yp, o);
+  if (!live) return;
+  *reinterpret_cast<float4 *>(a.state + ch * NM + 4 * g) = make_float4(hn[0], hn[1], hn[2], hn[3]);
+  if (g == 0) {
+    float y0 = yp + (a.D ? a.D[d] * uv : 0.f);
+    if (a.z) {
+      const float zv = to_f(static_cast<const T *>(a.z)[ch]);
+      y0 *= zv * rcpf(1.f + ex2f(-zv * kLog2e));
+    }
+    static_cast<T *>(a.y)[ch] = from_f<T>(y0);
+  }
+}
+
 }  // namespace mscan

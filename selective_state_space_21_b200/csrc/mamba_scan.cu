@@ -419,6 +419,27 @@ mamba_status_t mamba_scan_step(float *state, const void *u, const void *delta,
   a.bias = delta_bias; a.A = A; a.D = D; a.y = y;
   a.batch = batch; a.dim = dim; a.N = (int)N;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // four states per thread when N is 4, 8 or 16 and the state, A, B and C
+  // rows are 16- (B, C: 8-) byte aligned
+  const bool al16 = ((reinterpret_cast<uintptr_t>(state) | reinterpret_cast<uintptr_t>(A)) & 15) == 0;
+  const bool alBC = ((reinterpret_cast<uintptr_t>(B) | reinterpret_cast<uintptr_t>(C)) & (4 * es - 1)) == 0;
+  if ((N == 4 || N == 8 || N == 16) && al16 && alBC) {
+    const int64_t threads = int64_t(nbd) * (N / 4);
+    const int64_t g4 = (threads + kDecodeThreads - 1) / kDecodeThreads;
+    if (g4 > (int64_t(1) << 31) - 1) return MAMBA_ERR_UNSUPPORTED;
+#define MSCAN_VEC4(TT, NN) decode_step_vec4_kernel<TT, NN><<<unsigned(g4), kDecodeThreads, 0, s>>>(a)
+    if (dtype == MAMBA_BF16) {
+      if (N == 4) MSCAN_VEC4(__nv_bfloat16, 4);
+      else if (N == 8) MSCAN_VEC4(__nv_bfloat16, 8);
+      else MSCAN_VEC4(__nv_bfloat16, 16);
+    } else {
+      if (N == 4) MSCAN_VEC4(float, 4);
+      else if (N == 8) MSCAN_VEC4(float, 8);
+      else MSCAN_VEC4(float, 16);
+    }
+#undef MSCAN_VEC4
+    return launch_status();
+  }
   const int64_t grid = (int64_t(nbd) + kDecodeThreads - 1) / kDecodeThreads;
   if (grid > (int64_t(1) << 31) - 1) return MAMBA_ERR_UNSUPPORTED;
   auto launch = [&](auto tag, auto nm) {
