@@ -96,9 +96,10 @@ typedef struct {
                               1 = sequential hand-off (a bounded wait on the predecessor),
                               2 = three-phase (aggregate, scan over chunks, recompute) */
   int32_t wait_timeout_us; /* bound of every device-side wait; 0 = 2,000,000 (2 s) */
-  int32_t test_hook;       /* 0 in normal use.  1: the first chunk of the first channel
-                              group never publishes its end state, so that the waits on it
-                              expire (tests MAMBA_ERR_DEVICE_TIMEOUT; outputs undefined) */
+  int32_t test_hook;       /* 0 in normal use.  1: the first chunk processed of the first
+                              channel group (the first in time for the forward, the last for
+                              the backward) never publishes its state, so that the waits on
+                              it expire (tests MAMBA_ERR_DEVICE_TIMEOUT; outputs undefined) */
   int32_t reserved[3];     /* must be 0 */
 } mamba_scan_options_t;
 

@@ -80,6 +80,7 @@ struct BwdStagedArgs {
   float *part_bias;    // [G][K][128]
   uint64_t timeout_ns;
   int force_generic;
+  int test_hook;  // 1: the last chunk of group 0 never publishes its adjoint (tests the bounded wait)
 };
 
 // Byte offset of 16-byte chunk c of row r in a tile with RB-byte rows written
@@ -631,7 +632,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
       for (int n = 0; n < NM; ++n) p.carry[(int64_t(g) * NM + n) * kSThreads + tid] = gt[n];
       __threadfence();
       __syncthreads();
-      if (tid == 0) st_release_gpu(p.flags + g, r + 1);
+      if (tid == 0 && !(p.test_hook == 1 && g == 0 && r == 0)) st_release_gpu(p.flags + g, r + 1);
     }
     if (tid == 0) {  // claim the next unit and fill the free stages
       produce(true);
@@ -770,6 +771,7 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
   bp.part_bias = bp.part_D + n_D;
   bp.timeout_ns = o.timeout_us > 0 ? uint64_t(o.timeout_us) * 1000ull : kDefaultTimeoutNs;
   bp.force_generic = o.path == MAMBA_PATH_GENERIC ? 1 : 0;
+  bp.test_hook = o.test_hook;
 
   mamba_status_t st = MAMBA_OK;
   if (cudaMemsetAsync(ws, 0, int_bytes, s) != cudaSuccess) st = MAMBA_ERR_CUDA;
@@ -781,6 +783,7 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
     StagedOptions fo = o;
     fo.chunk_len = 0;
     fo.carry = 0;
+    fo.test_hook = 0;  // the hook targets the reverse hand-off
     st = staged_forward<T, NM>(fa, fo, s, launched, ckpt);
   }
   if (st == MAMBA_OK) {

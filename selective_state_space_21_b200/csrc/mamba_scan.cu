@@ -377,7 +377,7 @@ mamba_status_t mamba_scan_bwd_ex(const void *u, const void *delta, const float *
   so.chunk_len = options ? options->chunk_len : 0;
   so.carry = options ? options->carry : 0;
   so.timeout_us = options ? options->wait_timeout_us : 0;
-  so.test_hook = 0;
+  so.test_hook = options ? options->test_hook : 0;
   const bool stageable = staged_bwd_supported(a, es);
   if (so.path == MAMBA_PATH_REFERENCE || (!stageable && so.path == MAMBA_PATH_AUTO))
     return dispatch<BwdReferenceLauncher>(dtype, (int)N, a, s);

@@ -152,7 +152,8 @@ def mamba_scan_fwd(u, delta, delta_bias, A, B, C, D, z, y, last_state, *, path="
 
 
 def mamba_scan_bwd(u, delta, delta_bias, A, B, C, D, z, dy, du, ddelta, dA, dB, dC, dD, dz,
-                   ddelta_bias, *, path="auto", chunk_len=0, stream=None):
+                   ddelta_bias, *, path="auto", chunk_len=0, wait_timeout_us=0, test_hook=0,
+                   stream=None):
     """Enqueue the backward of sum(dy * y) on ``stream``; the gradient tensors
     are written."""
     batch, dim, L = u.shape
@@ -170,11 +171,11 @@ def mamba_scan_bwd(u, delta, delta_bias, A, B, C, D, z, dy, du, ddelta, dA, dB, 
         _ptr(dz, dt, bdl, "dz"), _ptr(ddelta_bias, f32, (dim,), "ddelta_bias"),
         batch, dim, L, N, _dtype_code(dt)]
     lib = load_library()
-    if path == "auto" and not chunk_len:
+    if path == "auto" and not chunk_len and not wait_timeout_us and not test_hook:
         rc = lib.mamba_scan_bwd(*args, _stream_handle(stream))
     else:
-        rc = lib.mamba_scan_bwd_ex(*args, ctypes.byref(_options(path, chunk_len)),
-                                   _stream_handle(stream))
+        opts = _options(path, chunk_len, "auto", wait_timeout_us, test_hook)
+        rc = lib.mamba_scan_bwd_ex(*args, ctypes.byref(opts), _stream_handle(stream))
     _check(rc, "mamba_scan_bwd")
 
 

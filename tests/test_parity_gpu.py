@@ -86,7 +86,7 @@ def test_fwd_generic_A(dtype):
 
 STAGED = [  # shapes the staged kernels take (rows of 16-byte multiples, N >= 3)
     (2, 300, 1024, 16), (1, 129, 2048, 4), (3, 40, 96, 16), (2, 256, 4096, 16), (1, 128, 64, 8),
-    (2, 70, 520, 3),
+    (2, 70, 520, 3), (1, 96, 256, 12), (2, 50, 128, 6),
 ]
 
 
@@ -206,7 +206,7 @@ def test_bwd_grid(shape, dtype):
 
 
 BWD_STAGED = [(2, 200, 1024, 16), (1, 130, 512, 8), (3, 40, 96, 4), (2, 128, 1000, 16),
-              (1, 64, 64, 3)]
+              (1, 64, 64, 3), (1, 96, 256, 12), (2, 50, 128, 6)]
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
@@ -236,6 +236,24 @@ def test_bwd_staged_structured_scaled_and_mixed_A():
     x["A"] = (-scale * torch.arange(1, 17, dtype=torch.float32)[None, :]).contiguous()
     x["A"][200, 3] = -7.25  # one group falls back to the generic arithmetic
     _bwd_case(x)
+
+
+def test_bwd_reverse_wait_times_out_without_hanging():
+    """The last chunk of group 0 never publishes its adjoint: the backward's
+    waits on it expire (bounded), the host reads MAMBA_ERR_DEVICE_TIMEOUT and a
+    normal backward afterwards is correct."""
+    xh = make_inputs(1, 256, 1024, 16, torch.bfloat16, seed=57, with_dy=True)
+    x = gc.to_device(xh)
+    g = {k: torch.empty_like(x[k]) for k in ("u", "B", "C")}
+    f32 = dict(device="cuda", dtype=torch.float32)
+    dA, dD, db = torch.empty(256, 16, **f32), torch.empty(256, **f32), torch.empty(256, **f32)
+    du, dd, dz = torch.empty_like(x["u"]), torch.empty_like(x["u"]), torch.empty_like(x["u"])
+    scan.mamba_scan_bwd(x["u"], x["delta"], x["delta_bias"], x["A"], x["B"], x["C"], x["D"],
+                        x["z"], x["dy"], du, dd, dA, g["B"], g["C"], dD, dz, db, chunk_len=128,
+                        wait_timeout_us=2000, test_hook=1)
+    assert scan.mamba_scan_stream_status() == 5  # MAMBA_ERR_DEVICE_TIMEOUT
+    assert scan.mamba_scan_stream_status() == 0
+    _bwd_case(xh)
 
 
 def test_bwd_staged_deterministic():
