@@ -280,8 +280,8 @@ struct StagedLayout {
   static constexpr int BSTR = (NM < 4 ? 4 : NM) + 4;     // fp32 row stride of B' / C
   static constexpr int OFF_Y = kStages * kStageBytes;
   static constexpr int OFF_BS = OFF_Y + 2 * kTileBytes;
-  static constexpr int OFF_CS = OFF_BS + TT * BSTR * 4;
-  static constexpr int OFF_BAR = OFF_CS + TT * BSTR * 4;
+  static constexpr int OFF_CS = OFF_BS + 2 * TT * BSTR * 4;   // B' and C: two buffers each
+  static constexpr int OFF_BAR = OFF_CS + 2 * TT * BSTR * 4;
   static constexpr int OFF_Q = OFF_BAR + 8 * kStages;
   static constexpr int BYTES = OFF_Q + 16 * 4;
   static constexpr int ALLOC = BYTES + 1024;  // slack to align the base to 1 KB
@@ -467,34 +467,43 @@ __global__ void __launch_bounds__(kSThreads, 2)
       const float A0 = Arow[0];
       const float invA0 = 1.f / A0;
 
-      for (int it = 0; it < ntiles; ++it, ++ctile) {
-        const int stage = ctile % kStages;
-        const uint32_t parity = uint32_t(ctile / kStages) & 1u;
-        unsigned char *st = sm + stage * kStageBytes;
-        if (!mbar_wait_bounded(&bars[stage], parity, p.timeout_ns)) {
+      // Waits for the tile in stage slot `ct % kStages` and writes its B and C
+      // rows as fp32, time-major, into buffer ct & 1 (B scaled by 1/(n+1) for
+      // the structured arithmetic).  The tables are double-buffered so that
+      // the next tile's are written at the end of the current one, under the
+      // same barrier as the y tile.
+      auto stage_tables = [&](int ct) {
+        const int stg = ct % kStages;
+        if (!mbar_wait_bounded(&bars[stg], uint32_t(ct / kStages) & 1u, p.timeout_ns)) {
           record_timeout();
           q[8] = 1;
         }
-        // B and C rows of this tile -> fp32, time-major, B scaled by 1/(n+1)
-        // for the structured arithmetic.
-        {
-          const T *Braw = reinterpret_cast<const T *>(st + 3 * kTileBytes);
-          const T *Craw = reinterpret_cast<const T *>(st + 3 * kTileBytes + kRawBytes);
-          constexpr int ITEMS = NM * (TT / 4);
-          for (int w = tid; w < (kOut ? 2 : 1) * ITEMS; w += kSThreads) {
-            const bool isC = w >= ITEMS;
-            const int r = isC ? w - ITEMS : w;
-            const int n = r % NM, tg = r / NM;
-            const T *src = (isC ? Craw : Braw) + n * TT + 4 * tg;
-            float *dst = (isC ? Cs : Bs) + 4 * tg * BSTR + n;
-            const float scale = (!isC && M != MODE_GEN) ? 1.f / float(n + 1) : 1.f;
+        const unsigned char *sst = sm + stg * kStageBytes;
+        const T *Braw = reinterpret_cast<const T *>(sst + 3 * kTileBytes);
+        const T *Craw = reinterpret_cast<const T *>(sst + 3 * kTileBytes + kRawBytes);
+        float *Bd = Bs + (ct & 1) * TT * BSTR;
+        float *Cd = Cs + (ct & 1) * TT * BSTR;
+        constexpr int ITEMS = NM * (TT / 4);
+        for (int w = tid; w < (kOut ? 2 : 1) * ITEMS; w += kSThreads) {
+          const bool isC = w >= ITEMS;
+          const int r = isC ? w - ITEMS : w;
+          const int n = r % NM, tg = r / NM;
+          const T *src = (isC ? Craw : Braw) + n * TT + 4 * tg;
+          float *dst = (isC ? Cd : Bd) + 4 * tg * BSTR + n;
+          const float scale = (!isC && M != MODE_GEN) ? 1.f / float(n + 1) : 1.f;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i * BSTR] = n < N ? raw_to_f(src, i) * scale : 0.f;
-          }
+          for (int i = 0; i < 4; ++i) dst[i * BSTR] = n < N ? raw_to_f(src, i) * scale : 0.f;
         }
-        __syncthreads();
-        if (q[8]) return;
+      };
+      stage_tables(ctile);
+      __syncthreads();
+      if (q[8]) return;
 
+      for (int it = 0; it < ntiles; ++it, ++ctile) {
+        const int stage = ctile % kStages;
+        unsigned char *st = sm + stage * kStageBytes;
+        const float *Bt = Bs + (ctile & 1) * TT * BSTR;
+        const float *Ct = Cs + (ctile & 1) * TT * BSTR;
         const int64_t t0 = tbeg + int64_t(it) * TT;
         const unsigned char *su = st;
         const unsigned char *sd = st + kTileBytes;
@@ -527,8 +536,8 @@ __global__ void __launch_bounds__(kSThreads, 2)
 #pragma unroll
           for (int i = 0; i < VEC; ++i) {
             const int tl = j * VEC + i;
-            const float *Brow = Bs + tl * BSTR;
-            const float *Crow = Cs + tl * BSTR;
+            const float *Brow = Bt + tl * BSTR;
+            const float *Crow = Ct + tl * BSTR;
             const float v = dv[i] + bias;
             float y0;
             if constexpr (M == MODE_SIG) {
@@ -570,8 +579,10 @@ __global__ void __launch_bounds__(kSThreads, 2)
           }
           if (kOut) *reinterpret_cast<uint4 *>(sy + off) = Vec<T>::pack(yv);
         }
+        if (it + 1 < ntiles) stage_tables(ctile + 1);
         if (kOut) fence_proxy_async_smem();
         __syncthreads();
+        if (q[8]) return;
         if (tid == 0) {
           if (kOut) {
             tma_store_3d(&tm_y, sy, int(t0), d0, b);
