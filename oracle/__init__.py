@@ -44,7 +44,7 @@ def build(force: bool = False) -> str:
 
 
 def load_library(path: str):
-    """Load an oracle shared library and declare its two entry points."""
+    """Load an oracle shared library and declare its entry points."""
     lib = ctypes.CDLL(path)
     dp = ctypes.c_void_p
     i64 = ctypes.c_longlong
@@ -52,6 +52,12 @@ def load_library(path: str):
     lib.s6_oracle_fwd.restype = ctypes.c_int
     lib.s6_oracle_bwd.argtypes = [dp] * 17 + [i64] * 5
     lib.s6_oracle_bwd.restype = ctypes.c_int
+    lib.s6_oracle_conv_silu.argtypes = [dp] * 3 + [i64] + [dp] * 2 + [i64] * 3
+    lib.s6_oracle_conv_silu.restype = ctypes.c_int
+    lib.s6_oracle_conv_fwd.argtypes = [dp] * 3 + [i64] + [dp] * 9 + [i64] * 5
+    lib.s6_oracle_conv_fwd.restype = ctypes.c_int
+    lib.s6_oracle_conv_bwd.argtypes = [dp] * 3 + [i64] + [dp] * 18 + [i64] * 5
+    lib.s6_oracle_conv_bwd.restype = ctypes.c_int
     return lib
 
 
@@ -126,6 +132,85 @@ def s6_backward(u, delta, A, B, C, dy, delta_bias=None, D=None, z=None, nthreads
     if rc != 0:
         raise RuntimeError(f"s6_oracle_bwd failed ({rc})")
     out = {"du": du, "ddelta": ddelta, "dA": dA, "dB": dB, "dC": dC, "ddelta_bias": dbias}
+    if dD is not None:
+        out["dD"] = dD
+    if dz is not None:
+        out["dz"] = dz
+    return out
+
+
+def conv_silu(x, conv_w, conv_b=None, lib=None):
+    """The convolution prologue alone: returns (pre, u) with
+    pre[b,d,t] = conv_b[d] + sum_k conv_w[d,k] x[b,d,t-(W-1)+k] (x = 0 before
+    t = 0) and u = SiLU(pre).  x (batch, dim, L); conv_w (dim, W); conv_b
+    (dim,) or None."""
+    x, conv_w, conv_b = _f64(x), _f64(conv_w), _f64(conv_b)
+    batch, dim, L = x.shape
+    W = conv_w.shape[1]
+    assert conv_w.shape == (dim, W)
+    pre = np.empty_like(x)
+    u = np.empty_like(x)
+    rc = (lib or _load()).s6_oracle_conv_silu(_ptr(x), _ptr(conv_w), _ptr(conv_b), W, _ptr(pre),
+                                              _ptr(u), batch, dim, L)
+    if rc != 0:
+        raise RuntimeError(f"s6_oracle_conv_silu failed ({rc})")
+    return pre, u
+
+
+def s6_conv_forward(x, conv_w, conv_b, delta, A, B, C, delta_bias=None, D=None, z=None,
+                    nthreads=None, lib=None):
+    """fp64 forward with the convolution prologue: u = SiLU(causal depthwise
+    conv of x), then the S6 forward.  Returns (y, last_state)."""
+    x, conv_w, conv_b = _f64(x), _f64(conv_w), _f64(conv_b)
+    delta, A, B, C = (_f64(t) for t in (delta, A, B, C))
+    delta_bias, D, z = _f64(delta_bias), _f64(D), _f64(z)
+    batch, dim, L = x.shape
+    N = A.shape[1]
+    W = conv_w.shape[1]
+    assert conv_w.shape == (dim, W) and delta.shape == x.shape and B.shape == (batch, N, L)
+    y = np.empty((batch, dim, L), np.float64)
+    last = np.empty((batch, dim, N), np.float64)
+    rc = (lib or _load()).s6_oracle_conv_fwd(
+        _ptr(x), _ptr(conv_w), _ptr(conv_b), W, _ptr(delta), _ptr(delta_bias), _ptr(A), _ptr(B),
+        _ptr(C), _ptr(D), _ptr(z), _ptr(y), _ptr(last), batch, dim, L, N,
+        nthreads or default_threads())
+    if rc != 0:
+        raise RuntimeError(f"s6_oracle_conv_fwd failed ({rc})")
+    return y, last
+
+
+def s6_conv_backward(x, conv_w, conv_b, delta, A, B, C, dy, delta_bias=None, D=None, z=None,
+                     nthreads=None, lib=None):
+    """fp64 backward of sum(dy * y) for the forward with the convolution
+    prologue.  Returns a dict with dx, dconv_w, ddelta, dA, dB, dC,
+    ddelta_bias and, when the matching input is given, dconv_b, dD, dz."""
+    x, conv_w, conv_b = _f64(x), _f64(conv_w), _f64(conv_b)
+    delta, A, B, C, dy = (_f64(t) for t in (delta, A, B, C, dy))
+    delta_bias, D, z = _f64(delta_bias), _f64(D), _f64(z)
+    batch, dim, L = x.shape
+    N = A.shape[1]
+    W = conv_w.shape[1]
+    dx = np.empty_like(x)
+    ddelta = np.empty_like(x)
+    dz = np.empty_like(x) if z is not None else None
+    dcw = np.empty((dim, W), np.float64)
+    dcb = np.empty((dim,), np.float64) if conv_b is not None else None
+    dA = np.empty((dim, N), np.float64)
+    dB = np.empty((batch, N, L), np.float64)
+    dC = np.empty((batch, N, L), np.float64)
+    dD = np.empty((dim,), np.float64) if D is not None else None
+    dbias = np.empty((dim,), np.float64)
+    rc = (lib or _load()).s6_oracle_conv_bwd(
+        _ptr(x), _ptr(conv_w), _ptr(conv_b), W, _ptr(delta), _ptr(delta_bias), _ptr(A), _ptr(B),
+        _ptr(C), _ptr(D), _ptr(z), _ptr(dy), _ptr(dx), _ptr(dcw), _ptr(dcb), _ptr(ddelta),
+        _ptr(dA), _ptr(dB), _ptr(dC), _ptr(dD), _ptr(dz), _ptr(dbias), batch, dim, L, N,
+        nthreads or default_threads())
+    if rc != 0:
+        raise RuntimeError(f"s6_oracle_conv_bwd failed ({rc})")
+    out = {"dx": dx, "dconv_w": dcw, "ddelta": ddelta, "dA": dA, "dB": dB, "dC": dC,
+           "ddelta_bias": dbias}
+    if dcb is not None:
+        out["dconv_b"] = dcb
     if dD is not None:
         out["dD"] = dD
     if dz is not None:

@@ -20,6 +20,12 @@
  *         (trishampatil.com engineering walk-through), Part II section 4
  *         (h_0 = 0) and section 6 (Algorithm 2 shapes).
  *  [TP-III4] same page, Part III section 4 (recomputation in the backward).
+ *  [KN3]  chapterpal.com page, Knowl 3 "Mamba Block Architecture", step 3:
+ *         the main branch runs a short 1D temporal convolution of width
+ *         d_conv = 4, then SiLU, then the S6 layer.
+ *  [PG34] paper-graph-ui summary, "The Mamba Architecture (Section 3.4)",
+ *         "The Mamba simplification": convolution (local context, the
+ *         "shift-SSM" of H3), SiLU, selective SSM on the main branch.
  *
  * What is computed (forward), for every batch b and channel d independently:
  *     Delta_t = softplus(delta[b,d,t] + bias[d])                     [PG33]
@@ -46,6 +52,16 @@
  * (the pages give no gradient formulas).  States are recomputed forward per
  * channel and kept in fp64 (the oracle has no memory constraint), then a
  * reverse sweep accumulates gradients [TP-III4].
+ *
+ * Convolution prologue (s6_oracle_conv_*), [KN3] / [PG34], with the readings
+ * the pages leave open: the convolution is depthwise (one filter of width W
+ * per channel, as the pages apply it per channel of the branch), causal
+ * (x = 0 before the first step, so that step t sees no later input, as a
+ * recurrent model needs) and has an optional per-channel bias:
+ *     pre[b,d,t] = conv_b[d] + sum_{k=0}^{W-1} conv_w[d,k] * x[b,d,t-(W-1)+k]
+ *     u[b,d,t]   = pre * sigmoid(pre)                                (SiLU)
+ * and u feeds the forward above.  Its backward is the chain rule through the
+ * SiLU and the convolution after the S6 backward has given du.
  *
  * Parity pins (the tests check this file against): Theorem 1 closed form,
  * the LTI convolution form, brute-force unrolling, an independent ZOH via the
@@ -329,5 +345,110 @@ int s6_oracle_bwd(const double *u, const double *delta, const double *bias, cons
   free(j.dA_part);
   free(j.dD_part);
   free(j.dbias_part);
+  return rc;
+}
+
+/* ------------------------------------------------ convolution prologue */
+
+/* pre and u = SiLU(pre) of the causal depthwise convolution (see the header). */
+static void conv_silu(const double *x, const double *w, const double *cb, i64 W, double *pre,
+                      double *u, i64 batch, i64 dim, i64 L) {
+  for (i64 b = 0; b < batch; ++b)
+    for (i64 d = 0; d < dim; ++d) {
+      const i64 off = (b * dim + d) * L;
+      for (i64 t = 0; t < L; ++t) {
+        double p = cb ? cb[d] : 0.0;
+        for (i64 k = 0; k < W; ++k) {
+          const i64 s = t - (W - 1) + k; /* the input step weight k looks at */
+          if (s >= 0) p += w[d * W + k] * x[off + s];
+        }
+        pre[off + t] = p;
+        u[off + t] = p * sigmoid(p);
+      }
+    }
+}
+
+/* The convolution prologue alone: u (and pre if non-NULL) from x.  Layouts:
+ * x, pre, u (batch, dim, L); conv_w (dim, W); conv_b (dim) or NULL. */
+int s6_oracle_conv_silu(const double *x, const double *conv_w, const double *conv_b, i64 W,
+                        double *pre, double *u, i64 batch, i64 dim, i64 L) {
+  if (batch < 0 || dim < 0 || L < 0 || W < 1 || W > 64) return -2;
+  const size_t n = (size_t)(batch * dim * L);
+  double *p = pre ? pre : (double *)malloc(sizeof(double) * (n ? n : 1));
+  if (!p) return -1;
+  conv_silu(x, conv_w, conv_b, W, p, u, batch, dim, L);
+  if (!pre) free(p);
+  return 0;
+}
+
+/* Forward with the prologue: u = SiLU(causal depthwise conv of x), then the
+ * S6 forward of s6_oracle_fwd (h = 0 before the first step). */
+int s6_oracle_conv_fwd(const double *x, const double *conv_w, const double *conv_b, i64 W,
+                       const double *delta, const double *bias, const double *A, const double *B,
+                       const double *C, const double *D, const double *z, double *y,
+                       double *last_state, i64 batch, i64 dim, i64 L, i64 N, i64 nthreads) {
+  if (batch < 0 || dim < 0 || L < 0 || W < 1 || W > 64) return -2;
+  const size_t n = (size_t)(batch * dim * L);
+  double *pre = (double *)malloc(sizeof(double) * (n ? n : 1));
+  double *u = (double *)malloc(sizeof(double) * (n ? n : 1));
+  int rc = -1;
+  if (pre && u) {
+    conv_silu(x, conv_w, conv_b, W, pre, u, batch, dim, L);
+    rc = s6_oracle_fwd(u, delta, bias, A, B, C, D, z, NULL, y, last_state, batch, dim, L, N,
+                       nthreads);
+  }
+  free(pre);
+  free(u);
+  return rc;
+}
+
+/* Backward of sum(dy * y) for the forward with the prologue.  Outputs as in
+ * s6_oracle_bwd, with dx (batch, dim, L) in place of du, plus dconv_w (dim, W)
+ * and dconv_b (dim; may be NULL).  The S6 backward gives du at u = SiLU(pre);
+ * then
+ *     dpre_t = du_t * sigmoid(pre_t) * (1 + pre_t * (1 - sigmoid(pre_t)))
+ * and each term conv_w[d,k] * x[s], s = t-(W-1)+k, of pre_t passes dpre_t on:
+ *     dx[s] += conv_w[d,k] * dpre_t,  dconv_w[d,k] += dpre_t * x[s],
+ *     dconv_b[d] += dpre_t. */
+int s6_oracle_conv_bwd(const double *x, const double *conv_w, const double *conv_b, i64 W,
+                       const double *delta, const double *bias, const double *A, const double *B,
+                       const double *C, const double *D, const double *z, const double *dy,
+                       double *dx, double *dconv_w, double *dconv_b, double *ddelta, double *dA,
+                       double *dB, double *dC, double *dD, double *dz, double *dbias, i64 batch,
+                       i64 dim, i64 L, i64 N, i64 nthreads) {
+  if (batch < 0 || dim < 0 || L < 0 || W < 1 || W > 64) return -2;
+  const size_t n = (size_t)(batch * dim * L);
+  double *pre = (double *)malloc(sizeof(double) * (n ? n : 1));
+  double *u = (double *)malloc(sizeof(double) * (n ? n : 1));
+  double *du = (double *)malloc(sizeof(double) * (n ? n : 1));
+  int rc = -1;
+  if (pre && u && du) {
+    conv_silu(x, conv_w, conv_b, W, pre, u, batch, dim, L);
+    rc = s6_oracle_bwd(u, delta, bias, A, B, C, D, z, dy, du, ddelta, dA, dB, dC, dD, dz, dbias,
+                       batch, dim, L, N, nthreads);
+  }
+  if (rc == 0) {
+    memset(dx, 0, sizeof(double) * n);
+    memset(dconv_w, 0, sizeof(double) * (size_t)(dim * W));
+    if (dconv_b) memset(dconv_b, 0, sizeof(double) * (size_t)dim);
+    for (i64 b = 0; b < batch; ++b)
+      for (i64 d = 0; d < dim; ++d) {
+        const i64 off = (b * dim + d) * L;
+        for (i64 t = 0; t < L; ++t) {
+          const double s = sigmoid(pre[off + t]);
+          const double dpre = du[off + t] * s * (1.0 + pre[off + t] * (1.0 - s));
+          for (i64 k = 0; k < W; ++k) {
+            const i64 src = t - (W - 1) + k;
+            if (src < 0) continue;
+            dx[off + src] += conv_w[d * W + k] * dpre;
+            dconv_w[d * W + k] += dpre * x[off + src];
+          }
+          if (dconv_b) dconv_b[d] += dpre;
+        }
+      }
+  }
+  free(pre);
+  free(u);
+  free(du);
   return rc;
 }

@@ -20,6 +20,13 @@ size N = 16 (same page, section 3.6 "State dimension N") and sequences up to
 
 A, D and the delta bias are always float32; u, delta, z, B, C and dy use the
 workload's I/O dtype.
+
+For the convolution prologue of the Mamba block (a short causal convolution
+of width d_conv = 4 in front of the S6 layer, Knowl 3 "Mamba Block
+Architecture" of the chapterpal.com page) the input x takes the place of u
+and is drawn the same way; the per-channel filter and bias are drawn
+uniform in [-1/sqrt(W), 1/sqrt(W)] (the usual default initialisation of a
+depthwise Conv1d layer, fan-in W; the pages give none).
 """
 from __future__ import annotations
 
@@ -102,6 +109,18 @@ def make_inputs(batch: int, dim: int, L: int, N: int, dtype: torch.dtype = torch
         "u": u, "delta": delta, "z": z if has_z else None, "B": B, "C": C, "A": A,
         "D": D if has_D else None, "delta_bias": delta_bias, "dy": dy,
     }
+
+
+def make_conv_params(dim: int, width: int = 4, device="cpu", seed: int = SEED_BASE,
+                     has_bias: bool = True) -> dict:
+    """Draw a depthwise convolution filter conv_w (dim, width) and bias conv_b
+    (dim,) (or None), float32, uniform in [-1/sqrt(width), 1/sqrt(width)]."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed + 7919)
+    bound = 1.0 / math.sqrt(width)
+    w = (torch.rand(dim, width, generator=g, device=device) * 2.0 - 1.0) * bound
+    b = (torch.rand(dim, generator=g, device=device) * 2.0 - 1.0) * bound
+    return {"conv_w": w.contiguous(), "conv_b": b if has_bias else None}
 
 
 def workload_inputs(index: int, device="cpu", with_dy: Optional[bool] = None) -> dict:

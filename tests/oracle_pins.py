@@ -20,7 +20,7 @@ import scipy.special
 import torch
 
 import oracle
-from selective_state_space_21_b200.inputs import gated_case, lti_case, make_inputs
+from selective_state_space_21_b200.inputs import gated_case, lti_case, make_conv_params, make_inputs
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_derived_exact.txt")
 
@@ -400,10 +400,124 @@ def pin_initial_state_decay(lib=None):
     return normwise(last[0], ref), 1e-13
 
 
+# ------------------------------------------------- convolution prologue
+
+def _silu(p):
+    return p * scipy.special.expit(p)  # scipy's logistic function
+
+
+def pin_conv_numpy(lib=None):
+    """The causal depthwise convolution against numpy's full convolution
+    (flipped filter, first L outputs) and SiLU through scipy's logistic."""
+    worst = 0.0
+    for W, seed, has_bias in ((4, 71, True), (3, 72, False), (1, 73, True), (2, 74, True)):
+        x = make_inputs(2, 3, 37, 2, seed=seed)["u"].double().numpy()
+        cp = make_conv_params(3, W, seed=seed, has_bias=has_bias)
+        w = cp["conv_w"].double().numpy()
+        cb = None if cp["conv_b"] is None else cp["conv_b"].double().numpy()
+        pre, u = oracle.conv_silu(x, w, cb, lib=lib)
+        ref = np.empty_like(x)
+        for b in range(2):
+            for d in range(3):
+                ref[b, d] = np.convolve(x[b, d], w[d, ::-1])[:37] + (cb[d] if cb is not None else 0.0)
+        worst = max(worst, normwise(pre, ref), normwise(u, _silu(ref)))
+    return worst, 1e-14
+
+
+def pin_conv_special_filters(lib=None):
+    """An identity filter (weight only on the current step, no bias) makes
+    the prologue u = SiLU(x); a filter on the oldest step makes it
+    u_t = SiLU(x_{t-3}) with zeros before the start.  Both then equal the
+    plain forward on that u."""
+    xi = make_inputs(2, 3, 29, 4, seed=75)
+    x = xi["u"].double().numpy()
+    common = dict(delta_bias=xi["delta_bias"], D=xi["D"], z=xi["z"], lib=lib)
+    worst = 0.0
+    for k_on, shift in ((3, 0), (0, 3)):
+        w = np.zeros((3, 4))
+        w[:, k_on] = 1.0
+        y, last = oracle.s6_conv_forward(x, w, None, xi["delta"], xi["A"], xi["B"], xi["C"],
+                                         **common)
+        u = np.zeros_like(x)
+        u[..., shift:] = _silu(x[..., :x.shape[2] - shift])
+        y_ref, last_ref = oracle.s6_forward(u, xi["delta"], xi["A"], xi["B"], xi["C"], **common)
+        worst = max(worst, normwise(y, y_ref), normwise(last, last_ref))
+    return worst, 1e-14
+
+
+def _conv_fd_inputs():
+    x = make_inputs(1, 2, 10, 3, seed=76, with_dy=True)
+    x = {k: (v.double() if v is not None else None) for k, v in x.items()}
+    x["A"] = x["A"] * 0.7
+    cp = make_conv_params(2, 4, seed=76)
+    x["conv_w"] = cp["conv_w"].double()
+    x["conv_b"] = cp["conv_b"].double()
+    return x
+
+
+def _conv_loss(x, lib):
+    y, _ = oracle.s6_conv_forward(x["u"], x["conv_w"], x["conv_b"], x["delta"], x["A"], x["B"],
+                                  x["C"], x["delta_bias"], x["D"], x["z"], lib=lib, nthreads=1)
+    return float(np.sum(_np(x["dy"]) * y))
+
+
+def _conv_grads(x, lib):
+    return oracle.s6_conv_backward(x["u"], x["conv_w"], x["conv_b"], x["delta"], x["A"], x["B"],
+                                   x["C"], x["dy"], x["delta_bias"], x["D"], x["z"], lib=lib,
+                                   nthreads=1)
+
+
+def pin_conv_finite_differences(lib=None):
+    """Central differences of sum(dy * y) through the prologue: x, the filter,
+    its bias, and delta and A behind it."""
+    x = _conv_fd_inputs()
+    g = _conv_grads(x, lib)
+    names = {"u": "dx", "conv_w": "dconv_w", "conv_b": "dconv_b", "delta": "ddelta", "A": "dA"}
+    worst = 0.0
+    for name, gname in names.items():
+        flat = x[name].reshape(-1)
+        fd = np.empty(x[name].shape)
+        for i in range(flat.numel()):
+            v = float(flat[i])
+            h = 1e-6 * max(1.0, abs(v))
+            flat[i] = v + h
+            lp = _conv_loss(x, lib)
+            flat[i] = v - h
+            lm = _conv_loss(x, lib)
+            flat[i] = v
+            fd.reshape(-1)[i] = (lp - lm) / (2.0 * h)
+        worst = max(worst, normwise(g[gname], fd))
+    return worst, 1e-6
+
+
+def pin_conv_autograd(lib=None):
+    """The prologue's chain rule against torch.autograd through torch's own
+    conv1d (causal by left padding, depthwise by groups) and silu, fed with
+    the (separately pinned) S6 gradient du at the prologue's output."""
+    x = _conv_fd_inputs()
+    xs = x["u"].clone().requires_grad_(True)
+    w = x["conv_w"].clone().requires_grad_(True)
+    cb = x["conv_b"].clone().requires_grad_(True)
+    dim, W = w.shape
+    L = xs.shape[2]
+    pre = torch.nn.functional.conv1d(xs, w[:, None, :], cb, padding=W - 1, groups=dim)[..., :L]
+    u = torch.nn.functional.silu(pre)
+    gs6 = oracle.s6_backward(u.detach(), x["delta"], x["A"], x["B"], x["C"], x["dy"],
+                             x["delta_bias"], x["D"], x["z"], lib=lib, nthreads=1)
+    ref = torch.autograd.grad(u, (xs, w, cb), grad_outputs=torch.from_numpy(gs6["du"]))
+    g = _conv_grads(x, lib)
+    worst = 0.0
+    for got, r in zip((g["dx"], g["dconv_w"], g["dconv_b"]), ref):
+        worst = max(worst, normwise(got, r.numpy()))
+    return worst, 1e-12
+
+
 ALL_PINS = [pin_golden, pin_theorem1, pin_zoh_expm, pin_lti_convolution, pin_brute_force,
             pin_held_input_exact, pin_skip_and_gate, pin_large_delta_limit,
             pin_small_delta_limit, pin_structure, pin_finite_differences, pin_autograd,
-            pin_threads_agree, pin_resume_from_state, pin_initial_state_decay]
+            pin_threads_agree, pin_resume_from_state, pin_initial_state_decay,
+            pin_conv_numpy, pin_conv_special_filters, pin_conv_finite_differences,
+            pin_conv_autograd]
 
 
 def run_all(lib=None):

@@ -33,6 +33,15 @@ MUTATIONS = {
     "bwd_adjoint_uses_current_Abar": ("Abar_next[n] * G[n];", "Abar * G[n];"),
     "bwd_dz_missing_factor": ("s * (1.0 + z[t] * (1.0 - s))", "s"),
     "bwd_dDelta_sign": ("(A[n] * hprev + Bt * u[t])", "(A[n] * hprev - Bt * u[t])"),
+    "conv_weight_reversed": ("if (s >= 0) p += w[d * W + k] * x[off + s];",
+                             "if (s >= 0) p += w[d * W + (W - 1 - k)] * x[off + s];"),
+    "conv_silu_dropped": ("u[off + t] = p * sigmoid(p);", "u[off + t] = p;"),
+    "conv_bias_ignored": ("double p = cb ? cb[d] : 0.0;", "double p = 0.0;"),
+    "bwd_conv_dx_wrong_weight": ("dx[off + src] += conv_w[d * W + k] * dpre;",
+                                 "dx[off + src] += conv_w[d * W + (W - 1 - k)] * dpre;"),
+    "bwd_conv_silu_derivative": ("s * (1.0 + pre[off + t] * (1.0 - s))", "s"),
+    "bwd_conv_dw_uses_output_step": ("dconv_w[d * W + k] += dpre * x[off + src];",
+                                     "dconv_w[d * W + k] += dpre * x[off + t];"),
     "bwd_dC_uses_prev_state": ("dCacc[(b * N + n) * L + t] += dy0 * H[(t + 1) * N + n];",
                                "dCacc[(b * N + n) * L + t] += dy0 * H[t * N + n];"),
 }
