@@ -391,6 +391,8 @@ def run_ours(args, world, rank, device):
 
     if not args.only and not args.no_decode:
         result["decode"] = run_decode(w, x, device, peaks)
+    if not args.only and not args.no_conv:
+        result["conv_prologue"] = run_conv(w, x, device, peaks)
     if args.only:
         result["note"] = f"--only {args.only}: a profiling run, not a benchmark result"
     if not args.no_e2e and not args.only:
@@ -411,6 +413,59 @@ def decode_bytes(w) -> int:
     s = w.io_bytes
     ch = w.batch * w.dim
     return ch * (8 * w.N + 4 * s) + 2 * w.batch * w.N * s + 4 * (w.dim * w.N + 2 * w.dim)
+
+
+def run_conv(w, x, device, peaks, steps=10):
+    """The same workload with the block's convolution prologue (width 4):
+    mamba_conv_scan_fwd / _bwd on x in place of u (u = SiLU(conv(x)) is made
+    inside the scan kernels).  Times each call with CUDA events; the bytes are
+    the algorithmic ones of the plain scan plus the filter."""
+    from selective_state_space_21_b200 import scan
+    from selective_state_space_21_b200.inputs import make_conv_params
+
+    cp = make_conv_params(w.dim, 4, device=device, seed=4321)
+    y = torch.empty_like(x["u"])
+    g = {k: torch.empty_like(x[k]) for k in ("u", "delta", "z", "B", "C")}
+    f32 = dict(device=device, dtype=torch.float32)
+    dcw, dcb = torch.empty(w.dim, 4, **f32), torch.empty(w.dim, **f32)
+    dA, dD, db = torch.empty(w.dim, w.N, **f32), torch.empty(w.dim, **f32), torch.empty(w.dim, **f32)
+
+    def fwd():
+        scan.mamba_conv_scan_fwd(x["u"], cp["conv_w"], cp["conv_b"], x["delta"], x["delta_bias"],
+                                 x["A"], x["B"], x["C"], x["D"], x["z"], y, None)
+
+    def bwd():
+        scan.mamba_conv_scan_bwd(x["u"], cp["conv_w"], cp["conv_b"], x["delta"], x["delta_bias"],
+                                 x["A"], x["B"], x["C"], x["D"], x["z"], x["dy"], g["u"],
+                                 dcw, dcb, g["delta"], dA, g["B"], g["C"], dD, g["z"], db)
+
+    for _ in range(3):
+        fwd()
+        bwd()
+    torch.cuda.synchronize(device)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for k in range(steps):
+        ev[k][0].record()
+        fwd()
+        ev[k][1].record()
+        bwd()
+        ev[k][2].record()
+    torch.cuda.synchronize(device)
+    if scan.mamba_scan_stream_status() != 0:
+        raise RuntimeError("device error in the convolution-prologue run")
+    fms = statistics.median(e[0].elapsed_time(e[1]) for e in ev)
+    bms = statistics.median(e[1].elapsed_time(e[2]) for e in ev)
+    extra = 4 * (w.dim * 4 + w.dim)
+    fb, bb = fwd_bytes(w) + extra, bwd_bytes(w) + 2 * extra
+    hbm = peaks["hbm_gbs"]
+    return {"fwd": {"ms": round(fms, 4), "gbs": round(fb / (fms * 1e-3) / 1e9, 1),
+                    "frac_hbm": round(fb / (fms * 1e-3) / 1e9 / hbm, 4),
+                    "tc_per_s": w.token_channels / (fms * 1e-3)},
+            "bwd": {"ms": round(bms, 4), "gbs": round(bb / (bms * 1e-3) / 1e9, 1),
+                    "frac_hbm": round(bb / (bms * 1e-3) / 1e9 / hbm, 4),
+                    "tc_per_s": w.token_channels / (bms * 1e-3)},
+            "steps": steps, "width": 4, "timing": "median of per-call CUDA events",
+            "shape": f"x in place of u, batch {w.batch} x dim {w.dim} x L {w.L}, N {w.N}"}
 
 
 def run_decode(w, x, device, peaks, steps=200):
@@ -598,6 +653,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-conv", action="store_true",
+                    help="skip the convolution-prologue timing")
     ap.add_argument("--only", choices=["fwd", "bwd"], default=None,
                     help="time one pass only (for profiling; not a benchmark result)")
     args = ap.parse_args(argv)

@@ -153,6 +153,59 @@ MAMBA_SCAN_API mamba_status_t mamba_scan_bwd_ex(const void *u, const void *delta
                                  const mamba_scan_options_t *options, mamba_stream_t stream);
 
 /*
+ * Forward with the convolution prologue of the Mamba block: the main branch
+ * runs a short causal 1D convolution and SiLU before the S6 layer
+ * ("Mamba: Linear-Time Sequence Modeling with Selective State Spaces",
+ * chapterpal.com, Knowl 3 "Mamba Block Architecture", step 3, width
+ * d_conv = 4; paper-graph-ui summary, "The Mamba Architecture (Section 3.4)").
+ * The pages do not spell the convolution out; it is read as depthwise (one
+ * filter per channel), causal (x = 0 before the first step) and with an
+ * optional bias:
+ *     pre[b,d,t] = conv_b[d] + sum_{k<W} conv_w[d,k] * x[b,d,t-(W-1)+k]
+ *     u[b,d,t]   = pre * sigmoid(pre)
+ * and u drives the scan of mamba_scan_fwd.  u is computed inside the scan
+ * kernels and never stored.
+ *   x            : (batch, dim, L) dtype, in place of u
+ *   conv_w       : (dim, W) float32, W = conv_width in 1..4 (4 in the Mamba
+ *                  block; other widths return MAMBA_ERR_UNSUPPORTED)
+ *   conv_b       : (dim) float32, nullable (no bias)
+ * Everything else as in mamba_scan_fwd_ex (options may be NULL).
+ */
+MAMBA_SCAN_API mamba_status_t mamba_conv_scan_fwd(const void *x, const float *conv_w,
+                                                  const float *conv_b, int64_t conv_width,
+                                                  const void *delta, const float *delta_bias,
+                                                  const float *A, const void *B, const void *C,
+                                                  const float *D, const void *z, void *y,
+                                                  float *last_state, int64_t batch, int64_t dim,
+                                                  int64_t L, int64_t N, mamba_dtype_t dtype,
+                                                  const mamba_scan_options_t *options,
+                                                  mamba_stream_t stream);
+
+/*
+ * Backward of sum(dy * y) for mamba_conv_scan_fwd, recomputing the prologue
+ * and the states from the inputs.  As mamba_scan_bwd_ex, with
+ *   dx           : (batch, dim, L) dtype, the gradient with respect to x (in
+ *                  place of du; it also serves as scratch for du, so it must
+ *                  not overlap any input)
+ *   dconv_w      : (dim, W) float32;  dconv_b : (dim) float32, nullable
+ *                  (both summed over batch and time)
+ * The scan backward writes du into dx; a second kernel then applies, in
+ * place, the chain rule through SiLU and the convolution:
+ *     dpre_t = du_t sigmoid(pre_t) (1 + pre_t (1 - sigmoid(pre_t)))
+ *     dx[s] = sum_k conv_w[d,k] dpre_{s+(W-1)-k},
+ *     dconv_w[d,k] = sum_{b,t} dpre_t x_{t-(W-1)+k},  dconv_b[d] = sum_{b,t} dpre_t.
+ * In bf16, du is rounded to bf16 once before that step.  Reductions run in a
+ * fixed order (bitwise reproducible).
+ */
+MAMBA_SCAN_API mamba_status_t mamba_conv_scan_bwd(
+    const void *x, const float *conv_w, const float *conv_b, int64_t conv_width,
+    const void *delta, const float *delta_bias, const float *A, const void *B, const void *C,
+    const float *D, const void *z, const void *dy, void *dx, float *dconv_w, float *dconv_b,
+    void *ddelta, float *dA, void *dB, void *dC, float *dD, void *dz, float *ddelta_bias,
+    int64_t batch, int64_t dim, int64_t L, int64_t N, mamba_dtype_t dtype,
+    const mamba_scan_options_t *options, mamba_stream_t stream);
+
+/*
  * One decoding step: the recurrent mode of the selective SSM, one token per
  * call with constant work per token ("Mamba: Linear-Time Sequence Modeling
  * with Selective State Spaces", trishampatil.com walk-through, Part II

@@ -72,6 +72,9 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_reference_kernel(BwdArgs a, B
   const float bias = a.bias ? a.bias[d] : 0.f;
   const float Dd = a.D ? a.D[d] : 0.f;
   float *ckpt = w.ckpt + ch * w.n_chunks * NM;
+  const bool conv = a.conv_w != nullptr;  // u is x; the scan input is SiLU(conv(x))
+  ConvFilter cf = {0.f, 0.f, 0.f, 1.f, 0.f};
+  if (conv) cf = load_conv_filter(a.conv_w, a.conv_b, a.conv_width, d);
 
   float Av[NM], invA[NM], h[NM];
 #pragma unroll
@@ -88,7 +91,7 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_reference_kernel(BwdArgs a, B
       for (int n = 0; n < NM; ++n) ckpt[(t / kBwdTC) * NM + n] = h[n];
     }
     const float Delta = softplus_acc(to_f(dl[t]) + bias);
-    const float ut = to_f(u[t]);
+    const float ut = conv ? conv_u_acc(cf, u, t) : to_f(u[t]);
 #pragma unroll
     for (int n = 0; n < NM; ++n) {
       if (n < N) {
@@ -115,7 +118,7 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_reference_kernel(BwdArgs a, B
 #pragma unroll
       for (int n = 0; n < NM; ++n) hs[(s * NM + n) * kBwdThreads + tid] = h[n];
       const float Delta = softplus_acc(to_f(dl[t]) + bias);
-      const float ut = to_f(u[t]);
+      const float ut = conv ? conv_u_acc(cf, u, t) : to_f(u[t]);
 #pragma unroll
       for (int n = 0; n < NM; ++n) {
         if (n < N) {
@@ -131,7 +134,7 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_reference_kernel(BwdArgs a, B
       const float v = to_f(dl[t]) + bias;
       const float Delta = softplus_acc(v);
       const float sv = sigmoid_acc(v);
-      const float ut = to_f(u[t]);
+      const float ut = conv ? conv_u_acc(cf, u, t) : to_f(u[t]);
       const float dyt = to_f(dy[t]);
       float dy0 = dyt, zt = 0.f, sz = 0.f;
       if (z) {

@@ -151,7 +151,29 @@ __device__ __forceinline__ float bfly_rest(float (&v)[16], int lane) {
   return v[0];
 }
 
-template <typename T, int NM>
+// Four consecutive x values of a row (16-byte aligned for float, 8-byte for
+// bf16), widened to float.
+__device__ __forceinline__ void load_x4(const float *p, float (&o)[4]) {
+  const float4 v = __ldg(reinterpret_cast<const float4 *>(p));
+  o[0] = v.x;
+  o[1] = v.y;
+  o[2] = v.z;
+  o[3] = v.w;
+}
+__device__ __forceinline__ void load_x4(const __nv_bfloat16 *p, float (&o)[4]) {
+  const uint2 v = __ldg(reinterpret_cast<const uint2 *>(p));
+  o[0] = __uint_as_float(v.x << 16);
+  o[1] = __uint_as_float(v.x & 0xffff0000u);
+  o[2] = __uint_as_float(v.y << 16);
+  o[3] = __uint_as_float(v.y & 0xffff0000u);
+}
+
+// CONV: the u tiles hold the input x of the block's causal depthwise
+// convolution; every read of a segment's u computes SiLU(conv(x)) from the
+// segment's x, the x just before it in the tile, and for the first steps of
+// a tile the four x values before the tile (read from global memory).  du is
+// the gradient with respect to u; the convolution's backward runs after.
+template <typename T, int NM, bool CONV = false>
 __global__ void __launch_bounds__(kSThreads, 2)
     bwd_staged_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_d,
                       const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_dy,
@@ -295,6 +317,10 @@ __global__ void __launch_bounds__(kSThreads, 2)
     }
     float dA[NM];
     float dDsum = 0.f, dbsum = 0.f;
+    ConvFilter cf = {0.f, 0.f, 0.f, 1.f, 0.f};
+    if constexpr (CONV) {
+      if (valid) cf = load_conv_filter(f.conv_w, f.conv_b, f.conv_width, d);
+    }
 
     auto run = [&](auto mode_tag) {
       constexpr int M = decltype(mode_tag)::value;
@@ -353,6 +379,12 @@ __global__ void __launch_bounds__(kSThreads, 2)
 #pragma unroll
           for (int n = 0; n < NM; ++n) h0[n] = __ldcg(ck + n * kSThreads);
         }
+        // convolution prologue: x at the four steps before the tile (0 before
+        // the sequence start and on padding channels)
+        [[maybe_unused]] float hx[4] = {0.f, 0.f, 0.f, 0.f};
+        if constexpr (CONV) {
+          if (valid && t0 > 0) load_x4(static_cast<const T *>(f.u) + row + t0 - 4, hx);
+        }
         if (!mbar_wait_bounded(&bars[stage], parity, p.timeout_ns)) {
           record_timeout();
           q[8] = 1;
@@ -380,6 +412,51 @@ __global__ void __launch_bounds__(kSThreads, 2)
         const unsigned char *sz = st + 2 * Lay::TILE;
         const unsigned char *sdy = st + 3 * Lay::TILE;
 
+        // u of one segment of the tile
+        auto load_u = [&](int seg, float (&uv)[SEG]) {
+          IO::load(su, tid, seg, uv);
+          if constexpr (CONV) {
+            float win[SEG + 3];  // x at the steps seg*SEG-3 .. seg*SEG+SEG-1 of the tile
+            if constexpr (SEG == 2) {
+              float p1[2], p2[2];
+              if (seg >= 1) {
+                IO::load(su, tid, seg - 1, p1);
+              } else {
+                p1[0] = hx[2];
+                p1[1] = hx[3];
+              }
+              if (seg >= 2) {
+                IO::load(su, tid, seg - 2, p2);
+              } else {
+                p2[0] = seg == 1 ? hx[2] : hx[0];
+                p2[1] = seg == 1 ? hx[3] : hx[1];
+              }
+              win[0] = p2[1];
+              win[1] = p1[0];
+              win[2] = p1[1];
+            } else {
+              static_assert(SEG == 4, "segments of 2 or 4 steps");
+              float p1[4];
+              if (seg >= 1) {
+                IO::load(su, tid, seg - 1, p1);
+              } else {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) p1[i] = hx[i];
+              }
+              win[0] = p1[1];
+              win[1] = p1[2];
+              win[2] = p1[3];
+            }
+#pragma unroll
+            for (int i = 0; i < SEG; ++i) win[3 + i] = uv[i];
+#pragma unroll
+            for (int i = 0; i < SEG; ++i) {
+              const float pre = conv_pre(cf, win[i], win[i + 1], win[i + 2], win[i + 3]);
+              uv[i] = pre * rcpf(1.f + ex2f(-pre * kLog2e));
+            }
+          }
+        };
+
         // forward over the tile: the state before every segment -> shared memory
         {
           f2 H[NP];
@@ -405,7 +482,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
             }
             if (seg == nseg - 1) break;  // the last segment is re-run below anyway
             float uv[SEG], dv[SEG];
-            IO::load(su, tid, seg, uv);
+            load_u(seg, uv);
             IO::load(sd, tid, seg, dv);
 #pragma unroll
             for (int i = 0; i < SEG; ++i) {
@@ -426,7 +503,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
         // segments from the last: re-run into registers, then walk backwards
         for (int seg = nseg - 1; seg >= 0; --seg) {
           float uv[SEG], dv[SEG], zv[SEG], dyv[SEG];
-          IO::load(su, tid, seg, uv);
+          load_u(seg, uv);
           IO::load(sd, tid, seg, dv);
           IO::load(sdy, tid, seg, dyv);
           if (has_z) IO::load(sz, tid, seg, zv);
@@ -705,7 +782,7 @@ inline bool staged_bwd_supported(const BwdArgs &a, size_t es) {
          al(a.ddelta) && al(a.dz);
 }
 
-template <typename T, int NM>
+template <typename T, int NM, bool CONV = false>
 mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStream_t s,
                                mamba_status_t (*launched)()) {
   using Lay = BwdLayout<T, NM>;
@@ -722,7 +799,7 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
       !make_map_3d(&maps[5], a.C, bf16, L, N, batch, kBTT, uint32_t(N), none)) {
     return MAMBA_ERR_UNSUPPORTED;
   }
-  auto kern = bwd_staged_kernel<T, NM>;
+  auto kern = bwd_staged_kernel<T, NM, CONV>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::ALLOC) != cudaSuccess)
     return MAMBA_ERR_CUDA;
   int bps = 0;
@@ -780,11 +857,12 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
     fa.u = a.u; fa.delta = a.delta; fa.z = nullptr; fa.B = a.B; fa.C = a.C;
     fa.bias = a.bias; fa.A = a.A; fa.D = nullptr; fa.y = nullptr; fa.last_state = nullptr;
     fa.batch = a.batch; fa.dim = a.dim; fa.L = a.L; fa.N = a.N;
+    fa.conv_w = a.conv_w; fa.conv_b = a.conv_b; fa.conv_width = a.conv_width;
     StagedOptions fo = o;
     fo.chunk_len = 0;
     fo.carry = 0;
     fo.test_hook = 0;  // the hook targets the reverse hand-off
-    st = staged_forward<T, NM>(fa, fo, s, launched, ckpt);
+    st = staged_forward<T, NM, CONV>(fa, fo, s, launched, ckpt);
   }
   if (st == MAMBA_OK) {
     kern<<<unsigned(std::min<int64_t>(gk, slots)), kSThreads, Lay::ALLOC, s>>>(

@@ -17,6 +17,9 @@ constexpr int kMaxN = 16;
 __device__ unsigned int g_error_word = 0;
 constexpr unsigned int kErrTimeout = 1u;
 
+// With conv_w set, `u` points at the input x of the Mamba block's causal
+// depthwise convolution, and the scan runs on u = SiLU(conv(x)) computed on
+// the fly (see ConvFilter); conv_w is (dim, conv_width), conv_b (dim) or null.
 struct FwdArgs {
   const void *u, *delta, *z, *B, *C;
   const float *bias, *A, *D;
@@ -24,8 +27,12 @@ struct FwdArgs {
   float *last_state;
   int64_t batch, dim, L;
   int N;
+  const float *conv_w = nullptr, *conv_b = nullptr;
+  int conv_width = 0;
 };
 
+// With conv_w set, `u` is x as in FwdArgs and `du` receives the gradient with
+// respect to u = SiLU(conv(x)); the convolution's own backward runs after.
 struct BwdArgs {
   const void *u, *delta, *z, *B, *C, *dy;
   const float *bias, *A, *D;
@@ -33,7 +40,37 @@ struct BwdArgs {
   float *dA, *dD, *dbias;
   int64_t batch, dim, L;
   int N;
+  const float *conv_w = nullptr, *conv_b = nullptr;
+  int conv_width = 0;
 };
+
+// The short causal depthwise convolution in front of the S6 layer (Knowl 3
+// "Mamba Block Architecture", step 3, chapterpal.com page: width d_conv = 4,
+// then SiLU), for widths W <= 4: the filter is held right-aligned, w3 on the
+// current step and w0 on the step three back, so that
+//     pre_t = b + w0 x_{t-3} + w1 x_{t-2} + w2 x_{t-1} + w3 x_t
+// with x = 0 before the first step, and u_t = pre_t sigmoid(pre_t).
+constexpr int kMaxConvWidth = 4;
+struct ConvFilter {
+  float w0, w1, w2, w3, b;
+};
+
+__device__ __forceinline__ ConvFilter load_conv_filter(const float *conv_w, const float *conv_b,
+                                                       int W, int64_t d) {
+  const float *r = conv_w + d * W;
+  ConvFilter c;
+  c.w3 = r[W - 1];
+  c.w2 = W >= 2 ? r[W - 2] : 0.f;
+  c.w1 = W >= 3 ? r[W - 3] : 0.f;
+  c.w0 = W >= 4 ? r[W - 4] : 0.f;
+  c.b = conv_b ? conv_b[d] : 0.f;
+  return c;
+}
+
+__device__ __forceinline__ float conv_pre(const ConvFilter &c, float xm3, float xm2, float xm1,
+                                          float x0) {
+  return fmaf(c.w0, xm3, fmaf(c.w1, xm2, fmaf(c.w2, xm1, fmaf(c.w3, x0, c.b))));
+}
 
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
@@ -51,6 +88,18 @@ __device__ __forceinline__ float softplus_acc(float v) {
 }
 
 __device__ __forceinline__ float sigmoid_acc(float v) { return 1.f / (1.f + expf(-v)); }
+
+// u_t of the convolution prologue at step t of the row x (I/O type), with
+// CUDA's accurate expf: the plain form used by the one-thread-per-channel
+// kernels.
+template <typename T>
+__device__ __forceinline__ float conv_u_acc(const ConvFilter &c, const T *x, int64_t t) {
+  const float xm3 = t >= 3 ? to_f(x[t - 3]) : 0.f;
+  const float xm2 = t >= 2 ? to_f(x[t - 2]) : 0.f;
+  const float xm1 = t >= 1 ? to_f(x[t - 1]) : 0.f;
+  const float p = conv_pre(c, xm3, xm2, xm1, to_f(x[t]));
+  return p * sigmoid_acc(p);
+}
 
 // (x e^x - expm1(x)) / x^2, the derivative of expm1(x)/x.  Taylor series
 // sum_k (k+1)/(k+2)! x^k near zero, where the closed form cancels.

@@ -6,7 +6,8 @@
 // chapterpal.com): discretize with zero-order hold, update the state, read it
 // out with C_t; plus softplus on Delta, the D skip and the SiLU gate.  It is
 // the path for shapes the staged kernels do not take (rows that are not
-// 16-byte multiples) and the slow-but-simple GPU comparison point.
+// 16-byte multiples) and the slow-but-simple GPU comparison point.  With a
+// convolution filter in the arguments, u is computed from x at every step.
 #pragma once
 #include "common.cuh"
 
@@ -29,6 +30,9 @@ __global__ void __launch_bounds__(kRefThreads) fwd_reference_kernel(FwdArgs a) {
   T *y = static_cast<T *>(a.y) + ch * L;
   const float bias = a.bias ? a.bias[d] : 0.f;
   const float Dd = a.D ? a.D[d] : 0.f;
+  const bool conv = a.conv_w != nullptr;  // u is x; the scan input is SiLU(conv(x))
+  ConvFilter cf = {0.f, 0.f, 0.f, 1.f, 0.f};
+  if (conv) cf = load_conv_filter(a.conv_w, a.conv_b, a.conv_width, d);
 
   float Av[NM], invA[NM], h[NM];
 #pragma unroll
@@ -39,7 +43,7 @@ __global__ void __launch_bounds__(kRefThreads) fwd_reference_kernel(FwdArgs a) {
   }
   for (int64_t t = 0; t < L; ++t) {
     const float Delta = softplus_acc(to_f(dl[t]) + bias);
-    const float ut = to_f(u[t]);
+    const float ut = conv ? conv_u_acc(cf, u, t) : to_f(u[t]);
     float y0 = 0.f;
 #pragma unroll
     for (int n = 0; n < NM; ++n) {

@@ -287,7 +287,11 @@ struct StagedLayout {
   static constexpr int ALLOC = BYTES + 1024;  // slack to align the base to 1 KB
 };
 
-template <typename T, int NM, int KIND>
+// CONV: the u tiles hold the input x of the block's causal depthwise
+// convolution, and each thread turns its row into u = SiLU(conv(x)) as it
+// reads it (the three inputs before the unit's first step come from global
+// memory; after that the last three stay in registers).
+template <typename T, int NM, int KIND, bool CONV = false>
 __global__ void __launch_bounds__(kSThreads, 2)
     fwd_staged_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_d,
                       const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_y,
@@ -447,6 +451,21 @@ __global__ void __launch_bounds__(kSThreads, 2)
 
     double Ssum = 0.0;  // sum of Delta over the chunk (aggregate pass)
 
+    // convolution prologue: the filter and x at the three steps before the chunk
+    ConvFilter cf = {0.f, 0.f, 0.f, 1.f, 0.f};
+    float xm1 = 0.f, xm2 = 0.f, xm3 = 0.f;
+    if constexpr (CONV) {
+      if (valid) {
+        cf = load_conv_filter(f.conv_w, f.conv_b, f.conv_width, d);
+        if (tbeg > 0) {  // chunks start at multiples of 64 steps
+          const T *xr = static_cast<const T *>(f.u) + (int64_t(b) * f.dim + d) * f.L + tbeg;
+          xm3 = to_f(xr[-3]);
+          xm2 = to_f(xr[-2]);
+          xm1 = to_f(xr[-1]);
+        }
+      }
+    }
+
     // Runs every tile of this unit with the arithmetic of mode M.
     auto run = [&](auto mode_tag) {
       constexpr int M = decltype(mode_tag)::value;
@@ -531,6 +550,17 @@ __global__ void __launch_bounds__(kSThreads, 2)
           const int off = swz64(tid, j);
           float uv[VEC], dv[VEC], zv[VEC], yv[VEC];
           Vec<T>::unpack(*reinterpret_cast<const uint4 *>(su + off), uv);
+          if constexpr (CONV) {  // x -> u = SiLU(conv(x)), in time order
+#pragma unroll
+            for (int i = 0; i < VEC; ++i) {
+              const float xv = uv[i];
+              const float pre = conv_pre(cf, xm3, xm2, xm1, xv);
+              uv[i] = pre * rcpf(1.f + ex2f(-pre * kLog2e));
+              xm3 = xm2;
+              xm2 = xm1;
+              xm1 = xv;
+            }
+          }
           Vec<T>::unpack(*reinterpret_cast<const uint4 *>(sd + off), dv);
           if (has_z) Vec<T>::unpack(*reinterpret_cast<const uint4 *>(sz + off), zv);
 #pragma unroll
@@ -693,18 +723,18 @@ inline bool staged_supported(const FwdArgs &a, size_t es) {
   return al(a.u) && al(a.delta) && al(a.z) && al(a.y) && al(a.B) && al(a.C);
 }
 
-template <typename T, int NM, int KIND>
+template <typename T, int NM, int KIND, bool CONV = false>
 inline cudaError_t prepare_kernel(int *blocks_per_sm) {
-  auto kern = fwd_staged_kernel<T, NM, KIND>;
+  auto kern = fwd_staged_kernel<T, NM, KIND, CONV>;
   const int bytes = StagedLayout<T, NM>::ALLOC;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return e;
   return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, kern, kSThreads, bytes);
 }
 
-template <typename T, int NM, int KIND>
+template <typename T, int NM, int KIND, bool CONV = false>
 inline void launch_staged(const CUtensorMap (&maps)[6], const StagedArgs &sa, int grid, cudaStream_t s) {
-  fwd_staged_kernel<T, NM, KIND><<<grid, kSThreads, StagedLayout<T, NM>::ALLOC, s>>>(
+  fwd_staged_kernel<T, NM, KIND, CONV><<<grid, kSThreads, StagedLayout<T, NM>::ALLOC, s>>>(
       maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], sa);
 }
 
@@ -743,7 +773,8 @@ inline StagedPlan plan_staged(int64_t G, int64_t L, int slots, const StagedOptio
 // tensor map.
 // With `ckpt` non-null the forward runs without y and stores the state before
 // every kCkptEvery-th step into ckpt ([G][ceil(L/16)][NM][128] floats).
-template <typename T, int NM>
+// CONV selects the kernels with the convolution prologue (a.conv_w set).
+template <typename T, int NM, bool CONV = false>
 mamba_status_t staged_forward(const FwdArgs &a, const StagedOptions &o, cudaStream_t s,
                               mamba_status_t (*launched)(), float *ckpt = nullptr) {
   using Lay = StagedLayout<T, NM>;
@@ -760,7 +791,7 @@ mamba_status_t staged_forward(const FwdArgs &a, const StagedOptions &o, cudaStre
     return MAMBA_ERR_UNSUPPORTED;
   }
   int bps_main = 0;
-  if (prepare_kernel<T, NM, KIND_SEQ>(&bps_main) != cudaSuccess) return MAMBA_ERR_CUDA;
+  if (prepare_kernel<T, NM, KIND_SEQ, CONV>(&bps_main) != cudaSuccess) return MAMBA_ERR_CUDA;
   const int sms = device_sm_count();
   const int slots = sms * std::max(1, bps_main);
   const int64_t gpb = ceil_div(a.dim, kSThreads);
@@ -809,10 +840,10 @@ mamba_status_t staged_forward(const FwdArgs &a, const StagedOptions &o, cudaStre
     const int grid = int(std::min<int64_t>(gk, slots));
     if (ckpt) {
       int bps = 0;
-      if (prepare_kernel<T, NM, KIND_CKPT_SEQ>(&bps) != cudaSuccess) st = MAMBA_ERR_CUDA;
-      else launch_staged<T, NM, KIND_CKPT_SEQ>(maps, sa, int(std::min<int64_t>(gk, sms * std::max(1, bps))), s);
+      if (prepare_kernel<T, NM, KIND_CKPT_SEQ, CONV>(&bps) != cudaSuccess) st = MAMBA_ERR_CUDA;
+      else launch_staged<T, NM, KIND_CKPT_SEQ, CONV>(maps, sa, int(std::min<int64_t>(gk, sms * std::max(1, bps))), s);
     } else {
-      launch_staged<T, NM, KIND_SEQ>(maps, sa, grid, s);
+      launch_staged<T, NM, KIND_SEQ, CONV>(maps, sa, grid, s);
     }
     if (st == MAMBA_OK) st = launched();
   } else if (st == MAMBA_OK) {
@@ -820,16 +851,16 @@ mamba_status_t staged_forward(const FwdArgs &a, const StagedOptions &o, cudaStre
     sa.agg_h = reinterpret_cast<float *>(ws + int_bytes + gk * kSThreads * 8);
     sa.hin = sa.agg_h + gk * NM * kSThreads;
     int bps_agg = 0, bps_par = 0;
-    if (prepare_kernel<T, NM, KIND_AGG>(&bps_agg) != cudaSuccess ||
-        (ckpt ? prepare_kernel<T, NM, KIND_CKPT_PAR>(&bps_par)
-              : prepare_kernel<T, NM, KIND_PAR>(&bps_par)) != cudaSuccess) {
+    if (prepare_kernel<T, NM, KIND_AGG, CONV>(&bps_agg) != cudaSuccess ||
+        (ckpt ? prepare_kernel<T, NM, KIND_CKPT_PAR, CONV>(&bps_par)
+              : prepare_kernel<T, NM, KIND_PAR, CONV>(&bps_par)) != cudaSuccess) {
       st = MAMBA_ERR_CUDA;
     }
     if (st == MAMBA_OK) {
       StagedArgs sg = sa;
       sg.counter = counters;
       sg.n_units = int(size_t(G) * size_t(pl.K - 1));
-      launch_staged<T, NM, KIND_AGG>(maps, sg, int(std::min<int64_t>(sg.n_units, sms * std::max(1, bps_agg))), s);
+      launch_staged<T, NM, KIND_AGG, CONV>(maps, sg, int(std::min<int64_t>(sg.n_units, sms * std::max(1, bps_agg))), s);
       st = launched();
     }
     if (st == MAMBA_OK) {
@@ -842,8 +873,8 @@ mamba_status_t staged_forward(const FwdArgs &a, const StagedOptions &o, cudaStre
       sm.counter = counters + 1;
       sm.n_units = int(gk);
       const int grid = int(std::min<int64_t>(gk, sms * std::max(1, bps_par)));
-      if (ckpt) launch_staged<T, NM, KIND_CKPT_PAR>(maps, sm, grid, s);
-      else launch_staged<T, NM, KIND_PAR>(maps, sm, grid, s);
+      if (ckpt) launch_staged<T, NM, KIND_CKPT_PAR, CONV>(maps, sm, grid, s);
+      else launch_staged<T, NM, KIND_PAR, CONV>(maps, sm, grid, s);
       st = launched();
     }
   }

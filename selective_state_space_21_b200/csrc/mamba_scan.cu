@@ -13,6 +13,7 @@
 #include "bwd_reference.cuh"
 #include "bwd_staged.cuh"
 #include "common.cuh"
+#include "conv_bwd.cuh"
 #include "decode.cuh"
 #include "fwd_reference.cuh"
 #include "fwd_staged.cuh"
@@ -157,18 +158,18 @@ struct FwdReferenceLauncher {
   }
 };
 
-template <typename T>
+template <typename T, bool CONV>
 mamba_status_t staged_bwd_dispatch(const BwdArgs &a, const StagedOptions &o, cudaStream_t s) {
-  if (a.N <= 4) return staged_backward<T, 4>(a, o, s, &launch_status);
-  if (a.N <= 8) return staged_backward<T, 8>(a, o, s, &launch_status);
-  return staged_backward<T, 16>(a, o, s, &launch_status);
+  if (a.N <= 4) return staged_backward<T, 4, CONV>(a, o, s, &launch_status);
+  if (a.N <= 8) return staged_backward<T, 8, CONV>(a, o, s, &launch_status);
+  return staged_backward<T, 16, CONV>(a, o, s, &launch_status);
 }
 
-template <typename T>
+template <typename T, bool CONV>
 mamba_status_t staged_dispatch(const FwdArgs &a, const StagedOptions &o, cudaStream_t s) {
-  if (a.N <= 4) return staged_forward<T, 4>(a, o, s, &launch_status);
-  if (a.N <= 8) return staged_forward<T, 8>(a, o, s, &launch_status);
-  return staged_forward<T, 16>(a, o, s, &launch_status);
+  if (a.N <= 4) return staged_forward<T, 4, CONV>(a, o, s, &launch_status);
+  if (a.N <= 8) return staged_forward<T, 8, CONV>(a, o, s, &launch_status);
+  return staged_forward<T, 16, CONV>(a, o, s, &launch_status);
 }
 
 template <typename T, int NM>
@@ -219,6 +220,47 @@ struct BwdReferenceLauncher {
     return st;
   }
 };
+
+StagedOptions staged_options(const mamba_scan_options_t *options) {
+  StagedOptions so;
+  so.path = options ? options->path : MAMBA_PATH_AUTO;
+  so.chunk_len = options ? options->chunk_len : 0;
+  so.carry = options ? options->carry : 0;
+  so.timeout_us = options ? options->wait_timeout_us : 0;
+  so.test_hook = options ? options->test_hook : 0;
+  return so;
+}
+
+// Kernel choice of the forward: the staged kernels where they apply (CONV:
+// their convolution-prologue instances), else the one-thread-per-channel
+// kernel (which handles the prologue at run time).
+template <bool CONV>
+mamba_status_t forward_paths(const FwdArgs &a, size_t es, mamba_dtype_t dtype,
+                             const StagedOptions &so, cudaStream_t s) {
+  const bool stageable = staged_supported(a, es);
+  if (so.path == MAMBA_PATH_REFERENCE || (!stageable && so.path == MAMBA_PATH_AUTO))
+    return dispatch<FwdReferenceLauncher>(dtype, a.N, a, s);
+  if (!stageable) return MAMBA_ERR_UNSUPPORTED;
+  const mamba_status_t st = dtype == MAMBA_BF16 ? staged_dispatch<__nv_bfloat16, CONV>(a, so, s)
+                                                : staged_dispatch<float, CONV>(a, so, s);
+  if (st == MAMBA_ERR_UNSUPPORTED && so.path == MAMBA_PATH_AUTO)
+    return dispatch<FwdReferenceLauncher>(dtype, a.N, a, s);
+  return st;
+}
+
+template <bool CONV>
+mamba_status_t backward_paths(const BwdArgs &a, size_t es, mamba_dtype_t dtype,
+                              const StagedOptions &so, cudaStream_t s) {
+  const bool stageable = staged_bwd_supported(a, es);
+  if (so.path == MAMBA_PATH_REFERENCE || (!stageable && so.path == MAMBA_PATH_AUTO))
+    return dispatch<BwdReferenceLauncher>(dtype, a.N, a, s);
+  if (!stageable) return MAMBA_ERR_UNSUPPORTED;
+  const mamba_status_t st = dtype == MAMBA_BF16 ? staged_bwd_dispatch<__nv_bfloat16, CONV>(a, so, s)
+                                                : staged_bwd_dispatch<float, CONV>(a, so, s);
+  if (st == MAMBA_ERR_UNSUPPORTED && so.path == MAMBA_PATH_AUTO)
+    return dispatch<BwdReferenceLauncher>(dtype, a.N, a, s);
+  return st;
+}
 
 }  // namespace
 
@@ -292,20 +334,7 @@ mamba_status_t mamba_scan_fwd_ex(const void *u, const void *delta, const float *
   a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
   a.bias = delta_bias; a.A = A; a.D = D; a.y = y; a.last_state = last_state;
   a.batch = batch; a.dim = dim; a.L = L; a.N = (int)N;
-  StagedOptions so;
-  so.path = options ? options->path : MAMBA_PATH_AUTO;
-  so.chunk_len = options ? options->chunk_len : 0;
-  so.carry = options ? options->carry : 0;
-  so.timeout_us = options ? options->wait_timeout_us : 0;
-  so.test_hook = options ? options->test_hook : 0;
-  const bool stageable = staged_supported(a, es);
-  if (so.path == MAMBA_PATH_REFERENCE || (!stageable && so.path == MAMBA_PATH_AUTO))
-    return dispatch<FwdReferenceLauncher>(dtype, (int)N, a, s);
-  if (!stageable) return MAMBA_ERR_UNSUPPORTED;
-  st = dtype == MAMBA_BF16 ? staged_dispatch<__nv_bfloat16>(a, so, s) : staged_dispatch<float>(a, so, s);
-  if (st == MAMBA_ERR_UNSUPPORTED && so.path == MAMBA_PATH_AUTO)
-    return dispatch<FwdReferenceLauncher>(dtype, (int)N, a, s);
-  return st;
+  return forward_paths<false>(a, es, dtype, staged_options(options), s);
 }
 
 mamba_status_t mamba_scan_fwd(const void *u, const void *delta, const float *delta_bias,
@@ -372,21 +401,7 @@ mamba_status_t mamba_scan_bwd_ex(const void *u, const void *delta, const float *
   a.du = du; a.ddelta = ddelta; a.dz = dz; a.dB = dB; a.dC = dC;
   a.dA = dA; a.dD = dD; a.dbias = ddelta_bias;
   a.batch = batch; a.dim = dim; a.L = L; a.N = (int)N;
-  StagedOptions so;
-  so.path = options ? options->path : MAMBA_PATH_AUTO;
-  so.chunk_len = options ? options->chunk_len : 0;
-  so.carry = options ? options->carry : 0;
-  so.timeout_us = options ? options->wait_timeout_us : 0;
-  so.test_hook = options ? options->test_hook : 0;
-  const bool stageable = staged_bwd_supported(a, es);
-  if (so.path == MAMBA_PATH_REFERENCE || (!stageable && so.path == MAMBA_PATH_AUTO))
-    return dispatch<BwdReferenceLauncher>(dtype, (int)N, a, s);
-  if (!stageable) return MAMBA_ERR_UNSUPPORTED;
-  st = dtype == MAMBA_BF16 ? staged_bwd_dispatch<__nv_bfloat16>(a, so, s)
-                           : staged_bwd_dispatch<float>(a, so, s);
-  if (st == MAMBA_ERR_UNSUPPORTED && so.path == MAMBA_PATH_AUTO)
-    return dispatch<BwdReferenceLauncher>(dtype, (int)N, a, s);
-  return st;
+  return backward_paths<false>(a, es, dtype, staged_options(options), s);
 }
 
 mamba_status_t mamba_scan_step(float *state, const void *u, const void *delta,
@@ -468,6 +483,155 @@ mamba_status_t mamba_scan_bwd(const void *u, const void *delta, const float *del
                               mamba_dtype_t dtype, mamba_stream_t stream) {
   return mamba_scan_bwd_ex(u, delta, delta_bias, A, B, C, D, z, dy, du, ddelta, dA, dB, dC, dD,
                            dz, ddelta_bias, batch, dim, L, N, dtype, nullptr, stream);
+}
+
+// ------------------------------------------------ convolution prologue
+
+mamba_status_t mamba_conv_scan_fwd(const void *x, const float *conv_w, const float *conv_b,
+                                   int64_t conv_width, const void *delta,
+                                   const float *delta_bias, const float *A, const void *B,
+                                   const void *C, const float *D, const void *z, void *y,
+                                   float *last_state, int64_t batch, int64_t dim, int64_t L,
+                                   int64_t N, mamba_dtype_t dtype,
+                                   const mamba_scan_options_t *options, mamba_stream_t stream) {
+  mamba_status_t st = check_shape(batch, dim, L, N, dtype);
+  if (st != MAMBA_OK) return st;
+  if ((st = check_options(options)) != MAMBA_OK) return st;
+  if (conv_width < 1 || conv_width > kMaxConvWidth) return MAMBA_ERR_UNSUPPORTED;
+  Checker ck;
+  if (cudaGetDevice(&ck.dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MAMBA_ERR_CUDA;
+  }
+  const size_t es = dtype_size(dtype);
+  const size_t nbdl = size_t(batch) * size_t(dim) * size_t(L);
+  const size_t nbnl = size_t(batch) * size_t(N) * size_t(L);
+  ck.buf(x, nbdl * es, es, true, false);
+  ck.buf(conv_w, size_t(dim) * size_t(conv_width) * 4, 4, true, false);
+  ck.buf(conv_b, size_t(dim) * 4, 4, false, false);
+  ck.buf(delta, nbdl * es, es, true, false);
+  ck.buf(z, nbdl * es, es, false, false);
+  ck.buf(B, nbnl * es, es, true, false);
+  ck.buf(C, nbnl * es, es, true, false);
+  ck.buf(A, size_t(dim) * N * 4, 4, true, false);
+  ck.buf(D, size_t(dim) * 4, 4, false, false);
+  ck.buf(delta_bias, size_t(dim) * 4, 4, false, false);
+  ck.buf(y, nbdl * es, es, true, true);
+  ck.buf(last_state, size_t(batch) * dim * N * 4, 4, false, true);
+  if (ck.st != MAMBA_OK) return ck.st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (batch == 0 || dim == 0) return MAMBA_OK;
+  if (L == 0) {
+    if (last_state && cudaMemsetAsync(last_state, 0, size_t(batch) * dim * N * 4, s) != cudaSuccess)
+      return cuda_status();
+    return MAMBA_OK;
+  }
+  FwdArgs a;
+  a.u = x; a.delta = delta; a.z = z; a.B = B; a.C = C;
+  a.bias = delta_bias; a.A = A; a.D = D; a.y = y; a.last_state = last_state;
+  a.batch = batch; a.dim = dim; a.L = L; a.N = (int)N;
+  a.conv_w = conv_w; a.conv_b = conv_b; a.conv_width = (int)conv_width;
+  return forward_paths<true>(a, es, dtype, staged_options(options), s);
+}
+
+mamba_status_t mamba_conv_scan_bwd(const void *x, const float *conv_w, const float *conv_b,
+                                   int64_t conv_width, const void *delta,
+                                   const float *delta_bias, const float *A, const void *B,
+                                   const void *C, const float *D, const void *z, const void *dy,
+                                   void *dx, float *dconv_w, float *dconv_b, void *ddelta,
+                                   float *dA, void *dB, void *dC, float *dD, void *dz,
+                                   float *ddelta_bias, int64_t batch, int64_t dim, int64_t L,
+                                   int64_t N, mamba_dtype_t dtype,
+                                   const mamba_scan_options_t *options, mamba_stream_t stream) {
+  mamba_status_t st = check_shape(batch, dim, L, N, dtype);
+  if (st != MAMBA_OK) return st;
+  if ((st = check_options(options)) != MAMBA_OK) return st;
+  if (conv_width < 1 || conv_width > kMaxConvWidth) return MAMBA_ERR_UNSUPPORTED;
+  if ((z == nullptr) != (dz == nullptr) || (D == nullptr) != (dD == nullptr))
+    return MAMBA_ERR_INVALID_ARG;
+  Checker ck;
+  if (cudaGetDevice(&ck.dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MAMBA_ERR_CUDA;
+  }
+  const size_t es = dtype_size(dtype);
+  const size_t nbdl = size_t(batch) * size_t(dim) * size_t(L);
+  const size_t nbnl = size_t(batch) * size_t(N) * size_t(L);
+  const size_t nw = size_t(dim) * size_t(conv_width) * 4;
+  ck.buf(x, nbdl * es, es, true, false);
+  ck.buf(conv_w, nw, 4, true, false);
+  ck.buf(conv_b, size_t(dim) * 4, 4, false, false);
+  ck.buf(delta, nbdl * es, es, true, false);
+  ck.buf(z, nbdl * es, es, false, false);
+  ck.buf(dy, nbdl * es, es, true, false);
+  ck.buf(B, nbnl * es, es, true, false);
+  ck.buf(C, nbnl * es, es, true, false);
+  ck.buf(A, size_t(dim) * N * 4, 4, true, false);
+  ck.buf(D, size_t(dim) * 4, 4, false, false);
+  ck.buf(delta_bias, size_t(dim) * 4, 4, false, false);
+  ck.buf(dx, nbdl * es, es, true, true);
+  ck.buf(dconv_w, nw, 4, true, true);
+  ck.buf(dconv_b, size_t(dim) * 4, 4, false, true);
+  ck.buf(ddelta, nbdl * es, es, true, true);
+  ck.buf(dz, nbdl * es, es, false, true);
+  ck.buf(dB, nbnl * es, es, true, true);
+  ck.buf(dC, nbnl * es, es, true, true);
+  ck.buf(dA, size_t(dim) * N * 4, 4, true, true);
+  ck.buf(dD, size_t(dim) * 4, 4, false, true);
+  ck.buf(ddelta_bias, size_t(dim) * 4, 4, false, true);
+  if (ck.st != MAMBA_OK) return ck.st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (dim == 0) return MAMBA_OK;
+  if (batch == 0 || L == 0) {  // empty sums
+    if (cudaMemsetAsync(dA, 0, size_t(dim) * N * 4, s) != cudaSuccess ||
+        cudaMemsetAsync(dconv_w, 0, nw, s) != cudaSuccess ||
+        (dconv_b && cudaMemsetAsync(dconv_b, 0, size_t(dim) * 4, s) != cudaSuccess) ||
+        (dD && cudaMemsetAsync(dD, 0, size_t(dim) * 4, s) != cudaSuccess) ||
+        (ddelta_bias && cudaMemsetAsync(ddelta_bias, 0, size_t(dim) * 4, s) != cudaSuccess))
+      return cuda_status();
+    return MAMBA_OK;
+  }
+  const int64_t rows = batch * dim;
+  const int64_t conv_grid = (rows + kConvWarps - 1) / kConvWarps;
+  if (conv_grid > (int64_t(1) << 31) - 1) return MAMBA_ERR_UNSUPPORTED;
+  // 1. the scan backward with the prologue recomputed; the gradient with
+  //    respect to u lands in dx
+  BwdArgs a;
+  a.u = x; a.delta = delta; a.z = z; a.B = B; a.C = C; a.dy = dy;
+  a.bias = delta_bias; a.A = A; a.D = D;
+  a.du = dx; a.ddelta = ddelta; a.dz = dz; a.dB = dB; a.dC = dC;
+  a.dA = dA; a.dD = dD; a.dbias = ddelta_bias;
+  a.batch = batch; a.dim = dim; a.L = L; a.N = (int)N;
+  a.conv_w = conv_w; a.conv_b = conv_b; a.conv_width = (int)conv_width;
+  if ((st = backward_paths<true>(a, es, dtype, staged_options(options), s)) != MAMBA_OK) return st;
+  // 2. through SiLU and the convolution, in place on dx, then the filter sums
+  float *part = nullptr;
+  if (ws_alloc(reinterpret_cast<void **>(&part), size_t(rows) * 5 * 4, s) != cudaSuccess) {
+    cudaGetLastError();
+    return MAMBA_ERR_OUT_OF_MEMORY;
+  }
+  const bool vec = (size_t(L) * es) % 16 == 0 &&
+                   ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(dx)) & 15) == 0;
+  const int W = (int)conv_width;
+#define MSCAN_CONV_BWD(TT, VV)                                                               \
+  conv_bwd_kernel<TT, VV><<<unsigned(conv_grid), 32 * kConvWarps, 0, s>>>(                    \
+      static_cast<const TT *>(x), static_cast<TT *>(dx), conv_w, conv_b, W, rows, dim, L, part)
+  if (dtype == MAMBA_BF16) {
+    if (vec) MSCAN_CONV_BWD(__nv_bfloat16, true);
+    else MSCAN_CONV_BWD(__nv_bfloat16, false);
+  } else {
+    if (vec) MSCAN_CONV_BWD(float, true);
+    else MSCAN_CONV_BWD(float, false);
+  }
+#undef MSCAN_CONV_BWD
+  st = launch_status();
+  if (st == MAMBA_OK) {
+    const int64_t g = std::min<int64_t>((dim + 255) / 256, 148 * 8);
+    conv_bwd_finalize<<<unsigned(g), 256, 0, s>>>(part, batch, dim, W, dconv_w, dconv_b);
+    st = launch_status();
+  }
+  if (ws_free(part, s) != cudaSuccess && st == MAMBA_OK) st = MAMBA_ERR_CUDA;
+  return st;
 }
 
 }  // extern "C"

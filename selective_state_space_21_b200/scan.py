@@ -3,9 +3,11 @@ step of the selective scan runs in the library's CUDA kernels.  There is no
 CPU fallback; a missing library or device raises.
 
 Low-level calls (same names and argument order as ``include/mamba_scan.h``):
-``mamba_scan_fwd``, ``mamba_scan_bwd``, ``mamba_scan_stream_status``.
-Convenience wrappers that allocate the outputs: ``selective_scan_fwd`` and
-``selective_scan_bwd``.
+``mamba_scan_fwd``, ``mamba_scan_bwd``, ``mamba_conv_scan_fwd``,
+``mamba_conv_scan_bwd``, ``mamba_scan_step``, ``mamba_scan_fwd_noalloc``,
+``mamba_scan_stream_status``.  Convenience wrappers that allocate the outputs:
+``selective_scan_fwd``, ``selective_scan_bwd``, ``conv_selective_scan_fwd``
+and ``conv_selective_scan_bwd``.
 """
 from __future__ import annotations
 
@@ -65,6 +67,10 @@ def load_library():
             lib.mamba_scan_fwd_noalloc.argtypes = [vp] * 10 + [i64] * 4 + [i32, vp]
             lib.mamba_scan_step.argtypes = [vp] * 10 + [i64] * 3 + [i32, vp]
             lib.mamba_scan_step.restype = ctypes.c_int
+            lib.mamba_conv_scan_fwd.argtypes = [vp] * 3 + [i64] + [vp] * 9 + [i64] * 4 + [i32, opt, vp]
+            lib.mamba_conv_scan_fwd.restype = ctypes.c_int
+            lib.mamba_conv_scan_bwd.argtypes = [vp] * 3 + [i64] + [vp] * 18 + [i64] * 4 + [i32, opt, vp]
+            lib.mamba_conv_scan_bwd.restype = ctypes.c_int
             for f in ("mamba_scan_fwd", "mamba_scan_fwd_ex", "mamba_scan_bwd",
                       "mamba_scan_bwd_ex", "mamba_scan_stream_status", "mamba_scan_fwd_noalloc"):
                 getattr(lib, f).restype = ctypes.c_int
@@ -179,6 +185,65 @@ def mamba_scan_bwd(u, delta, delta_bias, A, B, C, D, z, dy, du, ddelta, dA, dB, 
     _check(rc, "mamba_scan_bwd")
 
 
+def _opts_ptr(path, chunk_len, carry, wait_timeout_us, test_hook):
+    if path == "auto" and not chunk_len and carry == "auto" and not wait_timeout_us \
+            and not test_hook:
+        return None
+    return ctypes.byref(_options(path, chunk_len, carry, wait_timeout_us, test_hook))
+
+
+def mamba_conv_scan_fwd(x, conv_w, conv_b, delta, delta_bias, A, B, C, D, z, y, last_state, *,
+                        path="auto", chunk_len=0, carry="auto", wait_timeout_us=0, test_hook=0,
+                        stream=None):
+    """Enqueue the forward with the convolution prologue (u = SiLU(causal
+    depthwise conv of x) computed inside the scan kernels).  x (batch, dim, L)
+    in the I/O dtype; conv_w (dim, W) float32 with W in 1..4; conv_b (dim,)
+    float32 or None; the rest as ``mamba_scan_fwd``."""
+    batch, dim, L = x.shape
+    N = A.shape[1]
+    W = conv_w.shape[1]
+    dt = x.dtype
+    f32 = torch.float32
+    bdl, bnl = (batch, dim, L), (batch, N, L)
+    args = [
+        _ptr(x, dt, bdl, "x"), _ptr(conv_w, f32, (dim, W), "conv_w"),
+        _ptr(conv_b, f32, (dim,), "conv_b"), W,
+        _ptr(delta, dt, bdl, "delta"), _ptr(delta_bias, f32, (dim,), "delta_bias"),
+        _ptr(A, f32, (dim, N), "A"), _ptr(B, dt, bnl, "B"), _ptr(C, dt, bnl, "C"),
+        _ptr(D, f32, (dim,), "D"), _ptr(z, dt, bdl, "z"), _ptr(y, dt, bdl, "y"),
+        _ptr(last_state, f32, (batch, dim, N), "last_state"), batch, dim, L, N, _dtype_code(dt)]
+    opts = _opts_ptr(path, chunk_len, carry, wait_timeout_us, test_hook)
+    _check(load_library().mamba_conv_scan_fwd(*args, opts, _stream_handle(stream)),
+           "mamba_conv_scan_fwd")
+
+
+def mamba_conv_scan_bwd(x, conv_w, conv_b, delta, delta_bias, A, B, C, D, z, dy, dx, dconv_w,
+                        dconv_b, ddelta, dA, dB, dC, dD, dz, ddelta_bias, *, path="auto",
+                        chunk_len=0, wait_timeout_us=0, test_hook=0, stream=None):
+    """Enqueue the backward of sum(dy * y) for ``mamba_conv_scan_fwd``: dx
+    and dconv_w (and dconv_b if given) take the place of du."""
+    batch, dim, L = x.shape
+    N = A.shape[1]
+    W = conv_w.shape[1]
+    dt = x.dtype
+    f32 = torch.float32
+    bdl, bnl = (batch, dim, L), (batch, N, L)
+    args = [
+        _ptr(x, dt, bdl, "x"), _ptr(conv_w, f32, (dim, W), "conv_w"),
+        _ptr(conv_b, f32, (dim,), "conv_b"), W,
+        _ptr(delta, dt, bdl, "delta"), _ptr(delta_bias, f32, (dim,), "delta_bias"),
+        _ptr(A, f32, (dim, N), "A"), _ptr(B, dt, bnl, "B"), _ptr(C, dt, bnl, "C"),
+        _ptr(D, f32, (dim,), "D"), _ptr(z, dt, bdl, "z"), _ptr(dy, dt, bdl, "dy"),
+        _ptr(dx, dt, bdl, "dx"), _ptr(dconv_w, f32, (dim, W), "dconv_w"),
+        _ptr(dconv_b, f32, (dim,), "dconv_b"), _ptr(ddelta, dt, bdl, "ddelta"),
+        _ptr(dA, f32, (dim, N), "dA"), _ptr(dB, dt, bnl, "dB"), _ptr(dC, dt, bnl, "dC"),
+        _ptr(dD, f32, (dim,), "dD"), _ptr(dz, dt, bdl, "dz"),
+        _ptr(ddelta_bias, f32, (dim,), "ddelta_bias"), batch, dim, L, N, _dtype_code(dt)]
+    opts = _opts_ptr(path, chunk_len, "auto", wait_timeout_us, test_hook)
+    _check(load_library().mamba_conv_scan_bwd(*args, opts, _stream_handle(stream)),
+           "mamba_conv_scan_bwd")
+
+
 def mamba_scan_fwd_noalloc(u, delta, delta_bias, A, B, C, D, z, y, last_state, *, stream=None):
     """The forward without any device allocation by the library: for callers
     that cannot let a library allocate (their own allocator owns device
@@ -256,4 +321,41 @@ def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, p
     mamba_scan_bwd(u, delta, delta_bias, A, B, C, D, z, dy, g["du"], g["ddelta"], g["dA"],
                    g["dB"], g["dC"], g["dD"], g["dz"], g["ddelta_bias"], path=path,
                    chunk_len=chunk_len, stream=stream)
+    return {k: v for k, v in g.items() if v is not None}
+
+
+def conv_selective_scan_fwd(x, conv_w, conv_b, delta, A, B, C, D=None, z=None, delta_bias=None,
+                            return_last_state=False, path="auto", chunk_len=0, carry="auto",
+                            stream=None):
+    """Allocate y (and last_state) and run the forward with the convolution
+    prologue; returns y or (y, last_state)."""
+    batch, dim, L = x.shape
+    y = torch.empty_like(x)
+    last = (torch.empty(batch, dim, A.shape[1], device=x.device, dtype=torch.float32)
+            if return_last_state else None)
+    mamba_conv_scan_fwd(x, conv_w, conv_b, delta, delta_bias, A, B, C, D, z, y, last, path=path,
+                        chunk_len=chunk_len, carry=carry, stream=stream)
+    return (y, last) if return_last_state else y
+
+
+def conv_selective_scan_bwd(x, conv_w, conv_b, delta, A, B, C, dy, D=None, z=None,
+                            delta_bias=None, path="auto", chunk_len=0, stream=None) -> dict:
+    """Allocate the gradients and run the backward with the convolution
+    prologue; returns a dict of them (dx, dconv_w, dconv_b if conv_b is given,
+    and the scan's other gradients)."""
+    dim, N = A.shape
+    f32 = torch.float32
+    g = {
+        "dx": torch.empty_like(x), "dconv_w": torch.empty_like(conv_w),
+        "dconv_b": torch.empty(dim, device=x.device, dtype=f32) if conv_b is not None else None,
+        "ddelta": torch.empty_like(x),
+        "dA": torch.empty(dim, N, device=x.device, dtype=f32),
+        "dB": torch.empty_like(B), "dC": torch.empty_like(C),
+        "dD": torch.empty(dim, device=x.device, dtype=f32) if D is not None else None,
+        "dz": torch.empty_like(x) if z is not None else None,
+        "ddelta_bias": torch.empty(dim, device=x.device, dtype=f32),
+    }
+    mamba_conv_scan_bwd(x, conv_w, conv_b, delta, delta_bias, A, B, C, D, z, dy, g["dx"],
+                        g["dconv_w"], g["dconv_b"], g["ddelta"], g["dA"], g["dB"], g["dC"], g["dD"],
+                        g["dz"], g["ddelta_bias"], path=path, chunk_len=chunk_len, stream=stream)
     return {k: v for k, v in g.items() if v is not None}
