@@ -58,6 +58,10 @@ def load_library(path: str):
     lib.s6_oracle_conv_fwd.restype = ctypes.c_int
     lib.s6_oracle_conv_bwd.argtypes = [dp] * 3 + [i64] + [dp] * 18 + [i64] * 5
     lib.s6_oracle_conv_bwd.restype = ctypes.c_int
+    lib.s6_oracle_dtproj_fwd.argtypes = [dp] * 3 + [i64] + [dp] * 8 + [i64] * 5
+    lib.s6_oracle_dtproj_fwd.restype = ctypes.c_int
+    lib.s6_oracle_dtproj_bwd.argtypes = [dp] * 3 + [i64] + [dp] * 16 + [i64] * 5
+    lib.s6_oracle_dtproj_bwd.restype = ctypes.c_int
     return lib
 
 
@@ -211,6 +215,61 @@ def s6_conv_backward(x, conv_w, conv_b, delta, A, B, C, dy, delta_bias=None, D=N
            "ddelta_bias": dbias}
     if dcb is not None:
         out["dconv_b"] = dcb
+    if dD is not None:
+        out["dD"] = dD
+    if dz is not None:
+        out["dz"] = dz
+    return out
+
+
+def s6_dtproj_forward(u, dt_low, W_dt, A, B, C, delta_bias=None, D=None, z=None, nthreads=None,
+                      lib=None):
+    """fp64 forward with the low-rank Delta projection: delta = W_dt . dt_low
+    per batch row, then the S6 forward.  dt_low (batch, R, L); W_dt (dim, R).
+    Returns (y, last_state)."""
+    u, dt_low, W_dt, A, B, C = (_f64(t) for t in (u, dt_low, W_dt, A, B, C))
+    delta_bias, D, z = _f64(delta_bias), _f64(D), _f64(z)
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    R = W_dt.shape[1]
+    assert W_dt.shape == (dim, R) and dt_low.shape == (batch, R, L)
+    y = np.empty((batch, dim, L), np.float64)
+    last = np.empty((batch, dim, N), np.float64)
+    rc = (lib or _load()).s6_oracle_dtproj_fwd(
+        _ptr(u), _ptr(dt_low), _ptr(W_dt), R, _ptr(delta_bias), _ptr(A), _ptr(B), _ptr(C),
+        _ptr(D), _ptr(z), _ptr(y), _ptr(last), batch, dim, L, N, nthreads or default_threads())
+    if rc != 0:
+        raise RuntimeError(f"s6_oracle_dtproj_fwd failed ({rc})")
+    return y, last
+
+
+def s6_dtproj_backward(u, dt_low, W_dt, A, B, C, dy, delta_bias=None, D=None, z=None,
+                       nthreads=None, lib=None):
+    """fp64 backward of sum(dy * y) for the forward with the projection.
+    Returns a dict with du, d_dt_low, dW_dt, dA, dB, dC, ddelta_bias and, when
+    the matching input is given, dD, dz."""
+    u, dt_low, W_dt, A, B, C, dy = (_f64(t) for t in (u, dt_low, W_dt, A, B, C, dy))
+    delta_bias, D, z = _f64(delta_bias), _f64(D), _f64(z)
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    R = W_dt.shape[1]
+    du = np.empty_like(u)
+    dz = np.empty_like(u) if z is not None else None
+    ddl = np.empty((batch, R, L), np.float64)
+    dW = np.empty((dim, R), np.float64)
+    dA = np.empty((dim, N), np.float64)
+    dB = np.empty((batch, N, L), np.float64)
+    dC = np.empty((batch, N, L), np.float64)
+    dD = np.empty((dim,), np.float64) if D is not None else None
+    dbias = np.empty((dim,), np.float64)
+    rc = (lib or _load()).s6_oracle_dtproj_bwd(
+        _ptr(u), _ptr(dt_low), _ptr(W_dt), R, _ptr(delta_bias), _ptr(A), _ptr(B), _ptr(C),
+        _ptr(D), _ptr(z), _ptr(dy), _ptr(du), _ptr(ddl), _ptr(dW), _ptr(dA), _ptr(dB), _ptr(dC),
+        _ptr(dD), _ptr(dz), _ptr(dbias), batch, dim, L, N, nthreads or default_threads())
+    if rc != 0:
+        raise RuntimeError(f"s6_oracle_dtproj_bwd failed ({rc})")
+    out = {"du": du, "d_dt_low": ddl, "dW_dt": dW, "dA": dA, "dB": dB, "dC": dC,
+           "ddelta_bias": dbias}
     if dD is not None:
         out["dD"] = dD
     if dz is not None:

@@ -23,6 +23,9 @@
  *  [KN3]  chapterpal.com page, Knowl 3 "Mamba Block Architecture", step 3:
  *         the main branch runs a short 1D temporal convolution of width
  *         d_conv = 4, then SiLU, then the S6 layer.
+ *  [PG36] paper-graph-ui summary, section 3.6 "Additional Model Details",
+ *         "Parameterization of Delta's input projection" (the low-rank
+ *         s_Delta(x) = Linear_D(Linear_R(x))).
  *  [PG34] paper-graph-ui summary, "The Mamba Architecture (Section 3.4)",
  *         "The Mamba simplification": convolution (local context, the
  *         "shift-SSM" of H3), SiLU, selective SSM on the main branch.
@@ -62,6 +65,16 @@
  *     u[b,d,t]   = pre * sigmoid(pre)                                (SiLU)
  * and u feeds the forward above.  Its backward is the chain rule through the
  * SiLU and the convolution after the S6 backward has given du.
+ *
+ * Low-rank Delta projection (s6_oracle_dtproj_*), [PG36] "Parameterization
+ * of Delta's input projection": s_Delta(x) = Linear_D(Linear_R(x)) with a
+ * small rank R.  The scan takes the rank-R projection dt_low = Linear_R(x)
+ * (batch, R, L) and the weight W_dt (dim, R) of Linear_D, whose bias is
+ * delta_bias:
+ *     delta[b,d,t] = sum_r W_dt[d,r] * dt_low[b,r,t]
+ * and delta feeds the forward above (softplus(delta + delta_bias)).  Its
+ * backward is the chain rule through that product after the S6 backward has
+ * given ddelta.
  *
  * Parity pins (the tests check this file against): Theorem 1 closed form,
  * the LTI convolution form, brute-force unrolling, an independent ZOH via the
@@ -450,5 +463,77 @@ int s6_oracle_conv_bwd(const double *x, const double *conv_w, const double *conv
   free(pre);
   free(u);
   free(du);
+  return rc;
+}
+
+/* -------------------------------------------- low-rank Delta projection */
+
+/* delta = W_dt . dt_low per batch row (see the header). */
+static void dt_project(const double *dt_low, const double *W, i64 R, double *delta, i64 batch,
+                       i64 dim, i64 L) {
+  for (i64 b = 0; b < batch; ++b)
+    for (i64 d = 0; d < dim; ++d)
+      for (i64 t = 0; t < L; ++t) {
+        double s = 0.0;
+        for (i64 r = 0; r < R; ++r) s += W[d * R + r] * dt_low[(b * R + r) * L + t];
+        delta[(b * dim + d) * L + t] = s;
+      }
+}
+
+/* Forward with the low-rank Delta projection: delta = W_dt . dt_low, then
+ * the S6 forward of s6_oracle_fwd.  Layouts: dt_low (batch, R, L); W_dt
+ * (dim, R); the rest as s6_oracle_fwd. */
+int s6_oracle_dtproj_fwd(const double *u, const double *dt_low, const double *W_dt, i64 R,
+                         const double *bias, const double *A, const double *B, const double *C,
+                         const double *D, const double *z, double *y, double *last_state,
+                         i64 batch, i64 dim, i64 L, i64 N, i64 nthreads) {
+  if (batch < 0 || dim < 0 || L < 0 || R < 1) return -2;
+  const size_t n = (size_t)(batch * dim * L);
+  double *delta = (double *)malloc(sizeof(double) * (n ? n : 1));
+  if (!delta) return -1;
+  dt_project(dt_low, W_dt, R, delta, batch, dim, L);
+  const int rc = s6_oracle_fwd(u, delta, bias, A, B, C, D, z, NULL, y, last_state, batch, dim, L,
+                               N, nthreads);
+  free(delta);
+  return rc;
+}
+
+/* Backward of sum(dy * y) for the forward with the projection.  Outputs as
+ * in s6_oracle_bwd, with d_dt_low (batch, R, L) and dW_dt (dim, R) in place
+ * of ddelta.  With ddelta from the S6 backward, every term
+ * W_dt[d,r] * dt_low[b,r,t] of delta[b,d,t] passes ddelta[b,d,t] on:
+ *     d_dt_low[b,r,t] += W_dt[d,r] * ddelta[b,d,t],
+ *     dW_dt[d,r]      += ddelta[b,d,t] * dt_low[b,r,t]. */
+int s6_oracle_dtproj_bwd(const double *u, const double *dt_low, const double *W_dt, i64 R,
+                         const double *bias, const double *A, const double *B, const double *C,
+                         const double *D, const double *z, const double *dy, double *du,
+                         double *d_dt_low, double *dW_dt, double *dA, double *dB, double *dC,
+                         double *dD, double *dz, double *dbias, i64 batch, i64 dim, i64 L, i64 N,
+                         i64 nthreads) {
+  if (batch < 0 || dim < 0 || L < 0 || R < 1) return -2;
+  const size_t n = (size_t)(batch * dim * L);
+  double *delta = (double *)malloc(sizeof(double) * (n ? n : 1));
+  double *ddelta = (double *)malloc(sizeof(double) * (n ? n : 1));
+  int rc = -1;
+  if (delta && ddelta) {
+    dt_project(dt_low, W_dt, R, delta, batch, dim, L);
+    rc = s6_oracle_bwd(u, delta, bias, A, B, C, D, z, dy, du, ddelta, dA, dB, dC, dD, dz, dbias,
+                       batch, dim, L, N, nthreads);
+  }
+  if (rc == 0) {
+    memset(d_dt_low, 0, sizeof(double) * (size_t)(batch * R * L));
+    memset(dW_dt, 0, sizeof(double) * (size_t)(dim * R));
+    for (i64 b = 0; b < batch; ++b)
+      for (i64 d = 0; d < dim; ++d)
+        for (i64 t = 0; t < L; ++t) {
+          const double g = ddelta[(b * dim + d) * L + t];
+          for (i64 r = 0; r < R; ++r) {
+            d_dt_low[(b * R + r) * L + t] += W_dt[d * R + r] * g;
+            dW_dt[d * R + r] += g * dt_low[(b * R + r) * L + t];
+          }
+        }
+  }
+  free(delta);
+  free(ddelta);
   return rc;
 }

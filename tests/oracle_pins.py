@@ -512,12 +512,80 @@ def pin_conv_autograd(lib=None):
     return worst, 1e-12
 
 
+# -------------------------------------------- low-rank Delta projection
+
+def _dtproj_inputs(seed, b=2, d=3, L=23, N=4, R=2):
+    x = make_inputs(b, d, L, N, seed=seed, with_dy=True)
+    x = {k: (v.double() if v is not None else None) for k, v in x.items()}
+    g = torch.Generator().manual_seed(seed)
+    x["dt_low"] = torch.randn(b, R, L, generator=g, dtype=torch.float64)
+    x["W_dt"] = torch.randn(d, R, generator=g, dtype=torch.float64) / math.sqrt(R)
+    return x
+
+
+def pin_dtproj_matmul(lib=None):
+    """The projection against numpy's einsum: delta = W_dt . dt_low, then the
+    plain forward on that delta."""
+    x = _dtproj_inputs(81, R=5)
+    y, last = oracle.s6_dtproj_forward(x["u"], x["dt_low"], x["W_dt"], x["A"], x["B"], x["C"],
+                                       x["delta_bias"], x["D"], x["z"], lib=lib)
+    delta = np.einsum("dr,brl->bdl", _np(x["W_dt"]), _np(x["dt_low"]))
+    y_ref, last_ref = oracle.s6_forward(x["u"], delta, x["A"], x["B"], x["C"], x["delta_bias"],
+                                        x["D"], x["z"], lib=lib)
+    return max(normwise(y, y_ref), normwise(last, last_ref)), 1e-13
+
+
+def _dtproj_loss(x, lib):
+    y, _ = oracle.s6_dtproj_forward(x["u"], x["dt_low"], x["W_dt"], x["A"], x["B"], x["C"],
+                                    x["delta_bias"], x["D"], x["z"], lib=lib, nthreads=1)
+    return float(np.sum(_np(x["dy"]) * y))
+
+
+def pin_dtproj_finite_differences(lib=None):
+    """Central differences of sum(dy * y) through the projection: dt_low,
+    W_dt and u."""
+    x = _dtproj_inputs(82, b=1, d=2, L=9, N=3, R=2)
+    g = oracle.s6_dtproj_backward(x["u"], x["dt_low"], x["W_dt"], x["A"], x["B"], x["C"],
+                                  x["dy"], x["delta_bias"], x["D"], x["z"], lib=lib, nthreads=1)
+    worst = 0.0
+    for name, gname in {"dt_low": "d_dt_low", "W_dt": "dW_dt", "u": "du"}.items():
+        flat = x[name].reshape(-1)
+        fd = np.empty(x[name].shape)
+        for i in range(flat.numel()):
+            v = float(flat[i])
+            h = 1e-6 * max(1.0, abs(v))
+            flat[i] = v + h
+            lp = _dtproj_loss(x, lib)
+            flat[i] = v - h
+            lm = _dtproj_loss(x, lib)
+            flat[i] = v
+            fd.reshape(-1)[i] = (lp - lm) / (2.0 * h)
+        worst = max(worst, normwise(g[gname], fd))
+    return worst, 1e-6
+
+
+def pin_dtproj_autograd(lib=None):
+    """The projection's chain rule against torch.autograd through torch's
+    matmul, fed with the (separately pinned) S6 gradient ddelta."""
+    x = _dtproj_inputs(83, R=3)
+    dl = x["dt_low"].clone().requires_grad_(True)
+    W = x["W_dt"].clone().requires_grad_(True)
+    delta = torch.matmul(W, dl)  # (d, R) @ (b, R, L) -> (b, d, L)
+    gs6 = oracle.s6_backward(x["u"], delta.detach(), x["A"], x["B"], x["C"], x["dy"],
+                             x["delta_bias"], x["D"], x["z"], lib=lib)
+    ref = torch.autograd.grad(delta, (dl, W), grad_outputs=torch.from_numpy(gs6["ddelta"]))
+    g = oracle.s6_dtproj_backward(x["u"], x["dt_low"], x["W_dt"], x["A"], x["B"], x["C"],
+                                  x["dy"], x["delta_bias"], x["D"], x["z"], lib=lib)
+    return max(normwise(g["d_dt_low"], ref[0].numpy()), normwise(g["dW_dt"], ref[1].numpy())), 1e-12
+
+
 ALL_PINS = [pin_golden, pin_theorem1, pin_zoh_expm, pin_lti_convolution, pin_brute_force,
             pin_held_input_exact, pin_skip_and_gate, pin_large_delta_limit,
             pin_small_delta_limit, pin_structure, pin_finite_differences, pin_autograd,
             pin_threads_agree, pin_resume_from_state, pin_initial_state_decay,
             pin_conv_numpy, pin_conv_special_filters, pin_conv_finite_differences,
-            pin_conv_autograd]
+            pin_conv_autograd, pin_dtproj_matmul, pin_dtproj_finite_differences,
+            pin_dtproj_autograd]
 
 
 def run_all(lib=None):

@@ -42,6 +42,12 @@ MUTATIONS = {
     "bwd_conv_silu_derivative": ("s * (1.0 + pre[off + t] * (1.0 - s))", "s"),
     "bwd_conv_dw_uses_output_step": ("dconv_w[d * W + k] += dpre * x[off + src];",
                                      "dconv_w[d * W + k] += dpre * x[off + t];"),
+    "dtproj_W_transposed": ("s += W[d * R + r] * dt_low[(b * R + r) * L + t];",
+                            "s += W[r * dim + d] * dt_low[(b * R + r) * L + t];"),
+    "bwd_dtproj_dW_wrong_input": ("dW_dt[d * R + r] += g * dt_low[(b * R + r) * L + t];",
+                                  "dW_dt[d * R + r] += g * W_dt[d * R + r];"),
+    "bwd_dtproj_ddt_low_missing_W": ("d_dt_low[(b * R + r) * L + t] += W_dt[d * R + r] * g;",
+                                     "d_dt_low[(b * R + r) * L + t] += g;"),
     "bwd_dC_uses_prev_state": ("dCacc[(b * N + n) * L + t] += dy0 * H[(t + 1) * N + n];",
                                "dCacc[(b * N + n) * L + t] += dy0 * H[t * N + n];"),
 }
