@@ -102,8 +102,8 @@ def ncu_traffic(kernel_key: str):
         with open(p) as f:
             d = json.load(f)
         e = d[kernel_key]
-        from selective_state_space_21_b200.build import source_digest
-        if e.get("source_digest") != source_digest():
+        from selective_state_space_21_b200.build import STAGED_KERNEL_FILES, source_digest
+        if e.get("source_digest") != source_digest(STAGED_KERNEL_FILES):
             return None
         return e
     except Exception:
@@ -392,7 +392,7 @@ def run_ours(args, world, rank, device):
     if not args.only and not args.no_decode:
         result["decode"] = run_decode(w, x, device, peaks)
     if not args.only and not args.no_conv:
-        result["conv_prologue"] = run_conv(w, x, device, peaks)
+        result["conv_prologue"] = run_conv(w, x, device, peaks, steps=args.conv_steps)
     if args.only:
         result["note"] = f"--only {args.only}: a profiling run, not a benchmark result"
     if not args.no_e2e and not args.only:
@@ -655,6 +655,8 @@ def main(argv=None):
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-conv", action="store_true",
                     help="skip the convolution-prologue timing")
+    ap.add_argument("--conv-steps", type=int, default=10,
+                    help="timed calls of the convolution-prologue leg")
     ap.add_argument("--only", choices=["fwd", "bwd"], default=None,
                     help="time one pass only (for profiling; not a benchmark result)")
     args = ap.parse_args(argv)

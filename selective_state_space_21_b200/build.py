@@ -34,12 +34,21 @@ def deps():
         os.path.join(ROOT, "include", "mamba_scan.h")]
 
 
-def source_digest() -> str:
-    """Short hash of every source the library is built from (used to tell
+#: The files that define the staged forward and backward kernels and their
+#: launches (plus the compiler flags): a stored profile of those kernels stays
+#: valid while these are unchanged.
+STAGED_KERNEL_FILES = ("fwd_staged.cuh", "bwd_staged.cuh", "common.cuh", "tma.cuh")
+
+
+def source_digest(files=None) -> str:
+    """Short hash of the sources the library is built from -- all of them, or
+    only ``files`` (names under csrc/) -- and of the nvcc flags (used to tell
     whether a stored profile still describes the current kernels)."""
     import hashlib
     h = hashlib.sha256()
-    for p in deps():
+    h.update(" ".join(NVCC_FLAGS).encode())
+    paths = deps() if files is None else [os.path.join(CSRC, f) for f in files]
+    for p in paths:
         h.update(os.path.basename(p).encode())
         with open(p, "rb") as f:
             h.update(f.read())
