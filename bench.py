@@ -393,6 +393,8 @@ def run_ours(args, world, rank, device):
         result["decode"] = run_decode(w, x, device, peaks)
     if not args.only and not args.no_conv:
         result["conv_prologue"] = run_conv(w, x, device, peaks, steps=args.conv_steps)
+    if not args.only and not args.no_dtproj:
+        result["dt_projection"] = run_dtproj(w, x, device, steps=args.conv_steps)
     if args.only:
         result["note"] = f"--only {args.only}: a profiling run, not a benchmark result"
     if not args.no_e2e and not args.only:
@@ -466,6 +468,70 @@ def run_conv(w, x, device, peaks, steps=10):
                     "tc_per_s": w.token_channels / (bms * 1e-3)},
             "steps": steps, "width": 4, "timing": "median of per-call CUDA events",
             "shape": f"x in place of u, batch {w.batch} x dim {w.dim} x L {w.L}, N {w.N}"}
+
+
+def run_dtproj(w, x, device, steps=10):
+    """The same workload with the low-rank Delta projection of rank
+    ceil(d_model / 16) = ceil(dim / 32): mamba_dtproj_scan_fwd / _bwd take
+    dt_low (batch, R, L) and W_dt (dim, R) in place of delta.  Times each call
+    with CUDA events; the projection's own share is the difference to the
+    plain calls' times measured alongside."""
+    from selective_state_space_21_b200 import scan
+    from selective_state_space_21_b200.inputs import make_dtproj_params
+
+    R = -(-w.dim // 32)
+    pp = make_dtproj_params(w.batch, w.dim, w.L, R, w.dtype, device=device, seed=4322)
+    y = torch.empty_like(x["u"])
+    g = {k: torch.empty_like(x[k]) for k in ("u", "z", "B", "C", "delta")}
+    f32 = dict(device=device, dtype=torch.float32)
+    ddl = torch.empty_like(pp["dt_low"])
+    dW = torch.empty(w.dim, R, **f32)
+    dA, dD, db = torch.empty(w.dim, w.N, **f32), torch.empty(w.dim, **f32), torch.empty(w.dim, **f32)
+
+    def fwd():
+        scan.mamba_dtproj_scan_fwd(x["u"], pp["dt_low"], pp["W_dt"], x["delta_bias"], x["A"],
+                                   x["B"], x["C"], x["D"], x["z"], y, None)
+
+    def bwd():
+        scan.mamba_dtproj_scan_bwd(x["u"], pp["dt_low"], pp["W_dt"], x["delta_bias"], x["A"],
+                                   x["B"], x["C"], x["D"], x["z"], x["dy"], g["u"], ddl, dW, dA,
+                                   g["B"], g["C"], dD, g["z"], db)
+
+    def fwd_plain():
+        scan.mamba_scan_fwd(x["u"], x["delta"], x["delta_bias"], x["A"], x["B"], x["C"], x["D"],
+                            x["z"], y, None)
+
+    def bwd_plain():
+        scan.mamba_scan_bwd(x["u"], x["delta"], x["delta_bias"], x["A"], x["B"], x["C"], x["D"],
+                            x["z"], x["dy"], g["u"], g["delta"], dA, g["B"], g["C"], dD, g["z"],
+                            db)
+
+    def timed(fns):
+        for _ in range(3):
+            for f in fns:
+                f()
+        torch.cuda.synchronize(device)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(fns) + 1)]
+              for _ in range(steps)]
+        for k in range(steps):
+            for i, f in enumerate(fns):
+                ev[k][i].record()
+                f()
+            ev[k][-1].record()
+        torch.cuda.synchronize(device)
+        return [statistics.median(e[i].elapsed_time(e[i + 1]) for e in ev)
+                for i in range(len(fns))]
+
+    fms, bms, fpl, bpl = timed([fwd, bwd, fwd_plain, bwd_plain])
+    if scan.mamba_scan_stream_status() != 0:
+        raise RuntimeError("device error in the projection run")
+    return {"rank": R, "fwd_ms": round(fms, 4), "bwd_ms": round(bms, 4),
+            "plain_fwd_ms": round(fpl, 4), "plain_bwd_ms": round(bpl, 4),
+            "projection_fwd_ms": round(fms - fpl, 4), "projection_bwd_ms": round(bms - bpl, 4),
+            "fwd_tc_per_s": w.token_channels / (fms * 1e-3),
+            "bwd_tc_per_s": w.token_channels / (bms * 1e-3), "steps": steps,
+            "timing": "median of per-call CUDA events",
+            "shape": f"dt_low (batch {w.batch}, R {R}, L {w.L}), W_dt ({w.dim}, {R})"}
 
 
 def run_decode(w, x, device, peaks, steps=200):
@@ -656,7 +722,9 @@ def main(argv=None):
     ap.add_argument("--no-conv", action="store_true",
                     help="skip the convolution-prologue timing")
     ap.add_argument("--conv-steps", type=int, default=10,
-                    help="timed calls of the convolution-prologue leg")
+                    help="timed calls of the convolution-prologue and projection legs")
+    ap.add_argument("--no-dtproj", action="store_true",
+                    help="skip the Delta-projection timing")
     ap.add_argument("--only", choices=["fwd", "bwd"], default=None,
                     help="time one pass only (for profiling; not a benchmark result)")
     args = ap.parse_args(argv)

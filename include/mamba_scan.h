@@ -206,6 +206,48 @@ MAMBA_SCAN_API mamba_status_t mamba_conv_scan_bwd(
     const mamba_scan_options_t *options, mamba_stream_t stream);
 
 /*
+ * Forward with the low-rank Delta projection ("Mamba: Linear-Time Sequence
+ * Modeling with Selective State Spaces", paper-graph-ui summary, section 3.6
+ * "Parameterization of Delta's input projection": s_Delta(x) =
+ * Linear_D(Linear_R(x)) with a small rank R).  The caller passes the rank-R
+ * projection and the weight of Linear_D instead of delta:
+ *     delta[b,d,t] = sum_r W_dt[d,r] * dt_low[b,r,t]
+ * and delta_bias is Linear_D's bias (softplus(delta + delta_bias) as before).
+ *   dt_low : (batch, R, L) dtype
+ *   W_dt   : (dim, R) dtype (the I/O type, like a bf16 layer weight)
+ * Everything else as in mamba_scan_fwd_ex.  The contraction runs on the
+ * tensor cores through cuBLAS (fp32 accumulation, result rounded once to the
+ * I/O type) into a stream-ordered workspace of delta's size that the scan
+ * reads; cuBLAS is opened at run time (libcublas.so.12), and without it the
+ * call returns MAMBA_ERR_UNSUPPORTED.  R in 1..2^20; dim and L below 2^31.
+ */
+MAMBA_SCAN_API mamba_status_t mamba_dtproj_scan_fwd(const void *u, const void *dt_low,
+                                                    const void *W_dt, int64_t R,
+                                                    const float *delta_bias, const float *A,
+                                                    const void *B, const void *C, const float *D,
+                                                    const void *z, void *y, float *last_state,
+                                                    int64_t batch, int64_t dim, int64_t L,
+                                                    int64_t N, mamba_dtype_t dtype,
+                                                    const mamba_scan_options_t *options,
+                                                    mamba_stream_t stream);
+
+/*
+ * Backward of sum(dy * y) for mamba_dtproj_scan_fwd.  As mamba_scan_bwd_ex,
+ * with d_dt_low (batch, R, L) dtype and dW_dt (dim, R) float32 in place of
+ * ddelta:
+ *     d_dt_low[b] = W_dt^T . ddelta[b],   dW_dt = sum_b ddelta[b] . dt_low[b]^T
+ * where ddelta (the scan backward's gradient of delta, rounded once to the
+ * I/O type) lives in a workspace.  dW_dt is accumulated over the batch rows
+ * in a fixed order.
+ */
+MAMBA_SCAN_API mamba_status_t mamba_dtproj_scan_bwd(
+    const void *u, const void *dt_low, const void *W_dt, int64_t R, const float *delta_bias,
+    const float *A, const void *B, const void *C, const float *D, const void *z, const void *dy,
+    void *du, void *d_dt_low, float *dW_dt, float *dA, void *dB, void *dC, float *dD, void *dz,
+    float *ddelta_bias, int64_t batch, int64_t dim, int64_t L, int64_t N, mamba_dtype_t dtype,
+    const mamba_scan_options_t *options, mamba_stream_t stream);
+
+/*
  * One decoding step: the recurrent mode of the selective SSM, one token per
  * call with constant work per token ("Mamba: Linear-Time Sequence Modeling
  * with Selective State Spaces", trishampatil.com walk-through, Part II

@@ -14,6 +14,7 @@
 #include "bwd_staged.cuh"
 #include "common.cuh"
 #include "conv_bwd.cuh"
+#include "dtproj.h"
 #include "decode.cuh"
 #include "fwd_reference.cuh"
 #include "fwd_staged.cuh"
@@ -631,6 +632,148 @@ mamba_status_t mamba_conv_scan_bwd(const void *x, const float *conv_w, const flo
     st = launch_status();
   }
   if (ws_free(part, s) != cudaSuccess && st == MAMBA_OK) st = MAMBA_ERR_CUDA;
+  return st;
+}
+
+// ------------------------------------------- low-rank Delta projection
+
+mamba_status_t mamba_dtproj_scan_fwd(const void *u, const void *dt_low, const void *W_dt,
+                                     int64_t R, const float *delta_bias, const float *A,
+                                     const void *B, const void *C, const float *D, const void *z,
+                                     void *y, float *last_state, int64_t batch, int64_t dim,
+                                     int64_t L, int64_t N, mamba_dtype_t dtype,
+                                     const mamba_scan_options_t *options, mamba_stream_t stream) {
+  mamba_status_t st = check_shape(batch, dim, L, N, dtype);
+  if (st != MAMBA_OK) return st;
+  if ((st = check_options(options)) != MAMBA_OK) return st;
+  if (R < 1 || R > (int64_t(1) << 20)) return MAMBA_ERR_INVALID_ARG;
+  if (dim >= (int64_t(1) << 31) || L >= (int64_t(1) << 31)) return MAMBA_ERR_UNSUPPORTED;
+  Checker ck;
+  if (cudaGetDevice(&ck.dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MAMBA_ERR_CUDA;
+  }
+  const size_t es = dtype_size(dtype);
+  const size_t nbdl = size_t(batch) * size_t(dim) * size_t(L);
+  const size_t nbnl = size_t(batch) * size_t(N) * size_t(L);
+  ck.buf(u, nbdl * es, es, true, false);
+  ck.buf(dt_low, size_t(batch) * size_t(R) * size_t(L) * es, es, true, false);
+  ck.buf(W_dt, size_t(dim) * size_t(R) * es, es, true, false);
+  ck.buf(z, nbdl * es, es, false, false);
+  ck.buf(B, nbnl * es, es, true, false);
+  ck.buf(C, nbnl * es, es, true, false);
+  ck.buf(A, size_t(dim) * N * 4, 4, true, false);
+  ck.buf(D, size_t(dim) * 4, 4, false, false);
+  ck.buf(delta_bias, size_t(dim) * 4, 4, false, false);
+  ck.buf(y, nbdl * es, es, true, true);
+  ck.buf(last_state, size_t(batch) * dim * N * 4, 4, false, true);
+  if (ck.st != MAMBA_OK) return ck.st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (batch == 0 || dim == 0) return MAMBA_OK;
+  if (L == 0) {
+    if (last_state && cudaMemsetAsync(last_state, 0, size_t(batch) * dim * N * 4, s) != cudaSuccess)
+      return cuda_status();
+    return MAMBA_OK;
+  }
+  const cublasHandle_t h = cublas_handle(ck.dev);
+  if (!h || cublas_api().set_stream(h, s) != CUBLAS_STATUS_SUCCESS) return MAMBA_ERR_UNSUPPORTED;
+  void *delta = nullptr;
+  if (ws_alloc(&delta, nbdl * es, s) != cudaSuccess) {
+    cudaGetLastError();
+    return MAMBA_ERR_OUT_OF_MEMORY;
+  }
+  const DtProj pj{h, dtype == MAMBA_BF16 ? CUDA_R_16BF : CUDA_R_32F, batch, dim, L, R};
+  st = pj.forward(dt_low, W_dt, delta) ? MAMBA_OK : MAMBA_ERR_CUDA;
+  if (st == MAMBA_OK) {
+    FwdArgs a;
+    a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
+    a.bias = delta_bias; a.A = A; a.D = D; a.y = y; a.last_state = last_state;
+    a.batch = batch; a.dim = dim; a.L = L; a.N = (int)N;
+    st = forward_paths<false>(a, es, dtype, staged_options(options), s);
+  }
+  if (ws_free(delta, s) != cudaSuccess && st == MAMBA_OK) st = MAMBA_ERR_CUDA;
+  return st;
+}
+
+mamba_status_t mamba_dtproj_scan_bwd(const void *u, const void *dt_low, const void *W_dt,
+                                     int64_t R, const float *delta_bias, const float *A,
+                                     const void *B, const void *C, const float *D, const void *z,
+                                     const void *dy, void *du, void *d_dt_low, float *dW_dt,
+                                     float *dA, void *dB, void *dC, float *dD, void *dz,
+                                     float *ddelta_bias, int64_t batch, int64_t dim, int64_t L,
+                                     int64_t N, mamba_dtype_t dtype,
+                                     const mamba_scan_options_t *options, mamba_stream_t stream) {
+  mamba_status_t st = check_shape(batch, dim, L, N, dtype);
+  if (st != MAMBA_OK) return st;
+  if ((st = check_options(options)) != MAMBA_OK) return st;
+  if (R < 1 || R > (int64_t(1) << 20)) return MAMBA_ERR_INVALID_ARG;
+  if (dim >= (int64_t(1) << 31) || L >= (int64_t(1) << 31)) return MAMBA_ERR_UNSUPPORTED;
+  if ((z == nullptr) != (dz == nullptr) || (D == nullptr) != (dD == nullptr))
+    return MAMBA_ERR_INVALID_ARG;
+  Checker ck;
+  if (cudaGetDevice(&ck.dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MAMBA_ERR_CUDA;
+  }
+  const size_t es = dtype_size(dtype);
+  const size_t nbdl = size_t(batch) * size_t(dim) * size_t(L);
+  const size_t nbnl = size_t(batch) * size_t(N) * size_t(L);
+  const size_t nbrl = size_t(batch) * size_t(R) * size_t(L);
+  ck.buf(u, nbdl * es, es, true, false);
+  ck.buf(dt_low, nbrl * es, es, true, false);
+  ck.buf(W_dt, size_t(dim) * size_t(R) * es, es, true, false);
+  ck.buf(z, nbdl * es, es, false, false);
+  ck.buf(dy, nbdl * es, es, true, false);
+  ck.buf(B, nbnl * es, es, true, false);
+  ck.buf(C, nbnl * es, es, true, false);
+  ck.buf(A, size_t(dim) * N * 4, 4, true, false);
+  ck.buf(D, size_t(dim) * 4, 4, false, false);
+  ck.buf(delta_bias, size_t(dim) * 4, 4, false, false);
+  ck.buf(du, nbdl * es, es, true, true);
+  ck.buf(d_dt_low, nbrl * es, es, true, true);
+  ck.buf(dW_dt, size_t(dim) * size_t(R) * 4, 4, true, true);
+  ck.buf(dz, nbdl * es, es, false, true);
+  ck.buf(dB, nbnl * es, es, true, true);
+  ck.buf(dC, nbnl * es, es, true, true);
+  ck.buf(dA, size_t(dim) * N * 4, 4, true, true);
+  ck.buf(dD, size_t(dim) * 4, 4, false, true);
+  ck.buf(ddelta_bias, size_t(dim) * 4, 4, false, true);
+  if (ck.st != MAMBA_OK) return ck.st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (dim == 0) return MAMBA_OK;
+  if (batch == 0 || L == 0) {  // empty sums
+    if (cudaMemsetAsync(dA, 0, size_t(dim) * N * 4, s) != cudaSuccess ||
+        cudaMemsetAsync(dW_dt, 0, size_t(dim) * size_t(R) * 4, s) != cudaSuccess ||
+        (dD && cudaMemsetAsync(dD, 0, size_t(dim) * 4, s) != cudaSuccess) ||
+        (ddelta_bias && cudaMemsetAsync(ddelta_bias, 0, size_t(dim) * 4, s) != cudaSuccess))
+      return cuda_status();
+    return MAMBA_OK;
+  }
+  const cublasHandle_t h = cublas_handle(ck.dev);
+  if (!h || cublas_api().set_stream(h, s) != CUBLAS_STATUS_SUCCESS) return MAMBA_ERR_UNSUPPORTED;
+  // workspace: delta, then ddelta (the scan backward's gradient of delta)
+  const size_t half = (nbdl * es + 255) / 256 * 256;
+  unsigned char *ws = nullptr;
+  if (ws_alloc(reinterpret_cast<void **>(&ws), 2 * half, s) != cudaSuccess) {
+    cudaGetLastError();
+    return MAMBA_ERR_OUT_OF_MEMORY;
+  }
+  void *delta = ws, *ddelta = ws + half;
+  const DtProj pj{h, dtype == MAMBA_BF16 ? CUDA_R_16BF : CUDA_R_32F, batch, dim, L, R};
+  st = pj.forward(dt_low, W_dt, delta) ? MAMBA_OK : MAMBA_ERR_CUDA;
+  if (st == MAMBA_OK) {
+    BwdArgs a;
+    a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C; a.dy = dy;
+    a.bias = delta_bias; a.A = A; a.D = D;
+    a.du = du; a.ddelta = ddelta; a.dz = dz; a.dB = dB; a.dC = dC;
+    a.dA = dA; a.dD = dD; a.dbias = ddelta_bias;
+    a.batch = batch; a.dim = dim; a.L = L; a.N = (int)N;
+    st = backward_paths<false>(a, es, dtype, staged_options(options), s);
+  }
+  if (st == MAMBA_OK && !(pj.grad_input(ddelta, W_dt, d_dt_low) &&
+                          pj.grad_weight(ddelta, dt_low, dW_dt, es)))
+    st = MAMBA_ERR_CUDA;
+  if (ws_free(ws, s) != cudaSuccess && st == MAMBA_OK) st = MAMBA_ERR_CUDA;
   return st;
 }
 

@@ -27,6 +27,10 @@ Architecture" of the chapterpal.com page) the input x takes the place of u
 and is drawn the same way; the per-channel filter and bias are drawn
 uniform in [-1/sqrt(W), 1/sqrt(W)] (the usual default initialisation of a
 depthwise Conv1d layer, fan-in W; the pages give none).
+
+For the low-rank Delta projection (section 3.6 of the paper-graph-ui page,
+s_Delta = Linear_D(Linear_R(x))) the rank-R input dt_low is N(0, 1) and the
+weight W_dt is N(0, 1/R), so that their product has delta's unit variance.
 """
 from __future__ import annotations
 
@@ -121,6 +125,18 @@ def make_conv_params(dim: int, width: int = 4, device="cpu", seed: int = SEED_BA
     w = (torch.rand(dim, width, generator=g, device=device) * 2.0 - 1.0) * bound
     b = (torch.rand(dim, generator=g, device=device) * 2.0 - 1.0) * bound
     return {"conv_w": w.contiguous(), "conv_b": b if has_bias else None}
+
+
+def make_dtproj_params(batch: int, dim: int, L: int, R: int, dtype: torch.dtype = torch.float32,
+                       device="cpu", seed: int = SEED_BASE) -> dict:
+    """Draw the rank-R input of the low-rank Delta projection, dt_low (batch,
+    R, L) ~ N(0, 1), and the weight W_dt (dim, R) ~ N(0, 1/R), both in the I/O
+    dtype (so that W_dt . dt_low has unit variance, as delta has)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed + 104729)
+    dt_low = torch.randn(batch, R, L, generator=g, device=device).to(dtype)
+    W = (torch.randn(dim, R, generator=g, device=device) / math.sqrt(R)).to(dtype)
+    return {"dt_low": dt_low.contiguous(), "W_dt": W.contiguous()}
 
 
 def workload_inputs(index: int, device="cpu", with_dy: Optional[bool] = None) -> dict:

@@ -4,7 +4,8 @@ CPU fallback; a missing library or device raises.
 
 Low-level calls (same names and argument order as ``include/mamba_scan.h``):
 ``mamba_scan_fwd``, ``mamba_scan_bwd``, ``mamba_conv_scan_fwd``,
-``mamba_conv_scan_bwd``, ``mamba_scan_step``, ``mamba_scan_fwd_noalloc``,
+``mamba_conv_scan_bwd``, ``mamba_dtproj_scan_fwd``, ``mamba_dtproj_scan_bwd``,
+``mamba_scan_step``, ``mamba_scan_fwd_noalloc``,
 ``mamba_scan_stream_status``.  Convenience wrappers that allocate the outputs:
 ``selective_scan_fwd``, ``selective_scan_bwd``, ``conv_selective_scan_fwd``
 and ``conv_selective_scan_bwd``.
@@ -71,6 +72,10 @@ def load_library():
             lib.mamba_conv_scan_fwd.restype = ctypes.c_int
             lib.mamba_conv_scan_bwd.argtypes = [vp] * 3 + [i64] + [vp] * 18 + [i64] * 4 + [i32, opt, vp]
             lib.mamba_conv_scan_bwd.restype = ctypes.c_int
+            lib.mamba_dtproj_scan_fwd.argtypes = [vp] * 3 + [i64] + [vp] * 8 + [i64] * 4 + [i32, opt, vp]
+            lib.mamba_dtproj_scan_fwd.restype = ctypes.c_int
+            lib.mamba_dtproj_scan_bwd.argtypes = [vp] * 3 + [i64] + [vp] * 16 + [i64] * 4 + [i32, opt, vp]
+            lib.mamba_dtproj_scan_bwd.restype = ctypes.c_int
             for f in ("mamba_scan_fwd", "mamba_scan_fwd_ex", "mamba_scan_bwd",
                       "mamba_scan_bwd_ex", "mamba_scan_stream_status", "mamba_scan_fwd_noalloc"):
                 getattr(lib, f).restype = ctypes.c_int
@@ -242,6 +247,57 @@ def mamba_conv_scan_bwd(x, conv_w, conv_b, delta, delta_bias, A, B, C, D, z, dy,
     opts = _opts_ptr(path, chunk_len, "auto", wait_timeout_us, test_hook)
     _check(load_library().mamba_conv_scan_bwd(*args, opts, _stream_handle(stream)),
            "mamba_conv_scan_bwd")
+
+
+def mamba_dtproj_scan_fwd(u, dt_low, W_dt, delta_bias, A, B, C, D, z, y, last_state, *,
+                          path="auto", chunk_len=0, carry="auto", wait_timeout_us=0,
+                          test_hook=0, stream=None):
+    """Enqueue the forward with the low-rank Delta projection: delta =
+    W_dt . dt_low per batch row (a tensor-core GEMM), then the scan.  dt_low
+    (batch, R, L) and W_dt (dim, R) in the I/O dtype; the rest as
+    ``mamba_scan_fwd``."""
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    R = W_dt.shape[1]
+    dt = u.dtype
+    f32 = torch.float32
+    bdl, bnl = (batch, dim, L), (batch, N, L)
+    args = [
+        _ptr(u, dt, bdl, "u"), _ptr(dt_low, dt, (batch, R, L), "dt_low"),
+        _ptr(W_dt, dt, (dim, R), "W_dt"), R, _ptr(delta_bias, f32, (dim,), "delta_bias"),
+        _ptr(A, f32, (dim, N), "A"), _ptr(B, dt, bnl, "B"), _ptr(C, dt, bnl, "C"),
+        _ptr(D, f32, (dim,), "D"), _ptr(z, dt, bdl, "z"), _ptr(y, dt, bdl, "y"),
+        _ptr(last_state, f32, (batch, dim, N), "last_state"), batch, dim, L, N, _dtype_code(dt)]
+    opts = _opts_ptr(path, chunk_len, carry, wait_timeout_us, test_hook)
+    _check(load_library().mamba_dtproj_scan_fwd(*args, opts, _stream_handle(stream)),
+           "mamba_dtproj_scan_fwd")
+
+
+def mamba_dtproj_scan_bwd(u, dt_low, W_dt, delta_bias, A, B, C, D, z, dy, du, d_dt_low, dW_dt,
+                          dA, dB, dC, dD, dz, ddelta_bias, *, path="auto", chunk_len=0,
+                          wait_timeout_us=0, test_hook=0, stream=None):
+    """Enqueue the backward of sum(dy * y) for ``mamba_dtproj_scan_fwd``:
+    d_dt_low (batch, R, L, I/O dtype) and dW_dt (dim, R, float32) take the
+    place of ddelta."""
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    R = W_dt.shape[1]
+    dt = u.dtype
+    f32 = torch.float32
+    bdl, bnl = (batch, dim, L), (batch, N, L)
+    args = [
+        _ptr(u, dt, bdl, "u"), _ptr(dt_low, dt, (batch, R, L), "dt_low"),
+        _ptr(W_dt, dt, (dim, R), "W_dt"), R, _ptr(delta_bias, f32, (dim,), "delta_bias"),
+        _ptr(A, f32, (dim, N), "A"), _ptr(B, dt, bnl, "B"), _ptr(C, dt, bnl, "C"),
+        _ptr(D, f32, (dim,), "D"), _ptr(z, dt, bdl, "z"), _ptr(dy, dt, bdl, "dy"),
+        _ptr(du, dt, bdl, "du"), _ptr(d_dt_low, dt, (batch, R, L), "d_dt_low"),
+        _ptr(dW_dt, f32, (dim, R), "dW_dt"), _ptr(dA, f32, (dim, N), "dA"),
+        _ptr(dB, dt, bnl, "dB"), _ptr(dC, dt, bnl, "dC"), _ptr(dD, f32, (dim,), "dD"),
+        _ptr(dz, dt, bdl, "dz"), _ptr(ddelta_bias, f32, (dim,), "ddelta_bias"),
+        batch, dim, L, N, _dtype_code(dt)]
+    opts = _opts_ptr(path, chunk_len, "auto", wait_timeout_us, test_hook)
+    _check(load_library().mamba_dtproj_scan_bwd(*args, opts, _stream_handle(stream)),
+           "mamba_dtproj_scan_bwd")
 
 
 def mamba_scan_fwd_noalloc(u, delta, delta_bias, A, B, C, D, z, y, last_state, *, stream=None):
