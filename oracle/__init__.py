@@ -62,6 +62,10 @@ def load_library(path: str):
     lib.s6_oracle_dtproj_fwd.restype = ctypes.c_int
     lib.s6_oracle_dtproj_bwd.argtypes = [dp] * 3 + [i64] + [dp] * 16 + [i64] * 5
     lib.s6_oracle_dtproj_bwd.restype = ctypes.c_int
+    lib.s6_oracle_cplx_fwd.argtypes = [dp] * 10 + [i64] * 5
+    lib.s6_oracle_cplx_fwd.restype = ctypes.c_int
+    lib.s6_oracle_cplx_bwd.argtypes = [dp] * 17 + [i64] * 5
+    lib.s6_oracle_cplx_bwd.restype = ctypes.c_int
     return lib
 
 
@@ -270,6 +274,56 @@ def s6_dtproj_backward(u, dt_low, W_dt, A, B, C, dy, delta_bias=None, D=None, z=
         raise RuntimeError(f"s6_oracle_dtproj_bwd failed ({rc})")
     out = {"du": du, "d_dt_low": ddl, "dW_dt": dW, "dA": dA, "dB": dB, "dC": dC,
            "ddelta_bias": dbias}
+    if dD is not None:
+        out["dD"] = dD
+    if dz is not None:
+        out["dz"] = dz
+    return out
+
+
+def s6_cplx_forward(u, delta, A, B, C, delta_bias=None, D=None, z=None, nthreads=None, lib=None):
+    """fp64 forward with a complex diagonal A (and complex B, C, state).
+    Complex vectors are planar, real parts first: A (dim, 2N); B, C (batch,
+    2N, L).  Returns (y (batch, dim, L), last_state (batch, dim, 2N))."""
+    u, delta, A, B, C = (_f64(t) for t in (u, delta, A, B, C))
+    delta_bias, D, z = _f64(delta_bias), _f64(D), _f64(z)
+    batch, dim, L = u.shape
+    N = A.shape[1] // 2
+    assert A.shape == (dim, 2 * N) and B.shape == (batch, 2 * N, L) and C.shape == B.shape
+    y = np.empty((batch, dim, L), np.float64)
+    last = np.empty((batch, dim, 2 * N), np.float64)
+    rc = (lib or _load()).s6_oracle_cplx_fwd(
+        _ptr(u), _ptr(delta), _ptr(delta_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+        _ptr(y), _ptr(last), batch, dim, L, N, nthreads or default_threads())
+    if rc != 0:
+        raise RuntimeError(f"s6_oracle_cplx_fwd failed ({rc})")
+    return y, last
+
+
+def s6_cplx_backward(u, delta, A, B, C, dy, delta_bias=None, D=None, z=None, nthreads=None,
+                     lib=None):
+    """fp64 backward of sum(dy * y) for the complex forward.  Gradients of
+    complex inputs are (d/d re, d/d im) pairs in the planar layout.  Returns
+    a dict with du, ddelta, dA, dB, dC, ddelta_bias and, when given, dD, dz."""
+    u, delta, A, B, C, dy = (_f64(t) for t in (u, delta, A, B, C, dy))
+    delta_bias, D, z = _f64(delta_bias), _f64(D), _f64(z)
+    batch, dim, L = u.shape
+    N = A.shape[1] // 2
+    du = np.empty_like(u)
+    ddelta = np.empty_like(u)
+    dz = np.empty_like(u) if z is not None else None
+    dA = np.empty((dim, 2 * N), np.float64)
+    dB = np.empty((batch, 2 * N, L), np.float64)
+    dC = np.empty((batch, 2 * N, L), np.float64)
+    dD = np.empty((dim,), np.float64) if D is not None else None
+    dbias = np.empty((dim,), np.float64)
+    rc = (lib or _load()).s6_oracle_cplx_bwd(
+        _ptr(u), _ptr(delta), _ptr(delta_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+        _ptr(dy), _ptr(du), _ptr(ddelta), _ptr(dA), _ptr(dB), _ptr(dC), _ptr(dD), _ptr(dz),
+        _ptr(dbias), batch, dim, L, N, nthreads or default_threads())
+    if rc != 0:
+        raise RuntimeError(f"s6_oracle_cplx_bwd failed ({rc})")
+    out = {"du": du, "ddelta": ddelta, "dA": dA, "dB": dB, "dC": dC, "ddelta_bias": dbias}
     if dD is not None:
         out["dD"] = dD
     if dz is not None:

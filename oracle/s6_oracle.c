@@ -26,6 +26,8 @@
  *  [PG36] paper-graph-ui summary, section 3.6 "Additional Model Details",
  *         "Parameterization of Delta's input projection" (the low-rank
  *         s_Delta(x) = Linear_D(Linear_R(x))).
+ *  [PG-T8] paper-graph-ui summary, "Ablation Studies and Robustness Checks",
+ *         "Parameterization of A (Table 8)": S4D-Lin, A_n = -1/2 + n i.
  *  [PG34] paper-graph-ui summary, "The Mamba Architecture (Section 3.4)",
  *         "The Mamba simplification": convolution (local context, the
  *         "shift-SSM" of H3), SiLU, selective SSM on the main branch.
@@ -76,11 +78,24 @@
  * backward is the chain rule through that product after the S6 backward has
  * given ddelta.
  *
+ * Complex-valued diagonal A (s6_oracle_cplx_*), [PG36] "Real vs. Complex
+ * parameters" and [PG-T8] (S4D-Lin, A_n = -1/2 + n i): the state, A, B and C
+ * are complex, u, delta, z and y real.  Readings where the pages say no more:
+ * B_t and C_t are input-dependent complex vectors; the output is the real
+ * part of the readout; the same zero-order hold with complex exp and psi:
+ *     Abar = exp(Delta A_n),  Bbar = (exp(Delta A_n) - 1) / A_n * B_n,
+ *     h_n  = Abar h_n + Bbar u,   y0 = Re(sum_n C_n h_n) + D u.
+ * A complex vector of N entries is passed as 2N doubles, real parts first
+ * ("planar"): A (dim, 2N), B and C (batch, 2N, L), states (batch, dim, 2N).
+ * Gradients of complex inputs are the pairs (d/d re, d/d im), stored the
+ * same way.
+ *
  * Parity pins (the tests check this file against): Theorem 1 closed form,
  * the LTI convolution form, brute-force unrolling, an independent ZOH via the
  * matrix exponential, the exact ODE solution for a step input, finite
  * differences and autograd for the backward, and exact hand-derived values.
  */
+#include <complex.h>
 #include <math.h>
 #include <pthread.h>
 #include <stdlib.h>
@@ -535,5 +550,260 @@ int s6_oracle_dtproj_bwd(const double *u, const double *dt_low, const double *W_
   }
   free(delta);
   free(ddelta);
+  return rc;
+}
+
+/* ------------------------------------------------ complex diagonal A */
+
+typedef double complex cplx;
+
+/* psi(x) = (exp(x) - 1) / x for complex x; its series near 0. */
+static cplx cpsi(cplx x) {
+  if (cabs(x) < 1e-3) return 1.0 + x * (0.5 + x * (1.0 / 6.0 + x * (1.0 / 24.0 + x / 120.0)));
+  return (cexp(x) - 1.0) / x;
+}
+
+/* phi(x) = d psi / dx = (x e^x - (e^x - 1)) / x^2; its series near 0. */
+static cplx cphi(cplx x) {
+  if (cabs(x) < 1e-2)
+    return 0.5 + x * (1.0 / 3.0 + x * (1.0 / 8.0 + x * (1.0 / 30.0 + x * (1.0 / 144.0))));
+  return (x * cexp(x) - (cexp(x) - 1.0)) / (x * x);
+}
+
+/* element n of a planar complex row of N entries (stride between entries) */
+static cplx cget(const double *p, i64 n, i64 N, i64 stride) {
+  return p[n * stride] + I * p[(n + N) * stride];
+}
+
+typedef struct {
+  const double *u, *delta, *bias, *A, *B, *C, *D, *z, *dy;
+  double *y, *last_state, *du, *ddelta, *dz;
+  double *dA_part, *dD_part, *dbias_part, *dB_acc, *dC_acc;
+  i64 batch, dim, L, N, first, last;
+} cjob_t;
+
+static void cfwd_channel(const cjob_t *j, i64 b, i64 d, cplx *h) {
+  const i64 L = j->L, N = j->N, dim = j->dim;
+  const i64 off = (b * dim + d) * L;
+  const double *Bm = j->B + b * 2 * N * L, *Cm = j->C + b * 2 * N * L;
+  const double bias = j->bias ? j->bias[d] : 0.0;
+  for (i64 n = 0; n < N; ++n) h[n] = 0.0;
+  for (i64 t = 0; t < L; ++t) {
+    const double Delta = softplus(j->delta[off + t] + bias);
+    double y0 = 0.0;
+    for (i64 n = 0; n < N; ++n) {
+      const cplx An = cget(j->A + d * 2 * N, n, N, 1);
+      const cplx x = Delta * An;
+      const cplx Bbar = Delta * cpsi(x) * cget(Bm + t, n, N, L);
+      h[n] = cexp(x) * h[n] + Bbar * j->u[off + t];
+      y0 += creal(cget(Cm + t, n, N, L) * h[n]);
+    }
+    if (j->D) y0 += j->D[d] * j->u[off + t];
+    if (j->z) y0 *= j->z[off + t] * sigmoid(j->z[off + t]);
+    j->y[off + t] = y0;
+  }
+  if (j->last_state) {
+    double *ls = j->last_state + (b * dim + d) * 2 * N;
+    for (i64 n = 0; n < N; ++n) {
+      ls[n] = creal(h[n]);
+      ls[N + n] = cimag(h[n]);
+    }
+  }
+}
+
+static void *cfwd_worker(void *arg) {
+  cjob_t *j = (cjob_t *)arg;
+  cplx *h = (cplx *)malloc(sizeof(cplx) * (size_t)j->N);
+  for (i64 i = j->first; i < j->last; ++i) cfwd_channel(j, i / j->dim, i % j->dim, h);
+  free(h);
+  return NULL;
+}
+
+/* The adjoint of the complex forward, for the real loss sum(dy * y).  The
+ * gradient of a complex w is g = dl/d(re w) + i dl/d(im w); through a
+ * product v = a w it is conj(a) g_v, and through y = Re(c h) it is
+ * conj(c) dy.  So G_t = conj(C_t) dy0_t + conj(Abar_{t+1}) G_{t+1}, and with
+ * dh_t/dDelta = Abar (A h_{t-1} + B u), dh_t/dA = Delta Abar h_{t-1} +
+ * Delta^2 phi(x) B u:
+ *     du     += Re(conj(G) Bbar),        dDelta += Re(conj(G) dh/dDelta),
+ *     g_A    += conj(dh/dA) G,           g_B    += conj(Delta psi(x)) u G,
+ *     g_C    += conj(h_t) dy0. */
+static void cbwd_channel(cjob_t *j, i64 b, i64 d, cplx *H, cplx *G, cplx *Anext, cplx *gA) {
+  const i64 L = j->L, N = j->N, dim = j->dim;
+  const i64 off = (b * dim + d) * L;
+  const double *Bm = j->B + b * 2 * N * L, *Cm = j->C + b * 2 * N * L;
+  const double bias = j->bias ? j->bias[d] : 0.0;
+  const double Dd = j->D ? j->D[d] : 0.0;
+  for (i64 n = 0; n < N; ++n) H[n] = 0.0;
+  for (i64 t = 0; t < L; ++t) {
+    const double Delta = softplus(j->delta[off + t] + bias);
+    for (i64 n = 0; n < N; ++n) {
+      const cplx x = Delta * cget(j->A + d * 2 * N, n, N, 1);
+      H[(t + 1) * N + n] = cexp(x) * H[t * N + n] +
+                           Delta * cpsi(x) * cget(Bm + t, n, N, L) * j->u[off + t];
+    }
+  }
+  for (i64 n = 0; n < N; ++n) {
+    G[n] = 0.0;
+    Anext[n] = 0.0;
+    gA[n] = 0.0;
+  }
+  double dD = 0.0, dbias = 0.0;
+  for (i64 t = L - 1; t >= 0; --t) {
+    const double v = j->delta[off + t] + bias;
+    const double Delta = softplus(v);
+    const double ut = j->u[off + t];
+    double y0 = 0.0;
+    for (i64 n = 0; n < N; ++n) y0 += creal(cget(Cm + t, n, N, L) * H[(t + 1) * N + n]);
+    if (j->D) y0 += Dd * ut;
+    double dy0 = j->dy[off + t];
+    if (j->z) {
+      const double zt = j->z[off + t], sz = sigmoid(zt);
+      j->dz[off + t] = j->dy[off + t] * y0 * sz * (1.0 + zt * (1.0 - sz));
+      dy0 = j->dy[off + t] * zt * sz;
+    }
+    double du = j->D ? Dd * dy0 : 0.0, dDelta = 0.0;
+    if (j->D) dD += dy0 * ut;
+    for (i64 n = 0; n < N; ++n) {
+      const cplx An = cget(j->A + d * 2 * N, n, N, 1);
+      const cplx x = Delta * An;
+      const cplx Abar = cexp(x);
+      const cplx Bn = cget(Bm + t, n, N, L), Cn = cget(Cm + t, n, N, L);
+      const cplx hprev = H[t * N + n], hcur = H[(t + 1) * N + n];
+      G[n] = conj(Cn) * dy0 + conj(Anext[n]) * G[n];
+      Anext[n] = Abar;
+      const cplx E = Delta * cpsi(x); /* Bbar / B */
+      du += creal(conj(G[n]) * E * Bn);
+      dDelta += creal(conj(G[n]) * Abar * (An * hprev + Bn * ut));
+      gA[n] += conj(Delta * Abar * hprev + Delta * Delta * cphi(x) * Bn * ut) * G[n];
+      const cplx gB = conj(E) * ut * G[n];
+      const cplx gC = conj(hcur) * dy0;
+      j->dB_acc[(b * 2 * N + n) * L + t] += creal(gB);
+      j->dB_acc[(b * 2 * N + N + n) * L + t] += cimag(gB);
+      j->dC_acc[(b * 2 * N + n) * L + t] += creal(gC);
+      j->dC_acc[(b * 2 * N + N + n) * L + t] += cimag(gC);
+    }
+    const double dd = dDelta * sigmoid(v);
+    j->du[off + t] = du;
+    j->ddelta[off + t] = dd;
+    dbias += dd;
+  }
+  double *pa = j->dA_part + (b * dim + d) * 2 * N;
+  for (i64 n = 0; n < N; ++n) {
+    pa[n] = creal(gA[n]);
+    pa[N + n] = cimag(gA[n]);
+  }
+  j->dD_part[b * dim + d] = dD;
+  j->dbias_part[b * dim + d] = dbias;
+}
+
+static void *cbwd_worker(void *arg) {
+  cjob_t *j = (cjob_t *)arg;
+  const size_t N = (size_t)j->N;
+  cplx *H = (cplx *)malloc(sizeof(cplx) * (size_t)(j->L + 1) * N);
+  cplx *G = (cplx *)malloc(sizeof(cplx) * 3 * N);
+  for (i64 i = j->first; i < j->last; ++i) cbwd_channel(j, i / j->dim, i % j->dim, H, G, G + N, G + 2 * N);
+  free(H);
+  free(G);
+  return NULL;
+}
+
+static int run_cworkers(cjob_t *base, i64 nthreads, void *(*fn)(void *), int acc) {
+  const i64 total = base->batch * base->dim;
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > total) nthreads = total > 0 ? total : 1;
+  cjob_t *jobs = (cjob_t *)calloc((size_t)nthreads, sizeof(cjob_t));
+  pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+  if (!jobs || !th) { free(jobs); free(th); return -1; }
+  const size_t accn = (size_t)(base->batch * 2 * base->N * base->L);
+  int rc = 0;
+  for (i64 k = 0; k < nthreads; ++k) {
+    jobs[k] = *base;
+    jobs[k].first = total * k / nthreads;
+    jobs[k].last = total * (k + 1) / nthreads;
+    if (acc) {
+      jobs[k].dB_acc = (double *)calloc(accn ? accn : 1, sizeof(double));
+      jobs[k].dC_acc = (double *)calloc(accn ? accn : 1, sizeof(double));
+      if (!jobs[k].dB_acc || !jobs[k].dC_acc) rc = -1;
+    }
+  }
+  if (rc == 0) {
+    for (i64 k = 1; k < nthreads; ++k) pthread_create(&th[k], NULL, fn, &jobs[k]);
+    fn(&jobs[0]);
+    for (i64 k = 1; k < nthreads; ++k) pthread_join(th[k], NULL);
+  }
+  if (acc && rc == 0) {
+    for (size_t i = 0; i < accn; ++i) {
+      double sb = 0.0, sc = 0.0;
+      for (i64 k = 0; k < nthreads; ++k) { sb += jobs[k].dB_acc[i]; sc += jobs[k].dC_acc[i]; }
+      base->dB_acc[i] = sb;
+      base->dC_acc[i] = sc;
+    }
+  }
+  if (acc)
+    for (i64 k = 0; k < nthreads; ++k) { free(jobs[k].dB_acc); free(jobs[k].dC_acc); }
+  free(jobs);
+  free(th);
+  return rc;
+}
+
+/* Complex forward.  Layouts: u, delta, z, y (batch, dim, L); A (dim, 2N);
+ * B, C (batch, 2N, L); bias, D (dim); last_state (batch, dim, 2N); complex
+ * vectors planar (real parts first).  bias, D, z, last_state may be NULL. */
+int s6_oracle_cplx_fwd(const double *u, const double *delta, const double *bias, const double *A,
+                       const double *B, const double *C, const double *D, const double *z,
+                       double *y, double *last_state, i64 batch, i64 dim, i64 L, i64 N,
+                       i64 nthreads) {
+  if (batch < 0 || dim < 0 || L < 0 || N < 1 || N > 64) return -2;
+  cjob_t j;
+  memset(&j, 0, sizeof(j));
+  j.u = u; j.delta = delta; j.bias = bias; j.A = A; j.B = B; j.C = C; j.D = D; j.z = z;
+  j.y = y; j.last_state = last_state;
+  j.batch = batch; j.dim = dim; j.L = L; j.N = N;
+  if (batch * dim == 0) return 0;
+  return run_cworkers(&j, nthreads, cfwd_worker, 0);
+}
+
+/* Complex backward of sum(dy * y).  Outputs du, ddelta, dz (batch, dim, L);
+ * dA (dim, 2N); dB, dC (batch, 2N, L); dD, dbias (dim).  dz non-NULL iff z,
+ * dD iff D; dbias may be NULL. */
+int s6_oracle_cplx_bwd(const double *u, const double *delta, const double *bias, const double *A,
+                       const double *B, const double *C, const double *D, const double *z,
+                       const double *dy, double *du, double *ddelta, double *dA, double *dB,
+                       double *dC, double *dD, double *dz, double *dbias, i64 batch, i64 dim,
+                       i64 L, i64 N, i64 nthreads) {
+  if (batch < 0 || dim < 0 || L < 0 || N < 1 || N > 64) return -2;
+  if ((z == NULL) != (dz == NULL) || (D == NULL) != (dD == NULL)) return -2;
+  const size_t bd = (size_t)(batch * dim);
+  cjob_t j;
+  memset(&j, 0, sizeof(j));
+  j.u = u; j.delta = delta; j.bias = bias; j.A = A; j.B = B; j.C = C; j.D = D; j.z = z;
+  j.dy = dy; j.du = du; j.ddelta = ddelta; j.dz = dz;
+  j.batch = batch; j.dim = dim; j.L = L; j.N = N;
+  j.dB_acc = dB; j.dC_acc = dC;
+  memset(dB, 0, sizeof(double) * (size_t)(batch * 2 * N * L));
+  memset(dC, 0, sizeof(double) * (size_t)(batch * 2 * N * L));
+  memset(dA, 0, sizeof(double) * (size_t)(dim * 2 * N));
+  if (dD) memset(dD, 0, sizeof(double) * (size_t)dim);
+  if (dbias) memset(dbias, 0, sizeof(double) * (size_t)dim);
+  if (bd == 0) return 0;
+  j.dA_part = (double *)calloc(bd * 2 * (size_t)N, sizeof(double));
+  j.dD_part = (double *)calloc(bd, sizeof(double));
+  j.dbias_part = (double *)calloc(bd, sizeof(double));
+  int rc = -1;
+  if (j.dA_part && j.dD_part && j.dbias_part) {
+    rc = run_cworkers(&j, nthreads, cbwd_worker, 1);
+    if (rc == 0) {
+      for (i64 b = 0; b < batch; ++b)
+        for (i64 d = 0; d < dim; ++d) {
+          for (i64 n = 0; n < 2 * N; ++n) dA[d * 2 * N + n] += j.dA_part[(b * dim + d) * 2 * N + n];
+          if (dD) dD[d] += j.dD_part[b * dim + d];
+          if (dbias) dbias[d] += j.dbias_part[b * dim + d];
+        }
+    }
+  }
+  free(j.dA_part);
+  free(j.dD_part);
+  free(j.dbias_part);
   return rc;
 }

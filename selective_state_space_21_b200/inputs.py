@@ -31,6 +31,10 @@ depthwise Conv1d layer, fan-in W; the pages give none).
 For the low-rank Delta projection (section 3.6 of the paper-graph-ui page,
 s_Delta = Linear_D(Linear_R(x))) the rank-R input dt_low is N(0, 1) and the
 weight W_dt is N(0, 1/R), so that their product has delta's unit variance.
+
+For the complex-valued diagonal A (S4D-Lin, A_n = -1/2 + n i, Table 8 of the
+paper-graph-ui page's ablations) B and C are complex with N(0, 1/2) real and
+imaginary parts, stored planar (real parts first).
 """
 from __future__ import annotations
 
@@ -137,6 +141,27 @@ def make_dtproj_params(batch: int, dim: int, L: int, R: int, dtype: torch.dtype 
     dt_low = torch.randn(batch, R, L, generator=g, device=device).to(dtype)
     W = (torch.randn(dim, R, generator=g, device=device) / math.sqrt(R)).to(dtype)
     return {"dt_low": dt_low.contiguous(), "W_dt": W.contiguous()}
+
+
+def make_cplx_inputs(batch: int, dim: int, L: int, N: int, dtype: torch.dtype = torch.float32,
+                     device="cpu", seed: int = SEED_BASE, has_z: bool = True, has_D: bool = True,
+                     with_dy: bool = False) -> dict:
+    """Inputs for the complex-A scan: those of make_inputs (u, delta, z, D,
+    delta_bias, dy drawn the same way), with A = S4D-Lin, A[d, n] = -1/2 + n i,
+    and B, C complex with N(0, 1/2) real and imaginary parts.  Complex
+    vectors are planar, real parts first: A (dim, 2N) float32, B and C (batch,
+    2N, L) in the I/O dtype."""
+    x = make_inputs(batch, dim, L, N, dtype, device=device, seed=seed, has_z=has_z, has_D=has_D,
+                    with_dy=with_dy)
+    g = torch.Generator(device=device)
+    g.manual_seed(seed + 15485863)
+    s = math.sqrt(0.5)
+    x["B"] = (torch.randn(batch, 2 * N, L, generator=g, device=device) * s).to(dtype)
+    x["C"] = (torch.randn(batch, 2 * N, L, generator=g, device=device) * s).to(dtype)
+    n = torch.arange(N, device=device, dtype=torch.float32)
+    x["A"] = torch.cat([torch.full((dim, N), -0.5, device=device),
+                        n.repeat(dim, 1)], dim=1).contiguous()
+    return x
 
 
 def workload_inputs(index: int, device="cpu", with_dy: Optional[bool] = None) -> dict:

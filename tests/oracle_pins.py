@@ -20,7 +20,8 @@ import scipy.special
 import torch
 
 import oracle
-from selective_state_space_21_b200.inputs import gated_case, lti_case, make_conv_params, make_inputs
+from selective_state_space_21_b200.inputs import (gated_case, lti_case, make_conv_params,
+                                                  make_cplx_inputs, make_inputs)
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_derived_exact.txt")
 
@@ -579,13 +580,141 @@ def pin_dtproj_autograd(lib=None):
     return max(normwise(g["d_dt_low"], ref[0].numpy()), normwise(g["dW_dt"], ref[1].numpy())), 1e-12
 
 
+# ------------------------------------------------- complex diagonal A
+
+def _cplx(x, N):
+    """planar (..., 2N, ...) along axis -2 or -1 -> complex numpy array"""
+    return x[..., :N] + 1j * x[..., N:]
+
+
+def pin_cplx_real_case(lib=None):
+    """With zero imaginary parts the complex scan is the real one: y, the
+    state and the real-part gradients equal the (separately pinned) real
+    oracle's."""
+    xr = make_inputs(2, 3, 31, 4, seed=91, with_dy=True)
+    xr["A"] = xr["A"] * 0.6
+    N = 4
+    z2 = lambda t: torch.cat([t, torch.zeros_like(t)], dim=-2)  # (b, N, L) -> (b, 2N, L)
+    A2 = torch.cat([xr["A"], torch.zeros_like(xr["A"])], dim=1)
+    kw = dict(delta_bias=xr["delta_bias"], D=xr["D"], z=xr["z"], lib=lib)
+    y, last = oracle.s6_cplx_forward(xr["u"], xr["delta"], A2, z2(xr["B"]), z2(xr["C"]), **kw)
+    y_r, last_r = oracle.s6_forward(xr["u"], xr["delta"], xr["A"], xr["B"], xr["C"], **kw)
+    err = max(normwise(y, y_r), normwise(last[..., :N], last_r), float(np.abs(last[..., N:]).max()))
+    g = oracle.s6_cplx_backward(xr["u"], xr["delta"], A2, z2(xr["B"]), z2(xr["C"]), xr["dy"], **kw)
+    gr = oracle.s6_backward(xr["u"], xr["delta"], xr["A"], xr["B"], xr["C"], xr["dy"], **kw)
+    for k in ("du", "ddelta", "dz", "dD", "ddelta_bias"):
+        err = max(err, normwise(g[k], gr[k]))
+    err = max(err, normwise(g["dA"][:, :N], gr["dA"]))
+    for k in ("dB", "dC"):
+        err = max(err, normwise(g[k][:, :N], gr[k]))
+    return err, 1e-13
+
+
+def pin_cplx_zoh_expm(lib=None):
+    """Each complex state as the real 2-state system [[a, -b], [b, a]] with
+    input (Re B, Im B), discretized per step by scipy's matrix exponential of
+    the augmented matrix (Van Loan), and read out as Re(C h)."""
+    x = make_cplx_inputs(1, 2, 17, 3, seed=92)
+    N = 3
+    y, last = oracle.s6_cplx_forward(x["u"], x["delta"], x["A"], x["B"], x["C"], x["delta_bias"],
+                                     x["D"], x["z"], lib=lib)
+    u, dl, z = (_np(x[k])[0] for k in ("u", "delta", "z"))
+    A, B, C = _np(x["A"]), _np(x["B"])[0], _np(x["C"])[0]
+    bias, D = _np(x["delta_bias"]), _np(x["D"])
+    ref = np.empty((2, 17))
+    for d in range(2):
+        h = np.zeros((N, 2))
+        for t in range(17):
+            Delta = _softplus(dl[d, t] + bias[d])
+            y0 = D[d] * u[d, t]
+            for n in range(N):
+                a, b = A[d, n], A[d, N + n]
+                M = np.zeros((3, 3))
+                M[:2, :2] = [[a, -b], [b, a]]
+                M[:2, 2] = [B[n, t], B[N + n, t]]
+                E = scipy.linalg.expm(Delta * M)
+                h[n] = E[:2, :2] @ h[n] + E[:2, 2] * u[d, t]
+                y0 += C[n, t] * h[n, 0] - C[N + n, t] * h[n, 1]
+            ref[d, t] = y0 * z[d, t] * scipy.special.expit(z[d, t])
+    return normwise(y[0], ref), 1e-12
+
+
+def _cplx_fd_inputs():
+    x = make_cplx_inputs(1, 2, 9, 2, seed=93, with_dy=True)
+    return {k: (v.double() if v is not None else None) for k, v in x.items()}
+
+
+def _cplx_loss(x, lib):
+    y, _ = oracle.s6_cplx_forward(x["u"], x["delta"], x["A"], x["B"], x["C"], x["delta_bias"],
+                                  x["D"], x["z"], lib=lib, nthreads=1)
+    return float(np.sum(_np(x["dy"]) * y))
+
+
+def pin_cplx_finite_differences(lib=None):
+    """Central differences of sum(dy * y) over every real input, including
+    the real and imaginary parts of A, B and C."""
+    x = _cplx_fd_inputs()
+    g = oracle.s6_cplx_backward(x["u"], x["delta"], x["A"], x["B"], x["C"], x["dy"],
+                                x["delta_bias"], x["D"], x["z"], lib=lib, nthreads=1)
+    worst = 0.0
+    for name, gname in _GRAD_NAMES.items():
+        flat = x[name].reshape(-1)
+        fd = np.empty(x[name].shape)
+        for i in range(flat.numel()):
+            v = float(flat[i])
+            h = 1e-6 * max(1.0, abs(v))
+            flat[i] = v + h
+            lp = _cplx_loss(x, lib)
+            flat[i] = v - h
+            lm = _cplx_loss(x, lib)
+            flat[i] = v
+            fd.reshape(-1)[i] = (lp - lm) / (2.0 * h)
+        worst = max(worst, normwise(g[gname], fd))
+    return worst, 1e-6
+
+
+def pin_cplx_autograd(lib=None):
+    """The complex adjoint against torch.autograd of an independent complex128
+    forward (torch's gradient of a complex leaf under a real loss is
+    d/d re + i d/d im, the oracle's convention)."""
+    x = _cplx_fd_inputs()
+    N = x["A"].shape[1] // 2
+    to_c = lambda t: torch.complex(t[..., :N, :], t[..., N:, :]) if t.dim() == 3 else \
+        torch.complex(t[:, :N], t[:, N:])
+    Ac, Bc, Cc = to_c(x["A"]).requires_grad_(True), to_c(x["B"]).requires_grad_(True), \
+        to_c(x["C"]).requires_grad_(True)
+    leaves = {k: x[k].clone().requires_grad_(True) for k in ("u", "delta", "z", "D", "delta_bias")}
+    u, dl, z, D, bias = (leaves[k] for k in ("u", "delta", "z", "D", "delta_bias"))
+    Delta = torch.nn.functional.softplus(dl + bias[None, :, None], beta=1.0, threshold=1e9)
+    h = torch.zeros(u.shape[0], u.shape[1], N, dtype=torch.complex128)
+    ys = []
+    for t in range(u.shape[2]):
+        xa = Delta[:, :, t, None] * Ac[None]
+        Abar = torch.exp(xa)
+        Bbar = (Abar - 1.0) / Ac[None] * Bc[:, None, :, t]
+        h = Abar * h + Bbar * u[:, :, t, None]
+        y0 = (h * Cc[:, None, :, t]).sum(-1).real + D[None] * u[:, :, t]
+        ys.append(y0 * torch.nn.functional.silu(z[:, :, t]))
+    (torch.stack(ys, dim=-1) * x["dy"]).sum().backward()
+    g = oracle.s6_cplx_backward(x["u"], x["delta"], x["A"], x["B"], x["C"], x["dy"],
+                                x["delta_bias"], x["D"], x["z"], lib=lib, nthreads=1)
+    planar = lambda c, axis: torch.cat([c.real, c.imag], dim=axis).numpy()
+    worst = max(normwise(g["dA"], planar(Ac.grad, 1)), normwise(g["dB"], planar(Bc.grad, 1)),
+                normwise(g["dC"], planar(Cc.grad, 1)))
+    for k, gk in (("u", "du"), ("delta", "ddelta"), ("z", "dz"), ("D", "dD"),
+                  ("delta_bias", "ddelta_bias")):
+        worst = max(worst, normwise(g[gk], leaves[k].grad.numpy()))
+    return worst, 1e-10
+
+
 ALL_PINS = [pin_golden, pin_theorem1, pin_zoh_expm, pin_lti_convolution, pin_brute_force,
             pin_held_input_exact, pin_skip_and_gate, pin_large_delta_limit,
             pin_small_delta_limit, pin_structure, pin_finite_differences, pin_autograd,
             pin_threads_agree, pin_resume_from_state, pin_initial_state_decay,
             pin_conv_numpy, pin_conv_special_filters, pin_conv_finite_differences,
             pin_conv_autograd, pin_dtproj_matmul, pin_dtproj_finite_differences,
-            pin_dtproj_autograd]
+            pin_dtproj_autograd, pin_cplx_real_case, pin_cplx_zoh_expm,
+            pin_cplx_finite_differences, pin_cplx_autograd]
 
 
 def run_all(lib=None):

@@ -48,6 +48,14 @@ MUTATIONS = {
                                   "dW_dt[d * R + r] += g * W_dt[d * R + r];"),
     "bwd_dtproj_ddt_low_missing_W": ("d_dt_low[(b * R + r) * L + t] += W_dt[d * R + r] * g;",
                                      "d_dt_low[(b * R + r) * L + t] += g;"),
+    "cplx_readout_drops_imaginary_product": (
+        "y0 += creal(cget(Cm + t, n, N, L) * h[n]);",
+        "y0 += creal(cget(Cm + t, n, N, L)) * creal(h[n]);"),
+    "cplx_bwd_adjoint_without_conjugates": (
+        "G[n] = conj(Cn) * dy0 + conj(Anext[n]) * G[n];", "G[n] = Cn * dy0 + Anext[n] * G[n];"),
+    "cplx_bwd_dA_without_conjugate": (
+        "gA[n] += conj(Delta * Abar * hprev + Delta * Delta * cphi(x) * Bn * ut) * G[n];",
+        "gA[n] += (Delta * Abar * hprev + Delta * Delta * cphi(x) * Bn * ut) * G[n];"),
     "bwd_dC_uses_prev_state": ("dCacc[(b * N + n) * L + t] += dy0 * H[(t + 1) * N + n];",
                                "dCacc[(b * N + n) * L + t] += dy0 * H[t * N + n];"),
 }
