@@ -395,6 +395,8 @@ def run_ours(args, world, rank, device):
         result["conv_prologue"] = run_conv(w, x, device, peaks, steps=args.conv_steps)
     if not args.only and not args.no_dtproj:
         result["dt_projection"] = run_dtproj(w, x, device, steps=args.conv_steps)
+    if not args.only and not args.no_cplx:
+        result["complex_A"] = run_cplx(w, device, peaks, steps=3)
     if args.only:
         result["note"] = f"--only {args.only}: a profiling run, not a benchmark result"
     if not args.no_e2e and not args.only:
@@ -532,6 +534,61 @@ def run_dtproj(w, x, device, steps=10):
             "bwd_tc_per_s": w.token_channels / (bms * 1e-3), "steps": steps,
             "timing": "median of per-call CUDA events",
             "shape": f"dt_low (batch {w.batch}, R {R}, L {w.L}), W_dt ({w.dim}, {R})"}
+
+
+def run_cplx(w, device, peaks, steps=3):
+    """The workload's shape with a complex diagonal A (S4D-Lin) of N complex
+    states, complex B and C: mamba_cplx_scan_fwd / _bwd, timed per call with
+    CUDA events.  Bytes: the real scan's plus the doubled B, C (and dB, dC)
+    rows."""
+    from selective_state_space_21_b200 import scan
+    from selective_state_space_21_b200.inputs import make_cplx_inputs
+
+    x = make_cplx_inputs(w.batch, w.dim, w.L, w.N, w.dtype, device=device, seed=4323,
+                         with_dy=True)
+    f32 = dict(device=device, dtype=torch.float32)
+    y = torch.empty_like(x["u"])
+    g = {k: torch.empty_like(x[k]) for k in ("u", "delta", "z", "B", "C")}
+    dA = torch.empty(w.dim, 2 * w.N, **f32)
+    dD, db = torch.empty(w.dim, **f32), torch.empty(w.dim, **f32)
+
+    def fwd():
+        scan.mamba_cplx_scan_fwd(x["u"], x["delta"], x["delta_bias"], x["A"], x["B"], x["C"],
+                                 x["D"], x["z"], y, None)
+
+    def bwd():
+        scan.mamba_cplx_scan_bwd(x["u"], x["delta"], x["delta_bias"], x["A"], x["B"], x["C"],
+                                 x["D"], x["z"], x["dy"], g["u"], g["delta"], dA, g["B"], g["C"],
+                                 dD, g["z"], db)
+
+    fwd()
+    bwd()
+    torch.cuda.synchronize(device)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for k in range(steps):
+        ev[k][0].record()
+        fwd()
+        ev[k][1].record()
+        bwd()
+        ev[k][2].record()
+    torch.cuda.synchronize(device)
+    if scan.mamba_scan_stream_status() != 0:
+        raise RuntimeError("device error in the complex-A run")
+    fms = statistics.median(e[0].elapsed_time(e[1]) for e in ev)
+    bms = statistics.median(e[1].elapsed_time(e[2]) for e in ev)
+    s_io = w.io_bytes
+    bc = 2 * w.batch * (2 * w.N) * w.L * s_io
+    fb = 4 * s_io * w.token_channels + bc + 4 * (w.dim * 2 * w.N + 2 * w.dim)
+    bb = 7 * s_io * w.token_channels + 2 * bc + 8 * (w.dim * 2 * w.N + 2 * w.dim)
+    hbm = peaks["hbm_gbs"]
+    return {"fwd": {"ms": round(fms, 4), "gbs": round(fb / (fms * 1e-3) / 1e9, 1),
+                    "frac_hbm": round(fb / (fms * 1e-3) / 1e9 / hbm, 4),
+                    "tc_per_s": w.token_channels / (fms * 1e-3)},
+            "bwd": {"ms": round(bms, 4), "gbs": round(bb / (bms * 1e-3) / 1e9, 1),
+                    "frac_hbm": round(bb / (bms * 1e-3) / 1e9 / hbm, 4),
+                    "tc_per_s": w.token_channels / (bms * 1e-3)},
+            "steps": steps, "timing": "median of per-call CUDA events",
+            "shape": f"batch {w.batch} x dim {w.dim} x L {w.L}, {w.N} complex states"}
 
 
 def run_decode(w, x, device, peaks, steps=200):
@@ -725,6 +782,7 @@ def main(argv=None):
                     help="timed calls of the convolution-prologue and projection legs")
     ap.add_argument("--no-dtproj", action="store_true",
                     help="skip the Delta-projection timing")
+    ap.add_argument("--no-cplx", action="store_true", help="skip the complex-A timing")
     ap.add_argument("--only", choices=["fwd", "bwd"], default=None,
                     help="time one pass only (for profiling; not a benchmark result)")
     args = ap.parse_args(argv)

@@ -248,6 +248,44 @@ MAMBA_SCAN_API mamba_status_t mamba_dtproj_scan_bwd(
     const mamba_scan_options_t *options, mamba_stream_t stream);
 
 /*
+ * Forward with a complex-valued diagonal A ("Mamba: Linear-Time Sequence
+ * Modeling with Selective State Spaces", paper-graph-ui summary, section 3.6
+ * "Real vs. Complex parameters"; the S4D-Lin initialization A_n = -1/2 + n i
+ * of its Table 8 ablation).  A, B, C and the state are complex, u, delta, z
+ * and y real; the pages say no more, and the readings are: B_t and C_t are
+ * input-dependent complex vectors, the readout keeps the real part:
+ *     Abar = exp(Delta A_n),  Bbar = (exp(Delta A_n) - 1) / A_n * B_n,
+ *     h_n  = Abar h_n + Bbar u,   y = (Re(sum_n C_n h_n) + D u) * silu(z)
+ * A complex vector of N entries is stored planar, real parts first:
+ *   A          : (dim, 2N) float32
+ *   B, C       : (batch, 2N, L) dtype
+ *   last_state : (batch, dim, 2N) float32
+ * Everything else as in mamba_scan_fwd.  One thread per (batch, channel)
+ * with the B / C rows staged in shared memory; no chunking over time.
+ */
+MAMBA_SCAN_API mamba_status_t mamba_cplx_scan_fwd(const void *u, const void *delta,
+                                                  const float *delta_bias, const float *A,
+                                                  const void *B, const void *C, const float *D,
+                                                  const void *z, void *y, float *last_state,
+                                                  int64_t batch, int64_t dim, int64_t L, int64_t N,
+                                                  mamba_dtype_t dtype, mamba_stream_t stream);
+
+/*
+ * Backward of sum(dy * y) for mamba_cplx_scan_fwd, recomputing the states.
+ * As mamba_scan_bwd, with dA (dim, 2N) float32 and dB, dC (batch, 2N, L)
+ * dtype in the planar layout; the gradient of a complex input is the pair
+ * (d/d re, d/d im).  Reductions run in a fixed order.
+ */
+MAMBA_SCAN_API mamba_status_t mamba_cplx_scan_bwd(const void *u, const void *delta,
+                                                  const float *delta_bias, const float *A,
+                                                  const void *B, const void *C, const float *D,
+                                                  const void *z, const void *dy, void *du,
+                                                  void *ddelta, float *dA, void *dB, void *dC,
+                                                  float *dD, void *dz, float *ddelta_bias,
+                                                  int64_t batch, int64_t dim, int64_t L, int64_t N,
+                                                  mamba_dtype_t dtype, mamba_stream_t stream);
+
+/*
  * One decoding step: the recurrent mode of the selective SSM, one token per
  * call with constant work per token ("Mamba: Linear-Time Sequence Modeling
  * with Selective State Spaces", trishampatil.com walk-through, Part II

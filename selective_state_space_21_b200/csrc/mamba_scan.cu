@@ -14,6 +14,7 @@
 #include "bwd_staged.cuh"
 #include "common.cuh"
 #include "conv_bwd.cuh"
+#include "cplx.cuh"
 #include "dtproj.h"
 #include "decode.cuh"
 #include "fwd_reference.cuh"
@@ -215,6 +216,61 @@ struct BwdReferenceLauncher {
       const int64_t np = a.dim * a.N;
       const int64_t g = std::min<int64_t>((np + 255) / 256, 148 * 16);
       bwd_finalize_params_kernel<<<(unsigned)g, 256, 0, s>>>(a, w);
+      st = launch_status();
+    }
+    if (ws_free(ws, s) != cudaSuccess && st == MAMBA_OK) st = MAMBA_ERR_CUDA;
+    return st;
+  }
+};
+
+template <typename T, int NM>
+struct CplxFwdLauncher {
+  static mamba_status_t run(const CplxArgs &a, cudaStream_t s) {
+    const dim3 grid(unsigned((a.dim + kCplxThreads - 1) / kCplxThreads), unsigned(a.batch));
+    cplx_fwd_kernel<T, NM><<<grid, kCplxThreads, 0, s>>>(a);
+    return launch_status();
+  }
+};
+
+template <typename T, int NM>
+struct CplxBwdLauncher {
+  static mamba_status_t run(const CplxArgs &a, cudaStream_t s) {
+    CplxWork w;
+    w.n_blocks = (a.L + kCplxBwdTC - 1) / kCplxBwdTC;
+    w.n_dblk = (a.dim + kCplxBwdThreads - 1) / kCplxBwdThreads;
+    const size_t bd = size_t(a.batch * a.dim);
+    const size_t n_ckpt = bd * size_t(w.n_blocks) * 2 * NM;
+    const size_t n_bc = size_t(w.n_dblk) * size_t(a.batch) * 4 * kMaxN * size_t(a.L);
+    const size_t n_A = bd * 2 * size_t(a.N);
+    float *ws = nullptr;
+    if (ws_alloc(reinterpret_cast<void **>(&ws), (n_ckpt + n_bc + n_A + 2 * bd) * 4, s) != cudaSuccess) {
+      cudaGetLastError();
+      return MAMBA_ERR_OUT_OF_MEMORY;
+    }
+    w.ckpt = ws;
+    w.part_bc = w.ckpt + n_ckpt;
+    w.part_A = w.part_bc + n_bc;
+    w.part_D = w.part_A + n_A;
+    w.part_bias = w.part_D + bd;
+    const size_t smem = 4 * (size_t(kCplxBwdTC) * 2 * NM * kCplxBwdThreads +
+                             size_t(kCplxBwdTC) * 4 * NM + 2 * 4 * kMaxN * kCplxBwdTC);
+    mamba_status_t st = MAMBA_OK;
+    if (cudaFuncSetAttribute(cplx_bwd_kernel<T, NM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(smem)) != cudaSuccess)
+      st = MAMBA_ERR_CUDA;
+    if (st == MAMBA_OK) {
+      const dim3 grid(unsigned(w.n_dblk), unsigned(a.batch));
+      cplx_bwd_kernel<T, NM><<<grid, kCplxBwdThreads, smem, s>>>(a, w);
+      st = launch_status();
+    }
+    if (st == MAMBA_OK) {
+      const int64_t nbc = a.batch * 2 * a.N * a.L;
+      cplx_finalize_bc<T><<<unsigned(std::min<int64_t>((nbc + 255) / 256, 148 * 16)), 256, 0, s>>>(a, w);
+      st = launch_status();
+    }
+    if (st == MAMBA_OK) {
+      const int64_t np = a.dim * 2 * a.N;
+      cplx_finalize_params<<<unsigned(std::min<int64_t>((np + 255) / 256, 148 * 16)), 256, 0, s>>>(a, w);
       st = launch_status();
     }
     if (ws_free(ws, s) != cudaSuccess && st == MAMBA_OK) st = MAMBA_ERR_CUDA;
@@ -775,6 +831,105 @@ mamba_status_t mamba_dtproj_scan_bwd(const void *u, const void *dt_low, const vo
     st = MAMBA_ERR_CUDA;
   if (ws_free(ws, s) != cudaSuccess && st == MAMBA_OK) st = MAMBA_ERR_CUDA;
   return st;
+}
+
+// ------------------------------------------------ complex diagonal A
+
+mamba_status_t mamba_cplx_scan_fwd(const void *u, const void *delta, const float *delta_bias,
+                                   const float *A, const void *B, const void *C, const float *D,
+                                   const void *z, void *y, float *last_state, int64_t batch,
+                                   int64_t dim, int64_t L, int64_t N, mamba_dtype_t dtype,
+                                   mamba_stream_t stream) {
+  mamba_status_t st = check_shape(batch, dim, L, N, dtype);
+  if (st != MAMBA_OK) return st;
+  Checker ck;
+  if (cudaGetDevice(&ck.dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MAMBA_ERR_CUDA;
+  }
+  const size_t es = dtype_size(dtype);
+  const size_t nbdl = size_t(batch) * size_t(dim) * size_t(L);
+  const size_t nbnl = size_t(batch) * 2 * size_t(N) * size_t(L);
+  ck.buf(u, nbdl * es, es, true, false);
+  ck.buf(delta, nbdl * es, es, true, false);
+  ck.buf(z, nbdl * es, es, false, false);
+  ck.buf(B, nbnl * es, es, true, false);
+  ck.buf(C, nbnl * es, es, true, false);
+  ck.buf(A, size_t(dim) * 2 * N * 4, 4, true, false);
+  ck.buf(D, size_t(dim) * 4, 4, false, false);
+  ck.buf(delta_bias, size_t(dim) * 4, 4, false, false);
+  ck.buf(y, nbdl * es, es, true, true);
+  ck.buf(last_state, size_t(batch) * dim * 2 * N * 4, 4, false, true);
+  if (ck.st != MAMBA_OK) return ck.st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (batch == 0 || dim == 0) return MAMBA_OK;
+  if (L == 0) {
+    if (last_state && cudaMemsetAsync(last_state, 0, size_t(batch) * dim * 2 * N * 4, s) != cudaSuccess)
+      return cuda_status();
+    return MAMBA_OK;
+  }
+  if ((dim + kCplxThreads - 1) / kCplxThreads > (int64_t(1) << 31) - 1) return MAMBA_ERR_UNSUPPORTED;
+  CplxArgs a = {};
+  a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
+  a.bias = delta_bias; a.A = A; a.D = D; a.y = y; a.last_state = last_state;
+  a.batch = batch; a.dim = dim; a.L = L; a.N = (int)N;
+  return dispatch<CplxFwdLauncher>(dtype, (int)N, a, s);
+}
+
+mamba_status_t mamba_cplx_scan_bwd(const void *u, const void *delta, const float *delta_bias,
+                                   const float *A, const void *B, const void *C, const float *D,
+                                   const void *z, const void *dy, void *du, void *ddelta,
+                                   float *dA, void *dB, void *dC, float *dD, void *dz,
+                                   float *ddelta_bias, int64_t batch, int64_t dim, int64_t L,
+                                   int64_t N, mamba_dtype_t dtype, mamba_stream_t stream) {
+  mamba_status_t st = check_shape(batch, dim, L, N, dtype);
+  if (st != MAMBA_OK) return st;
+  if ((z == nullptr) != (dz == nullptr) || (D == nullptr) != (dD == nullptr))
+    return MAMBA_ERR_INVALID_ARG;
+  Checker ck;
+  if (cudaGetDevice(&ck.dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MAMBA_ERR_CUDA;
+  }
+  const size_t es = dtype_size(dtype);
+  const size_t nbdl = size_t(batch) * size_t(dim) * size_t(L);
+  const size_t nbnl = size_t(batch) * 2 * size_t(N) * size_t(L);
+  ck.buf(u, nbdl * es, es, true, false);
+  ck.buf(delta, nbdl * es, es, true, false);
+  ck.buf(z, nbdl * es, es, false, false);
+  ck.buf(dy, nbdl * es, es, true, false);
+  ck.buf(B, nbnl * es, es, true, false);
+  ck.buf(C, nbnl * es, es, true, false);
+  ck.buf(A, size_t(dim) * 2 * N * 4, 4, true, false);
+  ck.buf(D, size_t(dim) * 4, 4, false, false);
+  ck.buf(delta_bias, size_t(dim) * 4, 4, false, false);
+  ck.buf(du, nbdl * es, es, true, true);
+  ck.buf(ddelta, nbdl * es, es, true, true);
+  ck.buf(dz, nbdl * es, es, false, true);
+  ck.buf(dB, nbnl * es, es, true, true);
+  ck.buf(dC, nbnl * es, es, true, true);
+  ck.buf(dA, size_t(dim) * 2 * N * 4, 4, true, true);
+  ck.buf(dD, size_t(dim) * 4, 4, false, true);
+  ck.buf(ddelta_bias, size_t(dim) * 4, 4, false, true);
+  if (ck.st != MAMBA_OK) return ck.st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (dim == 0) return MAMBA_OK;
+  if (batch == 0 || L == 0) {
+    if (cudaMemsetAsync(dA, 0, size_t(dim) * 2 * N * 4, s) != cudaSuccess ||
+        (dD && cudaMemsetAsync(dD, 0, size_t(dim) * 4, s) != cudaSuccess) ||
+        (ddelta_bias && cudaMemsetAsync(ddelta_bias, 0, size_t(dim) * 4, s) != cudaSuccess))
+      return cuda_status();
+    return MAMBA_OK;
+  }
+  if ((dim + kCplxBwdThreads - 1) / kCplxBwdThreads > (int64_t(1) << 31) - 1)
+    return MAMBA_ERR_UNSUPPORTED;
+  CplxArgs a = {};
+  a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C; a.dy = dy;
+  a.bias = delta_bias; a.A = A; a.D = D;
+  a.du = du; a.ddelta = ddelta; a.dz = dz; a.dB = dB; a.dC = dC;
+  a.dA = dA; a.dD = dD; a.dbias = ddelta_bias;
+  a.batch = batch; a.dim = dim; a.L = L; a.N = (int)N;
+  return dispatch<CplxBwdLauncher>(dtype, (int)N, a, s);
 }
 
 }  // extern "C"

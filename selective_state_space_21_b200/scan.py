@@ -5,7 +5,8 @@ CPU fallback; a missing library or device raises.
 Low-level calls (same names and argument order as ``include/mamba_scan.h``):
 ``mamba_scan_fwd``, ``mamba_scan_bwd``, ``mamba_conv_scan_fwd``,
 ``mamba_conv_scan_bwd``, ``mamba_dtproj_scan_fwd``, ``mamba_dtproj_scan_bwd``,
-``mamba_scan_step``, ``mamba_scan_fwd_noalloc``,
+``mamba_cplx_scan_fwd``, ``mamba_cplx_scan_bwd``, ``mamba_scan_step``,
+``mamba_scan_fwd_noalloc``,
 ``mamba_scan_stream_status``.  Convenience wrappers that allocate the outputs:
 ``selective_scan_fwd``, ``selective_scan_bwd``, ``conv_selective_scan_fwd``
 and ``conv_selective_scan_bwd``.
@@ -76,6 +77,10 @@ def load_library():
             lib.mamba_dtproj_scan_fwd.restype = ctypes.c_int
             lib.mamba_dtproj_scan_bwd.argtypes = [vp] * 3 + [i64] + [vp] * 16 + [i64] * 4 + [i32, opt, vp]
             lib.mamba_dtproj_scan_bwd.restype = ctypes.c_int
+            lib.mamba_cplx_scan_fwd.argtypes = [vp] * 10 + [i64] * 4 + [i32, vp]
+            lib.mamba_cplx_scan_fwd.restype = ctypes.c_int
+            lib.mamba_cplx_scan_bwd.argtypes = [vp] * 17 + [i64] * 4 + [i32, vp]
+            lib.mamba_cplx_scan_bwd.restype = ctypes.c_int
             for f in ("mamba_scan_fwd", "mamba_scan_fwd_ex", "mamba_scan_bwd",
                       "mamba_scan_bwd_ex", "mamba_scan_stream_status", "mamba_scan_fwd_noalloc"):
                 getattr(lib, f).restype = ctypes.c_int
@@ -298,6 +303,49 @@ def mamba_dtproj_scan_bwd(u, dt_low, W_dt, delta_bias, A, B, C, D, z, dy, du, d_
     opts = _opts_ptr(path, chunk_len, "auto", wait_timeout_us, test_hook)
     _check(load_library().mamba_dtproj_scan_bwd(*args, opts, _stream_handle(stream)),
            "mamba_dtproj_scan_bwd")
+
+
+def mamba_cplx_scan_fwd(u, delta, delta_bias, A, B, C, D, z, y, last_state, *, stream=None):
+    """Enqueue the forward with a complex diagonal A.  Complex vectors are
+    planar, real parts first: A (dim, 2N) float32, B and C (batch, 2N, L) in
+    the I/O dtype, last_state (batch, dim, 2N) float32."""
+    batch, dim, L = u.shape
+    N = A.shape[1] // 2
+    dt = u.dtype
+    f32 = torch.float32
+    bdl, bnl = (batch, dim, L), (batch, 2 * N, L)
+    args = [
+        _ptr(u, dt, bdl, "u"), _ptr(delta, dt, bdl, "delta"),
+        _ptr(delta_bias, f32, (dim,), "delta_bias"), _ptr(A, f32, (dim, 2 * N), "A"),
+        _ptr(B, dt, bnl, "B"), _ptr(C, dt, bnl, "C"), _ptr(D, f32, (dim,), "D"),
+        _ptr(z, dt, bdl, "z"), _ptr(y, dt, bdl, "y"),
+        _ptr(last_state, f32, (batch, dim, 2 * N), "last_state"), batch, dim, L, N,
+        _dtype_code(dt)]
+    _check(load_library().mamba_cplx_scan_fwd(*args, _stream_handle(stream)),
+           "mamba_cplx_scan_fwd")
+
+
+def mamba_cplx_scan_bwd(u, delta, delta_bias, A, B, C, D, z, dy, du, ddelta, dA, dB, dC, dD, dz,
+                        ddelta_bias, *, stream=None):
+    """Enqueue the backward of sum(dy * y) for ``mamba_cplx_scan_fwd``; dA
+    (dim, 2N) float32 and dB, dC (batch, 2N, L) hold (d/d re, d/d im) pairs,
+    planar."""
+    batch, dim, L = u.shape
+    N = A.shape[1] // 2
+    dt = u.dtype
+    f32 = torch.float32
+    bdl, bnl = (batch, dim, L), (batch, 2 * N, L)
+    args = [
+        _ptr(u, dt, bdl, "u"), _ptr(delta, dt, bdl, "delta"),
+        _ptr(delta_bias, f32, (dim,), "delta_bias"), _ptr(A, f32, (dim, 2 * N), "A"),
+        _ptr(B, dt, bnl, "B"), _ptr(C, dt, bnl, "C"), _ptr(D, f32, (dim,), "D"),
+        _ptr(z, dt, bdl, "z"), _ptr(dy, dt, bdl, "dy"), _ptr(du, dt, bdl, "du"),
+        _ptr(ddelta, dt, bdl, "ddelta"), _ptr(dA, f32, (dim, 2 * N), "dA"),
+        _ptr(dB, dt, bnl, "dB"), _ptr(dC, dt, bnl, "dC"), _ptr(dD, f32, (dim,), "dD"),
+        _ptr(dz, dt, bdl, "dz"), _ptr(ddelta_bias, f32, (dim,), "ddelta_bias"),
+        batch, dim, L, N, _dtype_code(dt)]
+    _check(load_library().mamba_cplx_scan_bwd(*args, _stream_handle(stream)),
+           "mamba_cplx_scan_bwd")
 
 
 def mamba_scan_fwd_noalloc(u, delta, delta_bias, A, B, C, D, z, y, last_state, *, stream=None):

@@ -1,0 +1,154 @@
+"""GPU parity of the complex-A scan (mamba_cplx_scan_fwd / _bwd, S4D-Lin
+A_n = -1/2 + n i, complex B and C) against the fp64 oracle on the same seeded
+inputs.  Normwise max error <= 1e-4 for fp32 I/O and <= 2e-2 for bf16 I/O."""
+import pytest
+import torch
+
+import gpu_cases as gc
+import oracle
+from selective_state_space_21_b200 import build, scan
+from selective_state_space_21_b200.inputs import WORKLOADS, make_cplx_inputs, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+GRADS = ("du", "ddelta", "dA", "dB", "dC", "dD", "dz", "ddelta_bias")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    build.build()
+    scan.load_library()
+
+
+def gpu_fwd(x):
+    batch, dim, L = x["u"].shape
+    y = torch.empty_like(x["u"])
+    last = torch.empty(batch, dim, x["A"].shape[1], device="cuda")
+    scan.mamba_cplx_scan_fwd(x["u"], x["delta"], x["delta_bias"], x["A"], x["B"], x["C"], x["D"],
+                             x["z"], y, last)
+    assert scan.mamba_scan_stream_status() == 0
+    return y, last
+
+
+def gpu_bwd(x):
+    dim, N2 = x["A"].shape
+    f32 = dict(device="cuda", dtype=torch.float32)
+    g = {"du": torch.empty_like(x["u"]), "ddelta": torch.empty_like(x["u"]),
+         "dA": torch.empty(dim, N2, **f32), "dB": torch.empty_like(x["B"]),
+         "dC": torch.empty_like(x["C"]),
+         "dD": torch.empty(dim, **f32) if x["D"] is not None else None,
+         "dz": torch.empty_like(x["u"]) if x["z"] is not None else None,
+         "ddelta_bias": torch.empty(dim, **f32)}
+    scan.mamba_cplx_scan_bwd(x["u"], x["delta"], x["delta_bias"], x["A"], x["B"], x["C"], x["D"],
+                             x["z"], x["dy"], g["du"], g["ddelta"], g["dA"], g["dB"], g["dC"],
+                             g["dD"], g["dz"], g["ddelta_bias"])
+    assert scan.mamba_scan_stream_status() == 0
+    return {k: v for k, v in g.items() if v is not None}
+
+
+def check(xh, fwd=True, bwd=True):
+    x = gc.to_device(xh)
+    tol = gc.TOL[xh["u"].dtype]
+    args = (xh["u"], xh["delta"], xh["A"], xh["B"], xh["C"])
+    kw = dict(delta_bias=xh["delta_bias"], D=xh["D"], z=xh["z"])
+    if fwd:
+        y, last = gpu_fwd(x)
+        y_ref, last_ref = oracle.s6_cplx_forward(*args, **kw)
+        ey = gc.normwise(y.cpu().double().numpy(), y_ref)
+        el = gc.normwise(last.cpu().double().numpy(), last_ref)
+        assert ey <= tol and el <= max(tol, 1e-4), f"y err {ey:.2e}, last_state err {el:.2e}"
+    if bwd:
+        g = gpu_bwd(x)
+        ref = oracle.s6_cplx_backward(*args, xh["dy"], **kw)
+        errs = {k: gc.normwise(g[k].cpu().double().numpy(), ref[k]) for k in GRADS if k in g}
+        assert set(errs) == {k for k in GRADS if k in ref}
+        bad = {k: v for k, v in errs.items() if not v <= tol}
+        assert not bad, f"gradient errors above {tol}: {bad} (all: {errs})"
+
+
+SHAPES = [(2, 200, 300, 16), (1, 70, 129, 8), (3, 5, 40, 1), (2, 130, 77, 4), (1, 33, 20, 3)]
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_cplx_grid(shape, dtype):
+    b, d, L, N = shape
+    check(make_cplx_inputs(b, d, L, N, dtype, seed=1300 + L + d, with_dy=True))
+
+
+def test_cplx_without_gate_and_skip():
+    x = make_cplx_inputs(2, 96, 100, 16, torch.float32, seed=1390, has_z=False, has_D=False,
+                         with_dy=True)
+    x["delta_bias"] = None
+    check(x)
+
+
+def test_cplx_random_complex_A():
+    """A with random negative real parts and imaginary parts of either sign
+    (not the S4D-Lin pattern), including small |Delta A| where psi and phi
+    take their series."""
+    x = make_cplx_inputs(2, 64, 90, 8, torch.float32, seed=1391, with_dy=True)
+    g = torch.Generator().manual_seed(9)
+    re = -torch.exp(torch.randn(64, 8, generator=g) * 1.5)
+    im = torch.randn(64, 8, generator=g) * 3.0
+    re[0, :2] = -1e-4
+    im[0, :2] = 0.0
+    x["A"] = torch.cat([re, im], dim=1).contiguous()
+    check(x)
+
+
+def test_cplx_real_case_matches_real_scan():
+    """Zero imaginary parts: the complex kernels give the real kernels' y and
+    gradients."""
+    xr = gc.to_device(make_inputs(2, 150, 256, 8, torch.float32, seed=1392, with_dy=True))
+    z2 = lambda t: torch.cat([t, torch.zeros_like(t)], dim=1).contiguous()
+    xc = dict(xr, A=z2(xr["A"]), B=z2(xr["B"]), C=z2(xr["C"]))
+    y, last = gpu_fwd(xc)
+    y_r, last_r = gc.gpu_fwd(xr, path="reference")
+    assert gc.normwise(y.cpu().numpy(), y_r.cpu().numpy()) <= 1e-5
+    assert gc.normwise(last[..., :8].cpu().numpy(), last_r.cpu().numpy()) <= 1e-5
+    g = gpu_bwd(xc)
+    gr = gc.gpu_bwd(xr, path="reference")
+    for k in ("du", "ddelta", "dz", "dD", "ddelta_bias"):
+        assert gc.normwise(g[k].cpu().numpy(), gr[k].cpu().numpy()) <= 1e-4, k
+    assert gc.normwise(g["dA"][:, :8].cpu().numpy(), gr["dA"].cpu().numpy()) <= 1e-4
+    for k in ("dB", "dC"):
+        assert gc.normwise(g[k][:, :8].cpu().numpy(), gr[k].cpu().numpy()) <= 1e-4, k
+
+
+def test_cplx_bwd_deterministic():
+    x = gc.to_device(make_cplx_inputs(2, 300, 200, 16, torch.bfloat16, seed=1393, with_dy=True))
+    g1, g2 = gpu_bwd(x), gpu_bwd(x)
+    for k in g1:
+        assert torch.equal(g1[k], g2[k]), k
+
+
+def test_cplx_full_size_sampled():
+    """The bf16 4 x 2048 x 4096 workload shape with 16 complex states: y and
+    du, ddelta on sampled channels against the oracle."""
+    w = WORKLOADS[4]
+    xh = make_cplx_inputs(w.batch, w.dim, w.L, w.N, w.dtype, seed=1394, with_dy=True)
+    x = gc.to_device(xh)
+    y, _ = gpu_fwd(x)
+    g = gpu_bwd(x)
+    tol = gc.TOL[w.dtype]
+    yh, gh = y.cpu(), {k: v.cpu() for k, v in g.items()}
+    per_d = lambda t, idx: None if t is None else t.index_select(0, idx).contiguous()
+    for b, ds in gc.sample_channels(w.batch, w.dim, 8, seed=4).items():
+        idx = torch.tensor(ds)
+        sub = {k: (None if xh[k] is None else xh[k][b:b + 1].index_select(1, idx).contiguous())
+               for k in ("u", "delta", "z", "dy")}
+        sub.update(B=xh["B"][b:b + 1].contiguous(), C=xh["C"][b:b + 1].contiguous(),
+                   A=per_d(xh["A"], idx), D=per_d(xh["D"], idx),
+                   delta_bias=per_d(xh["delta_bias"], idx))
+        args = (sub["u"], sub["delta"], sub["A"], sub["B"], sub["C"])
+        kw = dict(delta_bias=sub["delta_bias"], D=sub["D"], z=sub["z"])
+        y_ref, _ = oracle.s6_cplx_forward(*args, **kw)
+        e = gc.normwise(yh[b].index_select(0, idx).double().numpy(), y_ref[0])
+        assert e <= tol, f"y (batch {b}): {e:.2e}"
+        ref = oracle.s6_cplx_backward(*args, sub["dy"], **kw)
+        for k in ("du", "ddelta", "dz"):
+            e = gc.normwise(gh[k][b].index_select(0, idx).double().numpy(), ref[k][0])
+            assert e <= tol, f"{k} (batch {b}): {e:.2e}"
