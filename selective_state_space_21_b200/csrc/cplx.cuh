@@ -16,8 +16,8 @@
 // over time; a CTA holds channels of one batch row, so the B and C rows of a
 // step are shared: they are staged per tile of steps in shared memory as
 // fp32 tables.  Each state costs three special-function operations per step
-// (exp of the real part, sine and cosine of the range-reduced imaginary
-// part) and about 25 FP32 operations.
+// (exp of the real part, sine and cosine of the range-reduced half of the
+// imaginary part) and about 35 FP32 operations, without branches.
 //
 // The backward follows the real one-thread-per-channel kernel: a forward
 // sweep keeps the state at the start of every block of steps, the reverse
@@ -32,6 +32,7 @@
 #pragma once
 
 #include "bwd_reference.cuh"
+#include "bwd_staged.cuh"
 #include "common.cuh"
 #include "fwd_staged.cuh"
 
@@ -52,66 +53,61 @@ constexpr int kCplxBwdThreads = 64;
 constexpr int kCplxBwdTC = 8;       // steps per recomputed block (backward)
 
 // exp(Delta a) and E = (exp(Delta a) - 1)/a = Delta psi(Delta a) for complex
-// a = ar + i ai (ira + i iai = 1/a).  The imaginary part of the exponent is
-// reduced to [-pi, pi] before the hardware sine and cosine; psi takes its
-// Taylor series where |Delta a| < 1/4 (the direct form cancels there).
+// a = ar + i ai (ira + i iai = 1/a), without branches.  With x = Delta a,
+//     exp(x) - 1 = (expm1(Re x) - 2 e^{Re x} sin^2(Im x / 2))
+//                  + i 2 e^{Re x} sin(Im x / 2) cos(Im x / 2),
+// which has no cancellation anywhere: expm1 takes its Taylor series below
+// |Re x| = 1/4 and the sine of the half angle (reduced to [-pi, pi]) its
+// series below 1/2, so that small arguments keep their relative accuracy.
+// a = 0 gives E = Delta (the limit).
 __device__ __forceinline__ void cplx_decay(float Delta, float ar, float ai, float ira, float iai,
                                            float &abr, float &abi, float &Er, float &Ei) {
   const float xr = Delta * ar, xi = Delta * ai;
-  const float mag = ex2f(xr * kLog2e);
-  const float k = rintf(xi * 0.15915494309189535f);
-  float r = fmaf(-k, 6.28318548202514648f, xi);
+  const float e = ex2f(xr * kLog2e);
+  const float pm = xr * (1.f + xr * (0.5f + xr * (1.f / 6.f + xr * (1.f / 24.f + xr * (1.f / 120.f +
+                   xr * (1.f / 720.f))))));
+  const float em1 = fabsf(xr) < 0.25f ? pm : e - 1.f;
+  const float hh = 0.5f * xi;
+  const float k = rintf(hh * 0.15915494309189535f);
+  float r = fmaf(-k, 6.28318548202514648f, hh);
   r = fmaf(-k, -1.7484556e-7f, r);  // 2 pi = 6.28318548 - 1.7484556e-7
-  float s, c;
-  __sincosf(r, &s, &c);
-  abr = mag * c;
-  abi = mag * s;
-  if (xr * xr + xi * xi < 0.0625f) {
-    // psi(x) = 1 + x/2 + x^2/6 + x^3/24 + x^4/120 + x^5/720
-    float pr = 1.f / 720.f, pi = 0.f;
-    const float cs[5] = {1.f / 120.f, 1.f / 24.f, 1.f / 6.f, 0.5f, 1.f};
-#pragma unroll
-    for (int j = 0; j < 5; ++j) {
-      const float tr = fmaf(pr, xr, fmaf(-pi, xi, cs[j]));
-      const float ti = fmaf(pr, xi, pi * xr);
-      pr = tr;
-      pi = ti;
-    }
-    Er = Delta * pr;
-    Ei = Delta * pi;
-  } else {
-    const float mr = abr - 1.f;
-    Er = fmaf(mr, ira, -abi * iai);
-    Ei = fmaf(mr, iai, abi * ira);
-  }
+  float s2, c2;
+  __sincosf(r, &s2, &c2);
+  const float r2 = r * r;
+  const float ps = r * (1.f - r2 * (1.f / 6.f - r2 * (1.f / 120.f - r2 * (1.f / 5040.f))));
+  s2 = fabsf(r) < 0.5f ? ps : s2;
+  const float es = 2.f * e * s2;
+  const float mr = fmaf(-es, s2, em1), mi = es * c2;
+  abr = 1.f + mr;
+  abi = mi;
+  const bool zero = ira == 0.f && iai == 0.f;
+  Er = zero ? Delta : fmaf(mr, ira, -mi * iai);
+  Ei = zero ? 0.f : fmaf(mr, iai, mi * ira);
 }
 
 // phi(x) = (x e^x - (e^x - 1)) / x^2 for complex x, from e^x = (er, ei);
 // its Taylor series where |x| < 1/4.
 __device__ __forceinline__ void cplx_phi(float xr, float xi, float er, float ei, float &pr,
                                          float &pi) {
-  if (xr * xr + xi * xi < 0.0625f) {
-    // sum_k (k+1)/(k+2)! x^k, k = 0..5
-    float ar = 1.f / 840.f, ai = 0.f;
-    const float cs[5] = {1.f / 144.f, 1.f / 30.f, 0.125f, 1.f / 3.f, 0.5f};
+  // both forms, then a select: no divergence between the channels of a warp
+  // sum_k (k+1)/(k+2)! x^k, k = 0..5
+  float ar = 1.f / 840.f, ai = 0.f;
+  const float cs[5] = {1.f / 144.f, 1.f / 30.f, 0.125f, 1.f / 3.f, 0.5f};
 #pragma unroll
-    for (int j = 0; j < 5; ++j) {
-      const float tr = fmaf(ar, xr, fmaf(-ai, xi, cs[j]));
-      const float ti = fmaf(ar, xi, ai * xr);
-      ar = tr;
-      ai = ti;
-    }
-    pr = ar;
-    pi = ai;
-  } else {
-    // numerator x e^x - e^x + 1, divided by x^2
-    const float nr = fmaf(xr, er, -xi * ei) - er + 1.f;
-    const float ni = fmaf(xr, ei, xi * er) - ei;
-    const float x2r = fmaf(xr, xr, -xi * xi), x2i = 2.f * xr * xi;
-    const float den = 1.f / fmaf(x2r, x2r, x2i * x2i);
-    pr = fmaf(nr, x2r, ni * x2i) * den;
-    pi = fmaf(ni, x2r, -nr * x2i) * den;
+  for (int j = 0; j < 5; ++j) {
+    const float tr = fmaf(ar, xr, fmaf(-ai, xi, cs[j]));
+    const float ti = fmaf(ar, xi, ai * xr);
+    ar = tr;
+    ai = ti;
   }
+  // numerator x e^x - e^x + 1, divided by x^2
+  const float nr = fmaf(xr, er, -xi * ei) - er + 1.f;
+  const float ni = fmaf(xr, ei, xi * er) - ei;
+  const float x2r = fmaf(xr, xr, -xi * xi), x2i = 2.f * xr * xi;
+  const float den = rcpf(fmaf(x2r, x2r, x2i * x2i));
+  const bool small = xr * xr + xi * xi < 0.0625f;
+  pr = small ? ar : fmaf(nr, x2r, ni * x2i) * den;
+  pi = small ? ai : fmaf(ni, x2r, -nr * x2i) * den;
 }
 
 // Stages the B and C columns of steps [t0, t0 + TT) of batch row b into
@@ -135,12 +131,17 @@ __device__ __forceinline__ void cplx_stage_bc(const CplxArgs &a, int64_t b, int6
   }
 }
 
-template <typename T, int NM>
+// TPC threads share one channel, NM / TPC states each (adjacent lanes; their
+// partial readouts are joined by shuffles): with few channels per SM, more
+// threads per channel hide more of the recurrence's latency.
+template <typename T, int NM, int TPC>
 __global__ void __launch_bounds__(kCplxThreads) cplx_fwd_kernel(const CplxArgs a) {
+  constexpr int NS = NM / TPC;  // states per thread
   __shared__ __align__(16) float tab[kCplxTT * 4 * NM];
   const int tid = threadIdx.x;
+  const int part = tid % TPC;
   const int64_t b = blockIdx.y;
-  const int64_t d_raw = int64_t(blockIdx.x) * kCplxThreads + tid;
+  const int64_t d_raw = int64_t(blockIdx.x) * (kCplxThreads / TPC) + tid / TPC;
   const bool valid = d_raw < a.dim;
   const int64_t d = valid ? d_raw : a.dim - 1;
   const int64_t row = (b * a.dim + d) * a.L;
@@ -150,16 +151,17 @@ __global__ void __launch_bounds__(kCplxThreads) cplx_fwd_kernel(const CplxArgs a
   const T *z = a.z ? static_cast<const T *>(a.z) + row : nullptr;
   T *y = static_cast<T *>(a.y) + row;
   const float bias = a.bias ? a.bias[d] : 0.f;
-  const float Dd = a.D ? a.D[d] : 0.f;
-  float ar[NM], ai[NM], ira[NM], iai[NM], hr[NM], hi[NM];
+  const float Dd = (a.D && part == 0) ? a.D[d] : 0.f;
+  float ar[NS], ai[NS], ira[NS], iai[NS], hr[NS], hi[NS];
 #pragma unroll
-  for (int n = 0; n < NM; ++n) {
-    ar[n] = n < N ? a.A[d * 2 * N + n] : -1.f;
-    ai[n] = n < N ? a.A[d * 2 * N + N + n] : 0.f;
-    const float m = ar[n] * ar[n] + ai[n] * ai[n];
-    ira[n] = m > 0.f ? ar[n] / m : 0.f;
-    iai[n] = m > 0.f ? -ai[n] / m : 0.f;
-    hr[n] = hi[n] = 0.f;
+  for (int j = 0; j < NS; ++j) {
+    const int n = part * NS + j;
+    ar[j] = n < N ? a.A[d * 2 * N + n] : -1.f;
+    ai[j] = n < N ? a.A[d * 2 * N + N + n] : 0.f;
+    const float m = ar[j] * ar[j] + ai[j] * ai[j];
+    ira[j] = m > 0.f ? ar[j] / m : 0.f;
+    iai[j] = m > 0.f ? -ai[j] / m : 0.f;
+    hr[j] = hi[j] = 0.f;
   }
   for (int64_t t0 = 0; t0 < a.L; t0 += kCplxTT) {
     __syncthreads();
@@ -170,36 +172,40 @@ __global__ void __launch_bounds__(kCplxThreads) cplx_fwd_kernel(const CplxArgs a
       const int64_t t = t0 + i;
       const float Delta = softplus_fast(to_f(dl[t]) + bias);
       const float ut = to_f(u[t]);
-      const float *tr = tab + i * 4 * NM;
+      const float *tr = tab + i * 4 * NM + part * NS;
       float y0 = Dd * ut;
 #pragma unroll
-      for (int n = 0; n < NM; ++n) {
+      for (int j = 0; j < NS; ++j) {
         float abr, abi, Er, Ei;
-        cplx_decay(Delta, ar[n], ai[n], ira[n], iai[n], abr, abi, Er, Ei);
-        const float br = tr[n], bi = tr[NM + n], cr = tr[2 * NM + n], ci = tr[3 * NM + n];
+        cplx_decay(Delta, ar[j], ai[j], ira[j], iai[j], abr, abi, Er, Ei);
+        const float br = tr[j], bi = tr[NM + j], cr = tr[2 * NM + j], ci = tr[3 * NM + j];
         // Bbar u = E B u
         const float bbr = fmaf(Er, br, -Ei * bi) * ut, bbi = fmaf(Er, bi, Ei * br) * ut;
-        const float nr = fmaf(abr, hr[n], fmaf(-abi, hi[n], bbr));
-        const float ni = fmaf(abr, hi[n], fmaf(abi, hr[n], bbi));
-        hr[n] = nr;
-        hi[n] = ni;
+        const float nr = fmaf(abr, hr[j], fmaf(-abi, hi[j], bbr));
+        const float ni = fmaf(abr, hi[j], fmaf(abi, hr[j], bbi));
+        hr[j] = nr;
+        hi[j] = ni;
         y0 = fmaf(cr, nr, fmaf(-ci, ni, y0));
       }
+#pragma unroll
+      for (int o = 1; o < TPC; o <<= 1) y0 += __shfl_xor_sync(0xffffffffu, y0, o);
       if (z) {
         const float zt = to_f(z[t]);
         y0 *= zt * rcpf(1.f + ex2f(-zt * kLog2e));
       }
-      if (valid) y[t] = from_f<T>(y0);
+      if (valid && part == 0) y[t] = from_f<T>(y0);
     }
   }
   if (valid && a.last_state) {
     float *ls = a.last_state + (b * a.dim + d) * 2 * N;
 #pragma unroll
-    for (int n = 0; n < NM; ++n)
+    for (int j = 0; j < NS; ++j) {
+      const int n = part * NS + j;
       if (n < N) {
-        ls[n] = hr[n];
-        ls[N + n] = hi[n];
+        ls[n] = hr[j];
+        ls[N + n] = hi[j];
       }
+    }
   }
 }
 
@@ -212,15 +218,54 @@ struct CplxWork {
   int64_t n_blocks, n_dblk;
 };
 
-template <typename T, int NM>
+// Sums S values over the lanes of a warp that share lane % TPC (the channels
+// of one state range), leaving S * TPC / 32 of the sums on each lane: a
+// butterfly reduce-scatter over lane bits 4 down to log2(TPC).  Lane l keeps
+// the sums of value indices base(l) + r, r < S * TPC / 32, where base(l) is
+// the sum of the upper half sizes of the stages whose lane bit is set.
+template <int S, int TPC>
+__device__ __forceinline__ void lane_reduce_scatter(float (&v)[S], int lane) {
+  int h = S / 2;
+#pragma unroll
+  for (int o = 16; o >= TPC; o >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < S / 2; ++i) {
+      if (i < h) {
+        const float send = up ? v[i] : v[i + h];
+        const float keep = up ? v[i + h] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      }
+    }
+    h /= 2;
+  }
+}
+
+template <int S, int TPC>
+__device__ __forceinline__ int lane_scatter_base(int lane) {
+  int base = 0, h = S / 2;
+  for (int o = 16; o >= TPC; o >>= 1) {
+    if (lane & o) base += h;
+    h /= 2;
+  }
+  return base;
+}
+
+// TPC threads share one channel, NM / TPC states each (adjacent lanes), as in
+// the forward: more threads per channel, fewer registers per thread.
+template <typename T, int NM, int TPC>
 __global__ void __launch_bounds__(kCplxBwdThreads) cplx_bwd_kernel(const CplxArgs a, const CplxWork w) {
+  constexpr int NS = NM / TPC;                 // states per thread
+  constexpr int NV = 4 * NS < 32 / TPC ? 32 / TPC : 4 * NS;  // dB / dC values (padded)
+  constexpr int NKEEP = NV * TPC / 32;         // sums left on each lane
   extern __shared__ __align__(16) float smem[];
-  float *hs = smem;                                          // [TC][2 NM][threads]
-  float *tab = hs + kCplxBwdTC * 2 * NM * kCplxBwdThreads;  // [TC][4 NM]
+  float *hs = smem;                                          // [TC][2 NS][threads]
+  float *tab = hs + kCplxBwdTC * 2 * NS * kCplxBwdThreads;  // [TC][4 NM]
   float *wsum = tab + kCplxBwdTC * 4 * NM;                   // [2 warps][4 kMaxN][TC]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int part = tid % TPC;
   const int64_t b = blockIdx.y;
-  const int64_t d_raw = int64_t(blockIdx.x) * kCplxBwdThreads + tid;
+  const int64_t d_raw = int64_t(blockIdx.x) * (kCplxBwdThreads / TPC) + tid / TPC;
   const bool valid = d_raw < a.dim;
   const int64_t d = valid ? d_raw : a.dim - 1;
   const int64_t ch = b * a.dim + d;
@@ -233,30 +278,32 @@ __global__ void __launch_bounds__(kCplxBwdThreads) cplx_bwd_kernel(const CplxArg
   const float bias = a.bias ? a.bias[d] : 0.f;
   const float Dd = a.D ? a.D[d] : 0.f;
   float *ckpt = w.ckpt + ch * w.n_blocks * 2 * NM;
+  for (int i = tid; i < 2 * 4 * kMaxN * kCplxBwdTC; i += kCplxBwdThreads) wsum[i] = 0.f;
 
-  float ar[NM], ai[NM], ira[NM], iai[NM], hr[NM], hi[NM];
+  float ar[NS], ai[NS], ira[NS], iai[NS], hr[NS], hi[NS];
 #pragma unroll
-  for (int n = 0; n < NM; ++n) {
-    ar[n] = n < N ? a.A[d * 2 * N + n] : -1.f;
-    ai[n] = n < N ? a.A[d * 2 * N + N + n] : 0.f;
-    const float m = ar[n] * ar[n] + ai[n] * ai[n];
-    ira[n] = m > 0.f ? ar[n] / m : 0.f;
-    iai[n] = m > 0.f ? -ai[n] / m : 0.f;
-    hr[n] = hi[n] = 0.f;
+  for (int j = 0; j < NS; ++j) {
+    const int n = part * NS + j;
+    ar[j] = n < N ? a.A[d * 2 * N + n] : -1.f;
+    ai[j] = n < N ? a.A[d * 2 * N + N + n] : 0.f;
+    const float m = ar[j] * ar[j] + ai[j] * ai[j];
+    ira[j] = m > 0.f ? ar[j] / m : 0.f;
+    iai[j] = m > 0.f ? -ai[j] / m : 0.f;
+    hr[j] = hi[j] = 0.f;
   }
 
-  // one forward step of the recurrence (B from the staged table row)
+  // one forward step of this thread's states (B from the staged table row)
   auto step = [&](float Delta, float ut, const float *trow) {
 #pragma unroll
-    for (int n = 0; n < NM; ++n) {
+    for (int j = 0; j < NS; ++j) {
       float abr, abi, Er, Ei;
-      cplx_decay(Delta, ar[n], ai[n], ira[n], iai[n], abr, abi, Er, Ei);
-      const float br = trow[n], bi = trow[NM + n];
+      cplx_decay(Delta, ar[j], ai[j], ira[j], iai[j], abr, abi, Er, Ei);
+      const float br = trow[part * NS + j], bi = trow[NM + part * NS + j];
       const float bbr = fmaf(Er, br, -Ei * bi) * ut, bbi = fmaf(Er, bi, Ei * br) * ut;
-      const float nr = fmaf(abr, hr[n], fmaf(-abi, hi[n], bbr));
-      const float ni = fmaf(abr, hi[n], fmaf(abi, hr[n], bbi));
-      hr[n] = nr;
-      hi[n] = ni;
+      const float nr = fmaf(abr, hr[j], fmaf(-abi, hi[j], bbr));
+      const float ni = fmaf(abr, hi[j], fmaf(abi, hr[j], bbi));
+      hr[j] = nr;
+      hi[j] = ni;
     }
   };
 
@@ -264,9 +311,9 @@ __global__ void __launch_bounds__(kCplxBwdThreads) cplx_bwd_kernel(const CplxArg
   for (int64_t c = 0; c < w.n_blocks; ++c) {
     const int64_t t0 = c * kCplxBwdTC;
 #pragma unroll
-    for (int n = 0; n < NM; ++n) {
-      ckpt[c * 2 * NM + n] = hr[n];
-      ckpt[c * 2 * NM + NM + n] = hi[n];
+    for (int j = 0; j < NS; ++j) {
+      ckpt[c * 2 * NM + part * NS + j] = hr[j];
+      ckpt[c * 2 * NM + NM + part * NS + j] = hi[j];
     }
     __syncthreads();
     cplx_stage_bc<T, NM, kCplxBwdTC>(a, b, t0, tab, false, kCplxBwdThreads);
@@ -276,10 +323,11 @@ __global__ void __launch_bounds__(kCplxBwdThreads) cplx_bwd_kernel(const CplxArg
       step(softplus_fast(to_f(dl[t0 + i]) + bias), to_f(u[t0 + i]), tab + i * 4 * NM);
   }
 
-  float Gr[NM], Gi[NM], Anr[NM], Ani[NM], gAr[NM], gAi[NM];
+  float Gr[NS], Gi[NS], Anr[NS], Ani[NS], gAr[NS], gAi[NS];
 #pragma unroll
-  for (int n = 0; n < NM; ++n) Gr[n] = Gi[n] = Anr[n] = Ani[n] = gAr[n] = gAi[n] = 0.f;
+  for (int j = 0; j < NS; ++j) Gr[j] = Gi[j] = Anr[j] = Ani[j] = gAr[j] = gAi[j] = 0.f;
   float dDacc = 0.f, dbacc = 0.f;
+  const int kbase = lane_scatter_base<NV, TPC>(lane);
 
   for (int64_t c = w.n_blocks - 1; c >= 0; --c) {
     const int64_t t0 = c * kCplxBwdTC;
@@ -289,15 +337,15 @@ __global__ void __launch_bounds__(kCplxBwdThreads) cplx_bwd_kernel(const CplxArg
     __syncthreads();
     // recompute the block; hs[s] holds the state before step t0 + s
 #pragma unroll
-    for (int n = 0; n < NM; ++n) {
-      hr[n] = ckpt[c * 2 * NM + n];
-      hi[n] = ckpt[c * 2 * NM + NM + n];
+    for (int j = 0; j < NS; ++j) {
+      hr[j] = ckpt[c * 2 * NM + part * NS + j];
+      hi[j] = ckpt[c * 2 * NM + NM + part * NS + j];
     }
     for (int s = 0; s < steps; ++s) {
 #pragma unroll
-      for (int n = 0; n < NM; ++n) {
-        hs[(s * 2 * NM + n) * kCplxBwdThreads + tid] = hr[n];
-        hs[(s * 2 * NM + NM + n) * kCplxBwdThreads + tid] = hi[n];
+      for (int j = 0; j < NS; ++j) {
+        hs[(s * 2 * NS + j) * kCplxBwdThreads + tid] = hr[j];
+        hs[(s * 2 * NS + NS + j) * kCplxBwdThreads + tid] = hi[j];
       }
       step(softplus_fast(to_f(dl[t0 + s]) + bias), to_f(u[t0 + s]), tab + s * 4 * NM);
     }
@@ -315,65 +363,78 @@ __global__ void __launch_bounds__(kCplxBwdThreads) cplx_bwd_kernel(const CplxArg
         sz = rcpf(1.f + ex2f(-zt * kLog2e));
         dy0 = dyt * zt * sz;
       }
-      const float *trow = tab + s * 4 * NM;
-      float y0 = Dd * ut, du = Dd * dy0, dDelta = 0.f;
-      float vb[32], vc[32];  // (Re, Im) of the dB and dC terms, for the channel sums
+      const float *trow = tab + s * 4 * NM + part * NS;
+      float y0 = 0.f, du = 0.f, dDelta = 0.f;
+      float vals[NV];  // per state j: Re dB, Im dB, Re dC, Im dC at j, NS + j, 2 NS + j, 3 NS + j
 #pragma unroll
-      for (int j = 0; j < 32; ++j) vb[j] = vc[j] = 0.f;
+      for (int i = 0; i < NV; ++i) vals[i] = 0.f;
+      const float m = valid ? 1.f : 0.f;
 #pragma unroll
-      for (int n = 0; n < NM; ++n) {
-        const float hpr = hs[(s * 2 * NM + n) * kCplxBwdThreads + tid];
-        const float hpi = hs[(s * 2 * NM + NM + n) * kCplxBwdThreads + tid];
+      for (int j = 0; j < NS; ++j) {
+        const float hpr = hs[(s * 2 * NS + j) * kCplxBwdThreads + tid];
+        const float hpi = hs[(s * 2 * NS + NS + j) * kCplxBwdThreads + tid];
         float abr, abi, Er, Ei;
-        cplx_decay(Delta, ar[n], ai[n], ira[n], iai[n], abr, abi, Er, Ei);
-        const float br = trow[n], bi = trow[NM + n], cr = trow[2 * NM + n], ci = trow[3 * NM + n];
+        cplx_decay(Delta, ar[j], ai[j], ira[j], iai[j], abr, abi, Er, Ei);
+        const float br = trow[j], bi = trow[NM + j], cr = trow[2 * NM + j], ci = trow[3 * NM + j];
         // h_t = Abar h_{t-1} + E B u
         const float bur = br * ut, bui = bi * ut;
         const float hcr = fmaf(abr, hpr, fmaf(-abi, hpi, fmaf(Er, bur, -Ei * bui)));
         const float hci = fmaf(abr, hpi, fmaf(abi, hpr, fmaf(Er, bui, Ei * bur)));
         y0 = fmaf(cr, hcr, fmaf(-ci, hci, y0));
         // G_t = conj(C) dy0 + conj(Abar_{t+1}) G_{t+1}
-        const float gr = fmaf(cr, dy0, fmaf(Anr[n], Gr[n], Ani[n] * Gi[n]));
-        const float gi = fmaf(-ci, dy0, fmaf(Anr[n], Gi[n], -Ani[n] * Gr[n]));
-        Gr[n] = gr;
-        Gi[n] = gi;
-        Anr[n] = abr;
-        Ani[n] = abi;
-        // du += Re(conj(G) E B) u-free part; dDelta += Re(conj(G) Abar (A h + B u))
+        const float gr = fmaf(cr, dy0, fmaf(Anr[j], Gr[j], Ani[j] * Gi[j]));
+        const float gi = fmaf(-ci, dy0, fmaf(Anr[j], Gi[j], -Ani[j] * Gr[j]));
+        Gr[j] = gr;
+        Gi[j] = gi;
+        Anr[j] = abr;
+        Ani[j] = abi;
+        // du += Re(conj(G) E B); dDelta += Re(conj(G) Abar (A h + B u))
         const float ebr = fmaf(Er, br, -Ei * bi), ebi = fmaf(Er, bi, Ei * br);
         du = fmaf(gr, ebr, fmaf(gi, ebi, du));
-        const float qr = fmaf(ar[n], hpr, fmaf(-ai[n], hpi, bur));
-        const float qi = fmaf(ar[n], hpi, fmaf(ai[n], hpr, bui));
+        const float qr = fmaf(ar[j], hpr, fmaf(-ai[j], hpi, bur));
+        const float qi = fmaf(ar[j], hpi, fmaf(ai[j], hpr, bui));
         const float pr_ = fmaf(abr, qr, -abi * qi), pi_ = fmaf(abr, qi, abi * qr);
         dDelta = fmaf(gr, pr_, fmaf(gi, pi_, dDelta));
         // gA += conj(Delta Abar h_{t-1} + Delta^2 phi(x) B u) G
         float phr, phi_;
-        cplx_phi(Delta * ar[n], Delta * ai[n], abr, abi, phr, phi_);
+        cplx_phi(Delta * ar[j], Delta * ai[j], abr, abi, phr, phi_);
         const float D2 = Delta * Delta;
         const float kr = fmaf(Delta, fmaf(abr, hpr, -abi * hpi), D2 * fmaf(phr, bur, -phi_ * bui));
         const float ki = fmaf(Delta, fmaf(abr, hpi, abi * hpr), D2 * fmaf(phr, bui, phi_ * bur));
-        gAr[n] = fmaf(kr, gr, fmaf(ki, gi, gAr[n]));
-        gAi[n] = fmaf(kr, gi, fmaf(-ki, gr, gAi[n]));
-        // gB = conj(E) u G, gC = conj(h_t) dy0 (zero on padding channels: dy0 = 0 there)
-        if (valid) {
-          vb[n] = fmaf(Er, gr, Ei * gi) * ut;
-          vb[16 + n] = fmaf(Er, gi, -Ei * gr) * ut;
-          vc[n] = hcr * dy0;
-          vc[16 + n] = -hci * dy0;
-        }
+        gAr[j] = fmaf(kr, gr, fmaf(ki, gi, gAr[j]));
+        gAi[j] = fmaf(kr, gi, fmaf(-ki, gr, gAi[j]));
+        // gB = conj(E) u G, gC = conj(h_t) dy0; padding channels contribute 0
+        vals[j] = m * fmaf(Er, gr, Ei * gi) * ut;
+        vals[NS + j] = m * fmaf(Er, gi, -Ei * gr) * ut;
+        vals[2 * NS + j] = m * hcr * dy0;
+        vals[3 * NS + j] = -m * hci * dy0;
       }
+      // join the partial sums of the TPC threads of this channel
+#pragma unroll
+      for (int o = 1; o < TPC; o <<= 1) {
+        y0 += __shfl_xor_sync(0xffffffffu, y0, o);
+        du += __shfl_xor_sync(0xffffffffu, du, o);
+        dDelta += __shfl_xor_sync(0xffffffffu, dDelta, o);
+      }
+      y0 = fmaf(Dd, ut, y0);
+      du = fmaf(Dd, dy0, du);
       const float ddl = dDelta * sv;
-      if (valid) {
+      if (valid && part == 0) {
         static_cast<T *>(a.du)[row + t] = from_f<T>(du);
         static_cast<T *>(a.ddelta)[row + t] = from_f<T>(ddl);
         if (z) static_cast<T *>(a.dz)[row + t] = from_f<T>(dyt * y0 * sz * (1.f + zt * (1.f - sz)));
         dDacc = fmaf(dy0, ut, dDacc);
         dbacc += ddl;
       }
-      const float rb = warp_reduce_scatter32(vb, lane);
-      const float rc = warp_reduce_scatter32(vc, lane);
-      wsum[(warp * 4 * kMaxN + lane) * kCplxBwdTC + s] = rb;
-      wsum[(warp * 4 * kMaxN + 32 + lane) * kCplxBwdTC + s] = rc;
+      lane_reduce_scatter<NV, TPC>(vals, lane);
+#pragma unroll
+      for (int r = 0; r < NKEEP; ++r) {
+        const int idx = kbase + r;  // value index of this lane's sum
+        if (idx < 4 * NS) {
+          const int q = idx / NS, n = part * NS + idx % NS;
+          wsum[(warp * 4 * kMaxN + q * kMaxN + n) * kCplxBwdTC + s] = vals[r];
+        }
+      }
     }
     __syncthreads();
     for (int idx = tid; idx < 4 * kMaxN * kCplxBwdTC; idx += kCplxBwdThreads) {
@@ -387,13 +448,17 @@ __global__ void __launch_bounds__(kCplxBwdThreads) cplx_bwd_kernel(const CplxArg
   }
   if (valid) {
 #pragma unroll
-    for (int n = 0; n < NM; ++n)
+    for (int j = 0; j < NS; ++j) {
+      const int n = part * NS + j;
       if (n < N) {
-        w.part_A[ch * 2 * N + n] = gAr[n];
-        w.part_A[ch * 2 * N + N + n] = gAi[n];
+        w.part_A[ch * 2 * N + n] = gAr[j];
+        w.part_A[ch * 2 * N + N + n] = gAi[j];
       }
-    w.part_D[ch] = dDacc;
-    w.part_bias[ch] = dbacc;
+    }
+    if (part == 0) {
+      w.part_D[ch] = dDacc;
+      w.part_bias[ch] = dbacc;
+    }
   }
 }
 

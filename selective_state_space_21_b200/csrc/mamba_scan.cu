@@ -225,19 +225,25 @@ struct BwdReferenceLauncher {
 
 template <typename T, int NM>
 struct CplxFwdLauncher {
+  // four threads per channel for 16 states, two for 8
+  static constexpr int TPC = NM >= 16 ? 4 : (NM >= 8 ? 2 : 1);
   static mamba_status_t run(const CplxArgs &a, cudaStream_t s) {
-    const dim3 grid(unsigned((a.dim + kCplxThreads - 1) / kCplxThreads), unsigned(a.batch));
-    cplx_fwd_kernel<T, NM><<<grid, kCplxThreads, 0, s>>>(a);
+    constexpr int per_block = kCplxThreads / TPC;
+    const dim3 grid(unsigned((a.dim + per_block - 1) / per_block), unsigned(a.batch));
+    cplx_fwd_kernel<T, NM, TPC><<<grid, kCplxThreads, 0, s>>>(a);
     return launch_status();
   }
 };
 
 template <typename T, int NM>
 struct CplxBwdLauncher {
+  // four threads per channel for 16 states, two for 8
+  static constexpr int TPC = NM >= 16 ? 4 : (NM >= 8 ? 2 : 1);
   static mamba_status_t run(const CplxArgs &a, cudaStream_t s) {
+    constexpr int per_block = kCplxBwdThreads / TPC;
     CplxWork w;
     w.n_blocks = (a.L + kCplxBwdTC - 1) / kCplxBwdTC;
-    w.n_dblk = (a.dim + kCplxBwdThreads - 1) / kCplxBwdThreads;
+    w.n_dblk = (a.dim + per_block - 1) / per_block;
     const size_t bd = size_t(a.batch * a.dim);
     const size_t n_ckpt = bd * size_t(w.n_blocks) * 2 * NM;
     const size_t n_bc = size_t(w.n_dblk) * size_t(a.batch) * 4 * kMaxN * size_t(a.L);
@@ -252,15 +258,15 @@ struct CplxBwdLauncher {
     w.part_A = w.part_bc + n_bc;
     w.part_D = w.part_A + n_A;
     w.part_bias = w.part_D + bd;
-    const size_t smem = 4 * (size_t(kCplxBwdTC) * 2 * NM * kCplxBwdThreads +
+    const size_t smem = 4 * (size_t(kCplxBwdTC) * 2 * (NM / TPC) * kCplxBwdThreads +
                              size_t(kCplxBwdTC) * 4 * NM + 2 * 4 * kMaxN * kCplxBwdTC);
     mamba_status_t st = MAMBA_OK;
-    if (cudaFuncSetAttribute(cplx_bwd_kernel<T, NM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(smem)) != cudaSuccess)
+    if (cudaFuncSetAttribute(cplx_bwd_kernel<T, NM, TPC>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
       st = MAMBA_ERR_CUDA;
     if (st == MAMBA_OK) {
       const dim3 grid(unsigned(w.n_dblk), unsigned(a.batch));
-      cplx_bwd_kernel<T, NM><<<grid, kCplxBwdThreads, smem, s>>>(a, w);
+      cplx_bwd_kernel<T, NM, TPC><<<grid, kCplxBwdThreads, smem, s>>>(a, w);
       st = launch_status();
     }
     if (st == MAMBA_OK) {
@@ -868,7 +874,8 @@ mamba_status_t mamba_cplx_scan_fwd(const void *u, const void *delta, const float
       return cuda_status();
     return MAMBA_OK;
   }
-  if ((dim + kCplxThreads - 1) / kCplxThreads > (int64_t(1) << 31) - 1) return MAMBA_ERR_UNSUPPORTED;
+  if ((dim + kCplxThreads / 4 - 1) / (kCplxThreads / 4) > (int64_t(1) << 31) - 1)
+    return MAMBA_ERR_UNSUPPORTED;
   CplxArgs a = {};
   a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
   a.bias = delta_bias; a.A = A; a.D = D; a.y = y; a.last_state = last_state;
