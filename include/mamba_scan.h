@@ -309,6 +309,26 @@ MAMBA_SCAN_API mamba_status_t mamba_scan_step(float *state, const void *u, const
                                               int64_t N, mamba_dtype_t dtype, mamba_stream_t stream);
 
 /*
+ * One decoding step of the block with its convolution prologue (the
+ * recurrent mode of mamba_conv_scan_fwd).  x is this token's block input
+ * (batch, dim) dtype; conv_state (batch, dim, W - 1) float32 holds the
+ * previous W - 1 inputs of each channel, oldest first (zeros before the
+ * first token; after a prompt, its last W - 1 inputs), and is shifted in
+ * place; NULL is allowed only for W = 1.  u = SiLU(conv_b + sum_k conv_w[d,k]
+ * (the W inputs ending with x)) then drives the step of mamba_scan_step.
+ * Repeating the call over the tokens of a sequence gives the result of
+ * mamba_conv_scan_fwd, up to rounding.
+ */
+MAMBA_SCAN_API mamba_status_t mamba_conv_scan_step(float *state, float *conv_state, const void *x,
+                                                   const float *conv_w, const float *conv_b,
+                                                   int64_t conv_width, const void *delta,
+                                                   const float *delta_bias, const float *A,
+                                                   const void *B, const void *C, const float *D,
+                                                   const void *z, void *y, int64_t batch,
+                                                   int64_t dim, int64_t N, mamba_dtype_t dtype,
+                                                   mamba_stream_t stream);
+
+/*
  * Forward that allocates nothing.  (An addition of this library for callers
  * that cannot allocate; the paper has no counterpart.)
  *

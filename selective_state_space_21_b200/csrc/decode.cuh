@@ -28,11 +28,36 @@ struct DecodeArgs {
   void *y;
   int64_t batch, dim;
   int N;
+  // convolution prologue (CONV kernels): u is the block input x of this token;
+  // conv_state (batch, dim, W - 1) fp32 holds the previous W - 1 inputs,
+  // oldest first, and is shifted in place.
+  float *conv_state = nullptr;
+  const float *conv_w = nullptr, *conv_b = nullptr;
+  int conv_width = 0;
 };
+
+// u of this token from x and the channel's convolution state (see ConvFilter
+// for the right-aligned filter), and the state shifted by one input.
+__device__ __forceinline__ float decode_conv_u(const DecodeArgs &a, int64_t ch, int64_t d, float x,
+                                               bool write_state) {
+  const int W = a.conv_width;
+  const ConvFilter c = load_conv_filter(a.conv_w, a.conv_b, W, d);
+  float *cs = a.conv_state + ch * (W - 1);
+  const float xm1 = W >= 2 ? cs[W - 2] : 0.f;
+  const float xm2 = W >= 3 ? cs[W - 3] : 0.f;
+  const float xm3 = W >= 4 ? cs[W - 4] : 0.f;
+  const float pre = conv_pre(c, xm3, xm2, xm1, x);
+  if (write_state && W >= 2) {
+    if (W >= 4) cs[W - 4] = xm2;
+    if (W >= 3) cs[W - 3] = xm1;
+    cs[W - 2] = x;
+  }
+  return pre * rcpf(1.f + ex2f(-pre * kLog2e));
+}
 
 constexpr int kDecodeThreads = 128;
 
-template <typename T, int NM>
+template <typename T, int NM, bool CONV = false>
 __global__ void __launch_bounds__(kDecodeThreads) decode_step_kernel(const DecodeArgs a) {
   const int64_t ch = int64_t(blockIdx.x) * kDecodeThreads + threadIdx.x;
   if (ch >= a.batch * a.dim) return;
@@ -41,7 +66,8 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_step_kernel(const Decod
   const T *Bp = static_cast<const T *>(a.B) + b * N;
   const T *Cp = static_cast<const T *>(a.C) + b * N;
   float *st = a.state + ch * N;
-  const float uv = to_f(static_cast<const T *>(a.u)[ch]);
+  float uv = to_f(static_cast<const T *>(a.u)[ch]);
+  if constexpr (CONV) uv = decode_conv_u(a, ch, d, uv, true);
   const float v = to_f(static_cast<const T *>(a.delta)[ch]) + (a.bias ? a.bias[d] : 0.f);
   const float Delta = softplus_fast(v);
   float y0 = a.D ? a.D[d] * uv : 0.f;
@@ -86,7 +112,7 @@ template <> struct Quad<__nv_bfloat16> {
   }
 };
 
-template <typename T, int NM>
+template <typename T, int NM, bool CONV = false>
 __global__ void __launch_bounds__(kDecodeThreads) decode_step_vec4_kernel(const DecodeArgs a) {
   constexpr int TPC = NM / 4;  // threads per channel
   const int64_t gid = int64_t(blockIdx.x) * kDecodeThreads + threadIdx.x;
@@ -99,7 +125,10 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_step_vec4_kernel(const 
   const float4 Av = *reinterpret_cast<const float4 *>(a.A + d * NM + 4 * g);
   const float4 Bv = Quad<T>::load(static_cast<const T *>(a.B) + b * NM + 4 * g);
   const float4 Cv = Quad<T>::load(static_cast<const T *>(a.C) + b * NM + 4 * g);
-  const float uv = to_f(static_cast<const T *>(a.u)[chs]);
+  float uv = to_f(static_cast<const T *>(a.u)[chs]);
+  // every thread of the channel forms u; the first one shifts the state (after
+  // all of them have read it: the shuffles below order the warp)
+  if constexpr (CONV) uv = decode_conv_u(a, chs, d, uv, false);
   const float v = to_f(static_cast<const T *>(a.delta)[chs]) + (a.bias ? a.bias[d] : 0.f);
   const float Delta = softplus_fast(v);
   const float hs[4] = {h.x, h.y, h.z, h.w}, As[4] = {Av.x, Av.y, Av.z, Av.w};
@@ -123,6 +152,15 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_step_vec4_kernel(const 
   if (!live) return;
   *reinterpret_cast<float4 *>(a.state + ch * NM + 4 * g) = make_float4(hn[0], hn[1], hn[2], hn[3]);
   if (g == 0) {
+    if constexpr (CONV) {
+      const int W = a.conv_width;
+      float *cs = a.conv_state + ch * (W - 1);
+      if (W >= 2) {
+        if (W >= 4) cs[W - 4] = cs[W - 3];
+        if (W >= 3) cs[W - 3] = cs[W - 2];
+        cs[W - 2] = to_f(static_cast<const T *>(a.u)[ch]);
+      }
+    }
     float y0 = yp + (a.D ? a.D[d] * uv : 0.f);
     if (a.z) {
       const float zv = to_f(static_cast<const T *>(a.z)[ch]);

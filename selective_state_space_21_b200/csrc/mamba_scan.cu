@@ -467,12 +467,20 @@ mamba_status_t mamba_scan_bwd_ex(const void *u, const void *delta, const float *
   return backward_paths<false>(a, es, dtype, staged_options(options), s);
 }
 
-mamba_status_t mamba_scan_step(float *state, const void *u, const void *delta,
-                               const float *delta_bias, const float *A, const void *B, const void *C,
-                               const float *D, const void *z, void *y, int64_t batch, int64_t dim,
-                               int64_t N, mamba_dtype_t dtype, mamba_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// One decoding token, with (CONV) or without the convolution prologue.
+template <bool CONV>
+mamba_status_t decode_step(float *state, float *conv_state, const void *u, const float *conv_w,
+                           const float *conv_b, int64_t conv_width, const void *delta,
+                           const float *delta_bias, const float *A, const void *B, const void *C,
+                           const float *D, const void *z, void *y, int64_t batch, int64_t dim,
+                           int64_t N, mamba_dtype_t dtype, mamba_stream_t stream) {
   mamba_status_t st = check_shape(batch, dim, 1, N, dtype);
   if (st != MAMBA_OK) return st;
+  if (CONV && (conv_width < 1 || conv_width > kMaxConvWidth)) return MAMBA_ERR_UNSUPPORTED;
   Checker ck;
   if (cudaGetDevice(&ck.dev) != cudaSuccess) {
     cudaGetLastError();
@@ -490,12 +498,20 @@ mamba_status_t mamba_scan_step(float *state, const void *u, const void *delta,
   ck.buf(delta_bias, size_t(dim) * 4, 4, false, false);
   ck.buf(state, nbd * N * 4, 4, true, true);
   ck.buf(y, nbd * es, es, true, true);
+  if (CONV) {
+    ck.buf(conv_w, size_t(dim) * size_t(conv_width) * 4, 4, true, false);
+    ck.buf(conv_b, size_t(dim) * 4, 4, false, false);
+    ck.buf(conv_state, nbd * size_t(conv_width - 1) * 4, 4, conv_width > 1, true);
+  }
   if (ck.st != MAMBA_OK) return ck.st;
   if (nbd == 0) return MAMBA_OK;
   DecodeArgs a;
   a.state = state; a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
   a.bias = delta_bias; a.A = A; a.D = D; a.y = y;
   a.batch = batch; a.dim = dim; a.N = (int)N;
+  if (CONV) {
+    a.conv_state = conv_state; a.conv_w = conv_w; a.conv_b = conv_b; a.conv_width = (int)conv_width;
+  }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   // four states per thread when N is 4, 8 or 16 and the state, A, B and C
   // rows are 16- (B, C: 8-) byte aligned
@@ -505,7 +521,7 @@ mamba_status_t mamba_scan_step(float *state, const void *u, const void *delta,
     const int64_t threads = int64_t(nbd) * (N / 4);
     const int64_t g4 = (threads + kDecodeThreads - 1) / kDecodeThreads;
     if (g4 > (int64_t(1) << 31) - 1) return MAMBA_ERR_UNSUPPORTED;
-#define MSCAN_VEC4(TT, NN) decode_step_vec4_kernel<TT, NN><<<unsigned(g4), kDecodeThreads, 0, s>>>(a)
+#define MSCAN_VEC4(TT, NN) decode_step_vec4_kernel<TT, NN, CONV><<<unsigned(g4), kDecodeThreads, 0, s>>>(a)
     if (dtype == MAMBA_BF16) {
       if (N == 4) MSCAN_VEC4(__nv_bfloat16, 4);
       else if (N == 8) MSCAN_VEC4(__nv_bfloat16, 8);
@@ -522,7 +538,7 @@ mamba_status_t mamba_scan_step(float *state, const void *u, const void *delta,
   if (grid > (int64_t(1) << 31) - 1) return MAMBA_ERR_UNSUPPORTED;
   auto launch = [&](auto tag, auto nm) {
     using T = typename decltype(tag)::type;
-    decode_step_kernel<T, decltype(nm)::value><<<unsigned(grid), kDecodeThreads, 0, s>>>(a);
+    decode_step_kernel<T, decltype(nm)::value, CONV><<<unsigned(grid), kDecodeThreads, 0, s>>>(a);
   };
   struct TF { using type = float; };
   struct TB { using type = __nv_bfloat16; };
@@ -536,6 +552,28 @@ mamba_status_t mamba_scan_step(float *state, const void *u, const void *delta,
     else launch(TF{}, std::integral_constant<int, 16>{});
   }
   return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+mamba_status_t mamba_scan_step(float *state, const void *u, const void *delta,
+                               const float *delta_bias, const float *A, const void *B, const void *C,
+                               const float *D, const void *z, void *y, int64_t batch, int64_t dim,
+                               int64_t N, mamba_dtype_t dtype, mamba_stream_t stream) {
+  return decode_step<false>(state, nullptr, u, nullptr, nullptr, 0, delta, delta_bias, A, B, C, D,
+                            z, y, batch, dim, N, dtype, stream);
+}
+
+mamba_status_t mamba_conv_scan_step(float *state, float *conv_state, const void *x,
+                                    const float *conv_w, const float *conv_b, int64_t conv_width,
+                                    const void *delta, const float *delta_bias, const float *A,
+                                    const void *B, const void *C, const float *D, const void *z,
+                                    void *y, int64_t batch, int64_t dim, int64_t N,
+                                    mamba_dtype_t dtype, mamba_stream_t stream) {
+  return decode_step<true>(state, conv_state, x, conv_w, conv_b, conv_width, delta, delta_bias, A,
+                           B, C, D, z, y, batch, dim, N, dtype, stream);
 }
 
 mamba_status_t mamba_scan_bwd(const void *u, const void *delta, const float *delta_bias,

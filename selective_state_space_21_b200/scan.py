@@ -69,6 +69,8 @@ def load_library():
             lib.mamba_scan_fwd_noalloc.argtypes = [vp] * 10 + [i64] * 4 + [i32, vp]
             lib.mamba_scan_step.argtypes = [vp] * 10 + [i64] * 3 + [i32, vp]
             lib.mamba_scan_step.restype = ctypes.c_int
+            lib.mamba_conv_scan_step.argtypes = [vp] * 5 + [i64] + [vp] * 8 + [i64] * 3 + [i32, vp]
+            lib.mamba_conv_scan_step.restype = ctypes.c_int
             lib.mamba_conv_scan_fwd.argtypes = [vp] * 3 + [i64] + [vp] * 9 + [i64] * 4 + [i32, opt, vp]
             lib.mamba_conv_scan_fwd.restype = ctypes.c_int
             lib.mamba_conv_scan_bwd.argtypes = [vp] * 3 + [i64] + [vp] * 18 + [i64] * 4 + [i32, opt, vp]
@@ -384,6 +386,29 @@ def mamba_scan_step(state, u, delta, delta_bias, A, B, C, D, z, y, *, stream=Non
         _ptr(D, f32, (dim,), "D"), _ptr(z, dt, (batch, dim), "z"), _ptr(y, dt, (batch, dim), "y"),
         batch, dim, N, _dtype_code(dt)]
     _check(load_library().mamba_scan_step(*args, _stream_handle(stream)), "mamba_scan_step")
+
+
+def mamba_conv_scan_step(state, conv_state, x, conv_w, conv_b, delta, delta_bias, A, B, C, D, z,
+                         y, *, stream=None):
+    """One decoding step with the convolution prologue: updates ``state``
+    (batch, dim, N) and ``conv_state`` (batch, dim, W - 1) float32 in place
+    and writes ``y`` (batch, dim).  x, delta, z, y: (batch, dim); B, C:
+    (batch, N); conv_w (dim, W), conv_b (dim,) or None."""
+    batch, dim = x.shape
+    N = A.shape[1]
+    W = conv_w.shape[1]
+    dt = x.dtype
+    f32 = torch.float32
+    args = [
+        _ptr(state, f32, (batch, dim, N), "state"),
+        _ptr(conv_state, f32, (batch, dim, W - 1), "conv_state"), _ptr(x, dt, (batch, dim), "x"),
+        _ptr(conv_w, f32, (dim, W), "conv_w"), _ptr(conv_b, f32, (dim,), "conv_b"), W,
+        _ptr(delta, dt, (batch, dim), "delta"), _ptr(delta_bias, f32, (dim,), "delta_bias"),
+        _ptr(A, f32, (dim, N), "A"), _ptr(B, dt, (batch, N), "B"), _ptr(C, dt, (batch, N), "C"),
+        _ptr(D, f32, (dim,), "D"), _ptr(z, dt, (batch, dim), "z"), _ptr(y, dt, (batch, dim), "y"),
+        batch, dim, N, _dtype_code(dt)]
+    _check(load_library().mamba_conv_scan_step(*args, _stream_handle(stream)),
+           "mamba_conv_scan_step")
 
 
 def launch_count() -> int:
