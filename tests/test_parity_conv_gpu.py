@@ -207,3 +207,23 @@ def test_conv_rejects_bad_width_and_aliasing():
         scan.mamba_conv_scan_fwd(x["u"], x["conv_w"], x["conv_b"], x["delta"], x["delta_bias"],
                                  x["A"], x["B"], x["C"], x["D"], x["z"], x["u"], None)
     assert e.value.status == 1  # MAMBA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("L", [1, 2, 3, 5])
+def test_conv_sequences_shorter_than_the_filter(L):
+    """L below the filter width: every step sees the zero padding before the
+    start (one-thread-per-channel kernels; rows are not 16-byte multiples)."""
+    x = conv_case(2, 40, L, 4, torch.float32, seed=992 + L)
+    fwd_case(x)
+    bwd_case(x)
+
+
+def test_conv_empty_sequence():
+    x = gc.to_device(conv_case(2, 8, 1, 4, torch.float32, seed=996))
+    e = {k: (v[..., :0].contiguous() if k in ("u", "delta", "z", "B", "C", "dy") else v)
+         for k, v in x.items()}
+    y, last = gpu_fwd(e)
+    assert y.numel() == 0 and torch.count_nonzero(last) == 0
+    g = gpu_bwd(e)
+    for k in ("dconv_w", "dconv_b", "dA", "dD", "ddelta_bias"):
+        assert torch.count_nonzero(g[k]) == 0, k

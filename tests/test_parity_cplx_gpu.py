@@ -68,7 +68,9 @@ def check(xh, fwd=True, bwd=True):
         assert not bad, f"gradient errors above {tol}: {bad} (all: {errs})"
 
 
-SHAPES = [(2, 200, 300, 16), (1, 70, 129, 8), (3, 5, 40, 1), (2, 130, 77, 4), (1, 33, 20, 3)]
+# N = 12 and 5 leave whole threads of a channel with padding states only
+SHAPES = [(2, 200, 300, 16), (1, 70, 129, 8), (3, 5, 40, 1), (2, 130, 77, 4), (1, 33, 20, 3),
+          (2, 50, 33, 12), (1, 40, 17, 5), (1, 9, 1, 16)]
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])

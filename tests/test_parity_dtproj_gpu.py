@@ -176,3 +176,11 @@ def test_dtproj_full_size_sampled():
     for k in ("dW_dt", "dA"):
         e = gc.normwise(gh[k].index_select(0, idx).double().numpy(), ref[k])
         assert e <= tol, f"{k}: {e:.2e}"
+
+
+@pytest.mark.parametrize("shape", [(2, 24, 1, 4, 3), (1, 16, 64, 8, 40)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_dtproj_edge_shapes(shape):
+    """A single step, and a rank above dim."""
+    b, d, L, N, R = shape
+    check(case(b, d, L, N, R, torch.float32, seed=1195 + L + R))
