@@ -81,6 +81,10 @@ struct BwdStagedArgs {
   uint64_t timeout_ns;
   int force_generic;
   int test_hook;  // 1: the last chunk of group 0 never publishes its adjoint (tests the bounded wait)
+  // three-phase carry of the adjoint (null in the sequential hand-off):
+  const float *gin;  // [G][K][NM][128] Abar G entering each chunk from the later one
+  float *agg_G;      // [G][K][NM][128] the same produced by each chunk from zero
+  double *agg_S;     // [G][K][128] sum of Delta over each chunk
 };
 
 // Byte offset of 16-byte chunk c of row r in a tile with RB-byte rows written
@@ -302,7 +306,11 @@ __global__ void __launch_bounds__(kSThreads, 2)
     float gt[NM];
 #pragma unroll
     for (int n = 0; n < NM; ++n) gt[n] = 0.f;
-    if (r > 0) {
+    if (p.gin) {  // three-phase carry: the entering adjoint is known
+#pragma unroll
+      for (int n = 0; n < NM; ++n)
+        gt[n] = __ldcg(p.gin + ((int64_t(g) * p.K + k) * NM + n) * kSThreads + tid);
+    } else if (r > 0) {
       if (tid == 0 && !wait_flag_geq(p.flags + g, r, p.timeout_ns)) {
         record_timeout();
         q[8] = 1;
@@ -704,7 +712,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
     for (int n = 0; n < NM; ++n) p.part_A[(pu * NM + n) * kSThreads + tid] = valid ? dA[n] : 0.f;
     p.part_D[pu * kSThreads + tid] = valid ? dDsum : 0.f;
     p.part_bias[pu * kSThreads + tid] = valid ? dbsum : 0.f;
-    if (k > 0) {
+    if (k > 0 && !p.gin) {
 #pragma unroll
       for (int n = 0; n < NM; ++n) p.carry[(int64_t(g) * NM + n) * kSThreads + tid] = gt[n];
       __threadfence();
@@ -721,6 +729,113 @@ __global__ void __launch_bounds__(kSThreads, 2)
   if (tid == 0 && aborted) {
     for (int t = ctile; t < p_issued; ++t)
       mbar_wait_bounded(&bars[t % kBStages], uint32_t(t / kBStages) & 1u, p.timeout_ns);
+  }
+}
+
+// Three-phase carry of the adjoint, used when there are too few channel groups
+// to fill the GPU with whole-sequence units.  The adjoint recurrence
+//     Ga_t = Abar_t (C_t dy0_t + Ga_{t+1})
+// does not involve the states, and it is linear: a chunk that starts from the
+// carried Ga_in produces  Ga_local + exp(A_n sum_chunk Delta) Ga_in,  where
+// Ga_local is what it produces from zero (the associative combine of affine
+// maps of the trishampatil.com walk-through, Part III section 2, run
+// backwards).  This kernel computes Ga_local and sum Delta of every chunk but
+// the first, one thread per (channel, chunk) walking the chunk from its end;
+// adjoint_carry_scan_kernel combines them, and the main reverse kernel then
+// runs every chunk from its true entering adjoint.
+template <typename T, int NM>
+__global__ void __launch_bounds__(kSThreads) bwd_adjoint_agg_kernel(const BwdStagedArgs p) {
+  constexpr int V = Vec<T>::kN;  // steps per 16-byte vector
+  __shared__ float cs[NM * V];   // the C rows of the current V steps
+  const BwdArgs &f = p.w;
+  const int unit = blockIdx.x;  // < G * (K - 1)
+  const int g = unit % p.G, k = p.K - 1 - unit / p.G;
+  const int b = g / p.gpb, d_raw = (g % p.gpb) * kSThreads + threadIdx.x;
+  const bool valid = d_raw < f.dim;
+  const int64_t d = valid ? d_raw : f.dim - 1;  // loads stay in bounds
+  const int N = f.N;
+  const int64_t row = (int64_t(b) * f.dim + d) * f.L;
+  const T *dl = static_cast<const T *>(f.delta) + row;
+  const T *dy = static_cast<const T *>(f.dy) + row;
+  const T *z = f.z ? static_cast<const T *>(f.z) + row : nullptr;
+  const T *Cp = static_cast<const T *>(f.C) + int64_t(b) * N * f.L;
+  const float bias = f.bias ? f.bias[d] : 0.f;
+  float Arow[NM], Ga[NM];
+#pragma unroll
+  for (int n = 0; n < NM; ++n) {
+    Arow[n] = n < N ? f.A[d * N + n] : float(n + 1) * f.A[d * N];
+    Ga[n] = 0.f;
+  }
+  // S4D-Real structure (as in the forward): all decays from one expm1
+  bool structured = Arow[0] < 0.f && isfinite(Arow[0]) && !p.force_generic;
+#pragma unroll
+  for (int n = 1; n < NM; ++n) structured = structured && (Arow[n] == float(n + 1) * Arow[0]);
+  const int64_t tbeg = int64_t(k) * p.chunk_len;
+  const int64_t tend = std::min<int64_t>(f.L, tbeg + p.chunk_len);
+  double S = 0.0;
+  // V steps at a time from the chunk's end (rows are 16-byte aligned multiples
+  // of 16 bytes and chunks start at multiples of 64 steps): every load of the V
+  // steps is issued before it is used
+  for (int64_t tb = tend - V; tb >= tbeg; tb -= V) {
+    float dv[V], dyv[V], zv[V];
+    Vec<T>::unpack(*reinterpret_cast<const uint4 *>(dl + tb), dv);
+    Vec<T>::unpack(*reinterpret_cast<const uint4 *>(dy + tb), dyv);
+    if (z) Vec<T>::unpack(*reinterpret_cast<const uint4 *>(z + tb), zv);
+    __syncthreads();  // the previous steps' C rows are no longer read
+    if (threadIdx.x < NM * V) {
+      const int n = threadIdx.x / V, i = threadIdx.x % V;
+      cs[threadIdx.x] = n < N ? to_f(Cp[int64_t(n) * f.L + tb + i]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = V - 1; i >= 0; --i) {
+      const float Delta = softplus_fast(dv[i] + bias);
+      S += double(Delta);
+      float dy0 = dyv[i];
+      if (z) dy0 *= zv[i] * rcpf(1.f + ex2f(-zv[i] * kLog2e));
+      if (structured) {
+        const float E1 = expm1_neg(Delta * Arow[0]);
+        f2 P[NM / 2];
+        decay_pairs<NM>(E1, 1.f + E1, P);
+        const f2 DY = pk(dy0, dy0);
+#pragma unroll
+        for (int j = 0; j < NM / 2; ++j) {
+          const f2 c = pk(cs[(2 * j) * V + i], cs[(2 * j + 1) * V + i]);
+          const f2 v = fma2(c, DY, pk(Ga[2 * j], Ga[2 * j + 1]));
+          const f2 w = fma2(P[j], v, v);  // Abar v = v + E v
+          Ga[2 * j] = lo_of(w);
+          Ga[2 * j + 1] = hi_of(w);
+        }
+      } else {
+#pragma unroll
+        for (int n = 0; n < NM; ++n)
+          if (n < N) Ga[n] = ex2f(Delta * Arow[n] * kLog2e) * fmaf(cs[n * V + i], dy0, Ga[n]);
+      }
+    }
+  }
+#pragma unroll
+  for (int n = 0; n < NM; ++n)
+    p.agg_G[((int64_t(g) * p.K + k) * NM + n) * kSThreads + threadIdx.x] = valid ? Ga[n] : 0.f;
+  p.agg_S[(int64_t(g) * p.K + k) * kSThreads + threadIdx.x] = valid ? S : 0.0;
+}
+
+// Ga_in(K-1) = 0, Ga_in(k-1) = exp(A_n S_k) Ga_in(k) + Ga_local(k), in fp64,
+// one thread per (group, state, channel).
+template <int NM>
+__global__ void adjoint_carry_scan_kernel(const BwdStagedArgs p) {
+  const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= int64_t(p.G) * NM * kSThreads) return;
+  const int c = int(idx % kSThreads);
+  const int n = int((idx / kSThreads) % NM);
+  const int g = int(idx / (int64_t(NM) * kSThreads));
+  const int d = (g % p.gpb) * kSThreads + c;
+  const double An = (d < p.w.dim && n < p.w.N) ? double(p.w.A[int64_t(d) * p.w.N + n]) : 0.0;
+  double G = 0.0;
+  for (int k = p.K - 1; k >= 0; --k) {
+    const int64_t base = int64_t(g) * p.K + k;
+    const_cast<float *>(p.gin)[(base * NM + n) * kSThreads + c] = float(G);
+    if (k > 0)
+      G = exp(An * p.agg_S[base * kSThreads + c]) * G + double(p.agg_G[(base * NM + n) * kSThreads + c]);
   }
 }
 
@@ -810,20 +925,25 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
   const int64_t gpb = ceil_div(a.dim, kSThreads);
   const int64_t G = int64_t(a.batch) * gpb;
   if (G > (int64_t(1) << 30)) return MAMBA_ERR_UNSUPPORTED;
-  StagedOptions ro = o;
-  ro.carry = 1;  // the adjoint crosses chunks by the sequential hand-off
-  StagedPlan pl = plan_staged(G, a.L, slots, ro);
+  // The adjoint crosses chunks by the sequential hand-off when the channel
+  // groups fill the GPU, else by the three-phase carry (whose aggregate pass is
+  // cheap here -- no states -- so it takes shorter chunks than the forward's).
+  StagedPlan pl = plan_staged(G, a.L, slots, o, 256);
+  const bool par = pl.kind == KIND_PAR;
   if (G * pl.K > (int64_t(1) << 30)) return MAMBA_ERR_UNSUPPORTED;
   const int64_t n16 = ceil_div(a.L, kBTT);
 
   // workspace: [ints][ckpt][carry][part_bc][part_A][part_D][part_bias]
+  //            (three-phase: + [agg_S][agg_G][gin])
   const size_t int_bytes = ceil_div((1 + size_t(G)) * 4, 256) * 256;
   const size_t n_ckpt = size_t(G) * size_t(n16) * NM * kSThreads;
   const size_t n_carry = size_t(G) * NM * kSThreads;
   const size_t n_bc = size_t(gpb) * size_t(a.batch) * 32 * size_t(a.L);
   const size_t gk = size_t(G) * size_t(pl.K);
   const size_t n_A = gk * NM * kSThreads, n_D = gk * kSThreads;
-  const size_t bytes = int_bytes + 4 * (n_ckpt + n_carry + n_bc + n_A + 2 * n_D);
+  const size_t n_par = par ? gk * NM * kSThreads : 0;  // agg_G and gin each
+  const size_t bytes = int_bytes + 4 * (n_ckpt + n_carry + n_bc + n_A + 2 * n_D) +
+                       (par ? 8 * n_D + 8 * n_par : 0);
   unsigned char *ws = nullptr;
   if (ws_alloc(reinterpret_cast<void **>(&ws), bytes, s) != cudaSuccess) {
     cudaGetLastError();
@@ -846,6 +966,14 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
   bp.part_A = bp.part_bc + n_bc;
   bp.part_D = bp.part_A + n_A;
   bp.part_bias = bp.part_D + n_D;
+  bp.gin = nullptr;
+  bp.agg_G = nullptr;
+  bp.agg_S = nullptr;
+  if (par) {
+    bp.agg_S = reinterpret_cast<double *>(bp.part_bias + n_D);  // 8-byte aligned: offsets are
+    bp.agg_G = reinterpret_cast<float *>(bp.agg_S + n_D);       // multiples of 128 floats
+    bp.gin = bp.agg_G + n_par;
+  }
   bp.timeout_ns = o.timeout_us > 0 ? uint64_t(o.timeout_us) * 1000ull : kDefaultTimeoutNs;
   bp.force_generic = o.path == MAMBA_PATH_GENERIC ? 1 : 0;
   bp.test_hook = o.test_hook;
@@ -863,6 +991,15 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
     fo.carry = 0;
     fo.test_hook = 0;  // the hook targets the reverse hand-off
     st = staged_forward<T, NM, CONV>(fa, fo, s, launched, ckpt);
+  }
+  if (st == MAMBA_OK && par) {
+    bwd_adjoint_agg_kernel<T, NM><<<unsigned(size_t(G) * size_t(pl.K - 1)), kSThreads, 0, s>>>(bp);
+    st = launched();
+    if (st == MAMBA_OK) {
+      const int64_t threads = G * NM * kSThreads;
+      adjoint_carry_scan_kernel<NM><<<unsigned(ceil_div(threads, 256)), 256, 0, s>>>(bp);
+      st = launched();
+    }
   }
   if (st == MAMBA_OK) {
     kern<<<unsigned(std::min<int64_t>(gk, slots)), kSThreads, Lay::ALLOC, s>>>(

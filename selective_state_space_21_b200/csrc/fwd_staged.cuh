@@ -747,7 +747,8 @@ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // Picks the chunking: the sequential hand-off when the channel groups alone
 // fill the resident CTAs (about eight chunks per group keeps the tail short),
 // else the three-phase scheme with about four units per resident CTA.
-inline StagedPlan plan_staged(int64_t G, int64_t L, int slots, const StagedOptions &o) {
+inline StagedPlan plan_staged(int64_t G, int64_t L, int slots, const StagedOptions &o,
+                              int64_t min_par_chunk = 512) {
   StagedPlan pl;
   int carry = o.carry;
   if (carry == 0) carry = G >= slots ? 1 : 2;
@@ -758,7 +759,7 @@ inline StagedPlan plan_staged(int64_t G, int64_t L, int slots, const StagedOptio
       chunk = std::max<int64_t>(256, ceil_div(ceil_div(L, kt), 64) * 64);
     } else {
       const int64_t kt = std::max<int64_t>(1, ceil_div(4 * int64_t(slots), G));
-      chunk = std::max<int64_t>(512, ceil_div(ceil_div(L, kt), 64) * 64);
+      chunk = std::max<int64_t>(min_par_chunk, ceil_div(ceil_div(L, kt), 64) * 64);
     }
   }
   chunk = std::min<int64_t>(chunk, ceil_div(L, 64) * 64);

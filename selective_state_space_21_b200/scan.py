@@ -170,8 +170,8 @@ def mamba_scan_fwd(u, delta, delta_bias, A, B, C, D, z, y, last_state, *, path="
 
 
 def mamba_scan_bwd(u, delta, delta_bias, A, B, C, D, z, dy, du, ddelta, dA, dB, dC, dD, dz,
-                   ddelta_bias, *, path="auto", chunk_len=0, wait_timeout_us=0, test_hook=0,
-                   stream=None):
+                   ddelta_bias, *, path="auto", chunk_len=0, carry="auto", wait_timeout_us=0,
+                   test_hook=0, stream=None):
     """Enqueue the backward of sum(dy * y) on ``stream``; the gradient tensors
     are written."""
     batch, dim, L = u.shape
@@ -189,10 +189,11 @@ def mamba_scan_bwd(u, delta, delta_bias, A, B, C, D, z, dy, du, ddelta, dA, dB, 
         _ptr(dz, dt, bdl, "dz"), _ptr(ddelta_bias, f32, (dim,), "ddelta_bias"),
         batch, dim, L, N, _dtype_code(dt)]
     lib = load_library()
-    if path == "auto" and not chunk_len and not wait_timeout_us and not test_hook:
+    if path == "auto" and not chunk_len and carry == "auto" and not wait_timeout_us \
+            and not test_hook:
         rc = lib.mamba_scan_bwd(*args, _stream_handle(stream))
     else:
-        opts = _options(path, chunk_len, "auto", wait_timeout_us, test_hook)
+        opts = _options(path, chunk_len, carry, wait_timeout_us, test_hook)
         rc = lib.mamba_scan_bwd_ex(*args, ctypes.byref(opts), _stream_handle(stream))
     _check(rc, "mamba_scan_bwd")
 
@@ -231,7 +232,7 @@ def mamba_conv_scan_fwd(x, conv_w, conv_b, delta, delta_bias, A, B, C, D, z, y, 
 
 def mamba_conv_scan_bwd(x, conv_w, conv_b, delta, delta_bias, A, B, C, D, z, dy, dx, dconv_w,
                         dconv_b, ddelta, dA, dB, dC, dD, dz, ddelta_bias, *, path="auto",
-                        chunk_len=0, wait_timeout_us=0, test_hook=0, stream=None):
+                        chunk_len=0, carry="auto", wait_timeout_us=0, test_hook=0, stream=None):
     """Enqueue the backward of sum(dy * y) for ``mamba_conv_scan_fwd``: dx
     and dconv_w (and dconv_b if given) take the place of du."""
     batch, dim, L = x.shape
@@ -251,7 +252,7 @@ def mamba_conv_scan_bwd(x, conv_w, conv_b, delta, delta_bias, A, B, C, D, z, dy,
         _ptr(dA, f32, (dim, N), "dA"), _ptr(dB, dt, bnl, "dB"), _ptr(dC, dt, bnl, "dC"),
         _ptr(dD, f32, (dim,), "dD"), _ptr(dz, dt, bdl, "dz"),
         _ptr(ddelta_bias, f32, (dim,), "ddelta_bias"), batch, dim, L, N, _dtype_code(dt)]
-    opts = _opts_ptr(path, chunk_len, "auto", wait_timeout_us, test_hook)
+    opts = _opts_ptr(path, chunk_len, carry, wait_timeout_us, test_hook)
     _check(load_library().mamba_conv_scan_bwd(*args, opts, _stream_handle(stream)),
            "mamba_conv_scan_bwd")
 
@@ -435,7 +436,7 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
 
 
 def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, path="auto",
-                       chunk_len=0, stream=None) -> dict:
+                       chunk_len=0, carry="auto", stream=None) -> dict:
     """Allocate the gradients and run the backward; returns a dict of them."""
     dim, N = A.shape
     f32 = torch.float32
@@ -449,7 +450,7 @@ def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, p
     }
     mamba_scan_bwd(u, delta, delta_bias, A, B, C, D, z, dy, g["du"], g["ddelta"], g["dA"],
                    g["dB"], g["dC"], g["dD"], g["dz"], g["ddelta_bias"], path=path,
-                   chunk_len=chunk_len, stream=stream)
+                   chunk_len=chunk_len, carry=carry, stream=stream)
     return {k: v for k, v in g.items() if v is not None}
 
 
@@ -468,7 +469,8 @@ def conv_selective_scan_fwd(x, conv_w, conv_b, delta, A, B, C, D=None, z=None, d
 
 
 def conv_selective_scan_bwd(x, conv_w, conv_b, delta, A, B, C, dy, D=None, z=None,
-                            delta_bias=None, path="auto", chunk_len=0, stream=None) -> dict:
+                            delta_bias=None, path="auto", chunk_len=0, carry="auto",
+                            stream=None) -> dict:
     """Allocate the gradients and run the backward with the convolution
     prologue; returns a dict of them (dx, dconv_w, dconv_b if conv_b is given,
     and the scan's other gradients)."""
@@ -486,5 +488,6 @@ def conv_selective_scan_bwd(x, conv_w, conv_b, delta, A, B, C, dy, D=None, z=Non
     }
     mamba_conv_scan_bwd(x, conv_w, conv_b, delta, delta_bias, A, B, C, D, z, dy, g["dx"],
                         g["dconv_w"], g["dconv_b"], g["ddelta"], g["dA"], g["dB"], g["dC"], g["dD"],
-                        g["dz"], g["ddelta_bias"], path=path, chunk_len=chunk_len, stream=stream)
+                        g["dz"], g["ddelta_bias"], path=path, chunk_len=chunk_len, carry=carry,
+                        stream=stream)
     return {k: v for k, v in g.items() if v is not None}

@@ -36,10 +36,10 @@ def gpu_fwd(x: dict, path="auto", chunk_len=0, last=True, carry="auto"):
     return out if last else (out, None)
 
 
-def gpu_bwd(x: dict, path="auto", chunk_len=0) -> dict:
+def gpu_bwd(x: dict, path="auto", chunk_len=0, carry="auto") -> dict:
     g = scan.selective_scan_bwd(x["u"], x["delta"], x["A"], x["B"], x["C"], x["dy"], D=x["D"],
                                 z=x["z"], delta_bias=x["delta_bias"], path=path,
-                                chunk_len=chunk_len)
+                                chunk_len=chunk_len, carry=carry)
     assert scan.mamba_scan_stream_status() == 0
     return g
 

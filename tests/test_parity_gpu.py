@@ -217,12 +217,15 @@ def test_bwd_staged_grid(shape, dtype, path):
     _bwd_case(make_inputs(b, d, L, N, dtype, seed=400 + L + d, with_dy=True), path)
 
 
+@pytest.mark.parametrize("carry", ["sequential", "three_phase"])
 @pytest.mark.parametrize("chunk_len", [64, 256, 4096])
-def test_bwd_chunking(chunk_len):
-    """The adjoint crosses chunk boundaries (backwards hand-off) exactly."""
+def test_bwd_chunking(chunk_len, carry):
+    """The adjoint crosses chunk boundaries exactly, by the backwards hand-off
+    and by the three-phase carry (chunk aggregates, a scan over chunks, then
+    every chunk from its true entering adjoint)."""
     x = make_inputs(2, 160, 2048, 16, torch.float32, seed=51, with_dy=True)
     xd = gc.to_device(x)
-    g = gc.gpu_bwd(xd, chunk_len=chunk_len)
+    g = gc.gpu_bwd(xd, chunk_len=chunk_len, carry=carry)
     ref = gc.oracle_bwd(x)
     for k in GRAD_KEYS:
         e = gc.normwise(g[k].cpu().double().numpy(), ref[k])
@@ -250,7 +253,7 @@ def test_bwd_reverse_wait_times_out_without_hanging():
     du, dd, dz = torch.empty_like(x["u"]), torch.empty_like(x["u"]), torch.empty_like(x["u"])
     scan.mamba_scan_bwd(x["u"], x["delta"], x["delta_bias"], x["A"], x["B"], x["C"], x["D"],
                         x["z"], x["dy"], du, dd, dA, g["B"], g["C"], dD, dz, db, chunk_len=128,
-                        wait_timeout_us=2000, test_hook=1)
+                        carry="sequential", wait_timeout_us=2000, test_hook=1)
     assert scan.mamba_scan_stream_status() == 5  # MAMBA_ERR_DEVICE_TIMEOUT
     assert scan.mamba_scan_stream_status() == 0
     _bwd_case(xh)
@@ -394,3 +397,20 @@ def test_invalid_arguments_are_rejected_on_the_host():
     # nothing was launched by the rejected calls: y still zero from the good call's input
     torch.cuda.synchronize()
     assert torch.isfinite(y).all()
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_bwd_three_phase_generic_and_mixed_A(dtype):
+    """The three-phase adjoint carry with channels off the structured form
+    (its aggregate pass takes one exp per state for every A)."""
+    x = make_inputs(1, 260, 1024, 16, dtype, seed=59, with_dy=True)
+    g = torch.Generator().manual_seed(5)
+    x["A"] = -torch.exp(torch.randn(260, 16, generator=g)).contiguous()
+    x["A"][:130] = -torch.arange(1, 17, dtype=torch.float32)  # one structured group
+    xd = gc.to_device(x)
+    gg = gc.gpu_bwd(xd, chunk_len=128, carry="three_phase")
+    ref = gc.oracle_bwd(x)
+    tol = gc.TOL[dtype]
+    for k in GRAD_KEYS:
+        e = gc.normwise(gg[k].cpu().double().numpy(), ref[k])
+        assert e <= tol, f"{k}: {e:.2e}"
