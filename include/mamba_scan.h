@@ -92,9 +92,12 @@ typedef struct {
   int32_t path;            /* a mamba_path_t */
   int32_t chunk_len;       /* time steps per chunk of the chunked kernels; 0 = automatic,
                               else a positive multiple of 64 */
-  int32_t carry;           /* how a chunk's end state reaches the next chunk: 0 = automatic,
-                              1 = sequential hand-off (a bounded wait on the predecessor),
-                              2 = three-phase (aggregate, scan over chunks, recompute) */
+  int32_t carry;           /* how a chunk's end state (in the backward: the adjoint entering
+                              from the later chunk) crosses chunk boundaries: 0 = automatic
+                              (sequential when the channel groups fill the GPU),
+                              1 = sequential hand-off (a bounded wait on the neighbour),
+                              2 = three-phase (chunk aggregates, a scan over chunks, then every
+                              chunk from its true entering value) */
   int32_t wait_timeout_us; /* bound of every device-side wait; 0 = 2,000,000 (2 s) */
   int32_t test_hook;       /* 0 in normal use.  1: the first chunk processed of the first
                               channel group (the first in time for the forward, the last for
