@@ -94,20 +94,26 @@ def measured_peaks() -> dict:
         return {"hbm_gbs": FALLBACK_HBM_GBS, "source": "fallback"}
 
 
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_bytes_per_launch_bf16_b8_d5120_L2048_N16.txt")
+
+
 def ncu_traffic(kernel_key: str):
-    """Per-launch DRAM bytes from a committed ncu summary, only if it was taken
-    on the current source of that kernel (else None)."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
+    """Per-launch DRAM bytes of one call ("fwd" or "bwd") from the committed ncu
+    summary, only if it was taken on the current source of the staged kernels
+    (else None).  Lines: <call> <bytes> <source digest> <launches>; # comments."""
     try:
-        with open(p) as f:
-            d = json.load(f)
-        e = d[kernel_key]
         from selective_state_space_21_b200.build import STAGED_KERNEL_FILES, source_digest
-        if e.get("source_digest") != source_digest(STAGED_KERNEL_FILES):
-            return None
-        return e
+        with open(TRAFFIC_FILE) as f:
+            for line in f:
+                parts = line.split()
+                if not parts or parts[0].startswith("#") or parts[0] != kernel_key:
+                    continue
+                if parts[2] != source_digest(STAGED_KERNEL_FILES):
+                    return None
+                return {"bytes_per_launch": int(parts[1]), "source_digest": parts[2]}
     except Exception:
         return None
+    return None
 
 
 # ------------------------------------------------------------------ clocks
