@@ -82,7 +82,7 @@ struct BwdStagedArgs {
   int force_generic;
   int test_hook;  // 1: the last chunk of group 0 never publishes its adjoint (tests the bounded wait)
   // three-phase carry of the adjoint (null in the sequential hand-off):
-  const float *gin;  // [G][K][NM][128] Abar G entering each chunk from the later one
+  float *gin;        // [G][K][NM][128] Abar G entering each chunk from the later one
   float *agg_G;      // [G][K][NM][128] the same produced by each chunk from zero
   double *agg_S;     // [G][K][128] sum of Delta over each chunk
 };
@@ -833,7 +833,7 @@ __global__ void adjoint_carry_scan_kernel(const BwdStagedArgs p) {
   double G = 0.0;
   for (int k = p.K - 1; k >= 0; --k) {
     const int64_t base = int64_t(g) * p.K + k;
-    const_cast<float *>(p.gin)[(base * NM + n) * kSThreads + c] = float(G);
+    p.gin[(base * NM + n) * kSThreads + c] = float(G);
     if (k > 0)
       G = exp(An * p.agg_S[base * kSThreads + c]) * G + double(p.agg_G[(base * NM + n) * kSThreads + c]);
   }

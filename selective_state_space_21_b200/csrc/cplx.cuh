@@ -31,8 +31,6 @@
 // with deterministic reductions as in the real kernels.
 #pragma once
 
-#include "bwd_reference.cuh"
-#include "bwd_staged.cuh"
 #include "common.cuh"
 #include "fwd_staged.cuh"
 

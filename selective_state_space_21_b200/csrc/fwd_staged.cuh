@@ -114,16 +114,8 @@ __device__ __forceinline__ f2 pk(float lo, float hi) {
   asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
   return r;
 }
-__device__ __forceinline__ float lo_of(f2 v) {
-  float lo, hi;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-  return lo;
-}
-__device__ __forceinline__ float hi_of(f2 v) {
-  float lo, hi;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-  return hi;
-}
+__device__ __forceinline__ float lo_of(f2 v) { return __uint_as_float(unsigned(v)); }
+__device__ __forceinline__ float hi_of(f2 v) { return __uint_as_float(unsigned(v >> 32)); }
 __device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
   f2 d;
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
