@@ -639,6 +639,25 @@ def pin_cplx_zoh_expm(lib=None):
     return normwise(y[0], ref), 1e-12
 
 
+def pin_cplx_held_input_exact(lib=None):
+    """u = 1, B = 1, C = 1 (complex ones), time-varying Delta: for a held
+    input the zero-order hold is exact, so each complex state is the ODE
+    solution h_n(t) = (exp(A_n T_t) - 1) / A_n with T_t = sum_{j<=t} Delta_j,
+    and y_t = Re(sum_n h_n(t)); numpy's complex exp on the closed form."""
+    N, L = 5, 120
+    x = make_inputs(1, 2, L, N, seed=304, has_z=False, has_D=False)
+    Ac = np.array([[-0.5 + 1j * n for n in range(N)], [-1.5 + 0.3j * n - 0.2j for n in range(N)]])
+    A = np.concatenate([Ac.real, Ac.imag], axis=1)
+    ones = np.concatenate([np.ones((1, N, L)), np.zeros((1, N, L))], axis=1)
+    y, last = oracle.s6_cplx_forward(np.ones((1, 2, L)), x["delta"], A, ones, ones,
+                                     x["delta_bias"], lib=lib)
+    Delta = _softplus(_np(x["delta"])[0] + _np(x["delta_bias"])[:, None])
+    T = np.cumsum(Delta, axis=1)  # (dim, L)
+    h = (np.exp(Ac[:, :, None] * T[:, None, :]) - 1.0) / Ac[:, :, None]  # (dim, N, L)
+    ref_last = np.concatenate([h[:, :, -1].real, h[:, :, -1].imag], axis=1)
+    return max(normwise(y[0], h.sum(axis=1).real), normwise(last[0], ref_last)), 1e-12
+
+
 def _cplx_fd_inputs():
     x = make_cplx_inputs(1, 2, 9, 2, seed=93, with_dy=True)
     return {k: (v.double() if v is not None else None) for k, v in x.items()}
@@ -713,7 +732,7 @@ ALL_PINS = [pin_golden, pin_theorem1, pin_zoh_expm, pin_lti_convolution, pin_bru
             pin_threads_agree, pin_resume_from_state, pin_initial_state_decay,
             pin_conv_numpy, pin_conv_special_filters, pin_conv_finite_differences,
             pin_conv_autograd, pin_dtproj_matmul, pin_dtproj_finite_differences,
-            pin_dtproj_autograd, pin_cplx_real_case, pin_cplx_zoh_expm,
+            pin_dtproj_autograd, pin_cplx_real_case, pin_cplx_zoh_expm, pin_cplx_held_input_exact,
             pin_cplx_finite_differences, pin_cplx_autograd]
 
 
