@@ -18,8 +18,10 @@
 // fp32 tables.  In general each state costs three special-function
 // operations per step (exp of the real part, sine and cosine of the
 // range-reduced half of the imaginary part) and about 35 FP32 operations,
-// without branches; states with the S4D-Lin structure share one exp and two
-// sine/cosine pairs per thread and step and take 14 FP32 operations each.
+// without branches.  A thread whose states have the S4D-Lin structure shares
+// one exp and two sine/cosine pairs per step over them; where also |A| >= 1/8
+// the update takes the form h += (Abar - 1)(h + (B/A) u), 10 FP32 operations
+// per state on top of the 7 of its decay.
 //
 // The backward follows the real one-thread-per-channel kernel: a forward
 // sweep keeps the state at the start of every block of steps, the reverse
@@ -28,7 +30,8 @@
 // product by the conjugate of the other factor):
 //     G_t = conj(C_t) dy0_t + conj(Abar_{t+1}) G_{t+1},
 //     du += Re(conj(G) Bbar),  dDelta += Re(conj(G) Abar (A h_{t-1} + B u)),
-//     gA += conj(Delta Abar h_{t-1} + Delta^2 phi(Delta A) B u) G,
+//     gA += conj(Delta Abar h_{t-1} + Delta^2 phi(Delta A) B u) G
+//        (= conj(1/A) conj(Delta dh/dDelta - Bbar u) G, used where |A| >= 1/8),
 //     gB += conj(Delta psi(Delta A)) u G,  gC += conj(h_t) dy0,
 // with deterministic reductions as in the real kernels.
 #pragma once
@@ -109,41 +112,89 @@ __device__ __forceinline__ bool cplx_lin_structure(const float (&ar)[NS], const 
   return lin && (ai[0] == 0.f || ai[0] * c >= 0.f);
 }
 
+// M_j = Abar_j - 1 = exp(Delta A_j) - 1 for a thread's NS states with the
+// S4D-Lin structure A_j = a + i (b + j c): M_j = expm1(Delta a) + e^{Delta a}
+// (e^{i th_j} - 1) with th_j = Delta (b + j c) and e^{i th} - 1 =
+// 2i sin(th/2) e^{i th/2}; the half angles e^{i th_j/2} follow from
+// e^{i th_0/2} by repeated multiplication with e^{i Delta c/2}.  One exp and
+// two sine/cosine pairs per step, 7 FP32 operations per state, all free of
+// cancellation.
+template <int NS>
+__device__ __forceinline__ void cplx_lin_m(float Delta, float a, float b, float c, float (&Mr)[NS],
+                                           float (&Mi)[NS]) {
+  const float xr = Delta * a;
+  const float ea = ex2f(xr * kLog2e);
+  const float pm = xr * (1.f + xr * (0.5f + xr * (1.f / 6.f + xr * (1.f / 24.f + xr * (1.f / 120.f +
+                   xr * (1.f / 720.f))))));
+  const float em = fabsf(xr) < 0.25f ? pm : ea - 1.f;
+  const float ea2 = 2.f * ea;
+  float qr, qi, zr, zi;
+  cis_reduced(0.5f * Delta * b, qr, qi);
+  cis_reduced(0.5f * Delta * c, zr, zi);
+#pragma unroll
+  for (int j = 0; j < NS; ++j) {
+    const float t = ea2 * qi;
+    Mr[j] = fmaf(-t, qi, em);  // expm1(Delta a) - 2 e^{Delta a} sin^2(th/2)
+    Mi[j] = t * qr;            // 2 e^{Delta a} sin(th/2) cos(th/2)
+    if (j + 1 < NS) {
+      const float nr = fmaf(qr, zr, -qi * zi);
+      qi = fmaf(qr, zi, qi * zr);
+      qr = nr;
+    }
+  }
+}
+
+// The spacing c of a thread's imaginary parts (0 with one state).
+template <int NS>
+__device__ __forceinline__ float cplx_lin_step(const float (&ai)[NS]) {
+  return NS > 1 ? ai[NS > 1 ? 1 : 0] - ai[0] : 0.f;
+}
+
+// Whether every state of the thread has |A| >= 1/8, so that forms divided by
+// A lose no more than a few ulp against the other terms.
+template <int NS>
+__device__ __forceinline__ bool cplx_not_small(const float (&ar)[NS], const float (&ai)[NS]) {
+  bool ok = true;
+#pragma unroll
+  for (int j = 0; j < NS; ++j) ok = ok && ar[j] * ar[j] + ai[j] * ai[j] >= 1.f / 64.f;
+  return ok;
+}
+
+// One step of a thread's states in the form h += M (h + (B/A) u), M = Abar - 1
+// (S4D-Lin structure and |A| >= 1/8): E B u = M (B/A) u without forming E.
+// bre / bim point at the staged Re B and Im B of this thread's states.
+template <int NS>
+__device__ __forceinline__ void cplx_update_m(const float (&Mr)[NS], const float (&Mi)[NS],
+                                              const float (&ira)[NS], const float (&iai)[NS],
+                                              float ut, const float *bre, const float *bim,
+                                              float (&hr)[NS], float (&hi)[NS]) {
+#pragma unroll
+  for (int j = 0; j < NS; ++j) {
+    const float br = bre[j], bi = bim[j];
+    const float wr = fmaf(br, ira[j], -bi * iai[j]), wi = fmaf(br, iai[j], bi * ira[j]);  // B/A
+    const float sr = fmaf(wr, ut, hr[j]), si = fmaf(wi, ut, hi[j]);
+    hr[j] = fmaf(Mr[j], sr, fmaf(-Mi[j], si, hr[j]));
+    hi[j] = fmaf(Mr[j], si, fmaf(Mi[j], sr, hi[j]));
+  }
+}
+
 // Decays of a thread's NS states at one step: Abar_j = exp(Delta A_j) and
-// E_j = (Abar_j - 1)/A_j.  With the S4D-Lin structure, Abar_j - 1 =
-// expm1(Delta a) + e^{Delta a} (e^{i th_j} - 1) with th_j = Delta (b + j c) and
-// e^{i th} - 1 = 2i sin(th/2) e^{i th/2}; the half angles e^{i th_j/2} follow
-// from e^{i th_0/2} by repeated multiplication with e^{i Delta c/2}.  That is
-// one exp and two sine/cosine pairs per step, and 14 FP32 operations per
-// state, all free of cancellation.  Otherwise each state takes cplx_decay.
+// E_j = (Abar_j - 1)/A_j, from cplx_lin_m with the S4D-Lin structure, else
+// per state from cplx_decay.
 template <int NS>
 __device__ __forceinline__ void cplx_decays(float Delta, bool lin, const float (&ar)[NS],
                                             const float (&ai)[NS], const float (&ira)[NS],
                                             const float (&iai)[NS], float (&abr)[NS],
                                             float (&abi)[NS], float (&Er)[NS], float (&Ei)[NS]) {
   if (lin) {
-    const float xr = Delta * ar[0];
-    const float ea = ex2f(xr * kLog2e);
-    const float pm = xr * (1.f + xr * (0.5f + xr * (1.f / 6.f + xr * (1.f / 24.f + xr * (1.f / 120.f +
-                     xr * (1.f / 720.f))))));
-    const float em = fabsf(xr) < 0.25f ? pm : ea - 1.f;
-    float qr, qi, zr, zi;
-    cis_reduced(0.5f * Delta * ai[0], qr, qi);
-    cis_reduced(0.5f * Delta * (NS > 1 ? ai[NS > 1 ? 1 : 0] - ai[0] : 0.f), zr, zi);
+    float Mr[NS], Mi[NS];
+    cplx_lin_m<NS>(Delta, ar[0], ai[0], cplx_lin_step<NS>(ai), Mr, Mi);
 #pragma unroll
     for (int j = 0; j < NS; ++j) {
-      const float t2 = 2.f * qi;
-      const float mr0 = -t2 * qi, mi0 = t2 * qr;  // e^{i th} - 1
-      const float Mr = fmaf(ea, mr0, em), Mi = ea * mi0;  // Abar - 1
-      abr[j] = 1.f + Mr;
-      abi[j] = Mi;
-      Er[j] = fmaf(Mr, ira[j], -Mi * iai[j]);
-      Ei[j] = fmaf(Mr, iai[j], Mi * ira[j]);
-      if (j + 1 < NS) {
-        const float nr = fmaf(qr, zr, -qi * zi);
-        qi = fmaf(qr, zi, qi * zr);
-        qr = nr;
-      }
+      abr[j] = 1.f + Mr[j];
+      abi[j] = Mi[j];
+      Er[j] = fmaf(Mr[j], ira[j], -Mi[j] * iai[j]);
+      Ei[j] = fmaf(Mr[j], iai[j], Mi[j] * ira[j]);
     }
   } else {
 #pragma unroll
@@ -176,8 +227,13 @@ __device__ __forceinline__ void cplx_phi(float xr, float xi, float er, float ei,
   pi = small ? ai : fmaf(ni, x2r, -nr * x2i) * den;
 }
 
+// Row stride of the staged tables: one float of padding, so that the staging
+// writes (consecutive threads, consecutive steps) fall in distinct banks.
+template <int NM> constexpr int cplx_tab_stride() { return 4 * NM + 1; }
+
 // Stages the B and C columns of steps [t0, t0 + TT) of batch row b into
-// tab[t][4 NM] = (Re B, Im B, Re C, Im C) as fp32, zero past N and past L.
+// tab[t][4 NM] = (Re B, Im B, Re C, Im C) as fp32 (rows cplx_tab_stride apart),
+// zero past N and past L.
 template <typename T, int NM, int TT>
 __device__ __forceinline__ void cplx_stage_bc(const CplxArgs &a, int64_t b, int64_t t0, float *tab,
                                               bool with_c, int nthreads) {
@@ -193,7 +249,7 @@ __device__ __forceinline__ void cplx_stage_bc(const CplxArgs &a, int64_t b, int6
       const T *src = part < 2 ? Bp : Cp;
       v = to_f(src[(int64_t(part & 1) * N + n) * a.L + tt]);
     }
-    tab[t * 4 * NM + slot] = v;
+    tab[t * cplx_tab_stride<NM>() + slot] = v;
   }
 }
 
@@ -203,7 +259,7 @@ __device__ __forceinline__ void cplx_stage_bc(const CplxArgs &a, int64_t b, int6
 template <typename T, int NM, int TPC>
 __global__ void __launch_bounds__(kCplxThreads) cplx_fwd_kernel(const CplxArgs a) {
   constexpr int NS = NM / TPC;  // states per thread
-  __shared__ __align__(16) float tab[kCplxTT * 4 * NM];
+  __shared__ __align__(16) float tab[kCplxTT * cplx_tab_stride<NM>()];
   const int tid = threadIdx.x;
   const int part = tid % TPC;
   const int64_t b = blockIdx.y;
@@ -230,6 +286,8 @@ __global__ void __launch_bounds__(kCplxThreads) cplx_fwd_kernel(const CplxArgs a
     hr[j] = hi[j] = 0.f;
   }
   const bool lin = cplx_lin_structure<NS>(ar, ai);
+  const bool mform = lin && cplx_not_small<NS>(ar, ai);
+  const float clin = cplx_lin_step<NS>(ai);
   for (int64_t t0 = 0; t0 < a.L; t0 += kCplxTT) {
     __syncthreads();
     cplx_stage_bc<T, NM, kCplxTT>(a, b, t0, tab, true, kCplxThreads);
@@ -239,22 +297,29 @@ __global__ void __launch_bounds__(kCplxThreads) cplx_fwd_kernel(const CplxArgs a
       const int64_t t = t0 + i;
       const float Delta = softplus_fast(to_f(dl[t]) + bias);
       const float ut = to_f(u[t]);
-      const float *tr = tab + i * 4 * NM + part * NS;
+      const float *tr = tab + i * cplx_tab_stride<NM>() + part * NS;
       float y0 = Dd * ut;
-      float Abr[NS], Abi[NS], Ebr[NS], Ebi[NS];
-      cplx_decays<NS>(Delta, lin, ar, ai, ira, iai, Abr, Abi, Ebr, Ebi);
+      if (mform) {
+        float Mr[NS], Mi[NS];
+        cplx_lin_m<NS>(Delta, ar[0], ai[0], clin, Mr, Mi);
+        cplx_update_m<NS>(Mr, Mi, ira, iai, ut, tr, tr + NM, hr, hi);
+      } else {
+        float Abr[NS], Abi[NS], Ebr[NS], Ebi[NS];
+        cplx_decays<NS>(Delta, lin, ar, ai, ira, iai, Abr, Abi, Ebr, Ebi);
 #pragma unroll
-      for (int j = 0; j < NS; ++j) {
-        const float abr = Abr[j], abi = Abi[j], Er = Ebr[j], Ei = Ebi[j];
-        const float br = tr[j], bi = tr[NM + j], cr = tr[2 * NM + j], ci = tr[3 * NM + j];
-        // Bbar u = E B u
-        const float bbr = fmaf(Er, br, -Ei * bi) * ut, bbi = fmaf(Er, bi, Ei * br) * ut;
-        const float nr = fmaf(abr, hr[j], fmaf(-abi, hi[j], bbr));
-        const float ni = fmaf(abr, hi[j], fmaf(abi, hr[j], bbi));
-        hr[j] = nr;
-        hi[j] = ni;
-        y0 = fmaf(cr, nr, fmaf(-ci, ni, y0));
+        for (int j = 0; j < NS; ++j) {
+          const float abr = Abr[j], abi = Abi[j], Er = Ebr[j], Ei = Ebi[j];
+          const float br = tr[j], bi = tr[NM + j];
+          // Bbar u = E B u
+          const float bbr = fmaf(Er, br, -Ei * bi) * ut, bbi = fmaf(Er, bi, Ei * br) * ut;
+          const float nr = fmaf(abr, hr[j], fmaf(-abi, hi[j], bbr));
+          const float ni = fmaf(abr, hi[j], fmaf(abi, hr[j], bbi));
+          hr[j] = nr;
+          hi[j] = ni;
+        }
       }
+#pragma unroll
+      for (int j = 0; j < NS; ++j) y0 = fmaf(tr[2 * NM + j], hr[j], fmaf(-tr[3 * NM + j], hi[j], y0));
 #pragma unroll
       for (int o = 1; o < TPC; o <<= 1) y0 += __shfl_xor_sync(0xffffffffu, y0, o);
       if (z) {
@@ -328,8 +393,8 @@ __global__ void __launch_bounds__(kCplxBwdThreads, 8) cplx_bwd_kernel(const Cplx
   constexpr int NKEEP = NV * TPC / 32;         // sums left on each lane
   extern __shared__ __align__(16) float smem[];
   float *hs = smem;                                          // [TC][2 NS][threads]
-  float *tab = hs + kCplxBwdTC * 2 * NS * kCplxBwdThreads;  // [TC][4 NM]
-  float *wsum = tab + kCplxBwdTC * 4 * NM;                   // [2 warps][4 kMaxN][TC]
+  float *tab = hs + kCplxBwdTC * 2 * NS * kCplxBwdThreads;  // [TC][stride]
+  float *wsum = tab + kCplxBwdTC * cplx_tab_stride<NM>();    // [2 warps][4 kMaxN][TC]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int part = tid % TPC;
   const int64_t b = blockIdx.y;
@@ -364,12 +429,18 @@ __global__ void __launch_bounds__(kCplxBwdThreads, 8) cplx_bwd_kernel(const Cplx
   // dA through A dh/dA = Delta dh/dDelta - E B u (no phi) where every state of
   // the thread has |A| >= 1/8; the fp32 error of that difference, relative to
   // the other terms of dA, is then about 8 eps.  Smaller |A| take phi.
-  bool ident = true;
-#pragma unroll
-  for (int j = 0; j < NS; ++j) ident = ident && ar[j] * ar[j] + ai[j] * ai[j] >= 1.f / 64.f;
+  const bool ident = cplx_not_small<NS>(ar, ai);
+  const bool mform = lin && ident;
+  const float clin = cplx_lin_step<NS>(ai);
 
   // one forward step of this thread's states (B from the staged table row)
   auto step = [&](float Delta, float ut, const float *trow) {
+    if (mform) {
+      float Mr[NS], Mi[NS];
+      cplx_lin_m<NS>(Delta, ar[0], ai[0], clin, Mr, Mi);
+      cplx_update_m<NS>(Mr, Mi, ira, iai, ut, trow + part * NS, trow + NM + part * NS, hr, hi);
+      return;
+    }
     float Abr[NS], Abi[NS], Ebr[NS], Ebi[NS];
     cplx_decays<NS>(Delta, lin, ar, ai, ira, iai, Abr, Abi, Ebr, Ebi);
 #pragma unroll
@@ -397,7 +468,7 @@ __global__ void __launch_bounds__(kCplxBwdThreads, 8) cplx_bwd_kernel(const Cplx
     __syncthreads();
     const int steps = int(a.L - t0 < kCplxBwdTC ? a.L - t0 : kCplxBwdTC);
     for (int i = 0; i < steps; ++i)
-      step(softplus_fast(to_f(dl[t0 + i]) + bias), to_f(u[t0 + i]), tab + i * 4 * NM);
+      step(softplus_fast(to_f(dl[t0 + i]) + bias), to_f(u[t0 + i]), tab + i * cplx_tab_stride<NM>());
   }
 
   float Gr[NS], Gi[NS], Anr[NS], Ani[NS], gAr[NS], gAi[NS];
@@ -424,7 +495,7 @@ __global__ void __launch_bounds__(kCplxBwdThreads, 8) cplx_bwd_kernel(const Cplx
         hs[(s * 2 * NS + j) * kCplxBwdThreads + tid] = hr[j];
         hs[(s * 2 * NS + NS + j) * kCplxBwdThreads + tid] = hi[j];
       }
-      step(softplus_fast(to_f(dl[t0 + s]) + bias), to_f(u[t0 + s]), tab + s * 4 * NM);
+      step(softplus_fast(to_f(dl[t0 + s]) + bias), to_f(u[t0 + s]), tab + s * cplx_tab_stride<NM>());
     }
     // reverse sweep over the block
     for (int s = steps - 1; s >= 0; --s) {
@@ -440,7 +511,7 @@ __global__ void __launch_bounds__(kCplxBwdThreads, 8) cplx_bwd_kernel(const Cplx
         sz = rcpf(1.f + ex2f(-zt * kLog2e));
         dy0 = dyt * zt * sz;
       }
-      const float *trow = tab + s * 4 * NM + part * NS;
+      const float *trow = tab + s * cplx_tab_stride<NM>() + part * NS;
       float y0 = 0.f, du = 0.f, dDelta = 0.f;
       float vals[NV];  // per state j: Re dB, Im dB, Re dC, Im dC at j, NS + j, 2 NS + j, 3 NS + j
 #pragma unroll

@@ -107,15 +107,20 @@ def test_cplx_mixed_structure_and_large_angles():
     rest the shared half-angle recurrence), spacings s up to 8 so that one
     step turns a state by up to some twenty full circles, a real part per
     channel, and channels whose spacing is not exact in fp32 next to ones
-    whose is.  (Much larger |Delta A| leaves fp32 short of the 1e-4 bound on
+    whose is.  Channels 3 and 11 have evenly spaced A with |A| below 1/8 in
+    their first states (the structured decay without the h += M (h + B u/A)
+    update).  (Much larger |Delta A| leaves fp32 short of the 1e-4 bound on
     ddelta whichever decay runs: dA/dDelta carries the factor A.)"""
     dim, N = 96, 16
     x = make_cplx_inputs(2, dim, 150, N, torch.float32, seed=1394, with_dy=True)
     n = torch.arange(N, dtype=torch.float32)
     s = (torch.arange(dim) % 8 + 1).float()
     s[1::2] += 0.1
-    re = -torch.linspace(0.05, 3.0, dim)[:, None].expand(dim, N)
+    re = -torch.linspace(0.05, 3.0, dim)[:, None].expand(dim, N).clone()
     im = (n - 5.0)[None, :] * s[:, None]
+    for d in (3, 11):
+        re[d] = -0.06
+        im[d] = 0.01 * n
     x["A"] = torch.cat([re, im], dim=1).contiguous()
     check(x)
 
