@@ -384,8 +384,76 @@ __device__ __forceinline__ int lane_scatter_base(int lane) {
   return base;
 }
 
+// Row stride of the per-block rows of u, delta, z, dy and of du, ddelta, dz
+// staged in shared memory (one float of padding: distinct banks for the
+// channels of a warp).
+constexpr int kCplxRow = kCplxBwdTC + 1;
+
+// Shared memory of cplx_bwd_kernel: block states, B / C table, dB / dC warp
+// sums, then the staged rows (4 inputs, 3 outputs) of the CTA's channels.
+template <int NM, int TPC>
+constexpr size_t cplx_bwd_smem() {
+  return 4 * (size_t(kCplxBwdTC) * 2 * (NM / TPC) * kCplxBwdThreads +
+              size_t(kCplxBwdTC) * cplx_tab_stride<NM>() + 2 * 4 * kMaxN * kCplxBwdTC +
+              7 * size_t(kCplxBwdThreads / TPC) * kCplxRow);
+}
+
+// Steps [t0, t0 + steps) of one (batch row, channel) row of a (batch, dim, L)
+// tensor to dst[0 .. kCplxBwdTC) as fp32, zero past `steps` (and for d past
+// dim): 16-byte loads where the rows are 16-byte aligned and the block whole.
+template <typename T>
+__device__ __forceinline__ void cplx_load_block(const void *src, const CplxArgs &a, int64_t b,
+                                                int64_t d, int64_t t0, int steps, bool vec,
+                                                float *dst) {
+  float v[kCplxBwdTC];
+#pragma unroll
+  for (int i = 0; i < kCplxBwdTC; ++i) v[i] = 0.f;
+  if (d < a.dim) {
+    const T *p = static_cast<const T *>(src) + (b * a.dim + d) * a.L + t0;
+    if (vec && steps == kCplxBwdTC) {
+      constexpr int V = Vec<T>::kN;
+#pragma unroll
+      for (int k = 0; k < kCplxBwdTC / V; ++k) {
+        float o[V];
+        Vec<T>::unpack(*reinterpret_cast<const uint4 *>(p + k * V), o);
+#pragma unroll
+        for (int i = 0; i < V; ++i) v[k * V + i] = o[i];
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < kCplxBwdTC; ++i)
+        if (i < steps) v[i] = to_f(p[i]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < kCplxBwdTC; ++i) dst[i] = v[i];
+}
+
+// The inverse of cplx_load_block for an output row (nothing for d past dim).
+template <typename T>
+__device__ __forceinline__ void cplx_store_block(void *dst, const CplxArgs &a, int64_t b, int64_t d,
+                                                 int64_t t0, int steps, bool vec, const float *src) {
+  if (d >= a.dim) return;
+  T *p = static_cast<T *>(dst) + (b * a.dim + d) * a.L + t0;
+  if (vec && steps == kCplxBwdTC) {
+    constexpr int V = Vec<T>::kN;
+#pragma unroll
+    for (int k = 0; k < kCplxBwdTC / V; ++k) {
+      float o[V];
+#pragma unroll
+      for (int i = 0; i < V; ++i) o[i] = src[k * V + i];
+      *reinterpret_cast<uint4 *>(p + k * V) = Vec<T>::pack(o);
+    }
+  } else {
+    for (int i = 0; i < steps; ++i) p[i] = from_f<T>(src[i]);
+  }
+}
+
 // TPC threads share one channel, NM / TPC states each (adjacent lanes), as in
-// the forward: more threads per channel, fewer registers per thread.
+// the forward: more threads per channel, fewer registers per thread.  Per
+// block of steps the CTA stages B and C and the u, delta, z, dy rows of its
+// channels in shared memory (one 16-byte load per row where aligned), and
+// writes its du, ddelta, dz rows back from there.
 template <typename T, int NM, int TPC>
 __global__ void __launch_bounds__(kCplxBwdThreads, 8) cplx_bwd_kernel(const CplxArgs a, const CplxWork w) {
   constexpr int NS = NM / TPC;                 // states per thread
@@ -395,19 +463,27 @@ __global__ void __launch_bounds__(kCplxBwdThreads, 8) cplx_bwd_kernel(const Cplx
   float *hs = smem;                                          // [TC][2 NS][threads]
   float *tab = hs + kCplxBwdTC * 2 * NS * kCplxBwdThreads;  // [TC][stride]
   float *wsum = tab + kCplxBwdTC * cplx_tab_stride<NM>();    // [2 warps][4 kMaxN][TC]
+  constexpr int CPB = kCplxBwdThreads / TPC;                 // channels per CTA
+  float *xs = wsum + 2 * 4 * kMaxN * kCplxBwdTC;             // [u, delta, z, dy][CPB][kCplxRow]
+  float *os = xs + 4 * CPB * kCplxRow;                       // [du, ddelta, dz][CPB][kCplxRow]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int part = tid % TPC;
+  const int part = tid % TPC, lc = tid / TPC;
   const int64_t b = blockIdx.y;
-  const int64_t d_raw = int64_t(blockIdx.x) * (kCplxBwdThreads / TPC) + tid / TPC;
+  const int64_t d0 = int64_t(blockIdx.x) * CPB;
+  const int64_t d_raw = d0 + lc;
   const bool valid = d_raw < a.dim;
   const int64_t d = valid ? d_raw : a.dim - 1;
   const int64_t ch = b * a.dim + d;
-  const int64_t row = ch * a.L;
   const int N = a.N;
-  const T *u = static_cast<const T *>(a.u) + row;
-  const T *dl = static_cast<const T *>(a.delta) + row;
-  const T *z = a.z ? static_cast<const T *>(a.z) + row : nullptr;
-  const T *dy = static_cast<const T *>(a.dy) + row;
+  const bool has_z = a.z != nullptr;
+  // 16-byte rows: every row start and block start is 16-byte aligned
+  const bool vec = (a.L * int64_t(sizeof(T))) % 16 == 0 &&
+                   ((reinterpret_cast<uintptr_t>(a.u) | reinterpret_cast<uintptr_t>(a.delta) |
+                     reinterpret_cast<uintptr_t>(a.z) | reinterpret_cast<uintptr_t>(a.dy) |
+                     reinterpret_cast<uintptr_t>(a.du) | reinterpret_cast<uintptr_t>(a.ddelta) |
+                     reinterpret_cast<uintptr_t>(a.dz)) & 15) == 0;
+  const float *xu = xs + lc * kCplxRow, *xd = xs + (CPB + lc) * kCplxRow;
+  const float *xz = xs + (2 * CPB + lc) * kCplxRow, *xdy = xs + (3 * CPB + lc) * kCplxRow;
   const float bias = a.bias ? a.bias[d] : 0.f;
   const float Dd = a.D ? a.D[d] : 0.f;
   float *ckpt = w.ckpt + ch * w.n_blocks * 2 * NM;
@@ -458,17 +534,23 @@ __global__ void __launch_bounds__(kCplxBwdThreads, 8) cplx_bwd_kernel(const Cplx
   // Forward sweep: the state at the start of every block.
   for (int64_t c = 0; c < w.n_blocks; ++c) {
     const int64_t t0 = c * kCplxBwdTC;
+    // (padding channels run on zero rows and share the last channel's slots:
+    // they must not write them)
+    if (valid) {
 #pragma unroll
-    for (int j = 0; j < NS; ++j) {
-      ckpt[c * 2 * NM + part * NS + j] = hr[j];
-      ckpt[c * 2 * NM + NM + part * NS + j] = hi[j];
+      for (int j = 0; j < NS; ++j) {
+        ckpt[c * 2 * NM + part * NS + j] = hr[j];
+        ckpt[c * 2 * NM + NM + part * NS + j] = hi[j];
+      }
     }
+    const int steps = int(a.L - t0 < kCplxBwdTC ? a.L - t0 : kCplxBwdTC);
     __syncthreads();
     cplx_stage_bc<T, NM, kCplxBwdTC>(a, b, t0, tab, false, kCplxBwdThreads);
+    for (int r = tid; r < 2 * CPB; r += kCplxBwdThreads)
+      cplx_load_block<T>(r < CPB ? a.u : a.delta, a, b, d0 + r % CPB, t0, steps, vec, xs + r * kCplxRow);
     __syncthreads();
-    const int steps = int(a.L - t0 < kCplxBwdTC ? a.L - t0 : kCplxBwdTC);
     for (int i = 0; i < steps; ++i)
-      step(softplus_fast(to_f(dl[t0 + i]) + bias), to_f(u[t0 + i]), tab + i * cplx_tab_stride<NM>());
+      step(softplus_fast(xd[i] + bias), xu[i], tab + i * cplx_tab_stride<NM>());
   }
 
   float Gr[NS], Gi[NS], Anr[NS], Ani[NS], gAr[NS], gAi[NS];
@@ -482,6 +564,11 @@ __global__ void __launch_bounds__(kCplxBwdThreads, 8) cplx_bwd_kernel(const Cplx
     const int steps = int(a.L - t0 < kCplxBwdTC ? a.L - t0 : kCplxBwdTC);
     __syncthreads();
     cplx_stage_bc<T, NM, kCplxBwdTC>(a, b, t0, tab, true, kCplxBwdThreads);
+    for (int r = tid; r < 4 * CPB; r += kCplxBwdThreads) {
+      const int k = r / CPB;  // u, delta, z, dy
+      const void *src = k == 0 ? a.u : k == 1 ? a.delta : k == 2 ? a.z : a.dy;
+      if (src) cplx_load_block<T>(src, a, b, d0 + r % CPB, t0, steps, vec, xs + r * kCplxRow);
+    }
     __syncthreads();
     // recompute the block; hs[s] holds the state before step t0 + s
 #pragma unroll
@@ -495,19 +582,18 @@ __global__ void __launch_bounds__(kCplxBwdThreads, 8) cplx_bwd_kernel(const Cplx
         hs[(s * 2 * NS + j) * kCplxBwdThreads + tid] = hr[j];
         hs[(s * 2 * NS + NS + j) * kCplxBwdThreads + tid] = hi[j];
       }
-      step(softplus_fast(to_f(dl[t0 + s]) + bias), to_f(u[t0 + s]), tab + s * cplx_tab_stride<NM>());
+      step(softplus_fast(xd[s] + bias), xu[s], tab + s * cplx_tab_stride<NM>());
     }
     // reverse sweep over the block
     for (int s = steps - 1; s >= 0; --s) {
-      const int64_t t = t0 + s;
-      const float v = to_f(dl[t]) + bias;
+      const float v = xd[s] + bias;
       const float Delta = softplus_fast(v);
       const float sv = rcpf(1.f + ex2f(-v * kLog2e));
-      const float ut = to_f(u[t]);
-      const float dyt = to_f(dy[t]);
+      const float ut = xu[s];
+      const float dyt = xdy[s];
       float dy0 = dyt, zt = 0.f, sz = 0.f;
-      if (z) {
-        zt = to_f(z[t]);
+      if (has_z) {
+        zt = xz[s];
         sz = rcpf(1.f + ex2f(-zt * kLog2e));
         dy0 = dyt * zt * sz;
       }
@@ -577,10 +663,10 @@ __global__ void __launch_bounds__(kCplxBwdThreads, 8) cplx_bwd_kernel(const Cplx
       y0 = fmaf(Dd, ut, y0);
       du = fmaf(Dd, dy0, du);
       const float ddl = dDelta * sv;
+      // du, ddelta, dz to the staged output rows, one per thread of the channel
+      const float dzv = dyt * y0 * sz * (1.f + zt * (1.f - sz));
+      for (int k = part; k < 3; k += TPC) os[(k * CPB + lc) * kCplxRow + s] = k == 0 ? du : k == 1 ? ddl : dzv;
       if (valid && part == 0) {
-        static_cast<T *>(a.du)[row + t] = from_f<T>(du);
-        static_cast<T *>(a.ddelta)[row + t] = from_f<T>(ddl);
-        if (z) static_cast<T *>(a.dz)[row + t] = from_f<T>(dyt * y0 * sz * (1.f + zt * (1.f - sz)));
         dDacc = fmaf(dy0, ut, dDacc);
         dbacc += ddl;
       }
@@ -602,6 +688,11 @@ __global__ void __launch_bounds__(kCplxBwdThreads, 8) cplx_bwd_kernel(const Cplx
                           wsum[(1 * 4 * kMaxN + slot) * kCplxBwdTC + s];
         w.part_bc[((int64_t(blockIdx.x) * a.batch + b) * 4 * kMaxN + slot) * a.L + t0 + s] = sum;
       }
+    }
+    for (int r = tid; r < 3 * CPB; r += kCplxBwdThreads) {
+      const int k = r / CPB;  // du, ddelta, dz
+      void *dst = k == 0 ? a.du : k == 1 ? a.ddelta : a.dz;
+      if (dst) cplx_store_block<T>(dst, a, b, d0 + r % CPB, t0, steps, vec, os + r * kCplxRow);
     }
   }
   if (ident) {  // conj(1/A) times the sums of conj(k A) G

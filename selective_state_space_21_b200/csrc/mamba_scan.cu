@@ -258,8 +258,7 @@ struct CplxBwdLauncher {
     w.part_A = w.part_bc + n_bc;
     w.part_D = w.part_A + n_A;
     w.part_bias = w.part_D + bd;
-    const size_t smem = 4 * (size_t(kCplxBwdTC) * 2 * (NM / TPC) * kCplxBwdThreads +
-                             size_t(kCplxBwdTC) * cplx_tab_stride<NM>() + 2 * 4 * kMaxN * kCplxBwdTC);
+    const size_t smem = cplx_bwd_smem<NM, TPC>();
     mamba_status_t st = MAMBA_OK;
     if (cudaFuncSetAttribute(cplx_bwd_kernel<T, NM, TPC>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
