@@ -29,7 +29,8 @@
 // adjoint (the gradient g = dl/d re + i dl/d im of a complex quantity passes a
 // product by the conjugate of the other factor):
 //     G_t = conj(C_t) dy0_t + conj(Abar_{t+1}) G_{t+1},
-//     du += Re(conj(G) Bbar),  dDelta += Re(conj(G) Abar (A h_{t-1} + B u)),
+//     du += Re(conj(G) Bbar),  dDelta += Re(conj(G) (A h_t + B u))
+//        (A h_t + B u = Abar (A h_{t-1} + B u)),
 //     gA += conj(Delta Abar h_{t-1} + Delta^2 phi(Delta A) B u) G
 //        (= conj(1/A) conj(Delta dh/dDelta - Bbar u) G, used where |A| >= 1/8),
 //     gB += conj(Delta psi(Delta A)) u G,  gC += conj(h_t) dy0,
@@ -625,11 +626,11 @@ __global__ void __launch_bounds__(kCplxBwdThreads, 8) cplx_bwd_kernel(const Cplx
         Gi[j] = gi;
         Anr[j] = abr;
         Ani[j] = abi;
-        // du += Re(conj(G) E B); dDelta += Re(conj(G) Abar (A h + B u))
+        // du += Re(conj(G) E B); dDelta += Re(conj(G) p) with
+        // p = dh_t/dDelta = Abar (A h_{t-1} + B u) = A h_t + B u
         du = fmaf(gr, ebr, fmaf(gi, ebi, du));
-        const float qr = fmaf(ar[j], hpr, fmaf(-ai[j], hpi, bur));
-        const float qi = fmaf(ar[j], hpi, fmaf(ai[j], hpr, bui));
-        const float pr_ = fmaf(abr, qr, -abi * qi), pi_ = fmaf(abr, qi, abi * qr);
+        const float pr_ = fmaf(ar[j], hcr, fmaf(-ai[j], hci, bur));
+        const float pi_ = fmaf(ar[j], hci, fmaf(ai[j], hcr, bui));
         dDelta = fmaf(gr, pr_, fmaf(gi, pi_, dDelta));
         // gA += conj(k) G with k = dh_t/dA = Delta Abar h_{t-1} + Delta^2 phi(x) B u;
         // with `ident` the sum runs over k A = Delta p - E B u and is divided
