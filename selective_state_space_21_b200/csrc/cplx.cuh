@@ -228,9 +228,10 @@ __device__ __forceinline__ void cplx_phi(float xr, float xi, float er, float ei,
   pi = small ? ai : fmaf(ni, x2r, -nr * x2i) * den;
 }
 
-// Row stride of the staged tables: one float of padding, so that the staging
-// writes (consecutive threads, consecutive steps) fall in distinct banks.
-template <int NM> constexpr int cplx_tab_stride() { return 4 * NM + 1; }
+// Row stride of the staged tables, padded so that the staging writes fall in
+// distinct banks: a warp writes 32 / TT slots of TT consecutive steps, which
+// wants a stride of 1 modulo 32 for TT = 32 and of 4 modulo 32 for TT = 8.
+template <int NM, int TT> constexpr int cplx_tab_stride() { return 4 * NM + (TT >= 32 ? 1 : 4); }
 
 // Stages the B and C columns of steps [t0, t0 + TT) of batch row b into
 // tab[t][4 NM] = (Re B, Im B, Re C, Im C) as fp32 (rows cplx_tab_stride apart),
@@ -250,7 +251,7 @@ __device__ __forceinline__ void cplx_stage_bc(const CplxArgs &a, int64_t b, int6
       const T *src = part < 2 ? Bp : Cp;
       v = to_f(src[(int64_t(part & 1) * N + n) * a.L + tt]);
     }
-    tab[t * cplx_tab_stride<NM>() + slot] = v;
+    tab[t * cplx_tab_stride<NM, TT>() + slot] = v;
   }
 }
 
@@ -260,7 +261,7 @@ __device__ __forceinline__ void cplx_stage_bc(const CplxArgs &a, int64_t b, int6
 template <typename T, int NM, int TPC>
 __global__ void __launch_bounds__(kCplxThreads) cplx_fwd_kernel(const CplxArgs a) {
   constexpr int NS = NM / TPC;  // states per thread
-  __shared__ __align__(16) float tab[kCplxTT * cplx_tab_stride<NM>()];
+  __shared__ __align__(16) float tab[kCplxTT * cplx_tab_stride<NM, kCplxTT>()];
   const int tid = threadIdx.x;
   const int part = tid % TPC;
   const int64_t b = blockIdx.y;
@@ -298,7 +299,7 @@ __global__ void __launch_bounds__(kCplxThreads) cplx_fwd_kernel(const CplxArgs a
       const int64_t t = t0 + i;
       const float Delta = softplus_fast(to_f(dl[t]) + bias);
       const float ut = to_f(u[t]);
-      const float *tr = tab + i * cplx_tab_stride<NM>() + part * NS;
+      const float *tr = tab + i * cplx_tab_stride<NM, kCplxTT>() + part * NS;
       float y0 = Dd * ut;
       if (mform) {
         float Mr[NS], Mi[NS];
@@ -395,7 +396,7 @@ constexpr int kCplxRow = kCplxBwdTC + 1;
 template <int NM, int TPC>
 constexpr size_t cplx_bwd_smem() {
   return 4 * (size_t(kCplxBwdTC) * 2 * (NM / TPC) * kCplxBwdThreads +
-              size_t(kCplxBwdTC) * cplx_tab_stride<NM>() + 2 * 4 * kMaxN * kCplxBwdTC +
+              size_t(kCplxBwdTC) * cplx_tab_stride<NM, kCplxBwdTC>() + 2 * 4 * kMaxN * kCplxRow +
               7 * size_t(kCplxBwdThreads / TPC) * kCplxRow);
 }
 
@@ -463,9 +464,9 @@ __global__ void __launch_bounds__(kCplxBwdThreads, 8) cplx_bwd_kernel(const Cplx
   extern __shared__ __align__(16) float smem[];
   float *hs = smem;                                          // [TC][2 NS][threads]
   float *tab = hs + kCplxBwdTC * 2 * NS * kCplxBwdThreads;  // [TC][stride]
-  float *wsum = tab + kCplxBwdTC * cplx_tab_stride<NM>();    // [2 warps][4 kMaxN][TC]
+  float *wsum = tab + kCplxBwdTC * cplx_tab_stride<NM, kCplxBwdTC>();  // [2 warps][4 kMaxN][kCplxRow]
   constexpr int CPB = kCplxBwdThreads / TPC;                 // channels per CTA
-  float *xs = wsum + 2 * 4 * kMaxN * kCplxBwdTC;             // [u, delta, z, dy][CPB][kCplxRow]
+  float *xs = wsum + 2 * 4 * kMaxN * kCplxRow;               // [u, delta, z, dy][CPB][kCplxRow]
   float *os = xs + 4 * CPB * kCplxRow;                       // [du, ddelta, dz][CPB][kCplxRow]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int part = tid % TPC, lc = tid / TPC;
@@ -488,7 +489,7 @@ __global__ void __launch_bounds__(kCplxBwdThreads, 8) cplx_bwd_kernel(const Cplx
   const float bias = a.bias ? a.bias[d] : 0.f;
   const float Dd = a.D ? a.D[d] : 0.f;
   float *ckpt = w.ckpt + ch * w.n_blocks * 2 * NM;
-  for (int i = tid; i < 2 * 4 * kMaxN * kCplxBwdTC; i += kCplxBwdThreads) wsum[i] = 0.f;
+  for (int i = tid; i < 2 * 4 * kMaxN * kCplxRow; i += kCplxBwdThreads) wsum[i] = 0.f;
 
   float ar[NS], ai[NS], ira[NS], iai[NS], hr[NS], hi[NS];
 #pragma unroll
@@ -551,7 +552,7 @@ __global__ void __launch_bounds__(kCplxBwdThreads, 8) cplx_bwd_kernel(const Cplx
       cplx_load_block<T>(r < CPB ? a.u : a.delta, a, b, d0 + r % CPB, t0, steps, vec, xs + r * kCplxRow);
     __syncthreads();
     for (int i = 0; i < steps; ++i)
-      step(softplus_fast(xd[i] + bias), xu[i], tab + i * cplx_tab_stride<NM>());
+      step(softplus_fast(xd[i] + bias), xu[i], tab + i * cplx_tab_stride<NM, kCplxBwdTC>());
   }
 
   float Gr[NS], Gi[NS], Anr[NS], Ani[NS], gAr[NS], gAi[NS];
@@ -583,7 +584,7 @@ __global__ void __launch_bounds__(kCplxBwdThreads, 8) cplx_bwd_kernel(const Cplx
         hs[(s * 2 * NS + j) * kCplxBwdThreads + tid] = hr[j];
         hs[(s * 2 * NS + NS + j) * kCplxBwdThreads + tid] = hi[j];
       }
-      step(softplus_fast(xd[s] + bias), xu[s], tab + s * cplx_tab_stride<NM>());
+      step(softplus_fast(xd[s] + bias), xu[s], tab + s * cplx_tab_stride<NM, kCplxBwdTC>());
     }
     // reverse sweep over the block
     for (int s = steps - 1; s >= 0; --s) {
@@ -598,7 +599,7 @@ __global__ void __launch_bounds__(kCplxBwdThreads, 8) cplx_bwd_kernel(const Cplx
         sz = rcpf(1.f + ex2f(-zt * kLog2e));
         dy0 = dyt * zt * sz;
       }
-      const float *trow = tab + s * cplx_tab_stride<NM>() + part * NS;
+      const float *trow = tab + s * cplx_tab_stride<NM, kCplxBwdTC>() + part * NS;
       float y0 = 0.f, du = 0.f, dDelta = 0.f;
       float vals[NV];  // per state j: Re dB, Im dB, Re dC, Im dC at j, NS + j, 2 NS + j, 3 NS + j
 #pragma unroll
@@ -677,7 +678,7 @@ __global__ void __launch_bounds__(kCplxBwdThreads, 8) cplx_bwd_kernel(const Cplx
         const int idx = kbase + r;  // value index of this lane's sum
         if (idx < 4 * NS) {
           const int q = idx / NS, n = part * NS + idx % NS;
-          wsum[(warp * 4 * kMaxN + q * kMaxN + n) * kCplxBwdTC + s] = vals[r];
+          wsum[(warp * 4 * kMaxN + q * kMaxN + n) * kCplxRow + s] = vals[r];
         }
       }
     }
@@ -685,8 +686,8 @@ __global__ void __launch_bounds__(kCplxBwdThreads, 8) cplx_bwd_kernel(const Cplx
     for (int idx = tid; idx < 4 * kMaxN * kCplxBwdTC; idx += kCplxBwdThreads) {
       const int slot = idx / kCplxBwdTC, s = idx % kCplxBwdTC;
       if (s < steps) {
-        const float sum = wsum[(0 * 4 * kMaxN + slot) * kCplxBwdTC + s] +
-                          wsum[(1 * 4 * kMaxN + slot) * kCplxBwdTC + s];
+        const float sum = wsum[(0 * 4 * kMaxN + slot) * kCplxRow + s] +
+                          wsum[(1 * 4 * kMaxN + slot) * kCplxRow + s];
         w.part_bc[((int64_t(blockIdx.x) * a.batch + b) * 4 * kMaxN + slot) * a.L + t0 + s] = sum;
       }
     }
