@@ -20,6 +20,7 @@ on the host cores instead (bounded channel samples of the same workload).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -270,6 +271,11 @@ def run_ours(args, world, rank, device):
     from selective_state_space_21_b200 import scan
 
     w = WORKLOADS[args.workload]
+    if args.only == "cplx":  # the complex-A calls alone, for profiling
+        if args.cplx_batch:
+            w = dataclasses.replace(w, batch=args.cplx_batch)
+        res = run_cplx(w, device, measured_peaks(), steps=args.steps)
+        return {"note": "--only cplx: a profiling run, not a benchmark result", "complex_A": res}
     x = make_inputs(w.batch, w.dim, w.L, w.N, w.dtype, device=device,
                     seed=shard_seed(1234 + args.workload, rank), has_z=w.has_z,
                     has_D=w.has_D, with_dy=True)
@@ -789,8 +795,11 @@ def main(argv=None):
     ap.add_argument("--no-dtproj", action="store_true",
                     help="skip the Delta-projection timing")
     ap.add_argument("--no-cplx", action="store_true", help="skip the complex-A timing")
-    ap.add_argument("--only", choices=["fwd", "bwd"], default=None,
-                    help="time one pass only (for profiling; not a benchmark result)")
+    ap.add_argument("--only", choices=["fwd", "bwd", "cplx"], default=None,
+                    help="time one pass, or the complex-A calls, only (for profiling; "
+                         "not a benchmark result)")
+    ap.add_argument("--cplx-batch", type=int, default=0,
+                    help="batch of the complex-A calls with --only cplx (0: the workload's)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
