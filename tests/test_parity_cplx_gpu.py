@@ -151,11 +151,14 @@ def test_cplx_bwd_deterministic():
         assert torch.equal(g1[k], g2[k]), k
 
 
-def test_cplx_full_size_sampled():
-    """The bf16 4 x 2048 x 4096 workload shape with 16 complex states: y and
-    du, ddelta on sampled channels against the oracle."""
-    w = WORKLOADS[4]
-    xh = make_cplx_inputs(w.batch, w.dim, w.L, w.N, w.dtype, seed=1394, with_dy=True)
+@pytest.mark.parametrize("wl", [2, 4], ids=["b8_d5120_L2048", "b4_d2048_L4096"])
+def test_cplx_full_size_sampled(wl):
+    """Workload shapes with 16 complex states (bf16 8 x 5120 x 2048, the one
+    the bench times, and 4 x 2048 x 4096): y, du, ddelta and dz on sampled
+    channels against the oracle, and dA, dD, dbias (sums over the batch) on
+    three channels."""
+    w = WORKLOADS[wl]
+    xh = make_cplx_inputs(w.batch, w.dim, w.L, w.N, w.dtype, seed=1394 + wl, with_dy=True)
     x = gc.to_device(xh)
     y, _ = gpu_fwd(x)
     g = gpu_bwd(x)
@@ -178,3 +181,11 @@ def test_cplx_full_size_sampled():
         for k in ("du", "ddelta", "dz"):
             e = gc.normwise(gh[k][b].index_select(0, idx).double().numpy(), ref[k][0])
             assert e <= tol, f"{k} (batch {b}): {e:.2e}"
+    idx = torch.tensor([0, w.dim // 2 + 1, w.dim - 1])
+    sub = {k: xh[k].index_select(1, idx).contiguous() for k in ("u", "delta", "z", "dy")}
+    sub.update(A=per_d(xh["A"], idx), D=per_d(xh["D"], idx), delta_bias=per_d(xh["delta_bias"], idx))
+    ref = oracle.s6_cplx_backward(sub["u"], sub["delta"], sub["A"], xh["B"], xh["C"], sub["dy"],
+                                  delta_bias=sub["delta_bias"], D=sub["D"], z=sub["z"])
+    for k in ("dA", "dD", "ddelta_bias"):
+        e = gc.normwise(gh[k].index_select(0, idx).double().numpy(), ref[k])
+        assert e <= tol, f"{k}: {e:.2e}"
