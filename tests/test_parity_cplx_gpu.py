@@ -189,3 +189,40 @@ def test_cplx_full_size_sampled(wl):
     for k in ("dA", "dD", "ddelta_bias"):
         e = gc.normwise(gh[k].index_select(0, idx).double().numpy(), ref[k])
         assert e <= tol, f"{k}: {e:.2e}"
+
+
+def test_cplx_rejects_bad_arguments():
+    """More than 16 complex states is unsupported, and an output over an input
+    is an invalid argument.  Nothing is launched for them."""
+    x = gc.to_device(make_cplx_inputs(1, 8, 32, 4, torch.float32, seed=1395, with_dy=True))
+    y = torch.empty_like(x["u"])
+    last = torch.empty(1, 8, 8, device="cuda")
+    base = (x["u"], x["delta"], x["delta_bias"], x["A"], x["B"], x["C"], x["D"], x["z"])
+    with pytest.raises(scan.MambaScanError) as e:  # y over u
+        scan.mamba_cplx_scan_fwd(*base, x["u"], last)
+    assert e.value.status == 1  # MAMBA_ERR_INVALID_ARG
+    A17 = torch.cat([torch.full((8, 17), -0.5), torch.zeros(8, 17)], dim=1).cuda()
+    B17 = torch.zeros(1, 34, 32, device="cuda")
+    with pytest.raises(scan.MambaScanError) as e:
+        scan.mamba_cplx_scan_fwd(x["u"], x["delta"], x["delta_bias"], A17, B17, B17, x["D"],
+                                 x["z"], y, None)
+    assert e.value.status == 2  # MAMBA_ERR_UNSUPPORTED
+    assert scan.mamba_scan_stream_status() == 0
+
+
+def test_cplx_bwd_rows_not_16_byte_aligned():
+    """Element-aligned tensors that are not 16-byte aligned take the backward's
+    per-element block loads and stores instead of the 16-byte ones: the
+    gradients are bitwise those of the aligned call."""
+    x = gc.to_device(make_cplx_inputs(2, 24, 64, 16, torch.float32, seed=1396, with_dy=True))
+    g = gpu_bwd(x)
+
+    def offset(t):  # same values, 4 bytes past a 16-byte boundary
+        o = torch.empty(t.numel() + 1, device="cuda", dtype=t.dtype)[1:].view(t.shape)
+        o.copy_(t)
+        return o
+
+    x2 = dict(x, u=offset(x["u"]), dy=offset(x["dy"]))
+    g2 = gpu_bwd(x2)
+    for k in g:
+        assert torch.equal(g[k], g2[k]), k
