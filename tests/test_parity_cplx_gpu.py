@@ -1,6 +1,7 @@
 """GPU parity of the complex-A scan (mamba_cplx_scan_fwd / _bwd, S4D-Lin
 A_n = -1/2 + n i, complex B and C) against the fp64 oracle on the same seeded
 inputs.  Normwise max error <= 1e-4 for fp32 I/O and <= 2e-2 for bf16 I/O."""
+import numpy as np
 import pytest
 import torch
 
@@ -226,3 +227,23 @@ def test_cplx_bwd_rows_not_16_byte_aligned():
     g2 = gpu_bwd(x2)
     for k in g:
         assert torch.equal(g[k], g2[k]), k
+
+
+def _random_cases(count, seed):
+    """Seeded shapes: batch 1-3, dim 1-120, L 1-300 (a multiple of 8 one time
+    in two, so that the backward's 16-byte block loads take part), N 1-16."""
+    g = np.random.default_rng(seed)
+    cases = []
+    for i in range(count):
+        L = int(g.integers(1, 301))
+        if i % 2 == 0:
+            L = max(8, L - L % 8)
+        cases.append((int(g.integers(1, 4)), int(g.integers(1, 121)), L, int(g.integers(1, 17))))
+    return cases
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("shape", _random_cases(8, 2027), ids=lambda s: "x".join(map(str, s)))
+def test_cplx_random_shapes(shape, dtype):
+    b, d, L, N = shape
+    check(make_cplx_inputs(b, d, L, N, dtype, seed=1400 + b * 131 + d + L, with_dy=True))

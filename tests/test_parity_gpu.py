@@ -414,3 +414,34 @@ def test_bwd_three_phase_generic_and_mixed_A(dtype):
     for k in GRAD_KEYS:
         e = gc.normwise(gg[k].cpu().double().numpy(), ref[k])
         assert e <= tol, f"{k}: {e:.2e}"
+
+
+# --------------------------------------------------- seeded random shapes
+
+def _random_cases(count, seed):
+    """Shapes and options drawn from a seeded generator: batch 1-3, dim 1-300,
+    L 1-700 (a multiple of 8 one time in three, so that the staged kernels
+    take part), N 1-16, with or without z, D and the bias."""
+    g = np.random.default_rng(seed)
+    cases = []
+    for i in range(count):
+        L = int(g.integers(1, 701))
+        if i % 3 == 0:
+            L = max(8, L - L % 8)
+        cases.append((int(g.integers(1, 4)), int(g.integers(1, 301)), L, int(g.integers(1, 17)),
+                      bool(g.integers(0, 2)), bool(g.integers(0, 2)), bool(g.integers(0, 2))))
+    return cases
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("case", _random_cases(12, 2026), ids=lambda c: "x".join(map(str, c[:4])))
+def test_fwd_bwd_random_shapes(case, dtype):
+    """Forward and backward through the auto path on seeded random shapes
+    against the oracle."""
+    b, d, L, N, has_z, has_D, has_bias = case
+    x = make_inputs(b, d, L, N, dtype, seed=b * 7919 + d * 31 + L, has_z=has_z, has_D=has_D,
+                    with_dy=True)
+    if not has_bias:
+        x["delta_bias"] = None
+    _fwd_case(x)
+    _bwd_case(x)
