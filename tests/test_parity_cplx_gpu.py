@@ -247,3 +247,14 @@ def _random_cases(count, seed):
 def test_cplx_random_shapes(shape, dtype):
     b, d, L, N = shape
     check(make_cplx_inputs(b, d, L, N, dtype, seed=1400 + b * 131 + d + L, with_dy=True))
+
+
+@pytest.mark.parametrize("shape", [(1, 19040, 40, 16), (2, 9600, 32, 16), (1, 36000, 24, 16),
+                                   (1, 38000, 17, 8)], ids=lambda s: "x".join(map(str, s)))
+def test_cplx_bwd_many_channels(shape):
+    """Channel counts that fill more than half a round of the backward's CTA
+    slots, so that it runs four (N = 16) or two (N = 8) threads per channel;
+    the smaller shapes above run one state per thread.  Every gradient, dB and
+    dC included, against the oracle."""
+    b, d, L, N = shape
+    check(make_cplx_inputs(b, d, L, N, torch.float32, seed=1500 + d + L, with_dy=True))
