@@ -740,7 +740,7 @@ def run_reference(args, world, rank):
     w = WORKLOADS[args.workload]
     x = make_inputs(w.batch, w.dim, w.L, w.N, w.dtype, device="cpu",
                     seed=1234 + args.workload, has_z=w.has_z, has_D=w.has_D, with_dy=True)
-    threads = oracle.default_threads()
+    threads = args.cpu_threads or oracle.default_threads()
     k = max(8, 2 * threads)
 
     def step(d0):
@@ -769,7 +769,8 @@ def run_reference(args, world, rank):
         "ms_per_step": round(per * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": f"{w.name} (forward + recompute backward per step)",
-                   "batch": w.batch, "dim": w.dim, "L": w.L, "N": w.N, "io_dtype": "bf16"},
+                   "batch": w.batch, "dim": w.dim, "L": w.L, "N": w.N,
+                   "io_dtype": "bf16" if w.dtype == torch.bfloat16 else "fp32"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -787,6 +788,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--cpu-threads", type=int, default=0,
+                    help="threads of the oracle in the reference arm (0: all host cores)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-conv", action="store_true",
                     help="skip the convolution-prologue timing")
