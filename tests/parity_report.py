@@ -1,6 +1,7 @@
 """Parity report: the measured error of the CUDA path against the fp64 oracle
 on every workload, per output tensor, at full size in the launch
-configuration the benchmark times (auto path).
+configuration the benchmark times (auto path), and of the convolution
+prologue, the Delta projection and complex A on the bf16 2K workload.
 
     python tests/parity_report.py            # needs a B200; prints a markdown table
 
@@ -77,6 +78,78 @@ def report(index: int, k: int, backward: bool):
     return w, acc
 
 
+def report_variant(kind: str, k: int = 16):
+    """The rows beyond the plain scan on the bf16 8 x 5120 x 2048 workload:
+    the convolution prologue (width 4), the rank-160 Delta projection and
+    complex A with 16 complex states.  y and the per-channel gradients on
+    sampled channels; the per-channel parameters' gradients (summed over the
+    batch) on three channels."""
+    import test_parity_conv_gpu as tc
+    import test_parity_cplx_gpu as tx
+    import test_parity_dtproj_gpu as td
+    from selective_state_space_21_b200.inputs import make_cplx_inputs
+
+    w = WORKLOADS[2]
+    if kind == "conv":
+        xh = tc.conv_case(w.batch, w.dim, w.L, w.N, w.dtype, seed=1236)
+        fwd, bwd, ofwd, obwd = tc.gpu_fwd, tc.gpu_bwd, tc.oracle_fwd, tc.oracle_bwd
+        rows, per_d, grads, params = ("u", "delta", "z", "dy"), ("A", "D", "delta_bias", "conv_w",
+                                      "conv_b"), ("dx", "ddelta", "dz"), ("dconv_w", "dconv_b", "dA")
+    elif kind == "dtproj":
+        xh = td.case(w.batch, w.dim, w.L, w.N, (w.dim // 2 + 15) // 16, w.dtype, seed=1194)
+        fwd, bwd, ofwd, obwd = td.gpu_fwd, td.gpu_bwd, td.oracle_fwd, td.oracle_bwd
+        rows, per_d, grads, params = ("u", "z", "dy"), ("A", "D", "delta_bias", "W_dt"), \
+            ("du", "dz"), ("dW_dt", "dA")
+    else:
+        xh = make_cplx_inputs(w.batch, w.dim, w.L, w.N, w.dtype, seed=1396, with_dy=True)
+        fwd, bwd = tx.gpu_fwd, tx.gpu_bwd
+        ofwd = lambda x: tx.oracle.s6_cplx_forward(x["u"], x["delta"], x["A"], x["B"], x["C"],
+                                                   delta_bias=x["delta_bias"], D=x["D"], z=x["z"])
+        obwd = lambda x: tx.oracle.s6_cplx_backward(x["u"], x["delta"], x["A"], x["B"], x["C"],
+                                                    x["dy"], delta_bias=x["delta_bias"], D=x["D"],
+                                                    z=x["z"])
+        rows, per_d, grads, params = ("u", "delta", "z", "dy"), ("A", "D", "delta_bias"), \
+            ("du", "ddelta", "dz"), ("dA", "dD", "ddelta_bias")
+    x = gc.to_device(xh)
+    y = fwd(x)[0].cpu()
+    g = {key: v.cpu() for key, v in bwd(x).items() if v is not None}
+    acc: dict = {}
+
+    def add(name, got, ref):
+        e = errors(got, ref)
+        a = acc.setdefault(name, [0.0, 0.0])
+        a[0], a[1] = max(a[0], e[0]), max(a[1], e[1])
+
+    def shared(b):  # tensors shared by the channels of batch row b
+        out = {"B": xh["B"][b:b + 1].contiguous(), "C": xh["C"][b:b + 1].contiguous()}
+        if "dt_low" in xh:
+            out["dt_low"] = xh["dt_low"][b:b + 1].contiguous()
+        return out
+
+    for b, ds in gc.sample_channels(w.batch, w.dim, k, seed=5).items():
+        idx = torch.tensor(ds)
+        sub = {n: xh[n][b:b + 1].index_select(1, idx).contiguous() for n in rows}
+        sub.update({n: xh[n].index_select(0, idx).contiguous() for n in per_d})
+        sub.update(shared(b))
+        if "delta" not in sub:
+            sub["delta"] = None
+        y_ref = ofwd(sub)[0]
+        add("y", y[b].index_select(0, idx).double().numpy(), y_ref[0])
+        ref = obwd(sub)
+        for key in grads:
+            add(key, g[key][b].index_select(0, idx).double().numpy(), ref[key][0])
+    idx = torch.tensor([0, w.dim // 2 + 1, w.dim - 1])
+    sub = {n: xh[n].index_select(1, idx).contiguous() for n in rows}
+    sub.update({n: xh[n].index_select(0, idx).contiguous() for n in per_d})
+    sub.update(B=xh["B"], C=xh["C"])
+    if "dt_low" in xh:
+        sub["dt_low"] = xh["dt_low"]
+    ref = obwd(sub)
+    for key in params:
+        add(key, g[key].index_select(0, idx).double().numpy(), ref[key])
+    return acc
+
+
 def main():
     build.build()
     scan.load_library()
@@ -88,6 +161,12 @@ def main():
         bar = gc.TOL[w.dtype]
         for name, (e, p) in acc.items():
             print(f"| {w.name} | {name} | {e:.2e} | {p:.2e} | {bar:g} |", flush=True)
+    names = {"conv": "convolution prologue (width 4)", "dtproj": "Δ projection (R = 160)",
+             "cplx": "complex A (16 complex states)"}
+    for kind in ("conv", "dtproj", "cplx"):
+        for name, (e, p) in report_variant(kind).items():
+            print(f"| {WORKLOADS[2].name}, {names[kind]} | {name} | {e:.2e} | {p:.2e} | 0.02 |",
+                  flush=True)
     return 0
 
 
