@@ -332,6 +332,64 @@ MAMBA_SCAN_API mamba_status_t mamba_conv_scan_step(float *state, float *conv_sta
                                                    mamba_stream_t stream);
 
 /*
+ * Decoding plans: mamba_scan_step / mamba_conv_scan_step with the argument
+ * checks done once.  A decoding loop usually steps the same buffers token
+ * after token (the state, this token's input slots, y); the plan records
+ * them, checks every pointer (device memory of the current device, aligned,
+ * no output overlapping an input) and picks the kernel, and each run is then
+ * a single kernel launch.  conv_width = 0 plans mamba_scan_step (x is u, and
+ * conv_state, conv_w, conv_b must be NULL); 1..4 plans mamba_conv_scan_step.
+ * All other arguments as there.  The plan holds only host memory and the
+ * pointers given: the caller keeps the buffers alive and unmoved while it
+ * runs the plan, and writes each token's values into them between runs (on
+ * the run's stream, or ordered with it).  A run on another device than the
+ * creating call's returns MAMBA_ERR_INVALID_ARG; runs of one plan on streams
+ * that overlap race on the state.  Destroying NULL does nothing.
+ */
+typedef struct mamba_step_plan_st *mamba_step_plan_t;
+
+MAMBA_SCAN_API mamba_status_t mamba_scan_step_plan_create(
+    mamba_step_plan_t *plan, float *state, float *conv_state, const void *x, const float *conv_w,
+    const float *conv_b, int64_t conv_width, const void *delta, const float *delta_bias,
+    const float *A, const void *B, const void *C, const float *D, const void *z, void *y,
+    int64_t batch, int64_t dim, int64_t N, mamba_dtype_t dtype);
+
+/* Enqueues one decoding token of `plan` on `stream` (one kernel launch). */
+MAMBA_SCAN_API mamba_status_t mamba_scan_step_plan_run(mamba_step_plan_t plan,
+                                                       mamba_stream_t stream);
+
+MAMBA_SCAN_API void mamba_scan_step_plan_destroy(mamba_step_plan_t plan);
+
+/*
+ * The workspace pool of the current device.  The library takes its temporary
+ * device memory from a pool of its own per device (see the conventions
+ * above), which keeps up to a reserve -- 4 GiB unless set here -- mapped
+ * between calls so that repeated calls do not map and unmap it.  That memory
+ * is not visible to other allocators in the process (torch's caching
+ * allocator, for one):
+ *  - mamba_scan_pool_set_reserve(bytes): the pool keeps at most `bytes`
+ *    reserved at each synchronization from now on (0: it gives all unused
+ *    memory back every time, at the cost of re-mapping it per call).
+ *  - mamba_scan_pool_trim(keep_bytes): gives unused memory back now, down to
+ *    `keep_bytes`; memory of calls still running on a stream is released by a
+ *    later trim, after that work completes.
+ *  - mamba_scan_pool_reserved(&bytes): the memory the pool holds now.
+ * Each returns MAMBA_ERR_CUDA if a CUDA call fails.
+ */
+MAMBA_SCAN_API mamba_status_t mamba_scan_pool_set_reserve(uint64_t bytes);
+MAMBA_SCAN_API mamba_status_t mamba_scan_pool_trim(uint64_t keep_bytes);
+MAMBA_SCAN_API mamba_status_t mamba_scan_pool_reserved(uint64_t *bytes);
+
+/*
+ * Test hook (not for production use): after `after` more successful
+ * workspace allocations by the calling thread, the next one fails as if the
+ * device were out of memory, so that tests can check that every call then
+ * returns MAMBA_ERR_OUT_OF_MEMORY without launching a kernel or writing an
+ * output.  A negative value disarms the hook.
+ */
+MAMBA_SCAN_API void mamba_scan_test_fail_alloc(int32_t after);
+
+/*
  * Forward that allocates nothing.  (An addition of this library for callers
  * that cannot allocate; the paper has no counterpart.)
  *

@@ -15,6 +15,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIBDIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIBDIR, "libmambascan.so")
+MICRO_SRC = os.path.join(CSRC, "micro", "throughput.cu")
+MICRO_LIB = os.path.join(LIBDIR, "libmambamicro.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 NVCC_FLAGS = [
@@ -62,7 +64,21 @@ def stale() -> bool:
     return any(os.path.getmtime(p) > t for p in deps())
 
 
+def build_micro(force: bool = False) -> str:
+    """Build libmambamicro.so, the instruction-throughput microbenchmark that
+    ``bench.py --micro`` runs (not part of the scan library)."""
+    if not force and os.path.exists(MICRO_LIB) and \
+            os.path.getmtime(MICRO_LIB) >= os.path.getmtime(MICRO_SRC):
+        return MICRO_LIB
+    os.makedirs(LIBDIR, exist_ok=True)
+    tmp = MICRO_LIB + f".tmp{os.getpid()}"
+    subprocess.check_call([NVCC, *NVCC_FLAGS, MICRO_SRC, "-o", tmp])
+    os.replace(tmp, MICRO_LIB)
+    return MICRO_LIB
+
+
 def build(force: bool = False, verbose_ptxas: bool = False) -> str:
+    build_micro(force)
     if not force and not stale():
         return LIB
     os.makedirs(LIBDIR, exist_ok=True)

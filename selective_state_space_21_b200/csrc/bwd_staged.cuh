@@ -942,10 +942,27 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
   const size_t gk = size_t(G) * size_t(pl.K);
   const size_t n_A = gk * NM * kSThreads, n_D = gk * kSThreads;
   const size_t n_par = par ? gk * NM * kSThreads : 0;  // agg_G and gin each
-  const size_t bytes = int_bytes + 4 * (n_ckpt + n_carry + n_bc + n_A + 2 * n_D) +
-                       (par ? 8 * n_D + 8 * n_par : 0);
+  const size_t bytes = ceil_div(int_bytes + 4 * (n_ckpt + n_carry + n_bc + n_A + 2 * n_D) +
+                                    (par ? 8 * n_D + 8 * n_par : 0), 256) * 256;
+  // The checkpoint pass (the forward without y) is prepared first so that one
+  // workspace holds both: a failed allocation then leaves nothing enqueued.
+  FwdArgs fa;
+  fa.u = a.u; fa.delta = a.delta; fa.z = nullptr; fa.B = a.B; fa.C = a.C;
+  fa.bias = a.bias; fa.A = a.A; fa.D = nullptr; fa.y = nullptr; fa.last_state = nullptr;
+  fa.batch = a.batch; fa.dim = a.dim; fa.L = a.L; fa.N = a.N;
+  fa.conv_w = a.conv_w; fa.conv_b = a.conv_b; fa.conv_width = a.conv_width;
+  StagedOptions fo = o;
+  fo.chunk_len = 0;
+  fo.carry = 0;
+  fo.test_hook = 0;  // the hook targets the reverse hand-off
+  StagedForward<T, NM, CONV> ckpt_pass;
   unsigned char *ws = nullptr;
-  if (ws_alloc(reinterpret_cast<void **>(&ws), bytes, s) != cudaSuccess) {
+  {
+    // the checkpoint buffer is set once the workspace exists (before run)
+    const mamba_status_t pst = ckpt_pass.prepare(fa, fo, nullptr);
+    if (pst != MAMBA_OK) return pst;
+  }
+  if (ws_alloc(reinterpret_cast<void **>(&ws), bytes + ckpt_pass.bytes, s) != cudaSuccess) {
     cudaGetLastError();
     return MAMBA_ERR_OUT_OF_MEMORY;
   }
@@ -981,16 +998,8 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
   mamba_status_t st = MAMBA_OK;
   if (cudaMemsetAsync(ws, 0, int_bytes, s) != cudaSuccess) st = MAMBA_ERR_CUDA;
   if (st == MAMBA_OK) {
-    FwdArgs fa;
-    fa.u = a.u; fa.delta = a.delta; fa.z = nullptr; fa.B = a.B; fa.C = a.C;
-    fa.bias = a.bias; fa.A = a.A; fa.D = nullptr; fa.y = nullptr; fa.last_state = nullptr;
-    fa.batch = a.batch; fa.dim = a.dim; fa.L = a.L; fa.N = a.N;
-    fa.conv_w = a.conv_w; fa.conv_b = a.conv_b; fa.conv_width = a.conv_width;
-    StagedOptions fo = o;
-    fo.chunk_len = 0;
-    fo.carry = 0;
-    fo.test_hook = 0;  // the hook targets the reverse hand-off
-    st = staged_forward<T, NM, CONV>(fa, fo, s, launched, ckpt);
+    ckpt_pass.sa.ckpt = ckpt;
+    st = ckpt_pass.run(ws + bytes, s, launched);
   }
   if (st == MAMBA_OK && par) {
     bwd_adjoint_agg_kernel<T, NM><<<unsigned(size_t(G) * size_t(pl.K - 1)), kSThreads, 0, s>>>(bp);

@@ -114,40 +114,76 @@ __device__ __forceinline__ float dpsi_acc(float x) {
 // ----------------------------------------------------------- host: workspace
 
 // Workspace comes stream-ordered from one library-owned memory pool per device
-// that keeps up to kPoolKeepBytes reserved between calls, so that repeated
-// calls do not map and unmap hundreds of megabytes each time (the default
-// pool gives memory back to the system at every synchronization).
+// that keeps up to a reserve (kPoolKeepBytes unless the caller sets another)
+// between calls, so that repeated calls do not map and unmap hundreds of
+// megabytes each time (the default pool gives memory back to the system at
+// every synchronization).
 constexpr uint64_t kPoolKeepBytes = uint64_t(4) << 30;
+constexpr int kMaxDevices = 64;
 
-inline cudaMemPool_t library_pool() {
-  static std::mutex mu;
-  static cudaMemPool_t pools[64] = {};
-  static bool tried[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
-    cudaGetLastError();
-    return nullptr;
+struct PoolRegistry {
+  std::mutex mu;
+  cudaMemPool_t pools[kMaxDevices] = {};
+  bool tried[kMaxDevices] = {};
+  uint64_t keep[kMaxDevices];
+  PoolRegistry() {
+    for (int i = 0; i < kMaxDevices; ++i) keep[i] = kPoolKeepBytes;
   }
-  std::lock_guard<std::mutex> lock(mu);
-  if (!tried[dev]) {
-    tried[dev] = true;
+};
+
+inline PoolRegistry &pool_registry() {
+  static PoolRegistry r;
+  return r;
+}
+
+inline int current_device_or(int fallback) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return fallback;
+  }
+  return dev;
+}
+
+// The pool of the current device (created on first use), or null.
+inline cudaMemPool_t library_pool() {
+  const int dev = current_device_or(-1);
+  if (dev < 0) return nullptr;
+  PoolRegistry &r = pool_registry();
+  std::lock_guard<std::mutex> lock(r.mu);
+  if (!r.tried[dev]) {
+    r.tried[dev] = true;
     cudaMemPoolProps props = {};
     props.allocType = cudaMemAllocationTypePinned;
     props.location.type = cudaMemLocationTypeDevice;
     props.location.id = dev;
     cudaMemPool_t pool = nullptr;
     if (cudaMemPoolCreate(&pool, &props) == cudaSuccess) {
-      uint64_t keep = kPoolKeepBytes;
+      uint64_t keep = r.keep[dev];
       cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
-      pools[dev] = pool;
+      r.pools[dev] = pool;
     } else {
       cudaGetLastError();
     }
   }
-  return pools[dev];
+  return r.pools[dev];
+}
+
+// Test hook: the number of workspace allocations of the calling thread that
+// still succeed before one fails (negative: none fails).
+inline int &alloc_failure_countdown() {
+  static thread_local int n = -1;
+  return n;
 }
 
 inline cudaError_t ws_alloc(void **ptr, size_t bytes, cudaStream_t s) {
+  int &countdown = alloc_failure_countdown();
+  if (countdown == 0) {
+    countdown = -1;
+    *ptr = nullptr;
+    return cudaErrorMemoryAllocation;
+  }
+  if (countdown > 0) --countdown;
   cudaMemPool_t pool = library_pool();
   if (pool) return cudaMallocFromPoolAsync(ptr, bytes, pool, s);
   return cudaMallocAsync(ptr, bytes, s);

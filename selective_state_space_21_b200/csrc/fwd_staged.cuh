@@ -761,103 +761,114 @@ inline StagedPlan plan_staged(int64_t G, int64_t L, int slots, const StagedOptio
   return pl;
 }
 
-// The staged forward: tensor maps, plan, stream-ordered workspace, launches.
-// Returns MAMBA_ERR_UNSUPPORTED (nothing enqueued) if the driver rejects a
-// tensor map.
-// With `ckpt` non-null the forward runs without y and stores the state before
-// every kCkptEvery-th step into ckpt ([G][ceil(L/16)][NM][128] floats).
-// CONV selects the kernels with the convolution prologue (a.conv_w set).
+// The staged forward, split into a preparation (tensor maps, plan, the
+// workspace size; nothing enqueued) and the launches on a given workspace, so
+// that a caller can take one workspace for several steps and fail before
+// enqueuing anything when it cannot be had.
 template <typename T, int NM, bool CONV = false>
-mamba_status_t staged_forward(const FwdArgs &a, const StagedOptions &o, cudaStream_t s,
-                              mamba_status_t (*launched)(), float *ckpt = nullptr) {
+struct StagedForward {
   using Lay = StagedLayout<T, NM>;
-  constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
   CUtensorMap maps[6];
-  const uint64_t L = a.L, dim = a.dim, batch = a.batch, N = a.N;
-  const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_64B, none = CU_TENSOR_MAP_SWIZZLE_NONE;
-  if (!make_map_3d(&maps[0], a.u, bf16, L, dim, batch, Lay::TT, kSThreads, sw) ||
-      !make_map_3d(&maps[1], a.delta, bf16, L, dim, batch, Lay::TT, kSThreads, sw) ||
-      !make_map_3d(&maps[2], a.z ? a.z : a.u, bf16, L, dim, batch, Lay::TT, kSThreads, sw) ||
-      !make_map_3d(&maps[3], a.y ? a.y : a.u, bf16, L, dim, batch, Lay::TT, kSThreads, sw) ||
-      !make_map_3d(&maps[4], a.B, bf16, L, N, batch, Lay::TT, uint32_t(N), none) ||
-      !make_map_3d(&maps[5], a.C, bf16, L, N, batch, Lay::TT, uint32_t(N), none)) {
-    return MAMBA_ERR_UNSUPPORTED;
-  }
-  int bps_main = 0;
-  if (prepare_kernel<T, NM, KIND_SEQ, CONV>(&bps_main) != cudaSuccess) return MAMBA_ERR_CUDA;
-  const int sms = device_sm_count();
-  const int slots = sms * std::max(1, bps_main);
-  const int64_t gpb = ceil_div(a.dim, kSThreads);
-  const int64_t G = int64_t(a.batch) * gpb;
-  if (G > (int64_t(1) << 30)) return MAMBA_ERR_UNSUPPORTED;
-  const StagedPlan pl = plan_staged(G, a.L, slots, o);
-  if (G * pl.K > (int64_t(1) << 30)) return MAMBA_ERR_UNSUPPORTED;
-
   StagedArgs sa;
-  sa.f = a;
-  sa.G = int(G);
-  sa.gpb = int(gpb);
-  sa.K = pl.K;
-  sa.chunk_len = pl.chunk_len;
-  sa.timeout_ns = o.timeout_us > 0 ? uint64_t(o.timeout_us) * 1000ull : kDefaultTimeoutNs;
-  sa.test_hook = o.test_hook;
-  sa.force_generic = o.path == MAMBA_PATH_GENERIC ? 1 : 0;
-  sa.flags = nullptr;
-  sa.carry = sa.agg_h = sa.hin = nullptr;
-  sa.agg_S = nullptr;
-  sa.ckpt = ckpt;
+  StagedPlan pl;
+  int sms = 0, slots = 0;
+  size_t int_bytes = 0, bytes = 0;
 
-  // workspace: [ints: 2 counters + G flags][carry | agg_h, agg_S, hin]
-  const size_t n_int = 2 + size_t(G);
-  const size_t int_bytes = ceil_div(n_int * 4, 256) * 256;
-  size_t bytes = int_bytes;
-  const size_t gk = size_t(G) * size_t(pl.K);
-  if (pl.kind == KIND_SEQ) {
-    bytes += size_t(G) * NM * kSThreads * 4;
-  } else {
-    bytes += gk * kSThreads * 8 + 2 * gk * NM * kSThreads * 4;
-  }
-  unsigned char *ws = nullptr;
-  if (ws_alloc(reinterpret_cast<void **>(&ws), bytes, s) != cudaSuccess) {
-    cudaGetLastError();
-    return MAMBA_ERR_OUT_OF_MEMORY;
-  }
-  mamba_status_t st = MAMBA_OK;
-  if (cudaMemsetAsync(ws, 0, int_bytes, s) != cudaSuccess) st = MAMBA_ERR_CUDA;
-  int *counters = reinterpret_cast<int *>(ws);
-  sa.flags = counters + 2;
-  if (st == MAMBA_OK && pl.kind == KIND_SEQ) {
-    sa.carry = reinterpret_cast<float *>(ws + int_bytes);
-    sa.counter = counters;
-    sa.n_units = int(gk);
-    const int grid = int(std::min<int64_t>(gk, slots));
-    if (ckpt) {
-      int bps = 0;
-      if (prepare_kernel<T, NM, KIND_CKPT_SEQ, CONV>(&bps) != cudaSuccess) st = MAMBA_ERR_CUDA;
-      else launch_staged<T, NM, KIND_CKPT_SEQ, CONV>(maps, sa, int(std::min<int64_t>(gk, sms * std::max(1, bps))), s);
-    } else {
-      launch_staged<T, NM, KIND_SEQ, CONV>(maps, sa, grid, s);
+  // Builds the tensor maps and the plan; with `ckpt` the forward runs without
+  // y and stores the state before every kCkptEvery-th step into ckpt
+  // ([G][ceil(L/16)][NM][128] floats).  Returns MAMBA_ERR_UNSUPPORTED if the
+  // driver rejects a tensor map.
+  mamba_status_t prepare(const FwdArgs &a, const StagedOptions &o, float *ckpt) {
+    constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
+    const uint64_t L = a.L, dim = a.dim, batch = a.batch, N = a.N;
+    const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_64B, none = CU_TENSOR_MAP_SWIZZLE_NONE;
+    if (!make_map_3d(&maps[0], a.u, bf16, L, dim, batch, Lay::TT, kSThreads, sw) ||
+        !make_map_3d(&maps[1], a.delta, bf16, L, dim, batch, Lay::TT, kSThreads, sw) ||
+        !make_map_3d(&maps[2], a.z ? a.z : a.u, bf16, L, dim, batch, Lay::TT, kSThreads, sw) ||
+        !make_map_3d(&maps[3], a.y ? a.y : a.u, bf16, L, dim, batch, Lay::TT, kSThreads, sw) ||
+        !make_map_3d(&maps[4], a.B, bf16, L, N, batch, Lay::TT, uint32_t(N), none) ||
+        !make_map_3d(&maps[5], a.C, bf16, L, N, batch, Lay::TT, uint32_t(N), none)) {
+      return MAMBA_ERR_UNSUPPORTED;
     }
-    if (st == MAMBA_OK) st = launched();
-  } else if (st == MAMBA_OK) {
+    int bps_main = 0;
+    if (prepare_kernel<T, NM, KIND_SEQ, CONV>(&bps_main) != cudaSuccess) return MAMBA_ERR_CUDA;
+    sms = device_sm_count();
+    slots = sms * std::max(1, bps_main);
+    const int64_t gpb = ceil_div(a.dim, kSThreads);
+    const int64_t G = int64_t(a.batch) * gpb;
+    if (G > (int64_t(1) << 30)) return MAMBA_ERR_UNSUPPORTED;
+    pl = plan_staged(G, a.L, slots, o);
+    if (G * pl.K > (int64_t(1) << 30)) return MAMBA_ERR_UNSUPPORTED;
+
+    sa.f = a;
+    sa.G = int(G);
+    sa.gpb = int(gpb);
+    sa.K = pl.K;
+    sa.chunk_len = pl.chunk_len;
+    sa.timeout_ns = o.timeout_us > 0 ? uint64_t(o.timeout_us) * 1000ull : kDefaultTimeoutNs;
+    sa.test_hook = o.test_hook;
+    sa.force_generic = o.path == MAMBA_PATH_GENERIC ? 1 : 0;
+    sa.flags = nullptr;
+    sa.counter = nullptr;
+    sa.carry = sa.agg_h = sa.hin = nullptr;
+    sa.agg_S = nullptr;
+    sa.ckpt = ckpt;
+
+    // workspace: [ints: 2 counters + G flags][carry | agg_S, agg_h, hin]
+    const size_t n_int = 2 + size_t(G);
+    int_bytes = ceil_div(n_int * 4, 256) * 256;
+    bytes = int_bytes;
+    const size_t gk = size_t(G) * size_t(pl.K);
+    if (pl.kind == KIND_SEQ) {
+      bytes += size_t(G) * NM * kSThreads * 4;
+    } else {
+      bytes += gk * kSThreads * 8 + 2 * gk * NM * kSThreads * 4;
+    }
+    bytes = ceil_div(bytes, 256) * 256;
+    return MAMBA_OK;
+  }
+
+  // Enqueues the launches on `ws` (at least `bytes`, 256-byte aligned).
+  mamba_status_t run(unsigned char *ws, cudaStream_t s, mamba_status_t (*launched)()) {
+    mamba_status_t st = MAMBA_OK;
+    if (cudaMemsetAsync(ws, 0, int_bytes, s) != cudaSuccess) return MAMBA_ERR_CUDA;
+    int *counters = reinterpret_cast<int *>(ws);
+    sa.flags = counters + 2;
+    const size_t gk = size_t(sa.G) * size_t(pl.K);
+    if (pl.kind == KIND_SEQ) {
+      sa.carry = reinterpret_cast<float *>(ws + int_bytes);
+      sa.counter = counters;
+      sa.n_units = int(gk);
+      const int grid = int(std::min<int64_t>(gk, slots));
+      if (sa.ckpt) {
+        int bps = 0;
+        if (prepare_kernel<T, NM, KIND_CKPT_SEQ, CONV>(&bps) != cudaSuccess) return MAMBA_ERR_CUDA;
+        launch_staged<T, NM, KIND_CKPT_SEQ, CONV>(maps, sa,
+                                                  int(std::min<int64_t>(gk, sms * std::max(1, bps))), s);
+      } else {
+        launch_staged<T, NM, KIND_SEQ, CONV>(maps, sa, grid, s);
+      }
+      return launched();
+    }
     sa.agg_S = reinterpret_cast<double *>(ws + int_bytes);
     sa.agg_h = reinterpret_cast<float *>(ws + int_bytes + gk * kSThreads * 8);
     sa.hin = sa.agg_h + gk * NM * kSThreads;
     int bps_agg = 0, bps_par = 0;
     if (prepare_kernel<T, NM, KIND_AGG, CONV>(&bps_agg) != cudaSuccess ||
-        (ckpt ? prepare_kernel<T, NM, KIND_CKPT_PAR, CONV>(&bps_par)
-              : prepare_kernel<T, NM, KIND_PAR, CONV>(&bps_par)) != cudaSuccess) {
-      st = MAMBA_ERR_CUDA;
+        (sa.ckpt ? prepare_kernel<T, NM, KIND_CKPT_PAR, CONV>(&bps_par)
+                 : prepare_kernel<T, NM, KIND_PAR, CONV>(&bps_par)) != cudaSuccess) {
+      return MAMBA_ERR_CUDA;
     }
-    if (st == MAMBA_OK) {
+    {
       StagedArgs sg = sa;
       sg.counter = counters;
-      sg.n_units = int(size_t(G) * size_t(pl.K - 1));
-      launch_staged<T, NM, KIND_AGG, CONV>(maps, sg, int(std::min<int64_t>(sg.n_units, sms * std::max(1, bps_agg))), s);
+      sg.n_units = int(size_t(sa.G) * size_t(pl.K - 1));
+      launch_staged<T, NM, KIND_AGG, CONV>(maps, sg,
+                                           int(std::min<int64_t>(sg.n_units, sms * std::max(1, bps_agg))), s);
       st = launched();
     }
     if (st == MAMBA_OK) {
-      const int64_t threads = G * NM * kSThreads;
+      const int64_t threads = int64_t(sa.G) * NM * kSThreads;
       carry_scan_kernel<NM><<<unsigned(ceil_div(threads, 256)), 256, 0, s>>>(sa);
       st = launched();
     }
@@ -866,11 +877,30 @@ mamba_status_t staged_forward(const FwdArgs &a, const StagedOptions &o, cudaStre
       sm.counter = counters + 1;
       sm.n_units = int(gk);
       const int grid = int(std::min<int64_t>(gk, sms * std::max(1, bps_par)));
-      if (ckpt) launch_staged<T, NM, KIND_CKPT_PAR, CONV>(maps, sm, grid, s);
+      if (sa.ckpt) launch_staged<T, NM, KIND_CKPT_PAR, CONV>(maps, sm, grid, s);
       else launch_staged<T, NM, KIND_PAR, CONV>(maps, sm, grid, s);
       st = launched();
     }
+    return st;
   }
+};
+
+// The staged forward with its own stream-ordered workspace.  Returns
+// MAMBA_ERR_UNSUPPORTED (nothing enqueued) if the driver rejects a tensor map,
+// MAMBA_ERR_OUT_OF_MEMORY (nothing enqueued) if the workspace cannot be had.
+// CONV selects the kernels with the convolution prologue (a.conv_w set).
+template <typename T, int NM, bool CONV = false>
+mamba_status_t staged_forward(const FwdArgs &a, const StagedOptions &o, cudaStream_t s,
+                              mamba_status_t (*launched)(), float *ckpt = nullptr) {
+  StagedForward<T, NM, CONV> sf;
+  mamba_status_t st = sf.prepare(a, o, ckpt);
+  if (st != MAMBA_OK) return st;
+  unsigned char *ws = nullptr;
+  if (ws_alloc(reinterpret_cast<void **>(&ws), sf.bytes, s) != cudaSuccess) {
+    cudaGetLastError();
+    return MAMBA_ERR_OUT_OF_MEMORY;
+  }
+  st = sf.run(ws, s, launched);
   if (ws_free(ws, s) != cudaSuccess && st == MAMBA_OK) st = MAMBA_ERR_CUDA;
   return st;
 }

@@ -8,6 +8,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <new>
 
 #include "../../include/mamba_scan.h"
 #include "bwd_reference.cuh"
@@ -498,13 +499,26 @@ mamba_status_t mamba_scan_bwd_ex(const void *u, const void *delta, const float *
 
 namespace {
 
-// One decoding token, with (CONV) or without the convolution prologue.
+// One decoding token, validated once: the kernel arguments and the launch
+// shape.  A plan (mamba_scan_step_plan_create) keeps one of these so that a
+// decoding loop pays the pointer checks once instead of every token.
+struct StepPlan {
+  DecodeArgs a;
+  bool conv = false;
+  bool vec4 = false;
+  mamba_dtype_t dtype = MAMBA_F32;
+  int64_t grid = 0;
+  int dev = 0;
+};
+
+// Validates one decoding token's arguments (CONV: with the convolution
+// prologue) and fills `p`; enqueues nothing.
 template <bool CONV>
-mamba_status_t decode_step(float *state, float *conv_state, const void *u, const float *conv_w,
-                           const float *conv_b, int64_t conv_width, const void *delta,
-                           const float *delta_bias, const float *A, const void *B, const void *C,
-                           const float *D, const void *z, void *y, int64_t batch, int64_t dim,
-                           int64_t N, mamba_dtype_t dtype, mamba_stream_t stream) {
+mamba_status_t decode_prepare(StepPlan *p, float *state, float *conv_state, const void *u,
+                              const float *conv_w, const float *conv_b, int64_t conv_width,
+                              const void *delta, const float *delta_bias, const float *A,
+                              const void *B, const void *C, const float *D, const void *z, void *y,
+                              int64_t batch, int64_t dim, int64_t N, mamba_dtype_t dtype) {
   mamba_status_t st = check_shape(batch, dim, 1, N, dtype);
   if (st != MAMBA_OK) return st;
   if (CONV && (conv_width < 1 || conv_width > kMaxConvWidth)) return MAMBA_ERR_UNSUPPORTED;
@@ -531,25 +545,37 @@ mamba_status_t decode_step(float *state, float *conv_state, const void *u, const
     ck.buf(conv_state, nbd * size_t(conv_width - 1) * 4, 4, conv_width > 1, true);
   }
   if (ck.st != MAMBA_OK) return ck.st;
-  if (nbd == 0) return MAMBA_OK;
-  DecodeArgs a;
+  DecodeArgs &a = p->a;
   a.state = state; a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
   a.bias = delta_bias; a.A = A; a.D = D; a.y = y;
   a.batch = batch; a.dim = dim; a.N = (int)N;
   if (CONV) {
     a.conv_state = conv_state; a.conv_w = conv_w; a.conv_b = conv_b; a.conv_width = (int)conv_width;
   }
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  p->conv = CONV;
+  p->dtype = dtype;
+  p->dev = ck.dev;
   // four states per thread when N is 4, 8 or 16 and the state, A, B and C
   // rows are 16- (B, C: 8-) byte aligned
   const bool al16 = ((reinterpret_cast<uintptr_t>(state) | reinterpret_cast<uintptr_t>(A)) & 15) == 0;
   const bool alBC = ((reinterpret_cast<uintptr_t>(B) | reinterpret_cast<uintptr_t>(C)) & (4 * es - 1)) == 0;
-  if ((N == 4 || N == 8 || N == 16) && al16 && alBC) {
-    const int64_t threads = int64_t(nbd) * (N / 4);
-    const int64_t g4 = (threads + kDecodeThreads - 1) / kDecodeThreads;
-    if (g4 > (int64_t(1) << 31) - 1) return MAMBA_ERR_UNSUPPORTED;
-#define MSCAN_VEC4(TT, NN) decode_step_vec4_kernel<TT, NN, CONV><<<unsigned(g4), kDecodeThreads, 0, s>>>(a)
-    if (dtype == MAMBA_BF16) {
+  p->vec4 = (N == 4 || N == 8 || N == 16) && al16 && alBC;
+  const int64_t threads = p->vec4 ? int64_t(nbd) * (N / 4) : int64_t(nbd);
+  p->grid = (threads + kDecodeThreads - 1) / kDecodeThreads;
+  if (p->grid > (int64_t(1) << 31) - 1) return MAMBA_ERR_UNSUPPORTED;
+  return MAMBA_OK;
+}
+
+// Enqueues the one launch of a validated decoding token (nothing for an
+// empty problem).
+template <bool CONV>
+mamba_status_t decode_launch_t(const StepPlan &p, cudaStream_t s) {
+  const DecodeArgs &a = p.a;
+  const int N = a.N;
+  const unsigned g = unsigned(p.grid);
+  if (p.vec4) {
+#define MSCAN_VEC4(TT, NN) decode_step_vec4_kernel<TT, NN, CONV><<<g, kDecodeThreads, 0, s>>>(a)
+    if (p.dtype == MAMBA_BF16) {
       if (N == 4) MSCAN_VEC4(__nv_bfloat16, 4);
       else if (N == 8) MSCAN_VEC4(__nv_bfloat16, 8);
       else MSCAN_VEC4(__nv_bfloat16, 16);
@@ -561,15 +587,13 @@ mamba_status_t decode_step(float *state, float *conv_state, const void *u, const
 #undef MSCAN_VEC4
     return launch_status();
   }
-  const int64_t grid = (int64_t(nbd) + kDecodeThreads - 1) / kDecodeThreads;
-  if (grid > (int64_t(1) << 31) - 1) return MAMBA_ERR_UNSUPPORTED;
   auto launch = [&](auto tag, auto nm) {
     using T = typename decltype(tag)::type;
-    decode_step_kernel<T, decltype(nm)::value, CONV><<<unsigned(grid), kDecodeThreads, 0, s>>>(a);
+    decode_step_kernel<T, decltype(nm)::value, CONV><<<g, kDecodeThreads, 0, s>>>(a);
   };
   struct TF { using type = float; };
   struct TB { using type = __nv_bfloat16; };
-  if (dtype == MAMBA_BF16) {
+  if (p.dtype == MAMBA_BF16) {
     if (N <= 4) launch(TB{}, std::integral_constant<int, 4>{});
     else if (N <= 8) launch(TB{}, std::integral_constant<int, 8>{});
     else launch(TB{}, std::integral_constant<int, 16>{});
@@ -579,6 +603,26 @@ mamba_status_t decode_step(float *state, float *conv_state, const void *u, const
     else launch(TF{}, std::integral_constant<int, 16>{});
   }
   return launch_status();
+}
+
+mamba_status_t decode_launch(const StepPlan &p, cudaStream_t s) {
+  if (p.a.batch == 0 || p.a.dim == 0) return MAMBA_OK;
+  return p.conv ? decode_launch_t<true>(p, s) : decode_launch_t<false>(p, s);
+}
+
+// One decoding token, with (CONV) or without the convolution prologue.
+template <bool CONV>
+mamba_status_t decode_step(float *state, float *conv_state, const void *u, const float *conv_w,
+                           const float *conv_b, int64_t conv_width, const void *delta,
+                           const float *delta_bias, const float *A, const void *B, const void *C,
+                           const float *D, const void *z, void *y, int64_t batch, int64_t dim,
+                           int64_t N, mamba_dtype_t dtype, mamba_stream_t stream) {
+  StepPlan p;
+  const mamba_status_t st = decode_prepare<CONV>(&p, state, conv_state, u, conv_w, conv_b,
+                                                 conv_width, delta, delta_bias, A, B, C, D, z, y,
+                                                 batch, dim, N, dtype);
+  if (st != MAMBA_OK) return st;
+  return decode_launch(p, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // namespace
@@ -731,13 +775,18 @@ mamba_status_t mamba_conv_scan_bwd(const void *x, const float *conv_w, const flo
   a.dA = dA; a.dD = dD; a.dbias = ddelta_bias;
   a.batch = batch; a.dim = dim; a.L = L; a.N = (int)N;
   a.conv_w = conv_w; a.conv_b = conv_b; a.conv_width = (int)conv_width;
-  if ((st = backward_paths<true>(a, es, dtype, staged_options(options), s)) != MAMBA_OK) return st;
-  // 2. through SiLU and the convolution, in place on dx, then the filter sums
+  // the per-row filter sums of step 2 are allocated first, so that a failed
+  // allocation leaves nothing enqueued
   float *part = nullptr;
   if (ws_alloc(reinterpret_cast<void **>(&part), size_t(rows) * 5 * 4, s) != cudaSuccess) {
     cudaGetLastError();
     return MAMBA_ERR_OUT_OF_MEMORY;
   }
+  if ((st = backward_paths<true>(a, es, dtype, staged_options(options), s)) != MAMBA_OK) {
+    ws_free(part, s);
+    return st;
+  }
+  // 2. through SiLU and the convolution, in place on dx, then the filter sums
   const bool vec = (size_t(L) * es) % 16 == 0 &&
                    ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(dx)) & 15) == 0;
   const int W = (int)conv_width;
@@ -1003,6 +1052,112 @@ mamba_status_t mamba_cplx_scan_bwd(const void *u, const void *delta, const float
   a.batch = batch; a.dim = dim; a.L = L; a.N = (int)N;
   return dispatch<CplxBwdLauncher>(dtype, (int)N, a, s);
 }
+
+}  // extern "C"
+
+// ------------------------------------------------ decoding plans, pool, hooks
+
+struct mamba_step_plan_st {
+  StepPlan p;
+};
+
+extern "C" {
+
+mamba_status_t mamba_scan_step_plan_create(mamba_step_plan_t *plan, float *state,
+                                           float *conv_state, const void *x, const float *conv_w,
+                                           const float *conv_b, int64_t conv_width,
+                                           const void *delta, const float *delta_bias,
+                                           const float *A, const void *B, const void *C,
+                                           const float *D, const void *z, void *y, int64_t batch,
+                                           int64_t dim, int64_t N, mamba_dtype_t dtype) {
+  if (!plan) return MAMBA_ERR_INVALID_ARG;
+  *plan = nullptr;
+  if (conv_width < 0) return MAMBA_ERR_INVALID_ARG;
+  if (conv_width == 0 && (conv_state || conv_w || conv_b)) return MAMBA_ERR_INVALID_ARG;
+  mamba_step_plan_st *h = new (std::nothrow) mamba_step_plan_st;
+  if (!h) return MAMBA_ERR_OUT_OF_MEMORY;
+  const mamba_status_t st =
+      conv_width == 0
+          ? decode_prepare<false>(&h->p, state, nullptr, x, nullptr, nullptr, 0, delta,
+                                  delta_bias, A, B, C, D, z, y, batch, dim, N, dtype)
+          : decode_prepare<true>(&h->p, state, conv_state, x, conv_w, conv_b, conv_width, delta,
+                                 delta_bias, A, B, C, D, z, y, batch, dim, N, dtype);
+  if (st != MAMBA_OK) {
+    delete h;
+    return st;
+  }
+  *plan = h;
+  return MAMBA_OK;
+}
+
+mamba_status_t mamba_scan_step_plan_run(mamba_step_plan_t plan, mamba_stream_t stream) {
+  if (!plan) return MAMBA_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MAMBA_ERR_CUDA;
+  }
+  if (dev != plan->p.dev) return MAMBA_ERR_INVALID_ARG;
+  return decode_launch(plan->p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+void mamba_scan_step_plan_destroy(mamba_step_plan_t plan) { delete plan; }
+
+mamba_status_t mamba_scan_pool_set_reserve(uint64_t bytes) {
+  const int dev = current_device_or(-1);
+  if (dev < 0) return MAMBA_ERR_CUDA;
+  PoolRegistry &r = pool_registry();
+  cudaMemPool_t pool = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(r.mu);
+    r.keep[dev] = bytes;
+    pool = r.pools[dev];
+  }
+  if (pool && cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &bytes) != cudaSuccess) {
+    cudaGetLastError();
+    return MAMBA_ERR_CUDA;
+  }
+  return MAMBA_OK;
+}
+
+mamba_status_t mamba_scan_pool_trim(uint64_t keep_bytes) {
+  const int dev = current_device_or(-1);
+  if (dev < 0) return MAMBA_ERR_CUDA;
+  PoolRegistry &r = pool_registry();
+  cudaMemPool_t pool = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(r.mu);
+    pool = r.pools[dev];
+  }
+  if (pool && cudaMemPoolTrimTo(pool, size_t(keep_bytes)) != cudaSuccess) {
+    cudaGetLastError();
+    return MAMBA_ERR_CUDA;
+  }
+  return MAMBA_OK;
+}
+
+mamba_status_t mamba_scan_pool_reserved(uint64_t *bytes) {
+  if (!bytes) return MAMBA_ERR_INVALID_ARG;
+  *bytes = 0;
+  const int dev = current_device_or(-1);
+  if (dev < 0) return MAMBA_ERR_CUDA;
+  PoolRegistry &r = pool_registry();
+  cudaMemPool_t pool = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(r.mu);
+    pool = r.pools[dev];
+  }
+  if (!pool) return MAMBA_OK;
+  cuuint64_t v = 0;
+  if (cudaMemPoolGetAttribute(pool, cudaMemPoolAttrReservedMemCurrent, &v) != cudaSuccess) {
+    cudaGetLastError();
+    return MAMBA_ERR_CUDA;
+  }
+  *bytes = uint64_t(v);
+  return MAMBA_OK;
+}
+
+void mamba_scan_test_fail_alloc(int32_t after) { alloc_failure_countdown() = after < 0 ? -1 : after; }
 
 }  // extern "C"
 

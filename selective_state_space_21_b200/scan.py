@@ -7,7 +7,9 @@ Low-level calls (same names and argument order as ``include/mamba_scan.h``):
 ``mamba_conv_scan_bwd``, ``mamba_dtproj_scan_fwd``, ``mamba_dtproj_scan_bwd``,
 ``mamba_cplx_scan_fwd``, ``mamba_cplx_scan_bwd``, ``mamba_scan_step``,
 ``mamba_scan_fwd_noalloc``,
-``mamba_scan_stream_status``.  Convenience wrappers that allocate the outputs:
+``mamba_scan_stream_status``; decoding plans (``StepPlan``), the workspace
+pool (``pool_set_reserve``, ``pool_trim``, ``pool_reserved``) and the
+allocation-failure test hook (``test_fail_alloc``).  Convenience wrappers that allocate the outputs:
 ``selective_scan_fwd``, ``selective_scan_bwd``, ``conv_selective_scan_fwd``
 and ``conv_selective_scan_bwd``.
 """
@@ -93,6 +95,21 @@ def load_library():
             lib.mamba_scan_launch_count.restype = ctypes.c_uint64
             lib.mamba_scan_abi_version.argtypes = []
             lib.mamba_scan_abi_version.restype = ctypes.c_int
+            lib.mamba_scan_step_plan_create.argtypes = (
+                [ctypes.POINTER(vp)] + [vp] * 5 + [i64] + [vp] * 8 + [i64] * 3 + [i32])
+            lib.mamba_scan_step_plan_create.restype = ctypes.c_int
+            lib.mamba_scan_step_plan_run.argtypes = [vp, vp]
+            lib.mamba_scan_step_plan_run.restype = ctypes.c_int
+            lib.mamba_scan_step_plan_destroy.argtypes = [vp]
+            lib.mamba_scan_step_plan_destroy.restype = None
+            lib.mamba_scan_pool_set_reserve.argtypes = [ctypes.c_uint64]
+            lib.mamba_scan_pool_set_reserve.restype = ctypes.c_int
+            lib.mamba_scan_pool_trim.argtypes = [ctypes.c_uint64]
+            lib.mamba_scan_pool_trim.restype = ctypes.c_int
+            lib.mamba_scan_pool_reserved.argtypes = [ctypes.POINTER(ctypes.c_uint64)]
+            lib.mamba_scan_pool_reserved.restype = ctypes.c_int
+            lib.mamba_scan_test_fail_alloc.argtypes = [ctypes.c_int32]
+            lib.mamba_scan_test_fail_alloc.restype = None
             _lib = lib
     return _lib
 
@@ -410,6 +427,78 @@ def mamba_conv_scan_step(state, conv_state, x, conv_w, conv_b, delta, delta_bias
         batch, dim, N, _dtype_code(dt)]
     _check(load_library().mamba_conv_scan_step(*args, _stream_handle(stream)),
            "mamba_conv_scan_step")
+
+
+class StepPlan:
+    """A decoding plan (``mamba_scan_step_plan_create``): the buffers of one
+    decoding token checked once; ``run()`` enqueues the step with a single
+    kernel launch.  Write each token's u (or x), delta, z, B and C into the
+    given tensors before its run.  With ``conv_w`` the plan steps the
+    convolution prologue too (``conv_state`` (batch, dim, W - 1) float32,
+    ``conv_b`` optional)."""
+
+    def __init__(self, state, u, delta, delta_bias, A, B, C, D, z, y, *, conv_state=None,
+                 conv_w=None, conv_b=None):
+        batch, dim = u.shape
+        N = A.shape[1]
+        dt = u.dtype
+        f32 = torch.float32
+        W = conv_w.shape[1] if conv_w is not None else 0
+        self._keep = (state, u, delta, delta_bias, A, B, C, D, z, y, conv_state, conv_w, conv_b)
+        self._lib = load_library()
+        self._h = ctypes.c_void_p()
+        rc = self._lib.mamba_scan_step_plan_create(
+            ctypes.byref(self._h), _ptr(state, f32, (batch, dim, N), "state"),
+            _ptr(conv_state, f32, (batch, dim, max(W - 1, 0)), "conv_state") if W > 1 else None,
+            _ptr(u, dt, (batch, dim), "u"),
+            _ptr(conv_w, f32, (dim, W), "conv_w") if W else None,
+            _ptr(conv_b, f32, (dim,), "conv_b") if W else None, W,
+            _ptr(delta, dt, (batch, dim), "delta"), _ptr(delta_bias, f32, (dim,), "delta_bias"),
+            _ptr(A, f32, (dim, N), "A"), _ptr(B, dt, (batch, N), "B"),
+            _ptr(C, dt, (batch, N), "C"), _ptr(D, f32, (dim,), "D"),
+            _ptr(z, dt, (batch, dim), "z"), _ptr(y, dt, (batch, dim), "y"),
+            batch, dim, N, _dtype_code(dt))
+        _check(rc, "mamba_scan_step_plan_create")
+
+    def run(self, stream=None):
+        _check(self._lib.mamba_scan_step_plan_run(self._h, _stream_handle(stream)),
+               "mamba_scan_step_plan_run")
+
+    def close(self):
+        if self._h:
+            self._lib.mamba_scan_step_plan_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def pool_set_reserve(nbytes: int) -> None:
+    """Memory the library's workspace pool of the current device keeps mapped
+    between calls (default 4 GiB)."""
+    _check(load_library().mamba_scan_pool_set_reserve(int(nbytes)), "mamba_scan_pool_set_reserve")
+
+
+def pool_trim(keep_bytes: int = 0) -> None:
+    """Give the pool's unused memory on the current device back, down to
+    ``keep_bytes``."""
+    _check(load_library().mamba_scan_pool_trim(int(keep_bytes)), "mamba_scan_pool_trim")
+
+
+def pool_reserved() -> int:
+    """Bytes the library's workspace pool of the current device holds."""
+    v = ctypes.c_uint64()
+    _check(load_library().mamba_scan_pool_reserved(ctypes.byref(v)), "mamba_scan_pool_reserved")
+    return int(v.value)
+
+
+def test_fail_alloc(after: int) -> None:
+    """Test hook: the workspace allocation after ``after`` more successful
+    ones (on this thread) fails; negative disarms."""
+    load_library().mamba_scan_test_fail_alloc(int(after))
 
 
 def launch_count() -> int:

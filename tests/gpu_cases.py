@@ -68,6 +68,25 @@ def sample_channels(batch: int, dim: int, k: int, seed: int = 0) -> dict:
     return by_b
 
 
+def sample_channels_per_group(batch: int, dim: int, per_group: int, seed: int = 0,
+                              group: int = 128) -> dict:
+    """``per_group`` channels of every channel group of ``group`` channels in
+    every batch row (the first and last channel of each group included, the
+    rest drawn from a seeded generator), grouped by batch row."""
+    g = torch.Generator().manual_seed(seed)
+    by_b: dict = {}
+    for b in range(batch):
+        picks = set()
+        for g0 in range(0, dim, group):
+            g1 = min(dim, g0 + group)
+            chosen = {g0, g1 - 1}
+            while len(chosen) < min(per_group, g1 - g0):
+                chosen.add(g0 + int(torch.randint(g1 - g0, (1,), generator=g)))
+            picks |= chosen
+        by_b[b] = sorted(picks)
+    return by_b
+
+
 def sub_problem(x: dict, b: int, ds: list) -> dict:
     """The inputs of batch row b restricted to channels ds (channels are
     independent, so the oracle can run on this slice alone)."""
@@ -82,14 +101,18 @@ def sub_problem(x: dict, b: int, ds: list) -> dict:
     }
 
 
-def check_fwd_sampled(x_dev: dict, y: torch.Tensor, last: torch.Tensor, k: int, seed=0):
-    """Compare sampled channels of a full-size GPU forward with the oracle.
+def check_fwd_sampled(x_dev: dict, y: torch.Tensor, last: torch.Tensor, k: int, seed=0,
+                      samples: dict = None):
+    """Compare sampled channels of a full-size GPU forward with the oracle
+    (``k`` channels from ``sample_channels``, or the given ``samples``).
     Returns the worst normwise errors of y and last_state."""
     batch, dim, _ = x_dev["u"].shape
     x = to_host(x_dev)
     y_h, last_h = y.cpu(), last.cpu() if last is not None else None
     ey = el = 0.0
-    for b, ds in sample_channels(batch, dim, k, seed).items():
+    if samples is None:
+        samples = sample_channels(batch, dim, k, seed)
+    for b, ds in samples.items():
         sub = sub_problem(x, b, ds)
         y_ref, last_ref = oracle_fwd(sub)
         idx = torch.tensor(ds)

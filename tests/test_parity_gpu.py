@@ -159,12 +159,19 @@ def test_fwd_sequential_wait_times_out_without_hanging():
 @pytest.mark.parametrize("index", [1, 2, 3], ids=lambda i: WORKLOADS[i].name)
 def test_fwd_full_workload_sampled(index):
     """The full-size workloads in the launch configuration the benchmark
-    times (auto path), checked on sampled channels over their full length."""
+    times (auto path), checked on sampled channels over their full length.
+    The 2^20-step workload is checked on six channels of each of its twelve
+    channel groups (72 channels, each over every chunk boundary of its
+    group); the others on 48 channels spread over the grid."""
     w = WORKLOADS[index]
     x = workload_inputs(index, device="cuda", with_dy=False)
     y, last = gc.gpu_fwd(x)
-    k = 12 if w.L > 100_000 else 48
-    ey, el = gc.check_fwd_sampled(x, y, last, k=k, seed=index)
+    if w.L > 100_000:
+        samples = gc.sample_channels_per_group(w.batch, w.dim, 6, seed=index)
+        assert sum(len(v) for v in samples.values()) >= 64
+        ey, el = gc.check_fwd_sampled(x, y, last, k=0, samples=samples)
+    else:
+        ey, el = gc.check_fwd_sampled(x, y, last, k=48, seed=index)
     tol = gc.TOL[w.dtype]
     assert ey <= tol and el <= tol, f"{w.name}: y err {ey:.2e}, last_state err {el:.2e}"
     assert torch.isfinite(y).all()
@@ -266,13 +273,17 @@ def test_bwd_staged_deterministic():
         assert torch.equal(g1[k], g2[k]), k
 
 
-def test_bwd_full_workload_sampled():
-    """Forward + recompute backward at the full bf16 4 x 2048 x 4096 size:
-    per-channel gradients on sampled channels, dB / dC on one full batch row
-    (they sum over all channels), dA / dD / dbias on sampled channels."""
-    index = 4
+@pytest.mark.parametrize("index", [4, 2], ids=lambda i: WORKLOADS[i].name)
+def test_bwd_full_workload_sampled(index):
+    """Forward + recompute backward at full size, in the launch configuration
+    the benchmark times: the bf16 4 x 2048 x 4096 workload (three-phase
+    adjoint carry) and the benchmark's own bf16 8 x 5120 x 2048 workload
+    (sequential adjoint hand-off over 320 channel groups).  Per-channel
+    gradients on sampled channels, dB / dC on one full batch row (they sum
+    over all channels), dA / dD / dbias on a few channels summed over every
+    batch row."""
     w = WORKLOADS[index]
-    x = workload_inputs(index, device="cuda")
+    x = workload_inputs(index, device="cuda", with_dy=True)
     y, last = gc.gpu_fwd(x)
     ey, el = gc.check_fwd_sampled(x, y, last, k=16, seed=index)
     assert ey <= gc.TOL[w.dtype] and el <= gc.TOL[w.dtype]
@@ -299,7 +310,7 @@ def test_bwd_full_workload_sampled():
             e = gc.normwise(gh[k][bb].index_select(0, idx).double().numpy(), v)
             assert e <= tol, f"{k} (batch {bb}): {e:.2e}"
     # parameter gradients sum over the batch: all rows for a few channels
-    ds = [0, 1, 777, w.dim - 1]
+    ds = [0, 1, 777, 1300, w.dim - 1]
     idx = torch.tensor(ds)
     sub = {k: (v.index_select(1, idx).contiguous() if k in ("u", "delta", "z", "dy") else v)
            for k, v in xh.items()}
