@@ -61,10 +61,27 @@ struct BwdLayout {
   static constexpr int OFF_BS = OFF_SUB + NSEG * NM * kSThreads * 4;
   static constexpr int OFF_CS = OFF_BS + kBTT * BSTR * 4;
   static constexpr int OFF_RED = OFF_CS + kBTT * BSTR * 4;
-  static constexpr int OFF_BAR = OFF_RED + (kSThreads / 32) * kBTT * 33 * 4;
-  static constexpr int OFF_Q = OFF_BAR + 8 * kBStages;
+  static constexpr int RED_BYTES = (kSThreads / 32) * kBTT * 33 * 4;
+  static constexpr int OFF_BAR = OFF_RED + RED_BYTES;
+  static constexpr int OFF_Q = OFF_BAR + 8 * 4;  // stage barriers (2) + MMA barriers (2)
   static constexpr int BYTES = OFF_Q + 16 * 4;
   static constexpr int ALLOC = BYTES + 512;
+};
+
+// Stage geometry of the backward: u, then delta (or, with the fused
+// projection, the Rp x 16 dt_low tile), z, dy, B and C.
+template <typename T, int NM>
+struct BwdStage {
+  uint32_t z, dy, B, C, bytes;
+  __host__ __device__ BwdStage(int Rp) {
+    using Lay = BwdLayout<T, NM>;
+    const uint32_t dsz = Rp > 0 ? uint32_t(Rp) * Lay::RB : uint32_t(Lay::TILE);
+    z = Lay::TILE + dsz;
+    dy = z + Lay::TILE;
+    B = dy + Lay::TILE;
+    C = B + Lay::RAW;
+    bytes = (C + Lay::RAW + 511u) & ~511u;
+  }
 };
 
 struct BwdStagedArgs {
@@ -85,6 +102,9 @@ struct BwdStagedArgs {
   float *gin;        // [G][K][NM][128] Abar G entering each chunk from the later one
   float *agg_G;      // [G][K][NM][128] the same produced by each chunk from zero
   double *agg_S;     // [G][K][128] sum of Delta over each chunk
+  // fused Delta projection (PROJ kernels): R padded to 16; bytes of a stage
+  int Rp = 0;
+  uint32_t stage_bytes = 0;
 };
 
 // Byte offset of 16-byte chunk c of row r in a tile with RB-byte rows written
@@ -155,6 +175,41 @@ __device__ __forceinline__ float bfly_rest(float (&v)[16], int lane) {
   return v[0];
 }
 
+// Smallest and largest delta of thread `r`'s row in a 16-step tile: from the
+// tile in shared memory (swizzled rows), or (PROJ) from its TMEM accumulator.
+template <typename T, bool PROJ>
+__device__ __forceinline__ void tile_delta_range(const unsigned char *tile, uint32_t dacc, int r,
+                                                 float &mn, float &mx) {
+  float v[kBTT];
+  if constexpr (PROJ) {
+    float a[8], b[8];
+    tmem_ld8(dacc, a);
+    tmem_ld8(dacc + 8u, b);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v[i] = a[i];
+      v[8 + i] = b[i];
+    }
+  } else {
+    constexpr int RB = kBTT * (int)sizeof(T);
+#pragma unroll
+    for (int c = 0; c < RB / 16; ++c) {
+      float o[Vec<T>::kN];
+      Vec<T>::unpack(*reinterpret_cast<const uint4 *>(tile + swz_rows<RB>(r, c)), o);
+#pragma unroll
+      for (int i = 0; i < Vec<T>::kN; ++i) v[c * Vec<T>::kN + i] = o[i];
+    }
+  }
+  mn = v[0];
+  mx = v[0];
+#pragma unroll
+  for (int i = 1; i < kBTT; ++i) {
+    mn = fminf(mn, v[i]);
+    mx = fmaxf(mx, v[i]);
+  }
+}
+
 // Four consecutive x values of a row (16-byte aligned for float, 8-byte for
 // bf16), widened to float.
 __device__ __forceinline__ void load_x4(const float *p, float (&o)[4]) {
@@ -177,7 +232,12 @@ __device__ __forceinline__ void load_x4(const __nv_bfloat16 *p, float (&o)[4]) {
 // segment's x, the x just before it in the tile, and for the first steps of
 // a tile the four x values before the tile (read from global memory).  du is
 // the gradient with respect to u; the convolution's backward runs after.
-template <typename T, int NM, bool CONV = false>
+//
+// PROJ: delta is formed on the tensor cores as in the forward's fused
+// projection (fwd_staged.cuh): the Rp x 16 dt_low tiles come through the
+// pipeline, W_dt's rows for the CTA's channels sit in TMEM, and each thread
+// reads its channel's delta for a segment with tcgen05.ld.
+template <typename T, int NM, bool CONV = false, bool PROJ = false>
 __global__ void __launch_bounds__(kSThreads, 2)
     bwd_staged_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_d,
                       const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_dy,
@@ -188,26 +248,48 @@ __global__ void __launch_bounds__(kSThreads, 2)
   constexpr int NP = NM / 2;
   constexpr int SEG = Lay::SEG;
   using IO = SegIO<T, SEG>;
+  static_assert(!PROJ || (std::is_same<T, __nv_bfloat16>::value && !CONV),
+                "the fused projection takes bf16 operands and no convolution prologue");
 
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *sm = smem_raw + ((512u - (smem_u32(smem_raw) & 511u)) & 511u);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sm + Lay::OFF_BAR);
-  int *q = reinterpret_cast<int *>(sm + Lay::OFF_Q);
-  float *sub = reinterpret_cast<float *>(sm + Lay::OFF_SUB);  // [NSEG][NM][128]
-  float *Bs = reinterpret_cast<float *>(sm + Lay::OFF_BS);
-  float *Cs = reinterpret_cast<float *>(sm + Lay::OFF_CS);
-  float *red = reinterpret_cast<float *>(sm + Lay::OFF_RED);  // [4 warps][kBTT][33] (padded rows)
+  const BwdStage<T, NM> bst(PROJ ? p.Rp : 0);
+  const uint32_t SST = PROJ ? bst.bytes : uint32_t(Lay::STAGE);
+  const uint32_t OFF_Z = PROJ ? bst.z : 2u * Lay::TILE;
+  const uint32_t OFF_DY = PROJ ? bst.dy : 3u * Lay::TILE;
+  const uint32_t OFF_B = PROJ ? bst.B : 4u * Lay::TILE;
+  const uint32_t OFF_C = PROJ ? bst.C : 4u * Lay::TILE + Lay::RAW;
+  const uint32_t OFF_SUB = kBStages * SST;
+  const uint32_t OFF_BS = OFF_SUB + uint32_t(Lay::OFF_BS - Lay::OFF_SUB);
+  const uint32_t OFF_CS = OFF_SUB + uint32_t(Lay::OFF_CS - Lay::OFF_SUB);
+  const uint32_t OFF_RED = OFF_SUB + uint32_t(Lay::OFF_RED - Lay::OFF_SUB);
+  const uint32_t OFF_BAR = OFF_SUB + uint32_t(Lay::OFF_BAR - Lay::OFF_SUB);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);  // [2 stages], then 2 MMA barriers
+  uint64_t *mma_bar = bars + 2;
+  int *q = reinterpret_cast<int *>(sm + OFF_BAR + 8 * 4);  // [0..7] tickets, [8] abort, [12] TMEM
+  float *sub = reinterpret_cast<float *>(sm + OFF_SUB);  // [NSEG][NM][128]
+  float *Bs = reinterpret_cast<float *>(sm + OFF_BS);
+  float *Cs = reinterpret_cast<float *>(sm + OFF_CS);
+  float *red = reinterpret_cast<float *>(sm + OFF_RED);  // [4 warps][kBTT][33] (padded rows)
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const BwdArgs &f = p.w;
   const int N = f.N;
   const bool has_z = f.z != nullptr;
   const int64_t n16 = (f.L + kBTT - 1) / kBTT;
-  const uint32_t tile_bytes = (has_z ? 4u : 3u) * Lay::TILE + 2u * uint32_t(N) * RB;
+  const uint32_t tile_bytes = (has_z ? 3u : 2u) * Lay::TILE +
+                              (PROJ ? uint32_t(p.Rp) * RB : uint32_t(Lay::TILE)) + 2u * uint32_t(N) * RB;
+  [[maybe_unused]] constexpr uint32_t kIdesc = mma_idesc_bf16(128, kBTT, false, true);
+  [[maybe_unused]] uint32_t tbase = 0;
+  [[maybe_unused]] int mma_issued = -1;
 
   if (tid == 0) {
 #pragma unroll
     for (int s = 0; s < kBStages; ++s) mbar_init(&bars[s], 1);
+    if (PROJ) {
+      mbar_init(&mma_bar[0], 1);
+      mbar_init(&mma_bar[1], 1);
+    }
     fence_barrier_init();
     prefetch_tensormap(&tm_u);
     prefetch_tensormap(&tm_d);
@@ -217,7 +299,38 @@ __global__ void __launch_bounds__(kSThreads, 2)
     if (has_z) prefetch_tensormap(&tm_z);
     q[8] = 0;
   }
+  if constexpr (PROJ) {
+    if (tid < 32) {
+      tmem_alloc(reinterpret_cast<uint32_t *>(&q[12]), kProjTmemCols);
+      tmem_relinquish();
+    }
+  }
   __syncthreads();
+  if constexpr (PROJ) {
+    tc_fence_after_sync();
+    tbase = uint32_t(q[12]);
+  }
+
+  // Issues (thread 0) the projection MMAs of consumed-tile index `ct` into
+  // accumulator ct & 1 once the tile's dt_low rows have landed: 16 rows of
+  // 32 bytes (two 256-byte swizzle atoms) per MMA.
+  [[maybe_unused]] auto issue_mma = [&](int ct) {
+    const int stg = ct % kBStages;
+    if (!mbar_wait_bounded(&bars[stg], uint32_t(ct / kBStages) & 1u, p.timeout_ns)) {
+      record_timeout();
+      q[8] = 1;
+      return;
+    }
+    tc_fence_after_sync();
+    const uint32_t dt_addr = smem_u32(sm + stg * SST + Lay::TILE);
+    const uint32_t acc = tbase + kProjAcc + uint32_t(ct & 1) * kBTT;
+    for (int kk = 0; kk < p.Rp / 16; ++kk) {
+      const uint64_t bdesc = smem_desc(dt_addr + uint32_t(kk) * 512u, 16u, 256u, 6u);
+      mma_ts(acc, tbase + uint32_t(kk) * 8u, bdesc, kIdesc, kk > 0);
+    }
+    mma_commit(&mma_bar[ct & 1]);
+    mma_issued = ct;
+  };
 
   // ---- producer (thread 0): tiles of the current unit, last tile first
   int p_ticket = 0, p_tile = 0, p_ntiles = 0, p_tail = 0, p_issued = 0;
@@ -246,15 +359,16 @@ __global__ void __launch_bounds__(kSThreads, 2)
     const int b = g / p.gpb, d0 = (g % p.gpb) * kSThreads;
     const int t0 = k * p.chunk_len + (p_ntiles - 1 - p_tile) * kBTT;
     const int stage = p_issued % kBStages;
-    unsigned char *st = sm + stage * Lay::STAGE;
+    unsigned char *st = sm + stage * SST;
     uint64_t *bar = &bars[stage];
     mbar_arrive_expect_tx(bar, tile_bytes);
     tma_load_3d(st, &tm_u, bar, t0, d0, b);
-    tma_load_3d(st + Lay::TILE, &tm_d, bar, t0, d0, b);
-    if (has_z) tma_load_3d(st + 2 * Lay::TILE, &tm_z, bar, t0, d0, b);
-    tma_load_3d(st + 3 * Lay::TILE, &tm_dy, bar, t0, d0, b);
-    tma_load_3d(st + 4 * Lay::TILE, &tm_B, bar, t0, 0, b);
-    tma_load_3d(st + 4 * Lay::TILE + Lay::RAW, &tm_C, bar, t0, 0, b);
+    if (PROJ) tma_load_3d(st + Lay::TILE, &tm_d, bar, t0, 0, b);  // dt_low rows 0..Rp-1
+    else tma_load_3d(st + Lay::TILE, &tm_d, bar, t0, d0, b);
+    if (has_z) tma_load_3d(st + OFF_Z, &tm_z, bar, t0, d0, b);
+    tma_load_3d(st + OFF_DY, &tm_dy, bar, t0, d0, b);
+    tma_load_3d(st + OFF_B, &tm_B, bar, t0, 0, b);
+    tma_load_3d(st + OFF_C, &tm_C, bar, t0, 0, b);
     ++p_tile;
     ++p_issued;
   };
@@ -296,6 +410,26 @@ __global__ void __launch_bounds__(kSThreads, 2)
 #pragma unroll
     for (int n = 1; n < NM; ++n) structured = structured && (Arow[n] == float(n + 1) * Arow[0]);
     const bool sig = structured && Arow[0] == -1.f;
+    if constexpr (PROJ) {
+      // this group's rows of W_dt into TMEM (as in the forward's fused projection)
+      const __nv_bfloat16 *wrow = static_cast<const __nv_bfloat16 *>(f.W_dt) +
+                                  (valid ? int64_t(d) * f.R : 0);
+      for (int c8 = 0; c8 < p.Rp / 16; ++c8) {
+        uint32_t r[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int k = 16 * c8 + 2 * i;
+          const uint32_t lo = (valid && k < f.R) ? __bfloat16_as_ushort(wrow[k]) : 0u;
+          const uint32_t hi = (valid && k + 1 < f.R) ? __bfloat16_as_ushort(wrow[k + 1]) : 0u;
+          r[i] = lo | (hi << 16);
+        }
+        tmem_st8(tmem_at(tbase, uint32_t(warp) * 32u, uint32_t(c8) * 8u), r);
+      }
+      tmem_st_wait();
+      tc_fence_before_sync();
+      __syncthreads();
+      if (tid == 0) issue_mma(ctile);
+    }
     int mode = MODE_GEN;
     if (!p.force_generic) {
       if (__syncthreads_and(sig)) mode = MODE_SIG;
@@ -335,6 +469,14 @@ __global__ void __launch_bounds__(kSThreads, 2)
       constexpr bool kS = M != MODE_GEN;
       const float A0 = Arow[0];
       const float invA0 = 1.f / A0;
+      // delta below d_lo or above d_hi gives Delta |A0| below 1e-5 or above 6
+      // (inverse softplus of those, less the bias)
+      [[maybe_unused]] float d_lo = 0.f, d_hi = 0.f;
+      if constexpr (kS) {
+        const float ylo = 1e-5f / fabsf(A0), yhi = 6.f / fabsf(A0);
+        d_lo = logf(expm1f(ylo)) - bias;
+        d_hi = yhi + logf(-expm1f(-yhi)) - bias;
+      }
       // per-mode state: pairs for the structured arithmetic, scalars otherwise
       f2 Gt[NP], Acc[NP];
       float gs[NM], accs[NM], A2[NM], invA[NM];
@@ -358,7 +500,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
       // arithmetic; also returns Delta and sigma(v).
       auto step_decay = [&](float v, f2 (&P)[NP], float &Delta, float &sv) {
         if constexpr (M == MODE_SIG) {
-          const float vc = fminf(fmaxf(v, -80.f), 80.f);
+          const float vc = fmaxf(v, -87.f);  // e^-v overflows below -88
           const float ev = ex2f(-vc * kLog2e);
           const float s = rcpf(1.f + ev);
           decay_pairs<NM>(-s, ev * s, P);
@@ -379,7 +521,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
         const int nseg = steps / SEG;
         const int stage = ctile % kBStages;
         const uint32_t parity = uint32_t(ctile / kBStages) & 1u;
-        unsigned char *st = sm + stage * Lay::STAGE;
+        unsigned char *st = sm + stage * SST;
         // checkpoint of the tile start (issued before the wait to overlap)
         float h0[NM];
         {
@@ -397,9 +539,18 @@ __global__ void __launch_bounds__(kSThreads, 2)
           record_timeout();
           q[8] = 1;
         }
+        [[maybe_unused]] uint32_t dacc = 0;
+        if constexpr (PROJ) {  // this tile's delta: wait for its MMA
+          if (!mbar_wait_bounded(&mma_bar[ctile & 1], uint32_t(ctile >> 1) & 1u, p.timeout_ns)) {
+            record_timeout();
+            q[8] = 1;
+          }
+          tc_fence_after_sync();
+          dacc = tmem_at(tbase + kProjAcc + uint32_t(ctile & 1) * kBTT, uint32_t(warp) * 32u, 0);
+        }
         {
-          const T *Braw = reinterpret_cast<const T *>(st + 4 * Lay::TILE);
-          const T *Craw = reinterpret_cast<const T *>(st + 4 * Lay::TILE + Lay::RAW);
+          const T *Braw = reinterpret_cast<const T *>(st + OFF_B);
+          const T *Craw = reinterpret_cast<const T *>(st + OFF_C);
           constexpr int ITEMS = NM * (kBTT / 4);
           for (int w = tid; w < 2 * ITEMS; w += kSThreads) {
             const bool isC = w >= ITEMS;
@@ -412,13 +563,31 @@ __global__ void __launch_bounds__(kSThreads, 2)
             for (int i = 0; i < 4; ++i) dst[i * BSTR] = n < N ? raw_to_f(src, i) * scale : 0.f;
           }
         }
-        __syncthreads();
+        bool tile_gen = false;
+        if constexpr (kS) {  // any step of the tile outside the structured range?
+          float dmin = 0.f, dmax = 0.f;
+          tile_delta_range<T, PROJ>(st + Lay::TILE, dacc, tid, dmin, dmax);
+          tile_gen = __syncthreads_or(valid && (dmax > d_hi || dmin < d_lo));
+        } else {
+          __syncthreads();
+        }
         if (q[8]) return;
 
         const unsigned char *su = st;
-        const unsigned char *sd = st + Lay::TILE;
-        const unsigned char *sz = st + 2 * Lay::TILE;
-        const unsigned char *sdy = st + 3 * Lay::TILE;
+        [[maybe_unused]] const unsigned char *sd = st + Lay::TILE;
+        const unsigned char *sz = st + OFF_Z;
+        const unsigned char *sdy = st + OFF_DY;
+
+        // delta of one segment: from the tile, or (PROJ) from TMEM
+        auto load_d = [&](int seg, float (&dv)[SEG]) {
+          if constexpr (PROJ) {
+            static_assert(SEG == 2, "two-step segments in bf16");
+            tmem_ld2(dacc + uint32_t(seg) * SEG, dv);
+            tmem_ld_wait();
+          } else {
+            IO::load(sd, tid, seg, dv);
+          }
+        };
 
         // u of one segment of the tile
         auto load_u = [&](int seg, float (&uv)[SEG]) {
@@ -465,208 +634,245 @@ __global__ void __launch_bounds__(kSThreads, 2)
           }
         };
 
-        // forward over the tile: the state before every segment -> shared memory
-        {
-          f2 H[NP];
-          float h[NM];
-          if constexpr (kS) {
-#pragma unroll
-            for (int i = 0; i < NP; ++i) H[i] = pk(h0[2 * i], h0[2 * i + 1]);
-          } else {
-#pragma unroll
-            for (int n = 0; n < NM; ++n) h[n] = h0[n];
-          }
-          for (int seg = 0; seg < nseg; ++seg) {
-            float *sp = sub + (seg * NM) * kSThreads + tid;
-            if constexpr (kS) {
-#pragma unroll
-              for (int i = 0; i < NP; ++i) {
-                sp[(2 * i) * kSThreads] = lo_of(H[i]);
-                sp[(2 * i + 1) * kSThreads] = hi_of(H[i]);
-              }
+        // One tile with the structured (S) or the generic arithmetic.
+        auto tile_body = [&](auto stag) {
+          constexpr bool S = decltype(stag)::value;
+          // forward over the tile: the state before every segment -> shared memory
+          {
+            f2 H[NP];
+            float h[NM];
+            if constexpr (S) {
+  #pragma unroll
+              for (int i = 0; i < NP; ++i) H[i] = pk(h0[2 * i], h0[2 * i + 1]);
             } else {
-#pragma unroll
-              for (int n = 0; n < NM; ++n) sp[n * kSThreads] = h[n];
+  #pragma unroll
+              for (int n = 0; n < NM; ++n) h[n] = h0[n];
             }
-            if (seg == nseg - 1) break;  // the last segment is re-run below anyway
-            float uv[SEG], dv[SEG];
+            for (int seg = 0; seg < nseg; ++seg) {
+              float *sp = sub + (seg * NM) * kSThreads + tid;
+              if constexpr (S) {
+  #pragma unroll
+                for (int i = 0; i < NP; ++i) {
+                  sp[(2 * i) * kSThreads] = lo_of(H[i]);
+                  sp[(2 * i + 1) * kSThreads] = hi_of(H[i]);
+                }
+              } else {
+  #pragma unroll
+                for (int n = 0; n < NM; ++n) sp[n * kSThreads] = h[n];
+              }
+              if (seg == nseg - 1) break;  // the last segment is re-run below anyway
+              float uv[SEG], dv[SEG];
+              load_u(seg, uv);
+              load_d(seg, dv);
+  #pragma unroll
+              for (int i = 0; i < SEG; ++i) {
+                const float *Brow = Bs + (seg * SEG + i) * BSTR;
+                if constexpr (S) {
+                  f2 P[NP];
+                  float Delta, sv;
+                  step_decay(dv[i] + bias, P, Delta, sv);
+                  struct_update<NM>(H, P, uv[i] * invA0, 0.f, Brow, Brow);
+                } else {
+                  const float Delta = softplus_fast(dv[i] + bias);
+                  generic_update<NM, kS>(h, Delta, uv[i], 0.f, Arow, A2, invA, Brow, Brow);
+                }
+              }
+            }
+          }
+
+          // the next tile's projection MMA, into the other accumulator
+          if constexpr (PROJ) {
+            if (tid == 0 && it + 1 < ntiles) issue_mma(ctile + 1);
+            __syncwarp();
+          }
+
+          // segments from the last: re-run into registers, then walk backwards
+          for (int seg = nseg - 1; seg >= 0; --seg) {
+            float uv[SEG], dv[SEG], zv[SEG], dyv[SEG];
             load_u(seg, uv);
-            IO::load(sd, tid, seg, dv);
-#pragma unroll
-            for (int i = 0; i < SEG; ++i) {
-              const float *Brow = Bs + (seg * SEG + i) * BSTR;
-              if constexpr (kS) {
+            load_d(seg, dv);
+            IO::load(sdy, tid, seg, dyv);
+            if (has_z) IO::load(sz, tid, seg, zv);
+            float du_o[SEG], dd_o[SEG], dz_o[SEG];
+            const float *sp = sub + (seg * NM) * kSThreads + tid;
+
+            if constexpr (S) {
+              // states before each step of the segment (the state after a step
+              // is recomputed in the reverse step from h_{t-1} and t1)
+              f2 Hs[SEG][NP];
+  #pragma unroll
+              for (int i = 0; i < NP; ++i)
+                Hs[0][i] = pk(sp[(2 * i) * kSThreads], sp[(2 * i + 1) * kSThreads]);
+  #pragma unroll
+              for (int i = 0; i + 1 < SEG; ++i) {
+                const float *Brow = Bs + (seg * SEG + i) * BSTR;
                 f2 P[NP];
                 float Delta, sv;
                 step_decay(dv[i] + bias, P, Delta, sv);
-                struct_update<NM>(H, P, uv[i] * invA0, 0.f, Brow, Brow);
-              } else {
-                const float Delta = softplus_fast(dv[i] + bias);
-                generic_update<NM>(h, Delta, uv[i], 0.f, Arow, A2, invA, Brow, Brow);
+  #pragma unroll
+                for (int j = 0; j < NP; ++j) Hs[i + 1][j] = Hs[i][j];
+                struct_update<NM>(Hs[i + 1], P, uv[i] * invA0, 0.f, Brow, Brow);
               }
+  #pragma unroll
+              for (int i = SEG - 1; i >= 0; --i) {
+                const int tl = seg * SEG + i;
+                const float *Brow = Bs + tl * BSTR;
+                const float *Crow = Cs + tl * BSTR;
+                f2 P[NP];
+                float Delta, sv;
+                step_decay(dv[i] + bias, P, Delta, sv);
+                float dy0 = dyv[i], sz = 0.f;
+                if (has_z) {
+                  sz = rcpf(1.f + ex2f(-zv[i] * kLog2e));
+                  dy0 *= zv[i] * sz;
+                }
+                const float up = uv[i] * invA0;
+                const float x1 = Delta * A0;
+                const f2 U = pk(up, up), DY = pk(dy0, dy0), X1n = pk(-x1, -x1), Z = pk(0.f, 0.f);
+                f2 DU = Z, DD = Z, Y0 = Z;
+                const bool up16 = (lane & 16) != 0;
+                float v16[16];
+  #pragma unroll
+                for (int j = 0; j < NP; j += 2) {
+                  const ulonglong2 bq = *reinterpret_cast<const ulonglong2 *>(Brow + 2 * j);
+                  const ulonglong2 cq2 = *reinterpret_cast<const ulonglong2 *>(Crow + 2 * j);
+  #pragma unroll
+                  for (int e = 0; e < 2; ++e) {
+                    const int jj = j + e;
+                    const f2 Bp = e ? bq.y : bq.x;
+                    const f2 Cp = e ? cq2.y : cq2.x;
+                    const f2 CN = pk(float(2 * jj + 1), float(2 * jj + 2));
+                    const f2 Gv = fma2(Cp, DY, Gt[jj]);
+                    const f2 Ga = fma2(Gv, P[jj], Gv);
+                    const f2 w = fma2(Gv, P[jj], Z);
+                    const f2 t1 = fma2(Bp, U, Hs[i][jj]);
+                    const f2 hcur = fma2(P[jj], t1, Hs[i][jj]);  // h_t
+                    const f2 cq = fma2(fma2(Ga, t1, Z), CN, Z);
+                    DD = fma2(cq, pk(1.f, 1.f), DD);
+                    Acc[jj] = fma2(X1n, cq, Acc[jj]);
+                    const f2 dBc = fma2(w, U, Z);
+                    Acc[jj] = fma2(dBc, Bp, Acc[jj]);
+                    DU = fma2(w, Bp, DU);
+                    Y0 = fma2(Cp, hcur, Y0);
+                    const f2 dCc = fma2(DY, hcur, Z);
+                    Gt[jj] = Ga;
+                    // Channels past `dim` contribute exact zeros: TMA fills their
+                    // rows with 0, so dy0 = 0 and their adjoint stays 0.
+                    v16[2 * jj] = bfly_first(lo_of(dBc), lo_of(dCc), up16);
+                    v16[2 * jj + 1] = bfly_first(hi_of(dBc), hi_of(dCc), up16);
+                  }
+                }
+  #pragma unroll
+                for (int n = NM; n < kMaxN; ++n) v16[n] = 0.f;
+                const float du = fmaf(lo_of(DU) + hi_of(DU), invA0, Dd * dy0);
+                const float dd = A0 * (lo_of(DD) + hi_of(DD)) * sv;
+                const float y0 = (lo_of(Y0) + hi_of(Y0)) + Dd * uv[i];
+                du_o[i] = du;
+                dd_o[i] = dd;
+                dz_o[i] = has_z ? dyv[i] * y0 * sz * (1.f + zv[i] * (1.f - sz)) : 0.f;
+                dDsum = fmaf(dy0, uv[i], dDsum);
+                dbsum += dd;
+                const float rsum = bfly_rest(v16, lane);
+                // lane l holds dB (l < 16, to be divided by l+1) or dC of state l-16
+                red[(warp * kBTT + tl) * 33 + lane] = (lane < kMaxN) ? rsum * (1.f / float(lane + 1)) : rsum;
+              }
+            } else {
+              float Hs[SEG][NM];
+  #pragma unroll
+              for (int n = 0; n < NM; ++n) Hs[0][n] = sp[n * kSThreads];
+  #pragma unroll
+              for (int i = 0; i + 1 < SEG; ++i) {
+                const float *Brow = Bs + (seg * SEG + i) * BSTR;
+                const float Delta = softplus_fast(dv[i] + bias);
+  #pragma unroll
+                for (int n = 0; n < NM; ++n) Hs[i + 1][n] = Hs[i][n];
+                generic_update<NM, kS>(Hs[i + 1], Delta, uv[i], 0.f, Arow, A2, invA, Brow, Brow);
+              }
+  #pragma unroll
+              for (int i = SEG - 1; i >= 0; --i) {
+                const int tl = seg * SEG + i;
+                const float *Brow = Bs + tl * BSTR;
+                const float *Crow = Cs + tl * BSTR;
+                const float v = dv[i] + bias;
+                const float Delta = softplus_fast(v);
+                const float sv = rcpf(1.f + ex2f(-v * kLog2e));
+                float dy0 = dyv[i], sz = 0.f;
+                if (has_z) {
+                  sz = rcpf(1.f + ex2f(-zv[i] * kLog2e));
+                  dy0 *= zv[i] * sz;
+                }
+                float du_acc = 0.f, dD_acc = 0.f, y0 = Dd * uv[i];
+                const bool up16 = (lane & 16) != 0;
+                float v16[16];
+  #pragma unroll
+                for (int n = 0; n < NM; ++n) {
+                  const float x = Delta * Arow[n];
+                  const float a = ex2f(Delta * A2[n]);
+                  float pp = fmaf(x, 1.f / 720.f, 1.f / 120.f);
+                  pp = fmaf(x, pp, 1.f / 24.f);
+                  pp = fmaf(x, pp, 1.f / 6.f);
+                  pp = fmaf(x, pp, 0.5f);
+                  pp = fmaf(x, pp, 1.f);
+                  const float Eb = fabsf(x) < 0.25f ? Delta * pp : (a - 1.f) * invA[n];  // Bbar / B
+                  const float Bn = kS ? Brow[n] * float(n + 1) : Brow[n], Cn = Crow[n];
+                  const float hprev = Hs[i][n];
+                  const float hcur = fmaf(a, hprev, Eb * (Bn * uv[i]));  // h_t, as in the forward
+                  const float Gv = fmaf(Cn, dy0, gs[n]);
+                  const float Ga = a * Gv;
+                  const float wv = Gv * Eb;
+                  du_acc = fmaf(wv, Bn, du_acc);
+                  dD_acc = fmaf(Ga, fmaf(Bn, uv[i], Arow[n] * hprev), dD_acc);
+                  accs[n] = fmaf(Gv, Delta * a * hprev + Bn * uv[i] * Delta * Delta * dpsi_fast(x, a), accs[n]);
+                  y0 = fmaf(Cn, hcur, y0);
+                  v16[n] = bfly_first(wv * uv[i], dy0 * hcur, up16);  // zero past `dim`
+                  gs[n] = Ga;
+                }
+  #pragma unroll
+                for (int n = NM; n < kMaxN; ++n) v16[n] = 0.f;
+                const float dd = dD_acc * sv;
+                du_o[i] = fmaf(Dd, dy0, du_acc);
+                dd_o[i] = dd;
+                dz_o[i] = has_z ? dyv[i] * y0 * sz * (1.f + zv[i] * (1.f - sz)) : 0.f;
+                dDsum = fmaf(dy0, uv[i], dDsum);
+                dbsum += dd;
+                red[(warp * kBTT + tl) * 33 + lane] = bfly_rest(v16, lane);
+              }
+            }
+            if (valid) {
+              const int64_t o = row + t0 + seg * SEG;
+              IO::store(static_cast<T *>(f.du) + o, du_o);
+              IO::store(static_cast<T *>(f.ddelta) + o, dd_o);
+              if (has_z) IO::store(static_cast<T *>(f.dz) + o, dz_o);
             }
           }
-        }
-
-        // segments from the last: re-run into registers, then walk backwards
-        for (int seg = nseg - 1; seg >= 0; --seg) {
-          float uv[SEG], dv[SEG], zv[SEG], dyv[SEG];
-          load_u(seg, uv);
-          IO::load(sd, tid, seg, dv);
-          IO::load(sdy, tid, seg, dyv);
-          if (has_z) IO::load(sz, tid, seg, zv);
-          float du_o[SEG], dd_o[SEG], dz_o[SEG];
-          const float *sp = sub + (seg * NM) * kSThreads + tid;
-
-          if constexpr (kS) {
-            // states before each step of the segment (the state after a step
-            // is recomputed in the reverse step from h_{t-1} and t1)
-            f2 Hs[SEG][NP];
+        };
+        if constexpr (kS) {
+          if (tile_gen) {
+            // A step of this tile has Delta |A0| outside the range where the
+            // structured arithmetic keeps its relative accuracy (1e-5 .. 6):
+            // the tile runs the generic arithmetic (one exp per state, dA
+            // through psi'), whose dA has no cancellation at small Delta and
+            // whose Abar keeps its relative accuracy at large Delta.
 #pragma unroll
-            for (int i = 0; i < NP; ++i)
-              Hs[0][i] = pk(sp[(2 * i) * kSThreads], sp[(2 * i + 1) * kSThreads]);
-#pragma unroll
-            for (int i = 0; i + 1 < SEG; ++i) {
-              const float *Brow = Bs + (seg * SEG + i) * BSTR;
-              f2 P[NP];
-              float Delta, sv;
-              step_decay(dv[i] + bias, P, Delta, sv);
-#pragma unroll
-              for (int j = 0; j < NP; ++j) Hs[i + 1][j] = Hs[i][j];
-              struct_update<NM>(Hs[i + 1], P, uv[i] * invA0, 0.f, Brow, Brow);
+            for (int n = 0; n < NM; ++n) {
+              gs[n] = (n & 1) ? hi_of(Gt[n >> 1]) : lo_of(Gt[n >> 1]);
+              accs[n] = 0.f;
+              A2[n] = Arow[n] * kLog2e;
+              invA[n] = Arow[n] != 0.f ? 1.f / Arow[n] : 0.f;
             }
+            tile_body(std::false_type{});
 #pragma unroll
-            for (int i = SEG - 1; i >= 0; --i) {
-              const int tl = seg * SEG + i;
-              const float *Brow = Bs + tl * BSTR;
-              const float *Crow = Cs + tl * BSTR;
-              f2 P[NP];
-              float Delta, sv;
-              step_decay(dv[i] + bias, P, Delta, sv);
-              float dy0 = dyv[i], sz = 0.f;
-              if (has_z) {
-                sz = rcpf(1.f + ex2f(-zv[i] * kLog2e));
-                dy0 *= zv[i] * sz;
-              }
-              const float up = uv[i] * invA0;
-              const float x1 = Delta * A0;
-              const f2 U = pk(up, up), DY = pk(dy0, dy0), X1n = pk(-x1, -x1), Z = pk(0.f, 0.f);
-              f2 DU = Z, DD = Z, Y0 = Z;
-              const bool up16 = (lane & 16) != 0;
-              float v16[16];
-#pragma unroll
-              for (int j = 0; j < NP; j += 2) {
-                const ulonglong2 bq = *reinterpret_cast<const ulonglong2 *>(Brow + 2 * j);
-                const ulonglong2 cq2 = *reinterpret_cast<const ulonglong2 *>(Crow + 2 * j);
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                  const int jj = j + e;
-                  const f2 Bp = e ? bq.y : bq.x;
-                  const f2 Cp = e ? cq2.y : cq2.x;
-                  const f2 CN = pk(float(2 * jj + 1), float(2 * jj + 2));
-                  const f2 Gv = fma2(Cp, DY, Gt[jj]);
-                  const f2 Ga = fma2(Gv, P[jj], Gv);
-                  const f2 w = fma2(Gv, P[jj], Z);
-                  const f2 t1 = fma2(Bp, U, Hs[i][jj]);
-                  const f2 hcur = fma2(P[jj], t1, Hs[i][jj]);  // h_t
-                  const f2 cq = fma2(fma2(Ga, t1, Z), CN, Z);
-                  DD = fma2(cq, pk(1.f, 1.f), DD);
-                  Acc[jj] = fma2(X1n, cq, Acc[jj]);
-                  const f2 dBc = fma2(w, U, Z);
-                  Acc[jj] = fma2(dBc, Bp, Acc[jj]);
-                  DU = fma2(w, Bp, DU);
-                  Y0 = fma2(Cp, hcur, Y0);
-                  const f2 dCc = fma2(DY, hcur, Z);
-                  Gt[jj] = Ga;
-                  // Channels past `dim` contribute exact zeros: TMA fills their
-                  // rows with 0, so dy0 = 0 and their adjoint stays 0.
-                  v16[2 * jj] = bfly_first(lo_of(dBc), lo_of(dCc), up16);
-                  v16[2 * jj + 1] = bfly_first(hi_of(dBc), hi_of(dCc), up16);
-                }
-              }
-#pragma unroll
-              for (int n = NM; n < kMaxN; ++n) v16[n] = 0.f;
-              const float du = fmaf(lo_of(DU) + hi_of(DU), invA0, Dd * dy0);
-              const float dd = A0 * (lo_of(DD) + hi_of(DD)) * sv;
-              const float y0 = (lo_of(Y0) + hi_of(Y0)) + Dd * uv[i];
-              du_o[i] = du;
-              dd_o[i] = dd;
-              dz_o[i] = has_z ? dyv[i] * y0 * sz * (1.f + zv[i] * (1.f - sz)) : 0.f;
-              dDsum = fmaf(dy0, uv[i], dDsum);
-              dbsum += dd;
-              const float rsum = bfly_rest(v16, lane);
-              // lane l holds dB (l < 16, to be divided by l+1) or dC of state l-16
-              red[(warp * kBTT + tl) * 33 + lane] = (lane < kMaxN) ? rsum * (1.f / float(lane + 1)) : rsum;
+            for (int i = 0; i < NP; ++i) {  // back to the structured units (Acc = -A_n dA_n)
+              Gt[i] = pk(gs[2 * i], gs[2 * i + 1]);
+              Acc[i] = fma2(pk(-Arow[2 * i], -Arow[2 * i + 1]), pk(accs[2 * i], accs[2 * i + 1]), Acc[i]);
             }
           } else {
-            float Hs[SEG][NM];
-#pragma unroll
-            for (int n = 0; n < NM; ++n) Hs[0][n] = sp[n * kSThreads];
-#pragma unroll
-            for (int i = 0; i + 1 < SEG; ++i) {
-              const float *Brow = Bs + (seg * SEG + i) * BSTR;
-              const float Delta = softplus_fast(dv[i] + bias);
-#pragma unroll
-              for (int n = 0; n < NM; ++n) Hs[i + 1][n] = Hs[i][n];
-              generic_update<NM>(Hs[i + 1], Delta, uv[i], 0.f, Arow, A2, invA, Brow, Brow);
-            }
-#pragma unroll
-            for (int i = SEG - 1; i >= 0; --i) {
-              const int tl = seg * SEG + i;
-              const float *Brow = Bs + tl * BSTR;
-              const float *Crow = Cs + tl * BSTR;
-              const float v = dv[i] + bias;
-              const float Delta = softplus_fast(v);
-              const float sv = rcpf(1.f + ex2f(-v * kLog2e));
-              float dy0 = dyv[i], sz = 0.f;
-              if (has_z) {
-                sz = rcpf(1.f + ex2f(-zv[i] * kLog2e));
-                dy0 *= zv[i] * sz;
-              }
-              float du_acc = 0.f, dD_acc = 0.f, y0 = Dd * uv[i];
-              const bool up16 = (lane & 16) != 0;
-              float v16[16];
-#pragma unroll
-              for (int n = 0; n < NM; ++n) {
-                const float x = Delta * Arow[n];
-                const float a = ex2f(Delta * A2[n]);
-                float pp = fmaf(x, 1.f / 720.f, 1.f / 120.f);
-                pp = fmaf(x, pp, 1.f / 24.f);
-                pp = fmaf(x, pp, 1.f / 6.f);
-                pp = fmaf(x, pp, 0.5f);
-                pp = fmaf(x, pp, 1.f);
-                const float Eb = fabsf(x) < 0.25f ? Delta * pp : (a - 1.f) * invA[n];  // Bbar / B
-                const float Bn = Brow[n], Cn = Crow[n];
-                const float hprev = Hs[i][n];
-                const float hcur = fmaf(a, hprev, Eb * (Bn * uv[i]));  // h_t, as in the forward
-                const float Gv = fmaf(Cn, dy0, gs[n]);
-                const float Ga = a * Gv;
-                const float wv = Gv * Eb;
-                du_acc = fmaf(wv, Bn, du_acc);
-                dD_acc = fmaf(Ga, fmaf(Bn, uv[i], Arow[n] * hprev), dD_acc);
-                accs[n] = fmaf(Gv, Delta * a * hprev + Bn * uv[i] * Delta * Delta * dpsi_fast(x, a), accs[n]);
-                y0 = fmaf(Cn, hcur, y0);
-                v16[n] = bfly_first(wv * uv[i], dy0 * hcur, up16);  // zero past `dim`
-                gs[n] = Ga;
-              }
-#pragma unroll
-              for (int n = NM; n < kMaxN; ++n) v16[n] = 0.f;
-              const float dd = dD_acc * sv;
-              du_o[i] = fmaf(Dd, dy0, du_acc);
-              dd_o[i] = dd;
-              dz_o[i] = has_z ? dyv[i] * y0 * sz * (1.f + zv[i] * (1.f - sz)) : 0.f;
-              dDsum = fmaf(dy0, uv[i], dDsum);
-              dbsum += dd;
-              red[(warp * kBTT + tl) * 33 + lane] = bfly_rest(v16, lane);
-            }
+            tile_body(std::true_type{});
           }
-          if (valid) {
-            const int64_t o = row + t0 + seg * SEG;
-            IO::store(static_cast<T *>(f.du) + o, du_o);
-            IO::store(static_cast<T *>(f.ddelta) + o, dd_o);
-            if (has_z) IO::store(static_cast<T *>(f.dz) + o, dz_o);
-          }
+        } else {
+          tile_body(std::false_type{});
         }
+        if (PROJ) tc_fence_before_sync();
         __syncthreads();
         // CTA sums of dB / dC for this tile -> partials
         for (int idx = tid; idx < 32 * kBTT; idx += kSThreads) {
@@ -730,6 +936,16 @@ __global__ void __launch_bounds__(kSThreads, 2)
     for (int t = ctile; t < p_issued; ++t)
       mbar_wait_bounded(&bars[t % kBStages], uint32_t(t / kBStages) & 1u, p.timeout_ns);
   }
+  if constexpr (PROJ) {  // every MMA issued must complete before TMEM is freed
+    if (tid == 0 && mma_issued >= 0)
+      mbar_wait_bounded(&mma_bar[mma_issued & 1], uint32_t(mma_issued >> 1) & 1u, p.timeout_ns);
+    tc_fence_before_sync();
+    __syncthreads();
+    if (tid < 32) {
+      tc_fence_after_sync();
+      tmem_dealloc(tbase, kProjTmemCols);
+    }
+  }
 }
 
 // Three-phase carry of the adjoint, used when there are too few channel groups
@@ -741,9 +957,10 @@ __global__ void __launch_bounds__(kSThreads, 2)
 // maps of the trishampatil.com walk-through, Part III section 2, run
 // backwards).  This kernel computes Ga_local and sum Delta of every chunk but
 // the first, one thread per (channel, chunk) walking the chunk from its end;
-// adjoint_carry_scan_kernel combines them, and the main reverse kernel then
-// runs every chunk from its true entering adjoint.
-template <typename T, int NM>
+// the parallel scan over chunks (chunk_scan_kernel, from the last chunk)
+// combines them, and the main reverse kernel then runs every chunk from its
+// true entering adjoint.
+template <typename T, int NM, typename TD = T>
 __global__ void __launch_bounds__(kSThreads) bwd_adjoint_agg_kernel(const BwdStagedArgs p) {
   constexpr int V = Vec<T>::kN;  // steps per 16-byte vector
   __shared__ float cs[NM * V];   // the C rows of the current V steps
@@ -755,7 +972,7 @@ __global__ void __launch_bounds__(kSThreads) bwd_adjoint_agg_kernel(const BwdSta
   const int64_t d = valid ? d_raw : f.dim - 1;  // loads stay in bounds
   const int N = f.N;
   const int64_t row = (int64_t(b) * f.dim + d) * f.L;
-  const T *dl = static_cast<const T *>(f.delta) + row;
+  const TD *dl = static_cast<const TD *>(f.delta) + row;
   const T *dy = static_cast<const T *>(f.dy) + row;
   const T *z = f.z ? static_cast<const T *>(f.z) + row : nullptr;
   const T *Cp = static_cast<const T *>(f.C) + int64_t(b) * N * f.L;
@@ -778,7 +995,17 @@ __global__ void __launch_bounds__(kSThreads) bwd_adjoint_agg_kernel(const BwdSta
   // steps is issued before it is used
   for (int64_t tb = tend - V; tb >= tbeg; tb -= V) {
     float dv[V], dyv[V], zv[V];
-    Vec<T>::unpack(*reinterpret_cast<const uint4 *>(dl + tb), dv);
+    if constexpr (std::is_same<TD, T>::value) {
+      Vec<T>::unpack(*reinterpret_cast<const uint4 *>(dl + tb), dv);
+    } else {  // fp32 delta beside bf16 tiles: V / 4 vectors of four
+#pragma unroll
+      for (int v4 = 0; v4 < V / 4; ++v4) {
+        float tmp[4];
+        Vec<float>::unpack(*reinterpret_cast<const uint4 *>(dl + tb + 4 * v4), tmp);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dv[4 * v4 + i] = tmp[i];
+      }
+    }
     Vec<T>::unpack(*reinterpret_cast<const uint4 *>(dy + tb), dyv);
     if (z) Vec<T>::unpack(*reinterpret_cast<const uint4 *>(z + tb), zv);
     __syncthreads();  // the previous steps' C rows are no longer read
@@ -817,26 +1044,6 @@ __global__ void __launch_bounds__(kSThreads) bwd_adjoint_agg_kernel(const BwdSta
   for (int n = 0; n < NM; ++n)
     p.agg_G[((int64_t(g) * p.K + k) * NM + n) * kSThreads + threadIdx.x] = valid ? Ga[n] : 0.f;
   p.agg_S[(int64_t(g) * p.K + k) * kSThreads + threadIdx.x] = valid ? S : 0.0;
-}
-
-// Ga_in(K-1) = 0, Ga_in(k-1) = exp(A_n S_k) Ga_in(k) + Ga_local(k), in fp64,
-// one thread per (group, state, channel).
-template <int NM>
-__global__ void adjoint_carry_scan_kernel(const BwdStagedArgs p) {
-  const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= int64_t(p.G) * NM * kSThreads) return;
-  const int c = int(idx % kSThreads);
-  const int n = int((idx / kSThreads) % NM);
-  const int g = int(idx / (int64_t(NM) * kSThreads));
-  const int d = (g % p.gpb) * kSThreads + c;
-  const double An = (d < p.w.dim && n < p.w.N) ? double(p.w.A[int64_t(d) * p.w.N + n]) : 0.0;
-  double G = 0.0;
-  for (int k = p.K - 1; k >= 0; --k) {
-    const int64_t base = int64_t(g) * p.K + k;
-    p.gin[(base * NM + n) * kSThreads + c] = float(G);
-    if (k > 0)
-      G = exp(An * p.agg_S[base * kSThreads + c]) * G + double(p.agg_G[(base * NM + n) * kSThreads + c]);
-  }
 }
 
 // dB / dC: sum of the per-CTA partials over the channel groups of a batch row.
@@ -897,7 +1104,24 @@ inline bool staged_bwd_supported(const BwdArgs &a, size_t es) {
          al(a.ddelta) && al(a.dz);
 }
 
-template <typename T, int NM, bool CONV = false>
+// Dynamic shared memory of the fused-projection backward (its stages hold the
+// Rp x 16 dt_low tile in place of delta's).
+template <typename T, int NM>
+inline int proj_bwd_smem_bytes(int Rp) {
+  using Lay = BwdLayout<T, NM>;
+  return int(kBStages * BwdStage<T, NM>(Rp).bytes) + (Lay::BYTES - Lay::OFF_SUB) + 512;
+}
+
+// Largest R the fused projection takes: its tiles must leave room for two
+// CTAs per SM in both the forward and the backward.
+template <typename T, int NM>
+inline int proj_max_rank() {
+  int r = 16;
+  while (r + 16 <= kProjMaxRp && proj_bwd_smem_bytes<T, NM>(r + 16) <= kTwoPerSmBytes) r += 16;
+  return r;
+}
+
+template <typename T, int NM, bool CONV = false, bool PROJ = false>
 mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStream_t s,
                                mamba_status_t (*launched)()) {
   using Lay = BwdLayout<T, NM>;
@@ -906,19 +1130,27 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
   const CUtensorMapSwizzle sw = bf16 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B;
   const CUtensorMapSwizzle none = CU_TENSOR_MAP_SWIZZLE_NONE;
   CUtensorMap maps[6];
-  if (!make_map_3d(&maps[0], a.u, bf16, L, dim, batch, kBTT, kSThreads, sw) ||
-      !make_map_3d(&maps[1], a.delta, bf16, L, dim, batch, kBTT, kSThreads, sw) ||
+  int Rp = 0, smem = Lay::ALLOC;
+  if (PROJ) {
+    Rp = (a.R + 15) / 16 * 16;
+    if (a.R < 1 || Rp > proj_max_rank<T, NM>()) return MAMBA_ERR_UNSUPPORTED;
+    smem = proj_bwd_smem_bytes<T, NM>(Rp);
+  }
+  const bool dmap = PROJ ? make_map_3d(&maps[1], a.dt_low, bf16, L, uint64_t(a.R), batch, kBTT,
+                                       uint32_t(Rp), sw)
+                         : make_map_3d(&maps[1], a.delta, bf16, L, dim, batch, kBTT, kSThreads, sw);
+  if (!make_map_3d(&maps[0], a.u, bf16, L, dim, batch, kBTT, kSThreads, sw) || !dmap ||
       !make_map_3d(&maps[2], a.z ? a.z : a.u, bf16, L, dim, batch, kBTT, kSThreads, sw) ||
       !make_map_3d(&maps[3], a.dy, bf16, L, dim, batch, kBTT, kSThreads, sw) ||
       !make_map_3d(&maps[4], a.B, bf16, L, N, batch, kBTT, uint32_t(N), none) ||
       !make_map_3d(&maps[5], a.C, bf16, L, N, batch, kBTT, uint32_t(N), none)) {
     return MAMBA_ERR_UNSUPPORTED;
   }
-  auto kern = bwd_staged_kernel<T, NM, CONV>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::ALLOC) != cudaSuccess)
+  auto kern = bwd_staged_kernel<T, NM, CONV, PROJ>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return MAMBA_ERR_CUDA;
   int bps = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, kern, kSThreads, Lay::ALLOC) != cudaSuccess)
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, kern, kSThreads, smem) != cudaSuccess)
     return MAMBA_ERR_CUDA;
   const int sms = device_sm_count();
   const int slots = sms * std::max(1, bps);
@@ -942,7 +1174,9 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
   const size_t gk = size_t(G) * size_t(pl.K);
   const size_t n_A = gk * NM * kSThreads, n_D = gk * kSThreads;
   const size_t n_par = par ? gk * NM * kSThreads : 0;  // agg_G and gin each
-  const size_t bytes = ceil_div(int_bytes + 4 * (n_ckpt + n_carry + n_bc + n_A + 2 * n_D) +
+  // the fused projection's three-phase carry: delta in fp32 for the aggregate pass
+  const size_t n_delta = (PROJ && par) ? size_t(a.batch) * size_t(a.dim) * size_t(a.L) : 0;
+  const size_t bytes = ceil_div(int_bytes + 4 * (n_ckpt + n_carry + n_bc + n_A + 2 * n_D + n_delta) +
                                     (par ? 8 * n_D + 8 * n_par : 0), 256) * 256;
   // The checkpoint pass (the forward without y) is prepared first so that one
   // workspace holds both: a failed allocation then leaves nothing enqueued.
@@ -951,11 +1185,12 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
   fa.bias = a.bias; fa.A = a.A; fa.D = nullptr; fa.y = nullptr; fa.last_state = nullptr;
   fa.batch = a.batch; fa.dim = a.dim; fa.L = a.L; fa.N = a.N;
   fa.conv_w = a.conv_w; fa.conv_b = a.conv_b; fa.conv_width = a.conv_width;
+  fa.dt_low = a.dt_low; fa.W_dt = a.W_dt; fa.R = a.R;
   StagedOptions fo = o;
   fo.chunk_len = 0;
   fo.carry = 0;
   fo.test_hook = 0;  // the hook targets the reverse hand-off
-  StagedForward<T, NM, CONV> ckpt_pass;
+  StagedForward<T, NM, CONV, PROJ> ckpt_pass;
   unsigned char *ws = nullptr;
   {
     // the checkpoint buffer is set once the workspace exists (before run)
@@ -986,11 +1221,15 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
   bp.gin = nullptr;
   bp.agg_G = nullptr;
   bp.agg_S = nullptr;
+  float *delta_f32 = nullptr;
   if (par) {
     bp.agg_S = reinterpret_cast<double *>(bp.part_bias + n_D);  // 8-byte aligned: offsets are
     bp.agg_G = reinterpret_cast<float *>(bp.agg_S + n_D);       // multiples of 128 floats
     bp.gin = bp.agg_G + n_par;
+    if (n_delta) delta_f32 = bp.gin + n_par;  // 16-byte aligned (multiples of 128 floats)
   }
+  bp.Rp = Rp;
+  bp.stage_bytes = PROJ ? BwdStage<T, NM>(Rp).bytes : 0;
   bp.timeout_ns = o.timeout_us > 0 ? uint64_t(o.timeout_us) * 1000ull : kDefaultTimeoutNs;
   bp.force_generic = o.path == MAMBA_PATH_GENERIC ? 1 : 0;
   bp.test_hook = o.test_hook;
@@ -999,19 +1238,35 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
   if (cudaMemsetAsync(ws, 0, int_bytes, s) != cudaSuccess) st = MAMBA_ERR_CUDA;
   if (st == MAMBA_OK) {
     ckpt_pass.sa.ckpt = ckpt;
+    ckpt_pass.sa.delta_out = delta_f32;
     st = ckpt_pass.run(ws + bytes, s, launched);
   }
   if (st == MAMBA_OK && par) {
-    bwd_adjoint_agg_kernel<T, NM><<<unsigned(size_t(G) * size_t(pl.K - 1)), kSThreads, 0, s>>>(bp);
+    if (delta_f32) {  // the aggregate pass reads the fp32 delta the checkpoint pass formed
+      BwdStagedArgs bq = bp;
+      bq.w.delta = delta_f32;
+      bwd_adjoint_agg_kernel<T, NM, float><<<unsigned(size_t(G) * size_t(pl.K - 1)), kSThreads, 0, s>>>(bq);
+    } else {
+      bwd_adjoint_agg_kernel<T, NM, T><<<unsigned(size_t(G) * size_t(pl.K - 1)), kSThreads, 0, s>>>(bp);
+    }
     st = launched();
-    if (st == MAMBA_OK) {
-      const int64_t threads = G * NM * kSThreads;
-      adjoint_carry_scan_kernel<NM><<<unsigned(ceil_div(threads, 256)), 256, 0, s>>>(bp);
+    if (st == MAMBA_OK) {  // Ga_in(K-1) = 0, Ga_in(k-1) = exp(A_n S_k) Ga_in(k) + Ga_local(k)
+      ChunkScanIO io;
+      io.S = bp.agg_S;
+      io.hl = bp.agg_G;
+      io.hin = bp.gin;
+      io.A = a.A;
+      io.G = int(G);
+      io.K = pl.K;
+      io.gpb = int(gpb);
+      io.N = a.N;
+      io.dim = a.dim;
+      chunk_scan_kernel<NM, true><<<unsigned(G * NM * kSThreads), 128, 0, s>>>(io);
       st = launched();
     }
   }
   if (st == MAMBA_OK) {
-    kern<<<unsigned(std::min<int64_t>(gk, slots)), kSThreads, Lay::ALLOC, s>>>(
+    kern<<<unsigned(std::min<int64_t>(gk, slots)), kSThreads, smem, s>>>(
         maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], bp);
     st = launched();
   }

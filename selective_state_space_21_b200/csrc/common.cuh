@@ -29,6 +29,10 @@ struct FwdArgs {
   int N;
   const float *conv_w = nullptr, *conv_b = nullptr;
   int conv_width = 0;
+  // With W_dt set (the fused low-rank Delta projection), delta is not read:
+  // delta[b,d,t] = sum_r W_dt[d,r] dt_low[b,r,t] is formed on the tensor cores.
+  const void *dt_low = nullptr, *W_dt = nullptr;
+  int R = 0;
 };
 
 // With conv_w set, `u` is x as in FwdArgs and `du` receives the gradient with
@@ -42,6 +46,9 @@ struct BwdArgs {
   int N;
   const float *conv_w = nullptr, *conv_b = nullptr;
   int conv_width = 0;
+  // fused low-rank Delta projection, as in FwdArgs (delta is not read)
+  const void *dt_low = nullptr, *W_dt = nullptr;
+  int R = 0;
 };
 
 // The short causal depthwise convolution in front of the S6 layer (Knowl 3

@@ -48,6 +48,7 @@
 
 #include "../../include/mamba_scan.h"
 #include "common.cuh"
+#include "tcgen05.cuh"
 #include "tma.cuh"
 
 namespace mscan {
@@ -63,7 +64,12 @@ constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
 // SEQ / PAR: the forward with y.  AGG: chunk aggregates for PAR.  CKPT_SEQ /
 // CKPT_PAR: the forward without y that stores the state every kCkptEvery
 // steps (the checkpoints the backward recomputes from).
-enum StagedKind { KIND_SEQ = 0, KIND_PAR = 1, KIND_AGG = 2, KIND_CKPT_SEQ = 3, KIND_CKPT_PAR = 4 };
+// LOC: the forward with y of every chunk from a zero entering state, which
+// also stores each chunk's end state and sum of Delta; the closed-form
+// correction (fwd_correct_kernel) then adds the entering state's
+// contribution once the scan over chunks has produced it.
+enum StagedKind { KIND_SEQ = 0, KIND_PAR = 1, KIND_AGG = 2, KIND_CKPT_SEQ = 3, KIND_CKPT_PAR = 4,
+                  KIND_LOC = 5 };
 constexpr int kCkptEvery = 16;
 enum UnitMode { MODE_SIG = 0, MODE_STRUCT = 1, MODE_GEN = 2 };
 
@@ -84,6 +90,32 @@ struct StagedArgs {
   uint64_t timeout_ns;
   int test_hook;   // 1: unit (group 0, chunk 0) never publishes (tests the bounded wait)
   int force_generic;  // 1: generic arithmetic for every channel
+  // fused Delta projection (PROJ kernels): R padded to a multiple of 16, the
+  // bytes of one pipeline stage and the number of stages; delta_out, when
+  // set, receives delta in fp32 (batch, dim, L) for kernels that read it later
+  int Rp = 0;
+  uint32_t stage_bytes = 0;
+  int nst = 0;
+  float *delta_out = nullptr;
+};
+
+// Fused Delta projection: TMEM columns of one CTA (W rows in [0, Rp/2), two
+// fp32 accumulators of one tile each after kProjAcc).
+constexpr int kProjMaxRp = 256;
+constexpr uint32_t kProjAcc = kProjMaxRp / 2;
+constexpr uint32_t kProjTmemCols = 256;
+
+// Shared-memory offsets of the fused-projection forward: a stage holds u,
+// the dt_low tile (Rp rows), z, B and C.
+struct ProjStage {
+  uint32_t dt, z, B, C, bytes;
+  __host__ __device__ ProjStage(int Rp) {
+    dt = kTileBytes;
+    z = dt + uint32_t(Rp) * kRowBytes;
+    B = z + kTileBytes;
+    C = B + kRawBytes;
+    bytes = (C + kRawBytes + 1023u) & ~1023u;
+  }
 };
 
 // ------------------------------------------------------------------ math
@@ -195,8 +227,9 @@ __device__ __forceinline__ float struct_update(f2 (&H)[NM / 2], const f2 (&P)[NM
 }
 
 // One generic step for one channel (any A): per state, Abar = exp(Delta A_n)
-// and Bbar/B = Delta psi(Delta A_n) with psi(x) = expm1(x)/x.
-template <int NM>
+// and Bbar/B = Delta psi(Delta A_n) with psi(x) = expm1(x)/x.  SCALED_B: the
+// B row holds B_n / (n + 1) (the structured arithmetic's table).
+template <int NM, bool SCALED_B = false>
 __device__ __forceinline__ float generic_update(float (&h)[NM], float Delta, float uv, float yinit,
                                                 const float (&A)[NM], const float (&A2)[NM],
                                                 const float (&invA)[NM], const float *Brow,
@@ -212,7 +245,8 @@ __device__ __forceinline__ float generic_update(float (&h)[NM], float Delta, flo
     p = fmaf(x, p, 0.5f);
     p = fmaf(x, p, 1.f);
     const float E = fabsf(x) < 0.25f ? Delta * p : (a - 1.f) * invA[n];
-    h[n] = fmaf(a, h[n], E * (Brow[n] * uv));
+    const float Bn = SCALED_B ? Brow[n] * float(n + 1) : Brow[n];
+    h[n] = fmaf(a, h[n], E * (Bn * uv));
     y = fmaf(Crow[n], h[n], y);
   }
   return y;
@@ -274,7 +308,7 @@ struct StagedLayout {
   static constexpr int OFF_BS = OFF_Y + 2 * kTileBytes;
   static constexpr int OFF_CS = OFF_BS + 2 * TT * BSTR * 4;   // B' and C: two buffers each
   static constexpr int OFF_BAR = OFF_CS + 2 * TT * BSTR * 4;
-  static constexpr int OFF_Q = OFF_BAR + 8 * kStages;
+  static constexpr int OFF_Q = OFF_BAR + 8 * 5;  // stage barriers (3) + MMA barriers (2)
   static constexpr int BYTES = OFF_Q + 16 * 4;
   static constexpr int ALLOC = BYTES + 1024;  // slack to align the base to 1 KB
 };
@@ -283,7 +317,15 @@ struct StagedLayout {
 // convolution, and each thread turns its row into u = SiLU(conv(x)) as it
 // reads it (the three inputs before the unit's first step come from global
 // memory; after that the last three stay in registers).
-template <typename T, int NM, int KIND, bool CONV = false>
+//
+// PROJ: delta is not read.  The tiles of the low-rank projection's input
+// dt_low (Rp x TT, bf16) come through the pipeline instead, the CTA's 128 rows
+// of W_dt sit in tensor memory, and one elected thread issues per tile the
+// tcgen05 MMA delta_tile (128 channels x TT steps, fp32 in TMEM) = W_g (128 x
+// Rp) . dt_low_tile (Rp x TT); each thread then reads its own channel's TT
+// values of delta with tcgen05.ld.  The MMA of the next tile is issued while
+// the current one is scanned, into the other of two accumulators.
+template <typename T, int NM, int KIND, bool CONV = false, bool PROJ = false>
 __global__ void __launch_bounds__(kSThreads, 2)
     fwd_staged_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_d,
                       const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_y,
@@ -291,7 +333,10 @@ __global__ void __launch_bounds__(kSThreads, 2)
                       const StagedArgs p) {
   using Lay = StagedLayout<T, NM>;
   constexpr int TT = Lay::TT, VEC = Lay::VEC, NV = Lay::NV, BSTR = Lay::BSTR;
-  constexpr bool kOut = KIND == KIND_SEQ || KIND == KIND_PAR;  // computes and stores y
+  static_assert(!PROJ || (std::is_same<T, __nv_bfloat16>::value && !CONV),
+                "the fused projection takes bf16 operands and no convolution prologue");
+  constexpr bool kOut = KIND == KIND_SEQ || KIND == KIND_PAR || KIND == KIND_LOC;  // stores y
+  constexpr bool kAgg = KIND == KIND_AGG || KIND == KIND_LOC;  // stores chunk aggregates
   constexpr bool kSeq = KIND == KIND_SEQ || KIND == KIND_CKPT_SEQ;
   constexpr bool kPar = KIND == KIND_PAR || KIND == KIND_CKPT_PAR;
   constexpr bool kCkpt = KIND == KIND_CKPT_SEQ || KIND == KIND_CKPT_PAR;
@@ -301,21 +346,43 @@ __global__ void __launch_bounds__(kSThreads, 2)
   // shared-memory loads and stores instead of generic ones.
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sm + Lay::OFF_BAR);
-  int *q = reinterpret_cast<int *>(sm + Lay::OFF_Q);  // [0..7] ticket ring, [8] abort
-  float *Bs = reinterpret_cast<float *>(sm + Lay::OFF_BS);
-  float *Cs = reinterpret_cast<float *>(sm + Lay::OFF_CS);
+  // stage geometry: fixed, or (PROJ) set by the dt_low tile's rows
+  const ProjStage ps(PROJ ? p.Rp : 0);
+  const uint32_t SST = PROJ ? ps.bytes : uint32_t(kStageBytes);
+  const int NST = PROJ ? p.nst : kStages;
+  const uint32_t OFF_Z = PROJ ? ps.z : 2u * kTileBytes;
+  const uint32_t OFF_B = PROJ ? ps.B : 3u * kTileBytes;
+  const uint32_t OFF_C = PROJ ? ps.C : 3u * kTileBytes + kRawBytes;
+  const uint32_t OFF_Y = uint32_t(NST) * SST;
+  const uint32_t OFF_BS = OFF_Y + 2 * kTileBytes;
+  const uint32_t OFF_CS = OFF_BS + 2 * TT * BSTR * 4;
+  const uint32_t OFF_BAR = OFF_CS + 2 * TT * BSTR * 4;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);  // [stages], then 2 MMA barriers
+  uint64_t *mma_bar = bars + 3;
+  int *q = reinterpret_cast<int *>(sm + OFF_BAR + 8 * 5);  // [0..7] ticket ring, [8] abort, [12] TMEM
+  float *Bs = reinterpret_cast<float *>(sm + OFF_BS);
+  float *Cs = reinterpret_cast<float *>(sm + OFF_CS);
 
   const int tid = threadIdx.x;
   const FwdArgs &f = p.f;
   const int N = f.N;
   const bool has_z = kOut && f.z != nullptr;
-  const uint32_t tile_bytes = (kOut ? (has_z ? 3u : 2u) : 2u) * kTileBytes +
+  const uint32_t tile_bytes = (kOut ? (has_z ? 2u : 1u) : 1u) * kTileBytes +
+                              (PROJ ? uint32_t(p.Rp) * kRowBytes : kTileBytes) +
                               (kOut ? 2u : 1u) * uint32_t(N) * kRowBytes;
+  // fused projection: the MMA's instruction descriptor (M = 128 channels,
+  // N = TT steps; A = W from TMEM, K-major; B = dt_low, MN-major) and TMEM
+  [[maybe_unused]] constexpr uint32_t kIdesc = mma_idesc_bf16(128, TT, false, true);
+  [[maybe_unused]] uint32_t tbase = 0;
+  [[maybe_unused]] int mma_issued = -1;  // thread 0: last tile whose MMA it issued
 
   if (tid == 0) {
 #pragma unroll
     for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
+    if (PROJ) {
+      mbar_init(&mma_bar[0], 1);
+      mbar_init(&mma_bar[1], 1);
+    }
     fence_barrier_init();
     prefetch_tensormap(&tm_u);
     prefetch_tensormap(&tm_d);
@@ -327,7 +394,38 @@ __global__ void __launch_bounds__(kSThreads, 2)
     }
     q[8] = 0;
   }
+  if constexpr (PROJ) {
+    if (tid < 32) {
+      tmem_alloc(reinterpret_cast<uint32_t *>(&q[12]), kProjTmemCols);
+      tmem_relinquish();
+    }
+  }
   __syncthreads();
+  if constexpr (PROJ) {
+    tc_fence_after_sync();
+    tbase = uint32_t(q[12]);
+  }
+
+  // Issues (thread 0) the projection MMAs of consumed-tile index `ct` into
+  // accumulator ct & 1, once the tile's dt_low rows have landed.
+  [[maybe_unused]] auto issue_mma = [&](int ct) {
+    const int stg = ct % NST;
+    if (!mbar_wait_bounded(&bars[stg], uint32_t(ct / NST) & 1u, p.timeout_ns)) {
+      record_timeout();
+      q[8] = 1;
+      return;
+    }
+    tc_fence_after_sync();
+    const uint32_t dt_addr = smem_u32(sm + stg * SST + ps.dt);
+    const uint32_t acc = tbase + kProjAcc + uint32_t(ct & 1) * TT;
+    for (int kk = 0; kk < p.Rp / 16; ++kk) {
+      // 16 rows of dt_low (two 8-row swizzle atoms of 512 bytes) per MMA
+      const uint64_t bdesc = smem_desc(dt_addr + uint32_t(kk) * 1024u, 16u, 512u, 4u);
+      mma_ts(acc, tbase + uint32_t(kk) * 8u, bdesc, kIdesc, kk > 0);
+    }
+    mma_commit(&mma_bar[ct & 1]);
+    mma_issued = ct;
+  };
 
   // ---- producer state (meaningful in thread 0 only)
   int p_ticket = 0, p_tile = 0, p_ntiles = 0, p_tail = 0, p_issued = 0;
@@ -361,15 +459,16 @@ __global__ void __launch_bounds__(kSThreads, 2)
     const int g = p_ticket % p.G, k = p_ticket / p.G;
     const int b = g / p.gpb, d0 = (g % p.gpb) * kSThreads;
     const int t0 = k * p.chunk_len + p_tile * TT;
-    const int stage = p_issued % kStages;
-    unsigned char *st = sm + stage * kStageBytes;
+    const int stage = p_issued % NST;
+    unsigned char *st = sm + stage * SST;
     uint64_t *bar = &bars[stage];
     mbar_arrive_expect_tx(bar, tile_bytes);
     tma_load_3d(st, &tm_u, bar, t0, d0, b);
-    tma_load_3d(st + kTileBytes, &tm_d, bar, t0, d0, b);
-    if (has_z) tma_load_3d(st + 2 * kTileBytes, &tm_z, bar, t0, d0, b);
-    tma_load_3d(st + 3 * kTileBytes, &tm_B, bar, t0, 0, b);
-    if (kOut) tma_load_3d(st + 3 * kTileBytes + kRawBytes, &tm_C, bar, t0, 0, b);
+    if (PROJ) tma_load_3d(st + kTileBytes, &tm_d, bar, t0, 0, b);  // dt_low rows 0..Rp-1
+    else tma_load_3d(st + kTileBytes, &tm_d, bar, t0, d0, b);
+    if (has_z) tma_load_3d(st + OFF_Z, &tm_z, bar, t0, d0, b);
+    tma_load_3d(st + OFF_B, &tm_B, bar, t0, 0, b);
+    if (kOut) tma_load_3d(st + OFF_C, &tm_C, bar, t0, 0, b);
     ++p_tile;
     ++p_issued;
   };
@@ -377,7 +476,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
   constexpr bool kLookahead = !kSeq;
   if (tid == 0) {
     produce(true);
-    for (int s = 1; s < kStages; ++s) produce(kLookahead);
+    for (int s = 1; s < NST; ++s) produce(kLookahead);
   }
 
   int head = 0;   // consumer position in the ticket ring
@@ -413,6 +512,29 @@ __global__ void __launch_bounds__(kSThreads, 2)
 #pragma unroll
     for (int n = 1; n < NM; ++n) structured = structured && (Arow[n] == float(n + 1) * Arow[0]);
     const bool sig = structured && Arow[0] == -1.f;
+    if constexpr (PROJ) {
+      // This group's rows of W_dt into TMEM columns [0, Rp/2), bf16 pairs
+      // (even k in the low half).  The previous unit's MMAs have completed:
+      // its threads waited for every one of them.
+      const __nv_bfloat16 *wrow = static_cast<const __nv_bfloat16 *>(f.W_dt) +
+                                  (valid ? int64_t(d) * f.R : 0);
+      const int warp = tid >> 5;
+      for (int c8 = 0; c8 < p.Rp / 16; ++c8) {
+        uint32_t r[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int k = 16 * c8 + 2 * i;
+          const uint32_t lo = (valid && k < f.R) ? __bfloat16_as_ushort(wrow[k]) : 0u;
+          const uint32_t hi = (valid && k + 1 < f.R) ? __bfloat16_as_ushort(wrow[k + 1]) : 0u;
+          r[i] = lo | (hi << 16);
+        }
+        tmem_st8(tmem_at(tbase, uint32_t(warp) * 32u, uint32_t(c8) * 8u), r);
+      }
+      tmem_st_wait();
+      tc_fence_before_sync();
+      __syncthreads();
+      if (tid == 0) issue_mma(ctile);
+    }
     int mode = MODE_GEN;
     if (!p.force_generic) {
       if (__syncthreads_and(sig)) mode = MODE_SIG;
@@ -484,14 +606,14 @@ __global__ void __launch_bounds__(kSThreads, 2)
       // the next tile's are written at the end of the current one, under the
       // same barrier as the y tile.
       auto stage_tables = [&](int ct) {
-        const int stg = ct % kStages;
-        if (!mbar_wait_bounded(&bars[stg], uint32_t(ct / kStages) & 1u, p.timeout_ns)) {
+        const int stg = ct % NST;
+        if (!mbar_wait_bounded(&bars[stg], uint32_t(ct / NST) & 1u, p.timeout_ns)) {
           record_timeout();
           q[8] = 1;
         }
-        const unsigned char *sst = sm + stg * kStageBytes;
-        const T *Braw = reinterpret_cast<const T *>(sst + 3 * kTileBytes);
-        const T *Craw = reinterpret_cast<const T *>(sst + 3 * kTileBytes + kRawBytes);
+        const unsigned char *sst = sm + stg * SST;
+        const T *Braw = reinterpret_cast<const T *>(sst + OFF_B);
+        const T *Craw = reinterpret_cast<const T *>(sst + OFF_C);
         float *Bd = Bs + (ct & 1) * TT * BSTR;
         float *Cd = Cs + (ct & 1) * TT * BSTR;
         constexpr int ITEMS = NM * (TT / 4);
@@ -511,15 +633,24 @@ __global__ void __launch_bounds__(kSThreads, 2)
       if (q[8]) return;
 
       for (int it = 0; it < ntiles; ++it, ++ctile) {
-        const int stage = ctile % kStages;
-        unsigned char *st = sm + stage * kStageBytes;
+        const int stage = ctile % NST;
+        unsigned char *st = sm + stage * SST;
         const float *Bt = Bs + (ctile & 1) * TT * BSTR;
         const float *Ct = Cs + (ctile & 1) * TT * BSTR;
         const int64_t t0 = tbeg + int64_t(it) * TT;
         const unsigned char *su = st;
-        const unsigned char *sd = st + kTileBytes;
-        const unsigned char *sz = st + 2 * kTileBytes;
-        unsigned char *sy = sm + Lay::OFF_Y + (ctile & 1) * kTileBytes;
+        [[maybe_unused]] const unsigned char *sd = st + kTileBytes;
+        const unsigned char *sz = st + OFF_Z;
+        unsigned char *sy = sm + OFF_Y + (ctile & 1) * kTileBytes;
+        [[maybe_unused]] uint32_t dacc = 0;
+        if constexpr (PROJ) {  // this tile's delta: wait for its MMA
+          if (!mbar_wait_bounded(&mma_bar[ctile & 1], uint32_t(ctile >> 1) & 1u, p.timeout_ns)) {
+            record_timeout();
+            q[8] = 1;
+          }
+          tc_fence_after_sync();
+          dacc = tmem_at(tbase + kProjAcc + uint32_t(ctile & 1) * TT, uint32_t(tid >> 5) * 32u, 0);
+        }
         for (int j = 0; j < NV; ++j) {
           if (t0 + int64_t(j) * VEC >= tend) break;  // past the end of the sequence
           if constexpr (kCkpt) {
@@ -553,7 +684,21 @@ __global__ void __launch_bounds__(kSThreads, 2)
               xm1 = xv;
             }
           }
-          Vec<T>::unpack(*reinterpret_cast<const uint4 *>(sd + off), dv);
+          if constexpr (PROJ) {
+            static_assert(VEC == 8, "eight steps per 16-byte chunk");
+            tmem_ld8(dacc + uint32_t(j) * 8u, dv);
+            tmem_ld_wait();
+            if (p.delta_out && valid) {
+              float *o = p.delta_out + (int64_t(b) * f.dim + d) * f.L + t0 + int64_t(j) * VEC;
+              *reinterpret_cast<float4 *>(o) = make_float4(dv[0], dv[1], dv[2], dv[3]);
+              *reinterpret_cast<float4 *>(o + 4) = make_float4(dv[4], dv[5], dv[6], dv[7]);
+            }
+            // the next tile's MMA, into the other accumulator, half-way through this one
+            if (tid == 0 && j == 1 && it + 1 < ntiles) issue_mma(ctile + 1);
+            __syncwarp();
+          } else {
+            Vec<T>::unpack(*reinterpret_cast<const uint4 *>(sd + off), dv);
+          }
           if (has_z) Vec<T>::unpack(*reinterpret_cast<const uint4 *>(sz + off), zv);
 #pragma unroll
           for (int i = 0; i < VEC; ++i) {
@@ -563,7 +708,9 @@ __global__ void __launch_bounds__(kSThreads, 2)
             const float v = dv[i] + bias;
             float y0;
             if constexpr (M == MODE_SIG) {
-              const float vc = fminf(fmaxf(v, -80.f), 80.f);
+              // e^-v overflows below v = -88; above +88 it flushes to 0 and
+              // the decays are exactly 0 (sigma = 1), as they should be
+              const float vc = fmaxf(v, -87.f);
               const float ev = ex2f(-vc * kLog2e);  // e^-v
               const float s = rcpf(1.f + ev);      // sigma(v) = 1 - exp(-Delta)
               f2 P[NM / 2];
@@ -572,8 +719,8 @@ __global__ void __launch_bounds__(kSThreads, 2)
                 y0 = struct_update<NM>(H, P, -uv[i], Dd * uv[i], Brow, Crow);
               } else {
                 struct_update<NM>(H, P, -uv[i], 0.f, Brow, Brow);
-                if constexpr (KIND == KIND_AGG) Ssum += double(softplus_fast(v));
               }
+              if constexpr (kAgg) Ssum += double(softplus_fast(v));
             } else if constexpr (M == MODE_STRUCT) {
               const float Delta = softplus_fast(v);
               const float E1 = expm1_neg(Delta * A0);
@@ -583,13 +730,13 @@ __global__ void __launch_bounds__(kSThreads, 2)
                 y0 = struct_update<NM>(H, P, uv[i] * invA0, Dd * uv[i], Brow, Crow);
               } else {
                 struct_update<NM>(H, P, uv[i] * invA0, 0.f, Brow, Brow);
-                if constexpr (KIND == KIND_AGG) Ssum += double(Delta);
               }
+              if constexpr (kAgg) Ssum += double(Delta);
             } else {
               const float Delta = softplus_fast(v);
               y0 = generic_update<NM>(h, Delta, uv[i], Dd * uv[i], Arow, A2, invA, Brow,
                                       kOut ? Crow : Brow);
-              if constexpr (KIND == KIND_AGG) Ssum += double(Delta);
+              if constexpr (kAgg) Ssum += double(Delta);
             }
             if (kOut) {
               if (has_z) {
@@ -603,6 +750,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
         }
         if (it + 1 < ntiles) stage_tables(ctile + 1);
         if (kOut) fence_proxy_async_smem();
+        if (PROJ) tc_fence_before_sync();
         __syncthreads();
         if (q[8]) return;
         if (tid == 0) {
@@ -635,7 +783,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
     }
 
     // hand the end state on
-    if (KIND == KIND_AGG) {
+    if (kAgg) {
 #pragma unroll
       for (int n = 0; n < NM; ++n)
         p.agg_h[((int64_t(g) * p.K + k) * NM + n) * kSThreads + tid] = hs[n];
@@ -655,38 +803,191 @@ __global__ void __launch_bounds__(kSThreads, 2)
     }
     if (!kLookahead && tid == 0) {  // claim the next unit and fill the free stages
       produce(true);
-      while (!p_done && p_issued < ctile + kStages && p_tile < p_ntiles) produce(false);
+      while (!p_done && p_issued < ctile + NST && p_tile < p_ntiles) produce(false);
     }
   }
 
-  // Drain: every TMA load this CTA issued must land before it exits.
+  // Drain: every TMA load this CTA issued must land before it exits, and
+  // (PROJ) every MMA it issued must complete before TMEM is freed.
   __syncthreads();
   if (tid == 0) {
     if (aborted) {
       for (int t = ctile; t < p_issued; ++t)
-        mbar_wait_bounded(&bars[t % kStages], uint32_t(t / kStages) & 1u, p.timeout_ns);
+        mbar_wait_bounded(&bars[t % NST], uint32_t(t / NST) & 1u, p.timeout_ns);
     }
+    if (PROJ && mma_issued >= 0)
+      mbar_wait_bounded(&mma_bar[mma_issued & 1], uint32_t(mma_issued >> 1) & 1u, p.timeout_ns);
     bulk_wait<0>();
+  }
+  if constexpr (PROJ) {
+    tc_fence_before_sync();
+    __syncthreads();
+    if (tid < 32) {
+      tc_fence_after_sync();
+      tmem_dealloc(tbase, kProjTmemCols);
+    }
   }
 }
 
-// Carry scan over chunks (PAR): h_in(0) = 0,
-// h_in(k+1) = exp(A_n S_k) h_in(k) + h_loc(k), one thread per (group, n, channel).
-template <int NM>
-__global__ void carry_scan_kernel(const StagedArgs p) {
-  const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t total = int64_t(p.G) * NM * kSThreads;
-  if (idx >= total) return;
-  const int c = int(idx % kSThreads);
-  const int n = int((idx / kSThreads) % NM);
-  const int g = int(idx / (int64_t(NM) * kSThreads));
+// The scan over chunks of the three-phase carry, as a parallel scan of the
+// associative operator of affine maps ("Mamba: Linear-Time Sequence Modeling
+// with Selective State Spaces", trishampatil.com walk-through, Part III
+// section 2, "Parallel scan: why a recurrence isn't as sequential as it
+// looks"; the chunking of section 3.3 of the paper-graph-ui summary).  Chunk
+// k maps an entering state h to exp(A_n S_k) h + hl_k (S_k its sum of Delta,
+// hl_k the state it produces from zero); two chunks compose as
+//     (S_a, hl_a) then (S_b, hl_b)  =  (S_a + S_b, exp(A_n S_b) hl_a + hl_b).
+// One CTA of 128 threads per (channel group, state, channel) walks the K
+// chunks in blocks of 128: a Kogge-Stone scan within each warp by shuffles,
+// the four warp totals combined through shared memory, and the state carried
+// from block to block; the chunk-entering states go back to HBM.  Element k
+// of the scan is chunk k (forward) or chunk K-1-k (REVERSE: the adjoint of
+// the backward runs from the end).  fp64 throughout.
+struct ChunkScanIO {
+  const double *S;   // [G][K][128] sum of Delta per chunk
+  const float *hl;   // [G][K][NM][128] value each chunk produces from zero
+  float *hin;        // [G][K][NM][128] value entering each chunk
+  const float *A;    // (dim, N)
+  int G, K, gpb, N;
+  int64_t dim;
+};
+
+template <int NM, bool REVERSE>
+__global__ void __launch_bounds__(128) chunk_scan_kernel(const ChunkScanIO io) {
+  __shared__ double wS[4], wh[4];
+  __shared__ double carry;
+  const int seq = blockIdx.x;  // (g * NM + n) * 128 + c
+  const int c = seq % kSThreads, n = (seq / kSThreads) % NM, g = seq / (kSThreads * NM);
+  const int d = (g % io.gpb) * kSThreads + c;
+  const double An = (d < io.dim && n < io.N) ? double(io.A[int64_t(d) * io.N + n]) : 0.0;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) carry = 0.0;
+  __syncthreads();
+  for (int k0 = 0; k0 < io.K; k0 += 128) {
+    const int e = k0 + threadIdx.x;  // element of the scan
+    const int k = REVERSE ? io.K - 1 - e : e;
+    const bool live = e < io.K - 1;  // the last element's map is never applied
+    const int64_t base = int64_t(g) * io.K + (live ? k : 0);
+    double S = live ? io.S[base * kSThreads + c] : 0.0;
+    double h = live ? double(io.hl[(base * NM + n) * kSThreads + c]) : 0.0;
+    // inclusive scan within the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const double So = __shfl_up_sync(0xffffffffu, S, o);
+      const double ho = __shfl_up_sync(0xffffffffu, h, o);
+      if (lane >= o) {
+        h = exp(An * S) * ho + h;
+        S = So + S;
+      }
+    }
+    if (lane == 31) {
+      wS[warp] = S;
+      wh[warp] = h;
+    }
+    __syncthreads();
+    // what enters this warp's first element: the carry through the earlier warps
+    double cin = carry;
+    for (int w = 0; w < warp; ++w) cin = exp(An * wS[w]) * cin + wh[w];
+    // exclusive prefix within the warp, applied to that
+    double Se = __shfl_up_sync(0xffffffffu, S, 1);
+    double he = __shfl_up_sync(0xffffffffu, h, 1);
+    if (lane == 0) {
+      Se = 0.0;
+      he = 0.0;
+    }
+    if (e < io.K) io.hin[((int64_t(g) * io.K + k) * NM + n) * kSThreads + c] = float(exp(An * Se) * cin + he);
+    __syncthreads();
+    if (threadIdx.x == 127) carry = exp(An * S) * cin + h;  // through the whole block
+    __syncthreads();
+  }
+}
+
+// Closed-form correction after the LOC pass (one CTA per channel group and
+// chunk k >= 1, one thread per channel).  A chunk run from a zero entering
+// state misses the contribution of its true entering state h_in: with
+// cumDelta_t the sum of Delta over the chunk up to step t, the state the
+// chunk really has is h_t + exp(A_n cumDelta_t) h_in,n (the homogeneous
+// solution of the recurrence, Abar multiplying it step by step), so
+//     y_t += silu(z_t) sum_n C_tn exp(A_n cumDelta_t) h_in,n
+// and the last chunk's final state gains exp(A_n S) h_in,n.  For the
+// structured A (A_n = (n+1) A_0 < 0) the sum is a polynomial in
+// q_t = exp(A_0 cumDelta_t), evaluated by Horner's rule; otherwise one exp per
+// state.  A thread stops once every decay has fallen below 2^-32 (the terms
+// left are below fp32 resolution of the state they correct).
+template <typename T, int NM>
+__global__ void __launch_bounds__(kSThreads) fwd_correct_kernel(const StagedArgs p) {
+  constexpr int V = 16 / int(sizeof(T));  // steps per 16-byte vector
+  const FwdArgs &f = p.f;
+  const int unit = blockIdx.x;  // (chunk - 1) * G + group
+  const int g = unit % p.G, k = 1 + unit / p.G;
+  const int b = g / p.gpb, c = threadIdx.x;
   const int d = (g % p.gpb) * kSThreads + c;
-  const double An = (d < p.f.dim && n < p.f.N) ? double(p.f.A[int64_t(d) * p.f.N + n]) : 0.0;
-  double h = 0.0;
-  for (int k = 0; k < p.K; ++k) {
-    const int64_t base = (int64_t(g) * p.K + k);
-    p.hin[(base * NM + n) * kSThreads + c] = float(h);
-    if (k < p.K - 1) h = exp(An * p.agg_S[base * kSThreads + c]) * h + double(p.agg_h[(base * NM + n) * kSThreads + c]);
+  if (d >= f.dim) return;
+  const int N = f.N;
+  float hin[NM], An[NM];
+  bool any = false;
+#pragma unroll
+  for (int n = 0; n < NM; ++n) {
+    hin[n] = __ldcg(p.hin + ((int64_t(g) * p.K + k) * NM + n) * kSThreads + c);
+    An[n] = n < N ? f.A[int64_t(d) * N + n] : -float(n + 1);
+    any = any || (n < N && hin[n] != 0.f);
+  }
+  const int64_t tbeg = int64_t(k) * p.chunk_len;
+  const int64_t tend = std::min<int64_t>(f.L, tbeg + p.chunk_len);
+  if (k == p.K - 1 && f.last_state) {  // the true final state
+    const double S = p.agg_S[(int64_t(g) * p.K + k) * kSThreads + c];
+#pragma unroll
+    for (int n = 0; n < NM; ++n)
+      if (n < N) {
+        const float hl = __ldcg(p.agg_h + ((int64_t(g) * p.K + k) * NM + n) * kSThreads + c);
+        f.last_state[(int64_t(b) * f.dim + d) * N + n] = hl + float(exp(double(An[n]) * S)) * hin[n];
+      }
+  }
+  if (!any) return;
+  bool structured = An[0] < 0.f && isfinite(An[0]);
+#pragma unroll
+  for (int n = 1; n < NM; ++n) structured = structured && (An[n] == float(n + 1) * An[0]);
+  float amax = An[0];  // slowest decay
+#pragma unroll
+  for (int n = 1; n < NM; ++n) amax = fmaxf(amax, An[n]);
+  const float bias = f.bias ? f.bias[d] : 0.f;
+  const int64_t row = (int64_t(b) * f.dim + d) * f.L;
+  const T *dl = static_cast<const T *>(f.delta) + row;
+  const T *zr = f.z ? static_cast<const T *>(f.z) + row : nullptr;
+  T *yr = static_cast<T *>(f.y) + row;
+  const T *Cb = static_cast<const T *>(f.C) + int64_t(b) * N * f.L;
+  float cum = 0.f;
+  // the chunk starts at a multiple of 64 steps and rows are 16-byte multiples
+  for (int64_t t0 = tbeg; t0 < tend; t0 += V) {
+    if (amax * cum < -22.2f) break;  // exp(amax cumDelta) < 2^-32
+    float dv[V], zv[V], yv[V];
+    Vec<T>::unpack(*reinterpret_cast<const uint4 *>(dl + t0), dv);
+    Vec<T>::unpack(*reinterpret_cast<const uint4 *>(yr + t0), yv);
+    if (zr) Vec<T>::unpack(*reinterpret_cast<const uint4 *>(zr + t0), zv);
+#pragma unroll
+    for (int i = 0; i < V; ++i) {
+      cum += softplus_fast(dv[i] + bias);
+      float corr;
+      if (structured) {
+        const float q = ex2f(An[0] * cum * kLog2e);
+        float r = 0.f;
+#pragma unroll
+        for (int n = NM - 1; n >= 0; --n) {
+          const float cn = n < N ? to_f(Cb[int64_t(n) * f.L + t0 + i]) * hin[n] : 0.f;
+          r = fmaf(r, q, cn);
+        }
+        corr = r * q;
+      } else {
+        corr = 0.f;
+#pragma unroll
+        for (int n = 0; n < NM; ++n)
+          if (n < N) corr = fmaf(to_f(Cb[int64_t(n) * f.L + t0 + i]) * hin[n],
+                                 ex2f(An[n] * cum * kLog2e), corr);
+      }
+      if (zr) corr *= zv[i] * rcpf(1.f + ex2f(-zv[i] * kLog2e));
+      yv[i] += corr;
+    }
+    *reinterpret_cast<uint4 *>(yr + t0) = Vec<T>::pack(yv);
   }
 }
 
@@ -715,18 +1016,30 @@ inline bool staged_supported(const FwdArgs &a, size_t es) {
   return al(a.u) && al(a.delta) && al(a.z) && al(a.y) && al(a.B) && al(a.C);
 }
 
-template <typename T, int NM, int KIND, bool CONV = false>
-inline cudaError_t prepare_kernel(int *blocks_per_sm) {
-  auto kern = fwd_staged_kernel<T, NM, KIND, CONV>;
-  const int bytes = StagedLayout<T, NM>::ALLOC;
+// Dynamic shared memory of the fused-projection forward with `nst` stages.
+template <typename T, int NM>
+inline int proj_smem_bytes(int Rp, int nst) {
+  using Lay = StagedLayout<T, NM>;
+  return int(uint32_t(nst) * ProjStage(Rp).bytes) + 2 * kTileBytes + 4 * Lay::TT * Lay::BSTR * 4 +
+         8 * 5 + 16 * 4 + 1024;
+}
+
+// Largest dynamic shared memory per CTA that still lets two CTAs share an SM
+// (228 KB per SM, 1 KB of it reserved per CTA).
+constexpr int kTwoPerSmBytes = (233472 - 2 * 1024) / 2;
+
+template <typename T, int NM, int KIND, bool CONV = false, bool PROJ = false>
+inline cudaError_t prepare_kernel(int *blocks_per_sm, int bytes = StagedLayout<T, NM>::ALLOC) {
+  auto kern = fwd_staged_kernel<T, NM, KIND, CONV, PROJ>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return e;
   return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, kern, kSThreads, bytes);
 }
 
-template <typename T, int NM, int KIND, bool CONV = false>
-inline void launch_staged(const CUtensorMap (&maps)[6], const StagedArgs &sa, int grid, cudaStream_t s) {
-  fwd_staged_kernel<T, NM, KIND, CONV><<<grid, kSThreads, StagedLayout<T, NM>::ALLOC, s>>>(
+template <typename T, int NM, int KIND, bool CONV = false, bool PROJ = false>
+inline void launch_staged(const CUtensorMap (&maps)[6], const StagedArgs &sa, int grid, cudaStream_t s,
+                          int bytes = StagedLayout<T, NM>::ALLOC) {
+  fwd_staged_kernel<T, NM, KIND, CONV, PROJ><<<grid, kSThreads, bytes, s>>>(
       maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], sa);
 }
 
@@ -765,7 +1078,7 @@ inline StagedPlan plan_staged(int64_t G, int64_t L, int slots, const StagedOptio
 // workspace size; nothing enqueued) and the launches on a given workspace, so
 // that a caller can take one workspace for several steps and fail before
 // enqueuing anything when it cannot be had.
-template <typename T, int NM, bool CONV = false>
+template <typename T, int NM, bool CONV = false, bool PROJ = false>
 struct StagedForward {
   using Lay = StagedLayout<T, NM>;
   CUtensorMap maps[6];
@@ -773,6 +1086,7 @@ struct StagedForward {
   StagedPlan pl;
   int sms = 0, slots = 0;
   size_t int_bytes = 0, bytes = 0;
+  int smem = Lay::ALLOC;  // dynamic shared memory per CTA
 
   // Builds the tensor maps and the plan; with `ckpt` the forward runs without
   // y and stores the state before every kCkptEvery-th step into ckpt
@@ -782,8 +1096,17 @@ struct StagedForward {
     constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
     const uint64_t L = a.L, dim = a.dim, batch = a.batch, N = a.N;
     const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_64B, none = CU_TENSOR_MAP_SWIZZLE_NONE;
-    if (!make_map_3d(&maps[0], a.u, bf16, L, dim, batch, Lay::TT, kSThreads, sw) ||
-        !make_map_3d(&maps[1], a.delta, bf16, L, dim, batch, Lay::TT, kSThreads, sw) ||
+    int Rp = 0, nst = kStages;
+    if (PROJ) {  // the dt_low tiles: Rp rows (R rounded up to 16, zero-filled) of TT steps
+      Rp = (a.R + 15) / 16 * 16;
+      if (a.R < 1 || Rp > kProjMaxRp) return MAMBA_ERR_UNSUPPORTED;
+      nst = proj_smem_bytes<T, NM>(Rp, 3) <= kTwoPerSmBytes ? 3 : 2;
+      smem = proj_smem_bytes<T, NM>(Rp, nst);
+    }
+    const bool dmap = PROJ ? make_map_3d(&maps[1], a.dt_low, bf16, L, uint64_t(a.R), batch, Lay::TT,
+                                         uint32_t(Rp), sw)
+                           : make_map_3d(&maps[1], a.delta, bf16, L, dim, batch, Lay::TT, kSThreads, sw);
+    if (!make_map_3d(&maps[0], a.u, bf16, L, dim, batch, Lay::TT, kSThreads, sw) || !dmap ||
         !make_map_3d(&maps[2], a.z ? a.z : a.u, bf16, L, dim, batch, Lay::TT, kSThreads, sw) ||
         !make_map_3d(&maps[3], a.y ? a.y : a.u, bf16, L, dim, batch, Lay::TT, kSThreads, sw) ||
         !make_map_3d(&maps[4], a.B, bf16, L, N, batch, Lay::TT, uint32_t(N), none) ||
@@ -791,7 +1114,7 @@ struct StagedForward {
       return MAMBA_ERR_UNSUPPORTED;
     }
     int bps_main = 0;
-    if (prepare_kernel<T, NM, KIND_SEQ, CONV>(&bps_main) != cudaSuccess) return MAMBA_ERR_CUDA;
+    if (prepare_kernel<T, NM, KIND_SEQ, CONV, PROJ>(&bps_main, smem) != cudaSuccess) return MAMBA_ERR_CUDA;
     sms = device_sm_count();
     slots = sms * std::max(1, bps_main);
     const int64_t gpb = ceil_div(a.dim, kSThreads);
@@ -813,6 +1136,10 @@ struct StagedForward {
     sa.carry = sa.agg_h = sa.hin = nullptr;
     sa.agg_S = nullptr;
     sa.ckpt = ckpt;
+    sa.Rp = Rp;
+    sa.nst = nst;
+    sa.stage_bytes = PROJ ? ProjStage(Rp).bytes : 0;
+    sa.delta_out = nullptr;
 
     // workspace: [ints: 2 counters + G flags][carry | agg_S, agg_h, hin]
     const size_t n_int = 2 + size_t(G);
@@ -826,6 +1153,22 @@ struct StagedForward {
     }
     bytes = ceil_div(bytes, 256) * 256;
     return MAMBA_OK;
+  }
+
+  // The scan over chunks (three-phase carry): h_in of every chunk.
+  mamba_status_t launch_chunk_scan(cudaStream_t s, mamba_status_t (*launched)()) {
+    ChunkScanIO io;
+    io.S = sa.agg_S;
+    io.hl = sa.agg_h;
+    io.hin = sa.hin;
+    io.A = sa.f.A;
+    io.G = sa.G;
+    io.K = sa.K;
+    io.gpb = sa.gpb;
+    io.N = sa.f.N;
+    io.dim = sa.f.dim;
+    chunk_scan_kernel<NM, false><<<unsigned(int64_t(sa.G) * NM * kSThreads), 128, 0, s>>>(io);
+    return launched();
   }
 
   // Enqueues the launches on `ws` (at least `bytes`, 256-byte aligned).
@@ -842,43 +1185,61 @@ struct StagedForward {
       const int grid = int(std::min<int64_t>(gk, slots));
       if (sa.ckpt) {
         int bps = 0;
-        if (prepare_kernel<T, NM, KIND_CKPT_SEQ, CONV>(&bps) != cudaSuccess) return MAMBA_ERR_CUDA;
-        launch_staged<T, NM, KIND_CKPT_SEQ, CONV>(maps, sa,
-                                                  int(std::min<int64_t>(gk, sms * std::max(1, bps))), s);
+        if (prepare_kernel<T, NM, KIND_CKPT_SEQ, CONV, PROJ>(&bps, smem) != cudaSuccess)
+          return MAMBA_ERR_CUDA;
+        launch_staged<T, NM, KIND_CKPT_SEQ, CONV, PROJ>(
+            maps, sa, int(std::min<int64_t>(gk, sms * std::max(1, bps))), s, smem);
       } else {
-        launch_staged<T, NM, KIND_SEQ, CONV>(maps, sa, grid, s);
+        launch_staged<T, NM, KIND_SEQ, CONV, PROJ>(maps, sa, grid, s, smem);
       }
       return launched();
     }
     sa.agg_S = reinterpret_cast<double *>(ws + int_bytes);
     sa.agg_h = reinterpret_cast<float *>(ws + int_bytes + gk * kSThreads * 8);
     sa.hin = sa.agg_h + gk * NM * kSThreads;
+    if (!sa.ckpt && !PROJ) {
+      // Every chunk from zero, with y and its aggregates; the scan over
+      // chunks; the closed-form correction of chunks 1..K-1 (and of the
+      // final state).  (The checkpoint pass needs the true states at every
+      // 16th step, and the fused projection does not store delta for the
+      // correction: those take the aggregate pass and a second full pass.)
+      int bps_loc = 0;
+      if (prepare_kernel<T, NM, KIND_LOC, CONV, PROJ>(&bps_loc, smem) != cudaSuccess) return MAMBA_ERR_CUDA;
+      StagedArgs sl = sa;
+      sl.counter = counters;
+      sl.n_units = int(gk);
+      launch_staged<T, NM, KIND_LOC, CONV, PROJ>(
+          maps, sl, int(std::min<int64_t>(gk, sms * std::max(1, bps_loc))), s, smem);
+      st = launched();
+      if (st == MAMBA_OK) st = launch_chunk_scan(s, launched);
+      if (st == MAMBA_OK) {
+        fwd_correct_kernel<T, NM><<<unsigned(size_t(sa.G) * size_t(pl.K - 1)), kSThreads, 0, s>>>(sa);
+        st = launched();
+      }
+      return st;
+    }
     int bps_agg = 0, bps_par = 0;
-    if (prepare_kernel<T, NM, KIND_AGG, CONV>(&bps_agg) != cudaSuccess ||
-        (sa.ckpt ? prepare_kernel<T, NM, KIND_CKPT_PAR, CONV>(&bps_par)
-                 : prepare_kernel<T, NM, KIND_PAR, CONV>(&bps_par)) != cudaSuccess) {
+    if (prepare_kernel<T, NM, KIND_AGG, CONV, PROJ>(&bps_agg, smem) != cudaSuccess ||
+        (sa.ckpt ? prepare_kernel<T, NM, KIND_CKPT_PAR, CONV, PROJ>(&bps_par, smem)
+                 : prepare_kernel<T, NM, KIND_PAR, CONV, PROJ>(&bps_par, smem)) != cudaSuccess) {
       return MAMBA_ERR_CUDA;
     }
     {
       StagedArgs sg = sa;
       sg.counter = counters;
       sg.n_units = int(size_t(sa.G) * size_t(pl.K - 1));
-      launch_staged<T, NM, KIND_AGG, CONV>(maps, sg,
-                                           int(std::min<int64_t>(sg.n_units, sms * std::max(1, bps_agg))), s);
+      launch_staged<T, NM, KIND_AGG, CONV, PROJ>(
+          maps, sg, int(std::min<int64_t>(sg.n_units, sms * std::max(1, bps_agg))), s, smem);
       st = launched();
     }
-    if (st == MAMBA_OK) {
-      const int64_t threads = int64_t(sa.G) * NM * kSThreads;
-      carry_scan_kernel<NM><<<unsigned(ceil_div(threads, 256)), 256, 0, s>>>(sa);
-      st = launched();
-    }
+    if (st == MAMBA_OK) st = launch_chunk_scan(s, launched);
     if (st == MAMBA_OK) {
       StagedArgs sm = sa;
       sm.counter = counters + 1;
       sm.n_units = int(gk);
       const int grid = int(std::min<int64_t>(gk, sms * std::max(1, bps_par)));
-      if (sa.ckpt) launch_staged<T, NM, KIND_CKPT_PAR, CONV>(maps, sm, grid, s);
-      else launch_staged<T, NM, KIND_PAR, CONV>(maps, sm, grid, s);
+      if (sa.ckpt) launch_staged<T, NM, KIND_CKPT_PAR, CONV, PROJ>(maps, sm, grid, s, smem);
+      else launch_staged<T, NM, KIND_PAR, CONV, PROJ>(maps, sm, grid, s, smem);
       st = launched();
     }
     return st;
@@ -889,10 +1250,10 @@ struct StagedForward {
 // MAMBA_ERR_UNSUPPORTED (nothing enqueued) if the driver rejects a tensor map,
 // MAMBA_ERR_OUT_OF_MEMORY (nothing enqueued) if the workspace cannot be had.
 // CONV selects the kernels with the convolution prologue (a.conv_w set).
-template <typename T, int NM, bool CONV = false>
+template <typename T, int NM, bool CONV = false, bool PROJ = false>
 mamba_status_t staged_forward(const FwdArgs &a, const StagedOptions &o, cudaStream_t s,
                               mamba_status_t (*launched)(), float *ckpt = nullptr) {
-  StagedForward<T, NM, CONV> sf;
+  StagedForward<T, NM, CONV, PROJ> sf;
   mamba_status_t st = sf.prepare(a, o, ckpt);
   if (st != MAMBA_OK) return st;
   unsigned char *ws = nullptr;

@@ -16,7 +16,8 @@
 #include "common.cuh"
 #include "conv_bwd.cuh"
 #include "cplx.cuh"
-#include "dtproj.h"
+#include "dtproj.cuh"
+#include "dtproj_gemm.cuh"
 #include "decode.cuh"
 #include "fwd_reference.cuh"
 #include "fwd_staged.cuh"
@@ -351,6 +352,130 @@ mamba_status_t backward_paths(const BwdArgs &a, size_t es, mamba_dtype_t dtype,
   if (st == MAMBA_ERR_UNSUPPORTED && so.path == MAMBA_PATH_AUTO)
     return dispatch<BwdReferenceLauncher>(dtype, a.N, a, s);
   return st;
+}
+
+// Whether the fused projection (delta formed on the tensor cores inside the
+// staged kernels) takes this forward: bf16, a shape the staged kernels take,
+// a rank its tiles fit, and no explicit path other than automatic/structured.
+bool proj_fused_ok(const FwdArgs &a, mamba_dtype_t dtype, const StagedOptions &so) {
+  if (dtype != MAMBA_BF16 || so.path == MAMBA_PATH_REFERENCE) return false;
+  if (!staged_supported(a, 2) || !a.dt_low || !a.W_dt) return false;
+  auto al = [](const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; };
+  if (!al(a.dt_low) || (int64_t(a.L) * 2) % 16 != 0) return false;
+  const int Rp = (a.R + 15) / 16 * 16;
+  return a.R >= 1 && Rp <= proj_max_rank<__nv_bfloat16, 16>();
+}
+
+mamba_status_t proj_fused_dispatch(const FwdArgs &a, const StagedOptions &o, cudaStream_t s) {
+  if (a.N <= 4) return staged_forward<__nv_bfloat16, 4, false, true>(a, o, s, &launch_status);
+  if (a.N <= 8) return staged_forward<__nv_bfloat16, 8, false, true>(a, o, s, &launch_status);
+  return staged_forward<__nv_bfloat16, 16, false, true>(a, o, s, &launch_status);
+}
+
+mamba_status_t proj_fused_bwd_dispatch(const BwdArgs &a, const StagedOptions &o, cudaStream_t s) {
+  if (a.N <= 4) return staged_backward<__nv_bfloat16, 4, false, true>(a, o, s, &launch_status);
+  if (a.N <= 8) return staged_backward<__nv_bfloat16, 8, false, true>(a, o, s, &launch_status);
+  return staged_backward<__nv_bfloat16, 16, false, true>(a, o, s, &launch_status);
+}
+
+// How the projection's gradient products split dW's contraction over the
+// grid (tensor-core path); 0 splits when the shapes or alignments do not suit
+// its TMA tiles (the CUDA-core contraction is used instead).
+struct ProjGradPlan {
+  int splits = 0, k_per_split = 0, k_tiles = 0;
+  size_t part_bytes = 0;  // fp32 partial sums of dW, one set per split
+};
+
+ProjGradPlan proj_grads_plan(const void *W, const void *dt_low, int64_t batch, int64_t dim,
+                             int64_t L, int64_t R, mamba_dtype_t dtype) {
+  ProjGradPlan pl;
+  auto al = [](const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; };
+  if (dtype != MAMBA_BF16 || R % 8 != 0 || L % 8 != 0 || !al(W) || !al(dt_low)) return pl;
+  const int Rp_in = int((R + 63) / 64 * 64), Rp_w = int((R + 15) / 16 * 16);
+  if (Rp_in > 256 || Rp_w > 256 || L > (int64_t(1) << 30) || dim > (int64_t(1) << 30) ||
+      batch > 65535)
+    return pl;
+  const int mt = int((dim + 127) / 128);
+  pl.k_tiles = int(batch * ((L + 63) / 64));
+  int splits = std::max(1, std::min(pl.k_tiles, (2 * device_sm_count() + mt - 1) / mt));
+  pl.k_per_split = (pl.k_tiles + splits - 1) / splits;
+  pl.splits = (pl.k_tiles + pl.k_per_split - 1) / pl.k_per_split;
+  pl.part_bytes = (size_t(pl.splits) * size_t(dim) * size_t(R) * 4 + 255) / 256 * 256;
+  return pl;
+}
+
+// The projection's gradient products on the tensor cores (bf16, tcgen05),
+// with the plan's partial sums in `part`: false (nothing enqueued) if a
+// tensor map is refused, so that the caller takes the CUDA-core contraction.
+bool proj_grads_tc(const ProjGradPlan &pl, float *part, const void *W, const void *dt_low,
+                   const void *ddelta, void *d_dt_low, float *dW, int64_t batch, int64_t dim,
+                   int64_t L, int64_t R, cudaStream_t s, mamba_status_t *st) {
+  auto al = [](const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; };
+  if (pl.splits == 0 || !part || !al(ddelta)) return false;
+  const int Rp_in = int((R + 63) / 64 * 64), Rp_w = int((R + 15) / 16 * 16);
+  const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  CUtensorMap a_in, b_in, a_w, b_w;
+  if (!make_map_3d(&a_in, ddelta, true, uint64_t(L), uint64_t(dim), uint64_t(batch), 64, 64, sw) ||
+      !make_map_3d(&b_in, W, true, uint64_t(R), uint64_t(dim), 1, 64, 64, sw) ||
+      !make_map_3d(&a_w, ddelta, true, uint64_t(L), uint64_t(dim), uint64_t(batch), 64, 128, sw) ||
+      !make_map_3d(&b_w, dt_low, true, uint64_t(L), uint64_t(R), uint64_t(batch), 64, uint32_t(Rp_w), sw))
+    return false;
+  const int smem_in = proj_gemm_smem<true>(Rp_in), smem_w = proj_gemm_smem<false>(Rp_w);
+  if (cudaFuncSetAttribute(proj_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem_in) != cudaSuccess ||
+      cudaFuncSetAttribute(proj_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem_w) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  const int mt = int((dim + 127) / 128);
+  ProjGemmArgs gi;
+  gi.batch = batch; gi.dim = dim; gi.L = L; gi.R = int(R); gi.Rp = Rp_in;
+  gi.k_tiles = int((dim + 63) / 64); gi.k_per_split = gi.k_tiles;
+  gi.out = d_dt_low; gi.timeout_ns = kDefaultTimeoutNs;
+  proj_gemm_kernel<true><<<dim3(unsigned((L + 127) / 128), unsigned(batch)), 128, smem_in, s>>>(a_in, b_in, gi);
+  *st = launch_status();
+  if (*st == MAMBA_OK) {
+    ProjGemmArgs gw = gi;
+    gw.Rp = Rp_w;
+    gw.k_tiles = pl.k_tiles;
+    gw.k_per_split = pl.k_per_split;
+    gw.out = part;
+    proj_gemm_kernel<false><<<dim3(unsigned(mt), unsigned(pl.splits)), 128, smem_w, s>>>(a_w, b_w, gw);
+    *st = launch_status();
+  }
+  if (*st == MAMBA_OK) {
+    const int64_t n = dim * R;
+    proj_grad_weight_finalize<<<unsigned(std::min<int64_t>((n + 255) / 256, 1184)), 256, 0, s>>>(
+        part, dW, n, pl.splits);
+    *st = launch_status();
+  }
+  return true;
+}
+
+// d_dt_low = W^T ddelta per batch row and dW = sum_b ddelta_b dt_low_b^T.
+mamba_status_t proj_grads(const ProjGradPlan &pl, float *part, const void *W, const void *dt_low,
+                          const void *ddelta, void *d_dt_low, float *dW, int64_t batch, int64_t dim,
+                          int64_t L, int64_t R, mamba_dtype_t dtype, cudaStream_t s) {
+  {
+    mamba_status_t st = MAMBA_OK;
+    if (proj_grads_tc(pl, part, W, dt_low, ddelta, d_dt_low, dW, batch, dim, L, R, s, &st)) return st;
+  }
+  const Contraction gi = proj_grad_input(W, ddelta, d_dt_low, batch, dim, L, R);
+  const Contraction gw = proj_grad_weight(ddelta, dt_low, dW, batch, dim, L, R);
+  cudaError_t e;
+  if (dtype == MAMBA_BF16) {
+    e = launch_contraction<__nv_bfloat16, __nv_bfloat16>(gi, s);
+    if (e == cudaSuccess && launch_status() == MAMBA_OK) e = launch_contraction<__nv_bfloat16, float>(gw, s);
+  } else {
+    e = launch_contraction<float, float>(gi, s);
+    if (e == cudaSuccess && launch_status() == MAMBA_OK) e = launch_contraction<float, float>(gw, s);
+  }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return MAMBA_ERR_CUDA;
+  }
+  return launch_status();
 }
 
 }  // namespace
@@ -851,21 +976,33 @@ mamba_status_t mamba_dtproj_scan_fwd(const void *u, const void *dt_low, const vo
       return cuda_status();
     return MAMBA_OK;
   }
-  const cublasHandle_t h = cublas_handle(ck.dev);
-  if (!h || cublas_api().set_stream(h, s) != CUBLAS_STATUS_SUCCESS) return MAMBA_ERR_UNSUPPORTED;
+  FwdArgs a;
+  a.u = u; a.delta = nullptr; a.z = z; a.B = B; a.C = C;
+  a.bias = delta_bias; a.A = A; a.D = D; a.y = y; a.last_state = last_state;
+  a.batch = batch; a.dim = dim; a.L = L; a.N = (int)N;
+  a.dt_low = dt_low; a.W_dt = W_dt; a.R = (int)R;
+  const StagedOptions so = staged_options(options);
+  // bf16 on the staged kernels: delta formed on the tensor cores inside the scan
+  if (proj_fused_ok(a, dtype, so)) {
+    st = proj_fused_dispatch(a, so, s);
+    if (st != MAMBA_ERR_UNSUPPORTED) return st;
+  }
+  // otherwise delta is formed first, in the I/O type, by the FP32 contraction
   void *delta = nullptr;
   if (ws_alloc(&delta, nbdl * es, s) != cudaSuccess) {
     cudaGetLastError();
     return MAMBA_ERR_OUT_OF_MEMORY;
   }
-  const DtProj pj{h, dtype == MAMBA_BF16 ? CUDA_R_16BF : CUDA_R_32F, batch, dim, L, R};
-  st = pj.forward(dt_low, W_dt, delta) ? MAMBA_OK : MAMBA_ERR_CUDA;
+  const Contraction cd = proj_delta(W_dt, dt_low, delta, batch, dim, L, R);
+  st = (dtype == MAMBA_BF16 ? launch_contraction<__nv_bfloat16, __nv_bfloat16>(cd, s)
+                            : launch_contraction<float, float>(cd, s)) == cudaSuccess
+           ? launch_status()
+           : MAMBA_ERR_CUDA;
   if (st == MAMBA_OK) {
-    FwdArgs a;
-    a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
-    a.bias = delta_bias; a.A = A; a.D = D; a.y = y; a.last_state = last_state;
-    a.batch = batch; a.dim = dim; a.L = L; a.N = (int)N;
-    st = forward_paths<false>(a, es, dtype, staged_options(options), s);
+    a.delta = delta;
+    a.dt_low = a.W_dt = nullptr;
+    a.R = 0;
+    st = forward_paths<false>(a, es, dtype, so, s);
   }
   if (ws_free(delta, s) != cudaSuccess && st == MAMBA_OK) st = MAMBA_ERR_CUDA;
   return st;
@@ -925,30 +1062,62 @@ mamba_status_t mamba_dtproj_scan_bwd(const void *u, const void *dt_low, const vo
       return cuda_status();
     return MAMBA_OK;
   }
-  const cublasHandle_t h = cublas_handle(ck.dev);
-  if (!h || cublas_api().set_stream(h, s) != CUBLAS_STATUS_SUCCESS) return MAMBA_ERR_UNSUPPORTED;
-  // workspace: delta, then ddelta (the scan backward's gradient of delta)
+  BwdArgs a;
+  a.u = u; a.delta = nullptr; a.z = z; a.B = B; a.C = C; a.dy = dy;
+  a.bias = delta_bias; a.A = A; a.D = D;
+  a.du = du; a.ddelta = nullptr; a.dz = dz; a.dB = dB; a.dC = dC;
+  a.dA = dA; a.dD = dD; a.dbias = ddelta_bias;
+  a.batch = batch; a.dim = dim; a.L = L; a.N = (int)N;
+  a.dt_low = dt_low; a.W_dt = W_dt; a.R = (int)R;
+  const StagedOptions so = staged_options(options);
+  FwdArgs fa;
+  fa.u = u; fa.delta = nullptr; fa.z = z; fa.B = B; fa.C = C; fa.bias = delta_bias; fa.A = A;
+  fa.D = D; fa.y = nullptr; fa.last_state = nullptr; fa.batch = batch; fa.dim = dim; fa.L = L;
+  fa.N = (int)N; fa.dt_low = dt_low; fa.W_dt = W_dt; fa.R = (int)R;
+  const bool fused = proj_fused_ok(fa, dtype, so) && staged_bwd_supported(a, es);
+  const ProjGradPlan gp = proj_grads_plan(W_dt, dt_low, batch, dim, L, R, dtype);
+  // workspace: the gradient products' partial sums, ddelta (the scan
+  // backward's gradient of delta, in the I/O type), then (unfused) delta
   const size_t half = (nbdl * es + 255) / 256 * 256;
   unsigned char *ws = nullptr;
-  if (ws_alloc(reinterpret_cast<void **>(&ws), 2 * half, s) != cudaSuccess) {
+  if (ws_alloc(reinterpret_cast<void **>(&ws), gp.part_bytes + (fused ? half : 2 * half), s) !=
+      cudaSuccess) {
     cudaGetLastError();
     return MAMBA_ERR_OUT_OF_MEMORY;
   }
-  void *delta = ws, *ddelta = ws + half;
-  const DtProj pj{h, dtype == MAMBA_BF16 ? CUDA_R_16BF : CUDA_R_32F, batch, dim, L, R};
-  st = pj.forward(dt_low, W_dt, delta) ? MAMBA_OK : MAMBA_ERR_CUDA;
-  if (st == MAMBA_OK) {
-    BwdArgs a;
-    a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C; a.dy = dy;
-    a.bias = delta_bias; a.A = A; a.D = D;
-    a.du = du; a.ddelta = ddelta; a.dz = dz; a.dB = dB; a.dC = dC;
-    a.dA = dA; a.dD = dD; a.dbias = ddelta_bias;
-    a.batch = batch; a.dim = dim; a.L = L; a.N = (int)N;
-    st = backward_paths<false>(a, es, dtype, staged_options(options), s);
+  float *part = gp.part_bytes ? reinterpret_cast<float *>(ws) : nullptr;
+  void *ddelta = ws + gp.part_bytes, *delta = fused ? nullptr : ws + gp.part_bytes + half;
+  a.ddelta = ddelta;
+  st = MAMBA_ERR_UNSUPPORTED;
+  if (fused) st = proj_fused_bwd_dispatch(a, so, s);
+  if (st == MAMBA_ERR_UNSUPPORTED && delta == nullptr) {  // the fused kernels declined
+    ws_free(ws, s);
+    ws = nullptr;
+    if (ws_alloc(reinterpret_cast<void **>(&ws), gp.part_bytes + 2 * half, s) != cudaSuccess) {
+      cudaGetLastError();
+      return MAMBA_ERR_OUT_OF_MEMORY;
+    }
+    part = gp.part_bytes ? reinterpret_cast<float *>(ws) : nullptr;
+    ddelta = ws + gp.part_bytes;
+    delta = ws + gp.part_bytes + half;
+    a.ddelta = ddelta;
   }
-  if (st == MAMBA_OK && !(pj.grad_input(ddelta, W_dt, d_dt_low) &&
-                          pj.grad_weight(ddelta, dt_low, dW_dt, es)))
-    st = MAMBA_ERR_CUDA;
+  if (st == MAMBA_ERR_UNSUPPORTED) {
+    const Contraction cd = proj_delta(W_dt, dt_low, delta, batch, dim, L, R);
+    st = (dtype == MAMBA_BF16 ? launch_contraction<__nv_bfloat16, __nv_bfloat16>(cd, s)
+                              : launch_contraction<float, float>(cd, s)) == cudaSuccess
+             ? launch_status()
+             : MAMBA_ERR_CUDA;
+    if (st == MAMBA_OK) {
+      a.delta = delta;
+      a.dt_low = a.W_dt = nullptr;
+      a.R = 0;
+      st = backward_paths<false>(a, es, dtype, so, s);
+    }
+  }
+  // the two gradient products of the projection, from ddelta
+  if (st == MAMBA_OK)
+    st = proj_grads(gp, part, W_dt, dt_low, ddelta, d_dt_low, dW_dt, batch, dim, L, R, dtype, s);
   if (ws_free(ws, s) != cudaSuccess && st == MAMBA_OK) st = MAMBA_ERR_CUDA;
   return st;
 }
