@@ -75,7 +75,9 @@ typedef enum {
   MAMBA_ERR_UNSUPPORTED = 2,   /* N outside 1..16, or a shape beyond the limits */
   MAMBA_ERR_CUDA = 3,          /* a CUDA runtime call or a launch failed */
   MAMBA_ERR_OUT_OF_MEMORY = 4, /* the stream-ordered workspace could not be allocated */
-  MAMBA_ERR_DEVICE_TIMEOUT = 5 /* a bounded device-side wait expired (sticky) */
+  MAMBA_ERR_DEVICE_TIMEOUT = 5, /* a bounded device-side wait expired (sticky) */
+  MAMBA_ERR_OUT_OF_BOUNDS = 6   /* bounds-checking build only: a kernel computed an index
+                                   outside its buffer and skipped the access (sticky) */
 } mamba_status_t;
 
 /* Kernel-path selection for mamba_scan_fwd_ex / mamba_scan_bwd_ex. */
@@ -397,17 +399,22 @@ MAMBA_SCAN_API void mamba_scan_test_fail_alloc(int32_t after);
  * that cannot let a library allocate device memory -- programs that give all
  * device memory to their own allocator up front, latency-critical loops that
  * must not enter the CUDA allocator, code that runs where allocation calls
- * are not allowed.  Instead of a workspace per call, the chunked kernel keeps
- * its scratch (ticket counter, hand-off flags, carried chunk-end states) in a
- * fixed 8 MiB array in the library's device memory; every GPU that loads the
- * library holds that array until the process exits.  The call makes no
- * cudaMalloc, cudaMallocAsync or cudaFree call.
+ * are not allowed.  Instead of a workspace per call, the chunked kernels keep
+ * their scratch (ticket counters, hand-off flags, carried chunk-end states,
+ * or the chunk aggregates of the three-phase carry) in a fixed 8 MiB array in
+ * the library's device memory; every GPU that loads the library holds that
+ * array until the process exits.  The call makes no cudaMalloc,
+ * cudaMallocAsync or cudaFree call.
  *
- *  - Limit: batch * ceil(dim / 128) channel groups must fit the array: at most
- *    1016 groups when N > 8, 2032 when 4 < N <= 8, 4064 when N <= 4.  Larger
- *    problems return MAMBA_ERR_UNSUPPORTED without enqueuing anything.  Shapes
- *    that the staged kernels do not take (see mamba_scan_fwd) run the
- *    one-thread-per-channel kernel, which needs no scratch.
+ *  - Plan: the regular call's (see mamba_scan_options_t.carry) when its
+ *    scratch fits the array; for the three-phase carry of few channel groups
+ *    and long sequences, fewer and longer chunks until it does.
+ *  - Limit: the sequential hand-off's scratch must fit: at most 1023 channel
+ *    groups (batch * ceil(dim / 128)) when N > 8, 2046 when 4 < N <= 8, 4088
+ *    when N <= 4.  Larger problems return MAMBA_ERR_UNSUPPORTED without
+ *    enqueuing anything.  Shapes that the staged kernels do not take (see
+ *    mamba_scan_fwd) run the one-thread-per-channel kernel, which needs no
+ *    scratch.
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress) for that device; make that first call before any
  *    stream capture.
@@ -425,7 +432,9 @@ MAMBA_SCAN_API mamba_status_t mamba_scan_fwd_noalloc(const void *u, const void *
 
 /* Synchronizes `stream`, then returns MAMBA_ERR_CUDA for a pending CUDA error,
  * else MAMBA_ERR_DEVICE_TIMEOUT if a kernel of this library recorded an
- * expired wait on the current device since the last call (the record is
+ * expired wait on the current device since the last call, else (in the
+ * bounds-checking build, libmambascan_debug.so) MAMBA_ERR_OUT_OF_BOUNDS if a
+ * kernel computed an index outside one of its buffers (the records are
  * cleared), else MAMBA_OK. */
 MAMBA_SCAN_API mamba_status_t mamba_scan_stream_status(mamba_stream_t stream);
 

@@ -77,6 +77,25 @@ def build_micro(force: bool = False) -> str:
     return MICRO_LIB
 
 
+DEBUG_LIB = os.path.join(LIBDIR, "libmambascan_debug.so")
+
+
+def build_debug(force: bool = False) -> str:
+    """Build libmambascan_debug.so: the same library with MAMBA_DEBUG_BOUNDS,
+    whose kernels check their computed indices against the buffers and record
+    a wrong one in the sticky status (MAMBA_ERR_OUT_OF_BOUNDS) instead of
+    making the access."""
+    if not force and os.path.exists(DEBUG_LIB) and \
+            all(os.path.getmtime(p) <= os.path.getmtime(DEBUG_LIB) for p in deps()):
+        return DEBUG_LIB
+    os.makedirs(LIBDIR, exist_ok=True)
+    tmp = DEBUG_LIB + f".tmp{os.getpid()}"
+    subprocess.check_call([NVCC, *NVCC_FLAGS, "-DMAMBA_DEBUG_BOUNDS", "-I",
+                           os.path.join(ROOT, "include"), *sources(), "-o", tmp])
+    os.replace(tmp, DEBUG_LIB)
+    return DEBUG_LIB
+
+
 def build(force: bool = False, verbose_ptxas: bool = False) -> str:
     build_micro(force)
     if not force and not stale():
@@ -96,6 +115,10 @@ if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose-ptxas", action="store_true")
+    ap.add_argument("--debug-bounds", action="store_true",
+                    help="also build the bounds-checking libmambascan_debug.so")
     args = ap.parse_args()
     print(build(force=args.force, verbose_ptxas=args.verbose_ptxas))
+    if args.debug_bounds:
+        print(build_debug(force=args.force))
     sys.exit(0)

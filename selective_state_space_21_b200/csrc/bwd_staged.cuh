@@ -105,6 +105,9 @@ struct BwdStagedArgs {
   // fused Delta projection (PROJ kernels): R padded to 16; bytes of a stage
   int Rp = 0;
   uint32_t stage_bytes = 0;
+  // element counts of the workspace buffers as allocated (the bounds-checking
+  // build checks every index against them)
+  int64_t n_ckpt = 0, n_carry = 0, n_bc = 0, n_unit = 0, n_gin = 0;
 };
 
 // Byte offset of 16-byte chunk c of row r in a tile with RB-byte rows written
@@ -443,7 +446,10 @@ __global__ void __launch_bounds__(kSThreads, 2)
     if (p.gin) {  // three-phase carry: the entering adjoint is known
 #pragma unroll
       for (int n = 0; n < NM; ++n)
-        gt[n] = __ldcg(p.gin + ((int64_t(g) * p.K + k) * NM + n) * kSThreads + tid);
+      {
+        const int64_t i = ((int64_t(g) * p.K + k) * NM + n) * kSThreads + tid;
+        gt[n] = in_bounds(i, p.n_gin) ? __ldcg(p.gin + i) : 0.f;
+      }
     } else if (r > 0) {
       if (tid == 0 && !wait_flag_geq(p.flags + g, r, p.timeout_ns)) {
         record_timeout();
@@ -455,7 +461,10 @@ __global__ void __launch_bounds__(kSThreads, 2)
         break;
       }
 #pragma unroll
-      for (int n = 0; n < NM; ++n) gt[n] = __ldcg(p.carry + (int64_t(g) * NM + n) * kSThreads + tid);
+      for (int n = 0; n < NM; ++n) {
+        const int64_t i = (int64_t(g) * NM + n) * kSThreads + tid;
+        gt[n] = in_bounds(i, p.n_carry) ? __ldcg(p.carry + i) : 0.f;
+      }
     }
     float dA[NM];
     float dDsum = 0.f, dbsum = 0.f;
@@ -525,7 +534,8 @@ __global__ void __launch_bounds__(kSThreads, 2)
         // checkpoint of the tile start (issued before the wait to overlap)
         float h0[NM];
         {
-          const float *ck = p.ckpt + ((int64_t(g) * n16 + t0 / kBTT) * NM) * kSThreads + tid;
+          const int64_t ci = ((int64_t(g) * n16 + t0 / kBTT) * NM) * kSThreads + tid;
+          const float *ck = p.ckpt + (in_bounds(ci + (NM - 1) * kSThreads, p.n_ckpt) ? ci : 0);
 #pragma unroll
           for (int n = 0; n < NM; ++n) h0[n] = __ldcg(ck + n * kSThreads);
         }
@@ -533,7 +543,8 @@ __global__ void __launch_bounds__(kSThreads, 2)
         // the sequence start and on padding channels)
         [[maybe_unused]] float hx[4] = {0.f, 0.f, 0.f, 0.f};
         if constexpr (CONV) {
-          if (valid && t0 > 0) load_x4(static_cast<const T *>(f.u) + row + t0 - 4, hx);
+          if (valid && t0 > 0 && in_bounds(row + t0 - 4, f.batch * f.dim * f.L))
+            load_x4(static_cast<const T *>(f.u) + row + t0 - 4, hx);
         }
         if (!mbar_wait_bounded(&bars[stage], parity, p.timeout_ns)) {
           record_timeout();
@@ -840,9 +851,11 @@ __global__ void __launch_bounds__(kSThreads, 2)
             }
             if (valid) {
               const int64_t o = row + t0 + seg * SEG;
-              IO::store(static_cast<T *>(f.du) + o, du_o);
-              IO::store(static_cast<T *>(f.ddelta) + o, dd_o);
-              if (has_z) IO::store(static_cast<T *>(f.dz) + o, dz_o);
+              if (in_bounds(o + SEG - 1, f.batch * f.dim * f.L)) {
+                IO::store(static_cast<T *>(f.du) + o, du_o);
+                IO::store(static_cast<T *>(f.ddelta) + o, dd_o);
+                if (has_z) IO::store(static_cast<T *>(f.dz) + o, dz_o);
+              }
             }
           }
         };
@@ -881,7 +894,8 @@ __global__ void __launch_bounds__(kSThreads, 2)
             float sum = 0.f;
 #pragma unroll
             for (int wv = 0; wv < kSThreads / 32; ++wv) sum += red[(wv * kBTT + tl) * 33 + slot];
-            p.part_bc[((int64_t(g % p.gpb) * f.batch + b) * 32 + slot) * f.L + t0 + tl] = sum;
+            const int64_t bi = ((int64_t(g % p.gpb) * f.batch + b) * 32 + slot) * f.L + t0 + tl;
+            if (in_bounds(bi, p.n_bc)) p.part_bc[bi] = sum;
           }
         }
         if (tid == 0) produce(false);
@@ -915,12 +929,18 @@ __global__ void __launch_bounds__(kSThreads, 2)
 
     const int64_t pu = int64_t(g) * p.K + k;
 #pragma unroll
-    for (int n = 0; n < NM; ++n) p.part_A[(pu * NM + n) * kSThreads + tid] = valid ? dA[n] : 0.f;
-    p.part_D[pu * kSThreads + tid] = valid ? dDsum : 0.f;
-    p.part_bias[pu * kSThreads + tid] = valid ? dbsum : 0.f;
+    for (int n = 0; n < NM; ++n)
+      if (in_bounds((pu * NM + n) * kSThreads + tid, p.n_unit * NM))
+        p.part_A[(pu * NM + n) * kSThreads + tid] = valid ? dA[n] : 0.f;
+    if (in_bounds(pu * kSThreads + tid, p.n_unit)) {
+      p.part_D[pu * kSThreads + tid] = valid ? dDsum : 0.f;
+      p.part_bias[pu * kSThreads + tid] = valid ? dbsum : 0.f;
+    }
     if (k > 0 && !p.gin) {
 #pragma unroll
-      for (int n = 0; n < NM; ++n) p.carry[(int64_t(g) * NM + n) * kSThreads + tid] = gt[n];
+      for (int n = 0; n < NM; ++n)
+        if (in_bounds((int64_t(g) * NM + n) * kSThreads + tid, p.n_carry))
+          p.carry[(int64_t(g) * NM + n) * kSThreads + tid] = gt[n];
       __threadfence();
       __syncthreads();
       if (tid == 0 && !(p.test_hook == 1 && g == 0 && r == 0)) st_release_gpu(p.flags + g, r + 1);
@@ -994,6 +1014,7 @@ __global__ void __launch_bounds__(kSThreads) bwd_adjoint_agg_kernel(const BwdSta
   // of 16 bytes and chunks start at multiples of 64 steps): every load of the V
   // steps is issued before it is used
   for (int64_t tb = tend - V; tb >= tbeg; tb -= V) {
+    if (!in_bounds(row + tb + V - 1, f.batch * f.dim * f.L)) break;
     float dv[V], dyv[V], zv[V];
     if constexpr (std::is_same<TD, T>::value) {
       Vec<T>::unpack(*reinterpret_cast<const uint4 *>(dl + tb), dv);
@@ -1042,8 +1063,10 @@ __global__ void __launch_bounds__(kSThreads) bwd_adjoint_agg_kernel(const BwdSta
   }
 #pragma unroll
   for (int n = 0; n < NM; ++n)
-    p.agg_G[((int64_t(g) * p.K + k) * NM + n) * kSThreads + threadIdx.x] = valid ? Ga[n] : 0.f;
-  p.agg_S[(int64_t(g) * p.K + k) * kSThreads + threadIdx.x] = valid ? S : 0.0;
+    if (in_bounds(((int64_t(g) * p.K + k) * NM + n) * kSThreads + threadIdx.x, p.n_gin))
+      p.agg_G[((int64_t(g) * p.K + k) * NM + n) * kSThreads + threadIdx.x] = valid ? Ga[n] : 0.f;
+  if (in_bounds((int64_t(g) * p.K + k) * kSThreads + threadIdx.x, p.n_unit))
+    p.agg_S[(int64_t(g) * p.K + k) * kSThreads + threadIdx.x] = valid ? S : 0.0;
 }
 
 // dB / dC: sum of the per-CTA partials over the channel groups of a batch row.
@@ -1230,6 +1253,11 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
   }
   bp.Rp = Rp;
   bp.stage_bytes = PROJ ? BwdStage<T, NM>(Rp).bytes : 0;
+  bp.n_ckpt = int64_t(n_ckpt);
+  bp.n_carry = int64_t(n_carry);
+  bp.n_bc = int64_t(n_bc);
+  bp.n_unit = int64_t(n_D);
+  bp.n_gin = int64_t(n_par);
   bp.timeout_ns = o.timeout_us > 0 ? uint64_t(o.timeout_us) * 1000ull : kDefaultTimeoutNs;
   bp.force_generic = o.path == MAMBA_PATH_GENERIC ? 1 : 0;
   bp.test_hook = o.test_hook;

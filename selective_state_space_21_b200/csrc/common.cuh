@@ -16,6 +16,21 @@ constexpr int kMaxN = 16;
 // translation unit that includes this header has its own copy.
 __device__ unsigned int g_error_word = 0;
 constexpr unsigned int kErrTimeout = 1u;
+constexpr unsigned int kErrBounds = 2u;
+
+// Index check of the bounds-checking build (MAMBA_DEBUG_BOUNDS): an index
+// outside [0, n) sets the sticky error word's bounds bit and the access that
+// it guards is skipped, so that a wrong index shows up as a status instead of
+// a fault.  In the normal build it is always true and costs nothing.
+#if defined(MAMBA_DEBUG_BOUNDS)
+__device__ __forceinline__ bool in_bounds(int64_t i, int64_t n) {
+  if (i >= 0 && i < n) return true;
+  atomicOr(&g_error_word, kErrBounds);
+  return false;
+}
+#else
+__device__ __forceinline__ constexpr bool in_bounds(int64_t, int64_t) { return true; }
+#endif
 
 // With conv_w set, `u` points at the input x of the Mamba block's causal
 // depthwise convolution, and the scan runs on u = SiLU(conv(x)) computed on

@@ -97,6 +97,9 @@ struct StagedArgs {
   uint32_t stage_bytes = 0;
   int nst = 0;
   float *delta_out = nullptr;
+  // element counts of the workspace buffers as allocated (the bounds-checking
+  // build checks every index against them)
+  int64_t n_carry = 0, n_agg = 0, n_aggS = 0, n_ckpt = 0;
 };
 
 // Fused Delta projection: TMEM columns of one CTA (W rows in [0, Rp/2), two
@@ -556,11 +559,17 @@ __global__ void __launch_bounds__(kSThreads, 2)
         break;
       }
 #pragma unroll
-      for (int n = 0; n < NM; ++n) hs[n] = __ldcg(p.carry + (int64_t(g) * NM + n) * kSThreads + tid);
+      for (int n = 0; n < NM; ++n) {
+        const int64_t i = (int64_t(g) * NM + n) * kSThreads + tid;
+        hs[n] = in_bounds(i, p.n_carry) ? __ldcg(p.carry + i) : 0.f;
+      }
     } else if (kPar && k > 0) {
 #pragma unroll
       for (int n = 0; n < NM; ++n)
-        hs[n] = __ldcg(p.hin + ((int64_t(g) * p.K + k) * NM + n) * kSThreads + tid);
+      {
+        const int64_t i = ((int64_t(g) * p.K + k) * NM + n) * kSThreads + tid;
+        hs[n] = in_bounds(i, p.n_agg) ? __ldcg(p.hin + i) : 0.f;
+      }
     }
 
     double Ssum = 0.0;  // sum of Delta over the chunk (aggregate pass)
@@ -573,9 +582,11 @@ __global__ void __launch_bounds__(kSThreads, 2)
         cf = load_conv_filter(f.conv_w, f.conv_b, f.conv_width, d);
         if (tbeg > 0) {  // chunks start at multiples of 64 steps
           const T *xr = static_cast<const T *>(f.u) + (int64_t(b) * f.dim + d) * f.L + tbeg;
-          xm3 = to_f(xr[-3]);
-          xm2 = to_f(xr[-2]);
-          xm1 = to_f(xr[-1]);
+          if (in_bounds((int64_t(b) * f.dim + d) * f.L + tbeg - 3, f.batch * f.dim * f.L)) {
+            xm3 = to_f(xr[-3]);
+            xm2 = to_f(xr[-2]);
+            xm1 = to_f(xr[-1]);
+          }
         }
       }
     }
@@ -656,8 +667,9 @@ __global__ void __launch_bounds__(kSThreads, 2)
           if constexpr (kCkpt) {
             const int64_t tj = t0 + int64_t(j) * VEC;
             if (tj % kCkptEvery == 0) {
-              float *dst = p.ckpt + ((int64_t(g) * ((f.L + kCkptEvery - 1) / kCkptEvery) +
-                                      tj / kCkptEvery) * NM) * kSThreads + tid;
+              const int64_t ci = ((int64_t(g) * ((f.L + kCkptEvery - 1) / kCkptEvery) +
+                                   tj / kCkptEvery) * NM) * kSThreads + tid;
+              float *dst = p.ckpt + (in_bounds(ci + (NM - 1) * kSThreads, p.n_ckpt) ? ci : 0);
               if constexpr (M == MODE_GEN) {
 #pragma unroll
                 for (int n = 0; n < NM; ++n) dst[n * kSThreads] = h[n];
@@ -688,7 +700,8 @@ __global__ void __launch_bounds__(kSThreads, 2)
             static_assert(VEC == 8, "eight steps per 16-byte chunk");
             tmem_ld8(dacc + uint32_t(j) * 8u, dv);
             tmem_ld_wait();
-            if (p.delta_out && valid) {
+            if (p.delta_out && valid &&
+                in_bounds((int64_t(b) * f.dim + d) * f.L + t0 + int64_t(j) * VEC + 7, f.batch * f.dim * f.L)) {
               float *o = p.delta_out + (int64_t(b) * f.dim + d) * f.L + t0 + int64_t(j) * VEC;
               *reinterpret_cast<float4 *>(o) = make_float4(dv[0], dv[1], dv[2], dv[3]);
               *reinterpret_cast<float4 *>(o + 4) = make_float4(dv[4], dv[5], dv[6], dv[7]);
@@ -786,17 +799,22 @@ __global__ void __launch_bounds__(kSThreads, 2)
     if (kAgg) {
 #pragma unroll
       for (int n = 0; n < NM; ++n)
-        p.agg_h[((int64_t(g) * p.K + k) * NM + n) * kSThreads + tid] = hs[n];
-      p.agg_S[(int64_t(g) * p.K + k) * kSThreads + tid] = Ssum;
+        if (in_bounds(((int64_t(g) * p.K + k) * NM + n) * kSThreads + tid, p.n_agg))
+          p.agg_h[((int64_t(g) * p.K + k) * NM + n) * kSThreads + tid] = hs[n];
+      if (in_bounds((int64_t(g) * p.K + k) * kSThreads + tid, p.n_aggS))
+        p.agg_S[(int64_t(g) * p.K + k) * kSThreads + tid] = Ssum;
     } else if (k == p.K - 1) {
       if (kOut && valid && f.last_state) {
 #pragma unroll
         for (int n = 0; n < NM; ++n)
-          if (n < N) f.last_state[(int64_t(b) * f.dim + d) * N + n] = hs[n];
+          if (n < N && in_bounds((int64_t(b) * f.dim + d) * N + n, f.batch * f.dim * N))
+            f.last_state[(int64_t(b) * f.dim + d) * N + n] = hs[n];
       }
     } else if (kSeq) {
 #pragma unroll
-      for (int n = 0; n < NM; ++n) p.carry[(int64_t(g) * NM + n) * kSThreads + tid] = hs[n];
+      for (int n = 0; n < NM; ++n)
+        if (in_bounds((int64_t(g) * NM + n) * kSThreads + tid, p.n_carry))
+          p.carry[(int64_t(g) * NM + n) * kSThreads + tid] = hs[n];
       __threadfence();
       __syncthreads();
       if (tid == 0 && !(p.test_hook == 1 && g == 0 && k == 0)) st_release_gpu(p.flags + g, k + 1);
@@ -851,6 +869,7 @@ struct ChunkScanIO {
   int G, K, gpb, N;
   int64_t dim;
 };
+// (its buffers hold G * K * 128 and G * K * NM * 128 elements)
 
 template <int NM, bool REVERSE>
 __global__ void __launch_bounds__(128) chunk_scan_kernel(const ChunkScanIO io) {
@@ -866,7 +885,8 @@ __global__ void __launch_bounds__(128) chunk_scan_kernel(const ChunkScanIO io) {
   for (int k0 = 0; k0 < io.K; k0 += 128) {
     const int e = k0 + threadIdx.x;  // element of the scan
     const int k = REVERSE ? io.K - 1 - e : e;
-    const bool live = e < io.K - 1;  // the last element's map is never applied
+    const int64_t nk = int64_t(io.G) * io.K;
+    const bool live = e < io.K - 1 && in_bounds(int64_t(g) * io.K + k, nk);  // the last map is never applied
     const int64_t base = int64_t(g) * io.K + (live ? k : 0);
     double S = live ? io.S[base * kSThreads + c] : 0.0;
     double h = live ? double(io.hl[(base * NM + n) * kSThreads + c]) : 0.0;
@@ -895,7 +915,8 @@ __global__ void __launch_bounds__(128) chunk_scan_kernel(const ChunkScanIO io) {
       Se = 0.0;
       he = 0.0;
     }
-    if (e < io.K) io.hin[((int64_t(g) * io.K + k) * NM + n) * kSThreads + c] = float(exp(An * Se) * cin + he);
+    if (e < io.K && in_bounds(int64_t(g) * io.K + k, nk))
+      io.hin[((int64_t(g) * io.K + k) * NM + n) * kSThreads + c] = float(exp(An * Se) * cin + he);
     __syncthreads();
     if (threadIdx.x == 127) carry = exp(An * S) * cin + h;  // through the whole block
     __syncthreads();
@@ -928,17 +949,20 @@ __global__ void __launch_bounds__(kSThreads) fwd_correct_kernel(const StagedArgs
   bool any = false;
 #pragma unroll
   for (int n = 0; n < NM; ++n) {
-    hin[n] = __ldcg(p.hin + ((int64_t(g) * p.K + k) * NM + n) * kSThreads + c);
+    const int64_t hi = ((int64_t(g) * p.K + k) * NM + n) * kSThreads + c;
+    hin[n] = in_bounds(hi, p.n_agg) ? __ldcg(p.hin + hi) : 0.f;
     An[n] = n < N ? f.A[int64_t(d) * N + n] : -float(n + 1);
     any = any || (n < N && hin[n] != 0.f);
   }
   const int64_t tbeg = int64_t(k) * p.chunk_len;
   const int64_t tend = std::min<int64_t>(f.L, tbeg + p.chunk_len);
   if (k == p.K - 1 && f.last_state) {  // the true final state
-    const double S = p.agg_S[(int64_t(g) * p.K + k) * kSThreads + c];
+    const int64_t si = (int64_t(g) * p.K + k) * kSThreads + c;
+    const double S = in_bounds(si, p.n_aggS) ? p.agg_S[si] : 0.0;
 #pragma unroll
     for (int n = 0; n < NM; ++n)
-      if (n < N) {
+      if (n < N && in_bounds(((int64_t(g) * p.K + k) * NM + n) * kSThreads + c, p.n_agg) &&
+          in_bounds((int64_t(b) * f.dim + d) * N + n, f.batch * f.dim * N)) {
         const float hl = __ldcg(p.agg_h + ((int64_t(g) * p.K + k) * NM + n) * kSThreads + c);
         f.last_state[(int64_t(b) * f.dim + d) * N + n] = hl + float(exp(double(An[n]) * S)) * hin[n];
       }
@@ -960,6 +984,9 @@ __global__ void __launch_bounds__(kSThreads) fwd_correct_kernel(const StagedArgs
   // the chunk starts at a multiple of 64 steps and rows are 16-byte multiples
   for (int64_t t0 = tbeg; t0 < tend; t0 += V) {
     if (amax * cum < -22.2f) break;  // exp(amax cumDelta) < 2^-32
+    if (!in_bounds(row + t0 + V - 1, f.batch * f.dim * f.L) ||
+        !in_bounds(int64_t(b) * N * f.L + int64_t(N - 1) * f.L + t0 + V - 1, f.batch * N * f.L))
+      break;
     float dv[V], zv[V], yv[V];
     Vec<T>::unpack(*reinterpret_cast<const uint4 *>(dl + t0), dv);
     Vec<T>::unpack(*reinterpret_cast<const uint4 *>(yr + t0), yv);
@@ -1178,6 +1205,10 @@ struct StagedForward {
     int *counters = reinterpret_cast<int *>(ws);
     sa.flags = counters + 2;
     const size_t gk = size_t(sa.G) * size_t(pl.K);
+    sa.n_carry = int64_t(sa.G) * NM * kSThreads;
+    sa.n_agg = int64_t(gk) * NM * kSThreads;
+    sa.n_aggS = int64_t(gk) * kSThreads;
+    sa.n_ckpt = int64_t(sa.G) * ((sa.f.L + kCkptEvery - 1) / kCkptEvery) * NM * kSThreads;
     if (pl.kind == KIND_SEQ) {
       sa.carry = reinterpret_cast<float *>(ws + int_bytes);
       sa.counter = counters;

@@ -494,6 +494,7 @@ const char *mamba_scan_status_string(mamba_status_t s) {
     case MAMBA_ERR_CUDA: return "MAMBA_ERR_CUDA";
     case MAMBA_ERR_OUT_OF_MEMORY: return "MAMBA_ERR_OUT_OF_MEMORY";
     case MAMBA_ERR_DEVICE_TIMEOUT: return "MAMBA_ERR_DEVICE_TIMEOUT";
+    case MAMBA_ERR_OUT_OF_BOUNDS: return "MAMBA_ERR_OUT_OF_BOUNDS";
   }
   return "MAMBA_ERR_UNKNOWN";
 }
@@ -509,7 +510,8 @@ mamba_status_t mamba_scan_stream_status(mamba_stream_t stream) {
     cudaGetLastError();
     return MAMBA_ERR_CUDA;
   }
-  return (word & kErrTimeout) ? MAMBA_ERR_DEVICE_TIMEOUT : MAMBA_OK;
+  if (word & kErrTimeout) return MAMBA_ERR_DEVICE_TIMEOUT;
+  return (word & kErrBounds) ? MAMBA_ERR_OUT_OF_BOUNDS : MAMBA_OK;
 }
 
 mamba_status_t mamba_scan_fwd_ex(const void *u, const void *delta, const float *delta_bias,
@@ -1347,7 +1349,6 @@ void mamba_scan_test_fail_alloc(int32_t after) { alloc_failure_countdown() = aft
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // per device
-constexpr size_t kNoAllocIntBytes = size_t(64) << 10;     // ticket counter + group flags
 constexpr int kNoAllocMaxDevices = 64;
 
 }  // namespace
@@ -1377,59 +1378,43 @@ mamba_status_t noalloc_scratch(int dev, unsigned char **out) {
   return MAMBA_OK;
 }
 
-// The staged forward with the sequential hand-off, its scratch carved out of
-// the fixed array.  Enqueues a memset of the counter and flags and one kernel.
+// The staged forward with its workspace carved out of the fixed array: the
+// plan the regular call would take (the sequential hand-off when the channel
+// groups fill the GPU, else chunks from zero with the parallel scan over
+// chunks and the closed-form correction) when its workspace fits; for the
+// latter, fewer and longer chunks until it does; else the sequential
+// hand-off.  Enqueues a memset of the counters and flags and the kernels.
 template <typename T, int NM>
 mamba_status_t noalloc_forward(const FwdArgs &a, unsigned char *scratch, cudaStream_t s) {
-  using Lay = StagedLayout<T, NM>;
-  constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
-  const uint64_t L = a.L, dim = a.dim, batch = a.batch, N = a.N;
-  const int64_t gpb = ceil_div(a.dim, kSThreads);
-  const int64_t G = int64_t(a.batch) * gpb;
-  // the limit: counter + flags in the first 64 KiB, one carried state per group after it
-  if (size_t(G + 1) * 4 > kNoAllocIntBytes ||
-      size_t(G) * NM * kSThreads * 4 > kNoAllocScratchBytes - kNoAllocIntBytes)
-    return MAMBA_ERR_UNSUPPORTED;
-  CUtensorMap maps[6];
-  const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_64B, none = CU_TENSOR_MAP_SWIZZLE_NONE;
-  if (!make_map_3d(&maps[0], a.u, bf16, L, dim, batch, Lay::TT, kSThreads, sw) ||
-      !make_map_3d(&maps[1], a.delta, bf16, L, dim, batch, Lay::TT, kSThreads, sw) ||
-      !make_map_3d(&maps[2], a.z ? a.z : a.u, bf16, L, dim, batch, Lay::TT, kSThreads, sw) ||
-      !make_map_3d(&maps[3], a.y, bf16, L, dim, batch, Lay::TT, kSThreads, sw) ||
-      !make_map_3d(&maps[4], a.B, bf16, L, N, batch, Lay::TT, uint32_t(N), none) ||
-      !make_map_3d(&maps[5], a.C, bf16, L, N, batch, Lay::TT, uint32_t(N), none))
-    return MAMBA_ERR_UNSUPPORTED;
-  int bps = 0;
-  if (prepare_kernel<T, NM, KIND_SEQ>(&bps) != cudaSuccess) return MAMBA_ERR_CUDA;
-  const int slots = device_sm_count() * std::max(1, bps);
   StagedOptions o;
   o.path = MAMBA_PATH_AUTO;
   o.chunk_len = 0;
-  o.carry = 1;
+  o.carry = 0;
   o.timeout_us = 0;
   o.test_hook = 0;
-  const StagedPlan pl = plan_staged(G, a.L, slots, o);
-  if (G * pl.K > (int64_t(1) << 30)) return MAMBA_ERR_UNSUPPORTED;
-  StagedArgs sa;
-  sa.f = a;
-  sa.G = int(G);
-  sa.gpb = int(gpb);
-  sa.K = pl.K;
-  sa.chunk_len = pl.chunk_len;
-  sa.n_units = int(G * pl.K);
-  sa.counter = reinterpret_cast<int *>(scratch);
-  sa.flags = sa.counter + 1;
-  sa.carry = reinterpret_cast<float *>(scratch + kNoAllocIntBytes);
-  sa.agg_h = sa.hin = sa.ckpt = nullptr;
-  sa.agg_S = nullptr;
-  sa.timeout_ns = kDefaultTimeoutNs;
-  sa.test_hook = 0;
-  sa.force_generic = 0;
-  // The array keeps whatever the previous call left: the counter and the
-  // flags must start at zero (the carried states are written before read).
-  if (cudaMemsetAsync(scratch, 0, size_t(G + 1) * 4, s) != cudaSuccess) return cuda_status();
-  launch_staged<T, NM, KIND_SEQ>(maps, sa, int(std::min<int64_t>(G * pl.K, slots)), s);
-  return launch_status();
+  StagedForward<T, NM> sf;
+  mamba_status_t st = sf.prepare(a, o, nullptr);
+  if (st != MAMBA_OK) return st;
+  if (sf.pl.kind == KIND_PAR && sf.bytes > kNoAllocScratchBytes) {
+    for (int64_t chunk = int64_t(sf.pl.chunk_len) * 2; chunk < a.L && chunk < (int64_t(1) << 30);
+         chunk *= 2) {
+      o.carry = 2;
+      o.chunk_len = int(chunk);
+      if ((st = sf.prepare(a, o, nullptr)) != MAMBA_OK) return st;
+      if (sf.bytes <= kNoAllocScratchBytes) break;
+    }
+  }
+  if (sf.bytes > kNoAllocScratchBytes || sf.pl.K < 2) {
+    o.carry = 1;
+    o.chunk_len = 0;
+    if ((st = sf.prepare(a, o, nullptr)) != MAMBA_OK) return st;
+  }
+  // the limit: what the sequential hand-off needs (counters, one flag and one
+  // carried state per channel group) must fit the array
+  if (sf.bytes > kNoAllocScratchBytes) return MAMBA_ERR_UNSUPPORTED;
+  // The array keeps whatever the previous call left: run() clears the
+  // counters and flags first; every other word is written before it is read.
+  return sf.run(scratch, s, &launch_status);
 }
 
 }  // namespace

@@ -22,14 +22,18 @@ from typing import Optional
 
 import torch
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libmambascan.so")
+# MAMBA_SCAN_LIBRARY selects another build of the same library (the
+# bounds-checking libmambascan_debug.so, for the tests that run against it).
+_LIB_PATH = os.environ.get("MAMBA_SCAN_LIBRARY") or os.path.join(
+    os.path.dirname(os.path.abspath(__file__)), "lib", "libmambascan.so")
 
 MAMBA_F32, MAMBA_BF16 = 0, 1
 PATH_AUTO, PATH_REFERENCE, PATH_GENERIC, PATH_STRUCTURED = 0, 1, 2, 3
 PATHS = {"auto": PATH_AUTO, "reference": PATH_REFERENCE, "generic": PATH_GENERIC,
          "structured": PATH_STRUCTURED}
 STATUS = {0: "MAMBA_OK", 1: "MAMBA_ERR_INVALID_ARG", 2: "MAMBA_ERR_UNSUPPORTED",
-          3: "MAMBA_ERR_CUDA", 4: "MAMBA_ERR_OUT_OF_MEMORY", 5: "MAMBA_ERR_DEVICE_TIMEOUT"}
+          3: "MAMBA_ERR_CUDA", 4: "MAMBA_ERR_OUT_OF_MEMORY", 5: "MAMBA_ERR_DEVICE_TIMEOUT",
+          6: "MAMBA_ERR_OUT_OF_BOUNDS"}
 
 
 class MambaScanError(RuntimeError):

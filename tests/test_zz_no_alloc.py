@@ -37,20 +37,33 @@ def _regular(x):
 
 
 def _noalloc_twice(x):
+    """Two calls in a row, each with the library's allocation-failure hook
+    armed (any workspace allocation the call made would fail it with
+    MAMBA_ERR_OUT_OF_MEMORY) and with its workspace pool emptied first (the
+    call must leave it empty)."""
     out = []
     for _ in range(2):
         y = torch.full_like(x["u"], float("nan"))
         last = torch.full((x["u"].shape[0], x["u"].shape[1], x["A"].shape[1]), float("nan"),
                           device="cuda")
-        scan.mamba_scan_fwd_noalloc(x["u"], x["delta"], x["delta_bias"], x["A"], x["B"], x["C"],
-                                    x["D"], x["z"], y, last)
+        torch.cuda.synchronize()
+        scan.pool_trim(0)
+        reserved0 = scan.pool_reserved()
+        scan.test_fail_alloc(0)
+        try:
+            scan.mamba_scan_fwd_noalloc(x["u"], x["delta"], x["delta_bias"], x["A"], x["B"],
+                                        x["C"], x["D"], x["z"], y, last)
+        finally:
+            scan.test_fail_alloc(-1)
         assert scan.mamba_scan_stream_status() == 0
+        assert scan.pool_reserved() == reserved0 == 0
         out.append((y, last))
     return out
 
 
 CASES = [  # (batch, dim, L, N, dtype): chunked hand-off, several group counts, N rounding,
     (8, 5120, 2048, 16, torch.bfloat16),  # the full bf16 2K-length workload
+    (1, 1536, 65536, 16, torch.bfloat16),  # few groups, long: chunks from zero, scan, correction
     (2, 300, 1024, 16, torch.float32),
     (3, 200, 1000, 8, torch.bfloat16),
     (1, 129, 512, 3, torch.float32),
@@ -75,8 +88,11 @@ def test_noalloc_matches_regular_forward_on_two_calls(case):
 
 
 def test_noalloc_rejects_problems_beyond_the_array():
-    """1024 channel groups of N = 16 need more than the fixed scratch holds:
-    the call is refused on the host and nothing is written."""
+    """1024 channel groups of N = 16 need more than the fixed scratch holds
+    even for the sequential hand-off: the call is refused on the host and
+    nothing is written (the scratch-free one-thread-per-channel kernel is
+    10-50 times slower, and a caller who sized for the fast path should
+    learn that its problem is beyond it)."""
     x = gc.to_device(make_inputs(8, 16384, 8, 16, torch.bfloat16, seed=9))
     y = torch.zeros_like(x["u"])
     with pytest.raises(scan.MambaScanError) as e:
