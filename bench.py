@@ -308,6 +308,13 @@ def run_ours(args, world, rank, device):
             w = dataclasses.replace(w, batch=args.cplx_batch)
         res = run_cplx(w, device, measured_peaks(), steps=args.steps)
         return {"note": "--only cplx: a profiling run, not a benchmark result", "complex_A": res}
+    if args.only == "dtproj":  # the projection calls alone, for profiling
+        if args.cplx_batch:
+            w = dataclasses.replace(w, batch=args.cplx_batch)
+        xp = make_inputs(w.batch, w.dim, w.L, w.N, w.dtype, device=device, seed=1234 + args.workload,
+                         has_z=w.has_z, has_D=w.has_D, with_dy=True)
+        res = run_dtproj(w, xp, device, steps=args.steps)
+        return {"note": "--only dtproj: a profiling run, not a benchmark result", "dt_projection": res}
     x = make_inputs(w.batch, w.dim, w.L, w.N, w.dtype, device=device,
                     seed=shard_seed(1234 + args.workload, rank), has_z=w.has_z,
                     has_D=w.has_D, with_dy=True)
@@ -945,11 +952,11 @@ def main(argv=None):
                          "then uses the nominal peak)")
     ap.add_argument("--micro", action="store_true",
                     help="run only the instruction-throughput microbenchmark and print it")
-    ap.add_argument("--only", choices=["fwd", "bwd", "cplx"], default=None,
-                    help="time one pass, or the complex-A calls, only (for profiling; "
-                         "not a benchmark result)")
+    ap.add_argument("--only", choices=["fwd", "bwd", "cplx", "dtproj"], default=None,
+                    help="time one pass, or the complex-A or projection calls, only (for "
+                         "profiling; not a benchmark result)")
     ap.add_argument("--cplx-batch", type=int, default=0,
-                    help="batch of the complex-A calls with --only cplx (0: the workload's)")
+                    help="batch of the calls with --only cplx / dtproj (0: the workload's)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

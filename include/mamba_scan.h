@@ -220,11 +220,18 @@ MAMBA_SCAN_API mamba_status_t mamba_conv_scan_bwd(
  * and delta_bias is Linear_D's bias (softplus(delta + delta_bias) as before).
  *   dt_low : (batch, R, L) dtype
  *   W_dt   : (dim, R) dtype (the I/O type, like a bf16 layer weight)
- * Everything else as in mamba_scan_fwd_ex.  The contraction runs on the
- * tensor cores through cuBLAS (fp32 accumulation, result rounded once to the
- * I/O type) into a stream-ordered workspace of delta's size that the scan
- * reads; cuBLAS is opened at run time (libcublas.so.12), and without it the
- * call returns MAMBA_ERR_UNSUPPORTED.  R in 1..2^20; dim and L below 2^31.
+ * Everything else as in mamba_scan_fwd_ex.  R in 1..2^20; dim and L below
+ * 2^31.  How delta is formed:
+ *   - bf16 with R <= 192, the staged kernels' shapes (L a multiple of 8,
+ *     16-byte aligned rows) and no MAMBA_PATH_REFERENCE: delta never reaches
+ *     memory.  Each CTA keeps its 128 rows of W_dt in tensor memory and forms
+ *     every 128-channel x 32-step tile of delta with one tensor-core MMA
+ *     (tcgen05, fp32 accumulation) from the dt_low tile that the scan's own
+ *     TMA pipeline brings in; the scan uses the fp32 result as it is.
+ *   - otherwise: delta is formed first by a CUDA-core contraction (fp32
+ *     accumulation, rounded once to the I/O type) into a stream-ordered
+ *     workspace of delta's size, and the regular scan reads it.
+ * No external library is called.
  */
 MAMBA_SCAN_API mamba_status_t mamba_dtproj_scan_fwd(const void *u, const void *dt_low,
                                                     const void *W_dt, int64_t R,
@@ -243,7 +250,13 @@ MAMBA_SCAN_API mamba_status_t mamba_dtproj_scan_fwd(const void *u, const void *d
  *     d_dt_low[b] = W_dt^T . ddelta[b],   dW_dt = sum_b ddelta[b] . dt_low[b]^T
  * where ddelta (the scan backward's gradient of delta, rounded once to the
  * I/O type) lives in a workspace.  dW_dt is accumulated over the batch rows
- * in a fixed order.
+ * in a fixed order.  Where the forward fuses the projection, so does the
+ * backward (delta recomputed per tile on the tensor cores, never stored);
+ * otherwise delta comes from the CUDA-core contraction into the workspace.
+ * The two products run as tcgen05 GEMMs (bf16 operands, fp32 accumulation;
+ * dW_dt's contraction over batch x L split across the grid and the parts
+ * summed in a fixed order) for bf16 with R and L multiples of 8, R <= 256 and
+ * 16-byte aligned W_dt / dt_low, else on the CUDA cores.
  */
 MAMBA_SCAN_API mamba_status_t mamba_dtproj_scan_bwd(
     const void *u, const void *dt_low, const void *W_dt, int64_t R, const float *delta_bias,

@@ -56,7 +56,7 @@ struct BwdLayout {
   // which leaves room for four-step segments only.
   static constexpr int SEG = sizeof(T) == 2 ? 2 : 4;
   static constexpr int NSEG = kBTT / SEG;
-  static constexpr int BSTR = NM + 4;
+  static constexpr int BSTR = NM;  // rows of B / C are read as broadcasts; no padding
   static constexpr int OFF_SUB = kBStages * STAGE;
   static constexpr int OFF_BS = OFF_SUB + NSEG * NM * kSThreads * 4;
   static constexpr int OFF_CS = OFF_BS + kBTT * BSTR * 4;
@@ -108,7 +108,13 @@ struct BwdStagedArgs {
   // element counts of the workspace buffers as allocated (the bounds-checking
   // build checks every index against them)
   int64_t n_ckpt = 0, n_carry = 0, n_bc = 0, n_unit = 0, n_gin = 0;
+  // [G][ceil(L/64)]: 1 where some channel's delta leaves the range the
+  // structured forms take (null: no check; the fused projection checks per tile)
+  const unsigned char *range_flags = nullptr;
+  int64_t n_flags = 0;
 };
+constexpr int kRangeBlock = 64;   // steps per range flag
+constexpr int kRangeSpan = 512;   // steps per CTA of delta_range_kernel
 
 // Byte offset of 16-byte chunk c of row r in a tile with RB-byte rows written
 // by TMA with RB-byte swizzling (chunk index XOR address bits from bit 7 up).
@@ -178,11 +184,12 @@ __device__ __forceinline__ float bfly_rest(float (&v)[16], int lane) {
   return v[0];
 }
 
-// Smallest and largest delta of thread `r`'s row in a 16-step tile: from the
-// tile in shared memory (swizzled rows), or (PROJ) from its TMEM accumulator.
+// Whether any step of thread `r`'s row in a 16-step tile has its delta in
+// [lo, hi]: from the tile in shared memory (swizzled rows), or (PROJ) from its
+// TMEM accumulator.
 template <typename T, bool PROJ>
-__device__ __forceinline__ void tile_delta_range(const unsigned char *tile, uint32_t dacc, int r,
-                                                 float &mn, float &mx) {
+__device__ __forceinline__ bool tile_delta_in_range(const unsigned char *tile, uint32_t dacc, int r,
+                                                    float lo, float hi) {
   float v[kBTT];
   if constexpr (PROJ) {
     float a[8], b[8];
@@ -204,13 +211,10 @@ __device__ __forceinline__ void tile_delta_range(const unsigned char *tile, uint
       for (int i = 0; i < Vec<T>::kN; ++i) v[c * Vec<T>::kN + i] = o[i];
     }
   }
-  mn = v[0];
-  mx = v[0];
+  bool in = false;
 #pragma unroll
-  for (int i = 1; i < kBTT; ++i) {
-    mn = fminf(mn, v[i]);
-    mx = fmaxf(mx, v[i]);
-  }
+  for (int i = 0; i < kBTT; ++i) in = in || (v[i] >= lo && v[i] <= hi);
+  return in;
 }
 
 // Four consecutive x values of a row (16-byte aligned for float, 8-byte for
@@ -228,6 +232,21 @@ __device__ __forceinline__ void load_x4(const __nv_bfloat16 *p, float (&o)[4]) {
   o[1] = __uint_as_float(v.x & 0xffff0000u);
   o[2] = __uint_as_float(v.y << 16);
   o[3] = __uint_as_float(v.y & 0xffff0000u);
+}
+
+// Where the backward's structured forms keep their relative accuracy:
+// Delta |A_0| in [1e-5, 6].  Above, the decay chain keeps the small decays'
+// absolute but not their relative accuracy, which ddelta needs; below, the dA
+// identity A dh/dA = Delta dh/dDelta - Bbar u cancels.  Either way the error
+// is at fp32 resolution of the terms of a step in the range, so it matters
+// only where no step is: a unit (or, with the fused projection, a tile) in
+// which every step of every channel lies outside takes the generic
+// arithmetic.  In terms of v = delta (before the bias): [lo, hi] with
+// softplus(lo + bias) = 1e-5 / |A_0| and softplus(hi + bias) = 6 / |A_0|.
+__device__ __forceinline__ void structured_delta_range(float A0, float bias, float &lo, float &hi) {
+  const float ylo = 1e-5f / fabsf(A0), yhi = 6.f / fabsf(A0);
+  lo = logf(expm1f(ylo)) - bias;
+  hi = yhi + logf(-expm1f(-yhi)) - bias;
 }
 
 // CONV: the u tiles hold the input x of the block's causal depthwise
@@ -314,7 +333,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
     tbase = uint32_t(q[12]);
   }
 
-  // Issues (thread 0) the projection MMAs of consumed-tile index `ct` into
+  // Issues (kMmaThread) the projection MMAs of consumed-tile index `ct` into
   // accumulator ct & 1 once the tile's dt_low rows have landed: 16 rows of
   // 32 bytes (two 256-byte swizzle atoms) per MMA.
   [[maybe_unused]] auto issue_mma = [&](int ct) {
@@ -415,28 +434,38 @@ __global__ void __launch_bounds__(kSThreads, 2)
     const bool sig = structured && Arow[0] == -1.f;
     if constexpr (PROJ) {
       // this group's rows of W_dt into TMEM (as in the forward's fused projection)
-      const __nv_bfloat16 *wrow = static_cast<const __nv_bfloat16 *>(f.W_dt) +
-                                  (valid ? int64_t(d) * f.R : 0);
-      for (int c8 = 0; c8 < p.Rp / 16; ++c8) {
-        uint32_t r[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int k = 16 * c8 + 2 * i;
-          const uint32_t lo = (valid && k < f.R) ? __bfloat16_as_ushort(wrow[k]) : 0u;
-          const uint32_t hi = (valid && k + 1 < f.R) ? __bfloat16_as_ushort(wrow[k + 1]) : 0u;
-          r[i] = lo | (hi << 16);
-        }
-        tmem_st8(tmem_at(tbase, uint32_t(warp) * 32u, uint32_t(c8) * 8u), r);
-      }
+      proj_load_w(static_cast<const __nv_bfloat16 *>(f.W_dt), d, valid, f.R, p.Rp,
+                  tmem_at(tbase, uint32_t(warp) * 32u, 0));
       tmem_st_wait();
       tc_fence_before_sync();
       __syncthreads();
-      if (tid == 0) issue_mma(ctile);
+      if (tid == kMmaThread) issue_mma(ctile);
+    }
+    // The structured arithmetic keeps its relative accuracy for Delta |A0| in
+    // 1e-5 .. 6: below, its dA cancels (Delta Abar B u against Bbar u); above,
+    // its Abar = 1 + expm1 has only absolute accuracy, and ddelta (~Abar) loses
+    // it.  A unit none of whose steps is in that range takes the generic
+    // arithmetic (one exp per state, dA through psi'), which has neither
+    // problem.  (The fused projection's kernels, whose delta is formed tile by
+    // tile, decide per tile.)
+    bool unit_extreme = false;
+    if constexpr (!PROJ) {  // the unit's range flags (delta_range_kernel): all set?
+      if (p.range_flags) {
+        const int64_t nblk = (f.L + kRangeBlock - 1) / kRangeBlock;
+        const int64_t ub = int64_t(k) * p.chunk_len;
+        const int64_t ue = std::min<int64_t>(f.L, ub + p.chunk_len);
+        unit_extreme = true;
+        for (int64_t i = ub / kRangeBlock + tid; i < (ue + kRangeBlock - 1) / kRangeBlock; i += kSThreads) {
+          const int64_t fi = int64_t(g) * nblk + i;
+          if (in_bounds(fi, p.n_flags) && !p.range_flags[fi]) unit_extreme = false;
+        }
+      }
     }
     int mode = MODE_GEN;
     if (!p.force_generic) {
-      if (__syncthreads_and(sig)) mode = MODE_SIG;
-      else if (__syncthreads_and(structured)) mode = MODE_STRUCT;
+      const bool ext = __syncthreads_and(unit_extreme);
+      if (!ext && __syncthreads_and(sig)) mode = MODE_SIG;
+      else if (!ext && __syncthreads_and(structured)) mode = MODE_STRUCT;
     }
 
     // adjoint entering from the later chunk
@@ -478,14 +507,8 @@ __global__ void __launch_bounds__(kSThreads, 2)
       constexpr bool kS = M != MODE_GEN;
       const float A0 = Arow[0];
       const float invA0 = 1.f / A0;
-      // delta below d_lo or above d_hi gives Delta |A0| below 1e-5 or above 6
-      // (inverse softplus of those, less the bias)
-      [[maybe_unused]] float d_lo = 0.f, d_hi = 0.f;
-      if constexpr (kS) {
-        const float ylo = 1e-5f / fabsf(A0), yhi = 6.f / fabsf(A0);
-        d_lo = logf(expm1f(ylo)) - bias;
-        d_hi = yhi + logf(-expm1f(-yhi)) - bias;
-      }
+      [[maybe_unused]] float d_lo = 0.f, d_hi = 0.f;  // the structured forms' range of delta
+      if constexpr (kS && PROJ) structured_delta_range(A0, bias, d_lo, d_hi);
       // per-mode state: pairs for the structured arithmetic, scalars otherwise
       f2 Gt[NP], Acc[NP];
       float gs[NM], accs[NM], A2[NM], invA[NM];
@@ -575,10 +598,10 @@ __global__ void __launch_bounds__(kSThreads, 2)
           }
         }
         bool tile_gen = false;
-        if constexpr (kS) {  // any step of the tile outside the structured range?
-          float dmin = 0.f, dmax = 0.f;
-          tile_delta_range<T, PROJ>(st + Lay::TILE, dacc, tid, dmin, dmax);
-          tile_gen = __syncthreads_or(valid && (dmax > d_hi || dmin < d_lo));
+        if constexpr (kS && PROJ) {  // no step of the tile in the structured range?
+          // (every thread reads its row: the TMEM load is warp-collective)
+          const bool in = tile_delta_in_range<T, PROJ>(st + Lay::TILE, dacc, tid, d_lo, d_hi);
+          tile_gen = !__syncthreads_or(valid && in);
         } else {
           __syncthreads();
         }
@@ -693,7 +716,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
 
           // the next tile's projection MMA, into the other accumulator
           if constexpr (PROJ) {
-            if (tid == 0 && it + 1 < ntiles) issue_mma(ctile + 1);
+            if (tid == kMmaThread && it + 1 < ntiles) issue_mma(ctile + 1);
             __syncwarp();
           }
 
@@ -859,9 +882,9 @@ __global__ void __launch_bounds__(kSThreads, 2)
             }
           }
         };
-        if constexpr (kS) {
+        if constexpr (kS && PROJ) {
           if (tile_gen) {
-            // A step of this tile has Delta |A0| outside the range where the
+            // No step of this tile has Delta |A0| in the range where the
             // structured arithmetic keeps its relative accuracy (1e-5 .. 6):
             // the tile runs the generic arithmetic (one exp per state, dA
             // through psi'), whose dA has no cancellation at small Delta and
@@ -883,7 +906,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
             tile_body(std::true_type{});
           }
         } else {
-          tile_body(std::false_type{});
+          tile_body(std::integral_constant<bool, kS>{});
         }
         if (PROJ) tc_fence_before_sync();
         __syncthreads();
@@ -957,7 +980,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
       mbar_wait_bounded(&bars[t % kBStages], uint32_t(t / kBStages) & 1u, p.timeout_ns);
   }
   if constexpr (PROJ) {  // every MMA issued must complete before TMEM is freed
-    if (tid == 0 && mma_issued >= 0)
+    if (tid == kMmaThread && mma_issued >= 0)
       mbar_wait_bounded(&mma_bar[mma_issued & 1], uint32_t(mma_issued >> 1) & 1u, p.timeout_ns);
     tc_fence_before_sync();
     __syncthreads();
@@ -966,6 +989,62 @@ __global__ void __launch_bounds__(kSThreads, 2)
       tmem_dealloc(tbase, kProjTmemCols);
     }
   }
+}
+
+// One flag per channel group and 64-step block: whether no step of any
+// channel of the group has its delta in structured_delta_range there
+// (channels whose A_0 is not negative take the generic arithmetic anyway and
+// are not checked).  Each CTA takes (group, 512-step span) units in turn, one
+// thread per channel; the reverse sweep takes the generic arithmetic for a
+// unit all of whose blocks are flagged.
+template <typename T, int V, int PER>
+__device__ __forceinline__ void delta_range_unit(const BwdStagedArgs &p, int g, int64_t t0, int64_t nblk) {
+  const BwdArgs &w = p.w;
+  const int b = g / p.gpb, d = (g % p.gpb) * kSThreads + int(threadIdx.x);
+  const float A0 = d < w.dim ? w.A[int64_t(d) * w.N] : 0.f;
+  const bool check = d < w.dim && A0 < 0.f && isfinite(A0);
+  float lo = 0.f, hi = 0.f;
+  if (check) structured_delta_range(A0, w.bias ? w.bias[d] : 0.f, lo, hi);
+  const int64_t row = (int64_t(b) * w.dim + (check ? d : 0)) * w.L;
+  const T *dl = static_cast<const T *>(w.delta) + row;
+  for (int j = 0; j < kRangeSpan / kRangeBlock; ++j) {
+    const int64_t tb = t0 + int64_t(j) * kRangeBlock;
+    if (tb >= w.L) break;  // (uniform over the CTA)
+    bool in = false;
+    if (check) {
+      uint4 raw[PER];
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {  // rows are 16-byte multiples: whole vectors up to L
+        const int64_t t = tb + int64_t(i) * V;
+        raw[i] = (t < w.L && in_bounds(row + t + V - 1, w.batch * w.dim * w.L))
+                     ? __ldg(reinterpret_cast<const uint4 *>(dl + t))
+                     : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        if (tb + int64_t(i) * V >= w.L) break;
+        float v[V];
+        Vec<T>::unpack(raw[i], v);
+#pragma unroll
+        for (int e = 0; e < V; ++e) in = in || (v[e] >= lo && v[e] <= hi);
+      }
+    }
+    const bool any_in = __syncthreads_or(in);
+    const int64_t fi = int64_t(g) * nblk + tb / kRangeBlock;
+    if (threadIdx.x == 0 && in_bounds(fi, p.n_flags))
+      const_cast<unsigned char *>(p.range_flags)[fi] = any_in ? 0 : 1;
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kSThreads) delta_range_kernel(const BwdStagedArgs p) {
+  constexpr int V = Vec<T>::kN;
+  constexpr int PER = kRangeBlock / V;  // 16-byte loads per block
+  const BwdArgs &w = p.w;
+  const int64_t nblk = (w.L + kRangeBlock - 1) / kRangeBlock;
+  const int64_t nspan = (w.L + kRangeSpan - 1) / kRangeSpan;
+  for (int64_t unit = blockIdx.x; unit < int64_t(p.G) * nspan; unit += gridDim.x)
+    delta_range_unit<T, V, PER>(p, int(unit % p.G), (unit / p.G) * kRangeSpan, nblk);
 }
 
 // Three-phase carry of the adjoint, used when there are too few channel groups
@@ -1173,7 +1252,7 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return MAMBA_ERR_CUDA;
   int bps = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, kern, kSThreads, smem) != cudaSuccess)
+  if (resident_ctas(kern, smem, PROJ, &bps) != cudaSuccess)
     return MAMBA_ERR_CUDA;
   const int sms = device_sm_count();
   const int slots = sms * std::max(1, bps);
@@ -1199,8 +1278,13 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
   const size_t n_par = par ? gk * NM * kSThreads : 0;  // agg_G and gin each
   // the fused projection's three-phase carry: delta in fp32 for the aggregate pass
   const size_t n_delta = (PROJ && par) ? size_t(a.batch) * size_t(a.dim) * size_t(a.L) : 0;
-  const size_t bytes = ceil_div(int_bytes + 4 * (n_ckpt + n_carry + n_bc + n_A + 2 * n_D + n_delta) +
-                                    (par ? 8 * n_D + 8 * n_par : 0), 256) * 256;
+  const size_t bytes_f = ceil_div(int_bytes + 4 * (n_ckpt + n_carry + n_bc + n_A + 2 * n_D + n_delta) +
+                                      (par ? 8 * n_D + 8 * n_par : 0), 256) * 256;
+  // the range flags of delta (not with the fused projection, which checks per
+  // tile, nor with the generic arithmetic forced)
+  const bool range = !PROJ && o.path != MAMBA_PATH_GENERIC;
+  const size_t n_flags = range ? size_t(G) * size_t(ceil_div(a.L, kRangeBlock)) : 0;
+  const size_t bytes = bytes_f + ceil_div(n_flags, 256) * 256;
   // The checkpoint pass (the forward without y) is prepared first so that one
   // workspace holds both: a failed allocation then leaves nothing enqueued.
   FwdArgs fa;
@@ -1258,6 +1342,8 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
   bp.n_bc = int64_t(n_bc);
   bp.n_unit = int64_t(n_D);
   bp.n_gin = int64_t(n_par);
+  bp.range_flags = range ? ws + bytes_f : nullptr;
+  bp.n_flags = int64_t(n_flags);
   bp.timeout_ns = o.timeout_us > 0 ? uint64_t(o.timeout_us) * 1000ull : kDefaultTimeoutNs;
   bp.force_generic = o.path == MAMBA_PATH_GENERIC ? 1 : 0;
   bp.test_hook = o.test_hook;
@@ -1268,6 +1354,11 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
     ckpt_pass.sa.ckpt = ckpt;
     ckpt_pass.sa.delta_out = delta_f32;
     st = ckpt_pass.run(ws + bytes, s, launched);
+  }
+  if (st == MAMBA_OK && range) {
+    const int64_t units = G * ceil_div(a.L, kRangeSpan);
+    delta_range_kernel<T><<<unsigned(std::min<int64_t>(units, int64_t(sms) * 16)), kSThreads, 0, s>>>(bp);
+    st = launched();
   }
   if (st == MAMBA_OK && par) {
     if (delta_f32) {  // the aggregate pass reads the fp32 delta the checkpoint pass formed
@@ -1289,7 +1380,8 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
       io.gpb = int(gpb);
       io.N = a.N;
       io.dim = a.dim;
-      chunk_scan_kernel<NM, true><<<unsigned(G * NM * kSThreads), 128, 0, s>>>(io);
+      const int64_t nseq = G * NM * kSThreads;
+      chunk_scan_kernel<NM, true><<<unsigned(chunk_scan_grid(nseq, pl.K)), 128, 0, s>>>(io);
       st = launched();
     }
   }

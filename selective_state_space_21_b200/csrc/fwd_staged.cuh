@@ -99,14 +99,61 @@ struct StagedArgs {
   float *delta_out = nullptr;
   // element counts of the workspace buffers as allocated (the bounds-checking
   // build checks every index against them)
-  int64_t n_carry = 0, n_agg = 0, n_aggS = 0, n_ckpt = 0;
+  int64_t n_carry = 0, n_agg = 0, n_aggS = 0, n_ckpt = 0, n_blk = 0;
+  // LOC: [G][ceil(L/64)][128] sum of Delta from the start of the chunk to the
+  // end of each 64-step block (where the correction of a block starts)
+  float *blk_cum = nullptr;
 };
+constexpr int kCorrBlock = 64;  // steps per CTA of the closed-form correction
 
 // Fused Delta projection: TMEM columns of one CTA (W rows in [0, Rp/2), two
 // fp32 accumulators of one tile each after kProjAcc).
 constexpr int kProjMaxRp = 256;
 constexpr uint32_t kProjAcc = kProjMaxRp / 2;
 constexpr uint32_t kProjTmemCols = 256;
+// The thread that issues the projection MMAs: lane 0 of the last warp, so that
+// warp 0, which issues the TMA loads and stores, does not carry both.
+constexpr int kMmaThread = 96;
+
+// Thread's row d of W_dt (bf16, R per row) into its TMEM lane from column
+// `taddr`'s on: Rp/2 columns of bf16 pairs (even k in the low half), zero
+// beyond R (and for a channel past dim).  With R a multiple of 8 and the row
+// 16-byte aligned, 16-byte loads, up to sixteen issued before the first use;
+// else 2-byte loads.
+__device__ __forceinline__ void proj_load_w(const __nv_bfloat16 *W, int64_t d, bool valid, int R, int Rp,
+                                            uint32_t taddr) {
+  const __nv_bfloat16 *wrow = W + (valid ? d * R : 0);
+  if (R % 8 == 0 && (reinterpret_cast<uintptr_t>(wrow) & 15) == 0) {
+    for (int c0 = 0; c0 < Rp / 16; c0 += 8) {  // eight 16-column groups per round of loads
+      uint4 v[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int k = 16 * c0 + 8 * i;
+        v[i] = (valid && k < R) ? __ldg(reinterpret_cast<const uint4 *>(wrow + k)) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        if (c0 + c < Rp / 16) {
+          const uint32_t r[8] = {v[2 * c].x,     v[2 * c].y,     v[2 * c].z,     v[2 * c].w,
+                                 v[2 * c + 1].x, v[2 * c + 1].y, v[2 * c + 1].z, v[2 * c + 1].w};
+          tmem_st8(taddr + uint32_t(c0 + c) * 8u, r);
+        }
+      }
+    }
+    return;
+  }
+  for (int c8 = 0; c8 < Rp / 16; ++c8) {
+    uint32_t r[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int k = 16 * c8 + 2 * i;
+      const uint32_t lo = (valid && k < R) ? __bfloat16_as_ushort(wrow[k]) : 0u;
+      const uint32_t hi = (valid && k + 1 < R) ? __bfloat16_as_ushort(wrow[k + 1]) : 0u;
+      r[i] = lo | (hi << 16);
+    }
+    tmem_st8(taddr + uint32_t(c8) * 8u, r);
+  }
+}
 
 // Shared-memory offsets of the fused-projection forward: a stage holds u,
 // the dt_low tile (Rp rows), z, B and C.
@@ -165,6 +212,17 @@ __device__ __forceinline__ float softplus_fast(float v) {
   const float l = lg2f(1.f + w) * kLn2;
   const float r = w < 0.0625f ? s : l;
   return v > 15.f ? v + ex2f(-v * kLog2e) : r;
+}
+
+// softplus(v) from e^-v and s = sigma(v), which the sigma form of the update
+// already has: softplus(v) = -ln(1 - s) with 1 - s = e^-v s.  Below s = 1/16
+// the series s + s^2/2 + ... + s^6/6 (relative error below 1e-8); above
+// v = 15, v + e^-v (e^-v s would leave fp32's range).
+__device__ __forceinline__ float softplus_from_sigmoid(float v, float ev, float s) {
+  const float ser = s * (1.f + s * (0.5f + s * (1.f / 3.f + s * (0.25f + s * (0.2f + s * (1.f / 6.f))))));
+  const float l = -lg2f(ev * s) * kLn2;
+  const float r = s < 0.0625f ? ser : l;
+  return v > 15.f ? v + ev : r;
 }
 
 // expm1(x) for x <= 0: a degree-6 Taylor polynomial for x > -1/4 (relative
@@ -377,7 +435,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
   // N = TT steps; A = W from TMEM, K-major; B = dt_low, MN-major) and TMEM
   [[maybe_unused]] constexpr uint32_t kIdesc = mma_idesc_bf16(128, TT, false, true);
   [[maybe_unused]] uint32_t tbase = 0;
-  [[maybe_unused]] int mma_issued = -1;  // thread 0: last tile whose MMA it issued
+  [[maybe_unused]] int mma_issued = -1;  // kMmaThread: last tile whose MMA it issued
 
   if (tid == 0) {
 #pragma unroll
@@ -409,7 +467,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
     tbase = uint32_t(q[12]);
   }
 
-  // Issues (thread 0) the projection MMAs of consumed-tile index `ct` into
+  // Issues (kMmaThread) the projection MMAs of consumed-tile index `ct` into
   // accumulator ct & 1, once the tile's dt_low rows have landed.
   [[maybe_unused]] auto issue_mma = [&](int ct) {
     const int stg = ct % NST;
@@ -519,24 +577,12 @@ __global__ void __launch_bounds__(kSThreads, 2)
       // This group's rows of W_dt into TMEM columns [0, Rp/2), bf16 pairs
       // (even k in the low half).  The previous unit's MMAs have completed:
       // its threads waited for every one of them.
-      const __nv_bfloat16 *wrow = static_cast<const __nv_bfloat16 *>(f.W_dt) +
-                                  (valid ? int64_t(d) * f.R : 0);
-      const int warp = tid >> 5;
-      for (int c8 = 0; c8 < p.Rp / 16; ++c8) {
-        uint32_t r[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int k = 16 * c8 + 2 * i;
-          const uint32_t lo = (valid && k < f.R) ? __bfloat16_as_ushort(wrow[k]) : 0u;
-          const uint32_t hi = (valid && k + 1 < f.R) ? __bfloat16_as_ushort(wrow[k + 1]) : 0u;
-          r[i] = lo | (hi << 16);
-        }
-        tmem_st8(tmem_at(tbase, uint32_t(warp) * 32u, uint32_t(c8) * 8u), r);
-      }
+      proj_load_w(static_cast<const __nv_bfloat16 *>(f.W_dt), d, valid, f.R, p.Rp,
+                  tmem_at(tbase, uint32_t(tid >> 5) * 32u, 0));
       tmem_st_wait();
       tc_fence_before_sync();
       __syncthreads();
-      if (tid == 0) issue_mma(ctile);
+      if (tid == kMmaThread) issue_mma(ctile);
     }
     int mode = MODE_GEN;
     if (!p.force_generic) {
@@ -644,6 +690,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
       if (q[8]) return;
 
       for (int it = 0; it < ntiles; ++it, ++ctile) {
+        [[maybe_unused]] float Stile = 0.f;  // Delta summed over the tile (fp32; fp64 across tiles)
         const int stage = ctile % NST;
         unsigned char *st = sm + stage * SST;
         const float *Bt = Bs + (ctile & 1) * TT * BSTR;
@@ -654,6 +701,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
         const unsigned char *sz = st + OFF_Z;
         unsigned char *sy = sm + OFF_Y + (ctile & 1) * kTileBytes;
         [[maybe_unused]] uint32_t dacc = 0;
+        [[maybe_unused]] bool mma_next = false;  // (kMmaThread) the next tile's MMA is issued
         if constexpr (PROJ) {  // this tile's delta: wait for its MMA
           if (!mbar_wait_bounded(&mma_bar[ctile & 1], uint32_t(ctile >> 1) & 1u, p.timeout_ns)) {
             record_timeout();
@@ -706,8 +754,13 @@ __global__ void __launch_bounds__(kSThreads, 2)
               *reinterpret_cast<float4 *>(o) = make_float4(dv[0], dv[1], dv[2], dv[3]);
               *reinterpret_cast<float4 *>(o + 4) = make_float4(dv[4], dv[5], dv[6], dv[7]);
             }
-            // the next tile's MMA, into the other accumulator, half-way through this one
-            if (tid == 0 && j == 1 && it + 1 < ntiles) issue_mma(ctile + 1);
+            // the next tile's MMA, into the other accumulator: as soon as its
+            // dt_low tile has landed, at this tile's last chunk at the latest
+            if (tid == kMmaThread && !mma_next && it + 1 < ntiles && j >= 1 &&
+                (j == NV - 1 || mbar_test_wait(&bars[(ctile + 1) % NST], uint32_t((ctile + 1) / NST) & 1u))) {
+              issue_mma(ctile + 1);
+              mma_next = true;
+            }
             __syncwarp();
           } else {
             Vec<T>::unpack(*reinterpret_cast<const uint4 *>(sd + off), dv);
@@ -733,7 +786,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
               } else {
                 struct_update<NM>(H, P, -uv[i], 0.f, Brow, Brow);
               }
-              if constexpr (kAgg) Ssum += double(softplus_fast(v));
+              if constexpr (kAgg) Stile += softplus_from_sigmoid(v, ev, s);
             } else if constexpr (M == MODE_STRUCT) {
               const float Delta = softplus_fast(v);
               const float E1 = expm1_neg(Delta * A0);
@@ -744,12 +797,12 @@ __global__ void __launch_bounds__(kSThreads, 2)
               } else {
                 struct_update<NM>(H, P, uv[i] * invA0, 0.f, Brow, Brow);
               }
-              if constexpr (kAgg) Ssum += double(Delta);
+              if constexpr (kAgg) Stile += Delta;
             } else {
               const float Delta = softplus_fast(v);
               y0 = generic_update<NM>(h, Delta, uv[i], Dd * uv[i], Arow, A2, invA, Brow,
                                       kOut ? Crow : Brow);
-              if constexpr (kAgg) Ssum += double(Delta);
+              if constexpr (kAgg) Stile += Delta;
             }
             if (kOut) {
               if (has_z) {
@@ -760,6 +813,14 @@ __global__ void __launch_bounds__(kSThreads, 2)
             }
           }
           if (kOut) *reinterpret_cast<uint4 *>(sy + off) = Vec<T>::pack(yv);
+        }
+        if constexpr (kAgg) Ssum += double(Stile);
+        if constexpr (KIND == KIND_LOC) {  // the block's running sum, where a block ends
+          if ((t0 + TT) % kCorrBlock == 0 || it + 1 == ntiles) {
+            const int64_t bi = (int64_t(g) * ((f.L + kCorrBlock - 1) / kCorrBlock) + t0 / kCorrBlock) *
+                               kSThreads + tid;
+            if (in_bounds(bi, p.n_blk)) p.blk_cum[bi] = float(Ssum);
+          }
         }
         if (it + 1 < ntiles) stage_tables(ctile + 1);
         if (kOut) fence_proxy_async_smem();
@@ -833,10 +894,10 @@ __global__ void __launch_bounds__(kSThreads, 2)
       for (int t = ctile; t < p_issued; ++t)
         mbar_wait_bounded(&bars[t % NST], uint32_t(t / NST) & 1u, p.timeout_ns);
     }
-    if (PROJ && mma_issued >= 0)
-      mbar_wait_bounded(&mma_bar[mma_issued & 1], uint32_t(mma_issued >> 1) & 1u, p.timeout_ns);
     bulk_wait<0>();
   }
+  if (PROJ && tid == kMmaThread && mma_issued >= 0)
+    mbar_wait_bounded(&mma_bar[mma_issued & 1], uint32_t(mma_issued >> 1) & 1u, p.timeout_ns);
   if constexpr (PROJ) {
     tc_fence_before_sync();
     __syncthreads();
@@ -855,12 +916,14 @@ __global__ void __launch_bounds__(kSThreads, 2)
 // k maps an entering state h to exp(A_n S_k) h + hl_k (S_k its sum of Delta,
 // hl_k the state it produces from zero); two chunks compose as
 //     (S_a, hl_a) then (S_b, hl_b)  =  (S_a + S_b, exp(A_n S_b) hl_a + hl_b).
-// One CTA of 128 threads per (channel group, state, channel) walks the K
-// chunks in blocks of 128: a Kogge-Stone scan within each warp by shuffles,
-// the four warp totals combined through shared memory, and the state carried
-// from block to block; the chunk-entering states go back to HBM.  Element k
-// of the scan is chunk k (forward) or chunk K-1-k (REVERSE: the adjoint of
-// the backward runs from the end).  fp64 throughout.
+// With few chunks (K <= kChunkScanSerialK) one thread takes a sequence -- one
+// (channel group, state, channel) -- in order, its loads issued eight chunks
+// at a time.  With more, a sequence is scanned by the CTA's four warps in
+// blocks of 128 chunks: a Kogge-Stone scan within each warp by shuffles, the
+// warp totals combined through shared memory, the state carried from block to
+// block.  The chunk-entering values go back to HBM.  Element e of a scan is
+// chunk e (forward) or chunk K-1-e (REVERSE: the adjoint of the backward runs
+// from the end).  fp32 with the hardware exp2.
 struct ChunkScanIO {
   const double *S;   // [G][K][128] sum of Delta per chunk
   const float *hl;   // [G][K][NM][128] value each chunk produces from zero
@@ -871,32 +934,63 @@ struct ChunkScanIO {
 };
 // (its buffers hold G * K * 128 and G * K * NM * 128 elements)
 
+constexpr int kChunkScanSerialK = 32;
+
+// CTAs of 128 threads for the scan of `nseq` sequences of K chunks.
+inline int64_t chunk_scan_grid(int64_t nseq, int K) {
+  return K <= kChunkScanSerialK ? (nseq + 127) / 128 : nseq;
+}
+
 template <int NM, bool REVERSE>
 __global__ void __launch_bounds__(128) chunk_scan_kernel(const ChunkScanIO io) {
-  __shared__ double wS[4], wh[4];
-  __shared__ double carry;
-  const int seq = blockIdx.x;  // (g * NM + n) * 128 + c
-  const int c = seq % kSThreads, n = (seq / kSThreads) % NM, g = seq / (kSThreads * NM);
-  const int d = (g % io.gpb) * kSThreads + c;
-  const double An = (d < io.dim && n < io.N) ? double(io.A[int64_t(d) * io.N + n]) : 0.0;
+  __shared__ float wS[4], wh[4];
+  __shared__ float carry;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (threadIdx.x == 0) carry = 0.0;
+  const bool serial = io.K <= kChunkScanSerialK;
+  const int64_t seq = serial ? int64_t(blockIdx.x) * 128 + threadIdx.x : int64_t(blockIdx.x);
+  const int64_t nseq = int64_t(io.G) * NM * kSThreads;
+  if (seq >= nseq) return;  // (uniform per CTA when not serial)
+  const int c = int(seq % kSThreads), n = int((seq / kSThreads) % NM), g = int(seq / (kSThreads * NM));
+  const int d = (g % io.gpb) * kSThreads + c;
+  const float A2 = (d < io.dim && n < io.N) ? io.A[int64_t(d) * io.N + n] * kLog2e : 0.f;
+  const int64_t nk = int64_t(io.G) * io.K;
+  if (serial) {
+    float h = 0.f;  // the value entering element e
+    for (int e0 = 0; e0 < io.K; e0 += 8) {
+      float S[8], hl[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int e = e0 + i, k = REVERSE ? io.K - 1 - e : e;
+        const bool live = e < io.K - 1 && in_bounds(int64_t(g) * io.K + k, nk);  // the last map is never applied
+        const int64_t base = int64_t(g) * io.K + (live ? k : 0);
+        S[i] = live ? float(io.S[base * kSThreads + c]) : 0.f;
+        hl[i] = live ? io.hl[(base * NM + n) * kSThreads + c] : 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int e = e0 + i, k = REVERSE ? io.K - 1 - e : e;
+        if (e < io.K && in_bounds(int64_t(g) * io.K + k, nk))
+          io.hin[((int64_t(g) * io.K + k) * NM + n) * kSThreads + c] = h;
+        h = fmaf(ex2f(A2 * S[i]), h, hl[i]);
+      }
+    }
+    return;
+  }
+  if (threadIdx.x == 0) carry = 0.f;
   __syncthreads();
   for (int k0 = 0; k0 < io.K; k0 += 128) {
-    const int e = k0 + threadIdx.x;  // element of the scan
+    const int e = k0 + int(threadIdx.x);  // element of the scan
     const int k = REVERSE ? io.K - 1 - e : e;
-    const int64_t nk = int64_t(io.G) * io.K;
-    const bool live = e < io.K - 1 && in_bounds(int64_t(g) * io.K + k, nk);  // the last map is never applied
+    const bool live = e < io.K - 1 && in_bounds(int64_t(g) * io.K + k, nk);
     const int64_t base = int64_t(g) * io.K + (live ? k : 0);
-    double S = live ? io.S[base * kSThreads + c] : 0.0;
-    double h = live ? double(io.hl[(base * NM + n) * kSThreads + c]) : 0.0;
-    // inclusive scan within the warp
+    float S = live ? float(io.S[base * kSThreads + c]) : 0.f;
+    float h = live ? io.hl[(base * NM + n) * kSThreads + c] : 0.f;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const double So = __shfl_up_sync(0xffffffffu, S, o);
-      const double ho = __shfl_up_sync(0xffffffffu, h, o);
+    for (int o = 1; o < 32; o <<= 1) {  // inclusive scan within the warp
+      const float So = __shfl_up_sync(0xffffffffu, S, o);
+      const float ho = __shfl_up_sync(0xffffffffu, h, o);
       if (lane >= o) {
-        h = exp(An * S) * ho + h;
+        h = fmaf(ex2f(A2 * S), ho, h);
         S = So + S;
       }
     }
@@ -905,45 +999,51 @@ __global__ void __launch_bounds__(128) chunk_scan_kernel(const ChunkScanIO io) {
       wh[warp] = h;
     }
     __syncthreads();
-    // what enters this warp's first element: the carry through the earlier warps
-    double cin = carry;
-    for (int w = 0; w < warp; ++w) cin = exp(An * wS[w]) * cin + wh[w];
-    // exclusive prefix within the warp, applied to that
-    double Se = __shfl_up_sync(0xffffffffu, S, 1);
-    double he = __shfl_up_sync(0xffffffffu, h, 1);
+    float cin = carry;  // through the earlier blocks, then the earlier warps
+    for (int w = 0; w < warp; ++w) cin = fmaf(ex2f(A2 * wS[w]), cin, wh[w]);
+    float Se = __shfl_up_sync(0xffffffffu, S, 1);  // exclusive prefix within the warp
+    float he = __shfl_up_sync(0xffffffffu, h, 1);
     if (lane == 0) {
-      Se = 0.0;
-      he = 0.0;
+      Se = 0.f;
+      he = 0.f;
     }
     if (e < io.K && in_bounds(int64_t(g) * io.K + k, nk))
-      io.hin[((int64_t(g) * io.K + k) * NM + n) * kSThreads + c] = float(exp(An * Se) * cin + he);
+      io.hin[((int64_t(g) * io.K + k) * NM + n) * kSThreads + c] = fmaf(ex2f(A2 * Se), cin, he);
     __syncthreads();
-    if (threadIdx.x == 127) carry = exp(An * S) * cin + h;  // through the whole block
+    if (threadIdx.x == 127) carry = fmaf(ex2f(A2 * S), cin, h);  // through the whole block
     __syncthreads();
   }
 }
 
 // Closed-form correction after the LOC pass (one CTA per channel group and
-// chunk k >= 1, one thread per channel).  A chunk run from a zero entering
-// state misses the contribution of its true entering state h_in: with
-// cumDelta_t the sum of Delta over the chunk up to step t, the state the
-// chunk really has is h_t + exp(A_n cumDelta_t) h_in,n (the homogeneous
-// solution of the recurrence, Abar multiplying it step by step), so
+// 64-step block of the chunks k >= 1, one thread per channel).  A chunk run
+// from a zero entering state misses the contribution of its true entering
+// state h_in: with cumDelta_t the sum of Delta over the chunk up to step t,
+// the state the chunk really has is h_t + exp(A_n cumDelta_t) h_in,n (the
+// homogeneous solution of the recurrence, Abar multiplying it step by step),
+// so
 //     y_t += silu(z_t) sum_n C_tn exp(A_n cumDelta_t) h_in,n
 // and the last chunk's final state gains exp(A_n S) h_in,n.  For the
 // structured A (A_n = (n+1) A_0 < 0) the sum is a polynomial in
 // q_t = exp(A_0 cumDelta_t), evaluated by Horner's rule; otherwise one exp per
-// state.  A thread stops once every decay has fallen below 2^-32 (the terms
-// left are below fp32 resolution of the state they correct).
+// state.  A block starts from the LOC pass's running sum at its start, and a
+// CTA has nothing to add once every decay of its channels has fallen below
+// 2^-32 (the terms left are below fp32 resolution of the state they correct).
 template <typename T, int NM>
 __global__ void __launch_bounds__(kSThreads) fwd_correct_kernel(const StagedArgs p) {
   constexpr int V = 16 / int(sizeof(T));  // steps per 16-byte vector
+  constexpr int BLK = kCorrBlock;
+  __shared__ float Cs[BLK][NM + 1];       // this block's C rows, fp32, time-major
   const FwdArgs &f = p.f;
-  const int unit = blockIdx.x;  // (chunk - 1) * G + group
-  const int g = unit % p.G, k = 1 + unit / p.G;
+  const int64_t nblk = (f.L + BLK - 1) / BLK;
+  const int64_t first = p.chunk_len / BLK;  // the first block of chunk 1
+  const int g = int(blockIdx.x % unsigned(p.G));
+  const int64_t jb = first + blockIdx.x / unsigned(p.G);
+  const int64_t t0 = jb * BLK;
+  const int k = int(t0 / p.chunk_len);
   const int b = g / p.gpb, c = threadIdx.x;
   const int d = (g % p.gpb) * kSThreads + c;
-  if (d >= f.dim) return;
+  const bool valid = d < f.dim;
   const int N = f.N;
   float hin[NM], An[NM];
   bool any = false;
@@ -951,12 +1051,10 @@ __global__ void __launch_bounds__(kSThreads) fwd_correct_kernel(const StagedArgs
   for (int n = 0; n < NM; ++n) {
     const int64_t hi = ((int64_t(g) * p.K + k) * NM + n) * kSThreads + c;
     hin[n] = in_bounds(hi, p.n_agg) ? __ldcg(p.hin + hi) : 0.f;
-    An[n] = n < N ? f.A[int64_t(d) * N + n] : -float(n + 1);
-    any = any || (n < N && hin[n] != 0.f);
+    An[n] = (valid && n < N) ? f.A[int64_t(d) * N + n] : -float(n + 1);
+    any = any || (valid && n < N && hin[n] != 0.f);
   }
-  const int64_t tbeg = int64_t(k) * p.chunk_len;
-  const int64_t tend = std::min<int64_t>(f.L, tbeg + p.chunk_len);
-  if (k == p.K - 1 && f.last_state) {  // the true final state
+  if (valid && k == p.K - 1 && t0 == int64_t(k) * p.chunk_len && f.last_state) {  // the true final state
     const int64_t si = (int64_t(g) * p.K + k) * kSThreads + c;
     const double S = in_bounds(si, p.n_aggS) ? p.agg_S[si] : 0.0;
 #pragma unroll
@@ -967,54 +1065,61 @@ __global__ void __launch_bounds__(kSThreads) fwd_correct_kernel(const StagedArgs
         f.last_state[(int64_t(b) * f.dim + d) * N + n] = hl + float(exp(double(An[n]) * S)) * hin[n];
       }
   }
-  if (!any) return;
-  bool structured = An[0] < 0.f && isfinite(An[0]);
-#pragma unroll
-  for (int n = 1; n < NM; ++n) structured = structured && (An[n] == float(n + 1) * An[0]);
+  float cum = 0.f;  // Delta summed from the chunk's start to step t0 - 1
+  if (t0 > int64_t(k) * p.chunk_len) {
+    const int64_t bi = (int64_t(g) * nblk + jb - 1) * kSThreads + c;
+    cum = in_bounds(bi, p.n_blk) ? __ldcg(p.blk_cum + bi) : 0.f;
+  }
   float amax = An[0];  // slowest decay
 #pragma unroll
   for (int n = 1; n < NM; ++n) amax = fmaxf(amax, An[n]);
+  const bool active = any && amax * cum >= -22.2f;  // exp(amax cumDelta) >= 2^-32
+  if (!__syncthreads_or(active)) return;
+  const int steps = int(std::min<int64_t>(BLK, f.L - t0));
+  const T *Cb = static_cast<const T *>(f.C) + int64_t(b) * N * f.L;
+  for (int i = threadIdx.x; i < BLK * NM; i += kSThreads) {
+    const int n = i / BLK, tl = i % BLK;  // consecutive threads read consecutive steps
+    Cs[tl][n] = (n < N && tl < steps && in_bounds(int64_t(b) * N * f.L + int64_t(n) * f.L + t0 + tl,
+                                                   f.batch * N * f.L))
+                    ? to_f(Cb[int64_t(n) * f.L + t0 + tl])
+                    : 0.f;
+  }
+  __syncthreads();
+  if (!active) return;
+  bool structured = An[0] < 0.f && isfinite(An[0]);
+#pragma unroll
+  for (int n = 1; n < NM; ++n) structured = structured && (An[n] == float(n + 1) * An[0]);
   const float bias = f.bias ? f.bias[d] : 0.f;
   const int64_t row = (int64_t(b) * f.dim + d) * f.L;
   const T *dl = static_cast<const T *>(f.delta) + row;
   const T *zr = f.z ? static_cast<const T *>(f.z) + row : nullptr;
   T *yr = static_cast<T *>(f.y) + row;
-  const T *Cb = static_cast<const T *>(f.C) + int64_t(b) * N * f.L;
-  float cum = 0.f;
-  // the chunk starts at a multiple of 64 steps and rows are 16-byte multiples
-  for (int64_t t0 = tbeg; t0 < tend; t0 += V) {
-    if (amax * cum < -22.2f) break;  // exp(amax cumDelta) < 2^-32
-    if (!in_bounds(row + t0 + V - 1, f.batch * f.dim * f.L) ||
-        !in_bounds(int64_t(b) * N * f.L + int64_t(N - 1) * f.L + t0 + V - 1, f.batch * N * f.L))
-      break;
+  for (int j = 0; j < steps; j += V) {  // rows are 16-byte multiples
+    if (!in_bounds(row + t0 + j + V - 1, f.batch * f.dim * f.L)) break;
     float dv[V], zv[V], yv[V];
-    Vec<T>::unpack(*reinterpret_cast<const uint4 *>(dl + t0), dv);
-    Vec<T>::unpack(*reinterpret_cast<const uint4 *>(yr + t0), yv);
-    if (zr) Vec<T>::unpack(*reinterpret_cast<const uint4 *>(zr + t0), zv);
+    Vec<T>::unpack(*reinterpret_cast<const uint4 *>(dl + t0 + j), dv);
+    Vec<T>::unpack(*reinterpret_cast<const uint4 *>(yr + t0 + j), yv);
+    if (zr) Vec<T>::unpack(*reinterpret_cast<const uint4 *>(zr + t0 + j), zv);
 #pragma unroll
     for (int i = 0; i < V; ++i) {
       cum += softplus_fast(dv[i] + bias);
+      const float *crow = Cs[j + i];
       float corr;
-      if (structured) {
+      if (structured) {  // sum_n (C_n hin_n) q^(n+1), q = exp(A_0 cumDelta)
         const float q = ex2f(An[0] * cum * kLog2e);
         float r = 0.f;
 #pragma unroll
-        for (int n = NM - 1; n >= 0; --n) {
-          const float cn = n < N ? to_f(Cb[int64_t(n) * f.L + t0 + i]) * hin[n] : 0.f;
-          r = fmaf(r, q, cn);
-        }
+        for (int n = NM - 1; n >= 0; --n) r = fmaf(r, q, crow[n] * hin[n]);
         corr = r * q;
       } else {
         corr = 0.f;
 #pragma unroll
-        for (int n = 0; n < NM; ++n)
-          if (n < N) corr = fmaf(to_f(Cb[int64_t(n) * f.L + t0 + i]) * hin[n],
-                                 ex2f(An[n] * cum * kLog2e), corr);
+        for (int n = 0; n < NM; ++n) corr = fmaf(crow[n] * hin[n], ex2f(An[n] * cum * kLog2e), corr);
       }
       if (zr) corr *= zv[i] * rcpf(1.f + ex2f(-zv[i] * kLog2e));
       yv[i] += corr;
     }
-    *reinterpret_cast<uint4 *>(yr + t0) = Vec<T>::pack(yv);
+    *reinterpret_cast<uint4 *>(yr + t0 + j) = Vec<T>::pack(yv);
   }
 }
 
@@ -1055,12 +1160,38 @@ inline int proj_smem_bytes(int Rp, int nst) {
 // (228 KB per SM, 1 KB of it reserved per CTA).
 constexpr int kTwoPerSmBytes = (233472 - 2 * 1024) / 2;
 
+// CTAs of `kern` resident per SM with `smem` bytes of dynamic shared memory.
+// The occupancy query answers one for any kernel that allocates tensor memory,
+// whatever its registers and shared memory; a fused-projection CTA holds
+// kProjTmemCols of the SM's 512 TMEM columns, so for those (`tmem`) the count
+// is taken from registers and shared memory, capped at 512 / kProjTmemCols.
+// (Should more CTAs than that land on one SM, the extra one waits in its TMEM
+// allocation, which comes before it claims any work, until one exits.)
+template <typename K>
+inline cudaError_t resident_ctas(K kern, int smem, bool tmem, int *bps) {
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(bps, kern, kSThreads, smem);
+  if (e != cudaSuccess || !tmem) return e;
+  cudaFuncAttributes at;
+  if ((e = cudaFuncGetAttributes(&at, kern)) != cudaSuccess) return e;
+  int dev = 0, sm_smem = 0, reserved = 0, sm_regs = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&sm_smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&sm_regs, cudaDevAttrMaxRegistersPerMultiprocessor, dev)) != cudaSuccess)
+    return e;
+  const int warp_regs = (at.numRegs * 32 + 255) / 256 * 256;  // allocated per warp in units of 256
+  const int by_regs = sm_regs / std::max(1, warp_regs * (kSThreads / 32));
+  const int by_smem = sm_smem / std::max(1, smem + int(at.sharedSizeBytes) + reserved);
+  *bps = std::max(*bps, std::min(std::min(by_regs, by_smem), 512 / int(kProjTmemCols)));
+  return cudaSuccess;
+}
+
 template <typename T, int NM, int KIND, bool CONV = false, bool PROJ = false>
 inline cudaError_t prepare_kernel(int *blocks_per_sm, int bytes = StagedLayout<T, NM>::ALLOC) {
   auto kern = fwd_staged_kernel<T, NM, KIND, CONV, PROJ>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return e;
-  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, kern, kSThreads, bytes);
+  return resident_ctas(kern, bytes, PROJ, blocks_per_sm);
 }
 
 template <typename T, int NM, int KIND, bool CONV = false, bool PROJ = false>
@@ -1177,6 +1308,8 @@ struct StagedForward {
       bytes += size_t(G) * NM * kSThreads * 4;
     } else {
       bytes += gk * kSThreads * 8 + 2 * gk * NM * kSThreads * 4;
+      if (!ckpt && !PROJ)  // the LOC pass's running sums of Delta
+        bytes += size_t(G) * size_t(ceil_div(a.L, kCorrBlock)) * kSThreads * 4;
     }
     bytes = ceil_div(bytes, 256) * 256;
     return MAMBA_OK;
@@ -1194,7 +1327,8 @@ struct StagedForward {
     io.gpb = sa.gpb;
     io.N = sa.f.N;
     io.dim = sa.f.dim;
-    chunk_scan_kernel<NM, false><<<unsigned(int64_t(sa.G) * NM * kSThreads), 128, 0, s>>>(io);
+    const int64_t nseq = int64_t(sa.G) * NM * kSThreads;
+    chunk_scan_kernel<NM, false><<<unsigned(chunk_scan_grid(nseq, sa.K)), 128, 0, s>>>(io);
     return launched();
   }
 
@@ -1228,6 +1362,7 @@ struct StagedForward {
     sa.agg_S = reinterpret_cast<double *>(ws + int_bytes);
     sa.agg_h = reinterpret_cast<float *>(ws + int_bytes + gk * kSThreads * 8);
     sa.hin = sa.agg_h + gk * NM * kSThreads;
+    const int64_t nblk = ceil_div(sa.f.L, kCorrBlock);
     if (!sa.ckpt && !PROJ) {
       // Every chunk from zero, with y and its aggregates; the scan over
       // chunks; the closed-form correction of chunks 1..K-1 (and of the
@@ -1236,6 +1371,8 @@ struct StagedForward {
       // correction: those take the aggregate pass and a second full pass.)
       int bps_loc = 0;
       if (prepare_kernel<T, NM, KIND_LOC, CONV, PROJ>(&bps_loc, smem) != cudaSuccess) return MAMBA_ERR_CUDA;
+      sa.blk_cum = sa.hin + gk * NM * kSThreads;
+      sa.n_blk = int64_t(sa.G) * nblk * kSThreads;
       StagedArgs sl = sa;
       sl.counter = counters;
       sl.n_units = int(gk);
@@ -1244,7 +1381,8 @@ struct StagedForward {
       st = launched();
       if (st == MAMBA_OK) st = launch_chunk_scan(s, launched);
       if (st == MAMBA_OK) {
-        fwd_correct_kernel<T, NM><<<unsigned(size_t(sa.G) * size_t(pl.K - 1)), kSThreads, 0, s>>>(sa);
+        const int64_t nb = nblk - pl.chunk_len / kCorrBlock;  // the blocks of chunks 1..K-1
+        fwd_correct_kernel<T, NM><<<unsigned(int64_t(sa.G) * nb), kSThreads, 0, s>>>(sa);
         st = launched();
       }
       return st;

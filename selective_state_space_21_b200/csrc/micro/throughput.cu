@@ -28,8 +28,10 @@ __device__ __forceinline__ float op_lg2(float x) {
   return -y;
 }
 __device__ __forceinline__ float op_rcp(float x) {
+  // 1 / (1 + |x|) stays in (0, 1]: the chain cannot fold two reciprocals
+  // into the identity (the add runs on the FMA pipe beside the MUFU one)
   float y;
-  asm volatile("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  asm volatile("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(1.f + fabsf(x)));
   return y;
 }
 

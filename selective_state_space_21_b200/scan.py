@@ -142,6 +142,11 @@ def _ptr(t: Optional[torch.Tensor], dtype=None, shape=None, name=""):
 
 def _stream_handle(stream) -> Optional[int]:
     if stream is None:
+        # torch's current stream of the current device, without building a
+        # Stream object per call (it matters for one-token decoding steps)
+        raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+        if raw is not None:
+            return raw(torch.cuda.current_device())
         stream = torch.cuda.current_stream()
     return stream.cuda_stream if isinstance(stream, torch.cuda.Stream) else int(stream)
 
