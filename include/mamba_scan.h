@@ -421,7 +421,9 @@ MAMBA_SCAN_API void mamba_scan_test_fail_alloc(int32_t after);
  *
  *  - Plan: the regular call's (see mamba_scan_options_t.carry) when its
  *    scratch fits the array; for the three-phase carry of few channel groups
- *    and long sequences, fewer and longer chunks until it does.
+ *    and long sequences, the variant with an aggregate pass (whose scratch
+ *    does not grow with L) and then fewer, longer chunks until it fits;
+ *    failing that, the sequential hand-off.
  *  - Limit: the sequential hand-off's scratch must fit: at most 1023 channel
  *    groups (batch * ceil(dim / 128)) when N > 8, 2046 when 4 < N <= 8, 4088
  *    when N <= 4.  Larger problems return MAMBA_ERR_UNSUPPORTED without

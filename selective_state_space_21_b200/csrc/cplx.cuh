@@ -347,10 +347,22 @@ __global__ void __launch_bounds__(kCplxThreads) cplx_fwd_kernel(const CplxArgs a
 struct CplxWork {
   float *ckpt;       // (batch*dim, n_blocks, 2 NM) block-start states
   float *part_bc;    // (n_dblk, batch, 4 kMaxN, L): Re dB, Im dB, Re dC, Im dC
-  float *part_A;     // (batch*dim, 2N)
-  float *part_D;     // (batch*dim)
-  float *part_bias;  // (batch*dim)
+  float *part_A;     // (K, batch*dim, 2N): per chunk
+  float *part_D;     // (K, batch*dim)
+  float *part_bias;  // (K, batch*dim)
   int64_t n_blocks, n_dblk;
+  // The sequence of every channel block splits into K chunks of `bpc` blocks
+  // (the last may be shorter).  The forward sweep hands each chunk's end
+  // state on to the next chunk, the reverse sweep each chunk's entering
+  // adjoint back to the previous one, through `carry` (per channel block
+  // and thread: the state, or G and Abar) and the flags (per channel block:
+  // how many chunks have handed on, in the sweep's order).
+  int K;
+  int64_t bpc;
+  int *counter;      // ticket counters of the two launches, zero before the first
+  int *flags;        // (n_dblk * batch): the forward sweep counts chunks 1..K, the reverse K+1..2K
+  float *carry;      // (n_dblk * batch, kCplxBwdThreads, 4 NS)
+  uint64_t timeout_ns;
 };
 
 // Sums S values over the lanes of a warp that share lane % TPC (the channels
@@ -456,7 +468,15 @@ __device__ __forceinline__ void cplx_store_block(void *dst, const CplxArgs &a, i
 // block of steps the CTA stages B and C and the u, delta, z, dy rows of its
 // channels in shared memory (one 16-byte load per row where aligned), and
 // writes its du, ddelta, dz rows back from there.
-template <typename T, int NM, int TPC>
+//
+// Two launches: REVERSE = false, the forward sweep storing the block-start
+// states; REVERSE = true, the reverse sweep.  The work units are (chunk,
+// channel block) pairs that persistent CTAs claim from a ticket counter,
+// chunk by chunk (the reverse sweep from the last chunk): a unit that waits
+// for its neighbour chunk's hand-off (bounded) waits only on a unit claimed
+// before it.  Splitting the sequences into chunks lets the units of the last
+// round fill the GPU instead of leaving most SMs idle for a whole sequence.
+template <typename T, int NM, int TPC, bool REVERSE>
 __global__ void __launch_bounds__(kCplxBwdThreads, 8) cplx_bwd_kernel(const CplxArgs a, const CplxWork w) {
   constexpr int NS = NM / TPC;                 // states per thread
   constexpr int NV = 4 * NS < 32 / TPC ? 32 / TPC : 4 * NS;  // dB / dC values (padded)
@@ -468,10 +488,26 @@ __global__ void __launch_bounds__(kCplxBwdThreads, 8) cplx_bwd_kernel(const Cplx
   constexpr int CPB = kCplxBwdThreads / TPC;                 // channels per CTA
   float *xs = wsum + 2 * 4 * kMaxN * kCplxRow;               // [u, delta, z, dy][CPB][kCplxRow]
   float *os = xs + 4 * CPB * kCplxRow;                       // [du, ddelta, dz][CPB][kCplxRow]
+  __shared__ int s_ticket, s_abort;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int part = tid % TPC, lc = tid / TPC;
-  const int64_t b = blockIdx.y;
-  const int64_t d0 = int64_t(blockIdx.x) * CPB;
+  for (int i = tid; i < 2 * 4 * kMaxN * kCplxRow; i += kCplxBwdThreads) wsum[i] = 0.f;
+  const int64_t n_cb = w.n_dblk * a.batch;  // channel blocks
+  for (;;) {  // one (chunk, channel block) unit per pass
+  __syncthreads();
+  if (tid == 0) {
+    s_ticket = atomicAdd(w.counter + (REVERSE ? 1 : 0), 1);
+    s_abort = 0;
+  }
+  __syncthreads();
+  if (int64_t(s_ticket) >= n_cb * w.K) break;
+  const int64_t cb = s_ticket % n_cb;
+  const int k = REVERSE ? w.K - 1 - int(s_ticket / n_cb) : int(s_ticket / n_cb);
+  const int64_t c_beg = int64_t(k) * w.bpc;
+  const int64_t c_end = std::min<int64_t>(w.n_blocks, c_beg + w.bpc);
+  const int64_t dblk = cb % w.n_dblk;
+  const int64_t b = cb / w.n_dblk;
+  const int64_t d0 = dblk * CPB;
   const int64_t d_raw = d0 + lc;
   const bool valid = d_raw < a.dim;
   const int64_t d = valid ? d_raw : a.dim - 1;
@@ -489,7 +525,7 @@ __global__ void __launch_bounds__(kCplxBwdThreads, 8) cplx_bwd_kernel(const Cplx
   const float bias = a.bias ? a.bias[d] : 0.f;
   const float Dd = a.D ? a.D[d] : 0.f;
   float *ckpt = w.ckpt + ch * w.n_blocks * 2 * NM;
-  for (int i = tid; i < 2 * 4 * kMaxN * kCplxRow; i += kCplxBwdThreads) wsum[i] = 0.f;
+  float *carry = w.carry + (cb * kCplxBwdThreads + tid) * 4 * NS;
 
   float ar[NS], ai[NS], ira[NS], iai[NS], hr[NS], hi[NS];
 #pragma unroll
@@ -533,8 +569,23 @@ __global__ void __launch_bounds__(kCplxBwdThreads, 8) cplx_bwd_kernel(const Cplx
     }
   };
 
-  // Forward sweep: the state at the start of every block.
-  for (int64_t c = 0; c < w.n_blocks; ++c) {
+  if constexpr (!REVERSE) {
+  // Forward sweep over the chunk: the state at the start of every block,
+  // from the state the previous chunk handed on.
+  if (k > 0) {
+    if (tid == 0 && !wait_flag_geq(w.flags + cb, k, w.timeout_ns)) {  // chunks 0..k-1 done
+      record_timeout();
+      s_abort = 1;
+    }
+    __syncthreads();
+    if (s_abort) return;
+#pragma unroll
+    for (int j = 0; j < NS; ++j) {
+      hr[j] = __ldcg(carry + j);
+      hi[j] = __ldcg(carry + NS + j);
+    }
+  }
+  for (int64_t c = c_beg; c < c_end; ++c) {
     const int64_t t0 = c * kCplxBwdTC;
     // (padding channels run on zero rows and share the last channel's slots:
     // they must not write them)
@@ -554,21 +605,49 @@ __global__ void __launch_bounds__(kCplxBwdThreads, 8) cplx_bwd_kernel(const Cplx
     for (int i = 0; i < steps; ++i)
       step(softplus_fast(xd[i] + bias), xu[i], tab + i * cplx_tab_stride<NM, kCplxBwdTC>());
   }
+  if (k + 1 < w.K) {  // the state at the chunk's end, for the next chunk
+#pragma unroll
+    for (int j = 0; j < NS; ++j) {
+      carry[j] = hr[j];
+      carry[NS + j] = hi[j];
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) st_release_gpu(w.flags + cb, k + 1);
+  continue;
+  } else {
 
   float Gr[NS], Gi[NS], Anr[NS], Ani[NS], gAr[NS], gAi[NS];
 #pragma unroll
   for (int j = 0; j < NS; ++j) Gr[j] = Gi[j] = Anr[j] = Ani[j] = gAr[j] = gAi[j] = 0.f;
   float dDacc = 0.f, dbacc = 0.f;
   const int kbase = lane_scatter_base<NV, TPC>(lane);
+  if (k + 1 < w.K) {  // the adjoint entering from the later chunk (and its Abar)
+    // (the reverse sweep counts on from the forward sweep's K)
+    if (tid == 0 && !wait_flag_geq(w.flags + cb, w.K + (w.K - 1 - k), w.timeout_ns)) {
+      record_timeout();
+      s_abort = 1;
+    }
+    __syncthreads();
+    if (s_abort) return;
+#pragma unroll
+    for (int j = 0; j < NS; ++j) {
+      Gr[j] = __ldcg(carry + j);
+      Gi[j] = __ldcg(carry + NS + j);
+      Anr[j] = __ldcg(carry + 2 * NS + j);
+      Ani[j] = __ldcg(carry + 3 * NS + j);
+    }
+  }
 
-  for (int64_t c = w.n_blocks - 1; c >= 0; --c) {
+  for (int64_t c = c_end - 1; c >= c_beg; --c) {
     const int64_t t0 = c * kCplxBwdTC;
     const int steps = int(a.L - t0 < kCplxBwdTC ? a.L - t0 : kCplxBwdTC);
     __syncthreads();
     cplx_stage_bc<T, NM, kCplxBwdTC>(a, b, t0, tab, true, kCplxBwdThreads);
     for (int r = tid; r < 4 * CPB; r += kCplxBwdThreads) {
-      const int k = r / CPB;  // u, delta, z, dy
-      const void *src = k == 0 ? a.u : k == 1 ? a.delta : k == 2 ? a.z : a.dy;
+      const int q = r / CPB;  // u, delta, z, dy
+      const void *src = q == 0 ? a.u : q == 1 ? a.delta : q == 2 ? a.z : a.dy;
       if (src) cplx_load_block<T>(src, a, b, d0 + r % CPB, t0, steps, vec, xs + r * kCplxRow);
     }
     __syncthreads();
@@ -688,13 +767,22 @@ __global__ void __launch_bounds__(kCplxBwdThreads, 8) cplx_bwd_kernel(const Cplx
       if (s < steps) {
         const float sum = wsum[(0 * 4 * kMaxN + slot) * kCplxRow + s] +
                           wsum[(1 * 4 * kMaxN + slot) * kCplxRow + s];
-        w.part_bc[((int64_t(blockIdx.x) * a.batch + b) * 4 * kMaxN + slot) * a.L + t0 + s] = sum;
+        w.part_bc[((dblk * a.batch + b) * 4 * kMaxN + slot) * a.L + t0 + s] = sum;
       }
     }
     for (int r = tid; r < 3 * CPB; r += kCplxBwdThreads) {
-      const int k = r / CPB;  // du, ddelta, dz
-      void *dst = k == 0 ? a.du : k == 1 ? a.ddelta : a.dz;
+      const int q = r / CPB;  // du, ddelta, dz
+      void *dst = q == 0 ? a.du : q == 1 ? a.ddelta : a.dz;
       if (dst) cplx_store_block<T>(dst, a, b, d0 + r % CPB, t0, steps, vec, os + r * kCplxRow);
+    }
+  }
+  if (k > 0) {  // the adjoint entering this chunk, for the previous one
+#pragma unroll
+    for (int j = 0; j < NS; ++j) {
+      carry[j] = Gr[j];
+      carry[NS + j] = Gi[j];
+      carry[2 * NS + j] = Anr[j];
+      carry[3 * NS + j] = Ani[j];
     }
   }
   if (ident) {  // conj(1/A) times the sums of conj(k A) G
@@ -705,19 +793,25 @@ __global__ void __launch_bounds__(kCplxBwdThreads, 8) cplx_bwd_kernel(const Cplx
       gAi[j] = fmaf(ira[j], si, -iai[j] * sr);
     }
   }
-  if (valid) {
+  if (valid) {  // this chunk's parts of dA, dD, dbias
+    const int64_t bd = a.batch * a.dim;
 #pragma unroll
     for (int j = 0; j < NS; ++j) {
       const int n = part * NS + j;
       if (n < N) {
-        w.part_A[ch * 2 * N + n] = gAr[j];
-        w.part_A[ch * 2 * N + N + n] = gAi[j];
+        w.part_A[(k * bd + ch) * 2 * N + n] = gAr[j];
+        w.part_A[(k * bd + ch) * 2 * N + N + n] = gAi[j];
       }
     }
     if (part == 0) {
-      w.part_D[ch] = dDacc;
-      w.part_bias[ch] = dbacc;
+      w.part_D[k * bd + ch] = dDacc;
+      w.part_bias[k * bd + ch] = dbacc;
     }
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) st_release_gpu(w.flags + cb, w.K + (w.K - k));
+  }
   }
 }
 
@@ -746,15 +840,18 @@ __global__ void cplx_finalize_params(const CplxArgs a, const CplxWork w) {
   for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
        i += int64_t(gridDim.x) * blockDim.x) {
     const int64_t d = i / (2 * a.N), j = i % (2 * a.N);
+    const int64_t bd = a.batch * a.dim;
     float s = 0.f;
-    for (int64_t b = 0; b < a.batch; ++b) s += w.part_A[(b * a.dim + d) * 2 * a.N + j];
+    for (int64_t b = 0; b < a.batch; ++b)
+      for (int k = 0; k < w.K; ++k) s += w.part_A[(k * bd + b * a.dim + d) * 2 * a.N + j];
     a.dA[i] = s;
     if (j == 0) {
       float sd = 0.f, sb = 0.f;
-      for (int64_t b = 0; b < a.batch; ++b) {
-        sd += w.part_D[b * a.dim + d];
-        sb += w.part_bias[b * a.dim + d];
-      }
+      for (int64_t b = 0; b < a.batch; ++b)
+        for (int k = 0; k < w.K; ++k) {
+          sd += w.part_D[k * bd + b * a.dim + d];
+          sb += w.part_bias[k * bd + b * a.dim + d];
+        }
       if (a.dD) a.dD[d] = sd;
       if (a.dbias) a.dbias[d] = sb;
     }

@@ -477,13 +477,12 @@ __global__ void __launch_bounds__(kSThreads, 2)
       return;
     }
     tc_fence_after_sync();
-    const uint32_t dt_addr = smem_u32(sm + stg * SST + ps.dt);
     const uint32_t acc = tbase + kProjAcc + uint32_t(ct & 1) * TT;
-    for (int kk = 0; kk < p.Rp / 16; ++kk) {
-      // 16 rows of dt_low (two 8-row swizzle atoms of 512 bytes) per MMA
-      const uint64_t bdesc = smem_desc(dt_addr + uint32_t(kk) * 1024u, 16u, 512u, 4u);
-      mma_ts(acc, tbase + uint32_t(kk) * 8u, bdesc, kIdesc, kk > 0);
-    }
+    // 16 rows of dt_low (two 8-row swizzle atoms of 512 bytes) per MMA: the
+    // descriptor's start address (in 16-byte units) advances by 1024 bytes
+    const uint64_t bdesc0 = smem_desc(smem_u32(sm + stg * SST + ps.dt), 16u, 512u, 4u);
+    for (int kk = 0; kk < p.Rp / 16; ++kk)
+      mma_ts(acc, tbase + uint32_t(kk) * 8u, bdesc0 + uint64_t(kk) * 64u, kIdesc, kk > 0);
     mma_commit(&mma_bar[ct & 1]);
     mma_issued = ct;
   };
@@ -1239,6 +1238,19 @@ inline StagedPlan plan_staged(int64_t G, int64_t L, int slots, const StagedOptio
 template <typename T, int NM, bool CONV = false, bool PROJ = false>
 struct StagedForward {
   using Lay = StagedLayout<T, NM>;
+  // The three-phase forward with y runs the chunks from zero and corrects
+  // them in closed form (LOC + scan + fwd_correct_kernel) for 16-bit I/O; the
+  // correction is a pass over delta, z, C and y, which in fp32 moves twice
+  // the bytes and costs more than the aggregate pass it replaces (measured on
+  // fp32 8 x 1536 x 2048: 0.304 against 0.256 ms).  The checkpoint pass needs
+  // the true states at every 16th step, and the fused projection does not
+  // store delta for the correction: those, and fp32, take the aggregate pass
+  // and a second full pass.
+  static constexpr bool kLocCarry = sizeof(T) == 2 && !PROJ;
+  // (a caller with a bounded workspace may turn the closed-form carry off:
+  // its running sums of Delta take L / 64 floats per channel whatever the
+  // chunking, where the aggregate pass needs none)
+  bool use_loc = true;
   CUtensorMap maps[6];
   StagedArgs sa;
   StagedPlan pl;
@@ -1308,7 +1320,7 @@ struct StagedForward {
       bytes += size_t(G) * NM * kSThreads * 4;
     } else {
       bytes += gk * kSThreads * 8 + 2 * gk * NM * kSThreads * 4;
-      if (!ckpt && !PROJ)  // the LOC pass's running sums of Delta
+      if (kLocCarry && use_loc && !ckpt)  // the LOC pass's running sums of Delta
         bytes += size_t(G) * size_t(ceil_div(a.L, kCorrBlock)) * kSThreads * 4;
     }
     bytes = ceil_div(bytes, 256) * 256;
@@ -1362,30 +1374,30 @@ struct StagedForward {
     sa.agg_S = reinterpret_cast<double *>(ws + int_bytes);
     sa.agg_h = reinterpret_cast<float *>(ws + int_bytes + gk * kSThreads * 8);
     sa.hin = sa.agg_h + gk * NM * kSThreads;
-    const int64_t nblk = ceil_div(sa.f.L, kCorrBlock);
-    if (!sa.ckpt && !PROJ) {
-      // Every chunk from zero, with y and its aggregates; the scan over
-      // chunks; the closed-form correction of chunks 1..K-1 (and of the
-      // final state).  (The checkpoint pass needs the true states at every
-      // 16th step, and the fused projection does not store delta for the
-      // correction: those take the aggregate pass and a second full pass.)
-      int bps_loc = 0;
-      if (prepare_kernel<T, NM, KIND_LOC, CONV, PROJ>(&bps_loc, smem) != cudaSuccess) return MAMBA_ERR_CUDA;
-      sa.blk_cum = sa.hin + gk * NM * kSThreads;
-      sa.n_blk = int64_t(sa.G) * nblk * kSThreads;
-      StagedArgs sl = sa;
-      sl.counter = counters;
-      sl.n_units = int(gk);
-      launch_staged<T, NM, KIND_LOC, CONV, PROJ>(
-          maps, sl, int(std::min<int64_t>(gk, sms * std::max(1, bps_loc))), s, smem);
-      st = launched();
-      if (st == MAMBA_OK) st = launch_chunk_scan(s, launched);
-      if (st == MAMBA_OK) {
-        const int64_t nb = nblk - pl.chunk_len / kCorrBlock;  // the blocks of chunks 1..K-1
-        fwd_correct_kernel<T, NM><<<unsigned(int64_t(sa.G) * nb), kSThreads, 0, s>>>(sa);
+    [[maybe_unused]] const int64_t nblk = ceil_div(sa.f.L, kCorrBlock);
+    if constexpr (kLocCarry) {
+      if (!sa.ckpt && use_loc) {
+        // Every chunk from zero, with y and its aggregates; the scan over
+        // chunks; the closed-form correction of chunks 1..K-1 (and of the
+        // final state).
+        int bps_loc = 0;
+        if (prepare_kernel<T, NM, KIND_LOC, CONV, PROJ>(&bps_loc, smem) != cudaSuccess) return MAMBA_ERR_CUDA;
+        sa.blk_cum = sa.hin + gk * NM * kSThreads;
+        sa.n_blk = int64_t(sa.G) * nblk * kSThreads;
+        StagedArgs sl = sa;
+        sl.counter = counters;
+        sl.n_units = int(gk);
+        launch_staged<T, NM, KIND_LOC, CONV, PROJ>(
+            maps, sl, int(std::min<int64_t>(gk, sms * std::max(1, bps_loc))), s, smem);
         st = launched();
+        if (st == MAMBA_OK) st = launch_chunk_scan(s, launched);
+        if (st == MAMBA_OK) {
+          const int64_t nb = nblk - pl.chunk_len / kCorrBlock;  // the blocks of chunks 1..K-1
+          fwd_correct_kernel<T, NM><<<unsigned(int64_t(sa.G) * nb), kSThreads, 0, s>>>(sa);
+          st = launched();
+        }
+        return st;
       }
-      return st;
     }
     int bps_agg = 0, bps_par = 0;
     if (prepare_kernel<T, NM, KIND_AGG, CONV, PROJ>(&bps_agg, smem) != cudaSuccess ||

@@ -248,30 +248,58 @@ struct CplxBwdLauncher {
   static mamba_status_t launch(const CplxArgs &a, cudaStream_t s) {
     constexpr int per_block = kCplxBwdThreads / P;
     constexpr size_t smem = cplx_bwd_smem<NM, P>();
+    auto kf = cplx_bwd_kernel<T, NM, P, false>;
+    auto kr = cplx_bwd_kernel<T, NM, P, true>;
+    int occ = 0;
+    if (cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess ||
+        cudaFuncSetAttribute(kr, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kr, kCplxBwdThreads, smem) != cudaSuccess) {
+      cudaGetLastError();
+      return MAMBA_ERR_CUDA;
+    }
+    const int64_t slots = int64_t(device_sm_count()) * std::max(occ, 1);
     CplxWork w;
     w.n_blocks = (a.L + kCplxBwdTC - 1) / kCplxBwdTC;
     w.n_dblk = (a.dim + per_block - 1) / per_block;
+    const int64_t n_cb = w.n_dblk * a.batch;
+    // More channel blocks than CTA slots: four chunks per sequence, so that
+    // the last round of units is a quarter of a sequence long.  Otherwise one
+    // (the units all run at once, and chunks would only wait on each other).
+    const int64_t K0 = n_cb > slots ? 4 : 1;
+    w.bpc = (w.n_blocks + K0 - 1) / K0;
+    w.K = int((w.n_blocks + w.bpc - 1) / w.bpc);
+    if (n_cb * w.K > (int64_t(1) << 30)) return MAMBA_ERR_UNSUPPORTED;
+    w.timeout_ns = kDefaultTimeoutNs;
     const size_t bd = size_t(a.batch * a.dim);
     const size_t n_ckpt = bd * size_t(w.n_blocks) * 2 * NM;
     const size_t n_bc = size_t(w.n_dblk) * size_t(a.batch) * 4 * kMaxN * size_t(a.L);
-    const size_t n_A = bd * 2 * size_t(a.N);
-    float *ws = nullptr;
-    if (ws_alloc(reinterpret_cast<void **>(&ws), (n_ckpt + n_bc + n_A + 2 * bd) * 4, s) != cudaSuccess) {
+    const size_t n_A = size_t(w.K) * bd * 2 * size_t(a.N);
+    const size_t n_par = size_t(w.K) * bd;
+    const size_t n_carry = size_t(n_cb) * kCplxBwdThreads * 4 * (NM / P);
+    const size_t int_bytes = (size_t(2 + n_cb) * 4 + 255) / 256 * 256;
+    unsigned char *ws = nullptr;
+    if (ws_alloc(reinterpret_cast<void **>(&ws),
+                 int_bytes + (n_ckpt + n_bc + n_A + 2 * n_par + n_carry) * 4, s) != cudaSuccess) {
       cudaGetLastError();
       return MAMBA_ERR_OUT_OF_MEMORY;
     }
-    w.ckpt = ws;
+    w.counter = reinterpret_cast<int *>(ws);
+    w.flags = w.counter + 2;
+    w.ckpt = reinterpret_cast<float *>(ws + int_bytes);
     w.part_bc = w.ckpt + n_ckpt;
     w.part_A = w.part_bc + n_bc;
     w.part_D = w.part_A + n_A;
-    w.part_bias = w.part_D + bd;
+    w.part_bias = w.part_D + n_par;
+    w.carry = w.part_bias + n_par;
     mamba_status_t st = MAMBA_OK;
-    if (cudaFuncSetAttribute(cplx_bwd_kernel<T, NM, P>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
-      st = MAMBA_ERR_CUDA;
+    if (cudaMemsetAsync(ws, 0, int_bytes, s) != cudaSuccess) st = MAMBA_ERR_CUDA;
+    const unsigned grid = unsigned(std::min<int64_t>(n_cb * w.K, slots));
+    if (st == MAMBA_OK) {  // the forward sweep (block-start states), then the reverse sweep
+      kf<<<grid, kCplxBwdThreads, smem, s>>>(a, w);
+      st = launch_status();
+    }
     if (st == MAMBA_OK) {
-      const dim3 grid(unsigned(w.n_dblk), unsigned(a.batch));
-      cplx_bwd_kernel<T, NM, P><<<grid, kCplxBwdThreads, smem, s>>>(a, w);
+      kr<<<grid, kCplxBwdThreads, smem, s>>>(a, w);
       st = launch_status();
     }
     if (st == MAMBA_OK) {
@@ -289,18 +317,18 @@ struct CplxBwdLauncher {
   }
 
   static mamba_status_t run(const CplxArgs &a, cudaStream_t s) {
-    // Each CTA runs its channels' whole sequence.  When they fill at most half
-    // of one round of CTA slots, every CTA is latency-bound, and one state per
-    // thread (more threads per channel, shorter per-step chains) finishes
-    // sooner: 3.66 against 4.02 ms at batch 1 x 5120 channels, L 2048.
+    // When the channel blocks fill at most half of one round of CTA slots,
+    // every CTA is latency-bound, and one state per thread (more threads per
+    // channel, shorter per-step chains) finishes sooner: 3.66 against 4.02 ms
+    // at batch 1 x 5120 channels, L 2048.
     constexpr size_t smem = cplx_bwd_smem<NM, TPC>();
-    if (cudaFuncSetAttribute(cplx_bwd_kernel<T, NM, TPC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(cplx_bwd_kernel<T, NM, TPC, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              int(smem)) != cudaSuccess) {
       cudaGetLastError();
       return MAMBA_ERR_CUDA;
     }
     int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, cplx_bwd_kernel<T, NM, TPC>,
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, cplx_bwd_kernel<T, NM, TPC, true>,
                                                       kCplxBwdThreads, smem) != cudaSuccess) {
       cudaGetLastError();
       return MAMBA_ERR_CUDA;
@@ -1395,6 +1423,11 @@ mamba_status_t noalloc_forward(const FwdArgs &a, unsigned char *scratch, cudaStr
   StagedForward<T, NM> sf;
   mamba_status_t st = sf.prepare(a, o, nullptr);
   if (st != MAMBA_OK) return st;
+  if (sf.pl.kind == KIND_PAR && sf.bytes > kNoAllocScratchBytes) {
+    // the aggregate pass (no running sums of Delta), then fewer, longer chunks
+    sf.use_loc = false;
+    if ((st = sf.prepare(a, o, nullptr)) != MAMBA_OK) return st;
+  }
   if (sf.pl.kind == KIND_PAR && sf.bytes > kNoAllocScratchBytes) {
     for (int64_t chunk = int64_t(sf.pl.chunk_len) * 2; chunk < a.L && chunk < (int64_t(1) << 30);
          chunk *= 2) {
