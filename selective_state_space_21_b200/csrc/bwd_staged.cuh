@@ -108,13 +108,12 @@ struct BwdStagedArgs {
   // element counts of the workspace buffers as allocated (the bounds-checking
   // build checks every index against them)
   int64_t n_ckpt = 0, n_carry = 0, n_bc = 0, n_unit = 0, n_gin = 0;
-  // [G][ceil(L/64)]: 1 where some channel's delta leaves the range the
-  // structured forms take (null: no check; the fused projection checks per tile)
+  // [G][ceil(L/64)]: 1 where no step of any channel has its delta in the
+  // range the structured forms take (written by the checkpoint pass; null: no
+  // check, and the fused projection checks per tile)
   const unsigned char *range_flags = nullptr;
   int64_t n_flags = 0;
 };
-constexpr int kRangeBlock = 64;   // steps per range flag
-constexpr int kRangeSpan = 512;   // steps per CTA of delta_range_kernel
 
 // Byte offset of 16-byte chunk c of row r in a tile with RB-byte rows written
 // by TMA with RB-byte swizzling (chunk index XOR address bits from bit 7 up).
@@ -232,21 +231,6 @@ __device__ __forceinline__ void load_x4(const __nv_bfloat16 *p, float (&o)[4]) {
   o[1] = __uint_as_float(v.x & 0xffff0000u);
   o[2] = __uint_as_float(v.y << 16);
   o[3] = __uint_as_float(v.y & 0xffff0000u);
-}
-
-// Where the backward's structured forms keep their relative accuracy:
-// Delta |A_0| in [1e-5, 6].  Above, the decay chain keeps the small decays'
-// absolute but not their relative accuracy, which ddelta needs; below, the dA
-// identity A dh/dA = Delta dh/dDelta - Bbar u cancels.  Either way the error
-// is at fp32 resolution of the terms of a step in the range, so it matters
-// only where no step is: a unit (or, with the fused projection, a tile) in
-// which every step of every channel lies outside takes the generic
-// arithmetic.  In terms of v = delta (before the bias): [lo, hi] with
-// softplus(lo + bias) = 1e-5 / |A_0| and softplus(hi + bias) = 6 / |A_0|.
-__device__ __forceinline__ void structured_delta_range(float A0, float bias, float &lo, float &hi) {
-  const float ylo = 1e-5f / fabsf(A0), yhi = 6.f / fabsf(A0);
-  lo = logf(expm1f(ylo)) - bias;
-  hi = yhi + logf(-expm1f(-yhi)) - bias;
 }
 
 // CONV: the u tiles hold the input x of the block's causal depthwise
@@ -449,7 +433,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
     // problem.  (The fused projection's kernels, whose delta is formed tile by
     // tile, decide per tile.)
     bool unit_extreme = false;
-    if constexpr (!PROJ) {  // the unit's range flags (delta_range_kernel): all set?
+    if constexpr (!PROJ) {  // the unit's range flags (from the checkpoint pass): all set?
       if (p.range_flags) {
         const int64_t nblk = (f.L + kRangeBlock - 1) / kRangeBlock;
         const int64_t ub = int64_t(k) * p.chunk_len;
@@ -991,62 +975,6 @@ __global__ void __launch_bounds__(kSThreads, 2)
   }
 }
 
-// One flag per channel group and 64-step block: whether no step of any
-// channel of the group has its delta in structured_delta_range there
-// (channels whose A_0 is not negative take the generic arithmetic anyway and
-// are not checked).  Each CTA takes (group, 512-step span) units in turn, one
-// thread per channel; the reverse sweep takes the generic arithmetic for a
-// unit all of whose blocks are flagged.
-template <typename T, int V, int PER>
-__device__ __forceinline__ void delta_range_unit(const BwdStagedArgs &p, int g, int64_t t0, int64_t nblk) {
-  const BwdArgs &w = p.w;
-  const int b = g / p.gpb, d = (g % p.gpb) * kSThreads + int(threadIdx.x);
-  const float A0 = d < w.dim ? w.A[int64_t(d) * w.N] : 0.f;
-  const bool check = d < w.dim && A0 < 0.f && isfinite(A0);
-  float lo = 0.f, hi = 0.f;
-  if (check) structured_delta_range(A0, w.bias ? w.bias[d] : 0.f, lo, hi);
-  const int64_t row = (int64_t(b) * w.dim + (check ? d : 0)) * w.L;
-  const T *dl = static_cast<const T *>(w.delta) + row;
-  for (int j = 0; j < kRangeSpan / kRangeBlock; ++j) {
-    const int64_t tb = t0 + int64_t(j) * kRangeBlock;
-    if (tb >= w.L) break;  // (uniform over the CTA)
-    bool in = false;
-    if (check) {
-      uint4 raw[PER];
-#pragma unroll
-      for (int i = 0; i < PER; ++i) {  // rows are 16-byte multiples: whole vectors up to L
-        const int64_t t = tb + int64_t(i) * V;
-        raw[i] = (t < w.L && in_bounds(row + t + V - 1, w.batch * w.dim * w.L))
-                     ? __ldg(reinterpret_cast<const uint4 *>(dl + t))
-                     : make_uint4(0u, 0u, 0u, 0u);
-      }
-#pragma unroll
-      for (int i = 0; i < PER; ++i) {
-        if (tb + int64_t(i) * V >= w.L) break;
-        float v[V];
-        Vec<T>::unpack(raw[i], v);
-#pragma unroll
-        for (int e = 0; e < V; ++e) in = in || (v[e] >= lo && v[e] <= hi);
-      }
-    }
-    const bool any_in = __syncthreads_or(in);
-    const int64_t fi = int64_t(g) * nblk + tb / kRangeBlock;
-    if (threadIdx.x == 0 && in_bounds(fi, p.n_flags))
-      const_cast<unsigned char *>(p.range_flags)[fi] = any_in ? 0 : 1;
-  }
-}
-
-template <typename T>
-__global__ void __launch_bounds__(kSThreads) delta_range_kernel(const BwdStagedArgs p) {
-  constexpr int V = Vec<T>::kN;
-  constexpr int PER = kRangeBlock / V;  // 16-byte loads per block
-  const BwdArgs &w = p.w;
-  const int64_t nblk = (w.L + kRangeBlock - 1) / kRangeBlock;
-  const int64_t nspan = (w.L + kRangeSpan - 1) / kRangeSpan;
-  for (int64_t unit = blockIdx.x; unit < int64_t(p.G) * nspan; unit += gridDim.x)
-    delta_range_unit<T, V, PER>(p, int(unit % p.G), (unit / p.G) * kRangeSpan, nblk);
-}
-
 // Three-phase carry of the adjoint, used when there are too few channel groups
 // to fill the GPU with whole-sequence units.  The adjoint recurrence
 //     Ga_t = Abar_t (C_t dy0_t + Ga_{t+1})
@@ -1157,6 +1085,7 @@ __global__ void bwd_staged_finalize_bc(const BwdStagedArgs p) {
        i += int64_t(gridDim.x) * blockDim.x) {
     const int64_t t = i % f.L, n = (i / f.L) % f.N, b = i / (f.L * f.N);
     float sb = 0.f, sc = 0.f;
+#pragma unroll 8
     for (int j = 0; j < p.gpb; ++j) {
       const float *pp = p.part_bc + ((int64_t(j) * f.batch + b) * 32) * f.L + t;
       sb += pp[n * f.L];
@@ -1280,8 +1209,9 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
   const size_t n_delta = (PROJ && par) ? size_t(a.batch) * size_t(a.dim) * size_t(a.L) : 0;
   const size_t bytes_f = ceil_div(int_bytes + 4 * (n_ckpt + n_carry + n_bc + n_A + 2 * n_D + n_delta) +
                                       (par ? 8 * n_D + 8 * n_par : 0), 256) * 256;
-  // the range flags of delta (not with the fused projection, which checks per
-  // tile, nor with the generic arithmetic forced)
+  // the range flags of delta, written by the checkpoint pass (not with the
+  // fused projection, which checks per tile, nor with the generic arithmetic
+  // forced)
   const bool range = !PROJ && o.path != MAMBA_PATH_GENERIC;
   const size_t n_flags = range ? size_t(G) * size_t(ceil_div(a.L, kRangeBlock)) : 0;
   const size_t bytes = bytes_f + ceil_div(n_flags, 256) * 256;
@@ -1353,12 +1283,9 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
   if (st == MAMBA_OK) {
     ckpt_pass.sa.ckpt = ckpt;
     ckpt_pass.sa.delta_out = delta_f32;
+    ckpt_pass.sa.range_flags = range ? ws + bytes_f : nullptr;
+    ckpt_pass.sa.n_flags = int64_t(n_flags);
     st = ckpt_pass.run(ws + bytes, s, launched);
-  }
-  if (st == MAMBA_OK && range) {
-    const int64_t units = G * ceil_div(a.L, kRangeSpan);
-    delta_range_kernel<T><<<unsigned(std::min<int64_t>(units, int64_t(sms) * 16)), kSThreads, 0, s>>>(bp);
-    st = launched();
   }
   if (st == MAMBA_OK && par) {
     if (delta_f32) {  // the aggregate pass reads the fp32 delta the checkpoint pass formed

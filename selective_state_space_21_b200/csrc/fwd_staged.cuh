@@ -97,6 +97,11 @@ struct StagedArgs {
   uint32_t stage_bytes = 0;
   int nst = 0;
   float *delta_out = nullptr;
+  // CKPT kinds, when set: [G][ceil(L/64)] flags, 1 where no step of any
+  // channel of the group has its delta in structured_delta_range (the
+  // backward's choice of arithmetic)
+  unsigned char *range_flags = nullptr;
+  int64_t n_flags = 0;
   // element counts of the workspace buffers as allocated (the bounds-checking
   // build checks every index against them)
   int64_t n_carry = 0, n_agg = 0, n_aggS = 0, n_ckpt = 0, n_blk = 0;
@@ -213,6 +218,22 @@ __device__ __forceinline__ float softplus_fast(float v) {
   const float r = w < 0.0625f ? s : l;
   return v > 15.f ? v + ex2f(-v * kLog2e) : r;
 }
+
+// Where the backward's structured forms keep their relative accuracy:
+// Delta |A_0| in [1e-5, 6].  Above, the decay chain keeps the small decays'
+// absolute but not their relative accuracy, which ddelta needs; below, the dA
+// identity A dh/dA = Delta dh/dDelta - Bbar u cancels.  Either way the error
+// is at fp32 resolution of the terms of a step in the range, so it matters
+// only where no step is: a unit (or, with the fused projection, a tile) in
+// which every step of every channel lies outside takes the generic
+// arithmetic.  In terms of v = delta (before the bias): [lo, hi] with
+// softplus(lo + bias) = 1e-5 / |A_0| and softplus(hi + bias) = 6 / |A_0|.
+__device__ __forceinline__ void structured_delta_range(float A0, float bias, float &lo, float &hi) {
+  const float ylo = 1e-5f / fabsf(A0), yhi = 6.f / fabsf(A0);
+  lo = logf(expm1f(ylo)) - bias;
+  hi = yhi + logf(-expm1f(-yhi)) - bias;
+}
+constexpr int kRangeBlock = 64;  // steps per range flag
 
 // softplus(v) from e^-v and s = sigma(v), which the sigma form of the update
 // already has: softplus(v) = -ln(1 - s) with 1 - s = e^-v s.  Below s = 1/16
@@ -572,6 +593,15 @@ __global__ void __launch_bounds__(kSThreads, 2)
 #pragma unroll
     for (int n = 1; n < NM; ++n) structured = structured && (Arow[n] == float(n + 1) * Arow[0]);
     const bool sig = structured && Arow[0] == -1.f;
+    // (CKPT with range flags) the structured range of delta + bias, empty
+    // for channels that are not checked
+    [[maybe_unused]] float rlo = 3.4e38f, rhi = -3.4e38f;
+    [[maybe_unused]] bool rin = false;  // a step of the current 64-step block in range
+    if constexpr (kCkpt) {
+      if (p.range_flags && valid && Arow[0] < 0.f && isfinite(Arow[0])) {
+        structured_delta_range(Arow[0], 0.f, rlo, rhi);
+      }
+    }
     if constexpr (PROJ) {
       // This group's rows of W_dt into TMEM columns [0, Rp/2), bf16 pairs
       // (even k in the low half).  The previous unit's MMAs have completed:
@@ -771,6 +801,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
             const float *Brow = Bt + tl * BSTR;
             const float *Crow = Ct + tl * BSTR;
             const float v = dv[i] + bias;
+            if constexpr (kCkpt) rin = rin || (v >= rlo && v <= rhi);
             float y0;
             if constexpr (M == MODE_SIG) {
               // e^-v overflows below v = -88; above +88 it flushes to 0 and
@@ -824,7 +855,15 @@ __global__ void __launch_bounds__(kSThreads, 2)
         if (it + 1 < ntiles) stage_tables(ctile + 1);
         if (kOut) fence_proxy_async_smem();
         if (PROJ) tc_fence_before_sync();
-        __syncthreads();
+        if (kCkpt && p.range_flags && ((t0 + TT) % kRangeBlock == 0 || it + 1 == ntiles)) {
+          // (uniform over the CTA) the flag of the 64-step block this tile ends
+          const bool any_in = __syncthreads_or(rin);
+          rin = false;
+          const int64_t fi = int64_t(g) * ((f.L + kRangeBlock - 1) / kRangeBlock) + t0 / kRangeBlock;
+          if (tid == 0 && in_bounds(fi, p.n_flags)) p.range_flags[fi] = any_in ? 0 : 1;
+        } else {
+          __syncthreads();
+        }
         if (q[8]) return;
         if (tid == 0) {
           if (kOut) {
@@ -1032,7 +1071,7 @@ template <typename T, int NM>
 __global__ void __launch_bounds__(kSThreads) fwd_correct_kernel(const StagedArgs p) {
   constexpr int V = 16 / int(sizeof(T));  // steps per 16-byte vector
   constexpr int BLK = kCorrBlock;
-  __shared__ float Cs[BLK][NM + 1];       // this block's C rows, fp32, time-major
+  __shared__ __align__(16) float Cs[BLK][NM + 2];  // this block's C rows, fp32, time-major (even rows)
   const FwdArgs &f = p.f;
   const int64_t nblk = (f.L + BLK - 1) / BLK;
   const int64_t first = p.chunk_len / BLK;  // the first block of chunk 1
@@ -1088,6 +1127,9 @@ __global__ void __launch_bounds__(kSThreads) fwd_correct_kernel(const StagedArgs
   bool structured = An[0] < 0.f && isfinite(An[0]);
 #pragma unroll
   for (int n = 1; n < NM; ++n) structured = structured && (An[n] == float(n + 1) * An[0]);
+  f2 H2[NM / 2];  // h_in in pairs (even, odd state)
+#pragma unroll
+  for (int i = 0; i < NM / 2; ++i) H2[i] = pk(hin[2 * i], hin[2 * i + 1]);
   const float bias = f.bias ? f.bias[d] : 0.f;
   const int64_t row = (int64_t(b) * f.dim + d) * f.L;
   const T *dl = static_cast<const T *>(f.delta) + row;
@@ -1104,12 +1146,18 @@ __global__ void __launch_bounds__(kSThreads) fwd_correct_kernel(const StagedArgs
       cum += softplus_fast(dv[i] + bias);
       const float *crow = Cs[j + i];
       float corr;
-      if (structured) {  // sum_n (C_n hin_n) q^(n+1), q = exp(A_0 cumDelta)
+      if (structured) {
+        // sum_n c_n q^(n+1) with c_n = C_n hin_n and q = exp(A_0 cumDelta):
+        // the even and the odd states as two polynomials in q^2, evaluated
+        // together by Horner's rule in packed pairs, then
+        // q (sum_k c_2k q^2k + q sum_k c_2k+1 q^2k)
         const float q = ex2f(An[0] * cum * kLog2e);
-        float r = 0.f;
+        const f2 X = pk(q * q, q * q), Z = pk(0.f, 0.f);
+        const f2 *c2 = reinterpret_cast<const f2 *>(crow);
+        f2 r = fma2(c2[NM / 2 - 1], H2[NM / 2 - 1], Z);
 #pragma unroll
-        for (int n = NM - 1; n >= 0; --n) r = fmaf(r, q, crow[n] * hin[n]);
-        corr = r * q;
+        for (int k = NM / 2 - 2; k >= 0; --k) r = fma2(r, X, fma2(c2[k], H2[k], Z));
+        corr = q * fmaf(q, hi_of(r), lo_of(r));
       } else {
         corr = 0.f;
 #pragma unroll
