@@ -183,36 +183,45 @@ __device__ __forceinline__ float bfly_rest(float (&v)[16], int lane) {
   return v[0];
 }
 
-// Whether any step of thread `r`'s row in a 16-step tile has its delta in
-// [lo, hi]: from the tile in shared memory (swizzled rows), or (PROJ) from its
-// TMEM accumulator.
-template <typename T, bool PROJ>
-__device__ __forceinline__ bool tile_delta_in_range(const unsigned char *tile, uint32_t dacc, int r,
-                                                    float lo, float hi) {
-  float v[kBTT];
-  if constexpr (PROJ) {
-    float a[8], b[8];
-    tmem_ld8(dacc, a);
-    tmem_ld8(dacc + 8u, b);
-    tmem_ld_wait();
+// The same two steps for values kept in packed pairs (v2[i] = values 2i, 2i+1):
+// the adds of a pair are one fma.rn.f32x2, the shuffles and selects as before.
+__device__ __forceinline__ f2 bfly_first2(f2 db, f2 dc, bool up) {
+  const f2 send = up ? db : dc;
+  const f2 keep = up ? dc : db;
+  const float rl = __shfl_xor_sync(0xffffffffu, lo_of(send), 16);
+  const float rh = __shfl_xor_sync(0xffffffffu, hi_of(send), 16);
+  return fma2(pk(rl, rh), pk(1.f, 1.f), keep);
+}
+__device__ __forceinline__ float bfly_rest2(f2 (&v2)[8], int lane) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      v[i] = a[i];
-      v[8 + i] = b[i];
-    }
-  } else {
-    constexpr int RB = kBTT * (int)sizeof(T);
+  for (int o = 4; o >= 1; o >>= 1) {  // lane bits 3, 2, 1: pairs o apart
+    const bool up = (lane & (2 * o)) != 0;
 #pragma unroll
-    for (int c = 0; c < RB / 16; ++c) {
-      float o[Vec<T>::kN];
-      Vec<T>::unpack(*reinterpret_cast<const uint4 *>(tile + swz_rows<RB>(r, c)), o);
-#pragma unroll
-      for (int i = 0; i < Vec<T>::kN; ++i) v[c * Vec<T>::kN + i] = o[i];
+    for (int i = 0; i < o; ++i) {
+      const f2 send = up ? v2[i] : v2[i + o];
+      const f2 keep = up ? v2[i + o] : v2[i];
+      const float rl = __shfl_xor_sync(0xffffffffu, lo_of(send), 2 * o);
+      const float rh = __shfl_xor_sync(0xffffffffu, hi_of(send), 2 * o);
+      v2[i] = fma2(pk(rl, rh), pk(1.f, 1.f), keep);
     }
   }
+  const bool up = (lane & 1) != 0;  // lane bit 0: the two halves of the last pair
+  const float send = up ? lo_of(v2[0]) : hi_of(v2[0]);
+  const float keep = up ? hi_of(v2[0]) : lo_of(v2[0]);
+  return keep + __shfl_xor_sync(0xffffffffu, send, 1);
+}
+
+// Whether any step of a 16-step tile of the thread's delta, from its fused-
+// projection accumulator in TMEM (lane = channel), lies in [lo, hi].  Every
+// lane of the warp must call it: the TMEM load is warp-collective.
+__device__ __forceinline__ bool tile_delta_in_range(uint32_t dacc, float lo, float hi) {
+  float a[8], b[8];
+  tmem_ld8(dacc, a);
+  tmem_ld8(dacc + 8u, b);
+  tmem_ld_wait();
   bool in = false;
 #pragma unroll
-  for (int i = 0; i < kBTT; ++i) in = in || (v[i] >= lo && v[i] <= hi);
+  for (int i = 0; i < 8; ++i) in = in || (a[i] >= lo && a[i] <= hi) || (b[i] >= lo && b[i] <= hi);
   return in;
 }
 
@@ -584,7 +593,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
         bool tile_gen = false;
         if constexpr (kS && PROJ) {  // no step of the tile in the structured range?
           // (every thread reads its row: the TMEM load is warp-collective)
-          const bool in = tile_delta_in_range<T, PROJ>(st + Lay::TILE, dacc, tid, d_lo, d_hi);
+          const bool in = tile_delta_in_range(dacc, d_lo, d_hi);
           tile_gen = !__syncthreads_or(valid && in);
         } else {
           __syncthreads();
@@ -668,12 +677,10 @@ __global__ void __launch_bounds__(kSThreads, 2)
             }
             for (int seg = 0; seg < nseg; ++seg) {
               float *sp = sub + (seg * NM) * kSThreads + tid;
-              if constexpr (S) {
+              if constexpr (S) {  // packed pairs of states, one 8-byte store each
+                f2 *sp2 = reinterpret_cast<f2 *>(sub) + (seg * NP) * kSThreads + tid;
   #pragma unroll
-                for (int i = 0; i < NP; ++i) {
-                  sp[(2 * i) * kSThreads] = lo_of(H[i]);
-                  sp[(2 * i + 1) * kSThreads] = hi_of(H[i]);
-                }
+                for (int i = 0; i < NP; ++i) sp2[i * kSThreads] = H[i];
               } else {
   #pragma unroll
                 for (int n = 0; n < NM; ++n) sp[n * kSThreads] = h[n];
@@ -718,9 +725,9 @@ __global__ void __launch_bounds__(kSThreads, 2)
               // states before each step of the segment (the state after a step
               // is recomputed in the reverse step from h_{t-1} and t1)
               f2 Hs[SEG][NP];
+              const f2 *sp2 = reinterpret_cast<const f2 *>(sub) + (seg * NP) * kSThreads + tid;
   #pragma unroll
-              for (int i = 0; i < NP; ++i)
-                Hs[0][i] = pk(sp[(2 * i) * kSThreads], sp[(2 * i + 1) * kSThreads]);
+              for (int i = 0; i < NP; ++i) Hs[0][i] = sp2[i * kSThreads];
   #pragma unroll
               for (int i = 0; i + 1 < SEG; ++i) {
                 const float *Brow = Bs + (seg * SEG + i) * BSTR;
@@ -749,7 +756,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
                 const f2 U = pk(up, up), DY = pk(dy0, dy0), X1n = pk(-x1, -x1), Z = pk(0.f, 0.f);
                 f2 DU = Z, DD = Z, Y0 = Z;
                 const bool up16 = (lane & 16) != 0;
-                float v16[16];
+                f2 v2[8];
   #pragma unroll
                 for (int j = 0; j < NP; j += 2) {
                   const ulonglong2 bq = *reinterpret_cast<const ulonglong2 *>(Brow + 2 * j);
@@ -776,12 +783,11 @@ __global__ void __launch_bounds__(kSThreads, 2)
                     Gt[jj] = Ga;
                     // Channels past `dim` contribute exact zeros: TMA fills their
                     // rows with 0, so dy0 = 0 and their adjoint stays 0.
-                    v16[2 * jj] = bfly_first(lo_of(dBc), lo_of(dCc), up16);
-                    v16[2 * jj + 1] = bfly_first(hi_of(dBc), hi_of(dCc), up16);
+                    v2[jj] = bfly_first2(dBc, dCc, up16);
                   }
                 }
   #pragma unroll
-                for (int n = NM; n < kMaxN; ++n) v16[n] = 0.f;
+                for (int jj = NM / 2; jj < kMaxN / 2; ++jj) v2[jj] = pk(0.f, 0.f);
                 const float du = fmaf(lo_of(DU) + hi_of(DU), invA0, Dd * dy0);
                 const float dd = A0 * (lo_of(DD) + hi_of(DD)) * sv;
                 const float y0 = (lo_of(Y0) + hi_of(Y0)) + Dd * uv[i];
@@ -790,7 +796,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
                 dz_o[i] = has_z ? dyv[i] * y0 * sz * (1.f + zv[i] * (1.f - sz)) : 0.f;
                 dDsum = fmaf(dy0, uv[i], dDsum);
                 dbsum += dd;
-                const float rsum = bfly_rest(v16, lane);
+                const float rsum = bfly_rest2(v2, lane);
                 // lane l holds dB (l < 16, to be divided by l+1) or dC of state l-16
                 red[(warp * kBTT + tl) * 33 + lane] = (lane < kMaxN) ? rsum * (1.f / float(lane + 1)) : rsum;
               }
