@@ -26,7 +26,12 @@
 
 namespace mscan {
 
-constexpr int kGStages = 4;
+// TMA ring stages: four for d_dt_low (its B tile is up to 256 rows of dt_low);
+// three for dW, so that two CTAs share an SM (108 KB each at R = 160).
+template <bool GRAD_INPUT>
+__host__ __device__ constexpr int proj_gemm_stages() {
+  return GRAD_INPUT ? 4 : 3;
+}
 constexpr int kGBK = 64;  // k per stage (128 bytes of bf16)
 constexpr uint32_t kGTileA = 128 * kGBK * 2;  // 16 KB
 
@@ -48,6 +53,7 @@ template <bool GRAD_INPUT>
 __global__ void __launch_bounds__(128, 1)
     proj_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const ProjGemmArgs p) {
+  constexpr int kGStages = proj_gemm_stages<GRAD_INPUT>();
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t btile = proj_gemm_btile<GRAD_INPUT>(p.Rp);
@@ -213,6 +219,7 @@ __global__ void proj_grad_weight_finalize(const float *part, float *dW, int64_t 
 
 template <bool GRAD_INPUT>
 inline int proj_gemm_smem(int Rp) {
+  constexpr int kGStages = proj_gemm_stages<GRAD_INPUT>();
   return int(kGStages * (kGTileA + proj_gemm_btile<GRAD_INPUT>(Rp))) + 8 * (2 * kGStages + 1) + 16 +
          1024;
 }

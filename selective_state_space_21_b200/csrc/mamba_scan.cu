@@ -425,7 +425,8 @@ ProjGradPlan proj_grads_plan(const void *W, const void *dt_low, int64_t batch, i
     return pl;
   const int mt = int((dim + 127) / 128);
   pl.k_tiles = int(batch * ((L + 63) / 64));
-  int splits = std::max(1, std::min(pl.k_tiles, (2 * device_sm_count() + mt - 1) / mt));
+  // one wave of two CTAs per SM
+  int splits = std::max(1, std::min(pl.k_tiles, (2 * device_sm_count()) / mt));
   pl.k_per_split = (pl.k_tiles + splits - 1) / splits;
   pl.splits = (pl.k_tiles + pl.k_per_split - 1) / pl.k_per_split;
   pl.part_bytes = (size_t(pl.splits) * size_t(dim) * size_t(R) * 4 + 255) / 256 * 256;
