@@ -67,9 +67,11 @@ constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
 // LOC: the forward with y of every chunk from a zero entering state, which
 // also stores each chunk's end state and sum of Delta; the closed-form
 // correction (fwd_correct_kernel) then adds the entering state's
-// contribution once the scan over chunks has produced it.
+// contribution once the scan over chunks has produced it.  CKPT_LOC: the same
+// without y, storing the checkpoints of every chunk from zero with the sum of
+// Delta up to each; the reader of a checkpoint adds exp(A_n cum) h_in,n.
 enum StagedKind { KIND_SEQ = 0, KIND_PAR = 1, KIND_AGG = 2, KIND_CKPT_SEQ = 3, KIND_CKPT_PAR = 4,
-                  KIND_LOC = 5 };
+                  KIND_LOC = 5, KIND_CKPT_LOC = 6 };
 constexpr int kCkptEvery = 16;
 enum UnitMode { MODE_SIG = 0, MODE_STRUCT = 1, MODE_GEN = 2 };
 
@@ -102,6 +104,10 @@ struct StagedArgs {
   // backward's choice of arithmetic)
   unsigned char *range_flags = nullptr;
   int64_t n_flags = 0;
+  // CKPT_LOC: [G][ceil(L/16)][128] sum of Delta from the chunk's start to each
+  // checkpoint
+  float *ckpt_cum = nullptr;
+  int64_t n_ckpt_cum = 0;
   // element counts of the workspace buffers as allocated (the bounds-checking
   // build checks every index against them)
   int64_t n_carry = 0, n_agg = 0, n_aggS = 0, n_ckpt = 0, n_blk = 0;
@@ -418,10 +424,10 @@ __global__ void __launch_bounds__(kSThreads, 2)
   static_assert(!PROJ || (std::is_same<T, __nv_bfloat16>::value && !CONV),
                 "the fused projection takes bf16 operands and no convolution prologue");
   constexpr bool kOut = KIND == KIND_SEQ || KIND == KIND_PAR || KIND == KIND_LOC;  // stores y
-  constexpr bool kAgg = KIND == KIND_AGG || KIND == KIND_LOC;  // stores chunk aggregates
+  constexpr bool kAgg = KIND == KIND_AGG || KIND == KIND_LOC || KIND == KIND_CKPT_LOC;  // chunk aggregates
   constexpr bool kSeq = KIND == KIND_SEQ || KIND == KIND_CKPT_SEQ;
   constexpr bool kPar = KIND == KIND_PAR || KIND == KIND_CKPT_PAR;
-  constexpr bool kCkpt = KIND == KIND_CKPT_SEQ || KIND == KIND_CKPT_PAR;
+  constexpr bool kCkpt = KIND == KIND_CKPT_SEQ || KIND == KIND_CKPT_PAR || KIND == KIND_CKPT_LOC;
 
   // Offsetting the __shared__ array itself (not a cast integer) keeps every
   // derived pointer in the shared address space, so the compiler emits
@@ -747,6 +753,11 @@ __global__ void __launch_bounds__(kSThreads, 2)
               const int64_t ci = ((int64_t(g) * ((f.L + kCkptEvery - 1) / kCkptEvery) +
                                    tj / kCkptEvery) * NM) * kSThreads + tid;
               float *dst = p.ckpt + (in_bounds(ci + (NM - 1) * kSThreads, p.n_ckpt) ? ci : 0);
+              if constexpr (KIND == KIND_CKPT_LOC) {  // Delta summed from the chunk's start
+                const int64_t cc = (int64_t(g) * ((f.L + kCkptEvery - 1) / kCkptEvery) + tj / kCkptEvery) *
+                                       kSThreads + tid;
+                if (in_bounds(cc, p.n_ckpt_cum)) p.ckpt_cum[cc] = float(Ssum + double(Stile));
+              }
               if constexpr (M == MODE_GEN) {
 #pragma unroll
                 for (int n = 0; n < NM; ++n) dst[n * kSThreads] = h[n];
@@ -1299,6 +1310,12 @@ struct StagedForward {
   // its running sums of Delta take L / 64 floats per channel whatever the
   // chunking, where the aggregate pass needs none)
   bool use_loc = true;
+  // The three-phase checkpoint pass runs the chunks from zero (CKPT_LOC +
+  // scan) in place of the aggregate pass and a second pass; its checkpoints
+  // in chunks k >= 1 then lack exp(A_n cum) h_in,n, which the backward adds
+  // as it reads them (cum in sa.ckpt_cum, h_in in sa.hin).
+  bool ckpt_loc = true;
+  bool for_ckpt = false;  // prepared for a checkpoint pass
   CUtensorMap maps[6];
   StagedArgs sa;
   StagedPlan pl;
@@ -1308,9 +1325,11 @@ struct StagedForward {
 
   // Builds the tensor maps and the plan; with `ckpt` the forward runs without
   // y and stores the state before every kCkptEvery-th step into ckpt
-  // ([G][ceil(L/16)][NM][128] floats).  Returns MAMBA_ERR_UNSUPPORTED if the
-  // driver rejects a tensor map.
-  mamba_status_t prepare(const FwdArgs &a, const StagedOptions &o, float *ckpt) {
+  // ([G][ceil(L/16)][NM][128] floats; `ckpt_mode` sizes the workspace for a
+  // checkpoint pass whose buffer is set later).  Returns
+  // MAMBA_ERR_UNSUPPORTED if the driver rejects a tensor map.
+  mamba_status_t prepare(const FwdArgs &a, const StagedOptions &o, float *ckpt, bool ckpt_mode = false) {
+    for_ckpt = ckpt_mode || ckpt != nullptr;
     constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
     const uint64_t L = a.L, dim = a.dim, batch = a.batch, N = a.N;
     const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_64B, none = CU_TENSOR_MAP_SWIZZLE_NONE;
@@ -1368,7 +1387,9 @@ struct StagedForward {
       bytes += size_t(G) * NM * kSThreads * 4;
     } else {
       bytes += gk * kSThreads * 8 + 2 * gk * NM * kSThreads * 4;
-      if (kLocCarry && use_loc && !ckpt)  // the LOC pass's running sums of Delta
+      if (for_ckpt && ckpt_loc)  // the CKPT_LOC pass's sums of Delta at the checkpoints
+        bytes += size_t(G) * size_t(ceil_div(a.L, kCkptEvery)) * kSThreads * 4;
+      else if (kLocCarry && use_loc && !for_ckpt)  // the LOC pass's running sums of Delta
         bytes += size_t(G) * size_t(ceil_div(a.L, kCorrBlock)) * kSThreads * 4;
     }
     bytes = ceil_div(bytes, 256) * 256;
@@ -1446,6 +1467,24 @@ struct StagedForward {
         }
         return st;
       }
+    }
+    if (sa.ckpt && ckpt_loc) {
+      // Every chunk from zero, storing its checkpoints with the sums of Delta
+      // up to them and its aggregates; the scan over chunks (h_in).
+      int bps_loc = 0;
+      if (prepare_kernel<T, NM, KIND_CKPT_LOC, CONV, PROJ>(&bps_loc, smem) != cudaSuccess)
+        return MAMBA_ERR_CUDA;
+      const int64_t n16 = ceil_div(sa.f.L, kCkptEvery);
+      sa.ckpt_cum = sa.hin + gk * NM * kSThreads;
+      sa.n_ckpt_cum = int64_t(sa.G) * n16 * kSThreads;
+      StagedArgs sl = sa;
+      sl.counter = counters;
+      sl.n_units = int(gk);
+      launch_staged<T, NM, KIND_CKPT_LOC, CONV, PROJ>(
+          maps, sl, int(std::min<int64_t>(gk, sms * std::max(1, bps_loc))), s, smem);
+      st = launched();
+      if (st == MAMBA_OK) st = launch_chunk_scan(s, launched);
+      return st;
     }
     int bps_agg = 0, bps_par = 0;
     if (prepare_kernel<T, NM, KIND_AGG, CONV, PROJ>(&bps_agg, smem) != cudaSuccess ||
