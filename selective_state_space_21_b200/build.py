@@ -39,7 +39,7 @@ def deps():
 #: The files that define the staged forward and backward kernels and their
 #: launches (plus the compiler flags): a stored profile of those kernels stays
 #: valid while these are unchanged.
-STAGED_KERNEL_FILES = ("fwd_staged.cuh", "bwd_staged.cuh", "common.cuh", "tma.cuh")
+STAGED_KERNEL_FILES = ("fwd_staged.cuh", "bwd_staged.cuh", "common.cuh", "tma.cuh", "tcgen05.cuh")
 
 
 def source_digest(files=None) -> str:

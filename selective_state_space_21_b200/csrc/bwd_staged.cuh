@@ -44,21 +44,28 @@ namespace mscan {
 constexpr int kBTT = kCkptEvery;  // time steps per backward tile
 constexpr int kBStages = 2;
 
-template <typename T, int NM>
+// TSUB: the state before every segment lives in tensor memory (each thread's
+// own lane, NSEG x NM columns): one tcgen05.st / tcgen05.ld of the NM states
+// in place of NM / 2 shared-memory stores / loads.  The fused projection's
+// kernels, whose tensor memory holds W_dt and the delta accumulators, keep
+// the states in shared memory.
+template <typename T, int NM, bool TSUB = false>
 struct BwdLayout {
   static constexpr int RB = kBTT * (int)sizeof(T);  // bytes of one channel row in a tile
   static constexpr int TILE = kSThreads * RB;
   static constexpr int RAW = kMaxN * RB;
   static constexpr int STAGE = 4 * TILE + 2 * RAW;  // u, delta, z, dy, B, C
   // Steps per recompute segment: the states of one segment live in
-  // registers, the state before every segment in shared memory.  Two-step
-  // segments keep the register footprint down; fp32 tiles are twice as large,
-  // which leaves room for four-step segments only.
+  // registers, the state before every segment in shared or tensor memory.
+  // Two-step segments keep the register footprint down; fp32 tiles are twice
+  // as large, which leaves room for four-step segments only.
   static constexpr int SEG = sizeof(T) == 2 ? 2 : 4;
   static constexpr int NSEG = kBTT / SEG;
   static constexpr int BSTR = NM;  // rows of B / C are read as broadcasts; no padding
   static constexpr int OFF_SUB = kBStages * STAGE;
-  static constexpr int OFF_BS = OFF_SUB + NSEG * NM * kSThreads * 4;
+  static constexpr int SUB_BYTES = TSUB ? 0 : NSEG * NM * kSThreads * 4;
+  static constexpr int TMEM_COLS = !TSUB ? 0 : (NSEG * NM < 32 ? 32 : NSEG * NM);
+  static constexpr int OFF_BS = OFF_SUB + SUB_BYTES;
   static constexpr int OFF_CS = OFF_BS + kBTT * BSTR * 4;
   static constexpr int OFF_RED = OFF_CS + kBTT * BSTR * 4;
   static constexpr int RED_BYTES = (kSThreads / 32) * kBTT * 33 * 4;
@@ -268,7 +275,8 @@ __global__ void __launch_bounds__(kSThreads, 2)
                       const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_dy,
                       const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_C,
                       const BwdStagedArgs p) {
-  using Lay = BwdLayout<T, NM>;
+  constexpr bool kTSub = !PROJ;  // segment states in tensor memory
+  using Lay = BwdLayout<T, NM, kTSub>;
   constexpr int RB = Lay::RB, BSTR = Lay::BSTR;
   constexpr int NP = NM / 2;
   constexpr int SEG = Lay::SEG;
@@ -324,17 +332,16 @@ __global__ void __launch_bounds__(kSThreads, 2)
     if (has_z) prefetch_tensormap(&tm_z);
     q[8] = 0;
   }
-  if constexpr (PROJ) {
-    if (tid < 32) {
-      tmem_alloc(reinterpret_cast<uint32_t *>(&q[12]), kProjTmemCols);
-      tmem_relinquish();
-    }
+  constexpr uint32_t kTmemCols = PROJ ? kProjTmemCols : uint32_t(Lay::TMEM_COLS);
+  if (tid < 32) {
+    tmem_alloc(reinterpret_cast<uint32_t *>(&q[12]), kTmemCols);
+    tmem_relinquish();
   }
   __syncthreads();
-  if constexpr (PROJ) {
-    tc_fence_after_sync();
-    tbase = uint32_t(q[12]);
-  }
+  tc_fence_after_sync();
+  tbase = uint32_t(q[12]);
+  // (TSUB) this thread's lane: the state before segment s in columns s*NM ..
+  [[maybe_unused]] const uint32_t tsub = tmem_at(tbase, uint32_t(warp) * 32u, 0);
 
   // Issues (kMmaThread) the projection MMAs of consumed-tile index `ct` into
   // accumulator ct & 1 once the tile's dt_low rows have landed: 16 rows of
@@ -705,8 +712,21 @@ __global__ void __launch_bounds__(kSThreads, 2)
               for (int n = 0; n < NM; ++n) h[n] = h0[n];
             }
             for (int seg = 0; seg < nseg; ++seg) {
-              float *sp = sub + (seg * NM) * kSThreads + tid;
-              if constexpr (S) {  // packed pairs of states, one 8-byte store each
+              [[maybe_unused]] float *sp = sub + (seg * NM) * kSThreads + tid;
+              if constexpr (kTSub) {  // one tensor-memory store of the NM states
+                float hv[NM];
+                if constexpr (S) {
+  #pragma unroll
+                  for (int i = 0; i < NP; ++i) {
+                    hv[2 * i] = lo_of(H[i]);
+                    hv[2 * i + 1] = hi_of(H[i]);
+                  }
+                } else {
+  #pragma unroll
+                  for (int n = 0; n < NM; ++n) hv[n] = h[n];
+                }
+                tmem_st_row<NM>(tsub + uint32_t(seg * NM), hv);
+              } else if constexpr (S) {  // packed pairs of states, one 8-byte store each
                 f2 *sp2 = reinterpret_cast<f2 *>(sub) + (seg * NP) * kSThreads + tid;
   #pragma unroll
                 for (int i = 0; i < NP; ++i) sp2[i * kSThreads] = H[i];
@@ -734,6 +754,8 @@ __global__ void __launch_bounds__(kSThreads, 2)
             }
           }
 
+          if constexpr (kTSub) tmem_st_wait();  // the segment states, before they are read back
+
           // the next tile's projection MMA, into the other accumulator
           if constexpr (PROJ) {
             if (tid == kMmaThread && it + 1 < ntiles) issue_mma(ctile + 1);
@@ -748,15 +770,23 @@ __global__ void __launch_bounds__(kSThreads, 2)
             IO::load(sdy, tid, seg, dyv);
             if (has_z) IO::load(sz, tid, seg, zv);
             float du_o[SEG], dd_o[SEG], dz_o[SEG];
-            const float *sp = sub + (seg * NM) * kSThreads + tid;
+            [[maybe_unused]] const float *sp = sub + (seg * NM) * kSThreads + tid;
 
             if constexpr (S) {
               // states before each step of the segment (the state after a step
               // is recomputed in the reverse step from h_{t-1} and t1)
               f2 Hs[SEG][NP];
-              const f2 *sp2 = reinterpret_cast<const f2 *>(sub) + (seg * NP) * kSThreads + tid;
+              if constexpr (kTSub) {
+                float hv[NM];
+                tmem_ld_row<NM>(tsub + uint32_t(seg * NM), hv);
+                tmem_ld_wait();
   #pragma unroll
-              for (int i = 0; i < NP; ++i) Hs[0][i] = sp2[i * kSThreads];
+                for (int i = 0; i < NP; ++i) Hs[0][i] = pk(hv[2 * i], hv[2 * i + 1]);
+              } else {
+                const f2 *sp2 = reinterpret_cast<const f2 *>(sub) + (seg * NP) * kSThreads + tid;
+  #pragma unroll
+                for (int i = 0; i < NP; ++i) Hs[0][i] = sp2[i * kSThreads];
+              }
   #pragma unroll
               for (int i = 0; i + 1 < SEG; ++i) {
                 const float *Brow = Bs + (seg * SEG + i) * BSTR;
@@ -831,8 +861,13 @@ __global__ void __launch_bounds__(kSThreads, 2)
               }
             } else {
               float Hs[SEG][NM];
+              if constexpr (kTSub) {
+                tmem_ld_row<NM>(tsub + uint32_t(seg * NM), Hs[0]);
+                tmem_ld_wait();
+              } else {
   #pragma unroll
-              for (int n = 0; n < NM; ++n) Hs[0][n] = sp[n * kSThreads];
+                for (int n = 0; n < NM; ++n) Hs[0][n] = sp[n * kSThreads];
+              }
   #pragma unroll
               for (int i = 0; i + 1 < SEG; ++i) {
                 const float *Brow = Bs + (seg * SEG + i) * BSTR;
@@ -1001,12 +1036,14 @@ __global__ void __launch_bounds__(kSThreads, 2)
   if constexpr (PROJ) {  // every MMA issued must complete before TMEM is freed
     if (tid == kMmaThread && mma_issued >= 0)
       mbar_wait_bounded(&mma_bar[mma_issued & 1], uint32_t(mma_issued >> 1) & 1u, p.timeout_ns);
-    tc_fence_before_sync();
-    __syncthreads();
-    if (tid < 32) {
-      tc_fence_after_sync();
-      tmem_dealloc(tbase, kProjTmemCols);
-    }
+  } else {
+    tmem_st_wait();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (tid < 32) {
+    tc_fence_after_sync();
+    tmem_dealloc(tbase, kTmemCols);
   }
 }
 
@@ -1190,7 +1227,7 @@ inline int proj_max_rank() {
 template <typename T, int NM, bool CONV = false, bool PROJ = false>
 mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStream_t s,
                                mamba_status_t (*launched)()) {
-  using Lay = BwdLayout<T, NM>;
+  using Lay = BwdLayout<T, NM, !PROJ>;
   constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
   const uint64_t L = a.L, dim = a.dim, batch = a.batch, N = a.N;
   const CUtensorMapSwizzle sw = bf16 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B;
@@ -1216,7 +1253,7 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return MAMBA_ERR_CUDA;
   int bps = 0;
-  if (resident_ctas(kern, smem, PROJ, &bps) != cudaSuccess)
+  if (resident_ctas(kern, smem, PROJ ? int(kProjTmemCols) : Lay::TMEM_COLS, &bps) != cudaSuccess)
     return MAMBA_ERR_CUDA;
   const int sms = device_sm_count();
   const int slots = sms * std::max(1, bps);

@@ -1220,15 +1220,15 @@ constexpr int kTwoPerSmBytes = (233472 - 2 * 1024) / 2;
 
 // CTAs of `kern` resident per SM with `smem` bytes of dynamic shared memory.
 // The occupancy query answers one for any kernel that allocates tensor memory,
-// whatever its registers and shared memory; a fused-projection CTA holds
-// kProjTmemCols of the SM's 512 TMEM columns, so for those (`tmem`) the count
-// is taken from registers and shared memory, capped at 512 / kProjTmemCols.
-// (Should more CTAs than that land on one SM, the extra one waits in its TMEM
-// allocation, which comes before it claims any work, until one exits.)
+// whatever its registers and shared memory; a CTA that holds `tmem_cols` of
+// the SM's 512 TMEM columns (0: none) has its count taken from registers and
+// shared memory, capped at 512 / tmem_cols.  (Should more CTAs than that land
+// on one SM, the extra one waits in its TMEM allocation, which comes before
+// it claims any work, until one exits.)
 template <typename K>
-inline cudaError_t resident_ctas(K kern, int smem, bool tmem, int *bps) {
+inline cudaError_t resident_ctas(K kern, int smem, int tmem_cols, int *bps) {
   cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(bps, kern, kSThreads, smem);
-  if (e != cudaSuccess || !tmem) return e;
+  if (e != cudaSuccess || tmem_cols <= 0) return e;
   cudaFuncAttributes at;
   if ((e = cudaFuncGetAttributes(&at, kern)) != cudaSuccess) return e;
   int dev = 0, sm_smem = 0, reserved = 0, sm_regs = 0;
@@ -1240,7 +1240,7 @@ inline cudaError_t resident_ctas(K kern, int smem, bool tmem, int *bps) {
   const int warp_regs = (at.numRegs * 32 + 255) / 256 * 256;  // allocated per warp in units of 256
   const int by_regs = sm_regs / std::max(1, warp_regs * (kSThreads / 32));
   const int by_smem = sm_smem / std::max(1, smem + int(at.sharedSizeBytes) + reserved);
-  *bps = std::max(*bps, std::min(std::min(by_regs, by_smem), 512 / int(kProjTmemCols)));
+  *bps = std::max(*bps, std::min(std::min(by_regs, by_smem), 512 / tmem_cols));
   return cudaSuccess;
 }
 
@@ -1249,7 +1249,7 @@ inline cudaError_t prepare_kernel(int *blocks_per_sm, int bytes = StagedLayout<T
   auto kern = fwd_staged_kernel<T, NM, KIND, CONV, PROJ>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return e;
-  return resident_ctas(kern, bytes, PROJ, blocks_per_sm);
+  return resident_ctas(kern, bytes, PROJ ? int(kProjTmemCols) : 0, blocks_per_sm);
 }
 
 template <typename T, int NM, int KIND, bool CONV = false, bool PROJ = false>

@@ -122,6 +122,53 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
                : "memory");
 }
 
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint32_t (&r)[4]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3])
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+      "%13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// A thread's NM (4, 8 or 16) fp32 values to / from NM consecutive columns of
+// its own lane (warp-collective: every lane of the warp takes part).
+template <int NM>
+__device__ __forceinline__ void tmem_st_row(uint32_t taddr, const float (&v)[NM]) {
+  static_assert(NM == 4 || NM == 8 || NM == 16, "rows of 4, 8 or 16 columns");
+  uint32_t r[NM];
+#pragma unroll
+  for (int i = 0; i < NM; ++i) r[i] = __float_as_uint(v[i]);
+  if constexpr (NM == 4) tmem_st4(taddr, r);
+  else if constexpr (NM == 8) tmem_st8(taddr, r);
+  else tmem_st16(taddr, r);
+}
+template <int NM>
+__device__ __forceinline__ void tmem_ld_row(uint32_t taddr, float (&v)[NM]) {
+  static_assert(NM == 4 || NM == 8 || NM == 16, "rows of 4, 8 or 16 columns");
+  if constexpr (NM == 4) tmem_ld4(taddr, v);
+  else if constexpr (NM == 8) tmem_ld8(taddr, v);
+  else tmem_ld16(taddr, v);
+}
+
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // TMEM address of lane `lane`, column `col` relative to `base`.
