@@ -299,6 +299,13 @@ def oracle_sample_rate(x_host: dict, w, seconds: float = 10.0, min_blocks: int =
 
 # ------------------------------------------------------------------- arms
 
+def workload_label(w, step: str) -> str:
+    if step == "pair":
+        return (f"{w.name} (training step: forward storing the 16-step states + backward "
+                f"reading them)")
+    return f"{w.name} (forward + recompute backward per step)"
+
+
 def run_ours(args, world, rank, device):
     from selective_state_space_21_b200 import scan
 
@@ -325,17 +332,40 @@ def run_ours(args, world, rank, device):
          "dC": torch.empty_like(x["C"]), "dD": torch.empty(w.dim, device=device),
          "dbias": torch.empty(w.dim, device=device)}
 
-    def fwd():
-        scan.mamba_scan_fwd(x["u"], x["delta"], x["delta_bias"], x["A"], x["B"], x["C"],
-                            x["D"], x["z"], y, None)
+    # The training step: by default the pair whose forward stores the 16-step
+    # states for its backward (mamba_scan_fwd_save / mamba_scan_bwd_saved);
+    # --step recompute times the backward that re-runs the forward instead.
+    pair = args.step == "pair"
+    saved = None
+    if pair:
+        nsaved = scan.saved_bytes(w.batch, w.dim, w.L, w.N, w.dtype)
+        saved = torch.empty(nsaved, device=device, dtype=torch.uint8) if nsaved else None
 
-    def bwd():
+    def fwd():
+        if pair:
+            scan.mamba_scan_fwd_save(x["u"], x["delta"], x["delta_bias"], x["A"], x["B"], x["C"],
+                                     x["D"], x["z"], y, None, saved)
+        else:
+            scan.mamba_scan_fwd(x["u"], x["delta"], x["delta_bias"], x["A"], x["B"], x["C"],
+                                x["D"], x["z"], y, None)
+
+    def bwd_recompute():
         scan.mamba_scan_bwd(x["u"], x["delta"], x["delta_bias"], x["A"], x["B"], x["C"],
                             x["D"], x["z"], x["dy"], g["du"], g["ddelta"], g["dA"], g["dB"],
                             g["dC"], g["dD"], g["dz"], g["dbias"])
 
+    def bwd():
+        if pair:
+            scan.mamba_scan_bwd_saved(x["u"], x["delta"], x["delta_bias"], x["A"], x["B"], x["C"],
+                                      x["D"], x["z"], x["dy"], g["du"], g["ddelta"], g["dA"],
+                                      g["dB"], g["dC"], g["dD"], g["dz"], g["dbias"], saved)
+        else:
+            bwd_recompute()
+
     do_fwd = args.only in (None, "fwd")
     do_bwd = args.only in (None, "bwd")
+    if pair and do_bwd and not do_fwd:
+        fwd()  # the backward reads what the forward saved
     for _ in range(args.warmup):
         if do_fwd:
             fwd()
@@ -390,8 +420,12 @@ def run_ours(args, world, rank, device):
                 "peak_source": f"{peaks['source']} hbm_gbs (copy bandwidth)",
                 "ms_per_launch": round(ms, 4)}
 
-    roof_fwd = roof("fwd", fb, fwd_ms_max, "mamba_scan_fwd call")
-    roof_bwd = roof("bwd", bb, bwd_ms_max, "mamba_scan_bwd call")
+    if pair:
+        roof_fwd = roof("fwd_save", fb, fwd_ms_max, "mamba_scan_fwd_save call")
+        roof_bwd = roof("bwd_saved", bb, bwd_ms_max, "mamba_scan_bwd_saved call")
+    else:
+        roof_fwd = roof("fwd", fb, fwd_ms_max, "mamba_scan_fwd call")
+        roof_bwd = roof("bwd", bb, bwd_ms_max, "mamba_scan_bwd call")
     clocks = sampler.summary()
     elements = w.token_channels * w.N
     micro = None
@@ -437,8 +471,9 @@ def run_ours(args, world, rank, device):
         "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded N(0,1) u, delta, z, B, C, D, dy; log-uniform dt bias; "
                 "A = -(n+1))",
-        "config": {"workload": f"{w.name} (forward + recompute backward per step)",
-                   "batch": w.batch, "dim": w.dim, "L": w.L, "N": w.N, "io_dtype": "bf16",
+        "config": {"workload": workload_label(w, args.step),
+                   "batch": w.batch, "dim": w.dim, "L": w.L, "N": w.N,
+                   "io_dtype": "bf16" if w.dtype == torch.bfloat16 else "fp32",
                    "state_dtype": "f32", "global_batch": w.batch * world,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "inputs larger than L2 (u, delta, z, dy 168 MB each; L2 126 MB)"},
@@ -455,6 +490,9 @@ def run_ours(args, world, rank, device):
     }
     if micro:
         result["micro"] = micro
+    if pair and not args.only:  # the recomputing backward, for context
+        result["bwd_recompute"] = time_calls(bwd_recompute, device, args.conv_steps)
+        result["bwd_recompute"]["call"] = "mamba_scan_bwd (re-runs the forward first)"
 
     if not args.only and not args.no_a_legs:
         result["structured_A"] = run_a_leg(w, x, device, peaks, "structured", steps=args.conv_steps)
@@ -470,7 +508,7 @@ def run_ours(args, world, rank, device):
     if args.only:
         result["note"] = f"--only {args.only}: a profiling run, not a benchmark result"
     if not args.no_e2e and not args.only:
-        result["e2e"] = run_e2e(args, w, x, y, g, fwd, bwd, device, world)
+        result["e2e"] = run_e2e(args, w, x, y, g, fwd, bwd, device, world, pair)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.only:
         xh = {k: (v.cpu() if torch.is_tensor(v) else v) for k, v in x.items()}
@@ -808,7 +846,24 @@ def run_decode(w, x, device, peaks, steps=200):
     return out
 
 
-def run_e2e(args, w, x, y, g, fwd, bwd, device, world):
+def time_calls(fn, device, steps=10) -> dict:
+    """Median of per-call CUDA-event times of fn() after three warm-up calls."""
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize(device)
+    times = []
+    for _ in range(steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize(device)
+        times.append(e0.elapsed_time(e1))
+    return {"ms": round(statistics.median(times), 4), "steps": steps,
+            "timing": "median of per-call CUDA events"}
+
+
+def run_e2e(args, w, x, y, g, fwd, bwd, device, world, pair=False):
     """Same step through the public API with host buffers: each step copies its
     inputs from pinned host memory to the device and reads every result back.
     Steps are pipelined the way a user would: copy-in, compute and copy-out run
@@ -826,6 +881,9 @@ def run_e2e(args, w, x, y, g, fwd, bwd, device, world):
     d2h = sum(t.numel() * t.element_size() for t in host_out.values())
     slots = [({k: torch.empty_like(x[k]) for k in names_in},
               {k: torch.empty_like(v) for k, v in out_like.items()}) for _ in range(2)]
+    nsaved = scan.saved_bytes(w.batch, w.dim, w.L, w.N, w.dtype) if pair else 0
+    saved = [torch.empty(nsaved, device=device, dtype=torch.uint8) if nsaved else None
+             for _ in range(2)]
     s_in, s_comp, s_out = (torch.cuda.Stream(device) for _ in range(3))
     ev = lambda: torch.cuda.Event()
     in_ready = [ev(), ev()]
@@ -845,11 +903,21 @@ def run_e2e(args, w, x, y, g, fwd, bwd, device, world):
         s_comp.wait_event(in_ready[k])
         if started[k]:
             s_comp.wait_event(out_done[k])  # step i-2's results have left this slot
-        scan.mamba_scan_fwd(xi["u"], xi["delta"], xi["delta_bias"], xi["A"], xi["B"], xi["C"],
-                            xi["D"], xi["z"], oi["y"], None, stream=s_comp)
-        scan.mamba_scan_bwd(xi["u"], xi["delta"], xi["delta_bias"], xi["A"], xi["B"], xi["C"],
-                            xi["D"], xi["z"], xi["dy"], oi["du"], oi["ddelta"], oi["dA"],
-                            oi["dB"], oi["dC"], oi["dD"], oi["dz"], oi["dbias"], stream=s_comp)
+        if pair:
+            scan.mamba_scan_fwd_save(xi["u"], xi["delta"], xi["delta_bias"], xi["A"], xi["B"],
+                                     xi["C"], xi["D"], xi["z"], oi["y"], None, saved[k],
+                                     stream=s_comp)
+            scan.mamba_scan_bwd_saved(xi["u"], xi["delta"], xi["delta_bias"], xi["A"], xi["B"],
+                                      xi["C"], xi["D"], xi["z"], xi["dy"], oi["du"], oi["ddelta"],
+                                      oi["dA"], oi["dB"], oi["dC"], oi["dD"], oi["dz"], oi["dbias"],
+                                      saved[k], stream=s_comp)
+        else:
+            scan.mamba_scan_fwd(xi["u"], xi["delta"], xi["delta_bias"], xi["A"], xi["B"],
+                                xi["C"], xi["D"], xi["z"], oi["y"], None, stream=s_comp)
+            scan.mamba_scan_bwd(xi["u"], xi["delta"], xi["delta_bias"], xi["A"], xi["B"],
+                                xi["C"], xi["D"], xi["z"], xi["dy"], oi["du"], oi["ddelta"],
+                                oi["dA"], oi["dB"], oi["dC"], oi["dD"], oi["dz"], oi["dbias"],
+                                stream=s_comp)
         comp_done[k].record(s_comp)
         s_out.wait_event(comp_done[k])
         with torch.cuda.stream(s_out):
@@ -915,7 +983,7 @@ def run_reference(args, world, rank):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(per * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{w.name} (forward + recompute backward per step)",
+        "config": {"workload": workload_label(w, args.step),
                    "batch": w.batch, "dim": w.dim, "L": w.L, "N": w.N,
                    "io_dtype": "bf16" if w.dtype == torch.bfloat16 else "fp32"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
@@ -933,6 +1001,9 @@ def main(argv=None):
     ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD,
                     help="index into the workload list (default: the bf16 2K-length one)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--step", choices=["pair", "recompute"], default="pair",
+                    help="the training step: the pair whose forward saves the 16-step states for "
+                         "its backward (default), or forward + the backward that re-runs it")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--cpu-threads", type=int, default=0,

@@ -158,6 +158,64 @@ MAMBA_SCAN_API mamba_status_t mamba_scan_bwd_ex(const void *u, const void *delta
                                  const mamba_scan_options_t *options, mamba_stream_t stream);
 
 /*
+ * The training pair: a forward that also stores what its backward would
+ * otherwise recompute, and a backward that reads it.  The recurrence is the
+ * one of mamba_scan_fwd ("Mamba: Linear-Time Sequence Modeling with Selective
+ * State Spaces", chapterpal.com, Knowl 1 "Selective State Space Model (S6)",
+ * the discretized recurrence; the backward as mamba_scan_bwd).  The stored
+ * states are the recurrence's h before every 16th step (for the three-phase
+ * carry: h from a zero state at each chunk start, with the chunk's entering
+ * state and the running sum of delta needed to complete it), so the backward
+ * skips the forward pass it would run first and re-runs only 16-step tiles.
+ *
+ * mamba_scan_saved_bytes writes into *bytes the size of the buffer `saved`
+ * for this shape, dtype and options on the current device.  It is 0 when the
+ * problem takes the one-thread-per-channel kernels (path REFERENCE, N <= 2,
+ * or rows of L * dtype size not a multiple of 16 bytes); the two calls are
+ * then mamba_scan_fwd_ex and mamba_scan_bwd_ex and `saved` may be NULL.
+ *
+ * mamba_scan_fwd_save: mamba_scan_fwd_ex (same arguments and results), and
+ * writes `saved` (device memory, 16-byte aligned, saved_bytes >= the size
+ * above; its contents are opaque).  With a nonzero size the staged kernels
+ * must take the call: u, delta, z, y, B and C 16-byte aligned, else
+ * MAMBA_ERR_INVALID_ARG (nothing enqueued).
+ *
+ * mamba_scan_bwd_saved: mamba_scan_bwd_ex (same arguments and results),
+ * reading `saved` as written by mamba_scan_fwd_save with the same u, delta,
+ * delta_bias, A, B, C, shape, dtype and options on the same device (any z,
+ * D and y; the stored states do not depend on them).  Stream order must put
+ * the forward before it; `saved` is not modified and may serve several
+ * backwards.  Anything else in `saved` gives undefined gradients.  The
+ * saved states are those the recomputing backward forms, by the same
+ * formulas on the same chunking when chunk_len and carry are automatic, so
+ * the gradients agree with mamba_scan_bwd_ex to rounding (bit for bit where
+ * the compiler forms both alike; the recomputing backward's own forward pass
+ * takes the automatic chunking whatever the options).  Only the plain
+ * scan has the pair (not the convolution prologue, the fused projection or
+ * complex A).
+ */
+MAMBA_SCAN_API mamba_status_t mamba_scan_saved_bytes(int64_t batch, int64_t dim, int64_t L, int64_t N,
+                                                     mamba_dtype_t dtype,
+                                                     const mamba_scan_options_t *options,
+                                                     uint64_t *bytes);
+
+MAMBA_SCAN_API mamba_status_t mamba_scan_fwd_save(const void *u, const void *delta,
+                                                  const float *delta_bias, const float *A,
+                                                  const void *B, const void *C, const float *D,
+                                                  const void *z, void *y, float *last_state,
+                                                  int64_t batch, int64_t dim, int64_t L, int64_t N,
+                                                  mamba_dtype_t dtype,
+                                                  const mamba_scan_options_t *options, void *saved,
+                                                  uint64_t saved_bytes, mamba_stream_t stream);
+
+MAMBA_SCAN_API mamba_status_t mamba_scan_bwd_saved(
+    const void *u, const void *delta, const float *delta_bias, const float *A, const void *B,
+    const void *C, const float *D, const void *z, const void *dy, void *du, void *ddelta, float *dA,
+    void *dB, void *dC, float *dD, void *dz, float *ddelta_bias, int64_t batch, int64_t dim, int64_t L,
+    int64_t N, mamba_dtype_t dtype, const mamba_scan_options_t *options, const void *saved,
+    uint64_t saved_bytes, mamba_stream_t stream);
+
+/*
  * Forward with the convolution prologue of the Mamba block: the main branch
  * runs a short causal 1D convolution and SiLU before the S6 layer
  * ("Mamba: Linear-Time Sequence Modeling with Selective State Spaces",

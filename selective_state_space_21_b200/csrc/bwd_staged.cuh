@@ -1224,9 +1224,19 @@ inline int proj_max_rank() {
   return r;
 }
 
+// With `saved` (the plain backward only: not with CONV or PROJ), the
+// checkpoints, range flags and (three-phase) h_in and sums of Delta come from
+// a saving forward of the same inputs and options, laid out as saved_layout
+// gives it, and the checkpoint pass does not run.
 template <typename T, int NM, bool CONV = false, bool PROJ = false>
 mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStream_t s,
-                               mamba_status_t (*launched)()) {
+                               mamba_status_t (*launched)(), const unsigned char *saved = nullptr) {
+  SavedLayout sl;
+  if (saved) {
+    if constexpr (CONV || PROJ) return MAMBA_ERR_UNSUPPORTED;
+    const mamba_status_t ls = saved_layout<T, NM>(a.batch, a.dim, a.L, o, &sl);
+    if (ls != MAMBA_OK) return ls;
+  }
   using Lay = BwdLayout<T, NM, !PROJ>;
   constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
   const uint64_t L = a.L, dim = a.dim, batch = a.batch, N = a.N;
@@ -1272,6 +1282,7 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
   //            (three-phase: + [agg_S][agg_G][gin])
   const size_t int_bytes = ceil_div((1 + size_t(G)) * 4, 256) * 256;
   const size_t n_ckpt = size_t(G) * size_t(n16) * NM * kSThreads;
+  const size_t n_ckpt_ws = saved ? 0 : n_ckpt;  // checkpoints in the workspace
   const size_t n_carry = size_t(G) * NM * kSThreads;
   const size_t n_bc = size_t(gpb) * size_t(a.batch) * 32 * size_t(a.L);
   const size_t gk = size_t(G) * size_t(pl.K);
@@ -1279,14 +1290,14 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
   const size_t n_par = par ? gk * NM * kSThreads : 0;  // agg_G and gin each
   // the fused projection's three-phase carry: delta in fp32 for the aggregate pass
   const size_t n_delta = (PROJ && par) ? size_t(a.batch) * size_t(a.dim) * size_t(a.L) : 0;
-  const size_t bytes_f = ceil_div(int_bytes + 4 * (n_ckpt + n_carry + n_bc + n_A + 2 * n_D + n_delta) +
+  const size_t bytes_f = ceil_div(int_bytes + 4 * (n_ckpt_ws + n_carry + n_bc + n_A + 2 * n_D + n_delta) +
                                       (par ? 8 * n_D + 8 * n_par : 0), 256) * 256;
   // the range flags of delta, written by the checkpoint pass (not with the
   // fused projection, which checks per tile, nor with the generic arithmetic
   // forced)
   const bool range = !PROJ && o.path != MAMBA_PATH_GENERIC;
   const size_t n_flags = range ? size_t(G) * size_t(ceil_div(a.L, kRangeBlock)) : 0;
-  const size_t bytes = bytes_f + ceil_div(n_flags, 256) * 256;
+  const size_t bytes = bytes_f + (saved ? 0 : ceil_div(n_flags, 256) * 256);
   // The checkpoint pass (the forward without y) is prepared first so that one
   // workspace holds both: a failed allocation then leaves nothing enqueued.
   FwdArgs fa;
@@ -1301,12 +1312,12 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
   fo.test_hook = 0;  // the hook targets the reverse hand-off
   StagedForward<T, NM, CONV, PROJ> ckpt_pass;
   unsigned char *ws = nullptr;
-  {
+  if (!saved) {
     // the checkpoint buffer is set once the workspace exists (before run)
     const mamba_status_t pst = ckpt_pass.prepare(fa, fo, nullptr, true);
     if (pst != MAMBA_OK) return pst;
   }
-  if (ws_alloc(reinterpret_cast<void **>(&ws), bytes + ckpt_pass.bytes, s) != cudaSuccess) {
+  if (ws_alloc(reinterpret_cast<void **>(&ws), bytes + (saved ? 0 : ckpt_pass.bytes), s) != cudaSuccess) {
     cudaGetLastError();
     return MAMBA_ERR_OUT_OF_MEMORY;
   }
@@ -1321,8 +1332,8 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
   bp.flags = bp.counter + 1;
   float *fws = reinterpret_cast<float *>(ws + int_bytes);
   float *ckpt = fws;
-  bp.ckpt = ckpt;
-  bp.carry = ckpt + n_ckpt;
+  bp.ckpt = saved ? reinterpret_cast<const float *>(saved + sl.ckpt) : ckpt;
+  bp.carry = ckpt + n_ckpt_ws;
   bp.part_bc = bp.carry + n_carry;
   bp.part_A = bp.part_bc + n_bc;
   bp.part_D = bp.part_A + n_A;
@@ -1344,7 +1355,7 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
   bp.n_bc = int64_t(n_bc);
   bp.n_unit = int64_t(n_D);
   bp.n_gin = int64_t(n_par);
-  bp.range_flags = range ? ws + bytes_f : nullptr;
+  bp.range_flags = !range ? nullptr : saved ? saved + sl.flags : ws + bytes_f;
   bp.n_flags = int64_t(n_flags);
   bp.timeout_ns = o.timeout_us > 0 ? uint64_t(o.timeout_us) * 1000ull : kDefaultTimeoutNs;
   bp.force_generic = o.path == MAMBA_PATH_GENERIC ? 1 : 0;
@@ -1352,7 +1363,15 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
 
   mamba_status_t st = MAMBA_OK;
   if (cudaMemsetAsync(ws, 0, int_bytes, s) != cudaSuccess) st = MAMBA_ERR_CUDA;
-  if (st == MAMBA_OK) {
+  if (saved && sl.n_hin > 0) {  // the forward's chunks ran from zero
+    bp.ckpt_hin = reinterpret_cast<const float *>(saved + sl.hin);
+    bp.ckpt_cum = reinterpret_cast<const float *>(saved + sl.cum);
+    bp.ckpt_chunk = sl.pl.chunk_len;
+    bp.ckpt_K = sl.pl.K;
+    bp.n_ckpt_hin = sl.n_hin;
+    bp.n_ckpt_cum = sl.n_cum;
+  }
+  if (st == MAMBA_OK && !saved) {
     ckpt_pass.sa.ckpt = ckpt;
     ckpt_pass.sa.delta_out = delta_f32;
     ckpt_pass.sa.range_flags = range ? ws + bytes_f : nullptr;

@@ -70,8 +70,13 @@ constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
 // contribution once the scan over chunks has produced it.  CKPT_LOC: the same
 // without y, storing the checkpoints of every chunk from zero with the sum of
 // Delta up to each; the reader of a checkpoint adds exp(A_n cum) h_in,n.
+// SEQ_SAVE, LOC_SAVE and PAR_SAVE: SEQ, LOC and PAR that also store the
+// checkpoints (and, for LOC, the sums of Delta up to them) and the
+// Delta-range flags, for a backward that reads them instead of re-running the
+// forward.
 enum StagedKind { KIND_SEQ = 0, KIND_PAR = 1, KIND_AGG = 2, KIND_CKPT_SEQ = 3, KIND_CKPT_PAR = 4,
-                  KIND_LOC = 5, KIND_CKPT_LOC = 6 };
+                  KIND_LOC = 5, KIND_CKPT_LOC = 6, KIND_SEQ_SAVE = 7, KIND_LOC_SAVE = 8,
+                  KIND_PAR_SAVE = 9 };
 constexpr int kCkptEvery = 16;
 enum UnitMode { MODE_SIG = 0, MODE_STRUCT = 1, MODE_GEN = 2 };
 
@@ -423,11 +428,16 @@ __global__ void __launch_bounds__(kSThreads, 2)
   constexpr int TT = Lay::TT, VEC = Lay::VEC, NV = Lay::NV, BSTR = Lay::BSTR;
   static_assert(!PROJ || (std::is_same<T, __nv_bfloat16>::value && !CONV),
                 "the fused projection takes bf16 operands and no convolution prologue");
-  constexpr bool kOut = KIND == KIND_SEQ || KIND == KIND_PAR || KIND == KIND_LOC;  // stores y
-  constexpr bool kAgg = KIND == KIND_AGG || KIND == KIND_LOC || KIND == KIND_CKPT_LOC;  // chunk aggregates
-  constexpr bool kSeq = KIND == KIND_SEQ || KIND == KIND_CKPT_SEQ;
-  constexpr bool kPar = KIND == KIND_PAR || KIND == KIND_CKPT_PAR;
-  constexpr bool kCkpt = KIND == KIND_CKPT_SEQ || KIND == KIND_CKPT_PAR || KIND == KIND_CKPT_LOC;
+  constexpr bool kLoc = KIND == KIND_LOC || KIND == KIND_LOC_SAVE;  // y from zero chunk starts
+  constexpr bool kOut = KIND == KIND_SEQ || KIND == KIND_PAR || kLoc || KIND == KIND_SEQ_SAVE ||
+                        KIND == KIND_PAR_SAVE;  // stores y
+  constexpr bool kAgg = KIND == KIND_AGG || kLoc || KIND == KIND_CKPT_LOC;  // chunk aggregates
+  constexpr bool kSeq = KIND == KIND_SEQ || KIND == KIND_CKPT_SEQ || KIND == KIND_SEQ_SAVE;
+  constexpr bool kPar = KIND == KIND_PAR || KIND == KIND_CKPT_PAR || KIND == KIND_PAR_SAVE;
+  constexpr bool kCkpt = KIND == KIND_CKPT_SEQ || KIND == KIND_CKPT_PAR || KIND == KIND_CKPT_LOC ||
+                         KIND == KIND_SEQ_SAVE || KIND == KIND_LOC_SAVE || KIND == KIND_PAR_SAVE;
+  // checkpoints of chunks run from zero: stored with the sums of Delta up to them
+  constexpr bool kCkptCum = KIND == KIND_CKPT_LOC || KIND == KIND_LOC_SAVE;
 
   // Offsetting the __shared__ array itself (not a cast integer) keeps every
   // derived pointer in the shared address space, so the compiler emits
@@ -753,7 +763,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
               const int64_t ci = ((int64_t(g) * ((f.L + kCkptEvery - 1) / kCkptEvery) +
                                    tj / kCkptEvery) * NM) * kSThreads + tid;
               float *dst = p.ckpt + (in_bounds(ci + (NM - 1) * kSThreads, p.n_ckpt) ? ci : 0);
-              if constexpr (KIND == KIND_CKPT_LOC) {  // Delta summed from the chunk's start
+              if constexpr (kCkptCum) {  // Delta summed from the chunk's start
                 const int64_t cc = (int64_t(g) * ((f.L + kCkptEvery - 1) / kCkptEvery) + tj / kCkptEvery) *
                                        kSThreads + tid;
                 if (in_bounds(cc, p.n_ckpt_cum)) p.ckpt_cum[cc] = float(Ssum + double(Stile));
@@ -856,7 +866,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
           if (kOut) *reinterpret_cast<uint4 *>(sy + off) = Vec<T>::pack(yv);
         }
         if constexpr (kAgg) Ssum += double(Stile);
-        if constexpr (KIND == KIND_LOC) {  // the block's running sum, where a block ends
+        if constexpr (kLoc) {  // the block's running sum, where a block ends
           if ((t0 + TT) % kCorrBlock == 0 || it + 1 == ntiles) {
             const int64_t bi = (int64_t(g) * ((f.L + kCorrBlock - 1) / kCorrBlock) + t0 / kCorrBlock) *
                                kSThreads + tid;
@@ -1196,13 +1206,18 @@ inline int device_sm_count() {
   return sms > 0 ? sms : 148;
 }
 
-// Whether the staged kernels can take this problem: rows of 16-byte
-// multiples, 16-byte aligned bases, N >= 3.
+// Whether the staged kernels can take a problem of this shape: rows of
+// 16-byte multiples, N >= 3, L and dim within the index limits.
+inline bool staged_shape_ok(int64_t L, int64_t dim, int64_t N, size_t es) {
+  if (N < 3) return false;
+  if ((L * int64_t(es)) % 16 != 0) return false;
+  return L <= (int64_t(1) << 31) - 1024 && dim <= (int64_t(1) << 31) - 1;
+}
+
+// ... and this problem: also 16-byte aligned bases.
 inline bool staged_supported(const FwdArgs &a, size_t es) {
   auto al = [](const void *ptr) { return ptr == nullptr || (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; };
-  if (a.N < 3) return false;
-  if ((a.L * int64_t(es)) % 16 != 0) return false;
-  if (a.L > (int64_t(1) << 31) - 1024 || a.dim > (int64_t(1) << 31) - 1) return false;
+  if (!staged_shape_ok(a.L, a.dim, a.N, es)) return false;
   return al(a.u) && al(a.delta) && al(a.z) && al(a.y) && al(a.B) && al(a.C);
 }
 
@@ -1290,6 +1305,66 @@ inline StagedPlan plan_staged(int64_t G, int64_t L, int slots, const StagedOptio
   return pl;
 }
 
+// The forward's chunking for a problem of this size on the current device
+// (what StagedForward::prepare decides, without tensor maps): G channel
+// groups, the plan, and the CTA slots of the main kernel.
+template <typename T, int NM, bool CONV = false, bool PROJ = false>
+inline mamba_status_t staged_forward_plan(int64_t batch, int64_t dim, int64_t L, const StagedOptions &o,
+                                          int smem, StagedPlan *pl, int64_t *G, int *sms, int *slots) {
+  int bps_main = 0;
+  if (prepare_kernel<T, NM, KIND_SEQ, CONV, PROJ>(&bps_main, smem) != cudaSuccess) return MAMBA_ERR_CUDA;
+  *sms = device_sm_count();
+  *slots = *sms * std::max(1, bps_main);
+  *G = batch * ceil_div(dim, kSThreads);
+  if (*G > (int64_t(1) << 30)) return MAMBA_ERR_UNSUPPORTED;
+  *pl = plan_staged(*G, L, *slots, o);
+  if (*G * pl->K > (int64_t(1) << 30)) return MAMBA_ERR_UNSUPPORTED;
+  return MAMBA_OK;
+}
+
+// What a saving forward stores for the backward (byte offsets into the
+// caller's buffer, each 256-byte aligned, and element counts):
+//   ckpt  [G][ceil(L/16)][NM][128] fp32  the state before every 16th step
+//   flags [G][ceil(L/64)] bytes         the Delta-range flags of the backward
+// and with the three-phase carry for 16-bit I/O, whose chunks run from zero
+// (LOC_SAVE; fp32 takes the aggregate pass and PAR_SAVE, whose checkpoints
+// are the true states),
+//   cum   [G][ceil(L/16)][128] fp32     Delta summed from the chunk's start
+//   hin   [G][K][NM][128] fp32          the state entering each chunk
+// (the backward adds exp(A_n cum) h_in,n to a checkpoint of chunk k >= 1).
+struct SavedLayout {
+  StagedPlan pl;
+  int64_t G = 0;
+  size_t ckpt = 0, flags = 0, cum = 0, hin = 0, bytes = 0;
+  int64_t n_ckpt = 0, n_flags = 0, n_cum = 0, n_hin = 0;
+};
+
+template <typename T, int NM>
+inline mamba_status_t saved_layout(int64_t batch, int64_t dim, int64_t L, const StagedOptions &o,
+                                   SavedLayout *out) {
+  SavedLayout sl;
+  int sms = 0, slots = 0;
+  const mamba_status_t st =
+      staged_forward_plan<T, NM>(batch, dim, L, o, StagedLayout<T, NM>::ALLOC, &sl.pl, &sl.G, &sms, &slots);
+  if (st != MAMBA_OK) return st;
+  auto up = [](size_t b) { return (b + 255) / 256 * 256; };
+  const int64_t n16 = ceil_div(L, kCkptEvery);
+  sl.n_ckpt = sl.G * n16 * NM * kSThreads;
+  sl.n_flags = sl.G * ceil_div(L, kRangeBlock);
+  sl.ckpt = 0;
+  sl.flags = up(size_t(sl.n_ckpt) * 4);
+  sl.bytes = sl.flags + up(size_t(sl.n_flags));
+  if (sl.pl.kind != KIND_SEQ && sizeof(T) == 2) {
+    sl.n_cum = sl.G * n16 * kSThreads;
+    sl.n_hin = sl.G * sl.pl.K * NM * kSThreads;
+    sl.cum = sl.bytes;
+    sl.hin = sl.cum + up(size_t(sl.n_cum) * 4);
+    sl.bytes = sl.hin + up(size_t(sl.n_hin) * 4);
+  }
+  *out = sl;
+  return MAMBA_OK;
+}
+
 // The staged forward, split into a preparation (tensor maps, plan, the
 // workspace size; nothing enqueued) and the launches on a given workspace, so
 // that a caller can take one workspace for several steps and fail before
@@ -1316,6 +1391,10 @@ struct StagedForward {
   // as it reads them (cum in sa.ckpt_cum, h_in in sa.hin).
   bool ckpt_loc = true;
   bool for_ckpt = false;  // prepared for a checkpoint pass
+  // A saving forward (set before prepare): y as usual, and the layout of
+  // what it stores for the backward into save_buf (set before run).
+  const SavedLayout *save = nullptr;
+  unsigned char *save_buf = nullptr;
   CUtensorMap maps[6];
   StagedArgs sa;
   StagedPlan pl;
@@ -1350,15 +1429,13 @@ struct StagedForward {
         !make_map_3d(&maps[5], a.C, bf16, L, N, batch, Lay::TT, uint32_t(N), none)) {
       return MAMBA_ERR_UNSUPPORTED;
     }
-    int bps_main = 0;
-    if (prepare_kernel<T, NM, KIND_SEQ, CONV, PROJ>(&bps_main, smem) != cudaSuccess) return MAMBA_ERR_CUDA;
-    sms = device_sm_count();
-    slots = sms * std::max(1, bps_main);
     const int64_t gpb = ceil_div(a.dim, kSThreads);
-    const int64_t G = int64_t(a.batch) * gpb;
-    if (G > (int64_t(1) << 30)) return MAMBA_ERR_UNSUPPORTED;
-    pl = plan_staged(G, a.L, slots, o);
-    if (G * pl.K > (int64_t(1) << 30)) return MAMBA_ERR_UNSUPPORTED;
+    int64_t G = 0;
+    {
+      const mamba_status_t st =
+          staged_forward_plan<T, NM, CONV, PROJ>(a.batch, a.dim, a.L, o, smem, &pl, &G, &sms, &slots);
+      if (st != MAMBA_OK) return st;
+    }
 
     sa.f = a;
     sa.G = int(G);
@@ -1385,6 +1462,9 @@ struct StagedForward {
     const size_t gk = size_t(G) * size_t(pl.K);
     if (pl.kind == KIND_SEQ) {
       bytes += size_t(G) * NM * kSThreads * 4;
+    } else if (save && sizeof(T) == 2) {  // agg_S, agg_h and the running sums (h_in is saved)
+      bytes += gk * kSThreads * 8 + gk * NM * kSThreads * 4 +
+               size_t(G) * size_t(ceil_div(a.L, kCorrBlock)) * kSThreads * 4;
     } else {
       bytes += gk * kSThreads * 8 + 2 * gk * NM * kSThreads * 4;
       if (for_ckpt && ckpt_loc)  // the CKPT_LOC pass's sums of Delta at the checkpoints
@@ -1413,6 +1493,73 @@ struct StagedForward {
     return launched();
   }
 
+  // The saving forward: SEQ_SAVE; for 16-bit I/O LOC_SAVE + scan +
+  // fwd_correct_kernel (with h_in and the checkpoints' sums of Delta in the
+  // saved buffer); for fp32 AGG + scan + PAR_SAVE.
+  mamba_status_t run_save(unsigned char *ws, cudaStream_t s, mamba_status_t (*launched)()) {
+    int *counters = reinterpret_cast<int *>(ws);
+    const size_t gk = size_t(sa.G) * size_t(pl.K);
+    sa.ckpt = reinterpret_cast<float *>(save_buf + save->ckpt);
+    sa.range_flags = sa.force_generic ? nullptr : save_buf + save->flags;
+    sa.n_flags = save->n_flags;
+    int bps = 0;
+    if (pl.kind == KIND_SEQ) {
+      if (prepare_kernel<T, NM, KIND_SEQ_SAVE, CONV, PROJ>(&bps, smem) != cudaSuccess) return MAMBA_ERR_CUDA;
+      sa.carry = reinterpret_cast<float *>(ws + int_bytes);
+      sa.counter = counters;
+      sa.n_units = int(gk);
+      launch_staged<T, NM, KIND_SEQ_SAVE, CONV, PROJ>(maps, sa, int(std::min<int64_t>(gk, sms * std::max(1, bps))),
+                                                      s, smem);
+      return launched();
+    }
+    if constexpr (sizeof(T) != 2) {
+      int bps_agg = 0;
+      if (prepare_kernel<T, NM, KIND_AGG, CONV, PROJ>(&bps_agg, smem) != cudaSuccess ||
+          prepare_kernel<T, NM, KIND_PAR_SAVE, CONV, PROJ>(&bps, smem) != cudaSuccess)
+        return MAMBA_ERR_CUDA;
+      sa.agg_S = reinterpret_cast<double *>(ws + int_bytes);
+      sa.agg_h = reinterpret_cast<float *>(ws + int_bytes + gk * kSThreads * 8);
+      sa.hin = sa.agg_h + gk * NM * kSThreads;
+      StagedArgs sg = sa;
+      sg.counter = counters;
+      sg.n_units = int(size_t(sa.G) * size_t(pl.K - 1));
+      launch_staged<T, NM, KIND_AGG, CONV, PROJ>(
+          maps, sg, int(std::min<int64_t>(sg.n_units, sms * std::max(1, bps_agg))), s, smem);
+      mamba_status_t st = launched();
+      if (st == MAMBA_OK) st = launch_chunk_scan(s, launched);
+      if (st == MAMBA_OK) {
+        StagedArgs sp = sa;
+        sp.counter = counters + 1;
+        sp.n_units = int(gk);
+        launch_staged<T, NM, KIND_PAR_SAVE, CONV, PROJ>(
+            maps, sp, int(std::min<int64_t>(gk, sms * std::max(1, bps))), s, smem);
+        st = launched();
+      }
+      return st;
+    }
+    if (prepare_kernel<T, NM, KIND_LOC_SAVE, CONV, PROJ>(&bps, smem) != cudaSuccess) return MAMBA_ERR_CUDA;
+    sa.agg_S = reinterpret_cast<double *>(ws + int_bytes);
+    sa.agg_h = reinterpret_cast<float *>(ws + int_bytes + gk * kSThreads * 8);
+    sa.blk_cum = sa.agg_h + gk * NM * kSThreads;
+    sa.n_blk = int64_t(sa.G) * ceil_div(sa.f.L, kCorrBlock) * kSThreads;
+    sa.hin = reinterpret_cast<float *>(save_buf + save->hin);
+    sa.ckpt_cum = reinterpret_cast<float *>(save_buf + save->cum);
+    sa.n_ckpt_cum = save->n_cum;
+    StagedArgs sl = sa;
+    sl.counter = counters;
+    sl.n_units = int(gk);
+    launch_staged<T, NM, KIND_LOC_SAVE, CONV, PROJ>(maps, sl, int(std::min<int64_t>(gk, sms * std::max(1, bps))),
+                                                    s, smem);
+    mamba_status_t st = launched();
+    if (st == MAMBA_OK) st = launch_chunk_scan(s, launched);
+    if (st == MAMBA_OK) {
+      const int64_t nb = ceil_div(sa.f.L, kCorrBlock) - pl.chunk_len / kCorrBlock;  // blocks of chunks 1..K-1
+      fwd_correct_kernel<T, NM><<<unsigned(int64_t(sa.G) * nb), kSThreads, 0, s>>>(sa);
+      st = launched();
+    }
+    return st;
+  }
+
   // Enqueues the launches on `ws` (at least `bytes`, 256-byte aligned).
   mamba_status_t run(unsigned char *ws, cudaStream_t s, mamba_status_t (*launched)()) {
     mamba_status_t st = MAMBA_OK;
@@ -1424,6 +1571,7 @@ struct StagedForward {
     sa.n_agg = int64_t(gk) * NM * kSThreads;
     sa.n_aggS = int64_t(gk) * kSThreads;
     sa.n_ckpt = int64_t(sa.G) * ((sa.f.L + kCkptEvery - 1) / kCkptEvery) * NM * kSThreads;
+    if (save) return run_save(ws, s, launched);
     if (pl.kind == KIND_SEQ) {
       sa.carry = reinterpret_cast<float *>(ws + int_bytes);
       sa.counter = counters;
@@ -1518,10 +1666,22 @@ struct StagedForward {
 // MAMBA_ERR_UNSUPPORTED (nothing enqueued) if the driver rejects a tensor map,
 // MAMBA_ERR_OUT_OF_MEMORY (nothing enqueued) if the workspace cannot be had.
 // CONV selects the kernels with the convolution prologue (a.conv_w set).
+// With `save` (the plain forward only: not with CONV or PROJ), the forward
+// also stores what the backward would recompute, laid out as saved_layout
+// gives it.
 template <typename T, int NM, bool CONV = false, bool PROJ = false>
 mamba_status_t staged_forward(const FwdArgs &a, const StagedOptions &o, cudaStream_t s,
-                              mamba_status_t (*launched)(), float *ckpt = nullptr) {
+                              mamba_status_t (*launched)(), float *ckpt = nullptr,
+                              unsigned char *save = nullptr) {
   StagedForward<T, NM, CONV, PROJ> sf;
+  SavedLayout lay;
+  if (save) {
+    if constexpr (CONV || PROJ) return MAMBA_ERR_UNSUPPORTED;  // only the plain forward saves
+    const mamba_status_t ls = saved_layout<T, NM>(a.batch, a.dim, a.L, o, &lay);
+    if (ls != MAMBA_OK) return ls;
+    sf.save = &lay;
+    sf.save_buf = save;
+  }
   mamba_status_t st = sf.prepare(a, o, ckpt);
   if (st != MAMBA_OK) return st;
   unsigned char *ws = nullptr;

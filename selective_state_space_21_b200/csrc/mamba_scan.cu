@@ -163,17 +163,44 @@ struct FwdReferenceLauncher {
 };
 
 template <typename T, bool CONV>
-mamba_status_t staged_bwd_dispatch(const BwdArgs &a, const StagedOptions &o, cudaStream_t s) {
-  if (a.N <= 4) return staged_backward<T, 4, CONV>(a, o, s, &launch_status);
-  if (a.N <= 8) return staged_backward<T, 8, CONV>(a, o, s, &launch_status);
-  return staged_backward<T, 16, CONV>(a, o, s, &launch_status);
+mamba_status_t staged_bwd_dispatch(const BwdArgs &a, const StagedOptions &o, cudaStream_t s,
+                                   const unsigned char *saved = nullptr) {
+  if (a.N <= 4) return staged_backward<T, 4, CONV>(a, o, s, &launch_status, saved);
+  if (a.N <= 8) return staged_backward<T, 8, CONV>(a, o, s, &launch_status, saved);
+  return staged_backward<T, 16, CONV>(a, o, s, &launch_status, saved);
 }
 
 template <typename T, bool CONV>
-mamba_status_t staged_dispatch(const FwdArgs &a, const StagedOptions &o, cudaStream_t s) {
-  if (a.N <= 4) return staged_forward<T, 4, CONV>(a, o, s, &launch_status);
-  if (a.N <= 8) return staged_forward<T, 8, CONV>(a, o, s, &launch_status);
-  return staged_forward<T, 16, CONV>(a, o, s, &launch_status);
+mamba_status_t staged_dispatch(const FwdArgs &a, const StagedOptions &o, cudaStream_t s,
+                               unsigned char *save = nullptr) {
+  if (a.N <= 4) return staged_forward<T, 4, CONV>(a, o, s, &launch_status, nullptr, save);
+  if (a.N <= 8) return staged_forward<T, 8, CONV>(a, o, s, &launch_status, nullptr, save);
+  return staged_forward<T, 16, CONV>(a, o, s, &launch_status, nullptr, save);
+}
+
+// Bytes a saving forward stores for its backward: 0 where the problem takes
+// the one-thread-per-channel kernels (then the saving calls are the plain
+// ones), else the layout of saved_layout on the current device.
+template <typename T>
+mamba_status_t saved_bytes_t(int64_t batch, int64_t dim, int64_t L, int64_t N, const StagedOptions &so,
+                             uint64_t *bytes) {
+  SavedLayout sl;
+  mamba_status_t st;
+  if (N <= 4) st = saved_layout<T, 4>(batch, dim, L, so, &sl);
+  else if (N <= 8) st = saved_layout<T, 8>(batch, dim, L, so, &sl);
+  else st = saved_layout<T, 16>(batch, dim, L, so, &sl);
+  *bytes = st == MAMBA_OK ? uint64_t(sl.bytes) : 0;
+  return st;
+}
+
+mamba_status_t saved_bytes_for(int64_t batch, int64_t dim, int64_t L, int64_t N, mamba_dtype_t dtype,
+                               const StagedOptions &so, uint64_t *bytes) {
+  *bytes = 0;
+  if (batch == 0 || dim == 0 || L == 0 || so.path == MAMBA_PATH_REFERENCE ||
+      !staged_shape_ok(L, dim, N, dtype_size(dtype)))
+    return MAMBA_OK;
+  return dtype == MAMBA_BF16 ? saved_bytes_t<__nv_bfloat16>(batch, dim, L, N, so, bytes)
+                             : saved_bytes_t<float>(batch, dim, L, N, so, bytes);
 }
 
 template <typename T, int NM>
@@ -356,8 +383,13 @@ StagedOptions staged_options(const mamba_scan_options_t *options) {
 // kernel (which handles the prologue at run time).
 template <bool CONV>
 mamba_status_t forward_paths(const FwdArgs &a, size_t es, mamba_dtype_t dtype,
-                             const StagedOptions &so, cudaStream_t s) {
+                             const StagedOptions &so, cudaStream_t s, unsigned char *save = nullptr) {
   const bool stageable = staged_supported(a, es);
+  if (save) {  // a saving forward: the staged kernels, no other path
+    if (!stageable) return MAMBA_ERR_INVALID_ARG;
+    return dtype == MAMBA_BF16 ? staged_dispatch<__nv_bfloat16, CONV>(a, so, s, save)
+                               : staged_dispatch<float, CONV>(a, so, s, save);
+  }
   if (so.path == MAMBA_PATH_REFERENCE || (!stageable && so.path == MAMBA_PATH_AUTO))
     return dispatch<FwdReferenceLauncher>(dtype, a.N, a, s);
   if (!stageable) return MAMBA_ERR_UNSUPPORTED;
@@ -370,8 +402,14 @@ mamba_status_t forward_paths(const FwdArgs &a, size_t es, mamba_dtype_t dtype,
 
 template <bool CONV>
 mamba_status_t backward_paths(const BwdArgs &a, size_t es, mamba_dtype_t dtype,
-                              const StagedOptions &so, cudaStream_t s) {
+                              const StagedOptions &so, cudaStream_t s,
+                              const unsigned char *saved = nullptr) {
   const bool stageable = staged_bwd_supported(a, es);
+  if (saved) {  // from a saving forward: the staged kernels, no other path
+    if (!stageable) return MAMBA_ERR_INVALID_ARG;
+    return dtype == MAMBA_BF16 ? staged_bwd_dispatch<__nv_bfloat16, CONV>(a, so, s, saved)
+                               : staged_bwd_dispatch<float, CONV>(a, so, s, saved);
+  }
   if (so.path == MAMBA_PATH_REFERENCE || (!stageable && so.path == MAMBA_PATH_AUTO))
     return dispatch<BwdReferenceLauncher>(dtype, a.N, a, s);
   if (!stageable) return MAMBA_ERR_UNSUPPORTED;
@@ -507,6 +545,126 @@ mamba_status_t proj_grads(const ProjGradPlan &pl, float *part, const void *W, co
   return launch_status();
 }
 
+// The forward and backward entry points with and without a saved buffer
+// (`saving`: the calls of the saving pair, whose buffer holds
+// mamba_scan_saved_bytes bytes or more).
+mamba_status_t fwd_entry(const void *u, const void *delta, const float *delta_bias,
+                                 const float *A, const void *B, const void *C, const float *D,
+                                 const void *z, void *y, float *last_state, int64_t batch,
+                                 int64_t dim, int64_t L, int64_t N, mamba_dtype_t dtype,
+                                 const mamba_scan_options_t *options, mamba_stream_t stream,
+                                 bool saving, void *saved, uint64_t saved_bytes) {
+  mamba_status_t st = check_shape(batch, dim, L, N, dtype);
+  if (st != MAMBA_OK) return st;
+  if ((st = check_options(options)) != MAMBA_OK) return st;
+  Checker ck;
+  if (cudaGetDevice(&ck.dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MAMBA_ERR_CUDA;
+  }
+  const size_t es = dtype_size(dtype);
+  const size_t nbdl = size_t(batch) * size_t(dim) * size_t(L);
+  const size_t nbnl = size_t(batch) * size_t(N) * size_t(L);
+  ck.buf(u, nbdl * es, es, true, false);
+  ck.buf(delta, nbdl * es, es, true, false);
+  ck.buf(z, nbdl * es, es, false, false);
+  ck.buf(B, nbnl * es, es, true, false);
+  ck.buf(C, nbnl * es, es, true, false);
+  ck.buf(A, size_t(dim) * N * 4, 4, true, false);
+  ck.buf(D, size_t(dim) * 4, 4, false, false);
+  ck.buf(delta_bias, size_t(dim) * 4, 4, false, false);
+  ck.buf(y, nbdl * es, es, true, true);
+  ck.buf(last_state, size_t(batch) * dim * N * 4, 4, false, true);
+  const StagedOptions so = staged_options(options);
+  uint64_t need = 0;
+  if (saving) {  // what this forward stores for its backward (0: nothing)
+    if ((st = saved_bytes_for(batch, dim, L, N, dtype, so, &need)) != MAMBA_OK) return st;
+    if (need > saved_bytes) return MAMBA_ERR_INVALID_ARG;
+    ck.buf(saved, need, 16, true, true);
+  }
+  if (ck.st != MAMBA_OK) return ck.st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (batch == 0 || dim == 0) return MAMBA_OK;
+  if (L == 0) {
+    if (last_state && cudaMemsetAsync(last_state, 0, size_t(batch) * dim * N * 4, s) != cudaSuccess)
+      return cuda_status();
+    return MAMBA_OK;
+  }
+  FwdArgs a;
+  a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
+  a.bias = delta_bias; a.A = A; a.D = D; a.y = y; a.last_state = last_state;
+  a.batch = batch; a.dim = dim; a.L = L; a.N = (int)N;
+  return forward_paths<false>(a, es, dtype, so, s, need ? static_cast<unsigned char *>(saved) : nullptr);
+}
+
+
+mamba_status_t bwd_entry(const void *u, const void *delta, const float *delta_bias,
+                                 const float *A, const void *B, const void *C, const float *D,
+                                 const void *z, const void *dy, void *du, void *ddelta,
+                                 float *dA, void *dB, void *dC, float *dD, void *dz,
+                                 float *ddelta_bias, int64_t batch, int64_t dim, int64_t L,
+                                 int64_t N, mamba_dtype_t dtype,
+                                 const mamba_scan_options_t *options, mamba_stream_t stream,
+                                 bool saving, const void *saved, uint64_t saved_bytes) {
+  mamba_status_t st = check_shape(batch, dim, L, N, dtype);
+  if (st != MAMBA_OK) return st;
+  if ((st = check_options(options)) != MAMBA_OK) return st;
+  if ((z == nullptr) != (dz == nullptr) || (D == nullptr) != (dD == nullptr))
+    return MAMBA_ERR_INVALID_ARG;
+  Checker ck;
+  if (cudaGetDevice(&ck.dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MAMBA_ERR_CUDA;
+  }
+  const size_t es = dtype_size(dtype);
+  const size_t nbdl = size_t(batch) * size_t(dim) * size_t(L);
+  const size_t nbnl = size_t(batch) * size_t(N) * size_t(L);
+  ck.buf(u, nbdl * es, es, true, false);
+  ck.buf(delta, nbdl * es, es, true, false);
+  ck.buf(z, nbdl * es, es, false, false);
+  ck.buf(dy, nbdl * es, es, true, false);
+  ck.buf(B, nbnl * es, es, true, false);
+  ck.buf(C, nbnl * es, es, true, false);
+  ck.buf(A, size_t(dim) * N * 4, 4, true, false);
+  ck.buf(D, size_t(dim) * 4, 4, false, false);
+  ck.buf(delta_bias, size_t(dim) * 4, 4, false, false);
+  ck.buf(du, nbdl * es, es, true, true);
+  ck.buf(ddelta, nbdl * es, es, true, true);
+  ck.buf(dz, nbdl * es, es, false, true);
+  ck.buf(dB, nbnl * es, es, true, true);
+  ck.buf(dC, nbnl * es, es, true, true);
+  ck.buf(dA, size_t(dim) * N * 4, 4, true, true);
+  ck.buf(dD, size_t(dim) * 4, 4, false, true);
+  ck.buf(ddelta_bias, size_t(dim) * 4, 4, false, true);
+  const StagedOptions so = staged_options(options);
+  uint64_t need = 0;
+  if (saving) {  // what the saving forward stored (0: nothing; recompute)
+    if ((st = saved_bytes_for(batch, dim, L, N, dtype, so, &need)) != MAMBA_OK) return st;
+    if (need > saved_bytes) return MAMBA_ERR_INVALID_ARG;
+    ck.buf(saved, need, 16, true, false);
+  }
+  if (ck.st != MAMBA_OK) return ck.st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (dim == 0) return MAMBA_OK;
+  if (batch == 0 || L == 0) {
+    // Empty sum: parameter gradients are zero, and dB / dC have no elements
+    // unless batch > 0 and L > 0.
+    if (cudaMemsetAsync(dA, 0, size_t(dim) * N * 4, s) != cudaSuccess) return cuda_status();
+    if (dD && cudaMemsetAsync(dD, 0, size_t(dim) * 4, s) != cudaSuccess) return cuda_status();
+    if (ddelta_bias && cudaMemsetAsync(ddelta_bias, 0, size_t(dim) * 4, s) != cudaSuccess)
+      return cuda_status();
+    return MAMBA_OK;
+  }
+  BwdArgs a;
+  a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C; a.dy = dy;
+  a.bias = delta_bias; a.A = A; a.D = D;
+  a.du = du; a.ddelta = ddelta; a.dz = dz; a.dB = dB; a.dC = dC;
+  a.dA = dA; a.dD = dD; a.dbias = ddelta_bias;
+  a.batch = batch; a.dim = dim; a.L = L; a.N = (int)N;
+  return backward_paths<false>(a, es, dtype, so, s,
+                               need ? static_cast<const unsigned char *>(saved) : nullptr);
+}
+
 }  // namespace
 
 extern "C" {
@@ -548,40 +706,29 @@ mamba_status_t mamba_scan_fwd_ex(const void *u, const void *delta, const float *
                                  const void *z, void *y, float *last_state, int64_t batch,
                                  int64_t dim, int64_t L, int64_t N, mamba_dtype_t dtype,
                                  const mamba_scan_options_t *options, mamba_stream_t stream) {
+  return fwd_entry(u, delta, delta_bias, A, B, C, D, z, y, last_state, batch, dim, L, N, dtype, options,
+                   stream, false, nullptr, 0);
+}
+
+mamba_status_t mamba_scan_saved_bytes(int64_t batch, int64_t dim, int64_t L, int64_t N,
+                                      mamba_dtype_t dtype, const mamba_scan_options_t *options,
+                                      uint64_t *bytes) {
+  if (!bytes) return MAMBA_ERR_INVALID_ARG;
+  *bytes = 0;
   mamba_status_t st = check_shape(batch, dim, L, N, dtype);
   if (st != MAMBA_OK) return st;
   if ((st = check_options(options)) != MAMBA_OK) return st;
-  Checker ck;
-  if (cudaGetDevice(&ck.dev) != cudaSuccess) {
-    cudaGetLastError();
-    return MAMBA_ERR_CUDA;
-  }
-  const size_t es = dtype_size(dtype);
-  const size_t nbdl = size_t(batch) * size_t(dim) * size_t(L);
-  const size_t nbnl = size_t(batch) * size_t(N) * size_t(L);
-  ck.buf(u, nbdl * es, es, true, false);
-  ck.buf(delta, nbdl * es, es, true, false);
-  ck.buf(z, nbdl * es, es, false, false);
-  ck.buf(B, nbnl * es, es, true, false);
-  ck.buf(C, nbnl * es, es, true, false);
-  ck.buf(A, size_t(dim) * N * 4, 4, true, false);
-  ck.buf(D, size_t(dim) * 4, 4, false, false);
-  ck.buf(delta_bias, size_t(dim) * 4, 4, false, false);
-  ck.buf(y, nbdl * es, es, true, true);
-  ck.buf(last_state, size_t(batch) * dim * N * 4, 4, false, true);
-  if (ck.st != MAMBA_OK) return ck.st;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (batch == 0 || dim == 0) return MAMBA_OK;
-  if (L == 0) {
-    if (last_state && cudaMemsetAsync(last_state, 0, size_t(batch) * dim * N * 4, s) != cudaSuccess)
-      return cuda_status();
-    return MAMBA_OK;
-  }
-  FwdArgs a;
-  a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
-  a.bias = delta_bias; a.A = A; a.D = D; a.y = y; a.last_state = last_state;
-  a.batch = batch; a.dim = dim; a.L = L; a.N = (int)N;
-  return forward_paths<false>(a, es, dtype, staged_options(options), s);
+  return saved_bytes_for(batch, dim, L, N, dtype, staged_options(options), bytes);
+}
+
+mamba_status_t mamba_scan_fwd_save(const void *u, const void *delta, const float *delta_bias,
+                                   const float *A, const void *B, const void *C, const float *D,
+                                   const void *z, void *y, float *last_state, int64_t batch,
+                                   int64_t dim, int64_t L, int64_t N, mamba_dtype_t dtype,
+                                   const mamba_scan_options_t *options, void *saved,
+                                   uint64_t saved_bytes, mamba_stream_t stream) {
+  return fwd_entry(u, delta, delta_bias, A, B, C, D, z, y, last_state, batch, dim, L, N, dtype, options,
+                   stream, true, saved, saved_bytes);
 }
 
 mamba_status_t mamba_scan_fwd(const void *u, const void *delta, const float *delta_bias,
@@ -600,55 +747,20 @@ mamba_status_t mamba_scan_bwd_ex(const void *u, const void *delta, const float *
                                  float *ddelta_bias, int64_t batch, int64_t dim, int64_t L,
                                  int64_t N, mamba_dtype_t dtype,
                                  const mamba_scan_options_t *options, mamba_stream_t stream) {
-  mamba_status_t st = check_shape(batch, dim, L, N, dtype);
-  if (st != MAMBA_OK) return st;
-  if ((st = check_options(options)) != MAMBA_OK) return st;
-  if ((z == nullptr) != (dz == nullptr) || (D == nullptr) != (dD == nullptr))
-    return MAMBA_ERR_INVALID_ARG;
-  Checker ck;
-  if (cudaGetDevice(&ck.dev) != cudaSuccess) {
-    cudaGetLastError();
-    return MAMBA_ERR_CUDA;
-  }
-  const size_t es = dtype_size(dtype);
-  const size_t nbdl = size_t(batch) * size_t(dim) * size_t(L);
-  const size_t nbnl = size_t(batch) * size_t(N) * size_t(L);
-  ck.buf(u, nbdl * es, es, true, false);
-  ck.buf(delta, nbdl * es, es, true, false);
-  ck.buf(z, nbdl * es, es, false, false);
-  ck.buf(dy, nbdl * es, es, true, false);
-  ck.buf(B, nbnl * es, es, true, false);
-  ck.buf(C, nbnl * es, es, true, false);
-  ck.buf(A, size_t(dim) * N * 4, 4, true, false);
-  ck.buf(D, size_t(dim) * 4, 4, false, false);
-  ck.buf(delta_bias, size_t(dim) * 4, 4, false, false);
-  ck.buf(du, nbdl * es, es, true, true);
-  ck.buf(ddelta, nbdl * es, es, true, true);
-  ck.buf(dz, nbdl * es, es, false, true);
-  ck.buf(dB, nbnl * es, es, true, true);
-  ck.buf(dC, nbnl * es, es, true, true);
-  ck.buf(dA, size_t(dim) * N * 4, 4, true, true);
-  ck.buf(dD, size_t(dim) * 4, 4, false, true);
-  ck.buf(ddelta_bias, size_t(dim) * 4, 4, false, true);
-  if (ck.st != MAMBA_OK) return ck.st;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (dim == 0) return MAMBA_OK;
-  if (batch == 0 || L == 0) {
-    // Empty sum: parameter gradients are zero, and dB / dC have no elements
-    // unless batch > 0 and L > 0.
-    if (cudaMemsetAsync(dA, 0, size_t(dim) * N * 4, s) != cudaSuccess) return cuda_status();
-    if (dD && cudaMemsetAsync(dD, 0, size_t(dim) * 4, s) != cudaSuccess) return cuda_status();
-    if (ddelta_bias && cudaMemsetAsync(ddelta_bias, 0, size_t(dim) * 4, s) != cudaSuccess)
-      return cuda_status();
-    return MAMBA_OK;
-  }
-  BwdArgs a;
-  a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C; a.dy = dy;
-  a.bias = delta_bias; a.A = A; a.D = D;
-  a.du = du; a.ddelta = ddelta; a.dz = dz; a.dB = dB; a.dC = dC;
-  a.dA = dA; a.dD = dD; a.dbias = ddelta_bias;
-  a.batch = batch; a.dim = dim; a.L = L; a.N = (int)N;
-  return backward_paths<false>(a, es, dtype, staged_options(options), s);
+  return bwd_entry(u, delta, delta_bias, A, B, C, D, z, dy, du, ddelta, dA, dB, dC, dD, dz, ddelta_bias,
+                   batch, dim, L, N, dtype, options, stream, false, nullptr, 0);
+}
+
+mamba_status_t mamba_scan_bwd_saved(const void *u, const void *delta, const float *delta_bias,
+                                    const float *A, const void *B, const void *C, const float *D,
+                                    const void *z, const void *dy, void *du, void *ddelta,
+                                    float *dA, void *dB, void *dC, float *dD, void *dz,
+                                    float *ddelta_bias, int64_t batch, int64_t dim, int64_t L,
+                                    int64_t N, mamba_dtype_t dtype,
+                                    const mamba_scan_options_t *options, const void *saved,
+                                    uint64_t saved_bytes, mamba_stream_t stream) {
+  return bwd_entry(u, delta, delta_bias, A, B, C, D, z, dy, du, ddelta, dA, dB, dC, dD, dz, ddelta_bias,
+                   batch, dim, L, N, dtype, options, stream, true, saved, saved_bytes);
 }
 
 }  // extern "C"

@@ -73,6 +73,13 @@ def load_library():
             lib.mamba_scan_bwd.argtypes = [vp] * 17 + [i64] * 4 + [i32, vp]
             lib.mamba_scan_bwd_ex.argtypes = [vp] * 17 + [i64] * 4 + [i32, opt, vp]
             lib.mamba_scan_fwd_noalloc.argtypes = [vp] * 10 + [i64] * 4 + [i32, vp]
+            u64 = ctypes.c_uint64
+            lib.mamba_scan_saved_bytes.argtypes = [i64] * 4 + [i32, opt, ctypes.POINTER(u64)]
+            lib.mamba_scan_saved_bytes.restype = ctypes.c_int
+            lib.mamba_scan_fwd_save.argtypes = [vp] * 10 + [i64] * 4 + [i32, opt, vp, u64, vp]
+            lib.mamba_scan_fwd_save.restype = ctypes.c_int
+            lib.mamba_scan_bwd_saved.argtypes = [vp] * 17 + [i64] * 4 + [i32, opt, vp, u64, vp]
+            lib.mamba_scan_bwd_saved.restype = ctypes.c_int
             lib.mamba_scan_step.argtypes = [vp] * 10 + [i64] * 3 + [i32, vp]
             lib.mamba_scan_step.restype = ctypes.c_int
             lib.mamba_conv_scan_step.argtypes = [vp] * 5 + [i64] + [vp] * 8 + [i64] * 3 + [i32, vp]
@@ -222,6 +229,81 @@ def mamba_scan_bwd(u, delta, delta_bias, A, B, C, D, z, dy, du, ddelta, dA, dB, 
         opts = _options(path, chunk_len, carry, wait_timeout_us, test_hook)
         rc = lib.mamba_scan_bwd_ex(*args, ctypes.byref(opts), _stream_handle(stream))
     _check(rc, "mamba_scan_bwd")
+
+
+def saved_bytes(batch, dim, L, N, dtype, *, path="auto", chunk_len=0, carry="auto",
+                wait_timeout_us=0, test_hook=0) -> int:
+    """Bytes of the buffer the saving forward (``mamba_scan_fwd_save``) fills
+    for its backward on the current device; 0 where the problem takes the
+    one-thread-per-channel kernels (then the pair is the plain forward and
+    backward, and ``saved`` may be None)."""
+    n = ctypes.c_uint64(0)
+    opts = _opts_ptr(path, chunk_len, carry, wait_timeout_us, test_hook)
+    _check(load_library().mamba_scan_saved_bytes(batch, dim, L, N, _dtype_code(dtype), opts,
+                                                 ctypes.byref(n)), "mamba_scan_saved_bytes")
+    return int(n.value)
+
+
+def _saved_arg(saved, need, name="saved"):
+    if need == 0:
+        return None, 0
+    if saved is None or saved.dtype != torch.uint8:
+        raise TypeError(f"{name} must be a uint8 CUDA tensor of at least {need} bytes")
+    if saved.numel() < need:
+        raise ValueError(f"{name} holds {saved.numel()} bytes; {need} are needed")
+    return _ptr(saved, torch.uint8, None, name), saved.numel()
+
+
+def mamba_scan_fwd_save(u, delta, delta_bias, A, B, C, D, z, y, last_state, saved, *,
+                        path="auto", chunk_len=0, carry="auto", wait_timeout_us=0, test_hook=0,
+                        stream=None):
+    """``mamba_scan_fwd`` that also fills ``saved`` (a uint8 CUDA tensor of
+    ``saved_bytes(...)`` bytes) with what ``mamba_scan_bwd_saved`` reads in
+    place of re-running the forward."""
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    dt = u.dtype
+    f32 = torch.float32
+    need = saved_bytes(batch, dim, L, N, dt, path=path, chunk_len=chunk_len, carry=carry,
+                       wait_timeout_us=wait_timeout_us, test_hook=test_hook)
+    sp, sn = _saved_arg(saved, need)
+    args = [
+        _ptr(u, dt, (batch, dim, L), "u"), _ptr(delta, dt, (batch, dim, L), "delta"),
+        _ptr(delta_bias, f32, (dim,), "delta_bias"), _ptr(A, f32, (dim, N), "A"),
+        _ptr(B, dt, (batch, N, L), "B"), _ptr(C, dt, (batch, N, L), "C"),
+        _ptr(D, f32, (dim,), "D"), _ptr(z, dt, (batch, dim, L), "z"),
+        _ptr(y, dt, (batch, dim, L), "y"), _ptr(last_state, f32, (batch, dim, N), "last_state"),
+        batch, dim, L, N, _dtype_code(dt)]
+    opts = _opts_ptr(path, chunk_len, carry, wait_timeout_us, test_hook)
+    _check(load_library().mamba_scan_fwd_save(*args, opts, sp, sn, _stream_handle(stream)),
+           "mamba_scan_fwd_save")
+
+
+def mamba_scan_bwd_saved(u, delta, delta_bias, A, B, C, D, z, dy, du, ddelta, dA, dB, dC, dD, dz,
+                         ddelta_bias, saved, *, path="auto", chunk_len=0, carry="auto",
+                         wait_timeout_us=0, test_hook=0, stream=None):
+    """``mamba_scan_bwd`` reading ``saved`` as ``mamba_scan_fwd_save`` wrote it
+    (same inputs and options) instead of re-running the forward."""
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    dt = u.dtype
+    f32 = torch.float32
+    bdl, bnl = (batch, dim, L), (batch, N, L)
+    need = saved_bytes(batch, dim, L, N, dt, path=path, chunk_len=chunk_len, carry=carry,
+                       wait_timeout_us=wait_timeout_us, test_hook=test_hook)
+    sp, sn = _saved_arg(saved, need)
+    args = [
+        _ptr(u, dt, bdl, "u"), _ptr(delta, dt, bdl, "delta"),
+        _ptr(delta_bias, f32, (dim,), "delta_bias"), _ptr(A, f32, (dim, N), "A"),
+        _ptr(B, dt, bnl, "B"), _ptr(C, dt, bnl, "C"), _ptr(D, f32, (dim,), "D"),
+        _ptr(z, dt, bdl, "z"), _ptr(dy, dt, bdl, "dy"), _ptr(du, dt, bdl, "du"),
+        _ptr(ddelta, dt, bdl, "ddelta"), _ptr(dA, f32, (dim, N), "dA"),
+        _ptr(dB, dt, bnl, "dB"), _ptr(dC, dt, bnl, "dC"), _ptr(dD, f32, (dim,), "dD"),
+        _ptr(dz, dt, bdl, "dz"), _ptr(ddelta_bias, f32, (dim,), "ddelta_bias"),
+        batch, dim, L, N, _dtype_code(dt)]
+    opts = _opts_ptr(path, chunk_len, carry, wait_timeout_us, test_hook)
+    _check(load_library().mamba_scan_bwd_saved(*args, opts, sp, sn, _stream_handle(stream)),
+           "mamba_scan_bwd_saved")
 
 
 def _opts_ptr(path, chunk_len, carry, wait_timeout_us, test_hook):
@@ -468,15 +550,27 @@ class StepPlan:
             _ptr(z, dt, (batch, dim), "z"), _ptr(y, dt, (batch, dim), "y"),
             batch, dim, N, _dtype_code(dt))
         _check(rc, "mamba_scan_step_plan_create")
+        # what run() needs, looked up once: the entry point, the handle as an
+        # integer, the plan's device and torch's raw-stream query
+        self._run = self._lib.mamba_scan_step_plan_run
+        self._hv = self._h.value
+        self._dev = u.device.index if u.device.index is not None else torch.cuda.current_device()
+        self._raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
 
     def run(self, stream=None):
-        _check(self._lib.mamba_scan_step_plan_run(self._h, _stream_handle(stream)),
-               "mamba_scan_step_plan_run")
+        if stream is None and self._raw is not None:
+            s = self._raw(self._dev)  # torch's current stream on the plan's device
+        else:
+            s = _stream_handle(stream)
+        rc = self._run(self._hv, s)
+        if rc:
+            _check(rc, "mamba_scan_step_plan_run")
 
     def close(self):
         if self._h:
             self._lib.mamba_scan_step_plan_destroy(self._h)
             self._h = ctypes.c_void_p()
+            self._hv = None
 
     def __del__(self):
         try:
@@ -549,6 +643,46 @@ def selective_scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, p
     mamba_scan_bwd(u, delta, delta_bias, A, B, C, D, z, dy, g["du"], g["ddelta"], g["dA"],
                    g["dB"], g["dC"], g["dD"], g["dz"], g["ddelta_bias"], path=path,
                    chunk_len=chunk_len, carry=carry, stream=stream)
+    return {k: v for k, v in g.items() if v is not None}
+
+
+def selective_scan_fwd_save(u, delta, A, B, C, D=None, z=None, delta_bias=None,
+                            return_last_state=False, path="auto", chunk_len=0, carry="auto",
+                            stream=None):
+    """The forward of the training pair: allocates y (and last_state) and the
+    saved buffer, runs ``mamba_scan_fwd_save``; returns (y, saved) or
+    (y, last_state, saved).  ``saved`` is None where the problem saves
+    nothing (``saved_bytes`` 0)."""
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    y = torch.empty_like(u)
+    last = (torch.empty(batch, dim, N, device=u.device, dtype=torch.float32)
+            if return_last_state else None)
+    need = saved_bytes(batch, dim, L, N, u.dtype, path=path, chunk_len=chunk_len, carry=carry)
+    saved = torch.empty(need, device=u.device, dtype=torch.uint8) if need else None
+    mamba_scan_fwd_save(u, delta, delta_bias, A, B, C, D, z, y, last, saved, path=path,
+                        chunk_len=chunk_len, carry=carry, stream=stream)
+    return (y, last, saved) if return_last_state else (y, saved)
+
+
+def selective_scan_bwd_saved(u, delta, A, B, C, dy, saved, D=None, z=None, delta_bias=None,
+                             path="auto", chunk_len=0, carry="auto", stream=None) -> dict:
+    """The backward of the training pair (``saved`` from
+    ``selective_scan_fwd_save`` with the same inputs and options); returns
+    the gradients as ``selective_scan_bwd`` does."""
+    dim, N = A.shape
+    f32 = torch.float32
+    g = {
+        "du": torch.empty_like(u), "ddelta": torch.empty_like(u),
+        "dA": torch.empty(dim, N, device=u.device, dtype=f32),
+        "dB": torch.empty_like(B), "dC": torch.empty_like(C),
+        "dD": torch.empty(dim, device=u.device, dtype=f32) if D is not None else None,
+        "dz": torch.empty_like(u) if z is not None else None,
+        "ddelta_bias": torch.empty(dim, device=u.device, dtype=f32),
+    }
+    mamba_scan_bwd_saved(u, delta, delta_bias, A, B, C, D, z, dy, g["du"], g["ddelta"], g["dA"],
+                         g["dB"], g["dC"], g["dD"], g["dz"], g["ddelta_bias"], saved, path=path,
+                         chunk_len=chunk_len, carry=carry, stream=stream)
     return {k: v for k, v in g.items() if v is not None}
 
 
