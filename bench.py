@@ -131,9 +131,10 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_bytes_per_launch_bf16_b8_d51
 
 
 def ncu_traffic(kernel_key: str):
-    """Per-launch DRAM bytes of one call ("fwd" or "bwd") from the committed ncu
-    summary, only if it was taken on the current source of the staged kernels
-    (else None).  Lines: <call> <bytes> <source digest> <launches>; # comments."""
+    """Per-launch DRAM bytes of one call ("fwd_save", "bwd_saved", "fwd" or
+    "bwd") from the committed ncu summary, only if it was taken on the current
+    source of the staged kernels (else None).  Lines: <call> <bytes> <source
+    digest> <launches>; # comments."""
     try:
         from selective_state_space_21_b200.build import STAGED_KERNEL_FILES, source_digest
         with open(TRAFFIC_FILE) as f:
@@ -453,8 +454,8 @@ def run_ours(args, world, rank, device):
                 "ops_per_launch": ops, "ops_per_element": ops_per_element,
                 "peak_source": alu_src, "ms_per_launch": round(ms, 4), "hbm_frac": hbm["frac"]}
 
-    alu_fwd = roof_alu("fwd", FWD_FP32_OPS_PER_ELEMENT, fwd_ms_max, roof_fwd)
-    alu_bwd = roof_alu("bwd", BWD_FP32_OPS_PER_ELEMENT, bwd_ms_max, roof_bwd)
+    alu_fwd = roof_alu(roof_fwd["kernel"], FWD_FP32_OPS_PER_ELEMENT, fwd_ms_max, roof_fwd)
+    alu_bwd = roof_alu(roof_bwd["kernel"], BWD_FP32_OPS_PER_ELEMENT, bwd_ms_max, roof_bwd)
     # The metric is throughput against the HBM roofline, so the roofline of
     # record is the HBM fraction of the dominant call; its FP32 fraction
     # (against the measured FMA rate) stands beside it, since both calls are
@@ -500,7 +501,8 @@ def run_ours(args, world, rank, device):
     if not args.only and not args.no_decode:
         result["decode"] = run_decode(w, x, device, peaks)
     if not args.only and not args.no_conv:
-        result["conv_prologue"] = run_conv(w, x, device, peaks, steps=args.conv_steps)
+        result["conv_prologue"] = run_conv(w, x, device, peaks, steps=args.conv_steps,
+                                           pair=args.step == "pair")
     if not args.only and not args.no_dtproj:
         result["dt_projection"] = run_dtproj(w, x, device, steps=args.conv_steps)
     if not args.only and not args.no_cplx:
@@ -594,11 +596,12 @@ def run_a_leg(w, x, device, peaks, kind, steps=10):
             "steps": steps, "timing": "median of per-call CUDA events"}
 
 
-def run_conv(w, x, device, peaks, steps=10):
+def run_conv(w, x, device, peaks, steps=10, pair=True):
     """The same workload with the block's convolution prologue (width 4):
-    mamba_conv_scan_fwd / _bwd on x in place of u (u = SiLU(conv(x)) is made
-    inside the scan kernels).  Times each call with CUDA events; the bytes are
-    the algorithmic ones of the plain scan plus the filter."""
+    the training pair mamba_conv_scan_fwd_save / _bwd_saved (pair=False: the
+    plain calls) on x in place of u (u = SiLU(conv(x)) is made inside the
+    scan kernels).  Times each call with CUDA events; the bytes are the
+    algorithmic ones of the plain scan plus the filter."""
     from selective_state_space_21_b200 import scan
     from selective_state_space_21_b200.inputs import make_conv_params
 
@@ -608,15 +611,30 @@ def run_conv(w, x, device, peaks, steps=10):
     f32 = dict(device=device, dtype=torch.float32)
     dcw, dcb = torch.empty(w.dim, 4, **f32), torch.empty(w.dim, **f32)
     dA, dD, db = torch.empty(w.dim, w.N, **f32), torch.empty(w.dim, **f32), torch.empty(w.dim, **f32)
+    nsaved = scan.conv_saved_bytes(w.batch, w.dim, w.L, w.N, 4, w.dtype) if pair else 0
+    saved = torch.empty(nsaved, device=device, dtype=torch.uint8) if nsaved else None
 
     def fwd():
-        scan.mamba_conv_scan_fwd(x["u"], cp["conv_w"], cp["conv_b"], x["delta"], x["delta_bias"],
-                                 x["A"], x["B"], x["C"], x["D"], x["z"], y, None)
+        if pair:
+            scan.mamba_conv_scan_fwd_save(x["u"], cp["conv_w"], cp["conv_b"], x["delta"],
+                                          x["delta_bias"], x["A"], x["B"], x["C"], x["D"], x["z"],
+                                          y, None, saved)
+        else:
+            scan.mamba_conv_scan_fwd(x["u"], cp["conv_w"], cp["conv_b"], x["delta"],
+                                     x["delta_bias"], x["A"], x["B"], x["C"], x["D"], x["z"], y,
+                                     None)
 
     def bwd():
-        scan.mamba_conv_scan_bwd(x["u"], cp["conv_w"], cp["conv_b"], x["delta"], x["delta_bias"],
-                                 x["A"], x["B"], x["C"], x["D"], x["z"], x["dy"], g["u"],
-                                 dcw, dcb, g["delta"], dA, g["B"], g["C"], dD, g["z"], db)
+        if pair:
+            scan.mamba_conv_scan_bwd_saved(x["u"], cp["conv_w"], cp["conv_b"], x["delta"],
+                                           x["delta_bias"], x["A"], x["B"], x["C"], x["D"],
+                                           x["z"], x["dy"], g["u"], dcw, dcb, g["delta"], dA,
+                                           g["B"], g["C"], dD, g["z"], db, saved)
+        else:
+            scan.mamba_conv_scan_bwd(x["u"], cp["conv_w"], cp["conv_b"], x["delta"],
+                                     x["delta_bias"], x["A"], x["B"], x["C"], x["D"], x["z"],
+                                     x["dy"], g["u"], dcw, dcb, g["delta"], dA, g["B"], g["C"], dD,
+                                     g["z"], db)
 
     for _ in range(3):
         fwd()
@@ -644,6 +662,8 @@ def run_conv(w, x, device, peaks, steps=10):
                     "frac_hbm": round(bb / (bms * 1e-3) / 1e9 / hbm, 4),
                     "tc_per_s": w.token_channels / (bms * 1e-3)},
             "steps": steps, "width": 4, "timing": "median of per-call CUDA events",
+            "calls": ("mamba_conv_scan_fwd_save + mamba_conv_scan_bwd_saved" if pair
+                      else "mamba_conv_scan_fwd + mamba_conv_scan_bwd"),
             "shape": f"x in place of u, batch {w.batch} x dim {w.dim} x L {w.L}, N {w.N}"}
 
 

@@ -190,9 +190,9 @@ MAMBA_SCAN_API mamba_status_t mamba_scan_bwd_ex(const void *u, const void *delta
  * formulas on the same chunking when chunk_len and carry are automatic, so
  * the gradients agree with mamba_scan_bwd_ex to rounding (bit for bit where
  * the compiler forms both alike; the recomputing backward's own forward pass
- * takes the automatic chunking whatever the options).  Only the plain
- * scan has the pair (not the convolution prologue, the fused projection or
- * complex A).
+ * takes the automatic chunking whatever the options).  The convolution
+ * prologue has the pair too (mamba_conv_scan_fwd_save and friends); the
+ * fused projection and complex A do not.
  */
 MAMBA_SCAN_API mamba_status_t mamba_scan_saved_bytes(int64_t batch, int64_t dim, int64_t L, int64_t N,
                                                      mamba_dtype_t dtype,
@@ -267,6 +267,36 @@ MAMBA_SCAN_API mamba_status_t mamba_conv_scan_bwd(
     void *ddelta, float *dA, void *dB, void *dC, float *dD, void *dz, float *ddelta_bias,
     int64_t batch, int64_t dim, int64_t L, int64_t N, mamba_dtype_t dtype,
     const mamba_scan_options_t *options, mamba_stream_t stream);
+
+/*
+ * The training pair with the convolution prologue: as mamba_scan_saved_bytes,
+ * mamba_scan_fwd_save and mamba_scan_bwd_saved, for mamba_conv_scan_fwd and
+ * mamba_conv_scan_bwd (same arguments; the stored states are those of the
+ * scan driven by u = SiLU(conv(x)), so x, conv_w, conv_b and conv_width must
+ * also be those of the forward).  The size depends on conv_width only
+ * through its range check.
+ */
+MAMBA_SCAN_API mamba_status_t mamba_conv_scan_saved_bytes(int64_t batch, int64_t dim, int64_t L,
+                                                          int64_t N, int64_t conv_width,
+                                                          mamba_dtype_t dtype,
+                                                          const mamba_scan_options_t *options,
+                                                          uint64_t *bytes);
+
+MAMBA_SCAN_API mamba_status_t mamba_conv_scan_fwd_save(
+    const void *x, const float *conv_w, const float *conv_b, int64_t conv_width, const void *delta,
+    const float *delta_bias, const float *A, const void *B, const void *C, const float *D,
+    const void *z, void *y, float *last_state, int64_t batch, int64_t dim, int64_t L, int64_t N,
+    mamba_dtype_t dtype, const mamba_scan_options_t *options, void *saved, uint64_t saved_bytes,
+    mamba_stream_t stream);
+
+MAMBA_SCAN_API mamba_status_t mamba_conv_scan_bwd_saved(
+    const void *x, const float *conv_w, const float *conv_b, int64_t conv_width,
+    const void *delta, const float *delta_bias, const float *A, const void *B, const void *C,
+    const float *D, const void *z, const void *dy, void *dx, float *dconv_w, float *dconv_b,
+    void *ddelta, float *dA, void *dB, void *dC, float *dD, void *dz, float *ddelta_bias,
+    int64_t batch, int64_t dim, int64_t L, int64_t N, mamba_dtype_t dtype,
+    const mamba_scan_options_t *options, const void *saved, uint64_t saved_bytes,
+    mamba_stream_t stream);
 
 /*
  * Forward with the low-rank Delta projection ("Mamba: Linear-Time Sequence

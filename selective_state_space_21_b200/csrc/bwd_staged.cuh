@@ -1224,8 +1224,8 @@ inline int proj_max_rank() {
   return r;
 }
 
-// With `saved` (the plain backward only: not with CONV or PROJ), the
-// checkpoints, range flags and (three-phase) h_in and sums of Delta come from
+// With `saved` (not with PROJ), the checkpoints, range flags and (three-phase)
+// h_in and sums of Delta come from
 // a saving forward of the same inputs and options, laid out as saved_layout
 // gives it, and the checkpoint pass does not run.
 template <typename T, int NM, bool CONV = false, bool PROJ = false>
@@ -1233,8 +1233,8 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
                                mamba_status_t (*launched)(), const unsigned char *saved = nullptr) {
   SavedLayout sl;
   if (saved) {
-    if constexpr (CONV || PROJ) return MAMBA_ERR_UNSUPPORTED;
-    const mamba_status_t ls = saved_layout<T, NM>(a.batch, a.dim, a.L, o, &sl);
+    if constexpr (PROJ) return MAMBA_ERR_UNSUPPORTED;
+    const mamba_status_t ls = saved_layout<T, NM, CONV>(a.batch, a.dim, a.L, o, &sl);
     if (ls != MAMBA_OK) return ls;
   }
   using Lay = BwdLayout<T, NM, !PROJ>;

@@ -1339,13 +1339,13 @@ struct SavedLayout {
   int64_t n_ckpt = 0, n_flags = 0, n_cum = 0, n_hin = 0;
 };
 
-template <typename T, int NM>
+template <typename T, int NM, bool CONV = false>
 inline mamba_status_t saved_layout(int64_t batch, int64_t dim, int64_t L, const StagedOptions &o,
                                    SavedLayout *out) {
   SavedLayout sl;
   int sms = 0, slots = 0;
-  const mamba_status_t st =
-      staged_forward_plan<T, NM>(batch, dim, L, o, StagedLayout<T, NM>::ALLOC, &sl.pl, &sl.G, &sms, &slots);
+  const mamba_status_t st = staged_forward_plan<T, NM, CONV>(batch, dim, L, o, StagedLayout<T, NM>::ALLOC,
+                                                             &sl.pl, &sl.G, &sms, &slots);
   if (st != MAMBA_OK) return st;
   auto up = [](size_t b) { return (b + 255) / 256 * 256; };
   const int64_t n16 = ceil_div(L, kCkptEvery);
@@ -1666,9 +1666,8 @@ struct StagedForward {
 // MAMBA_ERR_UNSUPPORTED (nothing enqueued) if the driver rejects a tensor map,
 // MAMBA_ERR_OUT_OF_MEMORY (nothing enqueued) if the workspace cannot be had.
 // CONV selects the kernels with the convolution prologue (a.conv_w set).
-// With `save` (the plain forward only: not with CONV or PROJ), the forward
-// also stores what the backward would recompute, laid out as saved_layout
-// gives it.
+// With `save` (not with PROJ), the forward also stores what the backward
+// would recompute, laid out as saved_layout gives it.
 template <typename T, int NM, bool CONV = false, bool PROJ = false>
 mamba_status_t staged_forward(const FwdArgs &a, const StagedOptions &o, cudaStream_t s,
                               mamba_status_t (*launched)(), float *ckpt = nullptr,
@@ -1676,8 +1675,8 @@ mamba_status_t staged_forward(const FwdArgs &a, const StagedOptions &o, cudaStre
   StagedForward<T, NM, CONV, PROJ> sf;
   SavedLayout lay;
   if (save) {
-    if constexpr (CONV || PROJ) return MAMBA_ERR_UNSUPPORTED;  // only the plain forward saves
-    const mamba_status_t ls = saved_layout<T, NM>(a.batch, a.dim, a.L, o, &lay);
+    if constexpr (PROJ) return MAMBA_ERR_UNSUPPORTED;  // the fused projection saves nothing
+    const mamba_status_t ls = saved_layout<T, NM, CONV>(a.batch, a.dim, a.L, o, &lay);
     if (ls != MAMBA_OK) return ls;
     sf.save = &lay;
     sf.save_buf = save;

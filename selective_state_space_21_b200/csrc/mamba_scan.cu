@@ -181,26 +181,31 @@ mamba_status_t staged_dispatch(const FwdArgs &a, const StagedOptions &o, cudaStr
 // Bytes a saving forward stores for its backward: 0 where the problem takes
 // the one-thread-per-channel kernels (then the saving calls are the plain
 // ones), else the layout of saved_layout on the current device.
-template <typename T>
+template <typename T, bool CONV>
 mamba_status_t saved_bytes_t(int64_t batch, int64_t dim, int64_t L, int64_t N, const StagedOptions &so,
                              uint64_t *bytes) {
   SavedLayout sl;
   mamba_status_t st;
-  if (N <= 4) st = saved_layout<T, 4>(batch, dim, L, so, &sl);
-  else if (N <= 8) st = saved_layout<T, 8>(batch, dim, L, so, &sl);
-  else st = saved_layout<T, 16>(batch, dim, L, so, &sl);
+  if (N <= 4) st = saved_layout<T, 4, CONV>(batch, dim, L, so, &sl);
+  else if (N <= 8) st = saved_layout<T, 8, CONV>(batch, dim, L, so, &sl);
+  else st = saved_layout<T, 16, CONV>(batch, dim, L, so, &sl);
   *bytes = st == MAMBA_OK ? uint64_t(sl.bytes) : 0;
   return st;
 }
 
+// (conv: the forward with the convolution prologue, whose kernels the chunking
+// is planned for)
 mamba_status_t saved_bytes_for(int64_t batch, int64_t dim, int64_t L, int64_t N, mamba_dtype_t dtype,
-                               const StagedOptions &so, uint64_t *bytes) {
+                               const StagedOptions &so, uint64_t *bytes, bool conv = false) {
   *bytes = 0;
   if (batch == 0 || dim == 0 || L == 0 || so.path == MAMBA_PATH_REFERENCE ||
       !staged_shape_ok(L, dim, N, dtype_size(dtype)))
     return MAMBA_OK;
-  return dtype == MAMBA_BF16 ? saved_bytes_t<__nv_bfloat16>(batch, dim, L, N, so, bytes)
-                             : saved_bytes_t<float>(batch, dim, L, N, so, bytes);
+  if (conv)
+    return dtype == MAMBA_BF16 ? saved_bytes_t<__nv_bfloat16, true>(batch, dim, L, N, so, bytes)
+                               : saved_bytes_t<float, true>(batch, dim, L, N, so, bytes);
+  return dtype == MAMBA_BF16 ? saved_bytes_t<__nv_bfloat16, false>(batch, dim, L, N, so, bytes)
+                             : saved_bytes_t<float, false>(batch, dim, L, N, so, bytes);
 }
 
 template <typename T, int NM>
@@ -927,13 +932,14 @@ mamba_status_t mamba_scan_bwd(const void *u, const void *delta, const float *del
 
 // ------------------------------------------------ convolution prologue
 
-mamba_status_t mamba_conv_scan_fwd(const void *x, const float *conv_w, const float *conv_b,
-                                   int64_t conv_width, const void *delta,
-                                   const float *delta_bias, const float *A, const void *B,
-                                   const void *C, const float *D, const void *z, void *y,
-                                   float *last_state, int64_t batch, int64_t dim, int64_t L,
-                                   int64_t N, mamba_dtype_t dtype,
-                                   const mamba_scan_options_t *options, mamba_stream_t stream) {
+static mamba_status_t conv_fwd_entry(const void *x, const float *conv_w, const float *conv_b,
+                                     int64_t conv_width, const void *delta,
+                                     const float *delta_bias, const float *A, const void *B,
+                                     const void *C, const float *D, const void *z, void *y,
+                                     float *last_state, int64_t batch, int64_t dim, int64_t L,
+                                     int64_t N, mamba_dtype_t dtype,
+                                     const mamba_scan_options_t *options, mamba_stream_t stream,
+                                     bool saving, void *saved, uint64_t saved_bytes) {
   mamba_status_t st = check_shape(batch, dim, L, N, dtype);
   if (st != MAMBA_OK) return st;
   if ((st = check_options(options)) != MAMBA_OK) return st;
@@ -958,6 +964,13 @@ mamba_status_t mamba_conv_scan_fwd(const void *x, const float *conv_w, const flo
   ck.buf(delta_bias, size_t(dim) * 4, 4, false, false);
   ck.buf(y, nbdl * es, es, true, true);
   ck.buf(last_state, size_t(batch) * dim * N * 4, 4, false, true);
+  const StagedOptions so = staged_options(options);
+  uint64_t need = 0;
+  if (saving) {  // what this forward stores for its backward (0: nothing)
+    if ((st = saved_bytes_for(batch, dim, L, N, dtype, so, &need, true)) != MAMBA_OK) return st;
+    if (need > saved_bytes) return MAMBA_ERR_INVALID_ARG;
+    ck.buf(saved, need, 16, true, true);
+  }
   if (ck.st != MAMBA_OK) return ck.st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (batch == 0 || dim == 0) return MAMBA_OK;
@@ -971,18 +984,54 @@ mamba_status_t mamba_conv_scan_fwd(const void *x, const float *conv_w, const flo
   a.bias = delta_bias; a.A = A; a.D = D; a.y = y; a.last_state = last_state;
   a.batch = batch; a.dim = dim; a.L = L; a.N = (int)N;
   a.conv_w = conv_w; a.conv_b = conv_b; a.conv_width = (int)conv_width;
-  return forward_paths<true>(a, es, dtype, staged_options(options), s);
+  return forward_paths<true>(a, es, dtype, so, s, need ? static_cast<unsigned char *>(saved) : nullptr);
 }
 
-mamba_status_t mamba_conv_scan_bwd(const void *x, const float *conv_w, const float *conv_b,
+mamba_status_t mamba_conv_scan_fwd(const void *x, const float *conv_w, const float *conv_b,
                                    int64_t conv_width, const void *delta,
                                    const float *delta_bias, const float *A, const void *B,
-                                   const void *C, const float *D, const void *z, const void *dy,
-                                   void *dx, float *dconv_w, float *dconv_b, void *ddelta,
-                                   float *dA, void *dB, void *dC, float *dD, void *dz,
-                                   float *ddelta_bias, int64_t batch, int64_t dim, int64_t L,
+                                   const void *C, const float *D, const void *z, void *y,
+                                   float *last_state, int64_t batch, int64_t dim, int64_t L,
                                    int64_t N, mamba_dtype_t dtype,
                                    const mamba_scan_options_t *options, mamba_stream_t stream) {
+  return conv_fwd_entry(x, conv_w, conv_b, conv_width, delta, delta_bias, A, B, C, D, z, y, last_state,
+                        batch, dim, L, N, dtype, options, stream, false, nullptr, 0);
+}
+
+mamba_status_t mamba_conv_scan_saved_bytes(int64_t batch, int64_t dim, int64_t L, int64_t N,
+                                           int64_t conv_width, mamba_dtype_t dtype,
+                                           const mamba_scan_options_t *options, uint64_t *bytes) {
+  if (!bytes) return MAMBA_ERR_INVALID_ARG;
+  *bytes = 0;
+  mamba_status_t st = check_shape(batch, dim, L, N, dtype);
+  if (st != MAMBA_OK) return st;
+  if ((st = check_options(options)) != MAMBA_OK) return st;
+  if (conv_width < 1 || conv_width > kMaxConvWidth) return MAMBA_ERR_UNSUPPORTED;
+  return saved_bytes_for(batch, dim, L, N, dtype, staged_options(options), bytes, true);
+}
+
+mamba_status_t mamba_conv_scan_fwd_save(const void *x, const float *conv_w, const float *conv_b,
+                                        int64_t conv_width, const void *delta,
+                                        const float *delta_bias, const float *A, const void *B,
+                                        const void *C, const float *D, const void *z, void *y,
+                                        float *last_state, int64_t batch, int64_t dim, int64_t L,
+                                        int64_t N, mamba_dtype_t dtype,
+                                        const mamba_scan_options_t *options, void *saved,
+                                        uint64_t saved_bytes, mamba_stream_t stream) {
+  return conv_fwd_entry(x, conv_w, conv_b, conv_width, delta, delta_bias, A, B, C, D, z, y, last_state,
+                        batch, dim, L, N, dtype, options, stream, true, saved, saved_bytes);
+}
+
+static mamba_status_t conv_bwd_entry(const void *x, const float *conv_w, const float *conv_b,
+                                     int64_t conv_width, const void *delta,
+                                     const float *delta_bias, const float *A, const void *B,
+                                     const void *C, const float *D, const void *z, const void *dy,
+                                     void *dx, float *dconv_w, float *dconv_b, void *ddelta,
+                                     float *dA, void *dB, void *dC, float *dD, void *dz,
+                                     float *ddelta_bias, int64_t batch, int64_t dim, int64_t L,
+                                     int64_t N, mamba_dtype_t dtype,
+                                     const mamba_scan_options_t *options, mamba_stream_t stream,
+                                     bool saving, const void *saved, uint64_t saved_bytes) {
   mamba_status_t st = check_shape(batch, dim, L, N, dtype);
   if (st != MAMBA_OK) return st;
   if ((st = check_options(options)) != MAMBA_OK) return st;
@@ -1019,6 +1068,13 @@ mamba_status_t mamba_conv_scan_bwd(const void *x, const float *conv_w, const flo
   ck.buf(dA, size_t(dim) * N * 4, 4, true, true);
   ck.buf(dD, size_t(dim) * 4, 4, false, true);
   ck.buf(ddelta_bias, size_t(dim) * 4, 4, false, true);
+  const StagedOptions so = staged_options(options);
+  uint64_t need = 0;
+  if (saving) {  // what the saving forward stored (0: nothing; recompute)
+    if ((st = saved_bytes_for(batch, dim, L, N, dtype, so, &need, true)) != MAMBA_OK) return st;
+    if (need > saved_bytes) return MAMBA_ERR_INVALID_ARG;
+    ck.buf(saved, need, 16, true, false);
+  }
   if (ck.st != MAMBA_OK) return ck.st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (dim == 0) return MAMBA_OK;
@@ -1050,7 +1106,9 @@ mamba_status_t mamba_conv_scan_bwd(const void *x, const float *conv_w, const flo
     cudaGetLastError();
     return MAMBA_ERR_OUT_OF_MEMORY;
   }
-  if ((st = backward_paths<true>(a, es, dtype, staged_options(options), s)) != MAMBA_OK) {
+  if ((st = backward_paths<true>(a, es, dtype, so, s,
+                                need ? static_cast<const unsigned char *>(saved) : nullptr)) !=
+      MAMBA_OK) {
     ws_free(part, s);
     return st;
   }
@@ -1077,6 +1135,35 @@ mamba_status_t mamba_conv_scan_bwd(const void *x, const float *conv_w, const flo
   }
   if (ws_free(part, s) != cudaSuccess && st == MAMBA_OK) st = MAMBA_ERR_CUDA;
   return st;
+}
+
+mamba_status_t mamba_conv_scan_bwd(const void *x, const float *conv_w, const float *conv_b,
+                                   int64_t conv_width, const void *delta,
+                                   const float *delta_bias, const float *A, const void *B,
+                                   const void *C, const float *D, const void *z, const void *dy,
+                                   void *dx, float *dconv_w, float *dconv_b, void *ddelta,
+                                   float *dA, void *dB, void *dC, float *dD, void *dz,
+                                   float *ddelta_bias, int64_t batch, int64_t dim, int64_t L,
+                                   int64_t N, mamba_dtype_t dtype,
+                                   const mamba_scan_options_t *options, mamba_stream_t stream) {
+  return conv_bwd_entry(x, conv_w, conv_b, conv_width, delta, delta_bias, A, B, C, D, z, dy, dx, dconv_w,
+                        dconv_b, ddelta, dA, dB, dC, dD, dz, ddelta_bias, batch, dim, L, N, dtype, options,
+                        stream, false, nullptr, 0);
+}
+
+mamba_status_t mamba_conv_scan_bwd_saved(const void *x, const float *conv_w, const float *conv_b,
+                                         int64_t conv_width, const void *delta,
+                                         const float *delta_bias, const float *A, const void *B,
+                                         const void *C, const float *D, const void *z, const void *dy,
+                                         void *dx, float *dconv_w, float *dconv_b, void *ddelta,
+                                         float *dA, void *dB, void *dC, float *dD, void *dz,
+                                         float *ddelta_bias, int64_t batch, int64_t dim, int64_t L,
+                                         int64_t N, mamba_dtype_t dtype,
+                                         const mamba_scan_options_t *options, const void *saved,
+                                         uint64_t saved_bytes, mamba_stream_t stream) {
+  return conv_bwd_entry(x, conv_w, conv_b, conv_width, delta, delta_bias, A, B, C, D, z, dy, dx, dconv_w,
+                        dconv_b, ddelta, dA, dB, dC, dD, dz, ddelta_bias, batch, dim, L, N, dtype, options,
+                        stream, true, saved, saved_bytes);
 }
 
 // ------------------------------------------- low-rank Delta projection

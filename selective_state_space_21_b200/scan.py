@@ -80,6 +80,14 @@ def load_library():
             lib.mamba_scan_fwd_save.restype = ctypes.c_int
             lib.mamba_scan_bwd_saved.argtypes = [vp] * 17 + [i64] * 4 + [i32, opt, vp, u64, vp]
             lib.mamba_scan_bwd_saved.restype = ctypes.c_int
+            lib.mamba_conv_scan_saved_bytes.argtypes = [i64] * 5 + [i32, opt, ctypes.POINTER(u64)]
+            lib.mamba_conv_scan_saved_bytes.restype = ctypes.c_int
+            lib.mamba_conv_scan_fwd_save.argtypes = (
+                [vp] * 3 + [i64] + [vp] * 9 + [i64] * 4 + [i32, opt, vp, u64, vp])
+            lib.mamba_conv_scan_fwd_save.restype = ctypes.c_int
+            lib.mamba_conv_scan_bwd_saved.argtypes = (
+                [vp] * 3 + [i64] + [vp] * 18 + [i64] * 4 + [i32, opt, vp, u64, vp])
+            lib.mamba_conv_scan_bwd_saved.restype = ctypes.c_int
             lib.mamba_scan_step.argtypes = [vp] * 10 + [i64] * 3 + [i32, vp]
             lib.mamba_scan_step.restype = ctypes.c_int
             lib.mamba_conv_scan_step.argtypes = [vp] * 5 + [i64] + [vp] * 8 + [i64] * 3 + [i32, vp]
@@ -313,13 +321,7 @@ def _opts_ptr(path, chunk_len, carry, wait_timeout_us, test_hook):
     return ctypes.byref(_options(path, chunk_len, carry, wait_timeout_us, test_hook))
 
 
-def mamba_conv_scan_fwd(x, conv_w, conv_b, delta, delta_bias, A, B, C, D, z, y, last_state, *,
-                        path="auto", chunk_len=0, carry="auto", wait_timeout_us=0, test_hook=0,
-                        stream=None):
-    """Enqueue the forward with the convolution prologue (u = SiLU(causal
-    depthwise conv of x) computed inside the scan kernels).  x (batch, dim, L)
-    in the I/O dtype; conv_w (dim, W) float32 with W in 1..4; conv_b (dim,)
-    float32 or None; the rest as ``mamba_scan_fwd``."""
+def _conv_fwd_args(x, conv_w, conv_b, delta, delta_bias, A, B, C, D, z, y, last_state):
     batch, dim, L = x.shape
     N = A.shape[1]
     W = conv_w.shape[1]
@@ -333,16 +335,51 @@ def mamba_conv_scan_fwd(x, conv_w, conv_b, delta, delta_bias, A, B, C, D, z, y, 
         _ptr(A, f32, (dim, N), "A"), _ptr(B, dt, bnl, "B"), _ptr(C, dt, bnl, "C"),
         _ptr(D, f32, (dim,), "D"), _ptr(z, dt, bdl, "z"), _ptr(y, dt, bdl, "y"),
         _ptr(last_state, f32, (batch, dim, N), "last_state"), batch, dim, L, N, _dtype_code(dt)]
+    return args
+
+
+def mamba_conv_scan_fwd(x, conv_w, conv_b, delta, delta_bias, A, B, C, D, z, y, last_state, *,
+                        path="auto", chunk_len=0, carry="auto", wait_timeout_us=0, test_hook=0,
+                        stream=None):
+    """Enqueue the forward with the convolution prologue (u = SiLU(causal
+    depthwise conv of x) computed inside the scan kernels).  x (batch, dim, L)
+    in the I/O dtype; conv_w (dim, W) float32 with W in 1..4; conv_b (dim,)
+    float32 or None; the rest as ``mamba_scan_fwd``."""
+    args = _conv_fwd_args(x, conv_w, conv_b, delta, delta_bias, A, B, C, D, z, y, last_state)
     opts = _opts_ptr(path, chunk_len, carry, wait_timeout_us, test_hook)
     _check(load_library().mamba_conv_scan_fwd(*args, opts, _stream_handle(stream)),
            "mamba_conv_scan_fwd")
 
 
-def mamba_conv_scan_bwd(x, conv_w, conv_b, delta, delta_bias, A, B, C, D, z, dy, dx, dconv_w,
-                        dconv_b, ddelta, dA, dB, dC, dD, dz, ddelta_bias, *, path="auto",
-                        chunk_len=0, carry="auto", wait_timeout_us=0, test_hook=0, stream=None):
-    """Enqueue the backward of sum(dy * y) for ``mamba_conv_scan_fwd``: dx
-    and dconv_w (and dconv_b if given) take the place of du."""
+def conv_saved_bytes(batch, dim, L, N, conv_width, dtype, *, path="auto", chunk_len=0,
+                     carry="auto", wait_timeout_us=0, test_hook=0) -> int:
+    """``saved_bytes`` for the training pair with the convolution prologue."""
+    n = ctypes.c_uint64(0)
+    opts = _opts_ptr(path, chunk_len, carry, wait_timeout_us, test_hook)
+    _check(load_library().mamba_conv_scan_saved_bytes(batch, dim, L, N, conv_width,
+                                                      _dtype_code(dtype), opts, ctypes.byref(n)),
+           "mamba_conv_scan_saved_bytes")
+    return int(n.value)
+
+
+def mamba_conv_scan_fwd_save(x, conv_w, conv_b, delta, delta_bias, A, B, C, D, z, y, last_state,
+                             saved, *, path="auto", chunk_len=0, carry="auto", wait_timeout_us=0,
+                             test_hook=0, stream=None):
+    """``mamba_conv_scan_fwd`` that also fills ``saved`` (``conv_saved_bytes``
+    bytes) for ``mamba_conv_scan_bwd_saved``."""
+    batch, dim, L = x.shape
+    need = conv_saved_bytes(batch, dim, L, A.shape[1], conv_w.shape[1], x.dtype, path=path,
+                            chunk_len=chunk_len, carry=carry, wait_timeout_us=wait_timeout_us,
+                            test_hook=test_hook)
+    sp, sn = _saved_arg(saved, need)
+    args = _conv_fwd_args(x, conv_w, conv_b, delta, delta_bias, A, B, C, D, z, y, last_state)
+    opts = _opts_ptr(path, chunk_len, carry, wait_timeout_us, test_hook)
+    _check(load_library().mamba_conv_scan_fwd_save(*args, opts, sp, sn, _stream_handle(stream)),
+           "mamba_conv_scan_fwd_save")
+
+
+def _conv_bwd_args(x, conv_w, conv_b, delta, delta_bias, A, B, C, D, z, dy, dx, dconv_w, dconv_b,
+                   ddelta, dA, dB, dC, dD, dz, ddelta_bias):
     batch, dim, L = x.shape
     N = A.shape[1]
     W = conv_w.shape[1]
@@ -360,9 +397,37 @@ def mamba_conv_scan_bwd(x, conv_w, conv_b, delta, delta_bias, A, B, C, D, z, dy,
         _ptr(dA, f32, (dim, N), "dA"), _ptr(dB, dt, bnl, "dB"), _ptr(dC, dt, bnl, "dC"),
         _ptr(dD, f32, (dim,), "dD"), _ptr(dz, dt, bdl, "dz"),
         _ptr(ddelta_bias, f32, (dim,), "ddelta_bias"), batch, dim, L, N, _dtype_code(dt)]
+    return args
+
+
+def mamba_conv_scan_bwd(x, conv_w, conv_b, delta, delta_bias, A, B, C, D, z, dy, dx, dconv_w,
+                        dconv_b, ddelta, dA, dB, dC, dD, dz, ddelta_bias, *, path="auto",
+                        chunk_len=0, carry="auto", wait_timeout_us=0, test_hook=0, stream=None):
+    """Enqueue the backward of sum(dy * y) for ``mamba_conv_scan_fwd``: dx
+    and dconv_w (and dconv_b if given) take the place of du."""
+    args = _conv_bwd_args(x, conv_w, conv_b, delta, delta_bias, A, B, C, D, z, dy, dx, dconv_w,
+                          dconv_b, ddelta, dA, dB, dC, dD, dz, ddelta_bias)
     opts = _opts_ptr(path, chunk_len, carry, wait_timeout_us, test_hook)
     _check(load_library().mamba_conv_scan_bwd(*args, opts, _stream_handle(stream)),
            "mamba_conv_scan_bwd")
+
+
+def mamba_conv_scan_bwd_saved(x, conv_w, conv_b, delta, delta_bias, A, B, C, D, z, dy, dx,
+                              dconv_w, dconv_b, ddelta, dA, dB, dC, dD, dz, ddelta_bias, saved, *,
+                              path="auto", chunk_len=0, carry="auto", wait_timeout_us=0,
+                              test_hook=0, stream=None):
+    """``mamba_conv_scan_bwd`` reading ``saved`` as ``mamba_conv_scan_fwd_save``
+    wrote it (same inputs and options)."""
+    batch, dim, L = x.shape
+    need = conv_saved_bytes(batch, dim, L, A.shape[1], conv_w.shape[1], x.dtype, path=path,
+                            chunk_len=chunk_len, carry=carry, wait_timeout_us=wait_timeout_us,
+                            test_hook=test_hook)
+    sp, sn = _saved_arg(saved, need)
+    args = _conv_bwd_args(x, conv_w, conv_b, delta, delta_bias, A, B, C, D, z, dy, dx, dconv_w,
+                          dconv_b, ddelta, dA, dB, dC, dD, dz, ddelta_bias)
+    opts = _opts_ptr(path, chunk_len, carry, wait_timeout_us, test_hook)
+    _check(load_library().mamba_conv_scan_bwd_saved(*args, opts, sp, sn, _stream_handle(stream)),
+           "mamba_conv_scan_bwd_saved")
 
 
 def mamba_dtproj_scan_fwd(u, dt_low, W_dt, delta_bias, A, B, C, D, z, y, last_state, *,
@@ -698,6 +763,48 @@ def conv_selective_scan_fwd(x, conv_w, conv_b, delta, A, B, C, D=None, z=None, d
     mamba_conv_scan_fwd(x, conv_w, conv_b, delta, delta_bias, A, B, C, D, z, y, last, path=path,
                         chunk_len=chunk_len, carry=carry, stream=stream)
     return (y, last) if return_last_state else y
+
+
+def conv_selective_scan_fwd_save(x, conv_w, conv_b, delta, A, B, C, D=None, z=None,
+                                 delta_bias=None, return_last_state=False, path="auto",
+                                 chunk_len=0, carry="auto", stream=None):
+    """The training pair's forward with the convolution prologue; returns
+    (y, saved) or (y, last_state, saved) as ``selective_scan_fwd_save``."""
+    batch, dim, L = x.shape
+    N = A.shape[1]
+    y = torch.empty_like(x)
+    last = (torch.empty(batch, dim, N, device=x.device, dtype=torch.float32)
+            if return_last_state else None)
+    need = conv_saved_bytes(batch, dim, L, N, conv_w.shape[1], x.dtype, path=path,
+                            chunk_len=chunk_len, carry=carry)
+    saved = torch.empty(need, device=x.device, dtype=torch.uint8) if need else None
+    mamba_conv_scan_fwd_save(x, conv_w, conv_b, delta, delta_bias, A, B, C, D, z, y, last, saved,
+                             path=path, chunk_len=chunk_len, carry=carry, stream=stream)
+    return (y, last, saved) if return_last_state else (y, saved)
+
+
+def conv_selective_scan_bwd_saved(x, conv_w, conv_b, delta, A, B, C, dy, saved, D=None, z=None,
+                                  delta_bias=None, path="auto", chunk_len=0, carry="auto",
+                                  stream=None) -> dict:
+    """The training pair's backward with the convolution prologue; returns
+    the gradients as ``conv_selective_scan_bwd``."""
+    dim, N = A.shape
+    f32 = torch.float32
+    g = {
+        "dx": torch.empty_like(x), "dconv_w": torch.empty_like(conv_w),
+        "dconv_b": torch.empty(dim, device=x.device, dtype=f32) if conv_b is not None else None,
+        "ddelta": torch.empty_like(x),
+        "dA": torch.empty(dim, N, device=x.device, dtype=f32),
+        "dB": torch.empty_like(B), "dC": torch.empty_like(C),
+        "dD": torch.empty(dim, device=x.device, dtype=f32) if D is not None else None,
+        "dz": torch.empty_like(x) if z is not None else None,
+        "ddelta_bias": torch.empty(dim, device=x.device, dtype=f32),
+    }
+    mamba_conv_scan_bwd_saved(x, conv_w, conv_b, delta, delta_bias, A, B, C, D, z, dy, g["dx"],
+                              g["dconv_w"], g["dconv_b"], g["ddelta"], g["dA"], g["dB"], g["dC"],
+                              g["dD"], g["dz"], g["ddelta_bias"], saved, path=path,
+                              chunk_len=chunk_len, carry=carry, stream=stream)
+    return {k: v for k, v in g.items() if v is not None}
 
 
 def conv_selective_scan_bwd(x, conv_w, conv_b, delta, A, B, C, dy, D=None, z=None,

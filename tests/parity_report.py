@@ -1,6 +1,7 @@
 """Parity report: the measured error of the CUDA path against the fp64 oracle
 on every workload, per output tensor, at full size in the launch
-configuration the benchmark times (auto path), and of the convolution
+configuration the benchmark times (auto path; the training pair where the
+workload has a backward), and of the convolution
 prologue, the Delta projection and complex A on the bf16 2K workload.
 
     python tests/parity_report.py            # needs a B200; prints a markdown table
@@ -39,8 +40,16 @@ def errors(got, ref):
 def report(index: int, k: int, backward: bool):
     w = WORKLOADS[index]
     x = workload_inputs(index, device="cuda", with_dy=backward)
-    y, last = gc.gpu_fwd(x)
-    g = gc.gpu_bwd(x) if backward else None
+    if backward:  # the training pair, as the benchmark times it
+        y, last, saved = scan.selective_scan_fwd_save(
+            x["u"], x["delta"], x["A"], x["B"], x["C"], D=x["D"], z=x["z"],
+            delta_bias=x["delta_bias"], return_last_state=True)
+        g = scan.selective_scan_bwd_saved(x["u"], x["delta"], x["A"], x["B"], x["C"], x["dy"],
+                                          saved, D=x["D"], z=x["z"], delta_bias=x["delta_bias"])
+        assert scan.mamba_scan_stream_status() == 0
+    else:
+        y, last = gc.gpu_fwd(x)
+        g = None
     xh = gc.to_host(x)
     yh, lh = y.cpu(), last.cpu()
     gh = {key: v.cpu() for key, v in g.items()} if g else {}

@@ -10,7 +10,7 @@ import torch
 
 import gpu_cases as gc
 from selective_state_space_21_b200 import build, scan
-from selective_state_space_21_b200.inputs import make_inputs
+from selective_state_space_21_b200.inputs import make_inputs, workload_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -151,3 +151,67 @@ def test_pair_refuses_a_short_buffer():
         None, 1, 128, 512, 16, scan._dtype_code(torch.bfloat16), None, short.data_ptr(),
         ctypes.c_uint64(short.numel()), None)
     assert rc == 1  # MAMBA_ERR_INVALID_ARG
+
+
+def test_pair_full_bench_workload():
+    """bf16 8 x 5120 x 2048 (the benchmark's step, in its launch configuration):
+    the pair's y and gradients equal the plain calls' bit for bit, which the
+    full-size sampled oracle tests check against the fp64 oracle."""
+    x = workload_inputs(2, device="cuda", with_dy=True)
+    y, last, saved, g = _pair(x)
+    y0, last0, g0 = _plain(x)
+    assert torch.equal(y, y0) and torch.equal(last, last0)
+    for k in g0:
+        assert torch.equal(g[k], g0[k]), k
+
+
+# ------------------------------------------------ with the convolution prologue
+
+CONV_GRADS = ("dx", "dconv_w", "dconv_b", "ddelta", "dA", "dB", "dC", "dD", "dz", "ddelta_bias")
+
+
+def _conv_case(b, d, L, N, dtype, W=4, seed=0):
+    from selective_state_space_21_b200.inputs import make_conv_params
+    x = make_inputs(b, d, L, N, dtype, seed=seed, with_dy=True)
+    x.update(make_conv_params(d, W, seed=seed, has_bias=True))
+    return x
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("shape", [(2, 256, 2048, 16), (8, 5120, 512, 16)],
+                         ids=["three_phase", "sequential"])
+def test_conv_pair(shape, dtype):
+    """mamba_conv_scan_fwd_save / _bwd_saved against the plain conv calls (bit
+    for bit in bf16) and, at the small shape, the fp64 conv oracle."""
+    import oracle
+    b, d, L, N = shape
+    xh = _conv_case(b, d, L, N, dtype, seed=800 + b)
+    x = gc.to_device(xh)
+    kw = dict(D=x["D"], z=x["z"], delta_bias=x["delta_bias"])
+    y, last, saved = scan.conv_selective_scan_fwd_save(x["u"], x["conv_w"], x["conv_b"],
+                                                       x["delta"], x["A"], x["B"], x["C"],
+                                                       return_last_state=True, **kw)
+    g = scan.conv_selective_scan_bwd_saved(x["u"], x["conv_w"], x["conv_b"], x["delta"], x["A"],
+                                           x["B"], x["C"], x["dy"], saved, **kw)
+    y0, last0 = scan.conv_selective_scan_fwd(x["u"], x["conv_w"], x["conv_b"], x["delta"],
+                                             x["A"], x["B"], x["C"], return_last_state=True, **kw)
+    g0 = scan.conv_selective_scan_bwd(x["u"], x["conv_w"], x["conv_b"], x["delta"], x["A"],
+                                      x["B"], x["C"], x["dy"], **kw)
+    assert scan.mamba_scan_stream_status() == 0
+    assert saved is not None
+    exact = dtype == torch.bfloat16
+    tol = gc.TOL[dtype]
+    if exact:
+        assert torch.equal(y, y0) and torch.equal(last, last0)
+    else:
+        assert _close(y, y0, tol) and _close(last, last0, 1e-5)
+    for k in CONV_GRADS:
+        if k in g0:
+            assert torch.equal(g[k], g0[k]) if exact else _close(g[k], g0[k], 1e-5), k
+    if b == 2:
+        ref = oracle.s6_conv_backward(xh["u"], xh["conv_w"], xh["conv_b"], xh["delta"], xh["A"],
+                                      xh["B"], xh["C"], xh["dy"], xh["delta_bias"], xh["D"],
+                                      xh["z"])
+        errs = {k: gc.normwise(g[k].cpu().double().numpy(), ref[k]) for k in CONV_GRADS
+                if k in g and k in ref}
+        assert all(e <= tol for e in errs.values()), errs
