@@ -89,7 +89,8 @@ def report(index: int, k: int, backward: bool):
 
 def report_variant(kind: str, k: int = 16):
     """The rows beyond the plain scan on the bf16 8 x 5120 x 2048 workload:
-    the convolution prologue (width 4), the rank-160 Delta projection and
+    the convolution prologue (width 4, through its training pair), the
+    rank-160 Delta projection and
     complex A with 16 complex states.  y and the per-channel gradients on
     sampled channels; the per-channel parameters' gradients (summed over the
     batch) on three channels."""
@@ -120,8 +121,18 @@ def report_variant(kind: str, k: int = 16):
         rows, per_d, grads, params = ("u", "delta", "z", "dy"), ("A", "D", "delta_bias"), \
             ("du", "ddelta", "dz"), ("dA", "dD", "ddelta_bias")
     x = gc.to_device(xh)
-    y = fwd(x)[0].cpu()
-    g = {key: v.cpu() for key, v in bwd(x).items() if v is not None}
+    if kind == "conv":  # the training pair, as the benchmark times it
+        kw = dict(D=x["D"], z=x["z"], delta_bias=x["delta_bias"])
+        yd, saved = scan.conv_selective_scan_fwd_save(x["u"], x["conv_w"], x["conv_b"], x["delta"],
+                                                      x["A"], x["B"], x["C"], **kw)
+        gd = scan.conv_selective_scan_bwd_saved(x["u"], x["conv_w"], x["conv_b"], x["delta"],
+                                                x["A"], x["B"], x["C"], x["dy"], saved, **kw)
+        assert scan.mamba_scan_stream_status() == 0
+        y = yd.cpu()
+        g = {key: v.cpu() for key, v in gd.items() if v is not None}
+    else:
+        y = fwd(x)[0].cpu()
+        g = {key: v.cpu() for key, v in bwd(x).items() if v is not None}
     acc: dict = {}
 
     def add(name, got, ref):

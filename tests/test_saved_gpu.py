@@ -57,8 +57,9 @@ def _check_pair(x_host, y_exact=True, g_exact=True, oracle=True, **opts):
         if k in g0:
             if g_exact:
                 assert torch.equal(g[k], g0[k]), f"{k} differs from the recomputing backward"
-            else:
-                assert _close(g[k], g0[k], 1e-5), f"{k} differs from the recomputing backward"
+            else:  # fp32: rounding of the states; bf16: that can flip an output's last bit
+                gt = 1e-5 if x_host["u"].dtype == torch.float32 else gc.TOL[x_host["u"].dtype]
+                assert _close(g[k], g0[k], gt), f"{k} differs from the recomputing backward"
     if oracle:
         ref = gc.oracle_bwd(x_host)
         tol = gc.TOL[x_host["u"].dtype]
@@ -215,3 +216,15 @@ def test_conv_pair(shape, dtype):
         errs = {k: gc.normwise(g[k].cpu().double().numpy(), ref[k]) for k in CONV_GRADS
                 if k in g and k in ref}
         assert all(e <= tol for e in errs.values()), errs
+
+
+@pytest.mark.parametrize("carry,chunk_len", [("sequential", 256), ("three_phase", 192),
+                                             ("three_phase", 0)])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_pair_explicit_chunking(carry, chunk_len, dtype):
+    """Explicit chunking options reach the saving forward and the backward
+    alike (the saved layout follows them): the gradients match the fp64
+    oracle and, within rounding, the recomputing backward (whose own forward
+    pass takes the automatic chunking)."""
+    xh = make_inputs(2, 160, 1100, 16, dtype, seed=900 + chunk_len, with_dy=True)
+    _check_pair(xh, y_exact=False, g_exact=False, carry=carry, chunk_len=chunk_len)
