@@ -198,10 +198,36 @@ def _calls():
         f["u"], pp["dt_low"], pp["W_dt"], f["delta_bias"], f["A"], f["B"], f["C"], f["D"], f["z"],
         f["dy"], o["du"], o["ddl"], o["dW"], o["dA"], o["dB"], o["dC"], o["dD"], o["dz"], o["db"]),
         dtp_outs))
+
+    # the training pairs: the backward reads a buffer its forward filled
+    saved = torch.empty(scan.saved_bytes(2, 200, 512, 16, torch.bfloat16), device="cuda",
+                        dtype=torch.uint8)
+    csaved = torch.empty(scan.conv_saved_bytes(2, 200, 512, 16, 4, torch.bfloat16),
+                         device="cuda", dtype=torch.uint8)
+    scan.mamba_scan_fwd_save(f["u"], f["delta"], f["delta_bias"], f["A"], f["B"], f["C"], f["D"],
+                             f["z"], torch.empty_like(f["u"]), None, saved)
+    scan.mamba_conv_scan_fwd_save(f["u"], cp["conv_w"], cp["conv_b"], f["delta"], f["delta_bias"],
+                                  f["A"], f["B"], f["C"], f["D"], f["z"], torch.empty_like(f["u"]),
+                                  None, csaved)
+    torch.cuda.synchronize()
+    out.append(("fwd save", lambda o: scan.mamba_scan_fwd_save(
+        f["u"], f["delta"], f["delta_bias"], f["A"], f["B"], f["C"], f["D"], f["z"], o["y"],
+        o["last"], torch.empty_like(saved)), lambda: fwd_outs(f)))
+    out.append(("bwd saved", lambda o: scan.mamba_scan_bwd_saved(
+        f["u"], f["delta"], f["delta_bias"], f["A"], f["B"], f["C"], f["D"], f["z"], f["dy"],
+        o["du"], o["dd"], o["dA"], o["dB"], o["dC"], o["dD"], o["dz"], o["db"], saved),
+        lambda: bwd_outs(f)))
+    out.append(("conv fwd save", lambda o: scan.mamba_conv_scan_fwd_save(
+        f["u"], cp["conv_w"], cp["conv_b"], f["delta"], f["delta_bias"], f["A"], f["B"], f["C"],
+        f["D"], f["z"], o["y"], o["last"], torch.empty_like(csaved)), lambda: fwd_outs(f)))
+    out.append(("conv bwd saved", lambda o: scan.mamba_conv_scan_bwd_saved(
+        f["u"], cp["conv_w"], cp["conv_b"], f["delta"], f["delta_bias"], f["A"], f["B"], f["C"],
+        f["D"], f["z"], f["dy"], o["du"], o["dcw"], o["dcb"], o["dd"], o["dA"], o["dB"], o["dC"],
+        o["dD"], o["dz"], o["db"], csaved), conv_outs))
     return out
 
 
-@pytest.mark.parametrize("index", range(10))
+@pytest.mark.parametrize("index", range(14))
 def test_allocation_failure_returns_oom_and_launches_nothing(index):
     calls = _calls()
     name, fn, make_out = calls[index]
