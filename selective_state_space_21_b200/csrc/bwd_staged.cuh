@@ -1148,23 +1148,57 @@ __global__ void __launch_bounds__(kSThreads) bwd_adjoint_agg_kernel(const BwdSta
     p.agg_S[(int64_t(g) * p.K + k) * kSThreads + threadIdx.x] = valid ? S : 0.0;
 }
 
-// dB / dC: sum of the per-CTA partials over the channel groups of a batch row.
+// Four consecutive outputs in one store (8 bytes of bf16, 16 of fp32).
+template <typename T> struct Vec4Out;
+template <> struct Vec4Out<float> {
+  __device__ static void store(float *dst, const float (&v)[4]) {
+    *reinterpret_cast<float4 *>(dst) = make_float4(v[0], v[1], v[2], v[3]);
+  }
+};
+template <> struct Vec4Out<__nv_bfloat16> {
+  __device__ static void store(__nv_bfloat16 *dst, const float (&v)[4]) {
+    const __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]), c = __floats2bfloat162_rn(v[2], v[3]);
+    uint2 w;
+    w.x = *reinterpret_cast<const uint32_t *>(&a);
+    w.y = *reinterpret_cast<const uint32_t *>(&c);
+    *reinterpret_cast<uint2 *>(dst) = w;
+  }
+};
+
+// dB / dC: sum of the per-CTA partials over the channel groups of a batch row,
+// four consecutive steps per thread (16-byte loads; L is a multiple of 4 on
+// this path), each element summed over the groups in order.
 template <typename T>
 __global__ void bwd_staged_finalize_bc(const BwdStagedArgs p) {
   const BwdArgs &f = p.w;
-  const int64_t total = f.batch * f.N * f.L;
+  const int64_t L4 = f.L / 4;
+  const int64_t total = f.batch * f.N * L4;
+  const bool vec_out = ((reinterpret_cast<uintptr_t>(f.dB) | reinterpret_cast<uintptr_t>(f.dC)) %
+                        (4 * sizeof(T))) == 0;
   for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
        i += int64_t(gridDim.x) * blockDim.x) {
-    const int64_t t = i % f.L, n = (i / f.L) % f.N, b = i / (f.L * f.N);
-    float sb = 0.f, sc = 0.f;
+    const int64_t t = (i % L4) * 4, n = (i / L4) % f.N, b = i / (L4 * f.N);
+    float4 sb = make_float4(0.f, 0.f, 0.f, 0.f), sc = sb;
 #pragma unroll 8
     for (int j = 0; j < p.gpb; ++j) {
-      const float *pp = p.part_bc + ((int64_t(j) * f.batch + b) * 32) * f.L + t;
-      sb += pp[n * f.L];
-      sc += pp[(kMaxN + n) * f.L];
+      const int64_t o = ((int64_t(j) * f.batch + b) * 32) * f.L + t;
+      if (!in_bounds(o + (kMaxN + n) * f.L + 3, p.n_bc)) break;
+      const float4 xb = __ldcs(reinterpret_cast<const float4 *>(p.part_bc + o + n * f.L));
+      const float4 xc = __ldcs(reinterpret_cast<const float4 *>(p.part_bc + o + (kMaxN + n) * f.L));
+      sb.x += xb.x; sb.y += xb.y; sb.z += xb.z; sb.w += xb.w;
+      sc.x += xc.x; sc.y += xc.y; sc.z += xc.z; sc.w += xc.w;
     }
-    static_cast<T *>(f.dB)[i] = from_f<T>(sb);
-    static_cast<T *>(f.dC)[i] = from_f<T>(sc);
+    const int64_t e = (b * f.N + n) * f.L + t;  // first of the four outputs
+    T *dB = static_cast<T *>(f.dB) + e;
+    T *dC = static_cast<T *>(f.dC) + e;
+    if (vec_out) {
+      const float vb[4] = {sb.x, sb.y, sb.z, sb.w}, vc[4] = {sc.x, sc.y, sc.z, sc.w};
+      Vec4Out<T>::store(dB, vb);
+      Vec4Out<T>::store(dC, vc);
+    } else {
+      dB[0] = from_f<T>(sb.x); dB[1] = from_f<T>(sb.y); dB[2] = from_f<T>(sb.z); dB[3] = from_f<T>(sb.w);
+      dC[0] = from_f<T>(sc.x); dC[1] = from_f<T>(sc.y); dC[2] = from_f<T>(sc.z); dC[3] = from_f<T>(sc.w);
+    }
   }
 }
 
@@ -1417,7 +1451,7 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
     st = launched();
   }
   if (st == MAMBA_OK) {
-    const int64_t nbc = a.batch * a.N * a.L;
+    const int64_t nbc = a.batch * a.N * (a.L / 4);
     bwd_staged_finalize_bc<T><<<unsigned(std::min<int64_t>(ceil_div(nbc, 256), sms * 8)), 256, 0, s>>>(bp);
     st = launched();
   }
