@@ -128,8 +128,12 @@ constexpr int kProjMaxRp = 256;
 constexpr uint32_t kProjAcc = kProjMaxRp / 2;
 constexpr uint32_t kProjTmemCols = 256;
 // The thread that issues the projection MMAs: lane 0 of the last warp, so that
-// warp 0, which issues the TMA loads and stores, does not carry both.
+// it is not one of the threads that store y and issue the TMA loads.
 constexpr int kMmaThread = 96;
+// The forward's TMA producer (tile loads, unit tickets): a thread of warp 1,
+// so that its work after each tile's barrier runs beside warp 0's store of
+// the y tile instead of after it.
+constexpr int kProdThread = 32;
 
 // Thread's row d of W_dt (bf16, R per row) into its TMEM lane from column
 // `taddr`'s on: Rp/2 columns of bf16 pairs (even k in the low half), zero
@@ -571,7 +575,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
   };
 
   constexpr bool kLookahead = !kSeq;
-  if (tid == 0) {
+  if (tid == kProdThread) {
     produce(true);
     for (int s = 1; s < NST; ++s) produce(kLookahead);
   }
@@ -886,14 +890,13 @@ __global__ void __launch_bounds__(kSThreads, 2)
           __syncthreads();
         }
         if (q[8]) return;
-        if (tid == 0) {
-          if (kOut) {
-            tma_store_3d(&tm_y, sy, int(t0), d0, b);
-            bulk_commit();
-            bulk_wait_read<1>();
-          }
-          produce(kLookahead);
+        // the y tile's store (warp 0) and the next loads (warp 1) in parallel
+        if (kOut && tid == 0) {
+          tma_store_3d(&tm_y, sy, int(t0), d0, b);
+          bulk_commit();
+          bulk_wait_read<1>();
         }
+        if (tid == kProdThread) produce(kLookahead);
       }
       if constexpr (M == MODE_GEN) {
 #pragma unroll
@@ -939,7 +942,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
       __syncthreads();
       if (tid == 0 && !(p.test_hook == 1 && g == 0 && k == 0)) st_release_gpu(p.flags + g, k + 1);
     }
-    if (!kLookahead && tid == 0) {  // claim the next unit and fill the free stages
+    if (!kLookahead && tid == kProdThread) {  // claim the next unit and fill the free stages
       produce(true);
       while (!p_done && p_issued < ctile + NST && p_tile < p_ntiles) produce(false);
     }
@@ -948,13 +951,11 @@ __global__ void __launch_bounds__(kSThreads, 2)
   // Drain: every TMA load this CTA issued must land before it exits, and
   // (PROJ) every MMA it issued must complete before TMEM is freed.
   __syncthreads();
-  if (tid == 0) {
-    if (aborted) {
-      for (int t = ctile; t < p_issued; ++t)
-        mbar_wait_bounded(&bars[t % NST], uint32_t(t / NST) & 1u, p.timeout_ns);
-    }
-    bulk_wait<0>();
+  if (tid == kProdThread && aborted) {
+    for (int t = ctile; t < p_issued; ++t)
+      mbar_wait_bounded(&bars[t % NST], uint32_t(t / NST) & 1u, p.timeout_ns);
   }
+  if (tid == 0) bulk_wait<0>();
   if (PROJ && tid == kMmaThread && mma_issued >= 0)
     mbar_wait_bounded(&mma_bar[mma_issued & 1], uint32_t(mma_issued >> 1) & 1u, p.timeout_ns);
   if constexpr (PROJ) {
