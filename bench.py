@@ -314,7 +314,7 @@ def run_ours(args, world, rank, device):
     if args.only == "cplx":  # the complex-A calls alone, for profiling
         if args.cplx_batch:
             w = dataclasses.replace(w, batch=args.cplx_batch)
-        res = run_cplx(w, device, measured_peaks(), steps=args.steps)
+        res = run_cplx(w, device, measured_peaks(), steps=args.steps, pair=args.step == "pair")
         return {"note": "--only cplx: a profiling run, not a benchmark result", "complex_A": res}
     if args.only == "dtproj":  # the projection calls alone, for profiling
         if args.cplx_batch:
@@ -506,7 +506,7 @@ def run_ours(args, world, rank, device):
     if not args.only and not args.no_dtproj:
         result["dt_projection"] = run_dtproj(w, x, device, steps=args.conv_steps)
     if not args.only and not args.no_cplx:
-        result["complex_A"] = run_cplx(w, device, peaks, steps=3)
+        result["complex_A"] = run_cplx(w, device, peaks, steps=3, pair=args.step == "pair")
     if args.only:
         result["note"] = f"--only {args.only}: a profiling run, not a benchmark result"
     if not args.no_e2e and not args.only:
@@ -731,11 +731,11 @@ def run_dtproj(w, x, device, steps=10):
             "shape": f"dt_low (batch {w.batch}, R {R}, L {w.L}), W_dt ({w.dim}, {R})"}
 
 
-def run_cplx(w, device, peaks, steps=3):
+def run_cplx(w, device, peaks, steps=3, pair=True):
     """The workload's shape with a complex diagonal A (S4D-Lin) of N complex
-    states, complex B and C: mamba_cplx_scan_fwd / _bwd, timed per call with
-    CUDA events.  Bytes: the real scan's plus the doubled B, C (and dB, dC)
-    rows."""
+    states, complex B and C: the training pair mamba_cplx_scan_fwd_save /
+    _bwd_saved (pair=False: the plain calls), timed per call with CUDA events.
+    Bytes: the real scan's plus the doubled B, C (and dB, dC) rows."""
     from selective_state_space_21_b200 import scan
     from selective_state_space_21_b200.inputs import make_cplx_inputs
 
@@ -746,15 +746,26 @@ def run_cplx(w, device, peaks, steps=3):
     g = {k: torch.empty_like(x[k]) for k in ("u", "delta", "z", "B", "C")}
     dA = torch.empty(w.dim, 2 * w.N, **f32)
     dD, db = torch.empty(w.dim, **f32), torch.empty(w.dim, **f32)
+    saved = (torch.empty(scan.cplx_saved_bytes(w.batch, w.dim, w.L, w.N, w.dtype), device=device,
+                         dtype=torch.uint8) if pair else None)
 
     def fwd():
-        scan.mamba_cplx_scan_fwd(x["u"], x["delta"], x["delta_bias"], x["A"], x["B"], x["C"],
-                                 x["D"], x["z"], y, None)
+        if pair:
+            scan.mamba_cplx_scan_fwd_save(x["u"], x["delta"], x["delta_bias"], x["A"], x["B"],
+                                          x["C"], x["D"], x["z"], y, None, saved)
+        else:
+            scan.mamba_cplx_scan_fwd(x["u"], x["delta"], x["delta_bias"], x["A"], x["B"], x["C"],
+                                     x["D"], x["z"], y, None)
 
     def bwd():
-        scan.mamba_cplx_scan_bwd(x["u"], x["delta"], x["delta_bias"], x["A"], x["B"], x["C"],
-                                 x["D"], x["z"], x["dy"], g["u"], g["delta"], dA, g["B"], g["C"],
-                                 dD, g["z"], db)
+        if pair:
+            scan.mamba_cplx_scan_bwd_saved(x["u"], x["delta"], x["delta_bias"], x["A"], x["B"],
+                                           x["C"], x["D"], x["z"], x["dy"], g["u"], g["delta"], dA,
+                                           g["B"], g["C"], dD, g["z"], db, saved)
+        else:
+            scan.mamba_cplx_scan_bwd(x["u"], x["delta"], x["delta_bias"], x["A"], x["B"], x["C"],
+                                     x["D"], x["z"], x["dy"], g["u"], g["delta"], dA, g["B"],
+                                     g["C"], dD, g["z"], db)
 
     fwd()
     bwd()
@@ -783,6 +794,8 @@ def run_cplx(w, device, peaks, steps=3):
                     "frac_hbm": round(bb / (bms * 1e-3) / 1e9 / hbm, 4),
                     "tc_per_s": w.token_channels / (bms * 1e-3)},
             "steps": steps, "timing": "median of per-call CUDA events",
+            "calls": ("mamba_cplx_scan_fwd_save + mamba_cplx_scan_bwd_saved" if pair
+                      else "mamba_cplx_scan_fwd + mamba_cplx_scan_bwd"),
             "shape": f"batch {w.batch} x dim {w.dim} x L {w.L}, {w.N} complex states"}
 
 

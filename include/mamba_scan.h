@@ -392,6 +392,40 @@ MAMBA_SCAN_API mamba_status_t mamba_cplx_scan_bwd(const void *u, const void *del
                                                   mamba_dtype_t dtype, mamba_stream_t stream);
 
 /*
+ * The training pair with complex A: mamba_cplx_scan_fwd_save is
+ * mamba_cplx_scan_fwd that also stores the state at the start of every
+ * 8-step block (the backward's block checkpoints: (batch*dim, ceil(L/8),
+ * 2 NM) fp32, NM = N rounded up to 1, 2, 4, 8 or 16) into `saved` (device
+ * memory, 16-byte aligned, at least mamba_cplx_scan_saved_bytes bytes);
+ * mamba_cplx_scan_bwd_saved is mamba_cplx_scan_bwd reading them in place of
+ * its forward sweep.  `saved` must come from mamba_cplx_scan_fwd_save with
+ * the same u, delta, delta_bias, A, B, shape and dtype on the same device,
+ * ordered before it on the stream; anything else gives undefined gradients.
+ * The gradients are those of mamba_cplx_scan_bwd to rounding (the states are
+ * the same recurrence, formed by the forward kernel).  A NULL `saved`, or one
+ * smaller than the size, returns MAMBA_ERR_INVALID_ARG with nothing enqueued.
+ */
+MAMBA_SCAN_API mamba_status_t mamba_cplx_scan_saved_bytes(int64_t batch, int64_t dim, int64_t L,
+                                                          int64_t N, mamba_dtype_t dtype,
+                                                          uint64_t *bytes);
+
+MAMBA_SCAN_API mamba_status_t mamba_cplx_scan_fwd_save(const void *u, const void *delta,
+                                                       const float *delta_bias, const float *A,
+                                                       const void *B, const void *C,
+                                                       const float *D, const void *z, void *y,
+                                                       float *last_state, int64_t batch,
+                                                       int64_t dim, int64_t L, int64_t N,
+                                                       mamba_dtype_t dtype, void *saved,
+                                                       uint64_t saved_bytes,
+                                                       mamba_stream_t stream);
+
+MAMBA_SCAN_API mamba_status_t mamba_cplx_scan_bwd_saved(
+    const void *u, const void *delta, const float *delta_bias, const float *A, const void *B,
+    const void *C, const float *D, const void *z, const void *dy, void *du, void *ddelta, float *dA,
+    void *dB, void *dC, float *dD, void *dz, float *ddelta_bias, int64_t batch, int64_t dim, int64_t L,
+    int64_t N, mamba_dtype_t dtype, const void *saved, uint64_t saved_bytes, mamba_stream_t stream);
+
+/*
  * One decoding step: the recurrent mode of the selective SSM, one token per
  * call with constant work per token ("Mamba: Linear-Time Sequence Modeling
  * with Selective State Spaces", trishampatil.com walk-through, Part II

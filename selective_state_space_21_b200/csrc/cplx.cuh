@@ -49,6 +49,14 @@ struct CplxArgs {
   float *last_state, *dA, *dD, *dbias;  // last_state (batch, dim, 2N), dA (dim, 2N)
   int64_t batch, dim, L;
   int N;
+  // (the saving forward) the state at the start of every kCplxBwdTC-step
+  // block, laid out as the backward's block checkpoints: (batch*dim,
+  // n_blocks, 2 NM), real parts first; null: not stored
+  float *save_ckpt = nullptr;
+  int64_t save_blocks = 0;
+  // (the backward from saved states) those checkpoints, written by the
+  // saving forward of the same inputs: the forward sweep does not run
+  const float *saved_ckpt = nullptr;
 };
 
 constexpr int kCplxThreads = 128;
@@ -297,6 +305,19 @@ __global__ void __launch_bounds__(kCplxThreads) cplx_fwd_kernel(const CplxArgs a
     const int steps = int(a.L - t0 < kCplxTT ? a.L - t0 : kCplxTT);
     for (int i = 0; i < steps; ++i) {
       const int64_t t = t0 + i;
+      if (a.save_ckpt && valid && t % kCplxBwdTC == 0) {  // the state at a block start
+        float *ck = a.save_ckpt + ((b * a.dim + d) * a.save_blocks + t / kCplxBwdTC) * 2 * NM + part * NS;
+        if constexpr (NS == 4) {  // 16-byte stores (the row is 128-byte aligned)
+          *reinterpret_cast<float4 *>(ck) = make_float4(hr[0], hr[1], hr[2], hr[3]);
+          *reinterpret_cast<float4 *>(ck + NM) = make_float4(hi[0], hi[1], hi[2], hi[3]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < NS; ++j) {
+            ck[j] = hr[j];
+            ck[NM + j] = hi[j];
+          }
+        }
+      }
       const float Delta = softplus_fast(to_f(dl[t]) + bias);
       const float ut = to_f(u[t]);
       const float *tr = tab + i * cplx_tab_stride<NM, kCplxTT>() + part * NS;
@@ -361,6 +382,8 @@ struct CplxWork {
   int64_t bpc;
   int *counter;      // ticket counters of the two launches, zero before the first
   int *flags;        // (n_dblk * batch): the forward sweep counts chunks 1..K, the reverse K+1..2K
+  int flag_base;     // the reverse sweep's count starts here: K, or 0 without a forward sweep
+                     // (block checkpoints saved by the forward)
   float *carry;      // (n_dblk * batch, kCplxBwdThreads, 4 NS)
   uint64_t timeout_ns;
 };
@@ -625,7 +648,7 @@ __global__ void __launch_bounds__(kCplxBwdThreads, 8) cplx_bwd_kernel(const Cplx
   const int kbase = lane_scatter_base<NV, TPC>(lane);
   if (k + 1 < w.K) {  // the adjoint entering from the later chunk (and its Abar)
     // (the reverse sweep counts on from the forward sweep's K)
-    if (tid == 0 && !wait_flag_geq(w.flags + cb, w.K + (w.K - 1 - k), w.timeout_ns)) {
+    if (tid == 0 && !wait_flag_geq(w.flags + cb, w.flag_base + (w.K - 1 - k), w.timeout_ns)) {
       record_timeout();
       s_abort = 1;
     }
@@ -810,7 +833,7 @@ __global__ void __launch_bounds__(kCplxBwdThreads, 8) cplx_bwd_kernel(const Cplx
   }
   __threadfence();
   __syncthreads();
-  if (tid == 0) st_release_gpu(w.flags + cb, w.K + (w.K - k));
+  if (tid == 0) st_release_gpu(w.flags + cb, w.flag_base + (w.K - k));
   }
   }
 }

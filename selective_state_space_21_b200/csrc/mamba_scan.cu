@@ -303,7 +303,8 @@ struct CplxBwdLauncher {
     if (n_cb * w.K > (int64_t(1) << 30)) return MAMBA_ERR_UNSUPPORTED;
     w.timeout_ns = kDefaultTimeoutNs;
     const size_t bd = size_t(a.batch * a.dim);
-    const size_t n_ckpt = bd * size_t(w.n_blocks) * 2 * NM;
+    const bool saved = a.saved_ckpt != nullptr;  // block checkpoints from the saving forward
+    const size_t n_ckpt = saved ? 0 : bd * size_t(w.n_blocks) * 2 * NM;
     const size_t n_bc = size_t(w.n_dblk) * size_t(a.batch) * 4 * kMaxN * size_t(a.L);
     const size_t n_A = size_t(w.K) * bd * 2 * size_t(a.N);
     const size_t n_par = size_t(w.K) * bd;
@@ -317,8 +318,9 @@ struct CplxBwdLauncher {
     }
     w.counter = reinterpret_cast<int *>(ws);
     w.flags = w.counter + 2;
-    w.ckpt = reinterpret_cast<float *>(ws + int_bytes);
-    w.part_bc = w.ckpt + n_ckpt;
+    w.flag_base = saved ? 0 : w.K;
+    w.ckpt = saved ? const_cast<float *>(a.saved_ckpt) : reinterpret_cast<float *>(ws + int_bytes);
+    w.part_bc = reinterpret_cast<float *>(ws + int_bytes) + n_ckpt;
     w.part_A = w.part_bc + n_bc;
     w.part_D = w.part_A + n_A;
     w.part_bias = w.part_D + n_par;
@@ -326,7 +328,7 @@ struct CplxBwdLauncher {
     mamba_status_t st = MAMBA_OK;
     if (cudaMemsetAsync(ws, 0, int_bytes, s) != cudaSuccess) st = MAMBA_ERR_CUDA;
     const unsigned grid = unsigned(std::min<int64_t>(n_cb * w.K, slots));
-    if (st == MAMBA_OK) {  // the forward sweep (block-start states), then the reverse sweep
+    if (st == MAMBA_OK && !saved) {  // the forward sweep (block-start states), then the reverse sweep
       kf<<<grid, kCplxBwdThreads, smem, s>>>(a, w);
       st = launch_status();
     }
@@ -1354,11 +1356,18 @@ mamba_status_t mamba_dtproj_scan_bwd(const void *u, const void *dt_low, const vo
 
 // ------------------------------------------------ complex diagonal A
 
-mamba_status_t mamba_cplx_scan_fwd(const void *u, const void *delta, const float *delta_bias,
-                                   const float *A, const void *B, const void *C, const float *D,
-                                   const void *z, void *y, float *last_state, int64_t batch,
-                                   int64_t dim, int64_t L, int64_t N, mamba_dtype_t dtype,
-                                   mamba_stream_t stream) {
+// Bytes of the complex forward's saved block checkpoints: (batch*dim,
+// ceil(L/8), 2 NM) fp32, NM the state count the kernels are instantiated for.
+static uint64_t cplx_saved_bytes_for(int64_t batch, int64_t dim, int64_t L, int64_t N) {
+  const int64_t nm = N <= 1 ? 1 : N <= 2 ? 2 : N <= 4 ? 4 : N <= 8 ? 8 : 16;
+  return uint64_t(batch) * uint64_t(dim) * uint64_t((L + kCplxBwdTC - 1) / kCplxBwdTC) * 2 * nm * 4;
+}
+
+static mamba_status_t cplx_fwd_entry(const void *u, const void *delta, const float *delta_bias,
+                                     const float *A, const void *B, const void *C, const float *D,
+                                     const void *z, void *y, float *last_state, int64_t batch,
+                                     int64_t dim, int64_t L, int64_t N, mamba_dtype_t dtype,
+                                     mamba_stream_t stream, void *saved, uint64_t saved_bytes) {
   mamba_status_t st = check_shape(batch, dim, L, N, dtype);
   if (st != MAMBA_OK) return st;
   Checker ck;
@@ -1379,6 +1388,11 @@ mamba_status_t mamba_cplx_scan_fwd(const void *u, const void *delta, const float
   ck.buf(delta_bias, size_t(dim) * 4, 4, false, false);
   ck.buf(y, nbdl * es, es, true, true);
   ck.buf(last_state, size_t(batch) * dim * 2 * N * 4, 4, false, true);
+  const uint64_t need = saved ? cplx_saved_bytes_for(batch, dim, L, N) : 0;
+  if (saved) {
+    if (need > saved_bytes) return MAMBA_ERR_INVALID_ARG;
+    ck.buf(saved, need, 16, true, true);
+  }
   if (ck.st != MAMBA_OK) return ck.st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (batch == 0 || dim == 0) return MAMBA_OK;
@@ -1393,15 +1407,49 @@ mamba_status_t mamba_cplx_scan_fwd(const void *u, const void *delta, const float
   a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
   a.bias = delta_bias; a.A = A; a.D = D; a.y = y; a.last_state = last_state;
   a.batch = batch; a.dim = dim; a.L = L; a.N = (int)N;
+  if (need) {
+    a.save_ckpt = static_cast<float *>(saved);
+    a.save_blocks = (L + kCplxBwdTC - 1) / kCplxBwdTC;
+  }
   return dispatch<CplxFwdLauncher>(dtype, (int)N, a, s);
 }
 
-mamba_status_t mamba_cplx_scan_bwd(const void *u, const void *delta, const float *delta_bias,
+mamba_status_t mamba_cplx_scan_fwd(const void *u, const void *delta, const float *delta_bias,
                                    const float *A, const void *B, const void *C, const float *D,
-                                   const void *z, const void *dy, void *du, void *ddelta,
-                                   float *dA, void *dB, void *dC, float *dD, void *dz,
-                                   float *ddelta_bias, int64_t batch, int64_t dim, int64_t L,
-                                   int64_t N, mamba_dtype_t dtype, mamba_stream_t stream) {
+                                   const void *z, void *y, float *last_state, int64_t batch,
+                                   int64_t dim, int64_t L, int64_t N, mamba_dtype_t dtype,
+                                   mamba_stream_t stream) {
+  return cplx_fwd_entry(u, delta, delta_bias, A, B, C, D, z, y, last_state, batch, dim, L, N, dtype,
+                        stream, nullptr, 0);
+}
+
+mamba_status_t mamba_cplx_scan_saved_bytes(int64_t batch, int64_t dim, int64_t L, int64_t N,
+                                           mamba_dtype_t dtype, uint64_t *bytes) {
+  if (!bytes) return MAMBA_ERR_INVALID_ARG;
+  *bytes = 0;
+  const mamba_status_t st = check_shape(batch, dim, L, N, dtype);
+  if (st != MAMBA_OK) return st;
+  *bytes = cplx_saved_bytes_for(batch, dim, L, N);
+  return MAMBA_OK;
+}
+
+mamba_status_t mamba_cplx_scan_fwd_save(const void *u, const void *delta, const float *delta_bias,
+                                        const float *A, const void *B, const void *C, const float *D,
+                                        const void *z, void *y, float *last_state, int64_t batch,
+                                        int64_t dim, int64_t L, int64_t N, mamba_dtype_t dtype,
+                                        void *saved, uint64_t saved_bytes, mamba_stream_t stream) {
+  if (!saved && cplx_saved_bytes_for(batch, dim, L, N) > 0) return MAMBA_ERR_INVALID_ARG;
+  return cplx_fwd_entry(u, delta, delta_bias, A, B, C, D, z, y, last_state, batch, dim, L, N, dtype,
+                        stream, saved, saved_bytes);
+}
+
+static mamba_status_t cplx_bwd_entry(const void *u, const void *delta, const float *delta_bias,
+                                     const float *A, const void *B, const void *C, const float *D,
+                                     const void *z, const void *dy, void *du, void *ddelta,
+                                     float *dA, void *dB, void *dC, float *dD, void *dz,
+                                     float *ddelta_bias, int64_t batch, int64_t dim, int64_t L,
+                                     int64_t N, mamba_dtype_t dtype, mamba_stream_t stream,
+                                     const void *saved, uint64_t saved_bytes) {
   mamba_status_t st = check_shape(batch, dim, L, N, dtype);
   if (st != MAMBA_OK) return st;
   if ((z == nullptr) != (dz == nullptr) || (D == nullptr) != (dD == nullptr))
@@ -1431,6 +1479,11 @@ mamba_status_t mamba_cplx_scan_bwd(const void *u, const void *delta, const float
   ck.buf(dA, size_t(dim) * 2 * N * 4, 4, true, true);
   ck.buf(dD, size_t(dim) * 4, 4, false, true);
   ck.buf(ddelta_bias, size_t(dim) * 4, 4, false, true);
+  if (saved) {
+    const uint64_t need = cplx_saved_bytes_for(batch, dim, L, N);
+    if (need > saved_bytes) return MAMBA_ERR_INVALID_ARG;
+    ck.buf(saved, need, 16, true, false);
+  }
   if (ck.st != MAMBA_OK) return ck.st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (dim == 0) return MAMBA_OK;
@@ -1449,7 +1502,30 @@ mamba_status_t mamba_cplx_scan_bwd(const void *u, const void *delta, const float
   a.du = du; a.ddelta = ddelta; a.dz = dz; a.dB = dB; a.dC = dC;
   a.dA = dA; a.dD = dD; a.dbias = ddelta_bias;
   a.batch = batch; a.dim = dim; a.L = L; a.N = (int)N;
+  a.saved_ckpt = static_cast<const float *>(saved);
   return dispatch<CplxBwdLauncher>(dtype, (int)N, a, s);
+}
+
+mamba_status_t mamba_cplx_scan_bwd(const void *u, const void *delta, const float *delta_bias,
+                                   const float *A, const void *B, const void *C, const float *D,
+                                   const void *z, const void *dy, void *du, void *ddelta,
+                                   float *dA, void *dB, void *dC, float *dD, void *dz,
+                                   float *ddelta_bias, int64_t batch, int64_t dim, int64_t L,
+                                   int64_t N, mamba_dtype_t dtype, mamba_stream_t stream) {
+  return cplx_bwd_entry(u, delta, delta_bias, A, B, C, D, z, dy, du, ddelta, dA, dB, dC, dD, dz,
+                        ddelta_bias, batch, dim, L, N, dtype, stream, nullptr, 0);
+}
+
+mamba_status_t mamba_cplx_scan_bwd_saved(const void *u, const void *delta, const float *delta_bias,
+                                         const float *A, const void *B, const void *C, const float *D,
+                                         const void *z, const void *dy, void *du, void *ddelta,
+                                         float *dA, void *dB, void *dC, float *dD, void *dz,
+                                         float *ddelta_bias, int64_t batch, int64_t dim, int64_t L,
+                                         int64_t N, mamba_dtype_t dtype, const void *saved,
+                                         uint64_t saved_bytes, mamba_stream_t stream) {
+  if (!saved && cplx_saved_bytes_for(batch, dim, L, N) > 0) return MAMBA_ERR_INVALID_ARG;
+  return cplx_bwd_entry(u, delta, delta_bias, A, B, C, D, z, dy, du, ddelta, dA, dB, dC, dD, dz,
+                        ddelta_bias, batch, dim, L, N, dtype, stream, saved, saved_bytes);
 }
 
 }  // extern "C"

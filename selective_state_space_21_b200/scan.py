@@ -104,6 +104,12 @@ def load_library():
             lib.mamba_cplx_scan_fwd.restype = ctypes.c_int
             lib.mamba_cplx_scan_bwd.argtypes = [vp] * 17 + [i64] * 4 + [i32, vp]
             lib.mamba_cplx_scan_bwd.restype = ctypes.c_int
+            lib.mamba_cplx_scan_saved_bytes.argtypes = [i64] * 4 + [i32, ctypes.POINTER(ctypes.c_uint64)]
+            lib.mamba_cplx_scan_saved_bytes.restype = ctypes.c_int
+            lib.mamba_cplx_scan_fwd_save.argtypes = [vp] * 10 + [i64] * 4 + [i32, vp, ctypes.c_uint64, vp]
+            lib.mamba_cplx_scan_fwd_save.restype = ctypes.c_int
+            lib.mamba_cplx_scan_bwd_saved.argtypes = [vp] * 17 + [i64] * 4 + [i32, vp, ctypes.c_uint64, vp]
+            lib.mamba_cplx_scan_bwd_saved.restype = ctypes.c_int
             for f in ("mamba_scan_fwd", "mamba_scan_fwd_ex", "mamba_scan_bwd",
                       "mamba_scan_bwd_ex", "mamba_scan_stream_status", "mamba_scan_fwd_noalloc"):
                 getattr(lib, f).restype = ctypes.c_int
@@ -481,10 +487,7 @@ def mamba_dtproj_scan_bwd(u, dt_low, W_dt, delta_bias, A, B, C, D, z, dy, du, d_
            "mamba_dtproj_scan_bwd")
 
 
-def mamba_cplx_scan_fwd(u, delta, delta_bias, A, B, C, D, z, y, last_state, *, stream=None):
-    """Enqueue the forward with a complex diagonal A.  Complex vectors are
-    planar, real parts first: A (dim, 2N) float32, B and C (batch, 2N, L) in
-    the I/O dtype, last_state (batch, dim, 2N) float32."""
+def _cplx_fwd_args(u, delta, delta_bias, A, B, C, D, z, y, last_state):
     batch, dim, L = u.shape
     N = A.shape[1] // 2
     dt = u.dtype
@@ -497,15 +500,41 @@ def mamba_cplx_scan_fwd(u, delta, delta_bias, A, B, C, D, z, y, last_state, *, s
         _ptr(z, dt, bdl, "z"), _ptr(y, dt, bdl, "y"),
         _ptr(last_state, f32, (batch, dim, 2 * N), "last_state"), batch, dim, L, N,
         _dtype_code(dt)]
+    return args
+
+
+def mamba_cplx_scan_fwd(u, delta, delta_bias, A, B, C, D, z, y, last_state, *, stream=None):
+    """Enqueue the forward with a complex diagonal A.  Complex vectors are
+    planar, real parts first: A (dim, 2N) float32, B and C (batch, 2N, L) in
+    the I/O dtype, last_state (batch, dim, 2N) float32."""
+    args = _cplx_fwd_args(u, delta, delta_bias, A, B, C, D, z, y, last_state)
     _check(load_library().mamba_cplx_scan_fwd(*args, _stream_handle(stream)),
            "mamba_cplx_scan_fwd")
 
 
-def mamba_cplx_scan_bwd(u, delta, delta_bias, A, B, C, D, z, dy, du, ddelta, dA, dB, dC, dD, dz,
-                        ddelta_bias, *, stream=None):
-    """Enqueue the backward of sum(dy * y) for ``mamba_cplx_scan_fwd``; dA
-    (dim, 2N) float32 and dB, dC (batch, 2N, L) hold (d/d re, d/d im) pairs,
-    planar."""
+def cplx_saved_bytes(batch, dim, L, N, dtype) -> int:
+    """Bytes of the block checkpoints the complex training pair keeps."""
+    n = ctypes.c_uint64(0)
+    _check(load_library().mamba_cplx_scan_saved_bytes(batch, dim, L, N, _dtype_code(dtype),
+                                                      ctypes.byref(n)),
+           "mamba_cplx_scan_saved_bytes")
+    return int(n.value)
+
+
+def mamba_cplx_scan_fwd_save(u, delta, delta_bias, A, B, C, D, z, y, last_state, saved, *,
+                             stream=None):
+    """``mamba_cplx_scan_fwd`` that also fills ``saved`` (``cplx_saved_bytes``
+    bytes, uint8) with the block checkpoints for ``mamba_cplx_scan_bwd_saved``."""
+    batch, dim, L = u.shape
+    need = cplx_saved_bytes(batch, dim, L, A.shape[1] // 2, u.dtype)
+    sp, sn = _saved_arg(saved, need)
+    args = _cplx_fwd_args(u, delta, delta_bias, A, B, C, D, z, y, last_state)
+    _check(load_library().mamba_cplx_scan_fwd_save(*args, sp, sn, _stream_handle(stream)),
+           "mamba_cplx_scan_fwd_save")
+
+
+def _cplx_bwd_args(u, delta, delta_bias, A, B, C, D, z, dy, du, ddelta, dA, dB, dC, dD, dz,
+                   ddelta_bias):
     batch, dim, L = u.shape
     N = A.shape[1] // 2
     dt = u.dtype
@@ -520,8 +549,31 @@ def mamba_cplx_scan_bwd(u, delta, delta_bias, A, B, C, D, z, dy, du, ddelta, dA,
         _ptr(dB, dt, bnl, "dB"), _ptr(dC, dt, bnl, "dC"), _ptr(dD, f32, (dim,), "dD"),
         _ptr(dz, dt, bdl, "dz"), _ptr(ddelta_bias, f32, (dim,), "ddelta_bias"),
         batch, dim, L, N, _dtype_code(dt)]
+    return args
+
+
+def mamba_cplx_scan_bwd(u, delta, delta_bias, A, B, C, D, z, dy, du, ddelta, dA, dB, dC, dD, dz,
+                        ddelta_bias, *, stream=None):
+    """Enqueue the backward of sum(dy * y) for ``mamba_cplx_scan_fwd``; dA
+    (dim, 2N) float32 and dB, dC (batch, 2N, L) hold (d/d re, d/d im) pairs,
+    planar."""
+    args = _cplx_bwd_args(u, delta, delta_bias, A, B, C, D, z, dy, du, ddelta, dA, dB, dC, dD, dz,
+                          ddelta_bias)
     _check(load_library().mamba_cplx_scan_bwd(*args, _stream_handle(stream)),
            "mamba_cplx_scan_bwd")
+
+
+def mamba_cplx_scan_bwd_saved(u, delta, delta_bias, A, B, C, D, z, dy, du, ddelta, dA, dB, dC, dD,
+                              dz, ddelta_bias, saved, *, stream=None):
+    """``mamba_cplx_scan_bwd`` reading the block checkpoints
+    ``mamba_cplx_scan_fwd_save`` stored, in place of its forward sweep."""
+    batch, dim, L = u.shape
+    need = cplx_saved_bytes(batch, dim, L, A.shape[1] // 2, u.dtype)
+    sp, sn = _saved_arg(saved, need)
+    args = _cplx_bwd_args(u, delta, delta_bias, A, B, C, D, z, dy, du, ddelta, dA, dB, dC, dD, dz,
+                          ddelta_bias)
+    _check(load_library().mamba_cplx_scan_bwd_saved(*args, sp, sn, _stream_handle(stream)),
+           "mamba_cplx_scan_bwd_saved")
 
 
 def mamba_scan_fwd_noalloc(u, delta, delta_bias, A, B, C, D, z, y, last_state, *, stream=None):

@@ -258,3 +258,69 @@ def test_cplx_bwd_many_channels(shape):
     dC included, against the oracle."""
     b, d, L, N = shape
     check(make_cplx_inputs(b, d, L, N, torch.float32, seed=1500 + d + L, with_dy=True))
+
+
+def pair(x):
+    """The complex training pair: the forward stores the block checkpoints, the
+    backward reads them in place of its forward sweep."""
+    batch, dim, L = x["u"].shape
+    saved = torch.empty(scan.cplx_saved_bytes(batch, dim, L, x["A"].shape[1] // 2, x["u"].dtype),
+                        device="cuda", dtype=torch.uint8)
+    y = torch.empty_like(x["u"])
+    last = torch.empty(batch, dim, x["A"].shape[1], device="cuda")
+    scan.mamba_cplx_scan_fwd_save(x["u"], x["delta"], x["delta_bias"], x["A"], x["B"], x["C"],
+                                  x["D"], x["z"], y, last, saved)
+    dim, N2 = x["A"].shape
+    f32 = dict(device="cuda", dtype=torch.float32)
+    g = {"du": torch.empty_like(x["u"]), "ddelta": torch.empty_like(x["u"]),
+         "dA": torch.empty(dim, N2, **f32), "dB": torch.empty_like(x["B"]),
+         "dC": torch.empty_like(x["C"]),
+         "dD": torch.empty(dim, **f32) if x["D"] is not None else None,
+         "dz": torch.empty_like(x["u"]) if x["z"] is not None else None,
+         "ddelta_bias": torch.empty(dim, **f32)}
+    scan.mamba_cplx_scan_bwd_saved(x["u"], x["delta"], x["delta_bias"], x["A"], x["B"], x["C"],
+                                   x["D"], x["z"], x["dy"], g["du"], g["ddelta"], g["dA"], g["dB"],
+                                   g["dC"], g["dD"], g["dz"], g["ddelta_bias"], saved)
+    assert scan.mamba_scan_stream_status() == 0
+    return y, last, {k: v for k, v in g.items() if v is not None}
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("shape", [(2, 200, 300, 16), (1, 70, 129, 8), (3, 5, 40, 1),
+                                   (1, 9, 1, 16), (2, 50, 33, 12), (8, 2560, 64, 16)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_cplx_pair(shape, dtype):
+    """y and the gradients of the pair against the plain calls (the same
+    recurrence: within 1e-5 normwise in fp32, within the bf16 bar in bf16) and,
+    at the small shapes, against the fp64 oracle.  The last shape has more
+    channel blocks than CTA slots: four chunks per sequence in the backward."""
+    b, d, L, N = shape
+    xh = make_cplx_inputs(b, d, L, N, dtype, seed=1600 + d + L, with_dy=True)
+    x = gc.to_device(xh)
+    y, last, g = pair(x)
+    y0, last0 = gpu_fwd(x)
+    g0 = gpu_bwd(x)
+    assert torch.equal(y, y0) and torch.equal(last, last0)  # the same forward kernel
+    gt = 1e-5 if dtype == torch.float32 else gc.TOL[dtype]
+    for k in g0:
+        if g0[k] is not None:
+            e = gc.normwise(g[k].cpu().double().numpy(), g0[k].cpu().double().numpy())
+            assert e <= gt, f"{k}: {e:.2e} from the backward with its own forward sweep"
+    if b * d * L <= 200 * 300 * 2:
+        tol = gc.TOL[dtype]
+        kw = dict(delta_bias=xh["delta_bias"], D=xh["D"], z=xh["z"])
+        ref = oracle.s6_cplx_backward(xh["u"], xh["delta"], xh["A"], xh["B"], xh["C"], xh["dy"],
+                                      **kw)
+        errs = {k: gc.normwise(g[k].cpu().double().numpy(), ref[k]) for k in GRADS if k in g}
+        assert all(e <= tol for e in errs.values()), errs
+
+
+def test_cplx_pair_refuses_a_missing_buffer():
+    x = gc.to_device(make_cplx_inputs(1, 8, 32, 4, torch.float32, seed=1601, with_dy=True))
+    lib = scan.load_library()
+    y = torch.empty_like(x["u"])
+    rc = lib.mamba_cplx_scan_fwd_save(
+        x["u"].data_ptr(), x["delta"].data_ptr(), x["delta_bias"].data_ptr(), x["A"].data_ptr(),
+        x["B"].data_ptr(), x["C"].data_ptr(), x["D"].data_ptr(), x["z"].data_ptr(), y.data_ptr(),
+        None, 1, 8, 32, 4, scan._dtype_code(torch.float32), None, 0, None)
+    assert rc == 1  # MAMBA_ERR_INVALID_ARG

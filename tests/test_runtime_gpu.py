@@ -224,10 +224,19 @@ def _calls():
         f["u"], cp["conv_w"], cp["conv_b"], f["delta"], f["delta_bias"], f["A"], f["B"], f["C"],
         f["D"], f["z"], f["dy"], o["du"], o["dcw"], o["dcb"], o["dd"], o["dA"], o["dB"], o["dC"],
         o["dD"], o["dz"], o["db"], csaved), conv_outs))
+    xsaved = torch.empty(scan.cplx_saved_bytes(2, 70, 64, 8, torch.float32), device="cuda",
+                         dtype=torch.uint8)
+    scan.mamba_cplx_scan_fwd_save(cx["u"], cx["delta"], cx["delta_bias"], cx["A"], cx["B"], cx["C"],
+                                  cx["D"], cx["z"], torch.empty_like(cx["u"]), None, xsaved)
+    torch.cuda.synchronize()
+    out.append(("cplx bwd saved", lambda o: scan.mamba_cplx_scan_bwd_saved(
+        cx["u"], cx["delta"], cx["delta_bias"], cx["A"], cx["B"], cx["C"], cx["D"], cx["z"],
+        cx["dy"], o["du"], o["dd"], o["dA"], o["dB"], o["dC"], o["dD"], o["dz"], o["db"], xsaved),
+        lambda: bwd_outs(cx)))
     return out
 
 
-@pytest.mark.parametrize("index", range(14))
+@pytest.mark.parametrize("index", range(15))
 def test_allocation_failure_returns_oom_and_launches_nothing(index):
     calls = _calls()
     name, fn, make_out = calls[index]
