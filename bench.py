@@ -321,7 +321,7 @@ def run_ours(args, world, rank, device):
             w = dataclasses.replace(w, batch=args.cplx_batch)
         xp = make_inputs(w.batch, w.dim, w.L, w.N, w.dtype, device=device, seed=1234 + args.workload,
                          has_z=w.has_z, has_D=w.has_D, with_dy=True)
-        res = run_dtproj(w, xp, device, steps=args.steps)
+        res = run_dtproj(w, xp, device, steps=args.steps, pair=args.step == "pair")
         return {"note": "--only dtproj: a profiling run, not a benchmark result", "dt_projection": res}
     x = make_inputs(w.batch, w.dim, w.L, w.N, w.dtype, device=device,
                     seed=shard_seed(1234 + args.workload, rank), has_z=w.has_z,
@@ -504,7 +504,8 @@ def run_ours(args, world, rank, device):
         result["conv_prologue"] = run_conv(w, x, device, peaks, steps=args.conv_steps,
                                            pair=args.step == "pair")
     if not args.only and not args.no_dtproj:
-        result["dt_projection"] = run_dtproj(w, x, device, steps=args.conv_steps)
+        result["dt_projection"] = run_dtproj(w, x, device, steps=args.conv_steps,
+                                             pair=args.step == "pair")
     if not args.only and not args.no_cplx:
         result["complex_A"] = run_cplx(w, device, peaks, steps=3, pair=args.step == "pair")
     if args.only:
@@ -667,12 +668,13 @@ def run_conv(w, x, device, peaks, steps=10, pair=True):
             "shape": f"x in place of u, batch {w.batch} x dim {w.dim} x L {w.L}, N {w.N}"}
 
 
-def run_dtproj(w, x, device, steps=10):
+def run_dtproj(w, x, device, steps=10, pair=True):
     """The same workload with the low-rank Delta projection of rank
-    ceil(d_model / 16) = ceil(dim / 32): mamba_dtproj_scan_fwd / _bwd take
-    dt_low (batch, R, L) and W_dt (dim, R) in place of delta.  Times each call
-    with CUDA events; the projection's own share is the difference to the
-    plain calls' times measured alongside."""
+    ceil(d_model / 16) = ceil(dim / 32): the training pair
+    mamba_dtproj_scan_fwd_save / _bwd_saved (pair=False: mamba_dtproj_scan_fwd
+    / _bwd) takes dt_low (batch, R, L) and W_dt (dim, R) in place of delta.
+    Times each call with CUDA events; the projection's own share is the
+    difference to the plain scan's calls of the same kind, timed alongside."""
     from selective_state_space_21_b200 import scan
     from selective_state_space_21_b200.inputs import make_dtproj_params
 
@@ -685,23 +687,43 @@ def run_dtproj(w, x, device, steps=10):
     dW = torch.empty(w.dim, R, **f32)
     dA, dD, db = torch.empty(w.dim, w.N, **f32), torch.empty(w.dim, **f32), torch.empty(w.dim, **f32)
 
+    def buf(n):
+        return torch.empty(n, device=device, dtype=torch.uint8) if n else None
+
+    psaved = buf(scan.dtproj_saved_bytes(w.batch, w.dim, w.L, w.N, R, w.dtype)) if pair else None
+    ssaved = buf(scan.saved_bytes(w.batch, w.dim, w.L, w.N, w.dtype)) if pair else None
+
     def fwd():
-        scan.mamba_dtproj_scan_fwd(x["u"], pp["dt_low"], pp["W_dt"], x["delta_bias"], x["A"],
-                                   x["B"], x["C"], x["D"], x["z"], y, None)
+        args = (x["u"], pp["dt_low"], pp["W_dt"], x["delta_bias"], x["A"], x["B"], x["C"], x["D"],
+                x["z"], y, None)
+        if pair:
+            scan.mamba_dtproj_scan_fwd_save(*args, psaved)
+        else:
+            scan.mamba_dtproj_scan_fwd(*args)
 
     def bwd():
-        scan.mamba_dtproj_scan_bwd(x["u"], pp["dt_low"], pp["W_dt"], x["delta_bias"], x["A"],
-                                   x["B"], x["C"], x["D"], x["z"], x["dy"], g["u"], ddl, dW, dA,
-                                   g["B"], g["C"], dD, g["z"], db)
+        args = (x["u"], pp["dt_low"], pp["W_dt"], x["delta_bias"], x["A"], x["B"], x["C"], x["D"],
+                x["z"], x["dy"], g["u"], ddl, dW, dA, g["B"], g["C"], dD, g["z"], db)
+        if pair:
+            scan.mamba_dtproj_scan_bwd_saved(*args, psaved)
+        else:
+            scan.mamba_dtproj_scan_bwd(*args)
 
     def fwd_plain():
-        scan.mamba_scan_fwd(x["u"], x["delta"], x["delta_bias"], x["A"], x["B"], x["C"], x["D"],
-                            x["z"], y, None)
+        args = (x["u"], x["delta"], x["delta_bias"], x["A"], x["B"], x["C"], x["D"], x["z"], y,
+                None)
+        if pair:
+            scan.mamba_scan_fwd_save(*args, ssaved)
+        else:
+            scan.mamba_scan_fwd(*args)
 
     def bwd_plain():
-        scan.mamba_scan_bwd(x["u"], x["delta"], x["delta_bias"], x["A"], x["B"], x["C"], x["D"],
-                            x["z"], x["dy"], g["u"], g["delta"], dA, g["B"], g["C"], dD, g["z"],
-                            db)
+        args = (x["u"], x["delta"], x["delta_bias"], x["A"], x["B"], x["C"], x["D"], x["z"],
+                x["dy"], g["u"], g["delta"], dA, g["B"], g["C"], dD, g["z"], db)
+        if pair:
+            scan.mamba_scan_bwd_saved(*args, ssaved)
+        else:
+            scan.mamba_scan_bwd(*args)
 
     def timed(fns):
         for _ in range(3):
@@ -722,11 +744,16 @@ def run_dtproj(w, x, device, steps=10):
     fms, bms, fpl, bpl = timed([fwd, bwd, fwd_plain, bwd_plain])
     if scan.mamba_scan_stream_status() != 0:
         raise RuntimeError("device error in the projection run")
+    calls = ("mamba_dtproj_scan_fwd_save + mamba_dtproj_scan_bwd_saved "
+             "(plain: mamba_scan_fwd_save + mamba_scan_bwd_saved)" if pair
+             else "mamba_dtproj_scan_fwd + mamba_dtproj_scan_bwd "
+                  "(plain: mamba_scan_fwd + mamba_scan_bwd)")
     return {"rank": R, "fwd_ms": round(fms, 4), "bwd_ms": round(bms, 4),
             "plain_fwd_ms": round(fpl, 4), "plain_bwd_ms": round(bpl, 4),
             "projection_fwd_ms": round(fms - fpl, 4), "projection_bwd_ms": round(bms - bpl, 4),
             "fwd_tc_per_s": w.token_channels / (fms * 1e-3),
             "bwd_tc_per_s": w.token_channels / (bms * 1e-3), "steps": steps,
+            "saved_bytes": psaved.numel() if psaved is not None else 0, "calls": calls,
             "timing": "median of per-call CUDA events",
             "shape": f"dt_low (batch {w.batch}, R {R}, L {w.L}), W_dt ({w.dim}, {R})"}
 

@@ -191,8 +191,9 @@ MAMBA_SCAN_API mamba_status_t mamba_scan_bwd_ex(const void *u, const void *delta
  * the gradients agree with mamba_scan_bwd_ex to rounding (bit for bit where
  * the compiler forms both alike; the recomputing backward's own forward pass
  * takes the automatic chunking whatever the options).  The convolution
- * prologue has the pair too (mamba_conv_scan_fwd_save and friends); the
- * fused projection and complex A do not.
+ * prologue, the fused Delta projection and complex A have the pair too
+ * (mamba_conv_scan_fwd_save, mamba_dtproj_scan_fwd_save,
+ * mamba_cplx_scan_fwd_save and their companions).
  */
 MAMBA_SCAN_API mamba_status_t mamba_scan_saved_bytes(int64_t batch, int64_t dim, int64_t L, int64_t N,
                                                      mamba_dtype_t dtype,
@@ -352,6 +353,38 @@ MAMBA_SCAN_API mamba_status_t mamba_dtproj_scan_bwd(
     void *du, void *d_dt_low, float *dW_dt, float *dA, void *dB, void *dC, float *dD, void *dz,
     float *ddelta_bias, int64_t batch, int64_t dim, int64_t L, int64_t N, mamba_dtype_t dtype,
     const mamba_scan_options_t *options, mamba_stream_t stream);
+
+/*
+ * The training pair with the low-rank Delta projection: as
+ * mamba_scan_saved_bytes, mamba_scan_fwd_save and mamba_scan_bwd_saved, for
+ * mamba_dtproj_scan_fwd and mamba_dtproj_scan_bwd (same arguments; dt_low,
+ * W_dt and R must also be those of the forward).  Only the fused kernels
+ * (bf16, R <= 192, L a multiple of 8, no MAMBA_PATH_REFERENCE) store or read
+ * states, and only on shapes whose backward carries its adjoint across the
+ * sequence in one pass: elsewhere mamba_dtproj_scan_saved_bytes gives 0 and
+ * the pair behaves as the plain calls.  Where it gives more, the saving
+ * forward refuses (MAMBA_ERR_INVALID_ARG, nothing enqueued) a call that the
+ * fused kernels cannot take, e.g. a dt_low that is not 16-byte aligned.
+ */
+MAMBA_SCAN_API mamba_status_t mamba_dtproj_scan_saved_bytes(int64_t batch, int64_t dim, int64_t L,
+                                                            int64_t N, int64_t R,
+                                                            mamba_dtype_t dtype,
+                                                            const mamba_scan_options_t *options,
+                                                            uint64_t *bytes);
+
+MAMBA_SCAN_API mamba_status_t mamba_dtproj_scan_fwd_save(
+    const void *u, const void *dt_low, const void *W_dt, int64_t R, const float *delta_bias,
+    const float *A, const void *B, const void *C, const float *D, const void *z, void *y,
+    float *last_state, int64_t batch, int64_t dim, int64_t L, int64_t N, mamba_dtype_t dtype,
+    const mamba_scan_options_t *options, void *saved, uint64_t saved_bytes, mamba_stream_t stream);
+
+MAMBA_SCAN_API mamba_status_t mamba_dtproj_scan_bwd_saved(
+    const void *u, const void *dt_low, const void *W_dt, int64_t R, const float *delta_bias,
+    const float *A, const void *B, const void *C, const float *D, const void *z, const void *dy,
+    void *du, void *d_dt_low, float *dW_dt, float *dA, void *dB, void *dC, float *dD, void *dz,
+    float *ddelta_bias, int64_t batch, int64_t dim, int64_t L, int64_t N, mamba_dtype_t dtype,
+    const mamba_scan_options_t *options, const void *saved, uint64_t saved_bytes,
+    mamba_stream_t stream);
 
 /*
  * Forward with a complex-valued diagonal A ("Mamba: Linear-Time Sequence

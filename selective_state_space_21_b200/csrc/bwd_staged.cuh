@@ -1258,8 +1258,32 @@ inline int proj_max_rank() {
   return r;
 }
 
-// With `saved` (not with PROJ), the checkpoints, range flags and (three-phase)
-// h_in and sums of Delta come from
+// The backward's chunking of its adjoint carry, as staged_backward decides it
+// (for a caller that must know it without launching anything).
+template <typename T, int NM, bool CONV = false, bool PROJ = false>
+inline mamba_status_t staged_backward_plan(int64_t batch, int64_t dim, int64_t L, const StagedOptions &o,
+                                           int R, StagedPlan *pl) {
+  using Lay = BwdLayout<T, NM, !PROJ>;
+  int smem = Lay::ALLOC;
+  if (PROJ) {
+    const int Rp = (R + 15) / 16 * 16;
+    if (R < 1 || Rp > proj_max_rank<T, NM>()) return MAMBA_ERR_UNSUPPORTED;
+    smem = proj_bwd_smem_bytes<T, NM>(Rp);
+  }
+  auto kern = bwd_staged_kernel<T, NM, CONV, PROJ>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return MAMBA_ERR_CUDA;
+  int bps = 0;
+  if (resident_ctas(kern, smem, PROJ ? int(kProjTmemCols) : Lay::TMEM_COLS, &bps) != cudaSuccess)
+    return MAMBA_ERR_CUDA;
+  const int slots = device_sm_count() * std::max(1, bps);
+  const int64_t G = batch * ceil_div(dim, kSThreads);
+  *pl = plan_staged(G, L, slots, o, 256);
+  return MAMBA_OK;
+}
+
+// With `saved`, the checkpoints, range flags and (three-phase) h_in and sums
+// of Delta come from
 // a saving forward of the same inputs and options, laid out as saved_layout
 // gives it, and the checkpoint pass does not run.
 template <typename T, int NM, bool CONV = false, bool PROJ = false>
@@ -1267,8 +1291,7 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
                                mamba_status_t (*launched)(), const unsigned char *saved = nullptr) {
   SavedLayout sl;
   if (saved) {
-    if constexpr (PROJ) return MAMBA_ERR_UNSUPPORTED;
-    const mamba_status_t ls = saved_layout<T, NM, CONV>(a.batch, a.dim, a.L, o, &sl);
+    const mamba_status_t ls = saved_layout<T, NM, CONV, PROJ>(a.batch, a.dim, a.L, o, &sl, a.R);
     if (ls != MAMBA_OK) return ls;
   }
   using Lay = BwdLayout<T, NM, !PROJ>;
@@ -1310,6 +1333,9 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
   StagedPlan pl = plan_staged(G, a.L, slots, o, 256);
   const bool par = pl.kind == KIND_PAR;
   if (G * pl.K > (int64_t(1) << 30)) return MAMBA_ERR_UNSUPPORTED;
+  // (the fused projection's three-phase adjoint carry reads delta from the
+  // checkpoint pass, which saved states replace: not taken from saved states)
+  if (PROJ && saved && par) return MAMBA_ERR_UNSUPPORTED;
   const int64_t n16 = ceil_div(a.L, kBTT);
 
   // workspace: [ints][ckpt][carry][part_bc][part_A][part_D][part_bias]

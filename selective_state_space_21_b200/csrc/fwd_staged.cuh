@@ -1340,13 +1340,19 @@ struct SavedLayout {
   int64_t n_ckpt = 0, n_flags = 0, n_cum = 0, n_hin = 0;
 };
 
-template <typename T, int NM, bool CONV = false>
+template <typename T, int NM, bool CONV = false, bool PROJ = false>
 inline mamba_status_t saved_layout(int64_t batch, int64_t dim, int64_t L, const StagedOptions &o,
-                                   SavedLayout *out) {
+                                   SavedLayout *out, int R = 0) {
   SavedLayout sl;
   int sms = 0, slots = 0;
-  const mamba_status_t st = staged_forward_plan<T, NM, CONV>(batch, dim, L, o, StagedLayout<T, NM>::ALLOC,
-                                                             &sl.pl, &sl.G, &sms, &slots);
+  int smem = StagedLayout<T, NM>::ALLOC;
+  if constexpr (PROJ) {  // the fused projection's stages (as StagedForward::prepare sizes them)
+    const int Rp = (R + 15) / 16 * 16;
+    if (R < 1 || Rp > kProjMaxRp) return MAMBA_ERR_UNSUPPORTED;
+    smem = proj_smem_bytes<T, NM>(Rp, proj_smem_bytes<T, NM>(Rp, 3) <= kTwoPerSmBytes ? 3 : 2);
+  }
+  const mamba_status_t st =
+      staged_forward_plan<T, NM, CONV, PROJ>(batch, dim, L, o, smem, &sl.pl, &sl.G, &sms, &slots);
   if (st != MAMBA_OK) return st;
   auto up = [](size_t b) { return (b + 255) / 256 * 256; };
   const int64_t n16 = ceil_div(L, kCkptEvery);
@@ -1355,7 +1361,7 @@ inline mamba_status_t saved_layout(int64_t batch, int64_t dim, int64_t L, const 
   sl.ckpt = 0;
   sl.flags = up(size_t(sl.n_ckpt) * 4);
   sl.bytes = sl.flags + up(size_t(sl.n_flags));
-  if (sl.pl.kind != KIND_SEQ && sizeof(T) == 2) {
+  if (sl.pl.kind != KIND_SEQ && sizeof(T) == 2 && !PROJ) {
     sl.n_cum = sl.G * n16 * kSThreads;
     sl.n_hin = sl.G * sl.pl.K * NM * kSThreads;
     sl.cum = sl.bytes;
@@ -1463,7 +1469,7 @@ struct StagedForward {
     const size_t gk = size_t(G) * size_t(pl.K);
     if (pl.kind == KIND_SEQ) {
       bytes += size_t(G) * NM * kSThreads * 4;
-    } else if (save && sizeof(T) == 2) {  // agg_S, agg_h and the running sums (h_in is saved)
+    } else if (save && sizeof(T) == 2 && !PROJ) {  // agg_S, agg_h and the running sums (h_in is saved)
       bytes += gk * kSThreads * 8 + gk * NM * kSThreads * 4 +
                size_t(G) * size_t(ceil_div(a.L, kCorrBlock)) * kSThreads * 4;
     } else {
@@ -1496,7 +1502,7 @@ struct StagedForward {
 
   // The saving forward: SEQ_SAVE; for 16-bit I/O LOC_SAVE + scan +
   // fwd_correct_kernel (with h_in and the checkpoints' sums of Delta in the
-  // saved buffer); for fp32 AGG + scan + PAR_SAVE.
+  // saved buffer); for fp32 and the fused projection AGG + scan + PAR_SAVE.
   mamba_status_t run_save(unsigned char *ws, cudaStream_t s, mamba_status_t (*launched)()) {
     int *counters = reinterpret_cast<int *>(ws);
     const size_t gk = size_t(sa.G) * size_t(pl.K);
@@ -1513,7 +1519,7 @@ struct StagedForward {
                                                       s, smem);
       return launched();
     }
-    if constexpr (sizeof(T) != 2) {
+    if constexpr (sizeof(T) != 2 || PROJ) {
       int bps_agg = 0;
       if (prepare_kernel<T, NM, KIND_AGG, CONV, PROJ>(&bps_agg, smem) != cudaSuccess ||
           prepare_kernel<T, NM, KIND_PAR_SAVE, CONV, PROJ>(&bps, smem) != cudaSuccess)
@@ -1667,8 +1673,8 @@ struct StagedForward {
 // MAMBA_ERR_UNSUPPORTED (nothing enqueued) if the driver rejects a tensor map,
 // MAMBA_ERR_OUT_OF_MEMORY (nothing enqueued) if the workspace cannot be had.
 // CONV selects the kernels with the convolution prologue (a.conv_w set).
-// With `save` (not with PROJ), the forward also stores what the backward
-// would recompute, laid out as saved_layout gives it.
+// With `save`, the forward also stores what the backward would recompute,
+// laid out as saved_layout gives it.
 template <typename T, int NM, bool CONV = false, bool PROJ = false>
 mamba_status_t staged_forward(const FwdArgs &a, const StagedOptions &o, cudaStream_t s,
                               mamba_status_t (*launched)(), float *ckpt = nullptr,
@@ -1676,8 +1682,7 @@ mamba_status_t staged_forward(const FwdArgs &a, const StagedOptions &o, cudaStre
   StagedForward<T, NM, CONV, PROJ> sf;
   SavedLayout lay;
   if (save) {
-    if constexpr (PROJ) return MAMBA_ERR_UNSUPPORTED;  // the fused projection saves nothing
-    const mamba_status_t ls = saved_layout<T, NM, CONV>(a.batch, a.dim, a.L, o, &lay);
+    const mamba_status_t ls = saved_layout<T, NM, CONV, PROJ>(a.batch, a.dim, a.L, o, &lay, a.R);
     if (ls != MAMBA_OK) return ls;
     sf.save = &lay;
     sf.save_buf = save;

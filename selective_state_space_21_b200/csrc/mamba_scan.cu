@@ -439,16 +439,49 @@ bool proj_fused_ok(const FwdArgs &a, mamba_dtype_t dtype, const StagedOptions &s
   return a.R >= 1 && Rp <= proj_max_rank<__nv_bfloat16, 16>();
 }
 
-mamba_status_t proj_fused_dispatch(const FwdArgs &a, const StagedOptions &o, cudaStream_t s) {
-  if (a.N <= 4) return staged_forward<__nv_bfloat16, 4, false, true>(a, o, s, &launch_status);
-  if (a.N <= 8) return staged_forward<__nv_bfloat16, 8, false, true>(a, o, s, &launch_status);
-  return staged_forward<__nv_bfloat16, 16, false, true>(a, o, s, &launch_status);
+mamba_status_t proj_fused_dispatch(const FwdArgs &a, const StagedOptions &o, cudaStream_t s,
+                                   unsigned char *save = nullptr) {
+  if (a.N <= 4) return staged_forward<__nv_bfloat16, 4, false, true>(a, o, s, &launch_status, nullptr, save);
+  if (a.N <= 8) return staged_forward<__nv_bfloat16, 8, false, true>(a, o, s, &launch_status, nullptr, save);
+  return staged_forward<__nv_bfloat16, 16, false, true>(a, o, s, &launch_status, nullptr, save);
 }
 
-mamba_status_t proj_fused_bwd_dispatch(const BwdArgs &a, const StagedOptions &o, cudaStream_t s) {
-  if (a.N <= 4) return staged_backward<__nv_bfloat16, 4, false, true>(a, o, s, &launch_status);
-  if (a.N <= 8) return staged_backward<__nv_bfloat16, 8, false, true>(a, o, s, &launch_status);
-  return staged_backward<__nv_bfloat16, 16, false, true>(a, o, s, &launch_status);
+mamba_status_t proj_fused_bwd_dispatch(const BwdArgs &a, const StagedOptions &o, cudaStream_t s,
+                                       const unsigned char *saved = nullptr) {
+  if (a.N <= 4) return staged_backward<__nv_bfloat16, 4, false, true>(a, o, s, &launch_status, saved);
+  if (a.N <= 8) return staged_backward<__nv_bfloat16, 8, false, true>(a, o, s, &launch_status, saved);
+  return staged_backward<__nv_bfloat16, 16, false, true>(a, o, s, &launch_status, saved);
+}
+
+// Bytes the fused projection's saving forward stores: 0 unless the fused
+// kernels take the shape and the backward hands its adjoint on in sequence
+// (its three-phase carry reads delta from the checkpoint pass).
+template <int NM>
+mamba_status_t dtproj_saved_nm(int64_t batch, int64_t dim, int64_t L, int64_t R, const StagedOptions &so,
+                               uint64_t *bytes) {
+  StagedPlan bpl;
+  mamba_status_t st = staged_backward_plan<__nv_bfloat16, NM, false, true>(batch, dim, L, so, int(R), &bpl);
+  if (st == MAMBA_ERR_UNSUPPORTED) return MAMBA_OK;
+  if (st != MAMBA_OK) return st;
+  if (bpl.kind != KIND_SEQ) return MAMBA_OK;
+  SavedLayout sl;
+  st = saved_layout<__nv_bfloat16, NM, false, true>(batch, dim, L, so, &sl, int(R));
+  if (st == MAMBA_ERR_UNSUPPORTED) return MAMBA_OK;
+  if (st != MAMBA_OK) return st;
+  *bytes = sl.bytes;
+  return MAMBA_OK;
+}
+
+mamba_status_t dtproj_saved_bytes_for(int64_t batch, int64_t dim, int64_t L, int64_t N, int64_t R,
+                                      mamba_dtype_t dtype, const StagedOptions &so, uint64_t *bytes) {
+  *bytes = 0;
+  if (batch == 0 || dim == 0 || L == 0 || dtype != MAMBA_BF16 || so.path == MAMBA_PATH_REFERENCE ||
+      !staged_shape_ok(L, dim, N, 2) || L % 8 != 0)
+    return MAMBA_OK;
+  if (R < 1 || (R + 15) / 16 * 16 > proj_max_rank<__nv_bfloat16, 16>()) return MAMBA_OK;
+  if (N <= 4) return dtproj_saved_nm<4>(batch, dim, L, R, so, bytes);
+  if (N <= 8) return dtproj_saved_nm<8>(batch, dim, L, R, so, bytes);
+  return dtproj_saved_nm<16>(batch, dim, L, R, so, bytes);
 }
 
 // How the projection's gradient products split dW's contraction over the
@@ -1170,12 +1203,13 @@ mamba_status_t mamba_conv_scan_bwd_saved(const void *x, const float *conv_w, con
 
 // ------------------------------------------- low-rank Delta projection
 
-mamba_status_t mamba_dtproj_scan_fwd(const void *u, const void *dt_low, const void *W_dt,
-                                     int64_t R, const float *delta_bias, const float *A,
-                                     const void *B, const void *C, const float *D, const void *z,
-                                     void *y, float *last_state, int64_t batch, int64_t dim,
-                                     int64_t L, int64_t N, mamba_dtype_t dtype,
-                                     const mamba_scan_options_t *options, mamba_stream_t stream) {
+static mamba_status_t dtproj_fwd_entry(const void *u, const void *dt_low, const void *W_dt,
+                                       int64_t R, const float *delta_bias, const float *A,
+                                       const void *B, const void *C, const float *D, const void *z,
+                                       void *y, float *last_state, int64_t batch, int64_t dim,
+                                       int64_t L, int64_t N, mamba_dtype_t dtype,
+                                       const mamba_scan_options_t *options, mamba_stream_t stream,
+                                       bool saving, void *saved, uint64_t saved_bytes) {
   mamba_status_t st = check_shape(batch, dim, L, N, dtype);
   if (st != MAMBA_OK) return st;
   if ((st = check_options(options)) != MAMBA_OK) return st;
@@ -1200,6 +1234,13 @@ mamba_status_t mamba_dtproj_scan_fwd(const void *u, const void *dt_low, const vo
   ck.buf(delta_bias, size_t(dim) * 4, 4, false, false);
   ck.buf(y, nbdl * es, es, true, true);
   ck.buf(last_state, size_t(batch) * dim * N * 4, 4, false, true);
+  uint64_t need = 0;
+  if (saving) {  // what this forward stores for its backward (0: nothing)
+    if ((st = dtproj_saved_bytes_for(batch, dim, L, N, R, dtype, staged_options(options), &need)) != MAMBA_OK)
+      return st;
+    if (need > saved_bytes) return MAMBA_ERR_INVALID_ARG;
+    ck.buf(saved, need, 16, true, true);
+  }
   if (ck.st != MAMBA_OK) return ck.st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (batch == 0 || dim == 0) return MAMBA_OK;
@@ -1214,6 +1255,10 @@ mamba_status_t mamba_dtproj_scan_fwd(const void *u, const void *dt_low, const vo
   a.batch = batch; a.dim = dim; a.L = L; a.N = (int)N;
   a.dt_low = dt_low; a.W_dt = W_dt; a.R = (int)R;
   const StagedOptions so = staged_options(options);
+  if (need) {  // a saving forward: the fused kernels, no other path
+    if (!proj_fused_ok(a, dtype, so)) return MAMBA_ERR_INVALID_ARG;
+    return proj_fused_dispatch(a, so, s, static_cast<unsigned char *>(saved));
+  }
   // bf16 on the staged kernels: delta formed on the tensor cores inside the scan
   if (proj_fused_ok(a, dtype, so)) {
     st = proj_fused_dispatch(a, so, s);
@@ -1240,14 +1285,48 @@ mamba_status_t mamba_dtproj_scan_fwd(const void *u, const void *dt_low, const vo
   return st;
 }
 
-mamba_status_t mamba_dtproj_scan_bwd(const void *u, const void *dt_low, const void *W_dt,
+mamba_status_t mamba_dtproj_scan_fwd(const void *u, const void *dt_low, const void *W_dt,
                                      int64_t R, const float *delta_bias, const float *A,
                                      const void *B, const void *C, const float *D, const void *z,
-                                     const void *dy, void *du, void *d_dt_low, float *dW_dt,
-                                     float *dA, void *dB, void *dC, float *dD, void *dz,
-                                     float *ddelta_bias, int64_t batch, int64_t dim, int64_t L,
-                                     int64_t N, mamba_dtype_t dtype,
+                                     void *y, float *last_state, int64_t batch, int64_t dim,
+                                     int64_t L, int64_t N, mamba_dtype_t dtype,
                                      const mamba_scan_options_t *options, mamba_stream_t stream) {
+  return dtproj_fwd_entry(u, dt_low, W_dt, R, delta_bias, A, B, C, D, z, y, last_state, batch, dim, L,
+                          N, dtype, options, stream, false, nullptr, 0);
+}
+
+mamba_status_t mamba_dtproj_scan_saved_bytes(int64_t batch, int64_t dim, int64_t L, int64_t N,
+                                             int64_t R, mamba_dtype_t dtype,
+                                             const mamba_scan_options_t *options, uint64_t *bytes) {
+  if (!bytes) return MAMBA_ERR_INVALID_ARG;
+  *bytes = 0;
+  mamba_status_t st = check_shape(batch, dim, L, N, dtype);
+  if (st != MAMBA_OK) return st;
+  if ((st = check_options(options)) != MAMBA_OK) return st;
+  if (R < 1 || R > (int64_t(1) << 20)) return MAMBA_ERR_INVALID_ARG;
+  return dtproj_saved_bytes_for(batch, dim, L, N, R, dtype, staged_options(options), bytes);
+}
+
+mamba_status_t mamba_dtproj_scan_fwd_save(const void *u, const void *dt_low, const void *W_dt,
+                                          int64_t R, const float *delta_bias, const float *A,
+                                          const void *B, const void *C, const float *D,
+                                          const void *z, void *y, float *last_state, int64_t batch,
+                                          int64_t dim, int64_t L, int64_t N, mamba_dtype_t dtype,
+                                          const mamba_scan_options_t *options, void *saved,
+                                          uint64_t saved_bytes, mamba_stream_t stream) {
+  return dtproj_fwd_entry(u, dt_low, W_dt, R, delta_bias, A, B, C, D, z, y, last_state, batch, dim, L,
+                          N, dtype, options, stream, true, saved, saved_bytes);
+}
+
+static mamba_status_t dtproj_bwd_entry(const void *u, const void *dt_low, const void *W_dt,
+                                       int64_t R, const float *delta_bias, const float *A,
+                                       const void *B, const void *C, const float *D, const void *z,
+                                       const void *dy, void *du, void *d_dt_low, float *dW_dt,
+                                       float *dA, void *dB, void *dC, float *dD, void *dz,
+                                       float *ddelta_bias, int64_t batch, int64_t dim, int64_t L,
+                                       int64_t N, mamba_dtype_t dtype,
+                                       const mamba_scan_options_t *options, mamba_stream_t stream,
+                                       bool saving, const void *saved, uint64_t saved_bytes) {
   mamba_status_t st = check_shape(batch, dim, L, N, dtype);
   if (st != MAMBA_OK) return st;
   if ((st = check_options(options)) != MAMBA_OK) return st;
@@ -1283,6 +1362,13 @@ mamba_status_t mamba_dtproj_scan_bwd(const void *u, const void *dt_low, const vo
   ck.buf(dA, size_t(dim) * N * 4, 4, true, true);
   ck.buf(dD, size_t(dim) * 4, 4, false, true);
   ck.buf(ddelta_bias, size_t(dim) * 4, 4, false, true);
+  uint64_t need = 0;
+  if (saving) {  // what the saving forward stored (0: nothing; recompute)
+    if ((st = dtproj_saved_bytes_for(batch, dim, L, N, R, dtype, staged_options(options), &need)) != MAMBA_OK)
+      return st;
+    if (need > saved_bytes) return MAMBA_ERR_INVALID_ARG;
+    ck.buf(saved, need, 16, true, false);
+  }
   if (ck.st != MAMBA_OK) return ck.st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (dim == 0) return MAMBA_OK;
@@ -1307,6 +1393,7 @@ mamba_status_t mamba_dtproj_scan_bwd(const void *u, const void *dt_low, const vo
   fa.D = D; fa.y = nullptr; fa.last_state = nullptr; fa.batch = batch; fa.dim = dim; fa.L = L;
   fa.N = (int)N; fa.dt_low = dt_low; fa.W_dt = W_dt; fa.R = (int)R;
   const bool fused = proj_fused_ok(fa, dtype, so) && staged_bwd_supported(a, es);
+  if (need && !fused) return MAMBA_ERR_INVALID_ARG;  // saved states: the fused kernels only
   const ProjGradPlan gp = proj_grads_plan(W_dt, dt_low, batch, dim, L, R, dtype);
   // workspace: the gradient products' partial sums, ddelta (the scan
   // backward's gradient of delta, in the I/O type), then (unfused) delta
@@ -1321,7 +1408,11 @@ mamba_status_t mamba_dtproj_scan_bwd(const void *u, const void *dt_low, const vo
   void *ddelta = ws + gp.part_bytes, *delta = fused ? nullptr : ws + gp.part_bytes + half;
   a.ddelta = ddelta;
   st = MAMBA_ERR_UNSUPPORTED;
-  if (fused) st = proj_fused_bwd_dispatch(a, so, s);
+  if (fused) st = proj_fused_bwd_dispatch(a, so, s, need ? static_cast<const unsigned char *>(saved) : nullptr);
+  if (need && st != MAMBA_OK) {  // no other path reads saved states
+    ws_free(ws, s);
+    return st;
+  }
   if (st == MAMBA_ERR_UNSUPPORTED && delta == nullptr) {  // the fused kernels declined
     ws_free(ws, s);
     ws = nullptr;
@@ -1352,6 +1443,33 @@ mamba_status_t mamba_dtproj_scan_bwd(const void *u, const void *dt_low, const vo
     st = proj_grads(gp, part, W_dt, dt_low, ddelta, d_dt_low, dW_dt, batch, dim, L, R, dtype, s);
   if (ws_free(ws, s) != cudaSuccess && st == MAMBA_OK) st = MAMBA_ERR_CUDA;
   return st;
+}
+
+mamba_status_t mamba_dtproj_scan_bwd(const void *u, const void *dt_low, const void *W_dt,
+                                     int64_t R, const float *delta_bias, const float *A,
+                                     const void *B, const void *C, const float *D, const void *z,
+                                     const void *dy, void *du, void *d_dt_low, float *dW_dt,
+                                     float *dA, void *dB, void *dC, float *dD, void *dz,
+                                     float *ddelta_bias, int64_t batch, int64_t dim, int64_t L,
+                                     int64_t N, mamba_dtype_t dtype,
+                                     const mamba_scan_options_t *options, mamba_stream_t stream) {
+  return dtproj_bwd_entry(u, dt_low, W_dt, R, delta_bias, A, B, C, D, z, dy, du, d_dt_low, dW_dt, dA, dB,
+                          dC, dD, dz, ddelta_bias, batch, dim, L, N, dtype, options, stream, false, nullptr,
+                          0);
+}
+
+mamba_status_t mamba_dtproj_scan_bwd_saved(const void *u, const void *dt_low, const void *W_dt,
+                                           int64_t R, const float *delta_bias, const float *A,
+                                           const void *B, const void *C, const float *D,
+                                           const void *z, const void *dy, void *du, void *d_dt_low,
+                                           float *dW_dt, float *dA, void *dB, void *dC, float *dD,
+                                           void *dz, float *ddelta_bias, int64_t batch, int64_t dim,
+                                           int64_t L, int64_t N, mamba_dtype_t dtype,
+                                           const mamba_scan_options_t *options, const void *saved,
+                                           uint64_t saved_bytes, mamba_stream_t stream) {
+  return dtproj_bwd_entry(u, dt_low, W_dt, R, delta_bias, A, B, C, D, z, dy, du, d_dt_low, dW_dt, dA, dB,
+                          dC, dD, dz, ddelta_bias, batch, dim, L, N, dtype, options, stream, true, saved,
+                          saved_bytes);
 }
 
 // ------------------------------------------------ complex diagonal A

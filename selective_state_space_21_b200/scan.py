@@ -4,7 +4,8 @@ CPU fallback; a missing library or device raises.
 
 Low-level calls (same names and argument order as ``include/mamba_scan.h``):
 ``mamba_scan_fwd``, ``mamba_scan_bwd``, ``mamba_conv_scan_fwd``,
-``mamba_conv_scan_bwd``, ``mamba_dtproj_scan_fwd``, ``mamba_dtproj_scan_bwd``,
+``mamba_conv_scan_bwd``, ``mamba_dtproj_scan_fwd``, ``mamba_dtproj_scan_bwd``
+(with the training pairs ``*_saved_bytes`` / ``*_fwd_save`` / ``*_bwd_saved``),
 ``mamba_cplx_scan_fwd``, ``mamba_cplx_scan_bwd``, ``mamba_scan_step``,
 ``mamba_scan_fwd_noalloc``,
 ``mamba_scan_stream_status``; decoding plans (``StepPlan``), the workspace
@@ -100,6 +101,14 @@ def load_library():
             lib.mamba_dtproj_scan_fwd.restype = ctypes.c_int
             lib.mamba_dtproj_scan_bwd.argtypes = [vp] * 3 + [i64] + [vp] * 16 + [i64] * 4 + [i32, opt, vp]
             lib.mamba_dtproj_scan_bwd.restype = ctypes.c_int
+            lib.mamba_dtproj_scan_saved_bytes.argtypes = [i64] * 5 + [i32, opt, ctypes.POINTER(u64)]
+            lib.mamba_dtproj_scan_saved_bytes.restype = ctypes.c_int
+            lib.mamba_dtproj_scan_fwd_save.argtypes = (
+                [vp] * 3 + [i64] + [vp] * 8 + [i64] * 4 + [i32, opt, vp, u64, vp])
+            lib.mamba_dtproj_scan_fwd_save.restype = ctypes.c_int
+            lib.mamba_dtproj_scan_bwd_saved.argtypes = (
+                [vp] * 3 + [i64] + [vp] * 16 + [i64] * 4 + [i32, opt, vp, u64, vp])
+            lib.mamba_dtproj_scan_bwd_saved.restype = ctypes.c_int
             lib.mamba_cplx_scan_fwd.argtypes = [vp] * 10 + [i64] * 4 + [i32, vp]
             lib.mamba_cplx_scan_fwd.restype = ctypes.c_int
             lib.mamba_cplx_scan_bwd.argtypes = [vp] * 17 + [i64] * 4 + [i32, vp]
@@ -436,6 +445,21 @@ def mamba_conv_scan_bwd_saved(x, conv_w, conv_b, delta, delta_bias, A, B, C, D, 
            "mamba_conv_scan_bwd_saved")
 
 
+def _dtproj_fwd_args(u, dt_low, W_dt, delta_bias, A, B, C, D, z, y, last_state):
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    R = W_dt.shape[1]
+    dt = u.dtype
+    f32 = torch.float32
+    bdl, bnl = (batch, dim, L), (batch, N, L)
+    return [
+        _ptr(u, dt, bdl, "u"), _ptr(dt_low, dt, (batch, R, L), "dt_low"),
+        _ptr(W_dt, dt, (dim, R), "W_dt"), R, _ptr(delta_bias, f32, (dim,), "delta_bias"),
+        _ptr(A, f32, (dim, N), "A"), _ptr(B, dt, bnl, "B"), _ptr(C, dt, bnl, "C"),
+        _ptr(D, f32, (dim,), "D"), _ptr(z, dt, bdl, "z"), _ptr(y, dt, bdl, "y"),
+        _ptr(last_state, f32, (batch, dim, N), "last_state"), batch, dim, L, N, _dtype_code(dt)]
+
+
 def mamba_dtproj_scan_fwd(u, dt_low, W_dt, delta_bias, A, B, C, D, z, y, last_state, *,
                           path="auto", chunk_len=0, carry="auto", wait_timeout_us=0,
                           test_hook=0, stream=None):
@@ -443,36 +467,49 @@ def mamba_dtproj_scan_fwd(u, dt_low, W_dt, delta_bias, A, B, C, D, z, y, last_st
     W_dt . dt_low per batch row (a tensor-core GEMM), then the scan.  dt_low
     (batch, R, L) and W_dt (dim, R) in the I/O dtype; the rest as
     ``mamba_scan_fwd``."""
-    batch, dim, L = u.shape
-    N = A.shape[1]
-    R = W_dt.shape[1]
-    dt = u.dtype
-    f32 = torch.float32
-    bdl, bnl = (batch, dim, L), (batch, N, L)
-    args = [
-        _ptr(u, dt, bdl, "u"), _ptr(dt_low, dt, (batch, R, L), "dt_low"),
-        _ptr(W_dt, dt, (dim, R), "W_dt"), R, _ptr(delta_bias, f32, (dim,), "delta_bias"),
-        _ptr(A, f32, (dim, N), "A"), _ptr(B, dt, bnl, "B"), _ptr(C, dt, bnl, "C"),
-        _ptr(D, f32, (dim,), "D"), _ptr(z, dt, bdl, "z"), _ptr(y, dt, bdl, "y"),
-        _ptr(last_state, f32, (batch, dim, N), "last_state"), batch, dim, L, N, _dtype_code(dt)]
+    args = _dtproj_fwd_args(u, dt_low, W_dt, delta_bias, A, B, C, D, z, y, last_state)
     opts = _opts_ptr(path, chunk_len, carry, wait_timeout_us, test_hook)
     _check(load_library().mamba_dtproj_scan_fwd(*args, opts, _stream_handle(stream)),
            "mamba_dtproj_scan_fwd")
 
 
-def mamba_dtproj_scan_bwd(u, dt_low, W_dt, delta_bias, A, B, C, D, z, dy, du, d_dt_low, dW_dt,
-                          dA, dB, dC, dD, dz, ddelta_bias, *, path="auto", chunk_len=0,
-                          wait_timeout_us=0, test_hook=0, stream=None):
-    """Enqueue the backward of sum(dy * y) for ``mamba_dtproj_scan_fwd``:
-    d_dt_low (batch, R, L, I/O dtype) and dW_dt (dim, R, float32) take the
-    place of ddelta."""
+def dtproj_saved_bytes(batch, dim, L, N, R, dtype, *, path="auto", chunk_len=0, carry="auto",
+                       wait_timeout_us=0, test_hook=0) -> int:
+    """``saved_bytes`` for the training pair with the Delta projection (0 where
+    the pair behaves as the plain calls)."""
+    n = ctypes.c_uint64(0)
+    opts = _opts_ptr(path, chunk_len, carry, wait_timeout_us, test_hook)
+    _check(load_library().mamba_dtproj_scan_saved_bytes(batch, dim, L, N, R, _dtype_code(dtype),
+                                                        opts, ctypes.byref(n)),
+           "mamba_dtproj_scan_saved_bytes")
+    return int(n.value)
+
+
+def mamba_dtproj_scan_fwd_save(u, dt_low, W_dt, delta_bias, A, B, C, D, z, y, last_state, saved,
+                               *, path="auto", chunk_len=0, carry="auto", wait_timeout_us=0,
+                               test_hook=0, stream=None):
+    """``mamba_dtproj_scan_fwd`` that also fills ``saved``
+    (``dtproj_saved_bytes`` bytes) for ``mamba_dtproj_scan_bwd_saved``."""
+    batch, dim, L = u.shape
+    need = dtproj_saved_bytes(batch, dim, L, A.shape[1], W_dt.shape[1], u.dtype, path=path,
+                              chunk_len=chunk_len, carry=carry, wait_timeout_us=wait_timeout_us,
+                              test_hook=test_hook)
+    sp, sn = _saved_arg(saved, need)
+    args = _dtproj_fwd_args(u, dt_low, W_dt, delta_bias, A, B, C, D, z, y, last_state)
+    opts = _opts_ptr(path, chunk_len, carry, wait_timeout_us, test_hook)
+    _check(load_library().mamba_dtproj_scan_fwd_save(*args, opts, sp, sn, _stream_handle(stream)),
+           "mamba_dtproj_scan_fwd_save")
+
+
+def _dtproj_bwd_args(u, dt_low, W_dt, delta_bias, A, B, C, D, z, dy, du, d_dt_low, dW_dt, dA, dB,
+                     dC, dD, dz, ddelta_bias):
     batch, dim, L = u.shape
     N = A.shape[1]
     R = W_dt.shape[1]
     dt = u.dtype
     f32 = torch.float32
     bdl, bnl = (batch, dim, L), (batch, N, L)
-    args = [
+    return [
         _ptr(u, dt, bdl, "u"), _ptr(dt_low, dt, (batch, R, L), "dt_low"),
         _ptr(W_dt, dt, (dim, R), "W_dt"), R, _ptr(delta_bias, f32, (dim,), "delta_bias"),
         _ptr(A, f32, (dim, N), "A"), _ptr(B, dt, bnl, "B"), _ptr(C, dt, bnl, "C"),
@@ -482,9 +519,37 @@ def mamba_dtproj_scan_bwd(u, dt_low, W_dt, delta_bias, A, B, C, D, z, dy, du, d_
         _ptr(dB, dt, bnl, "dB"), _ptr(dC, dt, bnl, "dC"), _ptr(dD, f32, (dim,), "dD"),
         _ptr(dz, dt, bdl, "dz"), _ptr(ddelta_bias, f32, (dim,), "ddelta_bias"),
         batch, dim, L, N, _dtype_code(dt)]
+
+
+def mamba_dtproj_scan_bwd(u, dt_low, W_dt, delta_bias, A, B, C, D, z, dy, du, d_dt_low, dW_dt,
+                          dA, dB, dC, dD, dz, ddelta_bias, *, path="auto", chunk_len=0,
+                          wait_timeout_us=0, test_hook=0, stream=None):
+    """Enqueue the backward of sum(dy * y) for ``mamba_dtproj_scan_fwd``:
+    d_dt_low (batch, R, L, I/O dtype) and dW_dt (dim, R, float32) take the
+    place of ddelta."""
+    args = _dtproj_bwd_args(u, dt_low, W_dt, delta_bias, A, B, C, D, z, dy, du, d_dt_low, dW_dt,
+                            dA, dB, dC, dD, dz, ddelta_bias)
     opts = _opts_ptr(path, chunk_len, "auto", wait_timeout_us, test_hook)
     _check(load_library().mamba_dtproj_scan_bwd(*args, opts, _stream_handle(stream)),
            "mamba_dtproj_scan_bwd")
+
+
+def mamba_dtproj_scan_bwd_saved(u, dt_low, W_dt, delta_bias, A, B, C, D, z, dy, du, d_dt_low,
+                                dW_dt, dA, dB, dC, dD, dz, ddelta_bias, saved, *, path="auto",
+                                chunk_len=0, carry="auto", wait_timeout_us=0, test_hook=0,
+                                stream=None):
+    """``mamba_dtproj_scan_bwd`` reading ``saved`` as
+    ``mamba_dtproj_scan_fwd_save`` wrote it (same inputs and options)."""
+    batch, dim, L = u.shape
+    need = dtproj_saved_bytes(batch, dim, L, A.shape[1], W_dt.shape[1], u.dtype, path=path,
+                              chunk_len=chunk_len, carry=carry, wait_timeout_us=wait_timeout_us,
+                              test_hook=test_hook)
+    sp, sn = _saved_arg(saved, need)
+    args = _dtproj_bwd_args(u, dt_low, W_dt, delta_bias, A, B, C, D, z, dy, du, d_dt_low, dW_dt,
+                            dA, dB, dC, dD, dz, ddelta_bias)
+    opts = _opts_ptr(path, chunk_len, carry, wait_timeout_us, test_hook)
+    _check(load_library().mamba_dtproj_scan_bwd_saved(*args, opts, sp, sn, _stream_handle(stream)),
+           "mamba_dtproj_scan_bwd_saved")
 
 
 def _cplx_fwd_args(u, delta, delta_bias, A, B, C, D, z, y, last_state):

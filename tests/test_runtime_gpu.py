@@ -233,10 +233,36 @@ def _calls():
         cx["u"], cx["delta"], cx["delta_bias"], cx["A"], cx["B"], cx["C"], cx["D"], cx["z"],
         cx["dy"], o["du"], o["dd"], o["dA"], o["dB"], o["dC"], o["dD"], o["dz"], o["db"], xsaved),
         lambda: bwd_outs(cx)))
+    # the projection's pair stores states where its backward runs in one
+    # chunk (L <= 256)
+    fs = gc.to_device(make_inputs(2, 200, 256, 16, torch.bfloat16, seed=70, with_dy=True))
+    ps = gc.to_device(make_dtproj_params(2, 200, 256, 8, torch.bfloat16, seed=71))
+    psaved = torch.empty(scan.dtproj_saved_bytes(2, 200, 256, 16, 8, torch.bfloat16),
+                         device="cuda", dtype=torch.uint8)
+    assert psaved.numel() > 0
+    scan.mamba_dtproj_scan_fwd_save(fs["u"], ps["dt_low"], ps["W_dt"], fs["delta_bias"], fs["A"],
+                                    fs["B"], fs["C"], fs["D"], fs["z"], torch.empty_like(fs["u"]),
+                                    None, psaved)
+    torch.cuda.synchronize()
+
+    def dtps_outs():
+        o = bwd_outs(fs)
+        del o["dd"]
+        o["ddl"] = _nan_like(ps["dt_low"])
+        o["dW"] = torch.full((200, 8), float("nan"), **f32)
+        return o
+
+    out.append(("dtproj fwd save", lambda o: scan.mamba_dtproj_scan_fwd_save(
+        fs["u"], ps["dt_low"], ps["W_dt"], fs["delta_bias"], fs["A"], fs["B"], fs["C"], fs["D"],
+        fs["z"], o["y"], o["last"], torch.empty_like(psaved)), lambda: fwd_outs(fs)))
+    out.append(("dtproj bwd saved", lambda o: scan.mamba_dtproj_scan_bwd_saved(
+        fs["u"], ps["dt_low"], ps["W_dt"], fs["delta_bias"], fs["A"], fs["B"], fs["C"], fs["D"],
+        fs["z"], fs["dy"], o["du"], o["ddl"], o["dW"], o["dA"], o["dB"], o["dC"], o["dD"],
+        o["dz"], o["db"], psaved), dtps_outs))
     return out
 
 
-@pytest.mark.parametrize("index", range(15))
+@pytest.mark.parametrize("index", range(17))
 def test_allocation_failure_returns_oom_and_launches_nothing(index):
     calls = _calls()
     name, fn, make_out = calls[index]
