@@ -43,12 +43,17 @@ namespace mscan {
 
 constexpr int kBTT = kCkptEvery;  // time steps per backward tile
 constexpr int kBStages = 2;
+// Tensor memory of the fused projection's backward (kProjTmemCols columns
+// per CTA): W_dt's rows in [0, Rp/2), the two 16-step delta accumulators in
+// [kProjBwdAcc, kProjBwdAcc + 32), the segment states from kProjBwdSub.
+constexpr uint32_t kProjBwdAcc = 96;
+constexpr uint32_t kProjBwdSub = 128;
+constexpr int kProjBwdMaxRp = 2 * int(kProjBwdAcc);
 
 // TSUB: the state before every segment lives in tensor memory (each thread's
 // own lane, NSEG x NM columns): one tcgen05.st / tcgen05.ld of the NM states
-// in place of NM / 2 shared-memory stores / loads.  The fused projection's
-// kernels, whose tensor memory holds W_dt and the delta accumulators, keep
-// the states in shared memory.
+// in place of NM / 2 shared-memory stores / loads.  The kernels take TSUB;
+// the layout without it sizes the rank limit of the fused projection.
 template <typename T, int NM, bool TSUB = false>
 struct BwdLayout {
   static constexpr int RB = kBTT * (int)sizeof(T);  // bytes of one channel row in a tile
@@ -275,14 +280,15 @@ __global__ void __launch_bounds__(kSThreads, 2)
                       const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_dy,
                       const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_C,
                       const BwdStagedArgs p) {
-  constexpr bool kTSub = !PROJ;  // segment states in tensor memory
-  using Lay = BwdLayout<T, NM, kTSub>;
+  using Lay = BwdLayout<T, NM, true>;  // segment states in tensor memory
   constexpr int RB = Lay::RB, BSTR = Lay::BSTR;
   constexpr int NP = NM / 2;
   constexpr int SEG = Lay::SEG;
   using IO = SegIO<T, SEG>;
   static_assert(!PROJ || (std::is_same<T, __nv_bfloat16>::value && !CONV),
                 "the fused projection takes bf16 operands and no convolution prologue");
+  static_assert(!PROJ || Lay::NSEG * NM <= int(kProjTmemCols - kProjBwdSub),
+                "the segment states must fit after the projection's columns");
 
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *sm = smem_raw + ((512u - (smem_u32(smem_raw) & 511u)) & 511u);
@@ -300,7 +306,6 @@ __global__ void __launch_bounds__(kSThreads, 2)
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);  // [2 stages], then 2 MMA barriers
   uint64_t *mma_bar = bars + 2;
   int *q = reinterpret_cast<int *>(sm + OFF_BAR + 8 * 4);  // [0..7] tickets, [8] abort, [12] TMEM
-  float *sub = reinterpret_cast<float *>(sm + OFF_SUB);  // [NSEG][NM][128]
   float *Bs = reinterpret_cast<float *>(sm + OFF_BS);
   float *Cs = reinterpret_cast<float *>(sm + OFF_CS);
   float *red = reinterpret_cast<float *>(sm + OFF_RED);  // [4 warps][kBTT][33] (padded rows)
@@ -340,8 +345,9 @@ __global__ void __launch_bounds__(kSThreads, 2)
   __syncthreads();
   tc_fence_after_sync();
   tbase = uint32_t(q[12]);
-  // (TSUB) this thread's lane: the state before segment s in columns s*NM ..
-  [[maybe_unused]] const uint32_t tsub = tmem_at(tbase, uint32_t(warp) * 32u, 0);
+  // this thread's lane: the state before segment s in columns s*NM .. (after
+  // the projection's columns with PROJ)
+  const uint32_t tsub = tmem_at(tbase, uint32_t(warp) * 32u, PROJ ? kProjBwdSub : 0u);
 
   // Issues (kMmaThread) the projection MMAs of consumed-tile index `ct` into
   // accumulator ct & 1 once the tile's dt_low rows have landed: 16 rows of
@@ -355,7 +361,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
     }
     tc_fence_after_sync();
     const uint32_t dt_addr = smem_u32(sm + stg * SST + Lay::TILE);
-    const uint32_t acc = tbase + kProjAcc + uint32_t(ct & 1) * kBTT;
+    const uint32_t acc = tbase + kProjBwdAcc + uint32_t(ct & 1) * kBTT;
     for (int kk = 0; kk < p.Rp / 16; ++kk) {
       const uint64_t bdesc = smem_desc(dt_addr + uint32_t(kk) * 512u, 16u, 256u, 6u);
       mma_ts(acc, tbase + uint32_t(kk) * 8u, bdesc, kIdesc, kk > 0);
@@ -609,7 +615,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
             q[8] = 1;
           }
           tc_fence_after_sync();
-          dacc = tmem_at(tbase + kProjAcc + uint32_t(ctile & 1) * kBTT, uint32_t(warp) * 32u, 0);
+          dacc = tmem_at(tbase + kProjBwdAcc + uint32_t(ctile & 1) * kBTT, uint32_t(warp) * 32u, 0);
         }
         {
           const T *Braw = reinterpret_cast<const T *>(st + OFF_B);
@@ -700,7 +706,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
         // One tile with the structured (S) or the generic arithmetic.
         auto tile_body = [&](auto stag) {
           constexpr bool S = decltype(stag)::value;
-          // forward over the tile: the state before every segment -> shared memory
+          // forward over the tile: the state before every segment -> tensor memory
           {
             f2 H[NP];
             float h[NM];
@@ -712,8 +718,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
               for (int n = 0; n < NM; ++n) h[n] = h0[n];
             }
             for (int seg = 0; seg < nseg; ++seg) {
-              [[maybe_unused]] float *sp = sub + (seg * NM) * kSThreads + tid;
-              if constexpr (kTSub) {  // one tensor-memory store of the NM states
+              {  // one tensor-memory store of the NM states
                 float hv[NM];
                 if constexpr (S) {
   #pragma unroll
@@ -726,13 +731,6 @@ __global__ void __launch_bounds__(kSThreads, 2)
                   for (int n = 0; n < NM; ++n) hv[n] = h[n];
                 }
                 tmem_st_row<NM>(tsub + uint32_t(seg * NM), hv);
-              } else if constexpr (S) {  // packed pairs of states, one 8-byte store each
-                f2 *sp2 = reinterpret_cast<f2 *>(sub) + (seg * NP) * kSThreads + tid;
-  #pragma unroll
-                for (int i = 0; i < NP; ++i) sp2[i * kSThreads] = H[i];
-              } else {
-  #pragma unroll
-                for (int n = 0; n < NM; ++n) sp[n * kSThreads] = h[n];
               }
               if (seg == nseg - 1) break;  // the last segment is re-run below anyway
               float uv[SEG], dv[SEG];
@@ -754,7 +752,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
             }
           }
 
-          if constexpr (kTSub) tmem_st_wait();  // the segment states, before they are read back
+          tmem_st_wait();  // the segment states, before they are read back
 
           // the next tile's projection MMA, into the other accumulator
           if constexpr (PROJ) {
@@ -770,22 +768,17 @@ __global__ void __launch_bounds__(kSThreads, 2)
             IO::load(sdy, tid, seg, dyv);
             if (has_z) IO::load(sz, tid, seg, zv);
             float du_o[SEG], dd_o[SEG], dz_o[SEG];
-            [[maybe_unused]] const float *sp = sub + (seg * NM) * kSThreads + tid;
 
             if constexpr (S) {
               // states before each step of the segment (the state after a step
               // is recomputed in the reverse step from h_{t-1} and t1)
               f2 Hs[SEG][NP];
-              if constexpr (kTSub) {
+              {
                 float hv[NM];
                 tmem_ld_row<NM>(tsub + uint32_t(seg * NM), hv);
                 tmem_ld_wait();
   #pragma unroll
                 for (int i = 0; i < NP; ++i) Hs[0][i] = pk(hv[2 * i], hv[2 * i + 1]);
-              } else {
-                const f2 *sp2 = reinterpret_cast<const f2 *>(sub) + (seg * NP) * kSThreads + tid;
-  #pragma unroll
-                for (int i = 0; i < NP; ++i) Hs[0][i] = sp2[i * kSThreads];
               }
   #pragma unroll
               for (int i = 0; i + 1 < SEG; ++i) {
@@ -861,13 +854,8 @@ __global__ void __launch_bounds__(kSThreads, 2)
               }
             } else {
               float Hs[SEG][NM];
-              if constexpr (kTSub) {
-                tmem_ld_row<NM>(tsub + uint32_t(seg * NM), Hs[0]);
-                tmem_ld_wait();
-              } else {
-  #pragma unroll
-                for (int n = 0; n < NM; ++n) Hs[0][n] = sp[n * kSThreads];
-              }
+              tmem_ld_row<NM>(tsub + uint32_t(seg * NM), Hs[0]);
+              tmem_ld_wait();
   #pragma unroll
               for (int i = 0; i + 1 < SEG; ++i) {
                 const float *Brow = Bs + (seg * SEG + i) * BSTR;
@@ -1245,16 +1233,17 @@ inline bool staged_bwd_supported(const BwdArgs &a, size_t es) {
 // Rp x 16 dt_low tile in place of delta's).
 template <typename T, int NM>
 inline int proj_bwd_smem_bytes(int Rp) {
-  using Lay = BwdLayout<T, NM>;
+  using Lay = BwdLayout<T, NM, true>;
   return int(kBStages * BwdStage<T, NM>(Rp).bytes) + (Lay::BYTES - Lay::OFF_SUB) + 512;
 }
 
 // Largest R the fused projection takes: its tiles must leave room for two
-// CTAs per SM in both the forward and the backward.
+// CTAs per SM in both the forward and the backward, and W_dt's columns must
+// end before the backward's delta accumulators in tensor memory.
 template <typename T, int NM>
 inline int proj_max_rank() {
   int r = 16;
-  while (r + 16 <= kProjMaxRp && proj_bwd_smem_bytes<T, NM>(r + 16) <= kTwoPerSmBytes) r += 16;
+  while (r + 16 <= kProjBwdMaxRp && proj_bwd_smem_bytes<T, NM>(r + 16) <= kTwoPerSmBytes) r += 16;
   return r;
 }
 
@@ -1263,7 +1252,7 @@ inline int proj_max_rank() {
 template <typename T, int NM, bool CONV = false, bool PROJ = false>
 inline mamba_status_t staged_backward_plan(int64_t batch, int64_t dim, int64_t L, const StagedOptions &o,
                                            int R, StagedPlan *pl) {
-  using Lay = BwdLayout<T, NM, !PROJ>;
+  using Lay = BwdLayout<T, NM, true>;
   int smem = Lay::ALLOC;
   if (PROJ) {
     const int Rp = (R + 15) / 16 * 16;
@@ -1294,7 +1283,7 @@ mamba_status_t staged_backward(const BwdArgs &a, const StagedOptions &o, cudaStr
     const mamba_status_t ls = saved_layout<T, NM, CONV, PROJ>(a.batch, a.dim, a.L, o, &sl, a.R);
     if (ls != MAMBA_OK) return ls;
   }
-  using Lay = BwdLayout<T, NM, !PROJ>;
+  using Lay = BwdLayout<T, NM, true>;
   constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
   const uint64_t L = a.L, dim = a.dim, batch = a.batch, N = a.N;
   const CUtensorMapSwizzle sw = bf16 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B;
