@@ -233,20 +233,6 @@ __device__ __forceinline__ float bfly_rest2(f2 (&v2)[8], int lane) {
   return keep + __shfl_xor_sync(0xffffffffu, send, 1);
 }
 
-// Whether any step of a 16-step tile of the thread's delta, from its fused-
-// projection accumulator in TMEM (lane = channel), lies in [lo, hi].  Every
-// lane of the warp must call it: the TMEM load is warp-collective.
-__device__ __forceinline__ bool tile_delta_in_range(uint32_t dacc, float lo, float hi) {
-  float a[8], b[8];
-  tmem_ld8(dacc, a);
-  tmem_ld8(dacc + 8u, b);
-  tmem_ld_wait();
-  bool in = false;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) in = in || (a[i] >= lo && a[i] <= hi) || (b[i] >= lo && b[i] <= hi);
-  return in;
-}
-
 // Four consecutive x values of a row (16-byte aligned for float, 8-byte for
 // bf16), widened to float.
 __device__ __forceinline__ void load_x4(const float *p, float (&o)[4]) {
@@ -273,7 +259,8 @@ __device__ __forceinline__ void load_x4(const __nv_bfloat16 *p, float (&o)[4]) {
 // PROJ: delta is formed on the tensor cores as in the forward's fused
 // projection (fwd_staged.cuh): the Rp x 16 dt_low tiles come through the
 // pipeline, W_dt's rows for the CTA's channels sit in TMEM, and each thread
-// reads its channel's delta for a segment with tcgen05.ld.
+// reads its channel's 16 values of the tile with one tcgen05.ld into its own
+// slots of shared memory, where both passes over the tile read them.
 template <typename T, int NM, bool CONV = false, bool PROJ = false>
 __global__ void __launch_bounds__(kSThreads, 2)
     bwd_staged_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_d,
@@ -303,6 +290,8 @@ __global__ void __launch_bounds__(kSThreads, 2)
   const uint32_t OFF_CS = OFF_SUB + uint32_t(Lay::OFF_CS - Lay::OFF_SUB);
   const uint32_t OFF_RED = OFF_SUB + uint32_t(Lay::OFF_RED - Lay::OFF_SUB);
   const uint32_t OFF_BAR = OFF_SUB + uint32_t(Lay::OFF_BAR - Lay::OFF_SUB);
+  // (PROJ) the tile's delta, fp32 pairs [segment][thread], each thread's own
+  const uint32_t OFF_DS = (OFF_SUB + uint32_t(Lay::BYTES - Lay::OFF_SUB) + 15u) & ~15u;
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);  // [2 stages], then 2 MMA barriers
   uint64_t *mma_bar = bars + 2;
   int *q = reinterpret_cast<int *>(sm + OFF_BAR + 8 * 4);  // [0..7] tickets, [8] abort, [12] TMEM
@@ -608,14 +597,23 @@ __global__ void __launch_bounds__(kSThreads, 2)
           record_timeout();
           q[8] = 1;
         }
-        [[maybe_unused]] uint32_t dacc = 0;
-        if constexpr (PROJ) {  // this tile's delta: wait for its MMA
+        [[maybe_unused]] bool d_in = false;  // (PROJ) a step of the tile in [d_lo, d_hi]
+        if constexpr (PROJ) {  // this tile's delta: wait for its MMA, then one TMEM load
           if (!mbar_wait_bounded(&mma_bar[ctile & 1], uint32_t(ctile >> 1) & 1u, p.timeout_ns)) {
             record_timeout();
             q[8] = 1;
           }
           tc_fence_after_sync();
-          dacc = tmem_at(tbase + kProjBwdAcc + uint32_t(ctile & 1) * kBTT, uint32_t(warp) * 32u, 0);
+          float dt16[kBTT];  // warp-collective load: every lane takes part
+          tmem_ld16(tmem_at(tbase + kProjBwdAcc + uint32_t(ctile & 1) * kBTT, uint32_t(warp) * 32u, 0), dt16);
+          tmem_ld_wait();
+          float2 *ds = reinterpret_cast<float2 *>(sm + OFF_DS);
+#pragma unroll
+          for (int sg = 0; sg < kBTT / 2; ++sg) ds[sg * kSThreads + tid] = make_float2(dt16[2 * sg], dt16[2 * sg + 1]);
+          if constexpr (kS) {
+#pragma unroll
+            for (int i = 0; i < kBTT; ++i) d_in = d_in || (dt16[i] >= d_lo && dt16[i] <= d_hi);
+          }
         }
         {
           const T *Braw = reinterpret_cast<const T *>(st + OFF_B);
@@ -634,9 +632,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
         }
         bool tile_gen = false;
         if constexpr (kS && PROJ) {  // no step of the tile in the structured range?
-          // (every thread reads its row: the TMEM load is warp-collective)
-          const bool in = tile_delta_in_range(dacc, d_lo, d_hi);
-          tile_gen = !__syncthreads_or(valid && in);
+          tile_gen = !__syncthreads_or(valid && d_in);
         } else {
           __syncthreads();
         }
@@ -649,10 +645,11 @@ __global__ void __launch_bounds__(kSThreads, 2)
 
         // delta of one segment: from the tile, or (PROJ) from TMEM
         auto load_d = [&](int seg, float (&dv)[SEG]) {
-          if constexpr (PROJ) {
+          if constexpr (PROJ) {  // this thread's pair, stored at the tile's start
             static_assert(SEG == 2, "two-step segments in bf16");
-            tmem_ld2(dacc + uint32_t(seg) * SEG, dv);
-            tmem_ld_wait();
+            const float2 v = reinterpret_cast<const float2 *>(sm + OFF_DS)[seg * kSThreads + tid];
+            dv[0] = v.x;
+            dv[1] = v.y;
           } else {
             IO::load(sd, tid, seg, dv);
           }
@@ -1230,11 +1227,12 @@ inline bool staged_bwd_supported(const BwdArgs &a, size_t es) {
 }
 
 // Dynamic shared memory of the fused-projection backward (its stages hold the
-// Rp x 16 dt_low tile in place of delta's).
+// Rp x 16 dt_low tile in place of delta's; the tile's fp32 delta follows).
 template <typename T, int NM>
 inline int proj_bwd_smem_bytes(int Rp) {
   using Lay = BwdLayout<T, NM, true>;
-  return int(kBStages * BwdStage<T, NM>(Rp).bytes) + (Lay::BYTES - Lay::OFF_SUB) + 512;
+  constexpr int kDeltaBytes = kBTT * kSThreads * 4 + 16;  // the tile's delta (and its alignment)
+  return int(kBStages * BwdStage<T, NM>(Rp).bytes) + (Lay::BYTES - Lay::OFF_SUB) + kDeltaBytes + 512;
 }
 
 // Largest R the fused projection takes: its tiles must leave room for two
