@@ -61,3 +61,19 @@ def test_binding_rejects_cpu_tensors():
     with pytest.raises(ValueError):
         scan.mamba_scan_fwd(x, x, None, torch.zeros(2, 4), torch.zeros(1, 4, 8),
                             torch.zeros(1, 4, 8), None, None, torch.zeros_like(x), None)
+
+
+def test_saved_bytes_queries_check_arguments_on_the_host(lib):
+    """The training pairs' size queries refuse a null result pointer and a bad
+    rank before touching a device; the projection's pair stores nothing for
+    fp32 (the fused kernels take bf16 only), which needs no device either."""
+    import ctypes
+    n = ctypes.c_uint64(7)
+    assert lib.mamba_scan_saved_bytes(2, 64, 128, 16, 1, None, None) == 1
+    assert lib.mamba_conv_scan_saved_bytes(2, 64, 128, 16, 4, 1, None, None) == 1
+    assert lib.mamba_dtproj_scan_saved_bytes(2, 64, 128, 16, 8, 1, None, None) == 1
+    assert lib.mamba_cplx_scan_saved_bytes(2, 64, 128, 8, 1, None) == 1
+    assert lib.mamba_dtproj_scan_saved_bytes(2, 64, 128, 16, 0, 1, None, ctypes.byref(n)) == 1
+    n.value = 7
+    assert lib.mamba_dtproj_scan_saved_bytes(2, 64, 128, 16, 8, 0, None, ctypes.byref(n)) == 0
+    assert n.value == 0
